@@ -1,0 +1,122 @@
+"""Seeded synthetic inputs for the MoE layer workloads.
+
+This module only draws random numbers and lays them out. It holds none of the
+layer's arithmetic: no routing, no capacity, no expert math. Both the CUDA
+path's tests/bench and the CPU oracle's tests take their inputs from here.
+
+Workloads (the shapes the pages' discussion turns on, made concrete):
+
+* ``tiny``            N=64,    d=128,  f=256,   E=8,   K=2, W=4, dropless
+* ``mixtral_prefill`` N=4096,  d=4096, f=14336, E=8,   K=2, W=8, dropless,
+                      uniform router init
+* ``e128_skew``       N=8192,  d=2048, f=768,   E=128, K=8, W=8, cf=1.25,
+                      Zipf(s=1.1) per-expert router bias
+* ``decode``          N=16,    d=7168, f=2048,  E=256, K=8, W=8, dropless
+* ``stack4``          N=32768, d=4096, f=1536,  E=64,  K=6, W=8, L=4 layers,
+                      cf in {1.0, 1.25, 2.0} x Zipf s in {0, 1.2}
+
+Recipe (one ``torch.Generator`` per call, ``manual_seed(seed)``; draw order
+x, router, W1, W3, W2; layer ``l`` of a stack re-seeds with ``seed + 1000*l``
+and skips x):
+
+* hidden states x ~ N(0, 1), rounded to bf16 (round-to-nearest-even);
+* router weight Wr [E][d] fp32 ~ N(0, 1/d) (std 1/sqrt(d)), or, for the
+  ``uniform`` init, U(-1/sqrt(d), 1/sqrt(d));
+* expert weights W1, W3 [E][f][d] and W2 [E][d][f] ~ N(0, 0.02^2) (std 0.02),
+  rounded to bf16;
+* Zipf(s) bias: bias[e] = -s * ln(e + 1), computed in float64, stored fp32
+  (expert 0 hottest); s = 0 means no bias (None).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+from typing import Optional
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    N: int
+    d: int
+    f: int
+    E: int
+    K: int
+    W: int
+    cf: float = 0.0          # <= 0 means dropless
+    s: float = 0.0           # Zipf exponent of the per-expert bias; 0 = none
+    router: str = "normal"   # "normal" (N(0,1/d)) or "uniform" (U(+-1/sqrt d))
+    layers: int = 1
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", N=64, d=128, f=256, E=8, K=2, W=4),
+    "mixtral_prefill": Workload("mixtral_prefill", N=4096, d=4096, f=14336, E=8, K=2, W=8,
+                                router="uniform"),
+    "e128_skew": Workload("e128_skew", N=8192, d=2048, f=768, E=128, K=8, W=8, cf=1.25, s=1.1),
+    "decode": Workload("decode", N=16, d=7168, f=2048, E=256, K=8, W=8),
+    "stack4": Workload("stack4", N=32768, d=4096, f=1536, E=64, K=6, W=8, cf=1.25, s=0.0,
+                       layers=4),
+}
+
+STACK_GRID_CF = (1.0, 1.25, 2.0)
+STACK_GRID_S = (0.0, 1.2)
+
+
+def zipf_bias(E: int, s: float) -> Optional[torch.Tensor]:
+    """bias[e] = -s*ln(e+1) (float64, stored fp32); None when s == 0."""
+    if s == 0.0:
+        return None
+    return torch.tensor([-s * math.log(e + 1.0) for e in range(E)], dtype=torch.float64).to(
+        torch.float32)
+
+
+def make_layer_inputs(w: Workload, seed: int = 0, device: str = "cpu", layer: int = 0,
+                      with_x: bool = True) -> dict:
+    """Draw one layer's inputs. Returns a dict of tensors on ``device``.
+
+    Keys: x (bf16 [N][d], only when ``with_x``), w_router (fp32 [E][d]),
+    bias (fp32 [E] or None), w1, w3 (bf16 [E][f][d]), w2 (bf16 [E][d][f]).
+    """
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 1000 * layer)
+    out = {}
+    if with_x:
+        out["x"] = torch.randn(w.N, w.d, generator=g, device=device,
+                               dtype=torch.float32).to(torch.bfloat16)
+    if w.router == "uniform":
+        bound = 1.0 / math.sqrt(w.d)
+        wr = torch.rand(w.E, w.d, generator=g, device=device, dtype=torch.float32)
+        out["w_router"] = (wr * 2.0 - 1.0) * bound
+    else:
+        out["w_router"] = torch.randn(w.E, w.d, generator=g, device=device,
+                                      dtype=torch.float32) * (1.0 / math.sqrt(w.d))
+    b = zipf_bias(w.E, w.s)
+    out["bias"] = None if b is None else b.to(device)
+    for name, shape in (("w1", (w.E, w.f, w.d)), ("w3", (w.E, w.f, w.d)), ("w2", (w.E, w.d, w.f))):
+        t = torch.empty(shape, device=device, dtype=torch.bfloat16)
+        # draw expert by expert to bound the fp32 temporary
+        for e in range(w.E):
+            t[e] = (torch.randn(shape[1:], generator=g, device=device, dtype=torch.float32)
+                    * 0.02).to(torch.bfloat16)
+        out[name] = t
+    return out
+
+
+def random_small_workload(rng: "torch.Generator", max_n: int = 16, max_e: int = 8) -> Workload:
+    """A random tiny shape for brute-force checks (N<=max_n, E<=max_e)."""
+    def ri(lo, hi):
+        return int(torch.randint(lo, hi + 1, (1,), generator=rng).item())
+    E = ri(1, max_e)
+    K = ri(1, E)
+    W = [w for w in range(1, E + 1) if E % w == 0][ri(0, len([w for w in range(1, E + 1) if E % w == 0]) - 1)]
+    n_per = ri(1, max(1, max_n // W))
+    N = n_per * W
+    cf = [0.0, 0.5, 1.0, 1.25, 2.0][ri(0, 4)]
+    s = [0.0, 1.1][ri(0, 1)]
+    return Workload("rand", N=N, d=8 * ri(1, 4), f=8 * ri(1, 4), E=E, K=K, W=W, cf=cf, s=s)

@@ -1,0 +1,319 @@
+/*
+ * CPU oracle for the single-GPU MoE FFN layer: route -> dispatch -> expert
+ * SwiGLU FFN -> combine.
+ *
+ * TEST INFRASTRUCTURE. Plain, slow, obviously correct loops that restate the
+ * definition of each step. Only the tests, the smoke check and the bench's
+ * CPU-baseline / reference arm load this file's library; the product path
+ * never does. It shares no code, header, table or helper with the CUDA path.
+ *
+ * Sources (page title, section):
+ *  [P1] "MoE 专家并行的 All-to-All 通信瓶颈：专家越多推理延迟为何反而上升"
+ *       §All-to-All 分发与回收的机制 (dataflow flowchart: route Top-K, pack by
+ *       destination card, group by expert, grouped GEMM, weighted merge back to
+ *       token order), §专家越多，通信为什么越重 (E/W experts per card, even
+ *       placement, per-card send volume N*K*d*b/W).
+ *  [P2] "MoE 推理服务工程真相 2026 ..." §2.2 Expert Capacity Factor (tokens above
+ *       an expert's capacity are dropped, router output set to zero) and the
+ *       moe_dispatch pseudo-code of §2.3 (bincount of expert ids, overflow mask).
+ *  [P3] "MoE Inference Communication" §DeepSpeed-MoE › MoE 计算核优化 (top-k,
+ *       cumsum, scatter; dense token->expert mapping table), §ExFlow 跨层专家
+ *       亲和性 (conditional routing between consecutive layers), §Aurora 定理
+ *       4.2 (traffic matrix D).
+ * Readings where the pages are silent (all fixed by the workload statement):
+ *  softmax over the K selected logits; ties to the lowest expert index; logits
+ *  accumulated in fp32 by one fused multiply-add per input element, i
+ *  ascending, then + bias; capacity C = ceil(cf*N*K/E) computed in double;
+ *  first-come drop in token-major (t, k) order; a dropped slot contributes 0
+ *  and the others keep their weights; SwiGLU experts y = W2 (silu(W1 x) * W3 x)
+ *  without biases; experts in contiguous blocks of E/W per rank; tokens in
+ *  contiguous shards of N/W per home rank.
+ *
+ * Floating point: logits in fp32 (the precision the selection is defined in);
+ * expert FFN, gate weights and combine in fp64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define EXPORT __attribute__((visibility("default")))
+
+static float bf16_to_float(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Router projection [P1 §All-to-All 分发与回收的机制, node B; P3 §Aurora, gate
+ * term G_i]. logits[t][e] = (sum_i x[t][i] * Wr[e][i]) + bias[e], the sum taken
+ * as one fmaf per i in ascending order starting from +0.0f. */
+EXPORT void orc_router_logits(int64_t N, int64_t d, int64_t E, const uint16_t *x,
+                              const float *w_router, const float *bias, float *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        for (int64_t e = 0; e < E; ++e) {
+            float acc = 0.0f;
+            for (int64_t i = 0; i < d; ++i)
+                acc = fmaf(bf16_to_float(x[t * d + i]), w_router[e * d + i], acc);
+            if (bias)
+                acc = acc + bias[e];
+            logits[t * E + e] = acc;
+        }
+    }
+}
+
+/* Top-K selection and gate weights [P1 §一个反直觉的扩容结果 (Top-K experts per
+ * token); P3 §MoE 计算核优化 (top-k)]. The K largest logits, larger value first,
+ * equal values ordered by lower expert index. Weights: softmax over the K
+ * selected logits, in fp64, stored as fp32. Returns the number of tokens that
+ * have a non-finite logit (their result is unspecified). */
+EXPORT int64_t orc_topk(int64_t N, int64_t E, int64_t K, const float *logits,
+                        int32_t *topk_idx, float *topk_w)
+{
+    int64_t nonfinite = 0;
+    char *chosen = (char *)malloc((size_t)E);
+    double *ex = (double *)malloc((size_t)K * sizeof(double));
+    for (int64_t t = 0; t < N; ++t) {
+        const float *l = logits + t * E;
+        int bad = 0;
+        for (int64_t e = 0; e < E; ++e) {
+            chosen[e] = 0;
+            if (!isfinite(l[e]))
+                bad = 1;
+        }
+        nonfinite += bad;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e) {
+                if (chosen[e])
+                    continue;
+                if (best < 0 || l[e] > l[best])
+                    best = e;
+            }
+            chosen[best] = 1;
+            topk_idx[t * K + k] = (int32_t)best;
+        }
+        double top = (double)l[topk_idx[t * K]];
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            ex[k] = exp((double)l[topk_idx[t * K + k]] - top);
+            sum += ex[k];
+        }
+        for (int64_t k = 0; k < K; ++k)
+            topk_w[t * K + k] = (float)(ex[k] / sum);
+    }
+    free(ex);
+    free(chosen);
+    return nonfinite;
+}
+
+/* Expert capacity [P2 §2.2]: C = ceil(cf * N * K / E), in double. cf <= 0 means
+ * dropless; then C = N * K, which no expert can exceed (each token picks K
+ * distinct experts, so an expert receives at most N). */
+EXPORT int64_t orc_capacity(int64_t N, int64_t E, int64_t K, float cf)
+{
+    if (!(cf > 0.0f))
+        return N * K;
+    return (int64_t)ceil((double)cf * (double)N * (double)K / (double)E);
+}
+
+/* Dispatch bookkeeping [P2 §2.3 pseudo-code (bincount, overflow mask); P3
+ * §MoE 计算核优化 (cumsum, scatter, mapping table); P1 §All-to-All 分发与回收的
+ * 机制 (pack by destination card)].
+ *
+ * Walk assignments a = t*K + k in increasing a. pos[a] = number of earlier
+ * assignments to the same expert. Kept iff pos < C. counts[e] = all
+ * assignments to e, kept[e] = min(counts[e], C). offsets = exclusive scan of
+ * kept (E+1 entries). row_of[a] = offsets[e] + pos[a] if kept else -1, and
+ * assign_of_row is its inverse over the R kept rows.
+ *
+ * Virtual ranks: expert e lives on rank e / (E/W); token t's home is
+ * t / (N/W). D[i][j] counts kept assignments from home i to expert rank j.
+ * The packed buffer holds blocks (i, j) in row-major order, each block's rows
+ * ordered by (expert, token); pk_off is the exclusive scan of D (W*W+1
+ * entries) and packed_row_of[a] the row of assignment a there (-1 if dropped).
+ *
+ * stats[0] R (kept rows), [1] dropped, [2] kept rows with rank(e) != home(t),
+ * [3] distinct (t, rank) pairs with rank != home(t) over kept assignments
+ * (what a deduplicating exchange would send), [4] experts with kept > 0,
+ * [5] max kept[e], [6] min kept[e], [7] C. */
+EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
+                          const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                          int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                          int64_t *D, int64_t *pk_off, int32_t *packed_row_of,
+                          int64_t *stats)
+{
+    int64_t e_per = E / W, n_per = N / W;
+    int64_t *seen = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *pos = (int64_t *)malloc((size_t)(N * K) * sizeof(int64_t));
+
+    for (int64_t a = 0; a < N * K; ++a) {
+        int64_t e = topk_idx[a];
+        pos[a] = seen[e];
+        seen[e] += 1;
+    }
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; ++e) {
+        counts[e] = (int32_t)seen[e];
+        kept[e] = (int32_t)(seen[e] < C ? seen[e] : C);
+        offsets[e + 1] = offsets[e] + kept[e];
+    }
+    for (int64_t i = 0; i < W * W; ++i)
+        D[i] = 0;
+    int64_t R = 0, cross = 0;
+    for (int64_t a = 0; a < N * K; ++a) {
+        int64_t e = topk_idx[a];
+        int64_t t = a / K;
+        if (pos[a] < C) {
+            int64_t r = offsets[e] + pos[a];
+            row_of[a] = (int32_t)r;
+            assign_of_row[r] = (int32_t)a;
+            int64_t i = t / n_per, j = e / e_per;
+            D[i * W + j] += 1;
+            if (i != j)
+                cross += 1;
+            R += 1;
+        } else {
+            row_of[a] = -1;
+        }
+    }
+    pk_off[0] = 0;
+    for (int64_t b = 0; b < W * W; ++b)
+        pk_off[b + 1] = pk_off[b] + D[b];
+
+    /* packed order: block (i, j), then expert e of rank j, then token t of
+     * shard i, then slot k (a token selects an expert at most once). */
+    for (int64_t a = 0; a < N * K; ++a)
+        packed_row_of[a] = -1;
+    int64_t next = 0;
+    for (int64_t i = 0; i < W; ++i)
+        for (int64_t j = 0; j < W; ++j)
+            for (int64_t e = j * e_per; e < (j + 1) * e_per; ++e)
+                for (int64_t t = i * n_per; t < (i + 1) * n_per; ++t)
+                    for (int64_t k = 0; k < K; ++k) {
+                        int64_t a = t * K + k;
+                        if (topk_idx[a] == e && row_of[a] >= 0)
+                            packed_row_of[a] = (int32_t)(next++);
+                    }
+
+    /* distinct destination ranks per token, excluding the home rank */
+    int64_t dedup = 0;
+    char *rank_seen = (char *)malloc((size_t)W);
+    for (int64_t t = 0; t < N; ++t) {
+        memset(rank_seen, 0, (size_t)W);
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t a = t * K + k;
+            if (row_of[a] < 0)
+                continue;
+            int64_t j = topk_idx[a] / e_per;
+            if (j != t / n_per && !rank_seen[j]) {
+                rank_seen[j] = 1;
+                dedup += 1;
+            }
+        }
+    }
+    int64_t active = 0, mx = 0, mn = -1;
+    for (int64_t e = 0; e < E; ++e) {
+        if (kept[e] > 0)
+            active += 1;
+        if (kept[e] > mx)
+            mx = kept[e];
+        if (mn < 0 || kept[e] < mn)
+            mn = kept[e];
+    }
+    stats[0] = R;
+    stats[1] = N * K - R;
+    stats[2] = cross;
+    stats[3] = dedup;
+    stats[4] = active;
+    stats[5] = mx;
+    stats[6] = mn;
+    stats[7] = C;
+    free(rank_seen);
+    free(pos);
+    free(seen);
+}
+
+/* Expert FFN for a list of rows [P1 §All-to-All 分发与回收的机制, node F: each
+ * expert's tokens through its own FFN]. Row r holds the hidden state of token
+ * row_token[r] for expert row_expert[r]:
+ *   g = W1[e] x, u = W3[e] x, h = g * sigmoid(g) * u, y = W2[e] h,
+ * all in fp64 from the bf16 inputs. W1, W3 are [E][f][d]; W2 is [E][d][f].
+ * h_out (nullable) receives h [nrows][f]; y_out receives y [nrows][d]. */
+EXPORT void orc_expert_rows(int64_t nrows, const int32_t *row_token, const int32_t *row_expert,
+                            int64_t d, int64_t f, const uint16_t *x, const uint16_t *w1,
+                            const uint16_t *w3, const uint16_t *w2, double *h_out, double *y_out)
+{
+#pragma omp parallel
+    {
+        double *xr = (double *)malloc((size_t)d * sizeof(double));
+        double *h = (double *)malloc((size_t)f * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t t = row_token[r], e = row_expert[r];
+            for (int64_t i = 0; i < d; ++i)
+                xr[i] = (double)bf16_to_float(x[t * d + i]);
+            for (int64_t j = 0; j < f; ++j) {
+                const uint16_t *a = w1 + (e * f + j) * d;
+                const uint16_t *b = w3 + (e * f + j) * d;
+                double g = 0.0, u = 0.0;
+                for (int64_t i = 0; i < d; ++i) {
+                    g += xr[i] * (double)bf16_to_float(a[i]);
+                    u += xr[i] * (double)bf16_to_float(b[i]);
+                }
+                h[j] = g / (1.0 + exp(-g)) * u;
+                if (h_out)
+                    h_out[r * f + j] = h[j];
+            }
+            for (int64_t i = 0; i < d; ++i) {
+                const uint16_t *c = w2 + (e * d + i) * f;
+                double y = 0.0;
+                for (int64_t j = 0; j < f; ++j)
+                    y += h[j] * (double)bf16_to_float(c[j]);
+                y_out[r * d + i] = y;
+            }
+        }
+        free(h);
+        free(xr);
+    }
+}
+
+/* Weighted combine [P1 §All-to-All 分发与回收的机制, node I: weighted merge back
+ * to the original token order; P2 §2.2: a dropped slot's router output is
+ * zero]. out[t] = sum over kept slots k, in k order, of w[t][k] * y[row], where
+ * y_of_slot[(t*K+k)*d ...] holds the expert output of slot (t, k). */
+EXPORT void orc_combine(int64_t N, int64_t K, int64_t d, const int32_t *row_of,
+                        const float *topk_w, const double *y_of_slot, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < N; ++t) {
+        for (int64_t i = 0; i < d; ++i)
+            out[t * d + i] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t a = t * K + k;
+            if (row_of[a] < 0)
+                continue;
+            double w = (double)topk_w[a];
+            for (int64_t i = 0; i < d; ++i)
+                out[t * d + i] += w * y_of_slot[a * d + i];
+        }
+    }
+}
+
+/* Inter-layer expert affinity counts [P3 §ExFlow 跨层专家亲和性]: for every
+ * token t, every expert i in its top-K at layer j and every expert p in its
+ * top-K at layer j+1, cnt[i][p] += 1 (pre-drop routing decisions). The
+ * conditional P(p | i) is cnt[i][p] / (number of tokens with i in their top-K
+ * at layer j); each row of cnt sums to K times that number. */
+EXPORT void orc_affinity(int64_t N, int64_t E, int64_t K, const int32_t *topk_j,
+                         const int32_t *topk_j1, int64_t *cnt)
+{
+    for (int64_t t = 0; t < N; ++t)
+        for (int64_t k = 0; k < K; ++k)
+            for (int64_t q = 0; q < K; ++q)
+                cnt[(int64_t)topk_j[t * K + k] * E + topk_j1[t * K + q]] += 1;
+}

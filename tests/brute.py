@@ -1,0 +1,123 @@
+"""Brute-force restatement of the layer for tiny inputs, used to pin the oracle.
+
+Independent of ``oracle/moe_oracle.c``: exact rational arithmetic for the fp32
+fused multiply-add chain, a full sort for top-K, an O(N*K*E) recount for
+positions, Python sets for deduplication and numpy float64 matmuls for the
+expert FFN. Pure Python loops: tiny shapes only.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+
+import numpy as np
+
+
+def _f32_bits(v: np.float32) -> int:
+    return int(np.array(v, dtype=np.float32).view(np.uint32))
+
+
+def round_to_f32(q: Fraction) -> float:
+    """Round an exact rational to binary32, nearest with ties to even."""
+    c0 = np.float32(float(q))
+    cands = [np.nextafter(c0, np.float32(-np.inf)), c0, np.nextafter(c0, np.float32(np.inf))]
+    best = None
+    for c in cands:
+        if not np.isfinite(c):
+            continue
+        dist = abs(Fraction(float(c)) - q)
+        if (best is None or dist < best[0]
+                or (dist == best[0] and (_f32_bits(c) & 1) == 0 and (_f32_bits(best[1]) & 1) == 1)):
+            best = (dist, c)
+    return float(best[1])
+
+
+def fmaf_exact(a: float, b: float, c: float) -> float:
+    return round_to_f32(Fraction(a) * Fraction(b) + Fraction(c))
+
+
+def bf16_bits_to_float(u: np.ndarray) -> np.ndarray:
+    return (u.astype(np.uint32) << 16).view(np.float32)
+
+
+def logits(x_u16: np.ndarray, wr: np.ndarray, bias) -> np.ndarray:
+    x = bf16_bits_to_float(x_u16)
+    N, d = x.shape
+    E = wr.shape[0]
+    out = np.empty((N, E), np.float32)
+    for t in range(N):
+        for e in range(E):
+            acc = 0.0
+            for i in range(d):
+                acc = fmaf_exact(float(x[t, i]), float(wr[e, i]), acc)
+            if bias is not None:
+                acc = round_to_f32(Fraction(acc) + Fraction(float(bias[e])))
+            out[t, e] = acc
+    return out
+
+
+def topk(lg: np.ndarray, K: int):
+    N, E = lg.shape
+    idx = np.empty((N, K), np.int32)
+    w = np.empty((N, K), np.float64)
+    for t in range(N):
+        order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))[:K]
+        idx[t] = order
+        ex = [math.exp(float(lg[t, e]) - float(lg[t, order[0]])) for e in order]
+        s = math.fsum(ex)
+        w[t] = [v / s for v in ex]
+    return idx, w
+
+
+def capacity(N: int, E: int, K: int, cf: float) -> int:
+    if not cf > 0:
+        return N * K
+    return math.ceil(Fraction(cf) * N * K / E)
+
+
+def dispatch(idx: np.ndarray, E: int, W: int, C: int) -> dict:
+    N, K = idx.shape
+    flat = idx.reshape(-1)
+    pos = [sum(1 for b in range(a) if flat[b] == flat[a]) for a in range(N * K)]
+    counts = [sum(1 for a in range(N * K) if flat[a] == e) for e in range(E)]
+    kept = [min(c, C) for c in counts]
+    offsets = [0]
+    for e in range(E):
+        offsets.append(offsets[-1] + kept[e])
+    row_of = [offsets[flat[a]] + pos[a] if pos[a] < C else -1 for a in range(N * K)]
+    e_per, n_per = E // W, N // W
+    D = np.zeros((W, W), np.int64)
+    keyed = []
+    for a in range(N * K):
+        if row_of[a] >= 0:
+            t, e = a // K, int(flat[a])
+            D[t // n_per, e // e_per] += 1
+            keyed.append(((t // n_per, e // e_per, e, t), a))
+    keyed.sort()
+    packed_row_of = [-1] * (N * K)
+    for p, (_, a) in enumerate(keyed):
+        packed_row_of[a] = p
+    dedup = 0
+    for t in range(N):
+        dests = {int(flat[t * K + k]) // e_per for k in range(K) if row_of[t * K + k] >= 0}
+        dests.discard(t // n_per)
+        dedup += len(dests)
+    return dict(counts=np.array(counts), kept=np.array(kept), offsets=np.array(offsets),
+                row_of=np.array(row_of), D=D, packed_row_of=np.array(packed_row_of), dedup=dedup)
+
+
+def swiglu_rows(x_u16, w1_u16, w3_u16, w2_u16, row_token, row_expert):
+    """Expert FFN through numpy float64 matmuls, one expert at a time."""
+    x = bf16_bits_to_float(x_u16).astype(np.float64)
+    w1 = bf16_bits_to_float(w1_u16).astype(np.float64)
+    w3 = bf16_bits_to_float(w3_u16).astype(np.float64)
+    w2 = bf16_bits_to_float(w2_u16).astype(np.float64)
+    y = np.zeros((len(row_token), x.shape[1]))
+    for e in sorted(set(int(v) for v in row_expert)):
+        sel = np.nonzero(np.asarray(row_expert) == e)[0]
+        X = x[np.asarray(row_token)[sel]]
+        G = X @ w1[e].T
+        U = X @ w3[e].T
+        H = G / (1.0 + np.exp(-G)) * U
+        y[sel] = H @ w2[e].T
+    return y

@@ -1,0 +1,337 @@
+"""Pins of the CPU oracle against things other than itself: hand-worked
+fixtures, brute force on tiny inputs, closed forms, library routines and
+invariants. CPU only."""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import brute
+from moe_workloads import Workload, WORKLOADS, make_layer_inputs, random_small_workload
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as fh:
+        return json.load(fh)
+
+
+# --------------------------------------------------------------------------- hand-worked
+
+def test_hand_routing_fixture(orc):
+    g = _load("hand_routing.json")
+    lg = np.array(g["logits"], np.float32)
+    idx, w, bad = orc.topk(lg, g["K"])
+    assert bad == 0
+    np.testing.assert_array_equal(idx, g["topk_idx"])
+    np.testing.assert_allclose(w, g["topk_w"], rtol=1e-6, atol=0)
+    C = orc.capacity(g["N"], g["E"], g["K"], g["cf"])
+    assert C == g["C"]
+    p = orc.positions(idx, g["E"], g["W"], C)
+    for key in ("counts", "kept", "offsets", "row_of", "assign_of_row", "pk_off", "packed_row_of"):
+        np.testing.assert_array_equal(p[key], g[key], err_msg=key)
+    np.testing.assert_array_equal(p["D"], g["D"])
+    assert p["stats"] == g["stats"]
+    rep = orc.derive_report(g["N"], g["E"], g["K"], g["W"], p["kept"], p["D"], p["stats"], d=1)
+    for key, v in g["report"].items():
+        assert rep[key] == pytest.approx(v, rel=1e-12), key
+
+
+def test_dispatch_volume_worked_example(orc):
+    g = _load("dispatch_volume.json")
+    for c in g["cases"]:
+        b = orc.dispatch_bytes(c["rows"], g["d"], g["elem_bytes"])
+        assert b == c["bytes"], c["name"]
+        assert abs(b - c["printed_value"]) <= c["rel_round"] * c["printed_value"], c["name"]
+
+
+def test_dispatch_volume_through_routing(orc):
+    # K=1 dropless routing of 2048 tokens at d=2048 carries the prefill figure
+    rng = np.random.default_rng(0)
+    lg = rng.standard_normal((2048, 16)).astype(np.float32)
+    idx, _, _ = orc.topk(lg, 1)
+    p = orc.positions(idx, 16, 4, orc.capacity(2048, 16, 1, 0.0))
+    rep = orc.derive_report(2048, 16, 1, 4, p["kept"], p["D"], p["stats"], d=2048, elem_bytes=2)
+    assert rep["dispatch_bytes"] == 8388608
+
+
+# --------------------------------------------------------------------------- brute force
+
+def _tiny_inputs(w: Workload, seed: int):
+    inp = make_layer_inputs(w, seed=seed)
+    return inp
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_brute_force_tiny(orc, seed):
+    rng = torch.Generator().manual_seed(100 + seed)
+    w = random_small_workload(rng, max_n=16, max_e=8)
+    inp = _tiny_inputs(w, seed)
+    xu = orc.as_u16(inp["x"])
+    wr = inp["w_router"].numpy()
+    bias = None if inp["bias"] is None else inp["bias"].numpy()
+
+    # logits: exact rational fmaf chain vs the oracle, bit for bit
+    lg_b = brute.logits(xu, wr, bias)
+    lg_o = orc.router_logits(inp["x"], inp["w_router"], inp["bias"])
+    np.testing.assert_array_equal(lg_o.view(np.uint32), lg_b.view(np.uint32))
+
+    # top-K by a full sort; weights by fp64 softmax
+    idx_b, w_b = brute.topk(lg_b, w.K)
+    idx_o, w_o, bad = orc.topk(lg_o, w.K)
+    assert bad == 0
+    np.testing.assert_array_equal(idx_o, idx_b)
+    np.testing.assert_allclose(w_o, w_b, rtol=2e-7, atol=0)
+
+    C = orc.capacity(w.N, w.E, w.K, w.cf)
+    assert C == brute.capacity(w.N, w.E, w.K, w.cf)
+    p = orc.positions(idx_o, w.E, w.W, C)
+    b = brute.dispatch(idx_b, w.E, w.W, C)
+    for key in ("counts", "kept", "offsets", "row_of", "packed_row_of"):
+        np.testing.assert_array_equal(p[key], b[key], err_msg=key)
+    np.testing.assert_array_equal(p["D"], b["D"])
+    assert p["stats"]["dedup_pairs"] == b["dedup"]
+
+    # whole layer output vs numpy float64 matmul experts + a Python combine
+    r = orc.layer(inp, w.K, w.W, w.cf)
+    aor = r["assign_of_row"]
+    y_b = brute.swiglu_rows(xu, orc.as_u16(inp["w1"]), orc.as_u16(inp["w3"]), orc.as_u16(inp["w2"]),
+                            aor // w.K, idx_b.reshape(-1)[aor])
+    np.testing.assert_allclose(r["y_rows"], y_b, rtol=1e-10, atol=1e-13)
+    out_b = np.zeros((w.N, w.d))
+    for t in range(w.N):
+        for k in range(w.K):
+            row = b["row_of"][t * w.K + k]
+            if row >= 0:
+                out_b[t] += float(w_o[t, k]) * y_b[row]
+    np.testing.assert_allclose(r["out"], out_b, rtol=1e-10, atol=1e-13)
+
+
+def test_brute_force_tiny_workload(orc):
+    """The 'tiny' workload, logits and routing checked by brute force."""
+    w = WORKLOADS["tiny"]
+    inp = make_layer_inputs(w, seed=0)
+    xu = orc.as_u16(inp["x"])
+    # brute-force logits on a token subset (exact rational arithmetic is slow)
+    sub = slice(0, 6)
+    lg_b = brute.logits(xu[sub], inp["w_router"].numpy(), None)
+    lg_o = orc.router_logits(inp["x"], inp["w_router"], None)
+    np.testing.assert_array_equal(lg_o[sub].view(np.uint32), lg_b.view(np.uint32))
+    idx_o, _, _ = orc.topk(lg_o, w.K)
+    idx_b, _ = brute.topk(lg_o, w.K)
+    np.testing.assert_array_equal(idx_o, idx_b)
+    p = orc.positions(idx_o, w.E, w.W, orc.capacity(w.N, w.E, w.K, w.cf))
+    b = brute.dispatch(idx_b, w.E, w.W, orc.capacity(w.N, w.E, w.K, w.cf))
+    np.testing.assert_array_equal(p["row_of"], b["row_of"])
+    np.testing.assert_array_equal(p["packed_row_of"], b["packed_row_of"])
+
+
+# --------------------------------------------------------------------------- special cases
+
+def test_single_expert_is_dense_swiglu(orc):
+    """E = 1, K = 1: the layer is the dense SwiGLU FFN, gate weight exactly 1."""
+    w = Workload("dense", N=24, d=64, f=96, E=1, K=1, W=1)
+    inp = make_layer_inputs(w, seed=3)
+    r = orc.layer(inp, 1, 1, 0.0)
+    assert np.all(r["topk_w"] == 1.0)
+    x = brute.bf16_bits_to_float(orc.as_u16(inp["x"])).astype(np.float64)
+    w1 = brute.bf16_bits_to_float(orc.as_u16(inp["w1"]))[0].astype(np.float64)
+    w3 = brute.bf16_bits_to_float(orc.as_u16(inp["w3"]))[0].astype(np.float64)
+    w2 = brute.bf16_bits_to_float(orc.as_u16(inp["w2"]))[0].astype(np.float64)
+    g = x @ w1.T
+    u = x @ w3.T
+    dense = (g * (1.0 / (1.0 + np.exp(-g))) * u) @ w2.T
+    np.testing.assert_allclose(r["out"], dense, rtol=1e-10, atol=1e-14)
+
+
+def test_swiglu_closed_form(orc):
+    """One-hot input: g_j = W1[j][0], u_j = W3[j][0] exactly, so
+    h_j = g_j * sigmoid(g_j) * u_j and y_i = sum_j h_j W2[i][j] in closed form."""
+    d, f = 8, 4
+    x = torch.zeros(1, d, dtype=torch.bfloat16)
+    x[0, 0] = 1.0
+    gvals = [-2.0, -0.5, 0.0, 3.0]
+    uvals = [1.5, -1.0, 2.0, 0.25]
+    w1 = torch.zeros(1, f, d, dtype=torch.bfloat16)
+    w3 = torch.zeros(1, f, d, dtype=torch.bfloat16)
+    w2 = torch.zeros(1, d, f, dtype=torch.bfloat16)
+    for j in range(f):
+        w1[0, j, 0] = gvals[j]
+        w3[0, j, 0] = uvals[j]
+    w2[0, 1, :] = torch.tensor([1.0, 2.0, -1.0, 0.5], dtype=torch.bfloat16)
+    h, y = orc.expert_rows(np.array([0]), np.array([0]), x, w1, w3, w2, want_h=True)
+    h_ref = [g / (1.0 + math.exp(-g)) * u for g, u in zip(gvals, uvals)]
+    np.testing.assert_allclose(h[0], h_ref, rtol=1e-15)
+    y_ref = np.zeros(d)
+    y_ref[1] = h_ref[0] * 1.0 + h_ref[1] * 2.0 - h_ref[2] + h_ref[3] * 0.5
+    np.testing.assert_allclose(y[0], y_ref, rtol=1e-15, atol=1e-300)
+
+
+def test_identity_experts_round_trip(orc):
+    """Identity experts (y row = the dispatched x row): combine(dispatch(x))
+    returns x * sum of kept weights; dropless, that sum is 1 up to fp32 weight
+    rounding."""
+    for cf in (0.0, 0.75):
+        w = Workload("id", N=64, d=32, f=8, E=8, K=3, W=4, cf=cf, s=1.1)
+        inp = make_layer_inputs(w, seed=7)
+        r = orc.route_and_dispatch(inp["x"], inp["w_router"], inp["bias"], w.K, w.W, w.cf)
+        x = brute.bf16_bits_to_float(orc.as_u16(inp["x"])).astype(np.float64)
+        y_rows = x[r["assign_of_row"] // w.K]
+        y_of_slot = np.zeros((w.N * w.K, w.d))
+        kept = r["row_of"] >= 0
+        y_of_slot[kept] = y_rows[r["row_of"][kept]]
+        out = orc.combine(r["row_of"], r["topk_w"], y_of_slot)
+        wsum = np.where(r["row_of"].reshape(w.N, w.K) >= 0, r["topk_w"].astype(np.float64), 0).sum(1)
+        np.testing.assert_allclose(out, x * wsum[:, None], rtol=1e-12, atol=1e-15)
+        if cf == 0.0:
+            np.testing.assert_allclose(wsum, 1.0, rtol=0, atol=4e-7)
+        else:
+            assert r["stats"]["dropped"] > 0
+
+
+def test_fully_dropped_token_outputs_zero(orc):
+    lg = np.array([[1.0, 0.0], [1.0, 0.0], [1.0, 0.0]], np.float32)  # all pick expert 0
+    idx, wts, _ = orc.topk(lg, 1)
+    p = orc.positions(idx, 2, 1, 2)
+    assert list(p["row_of"]) == [0, 1, -1]
+    out = orc.combine(p["row_of"], wts, np.ones((3, 4)))
+    np.testing.assert_array_equal(out[2], 0.0)
+    np.testing.assert_array_equal(out[:2], 1.0)
+
+
+def test_ties_and_signed_zero(orc):
+    lg = np.array([[0.0, -0.0, 0.0, -1.0], [2.0, 2.0, 2.0, 2.0]], np.float32)
+    idx, w, _ = orc.topk(lg, 3)
+    assert idx.tolist() == [[0, 1, 2], [0, 1, 2]]
+    np.testing.assert_allclose(w[1], [1 / 3] * 3, rtol=1e-7)
+
+
+def test_nonfinite_logit_counted(orc):
+    lg = np.array([[0.0, np.nan], [1.0, 2.0], [np.inf, 0.0]], np.float32)
+    _, _, bad = orc.topk(lg, 1)
+    assert bad == 2
+
+
+def test_capacity_exact():
+    import oracle
+    cases = [(8192, 128, 8, 1.25, 640), (32768, 64, 6, 1.0, 3072), (32768, 64, 6, 1.25, 3840),
+             (32768, 64, 6, 2.0, 6144), (4, 4, 2, 1.0, 2), (10, 3, 2, 1.0, 7), (7, 5, 3, 0.3, 2)]
+    for N, E, K, cf, want in cases:
+        assert oracle.capacity(N, E, K, cf) == want == math.ceil(Fraction(cf) * N * K / E)
+    assert oracle.capacity(16, 256, 8, 0.0) == 16 * 8
+
+
+# --------------------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("name,cf,s", [("e128_skew", 1.25, 1.1), ("stack4", 1.0, 1.2),
+                                        ("stack4", 2.0, 0.0)])
+def test_routing_invariants_at_scale(orc, name, cf, s):
+    """Integer invariants on full-size routing (logits drawn directly; the
+    invariants do not depend on how the logits arose)."""
+    w = WORKLOADS[name].with_(cf=cf, s=s)
+    rng = np.random.default_rng(11)
+    lg = rng.standard_normal((w.N, w.E)).astype(np.float32)
+    if s:
+        lg = lg + np.array([-s * math.log(e + 1) for e in range(w.E)], np.float32)
+    idx, wts, _ = orc.topk(lg, w.K)
+    C = orc.capacity(w.N, w.E, w.K, w.cf)
+    p = orc.positions(idx, w.E, w.W, C)
+    NK = w.N * w.K
+    assert p["counts"].sum() == NK
+    assert p["kept"].sum() == NK - p["stats"]["dropped"] == p["R"]
+    assert p["kept"].max() <= C
+    np.testing.assert_array_equal(p["counts"], np.bincount(idx.reshape(-1), minlength=w.E))
+    # every kept (t, k) exactly once among the rows; each token K - drops times
+    aor = p["assign_of_row"]
+    assert len(np.unique(aor)) == p["R"]
+    np.testing.assert_array_equal(p["row_of"][aor], np.arange(p["R"]))
+    drops = (p["row_of"].reshape(w.N, w.K) < 0).sum(1)
+    np.testing.assert_array_equal(np.bincount(aor // w.K, minlength=w.N), w.K - drops)
+    # rows inside each expert come in increasing token order
+    rows_e = idx.reshape(-1)[aor]
+    assert np.all(np.diff(rows_e) >= 0)
+    same = rows_e[1:] == rows_e[:-1]
+    assert np.all(np.diff(aor)[same] > 0)
+    # traffic matrix and packing
+    assert p["D"].sum() == p["R"]
+    assert p["pk_off"][-1] == p["R"]
+    pk = p["packed_row_of"][p["row_of"] >= 0]
+    assert sorted(pk.tolist()) == list(range(p["R"]))
+    # per-home-rank rows = row sums of D
+    home = (aor // w.K) // (w.N // w.W)
+    np.testing.assert_array_equal(np.bincount(home, minlength=w.W), p["D"].sum(1))
+
+
+def test_mean_send_volume_closed_form(orc):
+    """Dropless, the mean per-rank send equals N*K*d*b/W
+    [MoE 专家并行的 All-to-All 通信瓶颈, §专家越多，通信为什么越重]."""
+    N, E, K, W, d = 4096, 64, 6, 8, 4096
+    rng = np.random.default_rng(5)
+    idx, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    p = orc.positions(idx, E, W, orc.capacity(N, E, K, 0.0))
+    send_bytes = p["D"].sum(1) * d * 2
+    assert send_bytes.mean() == N * K * d * 2 / W
+
+
+def test_local_fraction_is_one_over_w(orc):
+    """Unbiased routing with experts spread evenly: a routed row stays on its
+    home rank with probability (E/W)/E = 1/W
+    [MoE 专家并行的 All-to-All 通信瓶颈, §专家越多，通信为什么越重]."""
+    N, E, K, W = 8192, 64, 6, 8
+    rng = np.random.default_rng(9)
+    idx, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    p = orc.positions(idx, E, W, orc.capacity(N, E, K, 0.0))
+    local = np.trace(p["D"]) / p["R"]
+    n = p["R"]
+    sigma = math.sqrt((1 / W) * (1 - 1 / W) / n) * math.sqrt(K)  # slots of a token correlate
+    assert abs(local - 1 / W) < 4 * sigma
+    rep = orc.derive_report(N, E, K, W, p["kept"], p["D"], p["stats"], d=1)
+    assert rep["cross_rank_fraction"] == pytest.approx(1 - local)
+
+
+def test_tau_min_identity(orc):
+    """Aurora's bound on a hand traffic matrix: the busiest sender or receiver
+    [MoE Inference Communication, §Aurora 定理 4.2]."""
+    D = np.array([[5, 2, 0], [1, 7, 4], [3, 0, 2]])
+    rep = orc.derive_report(3, 3, 1, 3, np.array([1, 1, 1]), D,
+                            dict(R=int(D.sum()), dropped=0, cross_rows=10, dedup_pairs=0,
+                                 active_experts=3), d=1)
+    # off-diagonal row sums 2, 5, 3; column sums 4, 2, 4
+    assert rep["tau_min_tokens"] == 5
+    assert rep["send_max"] == 12 and rep["recv_min"] == 6
+
+
+def test_affinity_invariants(orc):
+    """Affinity counts [MoE Inference Communication, §ExFlow 跨层专家亲和性]:
+    brute-force recount, row sums K * n_j(i), total K^2 N."""
+    N, E, K = 300, 16, 3
+    rng = np.random.default_rng(4)
+    a, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    b, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    cnt = orc.affinity(a, b, E)
+    ref = np.zeros((E, E), np.int64)
+    for t in range(N):
+        for i in a[t]:
+            for p_ in b[t]:
+                ref[i, p_] += 1
+    np.testing.assert_array_equal(cnt, ref)
+    n_i = np.bincount(a.reshape(-1), minlength=E)
+    np.testing.assert_array_equal(cnt.sum(1), K * n_i)
+    assert cnt.sum() == K * K * N
+    # identical consecutive routing: mass on the K x K blocks of each token
+    same = orc.affinity(a, a, E)
+    assert np.trace(same) == N * K
+
+
+def test_sampled_layer_matches_full(orc):
+    w = Workload("s", N=48, d=64, f=64, E=8, K=2, W=4, cf=1.0, s=1.1)
+    inp = make_layer_inputs(w, seed=2)
+    full = orc.layer(inp, w.K, w.W, w.cf)
+    toks = [0, 5, 17, 47]
+    smp = orc.layer_sampled(inp, w.K, w.W, w.cf, toks)
+    np.testing.assert_allclose(smp["out_tokens"], full["out"][toks], rtol=1e-13, atol=1e-15)
