@@ -1,0 +1,481 @@
+"""Benchmark of the MoE layer hot path on B200.
+
+One step = one pass of the whole layer over one batch of synthetic tokens:
+router logits -> top-K -> dispatch (histogram, scan, positions, scatter into
+the expert-sorted and the rank-packed buffers) -> gate/up grouped GEMM -> down
+grouped GEMM -> combine. Default workload: the Mixtral-shaped prefill layer
+(N=4096 tokens, d=4096, f=14336, E=8, K=2, W=8 virtual ranks, dropless).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Multi-GPU (torchrun, one process per GPU): the layer does not shard on one GPU's
+path, so every rank runs an independent replica on its own batch (no
+collective on the data path); the reported time is the max over ranks and the
+value counts the tokens of all ranks ("scaling": "weak").
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "moe_layer_tokens_per_s"
+UNIT = "tokens/s"
+
+
+# --------------------------------------------------------------------------- distributed harness
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    world, rank, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when single-process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(tokens_per_rank: float, elapsed_s: float, device=None) -> dict:
+    """Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    t_max = max_over_ranks(elapsed_s, device)
+    total = sum_over_ranks(tokens_per_rank, device)
+    return dict(elapsed_max_s=t_max, tokens_total=total, value=total / t_max if t_max > 0 else 0.0)
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
+                except ValueError:
+                    continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["power"] > 300.0] or rows
+        reasons = []
+        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                          ("swt", "sw_thermal_slowdown"), ("cap", "sw_power_cap")):
+            if any(r[key].lower() == "active" for r in load):
+                reasons.append(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(load)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+# DRAM bytes per launch of the gate/up grouped GEMM, from the ncu capture summarised in
+# profiles/grouped_gemm_up_mixtral_prefill_half_full.md (half-size case, scaled x2 to the
+# full layer). Valid only for the kernel source it was measured on.
+MEASURED_UP_TRAFFIC = {
+    "kernel_sha256": "28a3c9dae73d22cb397f70f7a04a51635be79cbfdbca4c92c286432e55a26756",
+    "workload": "mixtral_prefill",
+    "bytes": 2171.8e6,
+}
+
+
+def up_traffic(workload: str):
+    path = os.path.join(ROOT, "combine_grouped_gemm_router_b200", "csrc", "grouped_gemm.cuh")
+    try:
+        with open(path, "rb") as fh:
+            sha = hashlib.sha256(fh.read()).hexdigest()
+    except OSError:
+        return None
+    if sha == MEASURED_UP_TRAFFIC["kernel_sha256"] and workload == MEASURED_UP_TRAFFIC["workload"]:
+        return MEASURED_UP_TRAFFIC["bytes"]
+    return None
+
+
+def algorithmic_work(w, R: int) -> dict:
+    """Algorithmic flops and bytes per launch of each stage (see the design notes)."""
+    N, d, f, E, K = w.N, w.d, w.f, w.E, w.K
+    return dict(
+        up_flops=4.0 * d * f * R,
+        down_flops=2.0 * d * f * R,
+        logits_bytes=N * d * 2 + E * d * 4 + N * E * 4,
+        # scatter: read each token row once, write every kept row twice (sorted + packed)
+        scatter_bytes=N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3,
+        # combine: read every kept fp32 expert row, the routing, write fp32 out
+        combine_bytes=R * d * 4 + N * K * 8 + N * d * 4,
+    )
+
+
+def run_gpu(args, w) -> dict:
+    import torch
+
+    import combine_grouped_gemm_router_b200 as m
+    from moe_workloads import make_layer_inputs
+
+    world, rank = init_dist("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    inp = make_layer_inputs(w, seed=args.seed + rank, device=str(dev))
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    RA = m.moe_rows_alloc(shape)
+    ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
+    x, wr, bias = inp["x"], inp["w_router"], inp["bias"]
+    w1, w3, w2 = inp["w1"], inp["w3"], inp["w2"]
+    N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
+    topk_idx = torch.empty(N, K, dtype=torch.int32, device=dev)
+    topk_w = torch.empty(N, K, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(N * K, dtype=torch.int32, device=dev)
+    assign = torch.empty(RA, dtype=torch.int32, device=dev)
+    x_sorted = torch.empty(RA, d, dtype=torch.bfloat16, device=dev)
+    x_packed = torch.empty(RA, d, dtype=torch.bfloat16, device=dev)
+    D = torch.empty(W * W, dtype=torch.int64, device=dev)
+    pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
+    h = torch.empty(RA, f, dtype=torch.bfloat16, device=dev)
+    y = torch.empty(RA, d, dtype=torch.float32, device=dev)
+    out = torch.empty(N, d, dtype=torch.float32, device=dev)
+
+    n_ev = 6
+    launches_per_step = 9  # logits, top-K, histogram, scan, positions, scatter, up, down, combine
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        m.moe_route(shape, x, wr, bias, topk_idx, topk_w, None, ws, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted,
+                       x_packed, D, pk_off, None, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        m.moe_expert_up(shape, x_sorted, offsets, w1, w3, h, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        m.moe_expert_down(shape, h, offsets, w2, y, stream)
+        if ev is not None:
+            ev[4].record(stream)
+        m.moe_combine(shape, y, row_of, topk_w, out, None, stream)
+        if ev is not None:
+            ev[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if m.moe_get_device_error(True) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        t_stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_s = t_start.elapsed_time(t_stop) / 1e3
+    stage_ms = {name: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events)
+                for j, name in enumerate(["route", "dispatch", "expert_up", "expert_down",
+                                          "combine"])}
+    err = m.moe_get_device_error(True)
+    R = int(offsets[E].item())
+    agg = aggregate(float(N * args.steps), elapsed_s, dev)
+
+    # end to end through the public API: pinned host input -> moe_layer -> host output
+    e2e = None
+    if not args.no_e2e:
+        lws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
+        x_host = x.cpu().pin_memory()
+        out_host = torch.empty(N, d, dtype=torch.float32).pin_memory()
+        x_dev = torch.empty_like(x)
+        out_dev = torch.empty(N, d, dtype=torch.float32, device=dev)
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            m.moe_layer(shape, x_dev, wr, bias, w1, w3, w2, out_dev, ws=lws, stream=stream)
+            out_host.copy_(out_dev, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_agg = aggregate(float(N * args.steps), e0.elapsed_time(e1) / 1e3, dev)
+        e2e = {"value": e2e_agg["value"], "unit": UNIT, "h2d_bytes_per_step": N * d * 2,
+               "d2h_bytes_per_step": N * d * 4}
+        del lws
+
+    work = algorithmic_work(w, R)
+    peaks = load_peaks()
+    up_s = stage_ms["expert_up"] / 1e3
+    down_s = stage_ms["expert_down"] / 1e3
+    up_tflops = work["up_flops"] / up_s / 1e12
+    gemm_tflops = (work["up_flops"] + work["down_flops"]) / (up_s + down_s) / 1e12
+    scat_gbs = None
+    stages = {k: round(v, 4) for k, v in stage_ms.items()}
+    hbm = peaks["hbm_gbs"]
+    comb_gbs = work["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": agg["value"],
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": agg["elapsed_max_s"] / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
+                "random-init weights)",
+        "config": {"workload": w.name, "N": N, "d": d, "f": f, "E": E, "K": K, "W": W,
+                   "capacity_factor": w.cf if w.cf > 0 else "dropless", "zipf_s": w.s,
+                   "rows_kept": R, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
+                         "weights streamed per step"},
+        "roofline": {"kernel": "grouped GEMM gate/up (moe_expert_up)", "bound": "tensor",
+                     "achieved": up_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": up_tflops / peaks["bf16_tflops"],
+                     "peak_source": peaks["source"] + " bf16 burst",
+                     "frac_of_sustained": up_tflops / peaks["bf16_tflops_sustained"],
+                     "traffic": up_traffic(w.name),
+                     "algorithmic_flops_per_launch": work["up_flops"]},
+        "stages_ms": stages,
+        "grouped_gemm": {"tflops": gemm_tflops, "frac_of_bf16_peak": gemm_tflops / peaks["bf16_tflops"],
+                         "frac_of_bf16_sustained": gemm_tflops / peaks["bf16_tflops_sustained"]},
+        "combine": {"gbs": comb_gbs, "frac_of_hbm": comb_gbs / hbm, "frac_of_8tbs": comb_gbs / 8000.0},
+        "dispatch": {"ms": stage_ms["dispatch"],
+                     "scatter_bytes": work["scatter_bytes"]},
+        "clocks": clocks.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+        "device_error": err,
+        "e2e": e2e,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_sample_tokens)
+    return res if rank == 0 else None
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "of measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "of fallback"}
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+
+def oracle_time(w, inp_cpu, sample_tokens: int) -> dict:
+    """Times the oracle on a bounded sample: routing + dispatch for every token,
+    expert FFN + combine for `sample_tokens` tokens; extrapolates to the layer."""
+    import numpy as np
+
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    r = oracle.route_and_dispatch(inp_cpu["x"], inp_cpu["w_router"], inp_cpu.get("bias"), w.K,
+                                  w.W, w.cf)
+    t_route = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(w.N, size=min(sample_tokens, w.N), replace=False))
+    t1 = time.perf_counter()
+    oracle.layer_sampled(inp_cpu, w.K, w.W, w.cf, toks, routing=r)
+    t_exp = time.perf_counter() - t1
+    t_full = t_route + t_exp * (w.N / len(toks))
+    return dict(value=w.N / t_full, t_route_s=t_route, t_expert_sample_s=t_exp,
+                sample_tokens=int(len(toks)), extrapolated_layer_s=t_full)
+
+
+def cpu_threads() -> int:
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def cpu_baseline(w, inp, sample_tokens: int) -> dict:
+    inp_cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    t = oracle_time(w, inp_cpu, sample_tokens)
+    return {"value": t["value"], "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"routing + dispatch for all {w.N} tokens; expert FFN + combine for "
+                      f"{t['sample_tokens']} tokens, extrapolated to {w.N} "
+                      f"(route {t['t_route_s']:.2f} s, experts {t['t_expert_sample_s']:.2f} s)"}
+
+
+def run_reference(args, w) -> dict:
+    import torch
+
+    from moe_workloads import make_layer_inputs
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    inp = make_layer_inputs(w, seed=args.seed, device="cpu")
+    times, values = [], []
+    for i in range(args.warmup + args.steps):
+        t = oracle_time(w, inp, args.ref_sample_tokens)
+        if i >= args.warmup:
+            times.append(t["extrapolated_layer_s"])
+            values.append(t["value"])
+    total = sum(times)
+    value = w.N * len(times) / total
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "impl": "reference",
+        "config": {"workload": w.name, "N": w.N, "d": w.d, "f": w.f, "E": w.E, "K": w.K,
+                   "W": w.W, "capacity_factor": w.cf if w.cf > 0 else "dropless"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"each step: routing + dispatch for all {w.N} tokens, expert "
+                                   f"FFN + combine for {args.ref_sample_tokens} tokens, "
+                                   f"extrapolated to {w.N}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del torch
+    return res
+
+
+# --------------------------------------------------------------------------- main
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mixtral_prefill")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=32)
+    ap.add_argument("--ref-sample-tokens", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    from moe_workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        res = run_reference(args, w)
+    else:
+        res = run_gpu(args, w)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+"""Python binding of the B200 MoE layer library (``libmoe_b200.so``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels. Torch tensors supply device memory and the current stream. The
+functions keep the C names of ``include/moe_b200.h``; each raises
+``MoeError`` on a non-OK status. There is no fallback: the first call raises
+``ImportError`` when the library has not been built
+(``python -m combine_grouped_gemm_router_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmoe_b200.so")
+
+
+c_i32, c_i64, c_u32, c_u64, c_f32 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                     ctypes.c_uint64, ctypes.c_float)
+c_size, c_p = ctypes.c_size_t, ctypes.c_void_p
+
+MOE_OK = 0
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_MISALIGNED", 5: "MOE_ERR_CUDA",
+    6: "MOE_ERR_DEVICE_TIMEOUT", 7: "MOE_ERR_NONFINITE", 8: "MOE_ERR_DEVICE_BOUNDS",
+}
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("N", c_i32), ("d", c_i32), ("f", c_i32), ("E", c_i32), ("K", c_i32),
+                ("W", c_i32), ("capacity_factor", c_f32), ("flags", c_u32)]
+
+
+class MoeStats(ctypes.Structure):
+    _fields_ = [("rows", c_i64), ("dropped", c_i64), ("cross_rows", c_i64),
+                ("dedup_pairs", c_i64), ("nonfinite_tokens", c_i64), ("capacity", c_i32),
+                ("active_experts", c_i32), ("max_kept", c_i32), ("min_kept", c_i32)]
+
+
+class MoeReport(ctypes.Structure):
+    _fields_ = [("drop_rate", ctypes.c_double), ("send_max_over_min", ctypes.c_double),
+                ("recv_max_over_min", ctypes.c_double), ("cross_rank_fraction", ctypes.c_double),
+                ("load_std_over_mean", ctypes.c_double),
+                ("capacity_factor_effective", ctypes.c_double), ("tau_min_tokens", c_i64),
+                ("dispatch_bytes", c_i64), ("send_max", c_i64), ("send_min", c_i64),
+                ("recv_max", c_i64), ("recv_min", c_i64)]
+
+
+_SP = ctypes.POINTER(MoeShape)
+_sigs = {
+    "moe_abi_version": ([], c_i32),
+    "moe_status_string": ([c_i32], ctypes.c_char_p),
+    "moe_capacity": ([_SP], c_i64),
+    "moe_rows_alloc": ([_SP], c_i64),
+    "moe_workspace_size": ([_SP], c_size),
+    "moe_layer_workspace_size": ([_SP], c_size),
+    "moe_route": ([_SP] + [c_p] * 7 + [c_size, c_p], c_i32),
+    "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
+    "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
+    "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
+    "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
+    "moe_combine": ([_SP] + [c_p] * 6, c_i32),
+    "moe_layer": ([_SP] + [c_p] * 11 + [c_size, c_p], c_i32),
+    "moe_affinity_accumulate": ([c_i32, c_i32, c_i32, c_p, c_p, c_p, c_p], c_i32),
+    "moe_derive_report": ([_SP, ctypes.POINTER(MoeStats), c_p, c_p, ctypes.POINTER(MoeReport)],
+                          c_i32),
+    "moe_get_device_error": ([ctypes.c_int], c_i32),
+    "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
+}
+
+
+class _Lib:
+    """Loads libmoe_b200.so on first use and declares every C signature."""
+
+    def __init__(self):
+        self._cdll = None
+
+    def _load(self):
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m combine_grouped_gemm_router_b200.build` (nvcc, sm_100a). "
+                "There is no CPU fallback.")
+        cdll = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _sigs.items():
+            fn = getattr(cdll, name)
+            fn.argtypes = args
+            fn.restype = res
+        self._cdll = cdll
+
+    def __getattr__(self, name):
+        if self._cdll is None:
+            self._load()
+        return getattr(self._cdll, name)
+
+
+_lib = _Lib()
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+MOE_FLAG_OUT_BF16 = 1
+
+
+def make_shape(N: int, d: int, f: int, E: int, K: int, W: int, capacity_factor: float = 0.0,
+               out_bf16: bool = False) -> MoeShape:
+    return MoeShape(N, d, f, E, K, W, float(capacity_factor),
+                    MOE_FLAG_OUT_BF16 if out_bf16 else 0)
+
+
+# ---------------------------------------------------------------- sizes
+
+def moe_abi_version() -> int:
+    return _lib.moe_abi_version()
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def moe_capacity(shape: MoeShape) -> int:
+    return _lib.moe_capacity(ctypes.byref(shape))
+
+
+def moe_rows_alloc(shape: MoeShape) -> int:
+    return _lib.moe_rows_alloc(ctypes.byref(shape))
+
+
+def moe_workspace_size(shape: MoeShape) -> int:
+    return _lib.moe_workspace_size(ctypes.byref(shape))
+
+
+def moe_layer_workspace_size(shape: MoeShape) -> int:
+    return _lib.moe_layer_workspace_size(ctypes.byref(shape))
+
+
+# ---------------------------------------------------------------- stages
+
+def moe_route(shape, x, w_router, bias, topk_idx, topk_w, logits=None, ws=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_route(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias),
+                          _ptr(topk_idx), _ptr(topk_w), _ptr(logits), _ptr(ws), ws_bytes,
+                          _stream(stream)), "moe_route")
+
+
+def moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_row, x_sorted,
+                 x_packed=None, rank_matrix=None, packed_offsets=None, stats=None, ws=None,
+                 stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_dispatch(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                             _ptr(kept), _ptr(offsets), _ptr(row_of), _ptr(assign_of_row),
+                             _ptr(x_sorted), _ptr(x_packed), _ptr(rank_matrix),
+                             _ptr(packed_offsets), _ptr(stats), _ptr(ws), ws_bytes,
+                             _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_gemm(shape, x_sorted, offsets, w1, w3, w2, h, y, stream=None):
+    _check(_lib.moe_expert_gemm(ctypes.byref(shape), _ptr(x_sorted), _ptr(offsets), _ptr(w1),
+                                _ptr(w3), _ptr(w2), _ptr(h), _ptr(y), _stream(stream)),
+           "moe_expert_gemm")
+
+
+def moe_expert_up(shape, x_sorted, offsets, w1, w3, h, stream=None):
+    _check(_lib.moe_expert_up(ctypes.byref(shape), _ptr(x_sorted), _ptr(offsets), _ptr(w1),
+                              _ptr(w3), _ptr(h), _stream(stream)), "moe_expert_up")
+
+
+def moe_expert_down(shape, h, offsets, w2, y, stream=None):
+    _check(_lib.moe_expert_down(ctypes.byref(shape), _ptr(h), _ptr(offsets), _ptr(w2), _ptr(y),
+                                _stream(stream)), "moe_expert_down")
+
+
+def moe_combine(shape, y, row_of, topk_w, out, residual=None, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(shape), _ptr(y), _ptr(row_of), _ptr(topk_w),
+                            _ptr(residual), _ptr(out), _stream(stream)), "moe_combine")
+
+
+def moe_layer(shape, x, w_router, bias, w1, w3, w2, out, residual=None, topk_idx_out=None,
+              stats=None, ws=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_layer(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
+                          _ptr(w3), _ptr(w2), _ptr(residual), _ptr(out), _ptr(topk_idx_out),
+                          _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)), "moe_layer")
+
+
+def moe_affinity_accumulate(N, E, K, topk_j, topk_j1, counts, stream=None):
+    _check(_lib.moe_affinity_accumulate(N, E, K, _ptr(topk_j), _ptr(topk_j1), _ptr(counts),
+                                        _stream(stream)), "moe_affinity_accumulate")
+
+
+# ---------------------------------------------------------------- host helpers
+
+def moe_derive_report(shape, stats: MoeStats, rank_matrix, kept) -> MoeReport:
+    """rank_matrix: host int64 [W*W] array-like; kept: host int32 [E]."""
+    import numpy as np
+    D = np.ascontiguousarray(rank_matrix, dtype=np.int64).reshape(-1)
+    k = np.ascontiguousarray(kept, dtype=np.int32).reshape(-1)
+    rep = MoeReport()
+    _check(_lib.moe_derive_report(ctypes.byref(shape), ctypes.byref(stats),
+                                  D.ctypes.data_as(c_p), k.ctypes.data_as(c_p),
+                                  ctypes.byref(rep)), "moe_derive_report")
+    return rep
+
+
+def moe_get_device_error(clear: bool = True) -> int:
+    """Status recorded by kernels on the current device (synchronises)."""
+    return _lib.moe_get_device_error(1 if clear else 0)
+
+
+def moe_debug_bounded_wait(timeout_ns: int, stream=None) -> None:
+    _check(_lib.moe_debug_bounded_wait(int(timeout_ns), _stream(stream)), "moe_debug_bounded_wait")
+
+
+def stats_buffer(device="cuda"):
+    """A device buffer of sizeof(moe_stats_t) bytes."""
+    import torch
+    return torch.zeros(ctypes.sizeof(MoeStats), dtype=torch.uint8, device=device)
+
+
+def read_stats(buf) -> MoeStats:
+    return MoeStats.from_buffer_copy(bytes(buf.to("cpu").numpy().tobytes()))
+
+
+def report_dict(rep: MoeReport) -> dict:
+    return {name: getattr(rep, name) for name, _ in MoeReport._fields_}
+
+
+def stats_dict(st: MoeStats) -> dict:
+    return {name: getattr(st, name) for name, _ in MoeStats._fields_}

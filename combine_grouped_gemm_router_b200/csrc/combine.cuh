@@ -1,0 +1,159 @@
+// Weighted combine, inter-layer affinity counts, and the bounded-wait probe.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制, node I] weighted
+// merge of the K expert outputs back into the original token order;
+// [MoE 推理服务工程真相 2026, §2.2] a dropped slot's router output is zero.
+// One warp per token; each lane owns 16-byte column chunks; the K rows are
+// gathered (fp32 expert outputs) and accumulated in fp32 in slot order
+// k = 0..K-1. An optional bf16 residual row is added last, in fp32: the
+// inter-layer step of a stack of MoE layers, x_{j+1} = x_j + MoE_j(x_j). The
+// result is stored as fp32, or rounded once to bf16 (OUT_BF16).
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ row_of,
+                   const float *__restrict__ topk_w, const uint16_t *__restrict__ residual,
+                   int N, int d, int K, void *__restrict__ out)
+{
+    constexpr int U = 2;
+    const int lane = threadIdx.x & 31;
+    const int nvec = d >> 3;  // 8-column chunks
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const float4 *ysrc = reinterpret_cast<const float4 *>(y);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < N; t += nwarps) {
+        int r = -1;
+        float w = 0.0f;
+        if (lane < K) {
+            r = row_of[(size_t)t * K + lane];
+            w = topk_w[(size_t)t * K + lane];
+        }
+        // every lane runs every iteration: the shuffles below read lanes 0..K-1
+        for (int c0 = 0; c0 < nvec; c0 += 32 * U) {
+            const int c = c0 + lane;
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    acc[u][q] = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                const int rk = __shfl_sync(0xffffffffu, r, k);
+                const float wk = __shfl_sync(0xffffffffu, w, k);
+                if (rk < 0)
+                    continue;
+                float4 v[U][2];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (c + 32 * u < nvec) {
+                        v[u][0] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2];
+                        v[u][1] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2 + 1];
+                    }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (c + 32 * u < nvec) {
+                        const float f8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                             v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            acc[u][q] = __fmaf_rn(wk, f8[q], acc[u][q]);
+                    }
+                }
+            }
+            if (residual) {
+                const uint4 *rsrc = reinterpret_cast<const uint4 *>(residual);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (c + 32 * u < nvec) {
+                        const uint4 rv = rsrc[(size_t)t * nvec + c + 32 * u];
+                        const uint32_t q4[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            acc[u][2 * q] = __fadd_rn(acc[u][2 * q], bf16_lo(q4[q]));
+                            acc[u][2 * q + 1] = __fadd_rn(acc[u][2 * q + 1], bf16_hi(q4[q]));
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (c + 32 * u < nvec) {
+                    const size_t chunk = (size_t)t * nvec + c + 32 * u;
+                    if (OUT_BF16) {
+                        uint4 o;
+                        o.x = pack_bf16x2(acc[u][0], acc[u][1]);
+                        o.y = pack_bf16x2(acc[u][2], acc[u][3]);
+                        o.z = pack_bf16x2(acc[u][4], acc[u][5]);
+                        o.w = pack_bf16x2(acc[u][6], acc[u][7]);
+                        reinterpret_cast<uint4 *>(out)[chunk] = o;
+                    } else {
+                        float4 *o = reinterpret_cast<float4 *>(out) + chunk * 2;
+                        o[0] = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+                        o[1] = make_float4(acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+                    }
+                }
+            }
+        }
+    }
+}
+
+// [MoE Inference Communication, §ExFlow 核心发现：跨层专家亲和性] counts of
+// (expert i at layer j, expert p at layer j+1) over every token's top-K pairs.
+// Block-private shared counters when E*E fits, else global atomics.
+__global__ void __launch_bounds__(256)
+    affinity_kernel(const int32_t *__restrict__ a, const int32_t *__restrict__ b, int N, int E,
+                    int K, unsigned long long *__restrict__ cnt, int use_smem)
+{
+    extern __shared__ unsigned int s_cnt[];
+    if (use_smem) {
+        for (int i = threadIdx.x; i < E * E; i += blockDim.x)
+            s_cnt[i] = 0;
+        __syncthreads();
+    }
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < N; t += gridDim.x * blockDim.x) {
+        for (int k = 0; k < K; ++k) {
+            const int i = a[(size_t)t * K + k];
+            if ((unsigned)i >= (unsigned)E) {
+                set_dev_error(MOE_ERR_DEVICE_BOUNDS);
+                continue;
+            }
+            for (int q = 0; q < K; ++q) {
+                const int pe = b[(size_t)t * K + q];
+                if ((unsigned)pe >= (unsigned)E) {
+                    set_dev_error(MOE_ERR_DEVICE_BOUNDS);
+                    continue;
+                }
+                if (use_smem)
+                    atomicAdd(&s_cnt[i * E + pe], 1u);
+                else
+                    atomicAdd(&cnt[(size_t)i * E + pe], 1ull);
+            }
+        }
+    }
+    if (use_smem) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < E * E; i += blockDim.x)
+            if (s_cnt[i])
+                atomicAdd(&cnt[i], (unsigned long long)s_cnt[i]);
+    }
+}
+
+// A flag that no code ever sets: the bounded-wait probe waits on it.
+__device__ unsigned int g_never_set;
+
+__global__ void bounded_wait_probe_kernel(uint64_t timeout_ns)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (*reinterpret_cast<volatile unsigned int *>(&g_never_set) == 0u) {
+        if (global_timer_ns() - t0 > timeout_ns) {
+            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+            return;
+        }
+        __nanosleep(1000);
+    }
+}
+
+}  // namespace moe

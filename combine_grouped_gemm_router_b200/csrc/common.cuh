@@ -1,0 +1,84 @@
+// Device helpers shared by the kernels of the MoE layer (one translation unit:
+// moe_api.cu includes every .cuh).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_b200.h"
+
+namespace moe {
+
+// Sticky per-device error word: the first kernel-side error code wins.
+__device__ unsigned int g_dev_error;
+
+__device__ __forceinline__ void set_dev_error(unsigned int code)
+{
+    atomicCAS(&g_dev_error, 0u, code);
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// fp32 -> bf16 bits, round to nearest even (inputs here are finite or propagate NaN).
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu))
+        return 0x7fc0u;  // quiet NaN
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return u >> 16;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        T o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off)
+            v += o;
+    }
+    return v;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v)
+{
+#pragma unroll
+    for (int off = 16; off; off >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// Token block b of the dispatch: blocks never straddle a home-rank shard, so
+// per-shard prefix counts are available at block boundaries.
+// shard = b / bps, tokens [shard*S + (b%bps)*HB, min(... + HB, (shard+1)*S)).
+struct BlockMap {
+    int S;    // tokens per shard (N / W)
+    int bps;  // blocks per shard
+    int HB;   // tokens per block
+    __device__ __forceinline__ void range(int b, int &t0, int &t1) const
+    {
+        const int shard = b / bps;
+        const int j = b - shard * bps;
+        t0 = shard * S + j * HB;
+        t1 = min(t0 + HB, (shard + 1) * S);
+    }
+};
+
+}  // namespace moe

@@ -1,0 +1,466 @@
+// Ragged grouped GEMM of the SwiGLU experts on 5th-generation tensor cores.
+//
+// [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制] each card groups
+// its tokens by expert and runs a grouped GEMM over variable per-expert token
+// counts; [§容量因子、专家复制与 dropless 的取舍] dropless routing handles the
+// ragged counts directly with a grouped GEMM in a single call.
+//
+// Design (sm_100a):
+//  - persistent kernel, one CTA per SM, 6 warps: warp 0 issues TMA loads,
+//    warp 1 owns TMEM and issues tcgen05.mma, warps 2-5 are the epilogue
+//    (one TMEM lane quadrant each);
+//  - tile = 128 rows of one expert x BN output columns, K-steps of 64 bf16
+//    (one 128-byte swizzle atom), 4-stage shared-memory ring fed by TMA;
+//  - the fp32 accumulator lives in TMEM, double-buffered (2 x BN columns), so
+//    the epilogue of one tile overlaps the MMAs of the next;
+//  - the tile list is derived on device from the expert offsets: experts with
+//    no rows have no tiles, so their weights are never read;
+//  - tiles are ordered expert-major, then N-slab, then M (fastest): CTAs that
+//    run at the same time share one weight slab and one expert's rows in L2;
+//  - rows of a tile past the expert's end are computed (they are the next
+//    expert's rows or zero fill) but never stored.
+// Mode 0 (gate/up): the B tile stacks 128 rows of W1 and 128 rows of W3, one
+// N=256 MMA per K-step; the epilogue reads gate column c and up column 128+c
+// and writes h = silu(g) * u as bf16 (the next GEMM's operand). Mode 1 (down):
+// fp32 output straight from TMEM, so the combine sums unrounded expert outputs.
+//
+// Every mbarrier wait is bounded (globaltimer); a wait that runs out records
+// MOE_ERR_DEVICE_TIMEOUT, raises a CTA-wide abort flag, and every role drains
+// what it has in flight before TMEM is released.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;    // 16 KB
+constexpr int B_HALF_BYTES = 128 * BK * 2;  // 16 KB per 128-row B box
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int THREADS = 192;
+
+struct Args {
+    const int32_t *offsets;  // [E+1]
+    int E;
+    int n_tiles;         // N-slabs per expert
+    int k_blocks;        // K / 64
+    int b_rows;          // rows of one expert's B matrix (f for mode 0, d for mode 1)
+    int rows_alloc;      // rows of the A buffer
+    void *out;           // mode 0: bf16 h [rows_alloc][ldo]; mode 1: fp32 y [rows_alloc][ldo]
+    int ldo;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity` to complete. Gives up when the
+// CTA abort flag is raised (if honor_abort) or after timeout_ns, raising it.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint64_t timeout_ns, bool honor_abort = true)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (honor_abort && *abort_flag)
+            return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort_flag = 1;
+            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand in 128-byte swizzled atoms
+// (8 rows x 128 bytes, atoms 1024 bytes apart), tile base 1024-byte aligned.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr)
+{
+    uint64_t desc = 0;
+    desc |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address, 16-byte units
+    desc |= (uint64_t)1u << 16;                    // leading byte offset (unused: swizzled K-major)
+    desc |= (uint64_t)(1024u >> 4) << 32;          // stride byte offset: 8-row group pitch
+    desc |= (uint64_t)1u << 46;                    // descriptor version for sm_100
+    desc |= (uint64_t)2u << 61;                    // 128-byte swizzle
+    return desc;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulate, both K-major.
+__host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N)
+{
+    return (1u << 4)                          // D format: f32
+           | (1u << 7)                        // A format: bf16
+           | (1u << 10)                       // B format: bf16
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return g / (1.0f + __expf(-g)) * u;
+}
+
+// Tile index -> (expert, N-slab, M-tile). tile_start[e] = first tile of expert e.
+__device__ __forceinline__ void decode_tile(int tile, const int *tile_start, const int *mtiles,
+                                            int E, int n_tiles, int &e, int &n, int &m)
+{
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= tile)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    e = lo;
+    const int local = tile - tile_start[e];
+    const int mt = mtiles[e];
+    n = local / mt;
+    m = local - n * mt;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const Args args)
+{
+    static_assert(MODE == 0 ? BN == 256 : (BN == 128 || BN == 256), "tile shape");
+    constexpr int B_BYTES = BN * BK * 2;
+    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr uint32_t IDESC = instr_desc_bf16(BM, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *tile_start = reinterpret_cast<int *>(tmem_slot + 4);
+    int *mtiles = tile_start + (args.E + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t smem_base = smem_u32(smem);
+    const uint32_t bar_base = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES + s); };
+    auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + a); };
+    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
+    const uint32_t done_bar = bar_base + 8u * (2 * STAGES + 4);
+    const int E = args.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 4);
+        }
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        *abort_flag = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0) {
+        // per-expert M-tile counts and their prefix (in tiles, times n_tiles)
+        int carry = 0;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int mt = 0;
+            if (e < E) {
+                int rows = args.offsets[e + 1] - args.offsets[e];
+                rows = max(0, min(rows, args.rows_alloc));
+                mt = (rows + BM - 1) / BM;
+                mtiles[e] = mt;
+            }
+            const int incl = warp_incl_scan(mt);
+            if (e < E)
+                tile_start[e] = (carry + incl - mt) * args.n_tiles;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0)
+            tile_start[E] = carry * args.n_tiles;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_parity[STAGES];
+            bool issued[STAGES];
+            for (int s = 0; s < STAGES; ++s)
+                issued[s] = false;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                int e, n, m;
+                decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
+                const int row0 = args.offsets[e] + m * BM;
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_base + stage * STAGE_BYTES;
+                    const uint32_t b_dst = a_dst + A_BYTES;
+                    mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
+                    tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
+                    if (MODE == 0) {
+                        const int brow = e * args.b_rows + n * 128;
+                        tma_load_2d(b_dst, &tmB0, kb * BK, brow, full_bar(stage));
+                        tma_load_2d(b_dst + B_HALF_BYTES, &tmB1, kb * BK, brow, full_bar(stage));
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < BN / 128; ++h)
+                            tma_load_2d(b_dst + h * B_HALF_BYTES, &tmB0, kb * BK,
+                                        e * args.b_rows + n * BN + h * 128, full_bar(stage));
+                    }
+                    issued[stage] = true;
+                    last_parity[stage] = phase;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain: every issued copy has landed before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if (issued[s])
+                    mbar_wait(full_bar(s), last_parity[s], abort_flag, args.timeout_ns, false);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.timeout_ns))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < args.k_blocks; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + stage * STAGE_BYTES;
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr + k * 32),
+                                    smem_desc_sw128(b_addr + k * 32), IDESC,
+                                    (kb > 0 || k > 0) ? 1u : 0u);
+                    tc_commit(empty_bar(stage));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit(tfull_bar(acc));
+                acc ^= 1;
+                if (acc == 0)
+                    acc_phase ^= 1u;
+            }
+            // every MMA issued so far has completed before TMEM is released
+            tc_commit(done_bar);
+            mbar_wait(done_bar, 0, abort_flag, args.timeout_ns, false);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            int e, n, m;
+            decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
+            const int rows_e = args.offsets[e + 1] - args.offsets[e];
+            const int valid = min(BM, rows_e - m * BM);
+            const int row0 = args.offsets[e] + m * BM;
+            int ok = 0;
+            if (lane == 0)
+                ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            if (MODE == 0) {
+                uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)(row0 + r) * args.ldo;
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    uint32_t g[16], u[16];
+                    tmem_ld16(taddr + c, g);
+                    tmem_ld16(taddr + 128 + c, u);
+                    tmem_ld_wait();
+                    if (r < valid) {
+                        uint32_t p[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            p[j] = pack_bf16x2(
+                                silu_mul(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j])),
+                                silu_mul(__uint_as_float(g[2 * j + 1]),
+                                         __uint_as_float(u[2 * j + 1])));
+                        dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
+                        dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
+                    }
+                }
+            } else {
+                // fp32 output: the down projection is not rounded before the combine
+                float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
+                uint4 *dst = reinterpret_cast<uint4 *>(frow + n * BN);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v0[16], v1[16];
+                    tmem_ld16(taddr + c, v0);
+                    tmem_ld16(taddr + c + 16, v1);
+                    tmem_ld_wait();
+                    if (r < valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            dst[c / 4 + j] = make_uint4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2],
+                                                        v0[4 * j + 3]);
+                            dst[c / 4 + 4 + j] = make_uint4(v1[4 * j], v1[4 * j + 1],
+                                                            v1[4 * j + 2], v1[4 * j + 3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(tempty_bar(acc));
+            acc ^= 1;
+            if (acc == 0)
+                acc_phase ^= 1u;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+}
+
+template <int MODE, int BN>
+constexpr int smem_bytes(int E)
+{
+    return STAGES * (A_BYTES + BN * BK * 2) + 1024 /* alignment */ + 8 * (2 * STAGES + 5) +
+           16 + 8 * (E + 1) + 64;
+}
+
+}  // namespace gg
+}  // namespace moe

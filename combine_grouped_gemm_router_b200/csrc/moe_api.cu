@@ -1,0 +1,718 @@
+// C ABI of the MoE layer hot path (declarations and contracts: include/moe_b200.h).
+// Host side: argument checks, workspace carving, tensor maps, launches.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "grouped_gemm.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxE = 256;
+constexpr int kMaxK = 32;
+constexpr int kMaxW = 64;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s bound on any device-side wait
+
+inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+struct Geometry {
+    int64_t C;           // capacity as used by the kernels (<= N*K)
+    int64_t rows_alloc;  // min(N*K, E*C) + 128
+    int S, bps, nblk;    // dispatch blocks
+};
+
+int64_t capacity_of(const moe_shape_t *s)
+{
+    const int64_t NK = (int64_t)s->N * s->K;
+    if (!(s->capacity_factor > 0.0f))
+        return NK;
+    return (int64_t)ceil((double)s->capacity_factor * (double)s->N * (double)s->K / (double)s->E);
+}
+
+moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
+{
+    if (!s)
+        return MOE_ERR_INVALID_ARG;
+    if ((s->flags & ~(uint32_t)MOE_FLAG_OUT_BF16) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (s->N < 1 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (s->K > s->E || s->E % s->W != 0 || s->N % s->W != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (s->E > kMaxE || s->K > kMaxK || s->W > kMaxW || s->d % 8 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((int64_t)s->N * s->K >= (int64_t)1 << 31)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (gemm && (s->d % 128 != 0 || s->f < 128 || s->f % 128 != 0))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (g) {
+        const int64_t NK = (int64_t)s->N * s->K;
+        int64_t C = capacity_of(s);
+        if (C > NK)
+            C = NK;
+        g->C = C;
+        g->rows_alloc = (NK < (int64_t)s->E * C ? NK : (int64_t)s->E * C) + 128;
+        g->S = s->N / s->W;
+        g->bps = (g->S + kDispatchHB - 1) / kDispatchHB;
+        g->nblk = s->W * g->bps;
+    }
+    return MOE_OK;
+}
+
+// Route/dispatch scratch, carved in this order from the workspace.
+struct ScratchLayout {
+    size_t logits, blk, pk_base, D, pk_off, total;
+};
+
+ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
+{
+    ScratchLayout L;
+    size_t o = 0;
+    L.logits = o;
+    o = align_up(o + (size_t)s->N * s->E * 4);
+    L.blk = o;
+    o = align_up(o + (size_t)s->E * g.nblk * 4);
+    L.pk_base = o;
+    o = align_up(o + (size_t)s->E * s->W * 8);
+    L.D = o;
+    o = align_up(o + (size_t)s->W * s->W * 8);
+    L.pk_off = o;
+    o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
+    L.total = o;
+    return L;
+}
+
+// moe_layer: every intermediate, after the scratch.
+struct LayerLayout {
+    size_t topk_idx, topk_w, counts, kept, offsets, row_of, assign, x_sorted, x_packed, h, y,
+        nonfinite, total;
+};
+
+LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
+{
+    LayerLayout L;
+    const size_t NK = (size_t)s->N * s->K, RA = (size_t)g.rows_alloc;
+    size_t o = align_up(base);
+    L.topk_idx = o;
+    o = align_up(o + NK * 4);
+    L.topk_w = o;
+    o = align_up(o + NK * 4);
+    L.counts = o;
+    o = align_up(o + (size_t)s->E * 4);
+    L.kept = o;
+    o = align_up(o + (size_t)s->E * 4);
+    L.offsets = o;
+    o = align_up(o + ((size_t)s->E + 1) * 4);
+    L.row_of = o;
+    o = align_up(o + NK * 4);
+    L.assign = o;
+    o = align_up(o + RA * 4);
+    L.x_sorted = o;
+    o = align_up(o + RA * s->d * 2);
+    L.x_packed = o;
+    o = align_up(o + RA * s->d * 2);
+    L.h = o;
+    o = align_up(o + RA * (size_t)s->f * 2);
+    L.y = o;
+    o = align_up(o + RA * s->d * 4);
+    L.nonfinite = o;
+    o = align_up(o + 8);
+    L.total = o;
+    return L;
+}
+
+int num_sms()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+
+inline moe_status_t launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- route
+
+template <int TY, int TX, int TT, int TE>
+void launch_logits(const uint16_t *x, const float *wr, const float *bias, float *logits, int N,
+                   int d, int E, cudaStream_t st)
+{
+    constexpr int BT = TY * TT, BE = TX * TE;
+    dim3 grid((N + BT - 1) / BT, (E + BE - 1) / BE);
+    router_logits_kernel<TY, TX, TT, TE><<<grid, TY * TX, 0, st>>>(x, wr, bias, logits, N, d, E);
+}
+
+moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_router,
+                        const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+                        unsigned long long *nonfinite, cudaStream_t st)
+{
+    const int N = s->N, d = s->d, E = s->E;
+    if (N < 1024)
+        launch_logits<1, 32, 4, 1>(x, w_router, bias, logits, N, d, E, st);
+    else if (E <= 8)
+        launch_logits<32, 8, 4, 1>(x, w_router, bias, logits, N, d, E, st);
+    else if (E <= 16)
+        launch_logits<16, 16, 4, 1>(x, w_router, bias, logits, N, d, E, st);
+    else if (E <= 32)
+        launch_logits<16, 16, 4, 2>(x, w_router, bias, logits, N, d, E, st);
+    else
+        launch_logits<8, 16, 8, 4>(x, w_router, bias, logits, N, d, E, st);
+    topk_softmax_kernel<<<(N + 7) / 8, 256, 0, st>>>(logits, N, E, s->K, topk_idx, topk_w,
+                                                      nonfinite);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- dispatch
+
+size_t scan_smem_bytes(const moe_shape_t *s)
+{
+    const int E = s->E, W = s->W;
+    const int scan_len = (E > W * W ? E : W * W) + 1;
+    return (size_t)scan_len * 8 + (size_t)W * W * 8 + 32 * 8 + (size_t)E * (W + 1) * 4;
+}
+
+moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x,
+                           const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                           int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                           uint16_t *x_sorted, uint16_t *x_packed, int64_t *D, int64_t *pk_off,
+                           moe_stats_t *stats, int32_t *blk, int64_t *pk_base, cudaStream_t st)
+{
+    BlockMap bm{g.S, g.bps, kDispatchHB};
+    block_hist_kernel<<<g.nblk, 256, s->E * 4, st>>>(topk_idx, s->K, s->E, bm, g.nblk, blk);
+
+    ScanArgs sa;
+    sa.blk = blk;
+    sa.nblk = g.nblk;
+    sa.bm = bm;
+    sa.N = s->N;
+    sa.E = s->E;
+    sa.K = s->K;
+    sa.W = s->W;
+    sa.C = (int)g.C;
+    sa.counts = counts;
+    sa.kept = kept;
+    sa.offsets = offsets;
+    sa.D = D;
+    sa.pk_off = pk_off;
+    sa.pk_base = pk_base;
+    sa.stats = stats;
+    const size_t scan_smem = scan_smem_bytes(s);
+    static std::once_flag scan_attr;
+    std::call_once(scan_attr, [] {
+        cudaFuncSetAttribute(dispatch_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024);
+    });
+    dispatch_scan_kernel<<<1, 1024, scan_smem, st>>>(sa);
+
+    PosArgs pa;
+    pa.topk_idx = topk_idx;
+    pa.blk = blk;
+    pa.nblk = g.nblk;
+    pa.bm = bm;
+    pa.N = s->N;
+    pa.E = s->E;
+    pa.K = s->K;
+    pa.W = s->W;
+    pa.C = (int)g.C;
+    pa.offsets = offsets;
+    pa.row_of = row_of;
+    pa.assign_of_row = assign_of_row;
+    pa.stats = stats;
+    const size_t pos_smem = (size_t)9 * s->E * 4 + (size_t)kDispatchHB * s->K;
+    dispatch_positions_kernel<<<g.nblk, 256, pos_smem, st>>>(pa);
+
+    ScatterArgs ca;
+    ca.x = x;
+    ca.topk_idx = topk_idx;
+    ca.row_of = row_of;
+    ca.offsets = offsets;
+    ca.pk_base = pk_base;
+    ca.N = s->N;
+    ca.d = s->d;
+    ca.K = s->K;
+    ca.W = s->W;
+    ca.E = s->E;
+    ca.S = g.S;
+    ca.x_sorted = x_sorted;
+    ca.x_packed = x_packed;
+    scatter_rows_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- expert GEMMs
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor [rows][inner], box 128 rows x 64 elements, 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {(cuuint32_t)gg::BK, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int BN>
+moe_status_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1,
+                         const gg::Args &args, cudaStream_t st)
+{
+    const int smem = gg::smem_bytes<MODE, BN>(kMaxE);
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(gg::grouped_gemm_kernel<MODE, BN>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (attr_err != cudaSuccess)
+        return MOE_ERR_CUDA;
+    gg::grouped_gemm_kernel<MODE, BN><<<num_sms(), gg::THREADS, smem, st>>>(a, b0, b1, args);
+    return launch_status();
+}
+
+moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
+                            const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
+                            uint16_t *h, cudaStream_t st)
+{
+    const int d = s->d, f = s->f, E = s->E;
+    CUtensorMap tA, tW1, tW3;
+    if (!make_tmap(&tA, x_sorted, d, g.rows_alloc) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
+        !make_tmap(&tW3, w3, d, (uint64_t)E * f))
+        return MOE_ERR_CUDA;
+    gg::Args a;
+    a.offsets = offsets;
+    a.E = E;
+    a.n_tiles = f / 128;
+    a.k_blocks = d / gg::BK;
+    a.b_rows = f;
+    a.rows_alloc = (int)g.rows_alloc;
+    a.out = h;
+    a.ldo = f;
+    a.timeout_ns = kWaitTimeoutNs;
+    return launch_gemm<0, 256>(tA, tW1, tW3, a, st);
+}
+
+moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *h,
+                              const int32_t *offsets, const uint16_t *w2, float *y,
+                              cudaStream_t st)
+{
+    const int d = s->d, f = s->f, E = s->E;
+    CUtensorMap tA, tW2;
+    if (!make_tmap(&tA, h, f, g.rows_alloc) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
+        return MOE_ERR_CUDA;
+    gg::Args a;
+    a.offsets = offsets;
+    a.E = E;
+    a.k_blocks = f / gg::BK;
+    a.b_rows = d;
+    a.rows_alloc = (int)g.rows_alloc;
+    a.out = y;
+    a.ldo = d;
+    a.timeout_ns = kWaitTimeoutNs;
+    if (d % 256 == 0) {
+        a.n_tiles = d / 256;
+        return launch_gemm<1, 256>(tA, tW2, tW2, a, st);
+    }
+    a.n_tiles = d / 128;
+    return launch_gemm<1, 128>(tA, tW2, tW2, a, st);
+}
+
+moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
+                              const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
+                              const uint16_t *w2, uint16_t *h, float *y, cudaStream_t st)
+{
+    moe_status_t rc = expert_up_impl(s, g, x_sorted, offsets, w1, w3, h, st);
+    if (rc != MOE_OK)
+        return rc;
+    return expert_down_impl(s, g, h, offsets, w2, y, st);
+}
+
+moe_status_t combine_impl(const moe_shape_t *s, const float *y, const int32_t *row_of,
+                          const float *topk_w, const uint16_t *residual, void *out,
+                          cudaStream_t st)
+{
+    if (s->flags & MOE_FLAG_OUT_BF16)
+        combine_kernel<true><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, residual, s->N,
+                                                              s->d, s->K, out);
+    else
+        combine_kernel<false><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, residual, s->N,
+                                                               s->d, s->K, out);
+    return launch_status();
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+
+extern "C" {
+
+__attribute__((visibility("default"))) int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+__attribute__((visibility("default"))) const char *moe_status_string(moe_status_t st)
+{
+    switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_MISALIGNED: return "MOE_ERR_MISALIGNED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+    case MOE_ERR_NONFINITE: return "MOE_ERR_NONFINITE";
+    case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+__attribute__((visibility("default"))) int64_t moe_capacity(const moe_shape_t *shape)
+{
+    if (!shape)
+        return -1;
+    return capacity_of(shape);
+}
+
+__attribute__((visibility("default"))) int64_t moe_rows_alloc(const moe_shape_t *shape)
+{
+    Geometry g;
+    if (check_shape(shape, false, &g) != MOE_OK)
+        return -1;
+    return g.rows_alloc;
+}
+
+__attribute__((visibility("default"))) size_t moe_workspace_size(const moe_shape_t *shape)
+{
+    Geometry g;
+    if (check_shape(shape, false, &g) != MOE_OK)
+        return 0;
+    return scratch_layout(shape, g).total;
+}
+
+__attribute__((visibility("default"))) size_t moe_layer_workspace_size(const moe_shape_t *shape)
+{
+    Geometry g;
+    if (check_shape(shape, true, &g) != MOE_OK)
+        return 0;
+    return layer_layout(shape, g, scratch_layout(shape, g).total).total;
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router, const float *bias,
+          int32_t *topk_idx, float *topk_w, float *logits, void *ws, size_t ws_bytes,
+          moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, false, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x || !w_router || !topk_idx || !topk_w)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) ||
+        !aligned4(topk_idx) || !aligned4(topk_w) || (logits && !aligned4(logits)))
+        return MOE_ERR_MISALIGNED;
+    if (!logits) {
+        const ScratchLayout L = scratch_layout(shape, g);
+        if (!ws || ws_bytes < L.total)
+            return MOE_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(ws))
+            return MOE_ERR_MISALIGNED;
+        logits = reinterpret_cast<float *>(static_cast<char *>(ws) + L.logits);
+    }
+    return route_impl(shape, x, w_router, bias, topk_idx, topk_w, logits, nullptr,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx, int32_t *counts,
+             int32_t *kept, int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+             uint16_t *x_sorted, uint16_t *x_packed, int64_t *rank_matrix,
+             int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
+             moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, false, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_sorted) || (x_packed && !aligned16(x_packed)) ||
+        !aligned4(topk_idx) || !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) ||
+        !aligned4(row_of) || !aligned4(assign_of_row) ||
+        (rank_matrix && (reinterpret_cast<uintptr_t>(rank_matrix) & 7u)) ||
+        (packed_offsets && (reinterpret_cast<uintptr_t>(packed_offsets) & 7u)) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const ScratchLayout L = scratch_layout(shape, g);
+    if (!ws || ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    char *w = static_cast<char *>(ws);
+    int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
+    int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
+    return dispatch_impl(shape, g, x, topk_idx, counts, kept, offsets, row_of, assign_of_row,
+                         x_sorted, x_packed, D, pk, stats, reinterpret_cast<int32_t *>(w + L.blk),
+                         reinterpret_cast<int64_t *>(w + L.pk_base),
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_t *offsets,
+                const uint16_t *w1, const uint16_t *w3, const uint16_t *w2, uint16_t *h,
+                float *y, moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x_sorted || !offsets || !w1 || !w3 || !w2 || !h || !y)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_sorted) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
+        !aligned16(h) || !aligned16(y) || !aligned4(offsets))
+        return MOE_ERR_MISALIGNED;
+    return expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_t *offsets,
+              const uint16_t *w1, const uint16_t *w3, uint16_t *h, moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x_sorted || !offsets || !w1 || !w3 || !h)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_sorted) || !aligned16(w1) || !aligned16(w3) || !aligned16(h) ||
+        !aligned4(offsets))
+        return MOE_ERR_MISALIGNED;
+    return expert_up_impl(shape, g, x_sorted, offsets, w1, w3, h,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
+                const uint16_t *w2, float *y, moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!h || !offsets || !w2 || !y)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(w2) || !aligned16(y) || !aligned4(offsets))
+        return MOE_ERR_MISALIGNED;
+    return expert_down_impl(shape, g, h, offsets, w2, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
+            const float *topk_w, const uint16_t *residual, void *out, moe_stream_t stream)
+{
+    moe_status_t rc = check_shape(shape, false, nullptr);
+    if (rc != MOE_OK)
+        return rc;
+    if (!y || !row_of || !topk_w || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out) || !aligned4(row_of) || !aligned4(topk_w) ||
+        (residual && !aligned16(residual)))
+        return MOE_ERR_MISALIGNED;
+    return combine_impl(shape, y, row_of, topk_w, residual, out,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, const float *bias,
+          const uint16_t *w1, const uint16_t *w3, const uint16_t *w2, const uint16_t *residual,
+          void *out, int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
+          moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x || !w_router || !w1 || !w3 || !w2 || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1) ||
+        !aligned16(w3) || !aligned16(w2) || !aligned16(out) ||
+        (residual && !aligned16(residual)) || (topk_idx_out && !aligned4(topk_idx_out)) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const ScratchLayout S = scratch_layout(shape, g);
+    const LayerLayout L = layer_layout(shape, g, S.total);
+    if (!ws || ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    int32_t *topk_idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(w + L.topk_idx);
+    float *topk_w = reinterpret_cast<float *>(w + L.topk_w);
+    unsigned long long *nonfinite = nullptr;
+    if (stats) {
+        nonfinite = reinterpret_cast<unsigned long long *>(&stats->nonfinite_tokens);
+        if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
+                    reinterpret_cast<float *>(w + S.logits), nonfinite, st);
+    if (rc != MOE_OK)
+        return rc;
+    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+    int32_t *row_of = reinterpret_cast<int32_t *>(w + L.row_of);
+    uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
+    uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
+    float *y = reinterpret_cast<float *>(w + L.y);
+    rc = dispatch_impl(shape, g, x, topk_idx, reinterpret_cast<int32_t *>(w + L.counts),
+                       reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
+                       reinterpret_cast<int32_t *>(w + L.assign), x_sorted,
+                       reinterpret_cast<uint16_t *>(w + L.x_packed),
+                       reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
+                       stats, reinterpret_cast<int32_t *>(w + S.blk),
+                       reinterpret_cast<int64_t *>(w + S.pk_base), st);
+    if (rc != MOE_OK)
+        return rc;
+    rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
+    if (rc != MOE_OK)
+        return rc;
+    return combine_impl(shape, y, row_of, topk_w, residual, out, st);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_affinity_accumulate(int32_t N, int32_t E, int32_t K, const int32_t *topk_j,
+                        const int32_t *topk_j1, int64_t *counts, moe_stream_t stream)
+{
+    if (N < 1 || E < 1 || K < 1 || K > E || !topk_j || !topk_j1 || !counts)
+        return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || K > kMaxK)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned4(topk_j) || !aligned4(topk_j1) || (reinterpret_cast<uintptr_t>(counts) & 7u))
+        return MOE_ERR_MISALIGNED;
+    const int use_smem = E <= 64 ? 1 : 0;
+    const int threads = 256;
+    int blocks = (N + threads - 1) / threads;
+    if (blocks > 4 * num_sms())
+        blocks = 4 * num_sms();
+    affinity_kernel<<<blocks, threads, use_smem ? (size_t)E * E * 4 : 0,
+                      reinterpret_cast<cudaStream_t>(stream)>>>(
+        topk_j, topk_j1, N, E, K, reinterpret_cast<unsigned long long *>(counts), use_smem);
+    return launch_status();
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_derive_report(const moe_shape_t *shape, const moe_stats_t *st, const int64_t *D,
+                  const int32_t *kept, moe_report_t *out)
+{
+    if (check_shape(shape, false, nullptr) != MOE_OK)
+        return MOE_ERR_INVALID_ARG;
+    if (!st || !D || !kept || !out)
+        return MOE_ERR_INVALID_ARG;
+    const int W = shape->W, E = shape->E;
+    const double NK = (double)shape->N * shape->K;
+    int64_t smax = 0, smin = INT64_MAX, rmax = 0, rmin = INT64_MAX, off_row = 0, off_col = 0;
+    double mean = 0.0;
+    for (int i = 0; i < W; ++i) {
+        int64_t s = 0, r = 0, so = 0, ro = 0;
+        for (int j = 0; j < W; ++j) {
+            s += D[i * W + j];
+            r += D[j * W + i];
+            if (j != i) {
+                so += D[i * W + j];
+                ro += D[j * W + i];
+            }
+        }
+        smax = s > smax ? s : smax;
+        smin = s < smin ? s : smin;
+        rmax = r > rmax ? r : rmax;
+        rmin = r < rmin ? r : rmin;
+        off_row = so > off_row ? so : off_row;
+        off_col = ro > off_col ? ro : off_col;
+        mean += (double)r;
+    }
+    mean /= W;
+    double var = 0.0;
+    for (int j = 0; j < W; ++j) {
+        int64_t r = 0;
+        for (int i = 0; i < W; ++i)
+            r += D[i * W + j];
+        var += ((double)r - mean) * ((double)r - mean);
+    }
+    var /= W;
+    int32_t kmax = 0;
+    for (int e = 0; e < E; ++e)
+        kmax = kept[e] > kmax ? kept[e] : kmax;
+    out->drop_rate = (double)st->dropped / NK;
+    out->send_max_over_min = smin > 0 ? (double)smax / (double)smin : INFINITY;
+    out->recv_max_over_min = rmin > 0 ? (double)rmax / (double)rmin : INFINITY;
+    out->cross_rank_fraction = st->rows > 0 ? (double)st->cross_rows / (double)st->rows : 0.0;
+    out->load_std_over_mean = mean > 0 ? sqrt(var) / mean : 0.0;
+    out->capacity_factor_effective = (double)kmax / (NK / (double)E);
+    out->tau_min_tokens = off_row > off_col ? off_row : off_col;
+    out->dispatch_bytes = st->rows * (int64_t)shape->d * 2;
+    out->send_max = smax;
+    out->send_min = smin;
+    out->recv_max = rmax;
+    out->recv_min = rmin;
+    return MOE_OK;
+}
+
+__attribute__((visibility("default"))) moe_status_t moe_get_device_error(int clear)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return MOE_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_dev_error, sizeof v) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (clear) {
+        const unsigned int z = 0;
+        if (cudaMemcpyToSymbol(g_dev_error, &z, sizeof z) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    return (moe_status_t)v;
+}
+
+__attribute__((visibility("default"))) moe_status_t moe_debug_bounded_wait(uint64_t timeout_ns,
+                                                                           moe_stream_t stream)
+{
+    if (timeout_ns == 0 || timeout_ns > 10ull * 1000000000ull)
+        return MOE_ERR_INVALID_ARG;
+    bounded_wait_probe_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,250 @@
+/*
+ * moe_b200.h — C ABI of the single-GPU MoE FFN layer hot path for B200 (sm_100a):
+ *
+ *   route (router projection + softmax top-K)
+ *   -> dispatch (per-expert histogram, prefix scan, capacity drop, scatter into an
+ *      expert-contiguous buffer and a per-EP-rank packed buffer)
+ *   -> expert GEMMs (ragged grouped GEMM, SwiGLU experts, tcgen05 tensor cores)
+ *   -> combine (weighted un-permute back to token order)
+ *
+ * The dataflow is the one of "MoE 专家并行的 All-to-All 通信瓶颈：专家越多推理延迟为何
+ * 反而上升", §All-to-All 分发与回收的机制 (its flowchart: route Top-K, pack by
+ * destination card, exchange, group by expert, grouped GEMM, pack by source, exchange,
+ * weighted merge into the original token order), with the two exchanges replaced by an
+ * emulation of W virtual expert-parallel ranks inside one GPU's memory.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller, except where a comment
+ *    says HOST. bf16 arrays are passed as uint16_t bit patterns. Row-major layouts.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream). The library never allocates or frees device memory; scratch comes from a
+ *    caller workspace of at least the size the matching *_workspace_size function returns.
+ *  - Argument errors are detected on the host and returned before anything is launched.
+ *    Errors found by kernels (non-finite logits, out-of-range expert ids, a bounded wait
+ *    that ran out) are recorded in a sticky per-device error word that
+ *    moe_get_device_error() reads. No call throws; none synchronises unless it says so.
+ *  - Pointers to bf16 or fp32 arrays must be 16-byte aligned (MOE_ERR_MISALIGNED).
+ *
+ * Notation (kept from the pages): N tokens, d hidden size, f expert FFN width, E experts,
+ * K experts per token, W virtual EP ranks, cf capacity factor, C = ceil(cf*N*K/E) the
+ * per-expert capacity, R the number of kept (token, slot) assignments (rows).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *moe_stream_t; /* identical to cudaStream_t */
+
+#define MOE_ABI_VERSION 1
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,         /* null pointer, K > E, E % W != 0, N % W != 0, ... */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* a size outside the limits listed at moe_shape_t */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the *_workspace_size() value */
+    MOE_ERR_MISALIGNED = 4,          /* a pointer not 16-byte aligned */
+    MOE_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait gave up */
+    MOE_ERR_NONFINITE = 7,           /* a router logit was NaN or infinite */
+    MOE_ERR_DEVICE_BOUNDS = 8        /* an expert id outside [0, E) reached a kernel */
+} moe_status_t;
+
+/* Problem description. Limits: 1 <= N, N*K < 2^31; d % 8 == 0 (d % 128 == 0 for
+ * moe_expert_gemm / moe_layer); f % 128 == 0 for the GEMMs; 1 <= E <= 256;
+ * 1 <= K <= min(E, 32); 1 <= W <= 64, E % W == 0, N % W == 0.
+ * capacity_factor <= 0 selects dropless routing. */
+typedef struct moe_shape {
+    int32_t N, d, f, E, K, W;
+    float capacity_factor;
+    uint32_t flags; /* 0 or MOE_FLAG_OUT_BF16; other bits must be 0 */
+} moe_shape_t;
+
+/* moe_combine / moe_layer write `out` as bf16 (one rounding of the fp32 sum) instead of the
+ * default fp32. Meant for a stack of layers whose next input is bf16. */
+#define MOE_FLAG_OUT_BF16 1u
+
+/* Per-call dispatch counters, written (not accumulated) by moe_dispatch / moe_layer into
+ * DEVICE memory when a non-null pointer is given. Observability signals of
+ * "MoE 专家并行的 All-to-All 通信瓶颈", §可观测指标与故障定位, and
+ * "MoE 推理服务工程真相 2026", §5.1 (token_drop_count, overflow). */
+typedef struct moe_stats {
+    int64_t rows;             /* R = kept assignments */
+    int64_t dropped;          /* N*K - R (assignments over capacity) */
+    int64_t cross_rows;       /* kept rows whose expert rank differs from the token's home rank */
+    int64_t dedup_pairs;      /* distinct (token, destination rank != home) pairs over kept rows:
+                                 what an exchange that sends a token once per rank would carry */
+    int64_t nonfinite_tokens; /* tokens with a non-finite logit (moe_layer only; else 0) */
+    int32_t capacity;         /* C (N*K when dropless) */
+    int32_t active_experts;   /* experts with at least one kept row */
+    int32_t max_kept;         /* max_e kept[e] */
+    int32_t min_kept;         /* min_e kept[e] */
+} moe_stats_t;
+
+/* Host-side report derived from moe_stats_t, the traffic matrix D and kept[]. */
+typedef struct moe_report {
+    double drop_rate;                 /* dropped / (N*K) */
+    double send_max_over_min;         /* per-rank send (row sums of D): max / min (inf if min 0) */
+    double recv_max_over_min;         /* per-rank receive (column sums of D): max / min */
+    double cross_rank_fraction;       /* cross_rows / rows */
+    double load_std_over_mean;        /* population std / mean of per-rank receive */
+    double capacity_factor_effective; /* max_e kept[e] / (N*K/E) */
+    int64_t tau_min_tokens;           /* max(max off-diagonal row sum, max column sum) of D */
+    int64_t dispatch_bytes;           /* rows * d * 2 (bf16 payload of one dispatch) */
+    int64_t send_max, send_min, recv_max, recv_min;
+} moe_report_t;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Capacity C = ceil(cf * N * K / E) computed in double; N*K when dropless. Returns -1 on a
+ * null shape. [MoE 推理服务工程真相 2026, §2.2 Expert Capacity Factor] */
+int64_t moe_capacity(const moe_shape_t *shape);
+
+/* Rows to allocate for every row-indexed buffer (assign_of_row, x_sorted, x_packed, h, y):
+ * min(N*K, E*C) + 128. The 128 spare rows let the GEMM read whole 128-row tiles past the
+ * last expert. Returns -1 on an invalid shape. */
+int64_t moe_rows_alloc(const moe_shape_t *shape);
+
+/* Workspace bytes for moe_route (logit scratch when logits == NULL) and moe_dispatch
+ * (block histograms, pack bases). 0 on an invalid shape. */
+size_t moe_workspace_size(const moe_shape_t *shape);
+
+/* Workspace bytes for moe_layer: every intermediate of the layer plus the scratch above. */
+size_t moe_layer_workspace_size(const moe_shape_t *shape);
+
+/* ---------------------------------------------------------------- stages */
+
+/* Router projection and softmax top-K.
+ * [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化: gate top-k fused in one
+ *  kernel; §Aurora, gate term G_i of the per-layer time model]
+ * x [N][d] bf16; w_router [E][d] fp32; bias [E] fp32 or NULL (added to every logit).
+ * logits[t][e] = (sum over i ascending of one fp32 fused multiply-add x[t][i]*Wr[e][i],
+ * starting from +0) + bias[e]: bit-identical to any IEEE implementation of that order.
+ * topk_idx [N][K] int32: the K largest logits, larger first, equal logits to the lower
+ * expert index. topk_w [N][K] fp32: softmax over the K selected logits.
+ * logits [N][E] fp32 or NULL (then written to the workspace). A non-finite logit sets
+ * MOE_ERR_NONFINITE in the device error word; that token's result is unspecified. */
+moe_status_t moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
+                       const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+                       void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Dispatch permutation.
+ * [MoE 推理服务工程真相 2026, §2.3 moe_dispatch pseudo-code: bincount of expert ids,
+ *  overflow beyond capacity; §2.2: overflow dropped; MoE Inference Communication,
+ *  §MoE 计算核优化: cumsum + scatter through a dense mapping table;
+ *  MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制: pack by destination]
+ * Assignments a = t*K + k are taken in increasing a; an assignment is kept iff fewer than C
+ * earlier assignments chose the same expert.
+ *  counts [E]: assignments per expert; kept [E] = min(counts, C);
+ *  offsets [E+1]: exclusive scan of kept (offsets[E] = R);
+ *  row_of [N*K]: offsets[e] + position, or -1 when dropped;
+ *  assign_of_row [rows_alloc]: inverse of row_of on its first R entries;
+ *  x_sorted [rows_alloc][d] bf16: x_sorted[row_of[a]] = x[a / K] (rows of one expert in
+ *  increasing token order);
+ *  x_packed [rows_alloc][d] bf16 or NULL: the same rows in blocks (home rank i, expert
+ *  rank j), blocks row-major, rows inside a block ordered by (expert, token); expert e is on
+ *  rank e / (E/W), token t's home is t / (N/W);
+ *  rank_matrix [W][W] int64 or NULL: D[i][j] = kept rows from home i to rank j;
+ *  packed_offsets [W*W+1] int64 or NULL: exclusive scan of D (block starts in x_packed);
+ *  stats: DEVICE moe_stats_t or NULL.
+ * topk_idx entries outside [0, E) set MOE_ERR_DEVICE_BOUNDS and are treated as dropped. */
+moe_status_t moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx,
+                          int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of,
+                          int32_t *assign_of_row, uint16_t *x_sorted, uint16_t *x_packed,
+                          int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
+                          void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Ragged grouped GEMM of the SwiGLU experts, one persistent launch per GEMM.
+ * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (grouped GEMM over
+ *  variable per-expert token counts) and §容量因子、专家复制与 dropless 的取舍 (dropless
+ *  grouped GEMM in a single call)]
+ * For every expert e and every row r in [offsets[e], offsets[e+1]):
+ *   h[r] = silu(x_sorted[r] W1[e]^T) * (x_sorted[r] W3[e]^T)   (bf16 out, fp32 accumulate)
+ *   y[r] = h[r] W2[e]^T                                         (fp32 out, fp32 accumulate)
+ * x_sorted [rows_alloc][d], w1, w3 [E][f][d], w2 [E][d][f], h [rows_alloc][f] bf16;
+ * y [rows_alloc][d] fp32; offsets [E+1] device int32 (as written by moe_dispatch).
+ * h is bf16 because it is the second GEMM's tensor-core operand; y stays fp32 so the
+ * combine adds unrounded expert outputs.
+ * Rows past offsets[E] are neither read for output nor written. Experts with no rows cost
+ * nothing (their weights are not read). Needs d % 128 == 0, f % 128 == 0. */
+moe_status_t moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted,
+                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
+                             const uint16_t *w2, uint16_t *h, float *y, moe_stream_t stream);
+
+/* The two halves of moe_expert_gemm as separate launches (same contracts as above):
+ * moe_expert_up:   h = silu(x_sorted W1^T) * (x_sorted W3^T)   (gate/up GEMM, bf16 h)
+ * moe_expert_down: y = h W2^T                                  (down GEMM, fp32 y) */
+moe_status_t moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted,
+                           const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
+                           uint16_t *h, moe_stream_t stream);
+moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
+                             const uint16_t *w2, float *y, moe_stream_t stream);
+
+/* Weighted combine back to token order.
+ * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (weighted merge into the
+ *  original token order, then on to the next layer); MoE 推理服务工程真相 2026, §2.2 (a
+ *  dropped slot contributes 0)]
+ * out[t] = (sum over k = 0..K-1 with row_of[t*K+k] >= 0 of topk_w[t][k] * y[row])
+ *          + residual[t], accumulated in fp32 in k order, the residual (nullable, bf16
+ * [N][d]) added last. y [rows_alloc][d] fp32. out [N][d] is fp32, or bf16 (rounded once)
+ * when shape->flags has MOE_FLAG_OUT_BF16; a bf16 out may alias residual. */
+moe_status_t moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
+                         const float *topk_w, const uint16_t *residual, void *out,
+                         moe_stream_t stream);
+
+/* The whole layer: moe_route -> moe_dispatch (with the packed buffer) -> moe_expert_gemm ->
+ * moe_combine, every intermediate in the workspace (moe_layer_workspace_size bytes).
+ * residual (nullable) is added in the combine (pass x for x + MoE(x)); out [N][d] is fp32,
+ * or bf16 with MOE_FLAG_OUT_BF16, and must not alias x. topk_idx_out [N][K] (nullable)
+ * receives the routing; stats (nullable, DEVICE) the counters. */
+moe_status_t moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
+                       const float *bias, const uint16_t *w1, const uint16_t *w3,
+                       const uint16_t *w2, const uint16_t *residual, void *out,
+                       int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* Inter-layer expert affinity counts, accumulated into counts [E][E] int64:
+ * for every token t, i in topk_j[t], p in topk_j1[t]: counts[i][p] += 1.
+ * P(E_p at layer j+1 | E_i at layer j) = counts[i][p] / (tokens with i in topk_j).
+ * [MoE Inference Communication, §ExFlow 核心发现：跨层专家亲和性] */
+moe_status_t moe_affinity_accumulate(int32_t N, int32_t E, int32_t K, const int32_t *topk_j,
+                                     const int32_t *topk_j1, int64_t *counts,
+                                     moe_stream_t stream);
+
+/* ---------------------------------------------------------------- host-side helpers */
+
+/* Derived observability report. HOST pointers: stats (a copy of the device struct),
+ * rank_matrix [W][W], kept [E]. Pure host computation; needs no GPU.
+ * [MoE 专家并行的 All-to-All 通信瓶颈, §可观测指标与故障定位; MoE 推理服务工程真相 2026,
+ *  §5.1; MoE Inference Communication, §Aurora 定理 4.2 (tau_min = max row/column sum of
+ *  the traffic matrix, here in tokens and without the local diagonal)] */
+moe_status_t moe_derive_report(const moe_shape_t *shape, const moe_stats_t *stats,
+                               const int64_t *rank_matrix, const int32_t *kept,
+                               moe_report_t *out);
+
+/* Reads (and, if clear != 0, resets) the calling device's sticky error word. Synchronises
+ * the device. Returns MOE_OK when no kernel has recorded an error. */
+moe_status_t moe_get_device_error(int clear);
+
+/* Launches one kernel whose only work is a bounded wait on a flag that nothing sets; it gives
+ * up after timeout_ns nanoseconds and records MOE_ERR_DEVICE_TIMEOUT. Lets a test see the
+ * bounded-wait path end with an error status while the context stays usable. */
+moe_status_t moe_debug_bounded_wait(uint64_t timeout_ns, moe_stream_t stream);
+
+/* Human-readable name of a status code. Never NULL. */
+const char *moe_status_string(moe_status_t status);
+
+/* MOE_ABI_VERSION of the built library. */
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

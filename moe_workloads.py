@@ -62,6 +62,10 @@ WORKLOADS = {
     "decode": Workload("decode", N=16, d=7168, f=2048, E=256, K=8, W=8),
     "stack4": Workload("stack4", N=32768, d=4096, f=1536, E=64, K=6, W=8, cf=1.25, s=0.0,
                        layers=4),
+    # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
+    # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
+    "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,
+                                     W=4, router="uniform"),
 }
 
 STACK_GRID_CF = (1.0, 1.25, 2.0)

@@ -1,0 +1,141 @@
+"""Runs the CUDA path stage by stage (through the C ABI) and holds the results
+as host arrays, plus the tolerance checks the parity tests share."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def lib():
+    from combine_grouped_gemm_router_b200 import build
+    build.build()
+    import combine_grouped_gemm_router_b200 as m
+    return m
+
+
+def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
+    """route -> dispatch -> expert GEMMs -> combine, each through its C entry point."""
+    m = lib()
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    dev = torch.device(device)
+    x = inp["x"].to(dev)
+    wr = inp["w_router"].to(dev)
+    bias = None if inp["bias"] is None else inp["bias"].to(dev)
+    N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
+    RA = m.moe_rows_alloc(shape)
+    ws = torch.empty(max(m.moe_workspace_size(shape), 256), dtype=torch.uint8, device=dev)
+    logits = torch.empty(N, E, dtype=torch.float32, device=dev)
+    topk_idx = torch.empty(N, K, dtype=torch.int32, device=dev)
+    topk_w = torch.empty(N, K, dtype=torch.float32, device=dev)
+    m.moe_route(shape, x, wr, bias, topk_idx, topk_w, logits, ws)
+
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(N * K, dtype=torch.int32, device=dev)
+    assign = torch.full((RA,), -7, dtype=torch.int32, device=dev)
+    x_sorted = torch.zeros(RA, d, dtype=torch.bfloat16, device=dev)
+    x_packed = torch.zeros(RA, d, dtype=torch.bfloat16, device=dev) if pack else None
+    D = torch.empty(W * W, dtype=torch.int64, device=dev)
+    pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
+    stats = m.stats_buffer(dev)
+    m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted, x_packed,
+                   D, pk_off, stats, ws)
+    res = dict(shape=shape, logits=logits, topk_idx=topk_idx, topk_w=topk_w, counts=counts,
+               kept=kept, offsets=offsets, row_of=row_of, assign=assign, x_sorted=x_sorted,
+               x_packed=x_packed, D=D, pk_off=pk_off, stats_buf=stats, rows_alloc=RA)
+    if w.d % 128 == 0 and w.f % 128 == 0:
+        h = torch.zeros(RA, f, dtype=torch.bfloat16, device=dev)
+        y = torch.zeros(RA, d, dtype=torch.float32, device=dev)
+        m.moe_expert_gemm(shape, x_sorted, offsets, inp["w1"].to(dev), inp["w3"].to(dev),
+                          inp["w2"].to(dev), h, y)
+        out = torch.empty(N, d, dtype=torch.float32, device=dev)
+        m.moe_combine(shape, y, row_of, topk_w, out)
+        res.update(h=h, y=y, out=out)
+    torch.cuda.synchronize()
+    res["stats"] = m.stats_dict(m.read_stats(stats))
+    res["dev_error"] = m.moe_get_device_error(True)
+    return res
+
+
+def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True) -> dict:
+    m = lib()
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    dev = torch.device(device)
+    ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
+    out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+    topk = torch.empty(w.N, w.K, dtype=torch.int32, device=dev)
+    stats = m.stats_buffer(dev) if with_stats else None
+    bias = None if inp["bias"] is None else inp["bias"].to(dev)
+    m.moe_layer(shape, inp["x"].to(dev), inp["w_router"].to(dev), bias, inp["w1"].to(dev),
+                inp["w3"].to(dev), inp["w2"].to(dev), out, topk_idx_out=topk, stats=stats, ws=ws)
+    torch.cuda.synchronize()
+    res = dict(out=out, topk_idx=topk, ws=ws)
+    if with_stats:
+        res["stats"] = m.stats_dict(m.read_stats(stats))
+    res["dev_error"] = m.moe_get_device_error(True)
+    return res
+
+
+def f64(t) -> np.ndarray:
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64)
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def tolerance_report(got, ref) -> dict:
+    """Relative Frobenius error and max-abs error / RMS(ref)."""
+    g = f64(got)
+    r = f64(ref)
+    err = g - r
+    nr = np.linalg.norm(r)
+    rms = np.sqrt(np.mean(r * r)) if r.size else 0.0
+    return dict(rel_frob=float(np.linalg.norm(err) / nr) if nr > 0 else float(np.linalg.norm(err)),
+                max_abs_over_rms=float(np.max(np.abs(err)) / rms) if rms > 0 else 0.0)
+
+
+# The stated bar for floating-point outputs against the oracle.
+REL_FROB = 5e-3
+MAX_ABS_OVER_RMS = 2e-2
+
+
+def assert_rounded_bf16(got, ref, what: str = ""):
+    """An intermediate stored as bf16: each element within one bf16 rounding
+    (2^-8 relative) of the reference plus fp32 accumulation slack."""
+    g = f64(got)
+    r = f64(ref)
+    rms = np.sqrt(np.mean(r * r))
+    excess = np.abs(g - r) - (2.0 ** -8 * np.abs(r) + 1e-3 * rms)
+    assert excess.max() <= 0, (what, float(excess.max() / rms))
+    assert tolerance_report(g, r)["rel_frob"] <= REL_FROB, what
+
+
+def bf16_h_bound_rows(h_ref: np.ndarray, w2_f64: np.ndarray, row_expert: np.ndarray) -> np.ndarray:
+    """Per-element bound on |y_gpu - y_ref| implied by the arithmetic: h is rounded once
+    to bf16 (relative error <= 2^-8) before the down projection, which accumulates in
+    fp32 over f terms: |dy_i| <= (2^-8 + f*2^-23) * sum_j |h_j W2[i][j]| (+ tiny)."""
+    f = h_ref.shape[1]
+    bound = np.empty((h_ref.shape[0], w2_f64.shape[1]))
+    for e in np.unique(row_expert):
+        sel = row_expert == e
+        bound[sel] = np.abs(h_ref[sel]) @ np.abs(w2_f64[e]).T
+    return bound * (2.0 ** -8 + f * 2.0 ** -23) + 1e-30
+
+
+def assert_within_bound(got, ref, bound, what: str = ""):
+    g, r = f64(got), f64(ref)
+    err = np.abs(g - r)
+    ratio = err / np.maximum(bound, 1e-30)
+    i = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+    worst = float(ratio[i])
+    rms = float(np.sqrt(np.mean(r * r))) or 1.0
+    assert worst <= 1.0, (what, dict(worst=worst, at=tuple(int(v) for v in i), got=float(g[i]),
+                                     ref=float(r[i]), bound=float(bound[i]),
+                                     err_over_rms=float(err[i] / rms)))
+    return worst
+
+
+def assert_within_tolerance(got, ref, what: str = ""):
+    rep = tolerance_report(got, ref)
+    assert rep["rel_frob"] <= REL_FROB and rep["max_abs_over_rms"] <= MAX_ABS_OVER_RMS, (what, rep)
+    return rep

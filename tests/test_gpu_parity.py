@@ -1,0 +1,171 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on shapes the
+oracle finishes in seconds: several tiles per expert, ragged tails, drops,
+empty experts, K = E, E = 1. Integer outputs bit-exact; floating-point outputs
+within relative Frobenius 5e-3 and max-abs 2e-2 * RMS of the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from layer_runner import (assert_rounded_bf16, assert_within_bound, assert_within_tolerance,
+                          bf16_h_bound_rows, run_layer, run_stages, tolerance_report)
+from moe_workloads import WORKLOADS, Workload, make_layer_inputs
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    WORKLOADS["tiny"],
+    # ~260 rows per expert: 3 M-tiles with a ragged last tile; G2 with 256-wide N tiles
+    Workload("ragged", N=1040, d=256, f=384, E=8, K=2, W=4),
+    # capacity drops under Zipf skew; d = 384 takes the 128-wide N tile of G2
+    Workload("drop_bn128", N=384, d=384, f=256, E=6, K=3, W=3, cf=1.25, s=1.1),
+    # many experts with few rows, some with none; heavy Zipf skew with drops gives a
+    # heavy-tailed output (a few elements near 7x its RMS), where one bf16 rounding of h
+    # moves the largest element by about 2.1% of the RMS: see HEAVY_TAIL below
+    Workload("sparse_experts", N=256, d=128, f=128, E=64, K=6, W=8, cf=1.0, s=1.2),
+    Workload("k_eq_e", N=64, d=128, f=128, E=4, K=4, W=2),
+    Workload("dense_e1", N=300, d=256, f=256, E=1, K=1, W=1),
+    Workload("decode_like", N=16, d=512, f=256, E=64, K=8, W=8),
+    Workload("odd_e", N=100, d=128, f=128, E=5, K=2, W=5, cf=0.9),
+    Workload("one_token_per_rank", N=8, d=128, f=128, E=16, K=3, W=8, cf=0.5),
+    Workload("wide_k", N=96, d=128, f=128, E=48, K=32, W=4),
+]
+
+
+# Cases whose max-abs error against the fp64 oracle is set by the bf16 rounding of the
+# SwiGLU activation h (the down projection's tensor-core operand) on a heavy-tailed
+# output; for them the stated max-abs bar is not claimed, the derived per-element bound
+# and the relative Frobenius bar are.
+HEAVY_TAIL = {"sparse_experts"}
+
+
+def _u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("seed", [0, 1])
+def test_layer_stages_match_oracle(orc, w, seed):
+    inp = make_layer_inputs(w, seed=seed)
+    ref = orc.layer(inp, w.K, w.W, w.cf, want_h=True)
+    got = run_stages(inp, w)
+    assert got["dev_error"] == 0
+
+    # a1: logits bit for bit; a2: selection exact, weights to fp32 rounding
+    np.testing.assert_array_equal(got["logits"].cpu().numpy().view(np.uint32),
+                                  ref["logits"].view(np.uint32))
+    np.testing.assert_array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
+    np.testing.assert_allclose(got["topk_w"].cpu().numpy(), ref["topk_w"], rtol=2e-6, atol=1e-7)
+
+    # a3: integer bookkeeping, bit-exact
+    R = ref["R"]
+    for key, rk in (("counts", "counts"), ("kept", "kept"), ("offsets", "offsets"),
+                    ("row_of", "row_of")):
+        np.testing.assert_array_equal(got[key].cpu().numpy(), ref[rk], err_msg=key)
+    assign = got["assign"].cpu().numpy()
+    np.testing.assert_array_equal(assign[:R], ref["assign_of_row"])
+    assert np.all(assign[R:] == -7), "rows past R must not be written"
+    np.testing.assert_array_equal(got["D"].cpu().numpy().reshape(w.W, w.W), ref["D"])
+    np.testing.assert_array_equal(got["pk_off"].cpu().numpy(), ref["pk_off"])
+    st, rs = got["stats"], ref["stats"]
+    assert (st["rows"], st["dropped"], st["cross_rows"], st["dedup_pairs"]) == (
+        rs["R"], rs["dropped"], rs["cross_rows"], rs["dedup_pairs"])
+    assert (st["active_experts"], st["max_kept"], st["min_kept"]) == (
+        rs["active_experts"], rs["max_kept"], rs["min_kept"])
+    assert st["capacity"] == min(ref["C"], w.N * w.K)
+
+    # a4: scatter is an exact copy, in both layouts
+    xu = _u16(inp["x"])
+    np.testing.assert_array_equal(_u16(got["x_sorted"][:R]), xu[ref["assign_of_row"] // w.K])
+    kept_slots = np.nonzero(ref["row_of"] >= 0)[0]
+    packed = np.empty((R, w.d), np.uint16)
+    packed[ref["packed_row_of"][kept_slots]] = xu[kept_slots // w.K]
+    np.testing.assert_array_equal(_u16(got["x_packed"][:R]), packed)
+
+    # a5/a6: expert GEMMs; a7: combine
+    assert_rounded_bf16(got["h"][:R], ref["h_rows"], "h")
+    w2 = inp["w2"].double().numpy()
+    row_expert = ref["topk_idx"].reshape(-1)[ref["assign_of_row"]]
+    ybound = bf16_h_bound_rows(ref["h_rows"], w2, row_expert)
+    assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
+    obound = np.zeros((w.N, w.d))
+    for a in np.nonzero(ref["row_of"] >= 0)[0]:
+        wa = abs(float(ref["topk_w"].reshape(-1)[a]))
+        r = ref["row_of"][a]
+        # propagated y bound, plus the fp32 weights and the fp32 sum over K slots
+        obound[a // w.K] += wa * ybound[r] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(ref["y_rows"][r])
+    assert_within_bound(got["out"], ref["out"], obound, "out")
+    if w.name in HEAVY_TAIL:
+        rep = tolerance_report(got["out"], ref["out"])
+        assert rep["rel_frob"] <= 5e-3 and rep["max_abs_over_rms"] <= 3e-2, rep
+    else:
+        assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
+        assert_within_tolerance(got["out"], ref["out"], "out")
+
+    # the fused entry point runs the same kernels: identical bits
+    lay = run_layer(inp, w)
+    assert lay["dev_error"] == 0
+    np.testing.assert_array_equal(lay["out"].cpu().numpy().view(np.uint32),
+                                  got["out"].cpu().numpy().view(np.uint32))
+    np.testing.assert_array_equal(lay["topk_idx"].cpu().numpy(), ref["topk_idx"])
+    assert lay["stats"]["dedup_pairs"] == rs["dedup_pairs"]
+
+
+def test_residual_combine(orc):
+    w = Workload("res", N=128, d=256, f=256, E=8, K=2, W=4, cf=1.0)
+    inp = make_layer_inputs(w, seed=5)
+    ref = orc.layer(inp, w.K, w.W, w.cf)
+    import combine_grouped_gemm_router_b200 as m
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    dev = torch.device("cuda")
+    ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
+    x = inp["x"].to(dev)
+    out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+    m.moe_layer(shape, x, inp["w_router"].to(dev), None, inp["w1"].to(dev), inp["w3"].to(dev),
+                inp["w2"].to(dev), out, residual=x, ws=ws)
+    # bf16 output mode (the next layer's input), out of place
+    shape16 = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=True)
+    out16 = torch.empty(w.N, w.d, dtype=torch.bfloat16, device=dev)
+    m.moe_layer(shape16, x, inp["w_router"].to(dev), None, inp["w1"].to(dev), inp["w3"].to(dev),
+                inp["w2"].to(dev), out16, residual=x, ws=ws)
+    torch.cuda.synchronize()
+    xr = inp["x"].double().numpy()
+    assert_within_tolerance(out, xr + ref["out"], "x + moe(x)")
+    # the bf16 output is the fp32 output rounded once
+    assert torch.equal(out16, out.to(torch.bfloat16))
+
+
+def test_identity_experts_round_trip():
+    """Dispatch then combine with y := x_sorted returns x * sum of kept weights."""
+    import combine_grouped_gemm_router_b200 as m
+    w = Workload("id", N=512, d=256, f=128, E=16, K=4, W=4)
+    inp = make_layer_inputs(w, seed=3)
+    got = run_stages(inp, w)
+    shape = got["shape"]
+    out = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    m.moe_combine(shape, got["x_sorted"].float(), got["row_of"], got["topk_w"], out)
+    torch.cuda.synchronize()
+    wsum = got["topk_w"].double().sum(1, keepdim=True).cpu().numpy()
+    assert np.allclose(wsum, 1.0, atol=1e-6)
+    assert_within_tolerance(out, inp["x"].double().numpy() * wsum, "identity round trip")
+
+
+def test_affinity_kernel_matches_oracle(orc):
+    rng = np.random.default_rng(0)
+    N, E, K = 5000, 64, 6
+    a, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    b, _, _ = orc.topk(rng.standard_normal((N, E)).astype(np.float32), K)
+    import combine_grouped_gemm_router_b200 as m
+    cnt = torch.zeros(E, E, dtype=torch.int64, device="cuda")
+    m.moe_affinity_accumulate(N, E, K, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), cnt)
+    m.moe_affinity_accumulate(N, E, K, torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), cnt)
+    ref = orc.affinity(a, b, E)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), 2 * ref)
+    # the global-atomic path (E > 64)
+    E2 = 96
+    a2, _, _ = orc.topk(rng.standard_normal((N, E2)).astype(np.float32), K)
+    b2, _, _ = orc.topk(rng.standard_normal((N, E2)).astype(np.float32), K)
+    cnt2 = torch.zeros(E2, E2, dtype=torch.int64, device="cuda")
+    m.moe_affinity_accumulate(N, E2, K, torch.from_numpy(a2).cuda(), torch.from_numpy(b2).cuda(),
+                              cnt2)
+    np.testing.assert_array_equal(cnt2.cpu().numpy(), orc.affinity(a2, b2, E2))
+    assert m.moe_get_device_error(True) == 0
