@@ -149,13 +149,19 @@ inline moe_status_t launch_status()
 
 // ---------------------------------------------------------------- route
 
-template <int TY, int TX, int TT, int TE>
+template <int TY, int TX, int TT, int TE, int KC, int S>
 void launch_logits(const uint16_t *x, const float *wr, const float *bias, float *logits, int N,
                    int d, int E, cudaStream_t st)
 {
-    constexpr int BT = TY * TT, BE = TX * TE;
-    dim3 grid((N + BT - 1) / BT, (E + BE - 1) / BE);
-    router_logits_kernel<TY, TX, TT, TE><<<grid, TY * TX, 0, st>>>(x, wr, bias, logits, N, d, E);
+    using L = LogitTile<TY, TX, TT, TE, KC, S>;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(router_logits_kernel<TY, TX, TT, TE, KC, S>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+    });
+    dim3 grid((N + L::BT - 1) / L::BT, (E + L::BE - 1) / L::BE);
+    router_logits_kernel<TY, TX, TT, TE, KC, S>
+        <<<grid, L::NT, L::SMEM_BYTES, st>>>(x, wr, bias, logits, N, d, E);
 }
 
 moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_router,
@@ -163,16 +169,24 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
                         unsigned long long *nonfinite, cudaStream_t st)
 {
     const int N = s->N, d = s->d, E = s->E;
-    if (N < 1024)
-        launch_logits<1, 32, 4, 1>(x, w_router, bias, logits, N, d, E, st);
-    else if (E <= 8)
-        launch_logits<32, 8, 4, 1>(x, w_router, bias, logits, N, d, E, st);
-    else if (E <= 16)
-        launch_logits<16, 16, 4, 1>(x, w_router, bias, logits, N, d, E, st);
-    else if (E <= 32)
-        launch_logits<16, 16, 4, 2>(x, w_router, bias, logits, N, d, E, st);
-    else
-        launch_logits<8, 16, 8, 4>(x, w_router, bias, logits, N, d, E, st);
+    // Tile choice. Each output is one dependent chain of d fused multiply-adds, so
+    // the floor is d x (fma latency). Few outputs (small N or small E): one chain per
+    // thread and many warps per SM, so latency, not issue, is the limit. Many outputs
+    // (E >= 32 with large N): the fp32 FMA pipe is the limit; a thread owns 4 tokens x
+    // 8 experts so each bf16 -> fp32 conversion of x feeds 8 FMAs.
+    const long long outputs = (long long)N * E;
+    if (outputs < 148LL * 1024 || E <= 16) {
+        if (N < 64)
+            launch_logits<2, 32, 1, 1, 64, 6>(x, w_router, bias, logits, N, d, E, st);
+        else if (E <= 8)
+            launch_logits<32, 8, 1, 1, 64, 4>(x, w_router, bias, logits, N, d, E, st);
+        else
+            launch_logits<16, 16, 1, 1, 64, 4>(x, w_router, bias, logits, N, d, E, st);
+    } else if (E <= 32) {
+        launch_logits<8, 16, 2, 2, 64, 4>(x, w_router, bias, logits, N, d, E, st);
+    } else {
+        launch_logits<16, 8, 4, 8, 64, 3>(x, w_router, bias, logits, N, d, E, st);
+    }
     topk_softmax_kernel<<<(N + 7) / 8, 256, 0, st>>>(logits, N, E, s->K, topk_idx, topk_w,
                                                       nonfinite);
     return launch_status();

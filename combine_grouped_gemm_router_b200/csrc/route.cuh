@@ -15,30 +15,69 @@
 
 namespace moe {
 
-constexpr int kLogitKC = 32;  // d-chunk staged in shared memory per step
+// CTA tile: BT = TY*TT tokens x BE = TX*TE experts, TY*TX threads; d walked in
+// chunks of KC staged by cp.async into an S-deep shared-memory ring, so the
+// global-memory latency of later chunks overlaps the FMAs of earlier ones.
+// Thread (ty, tx) owns tokens ty*TT + i and experts tx + TX*j; per 8 elements of
+// d it reads one 16-byte bf16 vector per token and two 16-byte fp32 vectors per
+// expert, then runs the 8 fused multiply-adds of every owned output in i order.
+template <int TY, int TX, int TT, int TE, int KC, int S>
+struct LogitTile {
+    static constexpr int NT = TY * TX;
+    static constexpr int BT = TY * TT;
+    static constexpr int BE = TX * TE;
+    static constexpr int XROW = KC + 8;  // bf16 per staged x row (16-byte pad: no bank conflicts)
+    static constexpr int WROW = KC + 4;  // fp32 per staged Wr row (16-byte pad)
+    static constexpr int X_BYTES = BT * XROW * 2;
+    static constexpr int W_BYTES = BE * WROW * 4;
+    static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
+    static constexpr int SMEM_BYTES = S * STAGE_BYTES;
+};
 
-// CTA tile: BT = TY*TT tokens x BE = TX*TE experts, TY*TX threads.
-// Thread (ty, tx) owns tokens ty*TT + i (contiguous, float4 reads) and experts
-// tx + TX*j (strided, conflict-free scalar reads).
-template <int TY, int TX, int TT, int TE>
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int TY, int TX, int TT, int TE, int KC, int S>
 __global__ void __launch_bounds__(TY *TX)
     router_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
                          const float *__restrict__ bias, float *__restrict__ logits, int N, int d,
                          int E)
 {
-    static_assert(TT % 4 == 0, "tokens per thread must be a multiple of 4");
-    constexpr int NT = TY * TX;
-    constexpr int BT = TY * TT;
-    constexpr int BE = TX * TE;
-    constexpr int KC = kLogitKC;
-    constexpr int XS = BT + 4;  // keeps float4 alignment of every row
-    __shared__ __align__(16) float xs[KC][XS];
-    __shared__ float ws[KC][BE];
-
+    using L = LogitTile<TY, TX, TT, TE, KC, S>;
+    static_assert(KC % 8 == 0, "chunk must hold whole 16-byte vectors");
+    extern __shared__ __align__(16) unsigned char logit_smem[];
     const int tid = threadIdx.x;
     const int ty = tid / TX, tx = tid % TX;
-    const int t0 = blockIdx.x * BT;
-    const int e0 = blockIdx.y * BE;
+    const int t0 = blockIdx.x * L::BT;
+    const int e0 = blockIdx.y * L::BE;
+    const int nchunks = (d + KC - 1) / KC;
+
+    auto issue = [&](int c) {
+        if (c < nchunks) {
+            unsigned char *st = logit_smem + (c % S) * L::STAGE_BYTES;
+            uint16_t *xs = reinterpret_cast<uint16_t *>(st);
+            float *ws = reinterpret_cast<float *>(st + L::X_BYTES);
+            const int k0 = c * KC;
+            const int kc = min(KC, d - k0);  // a multiple of 8 (d % 8 == 0)
+            for (int idx = tid; idx < L::BT * (KC / 8); idx += L::NT) {
+                const int row = idx / (KC / 8), v = idx % (KC / 8);
+                if (t0 + row < N && v * 8 < kc)
+                    cp_async16(xs + row * L::XROW + v * 8, x + (size_t)(t0 + row) * d + k0 + v * 8);
+            }
+            for (int idx = tid; idx < L::BE * (KC / 4); idx += L::NT) {
+                const int row = idx / (KC / 4), v = idx % (KC / 4);
+                if (e0 + row < E && v * 4 < kc)
+                    cp_async16(ws + row * L::WROW + v * 4, wr + (size_t)(e0 + row) * d + k0 + v * 4);
+            }
+        }
+        cp_async_commit();  // possibly empty: keeps the group count uniform
+    };
 
     float acc[TT][TE];
 #pragma unroll
@@ -47,55 +86,44 @@ __global__ void __launch_bounds__(TY *TX)
         for (int j = 0; j < TE; ++j)
             acc[i][j] = 0.0f;
 
-    for (int k0 = 0; k0 < d; k0 += KC) {
-        const int kc = min(KC, d - k0);  // a multiple of 8 (d % 8 == 0)
-        for (int idx = tid; idx < BT * (KC / 8); idx += NT) {
-            const int row = idx % BT, c8 = idx / BT;
-            const int t = t0 + row;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (t < N && c8 * 8 < kc)
-                v = *reinterpret_cast<const uint4 *>(x + (size_t)t * d + k0 + c8 * 8);
-            xs[c8 * 8 + 0][row] = bf16_lo(v.x);
-            xs[c8 * 8 + 1][row] = bf16_hi(v.x);
-            xs[c8 * 8 + 2][row] = bf16_lo(v.y);
-            xs[c8 * 8 + 3][row] = bf16_hi(v.y);
-            xs[c8 * 8 + 4][row] = bf16_lo(v.z);
-            xs[c8 * 8 + 5][row] = bf16_hi(v.z);
-            xs[c8 * 8 + 6][row] = bf16_lo(v.w);
-            xs[c8 * 8 + 7][row] = bf16_hi(v.w);
-        }
-        for (int idx = tid; idx < BE * (KC / 4); idx += NT) {
-            const int col = idx % BE, c4 = idx / BE;
-            const int e = e0 + col;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (e < E && c4 * 4 < kc)
-                v = *reinterpret_cast<const float4 *>(wr + (size_t)e * d + k0 + c4 * 4);
-            ws[c4 * 4 + 0][col] = v.x;
-            ws[c4 * 4 + 1][col] = v.y;
-            ws[c4 * 4 + 2][col] = v.z;
-            ws[c4 * 4 + 3][col] = v.w;
-        }
-        __syncthreads();
-        for (int kk = 0; kk < kc; ++kk) {
-            float a[TT], b[TE];
 #pragma unroll
-            for (int i = 0; i < TT; i += 4) {
-                const float4 q = *reinterpret_cast<const float4 *>(&xs[kk][ty * TT + i]);
-                a[i] = q.x;
-                a[i + 1] = q.y;
-                a[i + 2] = q.z;
-                a[i + 3] = q.w;
+    for (int c = 0; c < S - 1; ++c)
+        issue(c);
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<S - 2>();
+        __syncthreads();
+        issue(c + S - 1);
+        const unsigned char *st = logit_smem + (c % S) * L::STAGE_BYTES;
+        const uint16_t *xs = reinterpret_cast<const uint16_t *>(st);
+        const float *ws = reinterpret_cast<const float *>(st + L::X_BYTES);
+        const int kc = min(KC, d - c * KC);
+        for (int kk = 0; kk < kc; kk += 8) {
+            float xv[TT][8];
+#pragma unroll
+            for (int i = 0; i < TT; ++i) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(xs + (ty * TT + i) * L::XROW + kk);
+                xv[i][0] = bf16_lo(q.x);
+                xv[i][1] = bf16_hi(q.x);
+                xv[i][2] = bf16_lo(q.y);
+                xv[i][3] = bf16_hi(q.y);
+                xv[i][4] = bf16_lo(q.z);
+                xv[i][5] = bf16_hi(q.z);
+                xv[i][6] = bf16_lo(q.w);
+                xv[i][7] = bf16_hi(q.w);
             }
 #pragma unroll
-            for (int j = 0; j < TE; ++j)
-                b[j] = ws[kk][tx + TX * j];
+            for (int j = 0; j < TE; ++j) {
+                const float *wrow = ws + (tx + TX * j) * L::WROW + kk;
+                const float4 a = *reinterpret_cast<const float4 *>(wrow);
+                const float4 b = *reinterpret_cast<const float4 *>(wrow + 4);
+                const float wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < TT; ++i)
+                for (int q = 0; q < 8; ++q)
 #pragma unroll
-                for (int j = 0; j < TE; ++j)
-                    acc[i][j] = __fmaf_rn(a[i], b[j], acc[i][j]);
+                    for (int i = 0; i < TT; ++i)
+                        acc[i][j] = __fmaf_rn(xv[i][q], wv[q], acc[i][j]);
+            }
         }
-        __syncthreads();
     }
 #pragma unroll
     for (int i = 0; i < TT; ++i) {
