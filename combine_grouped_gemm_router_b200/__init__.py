@@ -59,6 +59,7 @@ _sigs = {
     "moe_layer_workspace_size": ([_SP], c_size),
     "moe_route": ([_SP] + [c_p] * 7 + [c_size, c_p], c_i32),
     "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
+    "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
     "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
     "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
     "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
@@ -181,6 +182,21 @@ def moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_ro
                              _ptr(x_sorted), _ptr(x_packed), _ptr(rank_matrix),
                              _ptr(packed_offsets), _ptr(stats), _ptr(ws), ws_bytes,
                              _stream(stream)), "moe_dispatch")
+
+
+MOE_STATIC_SCRATCH_BYTES = 1 << 20
+
+
+def moe_dispatch_static(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_row,
+                        x_sorted, x_packed=None, rank_matrix=None, packed_offsets=None, stats=None,
+                        stream=None):
+    """moe_dispatch with the library's fixed device scratch instead of a caller workspace
+    (for callers that cannot allocate device memory)."""
+    _check(_lib.moe_dispatch_static(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                                    _ptr(kept), _ptr(offsets), _ptr(row_of), _ptr(assign_of_row),
+                                    _ptr(x_sorted), _ptr(x_packed), _ptr(rank_matrix),
+                                    _ptr(packed_offsets), _ptr(stats), _stream(stream)),
+           "moe_dispatch_static")
 
 
 def moe_expert_gemm(shape, x_sorted, offsets, w1, w3, w2, h, y, stream=None):

@@ -730,3 +730,91 @@ __attribute__((visibility("default"))) moe_status_t moe_debug_bounded_wait(uint6
 }
 
 }  // extern "C"
+
+// ================================================================ dispatch without a workspace
+//
+// Scratch of moe_dispatch_static: one fixed array per device. Host code never uses the
+// symbol itself as an address (on the host it is only a stand-in); the device address is
+// looked up once per device with cudaGetSymbolAddress while that device is current.
+
+static __device__ __align__(256) unsigned char g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_addr[kMaxDevices];
+
+moe_status_t static_scratch_address(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p)
+            return MOE_ERR_CUDA;
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return MOE_OK;
+}
+
+struct StaticLayout {
+    size_t blk, pk_base, D, pk_off, total;
+};
+
+StaticLayout static_layout(const moe_shape_t *s, const Geometry &g)
+{
+    StaticLayout L;
+    size_t o = 0;
+    L.blk = o;
+    o = align_up(o + (size_t)s->E * g.nblk * 4);
+    L.pk_base = o;
+    o = align_up(o + (size_t)s->E * s->W * 8);
+    L.D = o;
+    o = align_up(o + (size_t)s->W * s->W * 8);
+    L.pk_off = o;
+    o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+extern "C" __attribute__((visibility("default"))) moe_status_t
+moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx,
+                    int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of,
+                    int32_t *assign_of_row, uint16_t *x_sorted, uint16_t *x_packed,
+                    int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
+                    moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, false, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_sorted) || (x_packed && !aligned16(x_packed)) ||
+        !aligned4(topk_idx) || !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) ||
+        !aligned4(row_of) || !aligned4(assign_of_row) ||
+        (rank_matrix && (reinterpret_cast<uintptr_t>(rank_matrix) & 7u)) ||
+        (packed_offsets && (reinterpret_cast<uintptr_t>(packed_offsets) & 7u)) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const StaticLayout L = static_layout(shape, g);
+    if (L.total > MOE_STATIC_SCRATCH_BYTES)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    void *base = nullptr;
+    rc = static_scratch_address(&base);
+    if (rc != MOE_OK)
+        return rc;
+    char *w = static_cast<char *>(base);
+    int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
+    int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
+    return dispatch_impl(shape, g, x, topk_idx, counts, kept, offsets, row_of, assign_of_row,
+                         x_sorted, x_packed, D, pk, stats, reinterpret_cast<int32_t *>(w + L.blk),
+                         reinterpret_cast<int64_t *>(w + L.pk_base),
+                         reinterpret_cast<cudaStream_t>(stream));
+}

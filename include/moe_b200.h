@@ -160,6 +160,34 @@ moe_status_t moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int
                           int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
                           void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Size of the library's fixed device scratch array used by moe_dispatch_static. */
+#define MOE_STATIC_SCRATCH_BYTES (1u << 20)
+
+/* moe_dispatch for callers that cannot allocate device memory. The pages have no counterpart:
+ * this is an interface convenience, not a step of the method.
+ * Some callers cannot hand the library a workspace: a plugin whose host owns every device
+ * allocation and grants none to plugins, a process whose device-memory budget is fixed when it
+ * starts, or a latency-critical loop where a cudaMalloc (which can synchronise the device) is
+ * not acceptable. This entry point takes the same arguments and writes the same outputs as
+ * moe_dispatch, but its scratch (block histograms, pack bases, and the traffic matrix and pack
+ * offsets when those are NULL) lives in one static device array of MOE_STATIC_SCRATCH_BYTES
+ * inside the library. Every GPU that loads the library holds that array until the process
+ * exits. The call allocates and frees nothing.
+ *  - Shapes whose scratch does not fit (about E * W * ceil(N / (64 W)) * 4 bytes plus
+ *    E * W * 8 + 2 * W * W * 8) return MOE_ERR_WORKSPACE_TOO_SMALL before any launch.
+ *  - The first call on a device looks up the array's device address on that device (the
+ *    device must be current); make that first call before any stream capture.
+ *  - All calls share the one array, and it keeps the last call's contents; every scratch byte
+ *    a call reads it has written first in the same call, so nothing needs clearing. Two calls
+ *    that overlap on the GPU (other streams, other host threads) race on the array: serialise
+ *    them. */
+moe_status_t moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x,
+                                 const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                                 int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                                 uint16_t *x_sorted, uint16_t *x_packed, int64_t *rank_matrix,
+                                 int64_t *packed_offsets, moe_stats_t *stats,
+                                 moe_stream_t stream);
+
 /* Ragged grouped GEMM of the SwiGLU experts, one persistent launch per GEMM.
  * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (grouped GEMM over
  *  variable per-expert token counts) and §容量因子、专家复制与 dropless 的取舍 (dropless
