@@ -162,9 +162,9 @@ class ClockSampler:
 # profiles/grouped_gemm_up_mixtral_prefill_half_full.md (half-size case, scaled x2 to the
 # full layer). Valid only for the kernel source it was measured on.
 MEASURED_UP_TRAFFIC = {
-    "kernel_sha256": "28a3c9dae73d22cb397f70f7a04a51635be79cbfdbca4c92c286432e55a26756",
+    "kernel_sha256": "22c554d22716c0ea182bc63623776b24295dea3d04bfdfc1d0550202fb7781a5",
     "workload": "mixtral_prefill",
-    "bytes": 2171.8e6,
+    "bytes": 2287.6e6,
 }
 
 
@@ -337,7 +337,8 @@ def run_gpu(args, w) -> dict:
                    "rows_kept": R, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step"},
-        "roofline": {"kernel": "grouped GEMM gate/up (moe_expert_up)", "bound": "tensor",
+        "roofline": {"kernel": "grouped GEMM gate/up (moe_expert_up, CTA-pair tcgen05 kernel)",
+                     "bound": "tensor",
                      "achieved": up_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": up_tflops / peaks["bf16_tflops"],
                      "peak_source": peaks["source"] + " bf16 burst",

@@ -183,9 +183,11 @@ __device__ __forceinline__ void tmem_ld_wait()
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// silu(g) * u = g * u / (1 + e^-g), with the fast exponential and division
+// intrinsics (each within a few ulp; the result is rounded to bf16 next).
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
-    return g / (1.0f + __expf(-g)) * u;
+    return __fdividef(g * u, 1.0f + __expf(-g));
 }
 
 // Tile index -> (expert, N-slab, M-tile). tile_start[e] = first tile of expert e.
@@ -453,6 +455,343 @@ __global__ void __launch_bounds__(THREADS, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(TMEM_COLS)
                      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 cta_group::2). A cluster of 2 CTAs on 2 SMs computes
+// a 256 x 256 tile: CTA r loads rows [128 r, 128 r + 128) of A and rows
+// [128 r, 128 r + 128) of the 256-row B tile into its own shared memory at the
+// same offsets; the first CTA of the pair issues one M=256, N=256 MMA per K step
+// that reads A from each CTA and B from both, and each CTA's TMEM receives its 128
+// rows of the accumulator. Per CTA and 64-element K step that is 32 KB of
+// operands for the same MMA work that costs the single-CTA kernel 48 KB. A ring
+// stage holds two K steps (128 elements, two swizzle atoms per operand, 64 KB per
+// CTA, 3 stages): eight MMAs per barrier round trip instead of four, which the
+// issue path of the pair needs to keep the tensor pipe busy.
+// Barriers: full[s] lives in the first CTA and counts both CTAs' TMA bytes
+// (the loads name it by its cluster address); empty[s] and tfull[a] live in each
+// CTA and receive one tcgen05.commit each (two commits, one per CTA, to
+// mapa-resolved addresses); tempty[a] lives in the first CTA and counts the 8
+// epilogue warps of the pair.
+
+constexpr int KA2 = 2;                                      // 64-element K atoms per stage
+constexpr int STAGES2 = 3;
+constexpr int STAGE2_BYTES = KA2 * (A_BYTES + B_HALF_BYTES);  // 64 KB per CTA
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_addr), "r"(rank));
+    return out;
+}
+
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t bar_cluster_addr)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster_addr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar_cluster_addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                     bar_cluster_addr)
+                 : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                             const __grid_constant__ CUtensorMap tmB0,
+                             const __grid_constant__ CUtensorMap tmB1, const Args args)
+{
+    constexpr int BMP = 256;  // rows per pair tile
+    constexpr int BN = 256;
+    constexpr uint32_t IDESC = instr_desc_bf16(BMP, BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES2 * STAGE2_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES2 + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *tile_start = reinterpret_cast<int *>(tmem_slot + 4);
+    int *mtiles = tile_start + (args.E + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const uint32_t smem_base = smem_u32(smem);
+    const uint32_t bar_base = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (STAGES2 + s); };
+    auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * STAGES2 + a); };
+    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES2 + 2 + a); };
+    const uint32_t done_bar = bar_base + 8u * (2 * STAGES2 + 4);
+    const int E = args.E;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES2; ++st) {
+            mbar_init(full_bar(st), 1);
+            mbar_init(empty_bar(st), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 8);
+        }
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        *abort_flag = 0;
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0) {
+        int carry = 0;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int mt = 0;
+            if (e < E) {
+                int rows = args.offsets[e + 1] - args.offsets[e];
+                rows = max(0, min(rows, args.rows_alloc));
+                mt = (rows + BMP - 1) / BMP;
+                mtiles[e] = mt;
+            }
+            const int incl = warp_incl_scan(mt);
+            if (e < E)
+                tile_start[e] = (carry + incl - mt) * args.n_tiles;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0)
+            tile_start[E] = carry * args.n_tiles;
+    }
+    tc_fence_before();
+    cluster_sync_all();  // barriers initialised in both CTAs before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs)
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t last_parity[STAGES2];
+            bool issued[STAGES2];
+            for (int st = 0; st < STAGES2; ++st)
+                issued[st] = false;
+            bool ok = true;
+            const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? &tmB1 : &tmB0;
+            for (int tile = pair; tile < total && ok; tile += npairs) {
+                int e, n, m;
+                decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
+                const int row0 = args.offsets[e] + m * BMP + (int)rank * 128;
+                const int brow = MODE == 0 ? e * args.b_rows + n * 128
+                                           : e * args.b_rows + n * BN + (int)rank * 128;
+                for (int kb = 0; kb < args.k_blocks / KA2; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t a_dst = smem_base + stage * STAGE2_BYTES;
+                    const uint32_t full_leader = map_to_rank(full_bar(stage), 0);
+                    if (leader)
+                        mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE2_BYTES);
+#pragma unroll
+                    for (int at = 0; at < KA2; ++at) {
+                        const int kx = (kb * KA2 + at) * BK;
+                        tma_load_2d_pair(a_dst + at * A_BYTES, &tmA, kx, row0, full_leader);
+                        tma_load_2d_pair(a_dst + KA2 * A_BYTES + at * B_HALF_BYTES, bmap, kx, brow,
+                                         full_leader);
+                    }
+                    issued[stage] = true;
+                    last_parity[stage] = phase;
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain (first CTA: its full barriers count both CTAs' copies)
+            if (leader)
+                for (int st = 0; st < STAGES2; ++st)
+                    if (issued[st])
+                        mbar_wait(full_bar(st), last_parity[st], abort_flag, args.timeout_ns, false);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ---------------- MMA issuer (first CTA of the pair)
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < total && ok; tile += npairs) {
+                if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.timeout_ns))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < args.k_blocks / KA2; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_base + stage * STAGE2_BYTES;
+                    const uint32_t b_addr = a_addr + KA2 * A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < KA2 * BK / 16; ++k) {
+                        const uint32_t off = (uint32_t)((k / 4) * A_BYTES + (k % 4) * 32);
+                        tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + off),
+                                         smem_desc_sw128(b_addr + off), IDESC,
+                                         (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(map_to_rank(empty_bar(stage), 0));
+                    tc_commit_pair(map_to_rank(empty_bar(stage), 1));
+                    if (++stage == STAGES2) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit_pair(map_to_rank(tfull_bar(acc), 0));
+                tc_commit_pair(map_to_rank(tfull_bar(acc), 1));
+                acc ^= 1;
+                if (acc == 0)
+                    acc_phase ^= 1u;
+            }
+            tc_commit_pair(map_to_rank(done_bar, 0));
+            mbar_wait(done_bar, 0, abort_flag, args.timeout_ns, false);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5 of both CTAs
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = pair; tile < total; tile += npairs) {
+            int e, n, m;
+            decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
+            const int rows_e = args.offsets[e + 1] - args.offsets[e];
+            const int valid = min(128, rows_e - m * BMP - (int)rank * 128);
+            const int row0 = args.offsets[e] + m * BMP + (int)rank * 128;
+            int ok = 0;
+            if (lane == 0)
+                ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            if (MODE == 0) {
+                uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)(row0 + r) * args.ldo;
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    uint32_t g[16], u[16];
+                    tmem_ld16(taddr + c, g);
+                    tmem_ld16(taddr + 128 + c, u);
+                    tmem_ld_wait();
+                    if (r < valid) {
+                        uint32_t p[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            p[j] = pack_bf16x2(
+                                silu_mul(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j])),
+                                silu_mul(__uint_as_float(g[2 * j + 1]),
+                                         __uint_as_float(u[2 * j + 1])));
+                        dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
+                        dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
+                    }
+                }
+            } else {
+                float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
+                uint4 *dst = reinterpret_cast<uint4 *>(frow + n * BN);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v0[16], v1[16];
+                    tmem_ld16(taddr + c, v0);
+                    tmem_ld16(taddr + c + 16, v1);
+                    tmem_ld_wait();
+                    if (r < valid) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            dst[c / 4 + j] = make_uint4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2],
+                                                        v0[4 * j + 3]);
+                            dst[c / 4 + 4 + j] = make_uint4(v1[4 * j], v1[4 * j + 1],
+                                                            v1[4 * j + 2], v1[4 * j + 3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
+            acc ^= 1;
+            if (acc == 0)
+                acc_phase ^= 1u;
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    if (*abort_flag) {
+        // after a timeout, give copies already in flight time to land before the pair
+        // leaves (a CTA's shared memory must outlive the copies and MMAs that use it)
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
+    }
+    cluster_sync_all();  // neither CTA leaves while its partner may still use its memory
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+}
+
+constexpr int smem_bytes_pair(int E)
+{
+    return STAGES2 * STAGE2_BYTES + 1024 + 8 * (2 * STAGES2 + 5) + 16 + 8 * (E + 1) + 64;
 }
 
 template <int MODE, int BN>

@@ -319,6 +319,65 @@ moe_status_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b0, const CUte
     return launch_status();
 }
 
+// Launches the CTA-pair kernel with a 2-CTA cluster, as many pairs as fit on the
+// GPU at once (the tile schedule is static per pair, so every pair must be resident).
+template <int MODE>
+moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1,
+                              const gg::Args &args, cudaStream_t st)
+{
+    const int smem = gg::smem_bytes_pair(kMaxE);
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    static int pairs = 0;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(gg::grouped_gemm_pair_kernel<MODE>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (attr_err != cudaSuccess)
+            return;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+        cfg.blockDim = dim3(gg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        attr_err = cudaOccupancyMaxActiveClusters(&n, gg::grouped_gemm_pair_kernel<MODE>, &cfg);
+        pairs = n;
+    });
+    if (attr_err != cudaSuccess || pairs <= 0)
+        return MOE_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(gg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gg::grouped_gemm_pair_kernel<MODE>, a, b0, b1, args) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return launch_status();
+}
+
+// The pair kernel computes 256-row tiles: worth it when experts hold a few hundred rows
+// or more (prefill); with fewer, the 128-row single-CTA tiles waste less work.
+bool use_pair_tiles(const moe_shape_t *s, const Geometry &g)
+{
+    // (the pair kernel steps K by 128: d and f are multiples of 128 for every GEMM shape)
+    const int64_t mean_rows = ((int64_t)s->N * s->K) / s->E;
+    const int64_t rows = mean_rows < g.C ? mean_rows : g.C;
+    return rows >= 192;
+}
+
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                             uint16_t *h, cudaStream_t st)
@@ -338,6 +397,8 @@ moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint1
     a.out = h;
     a.ldo = f;
     a.timeout_ns = kWaitTimeoutNs;
+    if (use_pair_tiles(s, g))
+        return launch_gemm_pair<0>(tA, tW1, tW3, a, st);
     return launch_gemm<0, 256>(tA, tW1, tW3, a, st);
 }
 
@@ -360,6 +421,8 @@ moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uin
     a.timeout_ns = kWaitTimeoutNs;
     if (d % 256 == 0) {
         a.n_tiles = d / 256;
+        if (use_pair_tiles(s, g))
+            return launch_gemm_pair<1>(tA, tW2, tW2, a, st);
         return launch_gemm<1, 256>(tA, tW2, tW2, a, st);
     }
     a.n_tiles = d / 128;
