@@ -232,24 +232,25 @@ def run_gpu(args, w) -> dict:
     launches_per_step = 9  # logits, top-K, histogram, scan, positions, scatter, up, down, combine
 
     def step(ev=None):
+        st = torch.cuda.current_stream(dev)
         if ev is not None:
-            ev[0].record(stream)
-        m.moe_route(shape, x, wr, bias, topk_idx, topk_w, None, ws, stream)
+            ev[0].record(st)
+        m.moe_route(shape, x, wr, bias, topk_idx, topk_w, None, ws, st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted,
-                       x_packed, D, pk_off, None, ws, stream)
+                       x_packed, D, pk_off, None, ws, st)
         if ev is not None:
-            ev[2].record(stream)
-        m.moe_expert_up(shape, x_sorted, offsets, w1, w3, h, stream)
+            ev[2].record(st)
+        m.moe_expert_up(shape, x_sorted, offsets, w1, w3, h, st)
         if ev is not None:
-            ev[3].record(stream)
-        m.moe_expert_down(shape, h, offsets, w2, y, stream)
+            ev[3].record(st)
+        m.moe_expert_down(shape, h, offsets, w2, y, st)
         if ev is not None:
-            ev[4].record(stream)
-        m.moe_combine(shape, y, row_of, topk_w, out, None, stream)
+            ev[4].record(st)
+        m.moe_combine(shape, y, row_of, topk_w, out, None, st)
         if ev is not None:
-            ev[5].record(stream)
+            ev[5].record(st)
 
     for _ in range(args.warmup):
         step()
@@ -257,6 +258,8 @@ def run_gpu(args, w) -> dict:
     if m.moe_get_device_error(True) != 0:
         raise RuntimeError("device error during warm-up")
 
+    # the timed run: K eager steps, CUDA events between the stages of every step (on the
+    # stream the kernels run on), barrier + synchronize on both sides
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
@@ -273,39 +276,85 @@ def run_gpu(args, w) -> dict:
     stage_ms = {name: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events)
                 for j, name in enumerate(["route", "dispatch", "expert_up", "expert_down",
                                           "combine"])}
+
+    # the same step captured once in a CUDA graph (its 9 kernels) and replayed K times: the
+    # host launch overhead disappears, which matters for small (decode) steps
+    graph_res = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        barrier()
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        g_agg = aggregate(float(N * args.steps), g0.elapsed_time(g1) / 1e3, dev)
+        graph_res = {"value": g_agg["value"], "unit": UNIT,
+                     "ms_per_step": g_agg["elapsed_max_s"] / args.steps * 1e3}
+        del graph
     err = m.moe_get_device_error(True)
     R = int(offsets[E].item())
     agg = aggregate(float(N * args.steps), elapsed_s, dev)
 
     # end to end through the public API: pinned host input -> moe_layer -> host output
+    # end to end through the public API: every step copies its input from pinned host memory,
+    # runs moe_layer and copies the fp32 result back; the copies of one step overlap the layer
+    # of the previous one (two buffers, one copy stream each way)
     e2e = None
     if not args.no_e2e:
         lws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
         x_host = x.cpu().pin_memory()
-        out_host = torch.empty(N, d, dtype=torch.float32).pin_memory()
-        x_dev = torch.empty_like(x)
-        out_dev = torch.empty(N, d, dtype=torch.float32, device=dev)
+        out_host = [torch.empty(N, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+        x_dev = [torch.empty_like(x) for _ in range(2)]
+        out_dev = [torch.empty(N, d, dtype=torch.float32, device=dev) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            x_dev.copy_(x_host, non_blocking=True)
-            m.moe_layer(shape, x_dev, wr, bias, w1, w3, w2, out_dev, ws=lws, stream=stream)
-            out_host.copy_(out_dev, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            s_in.wait_event(ev_comp[b])  # buffer b's previous layer has read its input
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_out[b])  # buffer b's previous result has left the device
+            m.moe_layer(shape, x_dev[b], wr, bias, w1, w3, w2, out_dev[b], ws=lws, stream=stream)
+            ev_comp[b].record(stream)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-        for _ in range(args.warmup):
-            e2e_step()
+        for i in range(args.warmup):
+            e2e_step(i)
         torch.cuda.synchronize(dev)
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(args.steps):
+            e2e_step(i)
+        for b in range(2):
+            stream.wait_event(ev_out[b])
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         e2e_agg = aggregate(float(N * args.steps), e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": e2e_agg["value"], "unit": UNIT, "h2d_bytes_per_step": N * d * 2,
-               "d2h_bytes_per_step": N * d * 4}
+               "d2h_bytes_per_step": N * d * 4,
+               "note": "pinned host input and output; copies overlap the previous step's layer"}
         del lws
 
     work = algorithmic_work(w, R)
@@ -353,6 +402,7 @@ def run_gpu(args, w) -> dict:
                      "scatter_bytes": work["scatter_bytes"]},
         "clocks": clocks.summary(),
         "gpu_launches": launches_per_step * args.steps,
+        "graph": graph_res,
         "device_error": err,
         "e2e": e2e,
     }
@@ -457,6 +507,8 @@ def parse(argv=None):
     ap.add_argument("--cpu-sample-tokens", type=int, default=32)
     ap.add_argument("--ref-sample-tokens", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager launches instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args(argv)
 
