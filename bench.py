@@ -198,7 +198,7 @@ def run_gpu(args, w) -> dict:
     import torch
 
     import combine_grouped_gemm_router_b200 as m
-    from moe_workloads import make_layer_inputs
+    from moe_workloads import make_layer_inputs, make_shared_inputs
 
     world, rank = init_dist("nccl")
     _, _, local = dist_env()
@@ -206,18 +206,22 @@ def run_gpu(args, w) -> dict:
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
-    inp = make_layer_inputs(w, seed=args.seed + rank, device=str(dev))
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    # one step = the whole stack of w.layers layers (one layer unless the workload is a stack)
+    L = w.layers
+    shared = w.shared_f > 0
+    layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
+              for l in range(L)]
+    inp = layers[0]
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=L > 1)
     RA = m.moe_rows_alloc(shape)
     ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
-    x, wr, bias = inp["x"], inp["w_router"], inp["bias"]
-    w1, w3, w2 = inp["w1"], inp["w3"], inp["w2"]
+    x = inp["x"]
     N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
-    topk_idx = torch.empty(N, K, dtype=torch.int32, device=dev)
+    topk_idx = [torch.empty(N, K, dtype=torch.int32, device=dev) for _ in range(L)]
     topk_w = torch.empty(N, K, dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     kept = torch.empty(E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    offsets = [torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
     row_of = torch.empty(N * K, dtype=torch.int32, device=dev)
     assign = torch.empty(RA, dtype=torch.int32, device=dev)
     x_sorted = torch.empty(RA, d, dtype=torch.bfloat16, device=dev)
@@ -226,31 +230,62 @@ def run_gpu(args, w) -> dict:
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
     h = torch.empty(RA, f, dtype=torch.bfloat16, device=dev)
     y = torch.empty(RA, d, dtype=torch.float32, device=dev)
-    out = torch.empty(N, d, dtype=torch.float32, device=dev)
+    if L > 1:  # x_{l+1} = bf16(x_l + MoE_l(x_l)), ping-pong buffers
+        xbuf = [torch.empty(N, d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        affinity = torch.zeros(L - 1, E, E, dtype=torch.int64, device=dev)
+        out = xbuf[(L - 1) % 2]
+    else:
+        out = torch.empty(N, d, dtype=torch.float32, device=dev)
+    if shared:  # Residual-MoE: the shared dense MLP on every token
+        sh = make_shared_inputs(w, seed=args.seed + rank, device=str(dev))
+        h_s = torch.empty(N, w.shared_f, dtype=torch.bfloat16, device=dev)
+        y_s = torch.empty(N, d, dtype=torch.float32, device=dev)
+        ws_s = torch.empty(256, dtype=torch.uint8, device=dev)
 
-    n_ev = 6
-    launches_per_step = 9  # logits, top-K, histogram, scan, positions, scatter, up, down, combine
+    stage_names = ["route", "dispatch", "expert_up", "expert_down"] + (
+        ["shared_expert"] if shared else []) + ["combine"]
+    n_ev = len(stage_names) + 1
+    # per layer: logits, top-K, histogram, scan, positions, scatter, up, down, combine
+    # (+ offsets, shared up, shared down for the Residual-MoE layer); + affinity per layer pair
+    launches_per_step = L * (9 + (3 if shared else 0)) + (L - 1)
 
     def step(ev=None):
+        """One step; ev (optional) is [layer][n_ev] events around the stages."""
         st = torch.cuda.current_stream(dev)
-        if ev is not None:
-            ev[0].record(st)
-        m.moe_route(shape, x, wr, bias, topk_idx, topk_w, None, ws, st)
-        if ev is not None:
-            ev[1].record(st)
-        m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted,
-                       x_packed, D, pk_off, None, ws, st)
-        if ev is not None:
-            ev[2].record(st)
-        m.moe_expert_up(shape, x_sorted, offsets, w1, w3, h, st)
-        if ev is not None:
-            ev[3].record(st)
-        m.moe_expert_down(shape, h, offsets, w2, y, st)
-        if ev is not None:
-            ev[4].record(st)
-        m.moe_combine(shape, y, row_of, topk_w, out, None, st)
-        if ev is not None:
-            ev[5].record(st)
+        for l in range(L):
+            lw = layers[l]
+            xin = x if l == 0 else xbuf[(l - 1) % 2]
+            dst = xbuf[l % 2] if L > 1 else out
+            e = ev[l] if ev is not None else None
+            if e is not None:
+                e[0].record(st)
+            m.moe_route(shape, xin, lw["w_router"], lw["bias"], topk_idx[l], topk_w, None, ws, st)
+            if e is not None:
+                e[1].record(st)
+            m.moe_dispatch(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of, assign,
+                           x_sorted, x_packed, D, pk_off, None, ws, st)
+            if e is not None:
+                e[2].record(st)
+            m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
+            if e is not None:
+                e[3].record(st)
+            m.moe_expert_down(shape, h, offsets[l], lw["w2"], y, st)
+            j = 4
+            if e is not None:
+                e[j].record(st)
+            if shared:
+                m.moe_shared_expert(shape, w.shared_f, xin, sh["ws1"], sh["ws3"], sh["ws2"], h_s,
+                                    y_s, ws_s, st)
+                j += 1
+                if e is not None:
+                    e[j].record(st)
+            m.moe_combine(shape, y, row_of, topk_w, dst, residual=xin if L > 1 else None,
+                          shared_y=y_s if shared else None, stream=st)
+            if e is not None:
+                e[j + 1].record(st)
+            if l > 0:
+                m.moe_affinity_accumulate(N, E, K, topk_idx[l - 1], topk_idx[l], affinity[l - 1],
+                                          st)
 
     for _ in range(args.warmup):
         step()
@@ -260,7 +295,8 @@ def run_gpu(args, w) -> dict:
 
     # the timed run: K eager steps, CUDA events between the stages of every step (on the
     # stream the kernels run on), barrier + synchronize on both sides
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    events = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(L)]
+              for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -273,9 +309,10 @@ def run_gpu(args, w) -> dict:
         torch.cuda.synchronize(dev)
     barrier()
     elapsed_s = t_start.elapsed_time(t_stop) / 1e3
-    stage_ms = {name: statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in events)
-                for j, name in enumerate(["route", "dispatch", "expert_up", "expert_down",
-                                          "combine"])}
+    # per stage: mean over steps of the sum over the stack's layers
+    stage_ms = {name: statistics.mean(sum(ev[l][j].elapsed_time(ev[l][j + 1]) for l in range(L))
+                                      for ev in events)
+                for j, name in enumerate(stage_names)}
 
     # the same step captured once in a CUDA graph (its 9 kernels) and replayed K times: the
     # host launch overhead disappears, which matters for small (decode) steps
@@ -301,7 +338,8 @@ def run_gpu(args, w) -> dict:
                      "ms_per_step": g_agg["elapsed_max_s"] / args.steps * 1e3}
         del graph
     err = m.moe_get_device_error(True)
-    R = int(offsets[E].item())
+    R_layers = [int(o[E].item()) for o in offsets]
+    R = R_layers[0]
     agg = aggregate(float(N * args.steps), elapsed_s, dev)
 
     # end to end through the public API: pinned host input -> moe_layer -> host output
@@ -310,11 +348,15 @@ def run_gpu(args, w) -> dict:
     # of the previous one (two buffers, one copy stream each way)
     e2e = None
     if not args.no_e2e:
-        lws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
+        lws_bytes = (m.moe_layer_shared_workspace_size(shape, w.shared_f) if shared
+                     else m.moe_layer_workspace_size(shape))
+        lws = torch.empty(lws_bytes, dtype=torch.uint8, device=dev)
         x_host = x.cpu().pin_memory()
-        out_host = [torch.empty(N, d, dtype=torch.float32).pin_memory() for _ in range(2)]
+        out_dt = torch.bfloat16 if L > 1 else torch.float32
+        out_host = [torch.empty(N, d, dtype=out_dt).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]
-        out_dev = [torch.empty(N, d, dtype=torch.float32, device=dev) for _ in range(2)]
+        out_dev = [torch.empty(N, d, dtype=out_dt, device=dev) for _ in range(2)]
+        mid = [torch.empty_like(x) for _ in range(2)] if L > 1 else None
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_comp = [torch.cuda.Event() for _ in range(2)]
@@ -328,7 +370,22 @@ def run_gpu(args, w) -> dict:
             ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_out[b])  # buffer b's previous result has left the device
-            m.moe_layer(shape, x_dev[b], wr, bias, w1, w3, w2, out_dev[b], ws=lws, stream=stream)
+            l0 = layers[0]
+            if shared:
+                m.moe_layer_shared(shape, w.shared_f, x_dev[b], l0["w_router"], l0["bias"],
+                                   l0["w1"], l0["w3"], l0["w2"], sh["ws1"], sh["ws3"], sh["ws2"],
+                                   out_dev[b], ws=lws, stream=stream)
+            elif L == 1:
+                m.moe_layer(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1"], l0["w3"],
+                            l0["w2"], out_dev[b], ws=lws, stream=stream)
+            else:  # the stack: each layer adds its MoE output to its input, bf16 in between
+                xin = x_dev[b]
+                for l in range(L):
+                    lw = layers[l]
+                    dst = out_dev[b] if l == L - 1 else mid[l % 2]
+                    m.moe_layer(shape, xin, lw["w_router"], lw["bias"], lw["w1"], lw["w3"],
+                                lw["w2"], dst, residual=xin, ws=lws, stream=stream)
+                    xin = dst
             ev_comp[b].record(stream)
             s_out.wait_event(ev_comp[b])
             with torch.cuda.stream(s_out):
@@ -353,11 +410,15 @@ def run_gpu(args, w) -> dict:
         barrier()
         e2e_agg = aggregate(float(N * args.steps), e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": e2e_agg["value"], "unit": UNIT, "h2d_bytes_per_step": N * d * 2,
-               "d2h_bytes_per_step": N * d * 4,
+               "d2h_bytes_per_step": N * d * (2 if L > 1 else 4),
                "note": "pinned host input and output; copies overlap the previous step's layer"}
         del lws
 
-    work = algorithmic_work(w, R)
+    # algorithmic work of one step (all layers of a stack)
+    work = {}
+    for Rl in R_layers:
+        for k, v in algorithmic_work(w, Rl).items():
+            work[k] = work.get(k, 0.0) + v
     peaks = load_peaks()
     up_s = stage_ms["expert_up"] / 1e3
     down_s = stage_ms["expert_down"] / 1e3
@@ -382,8 +443,10 @@ def run_gpu(args, w) -> dict:
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",
         "config": {"workload": w.name, "N": N, "d": d, "f": f, "E": E, "K": K, "W": W,
+                   "shared_f": w.shared_f,
                    "capacity_factor": w.cf if w.cf > 0 else "dropless", "zipf_s": w.s,
-                   "rows_kept": R, "parallelism": f"replicas x{world}",
+                   "rows_kept": R_layers if L > 1 else R, "layers": L,
+                   "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step"},
         "roofline": {"kernel": "grouped GEMM gate/up (moe_expert_up, CTA-pair tcgen05 kernel)",
@@ -393,11 +456,14 @@ def run_gpu(args, w) -> dict:
                      "peak_source": peaks["source"] + " bf16 burst",
                      "frac_of_sustained": up_tflops / peaks["bf16_tflops_sustained"],
                      "traffic": up_traffic(w.name),
-                     "algorithmic_flops_per_launch": work["up_flops"]},
+                     "algorithmic_flops_per_launch": work["up_flops"] / L},
         "stages_ms": stages,
         "grouped_gemm": {"tflops": gemm_tflops, "frac_of_bf16_peak": gemm_tflops / peaks["bf16_tflops"],
                          "frac_of_bf16_sustained": gemm_tflops / peaks["bf16_tflops_sustained"]},
         "combine": {"gbs": comb_gbs, "frac_of_hbm": comb_gbs / hbm, "frac_of_8tbs": comb_gbs / 8000.0},
+        "shared_expert": ({"ms": stage_ms["shared_expert"],
+                           "tflops": 6.0 * d * w.shared_f * N / (stage_ms["shared_expert"] / 1e3) / 1e12}
+                          if shared else None),
         "dispatch": {"ms": stage_ms["dispatch"],
                      "scatter_bytes": work["scatter_bytes"]},
         "clocks": clocks.summary(),
@@ -407,7 +473,8 @@ def run_gpu(args, w) -> dict:
         "e2e": e2e,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_sample_tokens)
+        res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_sample_tokens,
+                                           sh if shared else None)
     return res if rank == 0 else None
 
 
@@ -426,9 +493,10 @@ def load_peaks() -> dict:
 
 # --------------------------------------------------------------------------- CPU oracle legs
 
-def oracle_time(w, inp_cpu, sample_tokens: int) -> dict:
+def oracle_time(w, inp_cpu, sample_tokens: int, shared_cpu=None) -> dict:
     """Times the oracle on a bounded sample: routing + dispatch for every token,
-    expert FFN + combine for `sample_tokens` tokens; extrapolates to the layer."""
+    expert FFN + combine (and the shared dense MLP, for a Residual-MoE layer) for
+    `sample_tokens` tokens; extrapolates to the layer."""
     import numpy as np
 
     import oracle
@@ -441,10 +509,18 @@ def oracle_time(w, inp_cpu, sample_tokens: int) -> dict:
     toks = np.sort(rng.choice(w.N, size=min(sample_tokens, w.N), replace=False))
     t1 = time.perf_counter()
     oracle.layer_sampled(inp_cpu, w.K, w.W, w.cf, toks, routing=r)
+    if shared_cpu is not None:
+        oracle.shared_expert(inp_cpu["x"][torch_index(toks)], shared_cpu["ws1"], shared_cpu["ws3"],
+                             shared_cpu["ws2"])
     t_exp = time.perf_counter() - t1
     t_full = t_route + t_exp * (w.N / len(toks))
     return dict(value=w.N / t_full, t_route_s=t_route, t_expert_sample_s=t_exp,
                 sample_tokens=int(len(toks)), extrapolated_layer_s=t_full)
+
+
+def torch_index(toks):
+    import torch
+    return torch.from_numpy(toks)
 
 
 def cpu_threads() -> int:
@@ -452,13 +528,16 @@ def cpu_threads() -> int:
     return int(n) if n else (os.cpu_count() or 1)
 
 
-def cpu_baseline(w, inp, sample_tokens: int) -> dict:
+def cpu_baseline(w, inp, sample_tokens: int, shared=None) -> dict:
     inp_cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
-    t = oracle_time(w, inp_cpu, sample_tokens)
-    return {"value": t["value"], "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+    sh_cpu = None if shared is None else {k: v.cpu() for k, v in shared.items()}
+    t = oracle_time(w, inp_cpu, sample_tokens, sh_cpu)
+    stack = f"; one layer timed, x{w.layers} for the stack" if w.layers > 1 else ""
+    return {"value": t["value"] / w.layers, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
             "sample": f"routing + dispatch for all {w.N} tokens; expert FFN + combine for "
                       f"{t['sample_tokens']} tokens, extrapolated to {w.N} "
-                      f"(route {t['t_route_s']:.2f} s, experts {t['t_expert_sample_s']:.2f} s)"}
+                      f"(route {t['t_route_s']:.2f} s, experts {t['t_expert_sample_s']:.2f} s)"
+                      + stack}
 
 
 def run_reference(args, w) -> dict:
@@ -469,12 +548,16 @@ def run_reference(args, w) -> dict:
     if rank != 0:
         return None
     inp = make_layer_inputs(w, seed=args.seed, device="cpu")
+    sh = None
+    if w.shared_f > 0:
+        from moe_workloads import make_shared_inputs
+        sh = make_shared_inputs(w, seed=args.seed, device="cpu")
     times, values = [], []
     for i in range(args.warmup + args.steps):
-        t = oracle_time(w, inp, args.ref_sample_tokens)
+        t = oracle_time(w, inp, args.ref_sample_tokens, sh)
         if i >= args.warmup:
-            times.append(t["extrapolated_layer_s"])
-            values.append(t["value"])
+            times.append(t["extrapolated_layer_s"] * w.layers)  # one layer timed, x layers
+            values.append(t["value"] / w.layers)
     total = sum(times)
     value = w.N * len(times) / total
     res = {

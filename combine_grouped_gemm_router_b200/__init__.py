@@ -63,7 +63,10 @@ _sigs = {
     "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
     "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
     "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
-    "moe_combine": ([_SP] + [c_p] * 6, c_i32),
+    "moe_combine": ([_SP] + [c_p] * 7, c_i32),
+    "moe_shared_expert": ([_SP, c_i32] + [c_p] * 7 + [c_size, c_p], c_i32),
+    "moe_layer_shared_workspace_size": ([_SP, c_i32], c_size),
+    "moe_layer_shared": ([_SP, c_i32] + [c_p] * 14 + [c_size, c_p], c_i32),
     "moe_layer": ([_SP] + [c_p] * 11 + [c_size, c_p], c_i32),
     "moe_affinity_accumulate": ([c_i32, c_i32, c_i32, c_p, c_p, c_p, c_p], c_i32),
     "moe_derive_report": ([_SP, ctypes.POINTER(MoeStats), c_p, c_p, ctypes.POINTER(MoeReport)],
@@ -215,9 +218,31 @@ def moe_expert_down(shape, h, offsets, w2, y, stream=None):
                                 _stream(stream)), "moe_expert_down")
 
 
-def moe_combine(shape, y, row_of, topk_w, out, residual=None, stream=None):
+def moe_combine(shape, y, row_of, topk_w, out, residual=None, shared_y=None, stream=None):
     _check(_lib.moe_combine(ctypes.byref(shape), _ptr(y), _ptr(row_of), _ptr(topk_w),
-                            _ptr(residual), _ptr(out), _stream(stream)), "moe_combine")
+                            _ptr(shared_y), _ptr(residual), _ptr(out), _stream(stream)),
+           "moe_combine")
+
+
+def moe_shared_expert(shape, f_shared, x, ws1, ws3, ws2, h_s, y_s, ws, stream=None):
+    _check(_lib.moe_shared_expert(ctypes.byref(shape), int(f_shared), _ptr(x), _ptr(ws1),
+                                  _ptr(ws3), _ptr(ws2), _ptr(h_s), _ptr(y_s), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_shared_expert")
+
+
+def moe_layer_shared_workspace_size(shape, f_shared) -> int:
+    return _lib.moe_layer_shared_workspace_size(ctypes.byref(shape), int(f_shared))
+
+
+def moe_layer_shared(shape, f_shared, x, w_router, bias, w1, w3, w2, ws1, ws3, ws2, out,
+                     residual=None, topk_idx_out=None, stats=None, ws=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_layer_shared(ctypes.byref(shape), int(f_shared), _ptr(x), _ptr(w_router),
+                                 _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(ws1), _ptr(ws3),
+                                 _ptr(ws2), _ptr(residual), _ptr(out), _ptr(topk_idx_out),
+                                 _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_layer_shared")
 
 
 def moe_layer(shape, x, w_router, bias, w1, w3, w2, out, residual=None, topk_idx_out=None,

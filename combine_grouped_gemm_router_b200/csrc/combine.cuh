@@ -10,14 +10,17 @@ namespace moe {
 // [MoE 推理服务工程真相 2026, §2.2] a dropped slot's router output is zero.
 // One warp per token; each lane owns 16-byte column chunks; the K rows are
 // gathered (fp32 expert outputs) and accumulated in fp32 in slot order
-// k = 0..K-1. An optional bf16 residual row is added last, in fp32: the
-// inter-layer step of a stack of MoE layers, x_{j+1} = x_j + MoE_j(x_j). The
+// k = 0..K-1. Then, optionally and in this order, the fp32 output of a shared
+// dense MLP is added ([MoE Inference Communication, §PR-MoE]: Residual-MoE adds
+// the shared MLP's and the routed experts' outputs) and a bf16 residual row (the
+// inter-layer step of a stack of MoE layers, x_{j+1} = x_j + MoE_j(x_j)). The
 // result is stored as fp32, or rounded once to bf16 (OUT_BF16).
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ row_of,
-                   const float *__restrict__ topk_w, const uint16_t *__restrict__ residual,
-                   int N, int d, int K, void *__restrict__ out)
+                   const float *__restrict__ topk_w, const float *__restrict__ shared_y,
+                   const uint16_t *__restrict__ residual, int N, int d, int K,
+                   void *__restrict__ out)
 {
     constexpr int U = 2;
     const int lane = threadIdx.x & 31;
@@ -60,6 +63,20 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             acc[u][q] = __fmaf_rn(wk, f8[q], acc[u][q]);
+                    }
+                }
+            }
+            if (shared_y) {
+                const float4 *ssrc = reinterpret_cast<const float4 *>(shared_y);
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (c + 32 * u < nvec) {
+                        const size_t chunk = (size_t)t * nvec + c + 32 * u;
+                        const float4 a = ssrc[chunk * 2], b = ssrc[chunk * 2 + 1];
+                        const float f8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            acc[u][q] = __fadd_rn(acc[u][q], f8[q]);
                     }
                 }
             }

@@ -378,55 +378,69 @@ bool use_pair_tiles(const moe_shape_t *s, const Geometry &g)
     return rows >= 192;
 }
 
+// Grouped GEMM launches for E experts of width f over an A buffer of a_rows rows (the
+// tensor map's extent: rows past it read as zeros). `pair` selects the CTA-pair kernel.
+moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *a,
+                     const int32_t *offsets, const uint16_t *w1, const uint16_t *w3, uint16_t *h,
+                     cudaStream_t st)
+{
+    CUtensorMap tA, tW1, tW3;
+    if (!make_tmap(&tA, a, d, (uint64_t)a_rows) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
+        !make_tmap(&tW3, w3, d, (uint64_t)E * f))
+        return MOE_ERR_CUDA;
+    gg::Args args;
+    args.offsets = offsets;
+    args.E = E;
+    args.n_tiles = f / 128;
+    args.k_blocks = d / gg::BK;
+    args.b_rows = f;
+    args.rows_alloc = (int)a_rows;
+    args.out = h;
+    args.ldo = f;
+    args.timeout_ns = kWaitTimeoutNs;
+    if (pair)
+        return launch_gemm_pair<0>(tA, tW1, tW3, args, st);
+    return launch_gemm<0, 256>(tA, tW1, tW3, args, st);
+}
+
+moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
+                       const int32_t *offsets, const uint16_t *w2, float *y, cudaStream_t st)
+{
+    CUtensorMap tA, tW2;
+    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
+        return MOE_ERR_CUDA;
+    gg::Args args;
+    args.offsets = offsets;
+    args.E = E;
+    args.k_blocks = f / gg::BK;
+    args.b_rows = d;
+    args.rows_alloc = (int)a_rows;
+    args.out = y;
+    args.ldo = d;
+    args.timeout_ns = kWaitTimeoutNs;
+    if (d % 256 == 0) {
+        args.n_tiles = d / 256;
+        if (pair)
+            return launch_gemm_pair<1>(tA, tW2, tW2, args, st);
+        return launch_gemm<1, 256>(tA, tW2, tW2, args, st);
+    }
+    args.n_tiles = d / 128;
+    return launch_gemm<1, 128>(tA, tW2, tW2, args, st);
+}
+
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                             uint16_t *h, cudaStream_t st)
 {
-    const int d = s->d, f = s->f, E = s->E;
-    CUtensorMap tA, tW1, tW3;
-    if (!make_tmap(&tA, x_sorted, d, g.rows_alloc) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
-        !make_tmap(&tW3, w3, d, (uint64_t)E * f))
-        return MOE_ERR_CUDA;
-    gg::Args a;
-    a.offsets = offsets;
-    a.E = E;
-    a.n_tiles = f / 128;
-    a.k_blocks = d / gg::BK;
-    a.b_rows = f;
-    a.rows_alloc = (int)g.rows_alloc;
-    a.out = h;
-    a.ldo = f;
-    a.timeout_ns = kWaitTimeoutNs;
-    if (use_pair_tiles(s, g))
-        return launch_gemm_pair<0>(tA, tW1, tW3, a, st);
-    return launch_gemm<0, 256>(tA, tW1, tW3, a, st);
+    return gemm_up(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), x_sorted, offsets, w1,
+                   w3, h, st);
 }
 
 moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *h,
                               const int32_t *offsets, const uint16_t *w2, float *y,
                               cudaStream_t st)
 {
-    const int d = s->d, f = s->f, E = s->E;
-    CUtensorMap tA, tW2;
-    if (!make_tmap(&tA, h, f, g.rows_alloc) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
-        return MOE_ERR_CUDA;
-    gg::Args a;
-    a.offsets = offsets;
-    a.E = E;
-    a.k_blocks = f / gg::BK;
-    a.b_rows = d;
-    a.rows_alloc = (int)g.rows_alloc;
-    a.out = y;
-    a.ldo = d;
-    a.timeout_ns = kWaitTimeoutNs;
-    if (d % 256 == 0) {
-        a.n_tiles = d / 256;
-        if (use_pair_tiles(s, g))
-            return launch_gemm_pair<1>(tA, tW2, tW2, a, st);
-        return launch_gemm<1, 256>(tA, tW2, tW2, a, st);
-    }
-    a.n_tiles = d / 128;
-    return launch_gemm<1, 128>(tA, tW2, tW2, a, st);
+    return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y, st);
 }
 
 moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
@@ -439,16 +453,35 @@ moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uin
     return expert_down_impl(s, g, h, offsets, w2, y, st);
 }
 
+// The shared dense MLP of a Residual-MoE layer: one "expert" that owns all N rows of x.
+__global__ void whole_range_offsets_kernel(int32_t *o, int n)
+{
+    o[0] = 0;
+    o[1] = n;
+}
+
+moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x,
+                                const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2,
+                                uint16_t *h_s, float *y_s, int32_t *offsets2, cudaStream_t st)
+{
+    whole_range_offsets_kernel<<<1, 1, 0, st>>>(offsets2, s->N);
+    const bool pair = s->N >= 192;
+    moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, st);
+    if (rc != MOE_OK)
+        return rc;
+    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, st);
+}
+
 moe_status_t combine_impl(const moe_shape_t *s, const float *y, const int32_t *row_of,
-                          const float *topk_w, const uint16_t *residual, void *out,
-                          cudaStream_t st)
+                          const float *topk_w, const float *shared_y, const uint16_t *residual,
+                          void *out, cudaStream_t st)
 {
     if (s->flags & MOE_FLAG_OUT_BF16)
-        combine_kernel<true><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, residual, s->N,
-                                                              s->d, s->K, out);
+        combine_kernel<true><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, shared_y,
+                                                              residual, s->N, s->d, s->K, out);
     else
-        combine_kernel<false><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, residual, s->N,
-                                                               s->d, s->K, out);
+        combine_kernel<false><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, shared_y,
+                                                               residual, s->N, s->d, s->K, out);
     return launch_status();
 }
 
@@ -619,7 +652,8 @@ moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offs
 
 __attribute__((visibility("default"))) moe_status_t
 moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
-            const float *topk_w, const uint16_t *residual, void *out, moe_stream_t stream)
+            const float *topk_w, const float *shared_y, const uint16_t *residual, void *out,
+            moe_stream_t stream)
 {
     moe_status_t rc = check_shape(shape, false, nullptr);
     if (rc != MOE_OK)
@@ -627,9 +661,9 @@ moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
     if (!y || !row_of || !topk_w || !out)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(y) || !aligned16(out) || !aligned4(row_of) || !aligned4(topk_w) ||
-        (residual && !aligned16(residual)))
+        (residual && !aligned16(residual)) || (shared_y && !aligned16(shared_y)))
         return MOE_ERR_MISALIGNED;
-    return combine_impl(shape, y, row_of, topk_w, residual, out,
+    return combine_impl(shape, y, row_of, topk_w, shared_y, residual, out,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -687,7 +721,108 @@ moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
     rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
     if (rc != MOE_OK)
         return rc;
-    return combine_impl(shape, y, row_of, topk_w, residual, out, st);
+    return combine_impl(shape, y, row_of, topk_w, nullptr, residual, out, st);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
+                  const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2, uint16_t *h_s,
+                  float *y_s, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    moe_status_t rc = check_shape(shape, true, nullptr);
+    if (rc != MOE_OK)
+        return rc;
+    if (f_shared < 128 || f_shared % 128 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !ws1 || !ws3 || !ws2 || !h_s || !y_s)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(ws1) || !aligned16(ws3) || !aligned16(ws2) ||
+        !aligned16(h_s) || !aligned16(y_s))
+        return MOE_ERR_MISALIGNED;
+    if (!ws || ws_bytes < kAlign)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    return shared_expert_impl(shape, f_shared, x, ws1, ws3, ws2, h_s, y_s,
+                              static_cast<int32_t *>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) size_t
+moe_layer_shared_workspace_size(const moe_shape_t *shape, int32_t f_shared)
+{
+    const size_t base = moe_layer_workspace_size(shape);
+    if (base == 0 || f_shared < 128 || f_shared % 128 != 0)
+        return 0;
+    return base + align_up((size_t)shape->N * f_shared * 2) + align_up((size_t)shape->N * shape->d * 4) +
+           kAlign;
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
+                 const float *w_router, const float *bias, const uint16_t *w1,
+                 const uint16_t *w3, const uint16_t *w2, const uint16_t *ws1, const uint16_t *ws3,
+                 const uint16_t *ws2, const uint16_t *residual, void *out, int32_t *topk_idx_out,
+                 moe_stats_t *stats, void *ws, size_t ws_bytes, moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (f_shared < 128 || f_shared % 128 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!x || !w_router || !w1 || !w3 || !w2 || !ws1 || !ws3 || !ws2 || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1) ||
+        !aligned16(w3) || !aligned16(w2) || !aligned16(ws1) || !aligned16(ws3) ||
+        !aligned16(ws2) || !aligned16(out) || (residual && !aligned16(residual)) ||
+        (topk_idx_out && !aligned4(topk_idx_out)) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const size_t need = moe_layer_shared_workspace_size(shape, f_shared);
+    if (!ws || ws_bytes < need)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    const ScratchLayout S = scratch_layout(shape, g);
+    const LayerLayout L = layer_layout(shape, g, S.total);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char *w = static_cast<char *>(ws);
+    uint16_t *h_s = reinterpret_cast<uint16_t *>(w + L.total);
+    float *y_s = reinterpret_cast<float *>(w + L.total + align_up((size_t)shape->N * f_shared * 2));
+    int32_t *off2 = reinterpret_cast<int32_t *>(w + need - kAlign);
+    int32_t *topk_idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(w + L.topk_idx);
+    float *topk_w = reinterpret_cast<float *>(w + L.topk_w);
+    unsigned long long *nonfinite = nullptr;
+    if (stats) {
+        nonfinite = reinterpret_cast<unsigned long long *>(&stats->nonfinite_tokens);
+        if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
+                    reinterpret_cast<float *>(w + S.logits), nonfinite, st);
+    if (rc != MOE_OK)
+        return rc;
+    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+    int32_t *row_of = reinterpret_cast<int32_t *>(w + L.row_of);
+    uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
+    uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
+    float *y = reinterpret_cast<float *>(w + L.y);
+    rc = dispatch_impl(shape, g, x, topk_idx, reinterpret_cast<int32_t *>(w + L.counts),
+                       reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
+                       reinterpret_cast<int32_t *>(w + L.assign), x_sorted,
+                       reinterpret_cast<uint16_t *>(w + L.x_packed),
+                       reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
+                       stats, reinterpret_cast<int32_t *>(w + S.blk),
+                       reinterpret_cast<int64_t *>(w + S.pk_base), st);
+    if (rc != MOE_OK)
+        return rc;
+    rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
+    if (rc != MOE_OK)
+        return rc;
+    rc = shared_expert_impl(shape, f_shared, x, ws1, ws3, ws2, h_s, y_s, off2, st);
+    if (rc != MOE_OK)
+        return rc;
+    return combine_impl(shape, y, row_of, topk_w, y_s, residual, out, st);
 }
 
 __attribute__((visibility("default"))) moe_status_t

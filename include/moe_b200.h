@@ -219,12 +219,35 @@ moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const 
  *  original token order, then on to the next layer); MoE 推理服务工程真相 2026, §2.2 (a
  *  dropped slot contributes 0)]
  * out[t] = (sum over k = 0..K-1 with row_of[t*K+k] >= 0 of topk_w[t][k] * y[row])
- *          + residual[t], accumulated in fp32 in k order, the residual (nullable, bf16
- * [N][d]) added last. y [rows_alloc][d] fp32. out [N][d] is fp32, or bf16 (rounded once)
- * when shape->flags has MOE_FLAG_OUT_BF16; a bf16 out may alias residual. */
+ *          + shared_y[t] + residual[t], accumulated in fp32 in k order, then the shared dense
+ * MLP's output (nullable, fp32 [N][d], see moe_shared_expert), then the residual (nullable,
+ * bf16 [N][d]). y [rows_alloc][d] fp32. out [N][d] is fp32, or bf16 (rounded once) when
+ * shape->flags has MOE_FLAG_OUT_BF16; a bf16 out may alias residual. */
 moe_status_t moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
-                         const float *topk_w, const uint16_t *residual, void *out,
-                         moe_stream_t stream);
+                         const float *topk_w, const float *shared_y, const uint16_t *residual,
+                         void *out, moe_stream_t stream);
+
+/* The shared dense MLP of a Residual-MoE layer, for every token, on the same tcgen05 grouped GEMM
+ * (one "expert" that owns all N rows of x).
+ * [MoE Inference Communication, §DeepSpeed-MoE › PR-MoE, 现象二 / Residual: a dense MLP every
+ *  token passes through, added to the output of the routed expert(s)]
+ * Same SwiGLU form as the experts: h_s = silu(x Ws1^T) * (x Ws3^T) (bf16), y_s = h_s Ws2^T (fp32).
+ * x [N][d]; ws1, ws3 [f_shared][d]; ws2 [d][f_shared]; h_s [N][f_shared]; y_s [N][d] fp32.
+ * f_shared % 128 == 0. ws: at least 256 bytes of device scratch. */
+moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
+                               const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2,
+                               uint16_t *h_s, float *y_s, void *ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/* Residual-MoE layer: moe_layer's routed path plus the shared dense MLP, the two outputs
+ * added in the combine (then the optional residual). Workspace: moe_layer_shared_workspace_size. */
+size_t moe_layer_shared_workspace_size(const moe_shape_t *shape, int32_t f_shared);
+moe_status_t moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
+                              const float *w_router, const float *bias, const uint16_t *w1,
+                              const uint16_t *w3, const uint16_t *w2, const uint16_t *ws1,
+                              const uint16_t *ws3, const uint16_t *ws2, const uint16_t *residual,
+                              void *out, int32_t *topk_idx_out, moe_stats_t *stats, void *ws,
+                              size_t ws_bytes, moe_stream_t stream);
 
 /* The whole layer: moe_route -> moe_dispatch (with the packed buffer) -> moe_expert_gemm ->
  * moe_combine, every intermediate in the workspace (moe_layer_workspace_size bytes).

@@ -14,6 +14,8 @@ Workloads (the shapes the pages' discussion turns on, made concrete):
 * ``decode``          N=16,    d=7168, f=2048,  E=256, K=8, W=8, dropless
 * ``stack4``          N=32768, d=4096, f=1536,  E=64,  K=6, W=8, L=4 layers,
                       cf in {1.0, 1.25, 2.0} x Zipf s in {0, 1.2}
+* ``residual_top1``   N=4096,  d=4096, f=14336, E=8,   K=1, W=8, dropless, plus a
+                      shared dense SwiGLU MLP of width 14336 (Residual-MoE)
 
 Recipe (one ``torch.Generator`` per call, ``manual_seed(seed)``; draw order
 x, router, W1, W3, W2; layer ``l`` of a stack re-seeds with ``seed + 1000*l``
@@ -49,6 +51,7 @@ class Workload:
     s: float = 0.0           # Zipf exponent of the per-expert bias; 0 = none
     router: str = "normal"   # "normal" (N(0,1/d)) or "uniform" (U(+-1/sqrt d))
     layers: int = 1
+    shared_f: int = 0        # width of the shared dense MLP (Residual-MoE); 0 = none
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -62,6 +65,9 @@ WORKLOADS = {
     "decode": Workload("decode", N=16, d=7168, f=2048, E=256, K=8, W=8),
     "stack4": Workload("stack4", N=32768, d=4096, f=1536, E=64, K=6, W=8, cf=1.25, s=0.0,
                        layers=4),
+    # Residual-MoE: top-1 routed experts plus a shared dense MLP of the same width
+    "residual_top1": Workload("residual_top1", N=4096, d=4096, f=14336, E=8, K=1, W=8,
+                              router="uniform", shared_f=14336),
     # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
     # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
     "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,
@@ -109,6 +115,19 @@ def make_layer_inputs(w: Workload, seed: int = 0, device: str = "cpu", layer: in
             t[e] = (torch.randn(shape[1:], generator=g, device=device, dtype=torch.float32)
                     * 0.02).to(torch.bfloat16)
         out[name] = t
+    return out
+
+
+def make_shared_inputs(w: Workload, seed: int = 0, device: str = "cpu", layer: int = 0) -> dict:
+    """Weights of the shared dense MLP (drawn after the layer's own inputs, from seed + 500):
+    ws1, ws3 [f_s][d], ws2 [d][f_s], bf16 ~ N(0, 0.02^2)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 500 + 1000 * layer)
+    out = {}
+    for name, shape in (("ws1", (w.shared_f, w.d)), ("ws3", (w.shared_f, w.d)),
+                        ("ws2", (w.d, w.shared_f))):
+        out[name] = (torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+                     * 0.02).to(torch.bfloat16)
     return out
 
 

@@ -242,6 +242,29 @@ def layer_sampled(inp: dict, K: int, W: int, cf: float, tokens: Sequence[int],
     return res
 
 
+def shared_expert(x, ws1, ws3, ws2) -> np.ndarray:
+    """The shared dense MLP of a Residual-MoE layer on every token: the same SwiGLU form as an
+    expert (W1s, W3s [f_s][d]; W2s [d][f_s]), computed by the expert routine with one expert
+    that owns every row [MoE Inference Communication, §PR-MoE, 现象二 (Residual-MoE)]."""
+    xs = as_u16(x)
+    N = xs.shape[0]
+    rows = np.arange(N, dtype=np.int32)
+    _, y = expert_rows(rows, np.zeros(N, np.int32), xs, as_u16(ws1)[None], as_u16(ws3)[None],
+                       as_u16(ws2)[None])
+    return y
+
+
+def layer_shared(inp: dict, shared: dict, K: int, W: int, cf: float, want_h: bool = False) -> dict:
+    """Residual-MoE layer: out = (sum over kept slots of w_k * expert output) + shared MLP(x).
+    [MoE Inference Communication, §PR-MoE: a shared dense MLP every token passes through plus
+    routed experts, the two outputs added]"""
+    r = layer(inp, K, W, cf, want_h)
+    r["shared_y"] = shared_expert(inp["x"], shared["ws1"], shared["ws3"], shared["ws2"])
+    r["out_routed"] = r["out"]
+    r["out"] = r["out_routed"] + r["shared_y"]
+    return r
+
+
 # --------------------------------------------------------------------------- report
 
 def dispatch_bytes(rows: int, d: int, elem_bytes: int) -> int:

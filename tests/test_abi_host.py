@@ -88,10 +88,15 @@ def test_argument_errors_return_before_launch(m):
     # null pointers
     assert lib.moe_route(by(s), None, P, None, P, P, P, None, 0, None) == 1
     assert lib.moe_expert_gemm(by(s), P, P, P, P, None, P, P, None) == 1
-    assert lib.moe_combine(by(s), P, P, P, None, None, None) == 1
+    assert lib.moe_combine(by(s), P, P, P, None, None, None, None) == 1
     # misaligned
     assert lib.moe_route(by(s), P + 2, P, None, P, P, P, None, 0, None) == 4
-    assert lib.moe_combine(by(s), P + 8, P, P, None, P, None) == 4
+    assert lib.moe_combine(by(s), P + 8, P, P, None, None, P, None) == 4
+    assert lib.moe_combine(by(s), P, P, P, P + 4, None, P, None) == 4  # misaligned shared_y
+    assert lib.moe_shared_expert(by(s), 100, P, P, P, P, P, P, P, 256, None) == 2
+    assert lib.moe_shared_expert(by(s), 128, P, P, P, P, P, P, P, 16, None) == 3
+    assert m.moe_layer_shared_workspace_size(s, 100) == 0
+    assert m.moe_layer_shared_workspace_size(s, 256) > m.moe_layer_workspace_size(s)
     # workspace too small (logits requested in the workspace)
     assert lib.moe_route(by(s), P, P, None, P, P, None, P, 16, None) == 3
     need = m.moe_workspace_size(s)

@@ -157,3 +157,41 @@ def test_stack_affinity_full_size(orc):
         P = c / np.maximum(n_i[:, None], 1)
         print(f"layer pair {j}->{j + 1}: max P(p|i) = {P.max():.3f}, diag mass "
               f"{np.trace(c) / c.sum():.4f}")
+
+
+def test_full_size_residual_moe(orc):
+    """Residual-MoE at the Mixtral shape with top-1 routing and a shared MLP of the same width:
+    routing in full, the layer output on sampled tokens (routed part + shared MLP)."""
+    import combine_grouped_gemm_router_b200 as m
+    from moe_workloads import make_shared_inputs
+    w = WORKLOADS["residual_top1"]
+    torch.cuda.empty_cache()
+    inp = make_layer_inputs(w, seed=0, device="cuda")
+    sh = make_shared_inputs(w, seed=0, device="cuda")
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    ws = torch.empty(m.moe_layer_shared_workspace_size(shape, w.shared_f), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
+    topk = torch.empty(w.N, w.K, dtype=torch.int32, device="cuda")
+    m.moe_layer_shared(shape, w.shared_f, inp["x"], inp["w_router"], inp["bias"], inp["w1"],
+                       inp["w3"], inp["w2"], sh["ws1"], sh["ws3"], sh["ws2"], out,
+                       topk_idx_out=topk, ws=ws)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_error(True) == 0
+    hx = host_inputs(inp, experts=[])
+    r = orc.route_and_dispatch(hx["x"], hx["w_router"], hx["bias"], w.K, w.W, w.cf)
+    np.testing.assert_array_equal(topk.cpu().numpy(), r["topk_idx"])
+    toks = sample_tokens(w.N, 16, 0)
+    slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
+    used = np.unique(r["topk_idx"].reshape(-1)[slots])
+    remap = np.full(w.E, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    hx = host_inputs(inp, experts=torch.from_numpy(used).cuda())
+    rr = dict(r)
+    rr["topk_idx"] = remap[r["topk_idx"]].astype(np.int32)
+    smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr)
+    dense = orc.shared_expert(hx["x"][torch.from_numpy(toks)], sh["ws1"].cpu(), sh["ws3"].cpu(),
+                              sh["ws2"].cpu())
+    rep = assert_within_tolerance(out[torch.from_numpy(toks).cuda()], smp["out_tokens"] + dense,
+                                  "residual-MoE sample")
+    print("residual_top1", rep)

@@ -169,3 +169,41 @@ def test_affinity_kernel_matches_oracle(orc):
                               cnt2)
     np.testing.assert_array_equal(cnt2.cpu().numpy(), orc.affinity(a2, b2, E2))
     assert m.moe_get_device_error(True) == 0
+
+
+def test_residual_moe_layer(orc):
+    """Residual-MoE: routed experts plus a shared dense MLP on every token, summed in the
+    combine. moe_shared_expert against the oracle's dense MLP; moe_layer_shared against the
+    oracle's layer and, bit for bit, against the same stages called one by one."""
+    import combine_grouped_gemm_router_b200 as m
+    from moe_workloads import make_shared_inputs
+    for w in (Workload("res_small", N=256, d=256, f=256, E=4, K=1, W=2, shared_f=384),
+              Workload("res_k2_drop", N=300, d=384, f=128, E=6, K=2, W=3, cf=1.0, s=1.1,
+                       shared_f=128)):
+        inp = make_layer_inputs(w, seed=1)
+        sh = make_shared_inputs(w, seed=1)
+        ref = orc.layer_shared(inp, sh, w.K, w.W, w.cf)
+        dev = torch.device("cuda")
+        shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+        shd = {k: v.to(dev) for k, v in sh.items()}
+        h_s = torch.empty(w.N, w.shared_f, dtype=torch.bfloat16, device=dev)
+        y_s = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+        ws_s = torch.empty(256, dtype=torch.uint8, device=dev)
+        x = inp["x"].to(dev)
+        m.moe_shared_expert(shape, w.shared_f, x, shd["ws1"], shd["ws3"], shd["ws2"], h_s, y_s, ws_s)
+        torch.cuda.synchronize()
+        assert_within_tolerance(y_s, ref["shared_y"], "shared MLP")
+        got = run_stages(inp, w)
+        out_st = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+        m.moe_combine(shape, got["y"], got["row_of"], got["topk_w"], out_st, shared_y=y_s)
+        ws = torch.empty(m.moe_layer_shared_workspace_size(shape, w.shared_f), dtype=torch.uint8,
+                         device=dev)
+        out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+        bias = None if inp["bias"] is None else inp["bias"].to(dev)
+        m.moe_layer_shared(shape, w.shared_f, x, inp["w_router"].to(dev), bias, inp["w1"].to(dev),
+                           inp["w3"].to(dev), inp["w2"].to(dev), shd["ws1"], shd["ws3"], shd["ws2"],
+                           out, ws=ws)
+        torch.cuda.synchronize()
+        assert m.moe_get_device_error(True) == 0
+        assert torch.equal(out, out_st)
+        assert_within_tolerance(out, ref["out"], w.name)

@@ -335,3 +335,27 @@ def test_sampled_layer_matches_full(orc):
     toks = [0, 5, 17, 47]
     smp = orc.layer_sampled(inp, w.K, w.W, w.cf, toks)
     np.testing.assert_allclose(smp["out_tokens"], full["out"][toks], rtol=1e-13, atol=1e-15)
+
+
+def test_residual_moe_oracle(orc):
+    """Residual-MoE [MoE Inference Communication, §PR-MoE]: the shared dense MLP equals a numpy
+    float64 SwiGLU on every token, and the layer output is the routed output plus it: with the
+    routed experts' down projections zeroed the layer is exactly the dense MLP."""
+    from moe_workloads import make_shared_inputs
+    w = Workload("res", N=40, d=64, f=64, E=4, K=1, W=2, shared_f=96)
+    inp = make_layer_inputs(w, seed=4)
+    sh = make_shared_inputs(w, seed=4)
+    r = orc.layer_shared(inp, sh, w.K, w.W, w.cf)
+    x = brute.bf16_bits_to_float(orc.as_u16(inp["x"])).astype(np.float64)
+    a = brute.bf16_bits_to_float(orc.as_u16(sh["ws1"])).astype(np.float64)
+    b = brute.bf16_bits_to_float(orc.as_u16(sh["ws3"])).astype(np.float64)
+    c = brute.bf16_bits_to_float(orc.as_u16(sh["ws2"])).astype(np.float64)
+    g, u = x @ a.T, x @ b.T
+    dense = (g / (1.0 + np.exp(-g)) * u) @ c.T
+    np.testing.assert_allclose(r["shared_y"], dense, rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(r["out"], r["out_routed"] + dense, rtol=1e-12, atol=1e-15)
+    assert np.all(r["topk_w"] == 1.0)  # top-1: the routed expert's weight is exactly 1
+    zero = dict(inp)
+    zero["w2"] = torch.zeros_like(inp["w2"])
+    r0 = orc.layer_shared(zero, sh, w.K, w.W, w.cf)
+    np.testing.assert_array_equal(r0["out"], r0["shared_y"])
