@@ -368,14 +368,16 @@ moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const
     return launch_status();
 }
 
-// The pair kernel computes 256-row tiles: worth it when experts hold a few hundred rows
-// or more (prefill); with fewer, the 128-row single-CTA tiles waste less work.
+// Kernel choice. With many rows per expert on average (prefill of a few large experts) both
+// kernels are launched and each expert goes to the one whose tiles waste less (on the device,
+// prefer_pair_tiles: 256-row pair tiles unless 128-row tiles save more than 10 %). With fewer
+// (decode, or many small experts where skewed routing leaves most experts a few hundred rows)
+// only the single-CTA kernel runs: measured faster there, its 128-row tiles wasting less.
 bool use_pair_tiles(const moe_shape_t *s, const Geometry &g)
 {
-    // (the pair kernel steps K by 128: d and f are multiples of 128 for every GEMM shape)
     const int64_t mean_rows = ((int64_t)s->N * s->K) / s->E;
     const int64_t rows = mean_rows < g.C ? mean_rows : g.C;
-    return rows >= 192;
+    return rows >= 768;
 }
 
 // Grouped GEMM launches for E experts of width f over an A buffer of a_rows rows (the
@@ -398,8 +400,14 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
     args.out = h;
     args.ldo = f;
     args.timeout_ns = kWaitTimeoutNs;
-    if (pair)
-        return launch_gemm_pair<0>(tA, tW1, tW3, args, st);
+    args.select = 0;
+    if (pair) {
+        args.select = 1;
+        moe_status_t rc = launch_gemm_pair<0>(tA, tW1, tW3, args, st);
+        if (rc != MOE_OK)
+            return rc;
+        args.select = 2;
+    }
     return launch_gemm<0, 256>(tA, tW1, tW3, args, st);
 }
 
@@ -418,10 +426,16 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     args.out = y;
     args.ldo = d;
     args.timeout_ns = kWaitTimeoutNs;
+    args.select = 0;
     if (d % 256 == 0) {
         args.n_tiles = d / 256;
-        if (pair)
-            return launch_gemm_pair<1>(tA, tW2, tW2, args, st);
+        if (pair) {
+            args.select = 1;
+            moe_status_t rc = launch_gemm_pair<1>(tA, tW2, tW2, args, st);
+            if (rc != MOE_OK)
+                return rc;
+            args.select = 2;
+        }
         return launch_gemm<1, 256>(tA, tW2, tW2, args, st);
     }
     args.n_tiles = d / 128;
@@ -465,7 +479,7 @@ moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x
                                 uint16_t *h_s, float *y_s, int32_t *offsets2, cudaStream_t st)
 {
     whole_range_offsets_kernel<<<1, 1, 0, st>>>(offsets2, s->N);
-    const bool pair = s->N >= 192;
+    const bool pair = s->N >= 768;
     moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, st);
     if (rc != MOE_OK)
         return rc;

@@ -28,6 +28,11 @@ CASES = [
     Workload("odd_e", N=100, d=128, f=128, E=5, K=2, W=5, cf=0.9),
     Workload("one_token_per_rank", N=8, d=128, f=128, E=16, K=3, W=8, cf=0.5),
     Workload("wide_k", N=96, d=128, f=128, E=48, K=32, W=4),
+    # >= 768 rows per expert on average: the CTA-pair GEMM kernel (256-row tiles)
+    Workload("pair_tiles", N=1600, d=256, f=256, E=2, K=1, W=2),
+    # skewed rows (Zipf bias): large experts on the pair kernel, small ones on the
+    # single-CTA kernel, in the same GEMM
+    Workload("pair_split", N=3200, d=256, f=256, E=4, K=1, W=4, s=1.6),
 ]
 
 
