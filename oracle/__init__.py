@@ -55,6 +55,8 @@ def _load():
         lib.orc_capacity.restype = _i64
         lib.orc_positions.argtypes = [_i64] * 5 + [_p] * 10
         lib.orc_positions.restype = None
+        lib.orc_positions_ordered.argtypes = [_i64] * 6 + [_p] * 10
+        lib.orc_positions_ordered.restype = None
         lib.orc_expert_rows.argtypes = [_i64, _p, _p, _i64, _i64, _p, _p, _p, _p, _p, _p]
         lib.orc_expert_rows.restype = None
         lib.orc_combine.argtypes = [_i64, _i64, _i64, _p, _p, _p, _p]
@@ -115,7 +117,10 @@ def capacity(N: int, E: int, K: int, cf: float) -> int:
     return int(_load().orc_capacity(N, E, K, float(cf)))
 
 
-def positions(topk_idx: np.ndarray, E: int, W: int, C: int) -> dict:
+SLOT_MAJOR = 1  # priority order of positions() / route_and_dispatch(): 0 token-major
+
+
+def positions(topk_idx: np.ndarray, E: int, W: int, C: int, order: int = 0) -> dict:
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
     N, K = topk_idx.shape
     counts = np.empty(E, np.int32)
@@ -127,9 +132,9 @@ def positions(topk_idx: np.ndarray, E: int, W: int, C: int) -> dict:
     pk_off = np.empty(W * W + 1, np.int64)
     packed_row_of = np.empty(N * K, np.int32)
     stats = np.empty(8, np.int64)
-    _load().orc_positions(N, E, K, W, C, _ptr(topk_idx), _ptr(counts), _ptr(kept), _ptr(offsets),
-                          _ptr(row_of), _ptr(assign_of_row), _ptr(D), _ptr(pk_off),
-                          _ptr(packed_row_of), _ptr(stats))
+    _load().orc_positions_ordered(N, E, K, W, C, order, _ptr(topk_idx), _ptr(counts), _ptr(kept),
+                                  _ptr(offsets), _ptr(row_of), _ptr(assign_of_row), _ptr(D),
+                                  _ptr(pk_off), _ptr(packed_row_of), _ptr(stats))
     R = int(offsets[E])
     return dict(counts=counts, kept=kept, offsets=offsets, row_of=row_of,
                 assign_of_row=assign_of_row[:R].copy(), D=D.reshape(W, W), pk_off=pk_off,
@@ -178,22 +183,22 @@ def affinity(topk_j: np.ndarray, topk_j1: np.ndarray, E: int,
 
 # --------------------------------------------------------------------------- compositions
 
-def route_and_dispatch(x, w_router, bias, K: int, W: int, cf: float) -> dict:
+def route_and_dispatch(x, w_router, bias, K: int, W: int, cf: float, order: int = 0) -> dict:
     """Steps a1-a3: logits, top-K + weights, capacity, positions, layout."""
     logits = router_logits(x, w_router, bias)
     N, E = logits.shape
     idx, w, bad = topk(logits, K)
     C = capacity(N, E, K, cf)
-    pos = positions(idx, E, W, C)
+    pos = positions(idx, E, W, C, order)
     pos.update(logits=logits, topk_idx=idx, topk_w=w, nonfinite=bad, C=C)
     return pos
 
 
-def layer(inp: dict, K: int, W: int, cf: float, want_h: bool = False) -> dict:
+def layer(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0) -> dict:
     """The whole layer on every token (small shapes only): returns the routing
     dict plus ``out`` [N][d] float64, ``y_rows`` [R][d] and optionally
     ``h_rows`` [R][f] (rows in expert-sorted order)."""
-    r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf)
+    r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order)
     N = r["logits"].shape[0]
     aor = r["assign_of_row"]
     row_token = (aor // K).astype(np.int32)

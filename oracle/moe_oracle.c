@@ -125,33 +125,38 @@ EXPORT int64_t orc_capacity(int64_t N, int64_t E, int64_t K, float cf)
  * §MoE 计算核优化 (cumsum, scatter, mapping table); P1 §All-to-All 分发与回收的
  * 机制 (pack by destination card)].
  *
- * Walk assignments a = t*K + k in increasing a. pos[a] = number of earlier
- * assignments to the same expert. Kept iff pos < C. counts[e] = all
- * assignments to e, kept[e] = min(counts[e], C). offsets = exclusive scan of
- * kept (E+1 entries). row_of[a] = offsets[e] + pos[a] if kept else -1, and
- * assign_of_row is its inverse over the R kept rows.
+ * Assignments are walked in priority order: token-major (order 0: a = t*K + k in
+ * increasing a) or slot-major (order 1: every token's slot 0, tokens ascending,
+ * then every token's slot 1, ...). pos[a] = number of earlier assignments (in that
+ * order) to the same expert. Kept iff pos < C. counts[e] = all assignments to e,
+ * kept[e] = min(counts[e], C). offsets = exclusive scan of kept (E+1 entries).
+ * row_of[a] = offsets[e] + pos[a] if kept else -1, and assign_of_row is its
+ * inverse over the R kept rows.
  *
  * Virtual ranks: expert e lives on rank e / (E/W); token t's home is
  * t / (N/W). D[i][j] counts kept assignments from home i to expert rank j.
- * The packed buffer holds blocks (i, j) in row-major order, each block's rows
- * ordered by (expert, token); pk_off is the exclusive scan of D (W*W+1
- * entries) and packed_row_of[a] the row of assignment a there (-1 if dropped).
+ * The packed buffer holds blocks (i, j) in row-major order; inside a block,
+ * expert by expert in increasing e, the rows of x_sorted of that expert whose
+ * token's home is i, in row order (for token-major priority that is token
+ * order). pk_off is the exclusive scan of D (W*W+1 entries) and
+ * packed_row_of[a] the row of assignment a there (-1 if dropped).
  *
  * stats[0] R (kept rows), [1] dropped, [2] kept rows with rank(e) != home(t),
  * [3] distinct (t, rank) pairs with rank != home(t) over kept assignments
  * (what a deduplicating exchange would send), [4] experts with kept > 0,
  * [5] max kept[e], [6] min kept[e], [7] C. */
-EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
-                          const int32_t *topk_idx, int32_t *counts, int32_t *kept,
-                          int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
-                          int64_t *D, int64_t *pk_off, int32_t *packed_row_of,
-                          int64_t *stats)
+EXPORT void orc_positions_ordered(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
+                                  int64_t order, const int32_t *topk_idx, int32_t *counts,
+                                  int32_t *kept, int32_t *offsets, int32_t *row_of,
+                                  int32_t *assign_of_row, int64_t *D, int64_t *pk_off,
+                                  int32_t *packed_row_of, int64_t *stats)
 {
     int64_t e_per = E / W, n_per = N / W;
     int64_t *seen = (int64_t *)calloc((size_t)E, sizeof(int64_t));
     int64_t *pos = (int64_t *)malloc((size_t)(N * K) * sizeof(int64_t));
 
-    for (int64_t a = 0; a < N * K; ++a) {
+    for (int64_t idx = 0; idx < N * K; ++idx) {
+        int64_t a = order == 0 ? idx : (idx % N) * K + idx / N;
         int64_t e = topk_idx[a];
         pos[a] = seen[e];
         seen[e] += 1;
@@ -185,20 +190,17 @@ EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
     for (int64_t b = 0; b < W * W; ++b)
         pk_off[b + 1] = pk_off[b] + D[b];
 
-    /* packed order: block (i, j), then expert e of rank j, then token t of
-     * shard i, then slot k (a token selects an expert at most once). */
     for (int64_t a = 0; a < N * K; ++a)
         packed_row_of[a] = -1;
     int64_t next = 0;
     for (int64_t i = 0; i < W; ++i)
         for (int64_t j = 0; j < W; ++j)
             for (int64_t e = j * e_per; e < (j + 1) * e_per; ++e)
-                for (int64_t t = i * n_per; t < (i + 1) * n_per; ++t)
-                    for (int64_t k = 0; k < K; ++k) {
-                        int64_t a = t * K + k;
-                        if (topk_idx[a] == e && row_of[a] >= 0)
-                            packed_row_of[a] = (int32_t)(next++);
-                    }
+                for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r) {
+                    int64_t a = assign_of_row[r];
+                    if ((a / K) / n_per == i)
+                        packed_row_of[a] = (int32_t)(next++);
+                }
 
     /* distinct destination ranks per token, excluding the home rank */
     int64_t dedup = 0;
@@ -236,6 +238,17 @@ EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
     free(rank_seen);
     free(pos);
     free(seen);
+}
+
+/* Token-major priority (the default reading). */
+EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
+                          const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                          int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                          int64_t *D, int64_t *pk_off, int32_t *packed_row_of,
+                          int64_t *stats)
+{
+    orc_positions_ordered(N, E, K, W, C, 0, topk_idx, counts, kept, offsets, row_of,
+                          assign_of_row, D, pk_off, packed_row_of, stats);
 }
 
 /* Expert FFN for a list of rows [P1 §All-to-All 分发与回收的机制, node F: each

@@ -75,10 +75,13 @@ def capacity(N: int, E: int, K: int, cf: float) -> int:
     return math.ceil(Fraction(cf) * N * K / E)
 
 
-def dispatch(idx: np.ndarray, E: int, W: int, C: int) -> dict:
+def dispatch(idx: np.ndarray, E: int, W: int, C: int, order: int = 0) -> dict:
+    """order 0: priority by (token, slot); 1: by (slot, token)."""
     N, K = idx.shape
     flat = idx.reshape(-1)
-    pos = [sum(1 for b in range(a) if flat[b] == flat[a]) for a in range(N * K)]
+    prio = (lambda a: a) if order == 0 else (lambda a: (a % K) * N + a // K)
+    pos = [sum(1 for b in range(N * K) if flat[b] == flat[a] and prio(b) < prio(a))
+           for a in range(N * K)]
     counts = [sum(1 for a in range(N * K) if flat[a] == e) for e in range(E)]
     kept = [min(c, C) for c in counts]
     offsets = [0]
@@ -92,7 +95,7 @@ def dispatch(idx: np.ndarray, E: int, W: int, C: int) -> dict:
         if row_of[a] >= 0:
             t, e = a // K, int(flat[a])
             D[t // n_per, e // e_per] += 1
-            keyed.append(((t // n_per, e // e_per, e, t), a))
+            keyed.append(((t // n_per, e // e_per, e, pos[a]), a))
     keyed.sort()
     packed_row_of = [-1] * (N * K)
     for p, (_, a) in enumerate(keyed):

@@ -359,3 +359,40 @@ def test_residual_moe_oracle(orc):
     zero["w2"] = torch.zeros_like(inp["w2"])
     r0 = orc.layer_shared(zero, sh, w.K, w.W, w.cf)
     np.testing.assert_array_equal(r0["out"], r0["shared_y"])
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_slot_major_priority_brute_force(orc, seed):
+    """Slot-major priority (every token's first choice before any second choice,
+    [MoE 推理服务工程真相 2026, §4.3: which assignments give way when an expert is full]):
+    positions, rows and the packed order against an O(N*K*E) recount."""
+    rng = np.random.default_rng(seed)
+    N, E, K, W = 12, 6, 3, 3
+    lg = rng.standard_normal((N, E)).astype(np.float32)
+    lg[:, 0] += 1.5  # a hot expert, so capacity binds
+    idx, _, _ = orc.topk(lg, K)
+    for C in (1, 3, 5, N * K):
+        p = orc.positions(idx, E, W, C, order=orc.SLOT_MAJOR)
+        b = brute.dispatch(idx, E, W, C, order=1)
+        for key in ("counts", "kept", "offsets", "row_of", "packed_row_of"):
+            np.testing.assert_array_equal(p[key], b[key], err_msg=(C, key))
+        np.testing.assert_array_equal(p["D"], b["D"])
+        assert p["stats"]["dedup_pairs"] == b["dedup"]
+        # the token-major and slot-major results agree when nothing is dropped
+        if C == N * K:
+            q = orc.positions(idx, E, W, C)
+            np.testing.assert_array_equal(q["kept"], p["kept"])
+
+
+def test_slot_major_keeps_first_choices(orc):
+    """Under slot-major priority, when capacity allows every first choice, no first
+    choice is dropped; token-major priority can drop a later token's first choice."""
+    idx = np.array([[0, 1], [0, 1], [1, 0]], np.int32)  # 3 tokens, K = 2, E = 2
+    C = 2
+    tm = orc.positions(idx, 2, 1, C)
+    sm = orc.positions(idx, 2, 1, C, order=orc.SLOT_MAJOR)
+    # token-major: expert 1 is filled by tokens 0 and 1 (their second choices), so token 2's
+    # first choice (expert 1) is dropped
+    assert tm["row_of"].reshape(3, 2)[2, 0] == -1
+    # slot-major: first choices (0, 0, 1) are placed before any second choice
+    assert np.all(sm["row_of"].reshape(3, 2)[:, 0] >= 0)
