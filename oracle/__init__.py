@@ -57,6 +57,8 @@ def _load():
         lib.orc_positions.restype = None
         lib.orc_positions_ordered.argtypes = [_i64] * 6 + [_p] * 10
         lib.orc_positions_ordered.restype = None
+        lib.orc_dispatch.argtypes = [_i64] * 7 + [_p] * 12
+        lib.orc_dispatch.restype = None
         lib.orc_expert_rows.argtypes = [_i64, _p, _p, _i64, _i64, _p, _p, _p, _p, _p, _p]
         lib.orc_expert_rows.restype = None
         lib.orc_combine.argtypes = [_i64, _i64, _i64, _p, _p, _p, _p]
@@ -120,28 +122,39 @@ def capacity(N: int, E: int, K: int, cf: float) -> int:
 SLOT_MAJOR = 1  # priority order of positions() / route_and_dispatch(): 0 token-major
 
 
-def positions(topk_idx: np.ndarray, E: int, W: int, C: int, order: int = 0) -> dict:
+def positions(topk_idx: np.ndarray, E: int, W: int, C: int, order: int = 0,
+              reroute: bool = False, logits: Optional[np.ndarray] = None) -> dict:
+    """Dispatch bookkeeping in priority ``order`` (0 token-major, SLOT_MAJOR), with
+    overflowed assignments re-routed to the next-best non-full expert when
+    ``reroute`` (then ``logits`` [N][E] fp32 rank the candidates)."""
     topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
     N, K = topk_idx.shape
+    if reroute:
+        logits = np.ascontiguousarray(logits, dtype=np.float32)
+        assert logits.shape == (N, E)
     counts = np.empty(E, np.int32)
     kept = np.empty(E, np.int32)
     offsets = np.empty(E + 1, np.int32)
     row_of = np.empty(N * K, np.int32)
     assign_of_row = np.full(N * K, -1, np.int32)
+    expert_of = np.empty(N * K, np.int32)
     D = np.empty(W * W, np.int64)
     pk_off = np.empty(W * W + 1, np.int64)
     packed_row_of = np.empty(N * K, np.int32)
-    stats = np.empty(8, np.int64)
-    _load().orc_positions_ordered(N, E, K, W, C, order, _ptr(topk_idx), _ptr(counts), _ptr(kept),
-                                  _ptr(offsets), _ptr(row_of), _ptr(assign_of_row), _ptr(D),
-                                  _ptr(pk_off), _ptr(packed_row_of), _ptr(stats))
+    stats = np.empty(9, np.int64)
+    _load().orc_dispatch(N, E, K, W, C, order, int(bool(reroute)),
+                         _ptr(logits) if reroute else None, _ptr(topk_idx), _ptr(counts),
+                         _ptr(kept), _ptr(offsets), _ptr(row_of), _ptr(assign_of_row),
+                         _ptr(expert_of), _ptr(D), _ptr(pk_off), _ptr(packed_row_of),
+                         _ptr(stats))
     R = int(offsets[E])
     return dict(counts=counts, kept=kept, offsets=offsets, row_of=row_of,
-                assign_of_row=assign_of_row[:R].copy(), D=D.reshape(W, W), pk_off=pk_off,
-                packed_row_of=packed_row_of, R=R,
+                assign_of_row=assign_of_row[:R].copy(), expert_of=expert_of, D=D.reshape(W, W),
+                pk_off=pk_off, packed_row_of=packed_row_of, R=R,
                 stats=dict(R=int(stats[0]), dropped=int(stats[1]), cross_rows=int(stats[2]),
                            dedup_pairs=int(stats[3]), active_experts=int(stats[4]),
-                           max_kept=int(stats[5]), min_kept=int(stats[6]), C=int(stats[7])))
+                           max_kept=int(stats[5]), min_kept=int(stats[6]), C=int(stats[7]),
+                           rerouted=int(stats[8])))
 
 
 def expert_rows(row_token: np.ndarray, row_expert: np.ndarray, x, w1, w3, w2,
@@ -183,26 +196,28 @@ def affinity(topk_j: np.ndarray, topk_j1: np.ndarray, E: int,
 
 # --------------------------------------------------------------------------- compositions
 
-def route_and_dispatch(x, w_router, bias, K: int, W: int, cf: float, order: int = 0) -> dict:
+def route_and_dispatch(x, w_router, bias, K: int, W: int, cf: float, order: int = 0,
+                       reroute: bool = False) -> dict:
     """Steps a1-a3: logits, top-K + weights, capacity, positions, layout."""
     logits = router_logits(x, w_router, bias)
     N, E = logits.shape
     idx, w, bad = topk(logits, K)
     C = capacity(N, E, K, cf)
-    pos = positions(idx, E, W, C, order)
+    pos = positions(idx, E, W, C, order, reroute, logits)
     pos.update(logits=logits, topk_idx=idx, topk_w=w, nonfinite=bad, C=C)
     return pos
 
 
-def layer(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0) -> dict:
+def layer(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0,
+          reroute: bool = False) -> dict:
     """The whole layer on every token (small shapes only): returns the routing
     dict plus ``out`` [N][d] float64, ``y_rows`` [R][d] and optionally
     ``h_rows`` [R][f] (rows in expert-sorted order)."""
-    r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order)
+    r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order, reroute)
     N = r["logits"].shape[0]
     aor = r["assign_of_row"]
     row_token = (aor // K).astype(np.int32)
-    row_expert = r["topk_idx"].reshape(-1)[aor].astype(np.int32)
+    row_expert = r["expert_of"][aor].astype(np.int32)
     h, y = expert_rows(row_token, row_expert, inp["x"], inp["w1"], inp["w3"], inp["w2"], want_h)
     d = y.shape[1]
     y_of_slot = np.zeros((N * K, d), np.float64)
@@ -225,7 +240,7 @@ def layer_sampled(inp: dict, K: int, W: int, cf: float, tokens: Sequence[int],
     slots = (tokens[:, None] * K + np.arange(K)[None, :]).reshape(-1)
     kept_slots = slots[r["row_of"][slots] >= 0]
     row_token = (kept_slots // K).astype(np.int32)
-    row_expert = r["topk_idx"].reshape(-1)[kept_slots].astype(np.int32)
+    row_expert = r["expert_of"][kept_slots].astype(np.int32)
     h, y = expert_rows(row_token, row_expert, inp["x"], inp["w1"], inp["w3"], inp["w2"], want_h)
     d = y.shape[1]
     n = tokens.shape[0]

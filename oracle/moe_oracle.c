@@ -121,76 +121,155 @@ EXPORT int64_t orc_capacity(int64_t N, int64_t E, int64_t K, float cf)
     return (int64_t)ceil((double)cf * (double)N * (double)K / (double)E);
 }
 
-/* Dispatch bookkeeping [P2 §2.3 pseudo-code (bincount, overflow mask); P3
- * §MoE 计算核优化 (cumsum, scatter, mapping table); P1 §All-to-All 分发与回收的
- * 机制 (pack by destination card)].
- *
- * Assignments are walked in priority order: token-major (order 0: a = t*K + k in
- * increasing a) or slot-major (order 1: every token's slot 0, tokens ascending,
- * then every token's slot 1, ...). pos[a] = number of earlier assignments (in that
- * order) to the same expert. Kept iff pos < C. counts[e] = all assignments to e,
- * kept[e] = min(counts[e], C). offsets = exclusive scan of kept (E+1 entries).
- * row_of[a] = offsets[e] + pos[a] if kept else -1, and assign_of_row is its
- * inverse over the R kept rows.
- *
- * Virtual ranks: expert e lives on rank e / (E/W); token t's home is
- * t / (N/W). D[i][j] counts kept assignments from home i to expert rank j.
- * The packed buffer holds blocks (i, j) in row-major order; inside a block,
- * expert by expert in increasing e, the rows of x_sorted of that expert whose
- * token's home is i, in row order (for token-major priority that is token
- * order). pk_off is the exclusive scan of D (W*W+1 entries) and
- * packed_row_of[a] the row of assignment a there (-1 if dropped).
- *
- * stats[0] R (kept rows), [1] dropped, [2] kept rows with rank(e) != home(t),
- * [3] distinct (t, rank) pairs with rank != home(t) over kept assignments
- * (what a deduplicating exchange would send), [4] experts with kept > 0,
- * [5] max kept[e], [6] min kept[e], [7] C. */
-EXPORT void orc_positions_ordered(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
-                                  int64_t order, const int32_t *topk_idx, int32_t *counts,
-                                  int32_t *kept, int32_t *offsets, int32_t *row_of,
-                                  int32_t *assign_of_row, int64_t *D, int64_t *pk_off,
-                                  int32_t *packed_row_of, int64_t *stats)
+/* Position of each assignment in its expert's sequence, walking the N*K assignments in
+ * priority order: token-major (order 0: a = t*K + k in increasing a) or slot-major
+ * (order 1: every token's slot 0, tokens ascending, then every token's slot 1, ...).
+ * Only assignments with expert[a] >= 0 take part; start[e] is where expert e's count
+ * begins (0 for a first pass). */
+static void walk_positions(int64_t N, int64_t E, int64_t K, int64_t order,
+                           const int64_t *expert, const int64_t *start, int64_t *pos,
+                           int64_t *total)
 {
-    int64_t e_per = E / W, n_per = N / W;
-    int64_t *seen = (int64_t *)calloc((size_t)E, sizeof(int64_t));
-    int64_t *pos = (int64_t *)malloc((size_t)(N * K) * sizeof(int64_t));
-
+    for (int64_t e = 0; e < E; ++e)
+        total[e] = start ? start[e] : 0;
     for (int64_t idx = 0; idx < N * K; ++idx) {
         int64_t a = order == 0 ? idx : (idx % N) * K + idx / N;
-        int64_t e = topk_idx[a];
-        pos[a] = seen[e];
-        seen[e] += 1;
+        int64_t e = expert[a];
+        if (e < 0)
+            continue;
+        pos[a] = total[e];
+        total[e] += 1;
     }
-    offsets[0] = 0;
+}
+
+/* Dispatch bookkeeping [P2 §2.3 pseudo-code (bincount, overflow mask, remapping of
+ * overflowed assignments); §2.2 (capacity, expert drop); §4.3 (token drop: re-route
+ * to the next-best expert); P3 §MoE 计算核优化 (cumsum, scatter, mapping table);
+ * P1 §All-to-All 分发与回收的机制 (pack by destination card)].
+ *
+ * First pass: pos0[a] = number of earlier assignments (in priority order) to the
+ * same expert; the assignment is kept iff pos0 < C. demand counts[e] = all
+ * assignments routed to e.
+ *
+ * With reroute: an expert is full when counts[e] >= C. Each assignment that
+ * overflowed (pos0 >= C) moves to its token's best-ranked expert (larger logit
+ * first, ties to the lower index) that is neither one of the token's K routed
+ * experts, nor full, nor already taken by an earlier overflowed slot (in k order)
+ * of the same token; none such: it stays dropped. The moved assignments then take
+ * positions at their new expert after all of its first-pass assignments, in the
+ * same priority order, and are kept iff that position < C. They keep their gate
+ * weight. One round: a moved assignment that does not fit is dropped.
+ *
+ * Results: expert_of[a] = the expert whose row a uses, -1 if dropped.
+ * kept[e] = rows of expert e; offsets = exclusive scan of kept (E+1 entries);
+ * row_of[a] = offsets[expert_of[a]] + position, or -1; assign_of_row its inverse.
+ *
+ * Virtual ranks: expert e lives on rank e / (E/W); token t's home is t / (N/W).
+ * D[i][j] counts rows from home i at experts on rank j. The packed buffer holds
+ * blocks (i, j) in row-major order; inside a block, expert by expert in
+ * increasing e, the rows of that expert whose token's home is i, in row order.
+ * pk_off is the exclusive scan of D (W*W+1 entries) and packed_row_of[a] the row
+ * of assignment a there (-1 if dropped).
+ *
+ * stats[0] R (rows), [1] dropped = N*K - R, [2] rows with rank(e) != home(t),
+ * [3] distinct (t, rank) pairs with rank != home(t) over the rows (what a
+ * deduplicating exchange would send), [4] experts with rows, [5] max kept[e],
+ * [6] min kept[e], [7] C, [8] rows at a re-routed expert. */
+EXPORT void orc_dispatch(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C, int64_t order,
+                         int64_t reroute, const float *logits, const int32_t *topk_idx,
+                         int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of,
+                         int32_t *assign_of_row, int32_t *expert_of, int64_t *D,
+                         int64_t *pk_off, int32_t *packed_row_of, int64_t *stats)
+{
+    int64_t e_per = E / W, n_per = N / W;
+    int64_t NK = N * K;
+    int64_t *route = (int64_t *)malloc((size_t)NK * sizeof(int64_t));
+    int64_t *pos = (int64_t *)malloc((size_t)NK * sizeof(int64_t));
+    int64_t *moved = (int64_t *)malloc((size_t)NK * sizeof(int64_t));
+    int64_t *pos1 = (int64_t *)malloc((size_t)NK * sizeof(int64_t));
+    int64_t *demand = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    int64_t *total = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    char *taken = (char *)malloc((size_t)E);
+
+    for (int64_t a = 0; a < NK; ++a) {
+        route[a] = topk_idx[a];
+        moved[a] = -1;
+    }
+    walk_positions(N, E, K, order, route, NULL, pos, demand);
+
+    int64_t n_moved = 0;
+    if (reroute) {
+        for (int64_t t = 0; t < N; ++t) {
+            memset(taken, 0, (size_t)E);
+            for (int64_t k = 0; k < K; ++k)
+                taken[topk_idx[t * K + k]] = 1;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t a = t * K + k;
+                if (pos[a] < C)
+                    continue;
+                const float *l = logits + t * E;
+                int64_t best = -1;
+                for (int64_t e = 0; e < E; ++e) {
+                    if (taken[e] || demand[e] >= C)
+                        continue;
+                    if (best < 0 || l[e] > l[best])
+                        best = e;
+                }
+                if (best >= 0) {
+                    taken[best] = 1;
+                    moved[a] = best;
+                }
+            }
+        }
+        /* second pass starts after each expert's first-pass assignments */
+        walk_positions(N, E, K, order, moved, demand, pos1, total);
+    }
+
+    for (int64_t a = 0; a < NK; ++a) {
+        if (pos[a] < C) {
+            expert_of[a] = (int32_t)route[a];
+        } else if (moved[a] >= 0 && pos1[a] < C) {
+            expert_of[a] = (int32_t)moved[a];
+            pos[a] = pos1[a];
+            n_moved += 1;
+        } else {
+            expert_of[a] = -1;
+        }
+    }
+
     for (int64_t e = 0; e < E; ++e) {
-        counts[e] = (int32_t)seen[e];
-        kept[e] = (int32_t)(seen[e] < C ? seen[e] : C);
-        offsets[e + 1] = offsets[e] + kept[e];
+        counts[e] = (int32_t)demand[e];
+        kept[e] = 0;
     }
+    for (int64_t a = 0; a < NK; ++a)
+        if (expert_of[a] >= 0)
+            kept[expert_of[a]] += 1;
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + kept[e];
     for (int64_t i = 0; i < W * W; ++i)
         D[i] = 0;
     int64_t R = 0, cross = 0;
-    for (int64_t a = 0; a < N * K; ++a) {
-        int64_t e = topk_idx[a];
-        int64_t t = a / K;
-        if (pos[a] < C) {
-            int64_t r = offsets[e] + pos[a];
-            row_of[a] = (int32_t)r;
-            assign_of_row[r] = (int32_t)a;
-            int64_t i = t / n_per, j = e / e_per;
-            D[i * W + j] += 1;
-            if (i != j)
-                cross += 1;
-            R += 1;
-        } else {
+    for (int64_t a = 0; a < NK; ++a) {
+        int64_t e = expert_of[a];
+        if (e < 0) {
             row_of[a] = -1;
+            continue;
         }
+        int64_t r = offsets[e] + pos[a];
+        row_of[a] = (int32_t)r;
+        assign_of_row[r] = (int32_t)a;
+        int64_t i = (a / K) / n_per, j = e / e_per;
+        D[i * W + j] += 1;
+        if (i != j)
+            cross += 1;
+        R += 1;
     }
     pk_off[0] = 0;
     for (int64_t b = 0; b < W * W; ++b)
         pk_off[b + 1] = pk_off[b] + D[b];
 
-    for (int64_t a = 0; a < N * K; ++a)
+    for (int64_t a = 0; a < NK; ++a)
         packed_row_of[a] = -1;
     int64_t next = 0;
     for (int64_t i = 0; i < W; ++i)
@@ -208,10 +287,10 @@ EXPORT void orc_positions_ordered(int64_t N, int64_t E, int64_t K, int64_t W, in
     for (int64_t t = 0; t < N; ++t) {
         memset(rank_seen, 0, (size_t)W);
         for (int64_t k = 0; k < K; ++k) {
-            int64_t a = t * K + k;
-            if (row_of[a] < 0)
+            int64_t e = expert_of[t * K + k];
+            if (e < 0)
                 continue;
-            int64_t j = topk_idx[a] / e_per;
+            int64_t j = e / e_per;
             if (j != t / n_per && !rank_seen[j]) {
                 rank_seen[j] = 1;
                 dedup += 1;
@@ -228,19 +307,41 @@ EXPORT void orc_positions_ordered(int64_t N, int64_t E, int64_t K, int64_t W, in
             mn = kept[e];
     }
     stats[0] = R;
-    stats[1] = N * K - R;
+    stats[1] = NK - R;
     stats[2] = cross;
     stats[3] = dedup;
     stats[4] = active;
     stats[5] = mx;
     stats[6] = mn;
     stats[7] = C;
+    stats[8] = n_moved;
     free(rank_seen);
+    free(taken);
+    free(total);
+    free(demand);
+    free(pos1);
+    free(moved);
     free(pos);
-    free(seen);
+    free(route);
 }
 
-/* Token-major priority (the default reading). */
+/* Without re-routing: the priority order alone decides. */
+EXPORT void orc_positions_ordered(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
+                                  int64_t order, const int32_t *topk_idx, int32_t *counts,
+                                  int32_t *kept, int32_t *offsets, int32_t *row_of,
+                                  int32_t *assign_of_row, int64_t *D, int64_t *pk_off,
+                                  int32_t *packed_row_of, int64_t *stats)
+{
+    int32_t *expert_of = (int32_t *)malloc((size_t)(N * K) * sizeof(int32_t));
+    int64_t st[9];
+    orc_dispatch(N, E, K, W, C, order, 0, NULL, topk_idx, counts, kept, offsets, row_of,
+                 assign_of_row, expert_of, D, pk_off, packed_row_of, st);
+    for (int i = 0; i < 8; ++i)
+        stats[i] = st[i];
+    free(expert_of);
+}
+
+/* Token-major priority without re-routing (the default reading). */
 EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
                           const int32_t *topk_idx, int32_t *counts, int32_t *kept,
                           int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,

@@ -75,25 +75,44 @@ def capacity(N: int, E: int, K: int, cf: float) -> int:
     return math.ceil(Fraction(cf) * N * K / E)
 
 
-def dispatch(idx: np.ndarray, E: int, W: int, C: int, order: int = 0) -> dict:
-    """order 0: priority by (token, slot); 1: by (slot, token)."""
+def dispatch(idx: np.ndarray, E: int, W: int, C: int, order: int = 0, reroute: bool = False,
+             logits=None) -> dict:
+    """order 0: priority by (token, slot); 1: by (slot, token). With ``reroute``, an
+    overflowed assignment moves to the token's best remaining expert (by logit, then
+    index) outside its top-K whose demand is below C, and queues behind that expert's
+    first-pass assignments."""
     N, K = idx.shape
     flat = idx.reshape(-1)
     prio = (lambda a: a) if order == 0 else (lambda a: (a % K) * N + a // K)
     pos = [sum(1 for b in range(N * K) if flat[b] == flat[a] and prio(b) < prio(a))
            for a in range(N * K)]
     counts = [sum(1 for a in range(N * K) if flat[a] == e) for e in range(E)]
-    kept = [min(c, C) for c in counts]
+    expert_of = [int(flat[a]) if pos[a] < C else -1 for a in range(N * K)]
+    if reroute:
+        moved = {}
+        for t in range(N):
+            mine = {int(e) for e in idx[t]}
+            cands = [e for e in sorted(range(E), key=lambda e: (-float(logits[t, e]), e))
+                     if e not in mine and counts[e] < C]
+            over = [t * K + k for k in range(K) if pos[t * K + k] >= C]
+            for a, e in zip(over, cands):
+                moved[a] = e
+        for a, e in moved.items():
+            p1 = counts[e] + sum(1 for b, e2 in moved.items() if e2 == e and prio(b) < prio(a))
+            if p1 < C:
+                expert_of[a] = e
+                pos[a] = p1
+    kept = [sum(1 for a in range(N * K) if expert_of[a] == e) for e in range(E)]
     offsets = [0]
     for e in range(E):
         offsets.append(offsets[-1] + kept[e])
-    row_of = [offsets[flat[a]] + pos[a] if pos[a] < C else -1 for a in range(N * K)]
+    row_of = [offsets[expert_of[a]] + pos[a] if expert_of[a] >= 0 else -1 for a in range(N * K)]
     e_per, n_per = E // W, N // W
     D = np.zeros((W, W), np.int64)
     keyed = []
     for a in range(N * K):
         if row_of[a] >= 0:
-            t, e = a // K, int(flat[a])
+            t, e = a // K, expert_of[a]
             D[t // n_per, e // e_per] += 1
             keyed.append(((t // n_per, e // e_per, e, pos[a]), a))
     keyed.sort()
@@ -102,11 +121,13 @@ def dispatch(idx: np.ndarray, E: int, W: int, C: int, order: int = 0) -> dict:
         packed_row_of[a] = p
     dedup = 0
     for t in range(N):
-        dests = {int(flat[t * K + k]) // e_per for k in range(K) if row_of[t * K + k] >= 0}
+        dests = {expert_of[t * K + k] // e_per for k in range(K) if expert_of[t * K + k] >= 0}
         dests.discard(t // n_per)
         dedup += len(dests)
+    rerouted = sum(1 for a in range(N * K) if expert_of[a] >= 0 and expert_of[a] != flat[a])
     return dict(counts=np.array(counts), kept=np.array(kept), offsets=np.array(offsets),
-                row_of=np.array(row_of), D=D, packed_row_of=np.array(packed_row_of), dedup=dedup)
+                row_of=np.array(row_of), D=D, packed_row_of=np.array(packed_row_of), dedup=dedup,
+                expert_of=np.array(expert_of), rerouted=rerouted)
 
 
 def swiglu_rows(x_u16, w1_u16, w3_u16, w2_u16, row_token, row_expert):

@@ -36,7 +36,8 @@ def test_hand_routing_fixture(orc):
     for key in ("counts", "kept", "offsets", "row_of", "assign_of_row", "pk_off", "packed_row_of"):
         np.testing.assert_array_equal(p[key], g[key], err_msg=key)
     np.testing.assert_array_equal(p["D"], g["D"])
-    assert p["stats"] == g["stats"]
+    assert {k: p["stats"][k] for k in g["stats"]} == g["stats"]
+    assert p["stats"]["rerouted"] == 0  # no re-routing unless asked
     rep = orc.derive_report(g["N"], g["E"], g["K"], g["W"], p["kept"], p["D"], p["stats"], d=1)
     for key, v in g["report"].items():
         assert rep[key] == pytest.approx(v, rel=1e-12), key
@@ -396,3 +397,59 @@ def test_slot_major_keeps_first_choices(orc):
     assert tm["row_of"].reshape(3, 2)[2, 0] == -1
     # slot-major: first choices (0, 0, 1) are placed before any second choice
     assert np.all(sm["row_of"].reshape(3, 2)[:, 0] >= 0)
+
+
+def test_drop_policies_hand_worked_example(orc):
+    """The four drop policies on a 4-token example worked by hand
+    (tests/golden/reroute_example.json)."""
+    with open(os.path.join(GOLDEN, "reroute_example.json"), encoding="utf-8") as fh:
+        g = json.load(fh)
+    lg = np.array(g["logits"], np.float32)
+    idx, _, _ = orc.topk(lg, g["K"])
+    np.testing.assert_array_equal(idx, g["topk_idx"])
+    for name, c in g["cases"].items():
+        p = orc.positions(idx, g["E"], g["W"], g["C"], order=c["order"], reroute=c["reroute"],
+                          logits=lg)
+        np.testing.assert_array_equal(p["expert_of"], c["expert_of"], err_msg=name)
+        np.testing.assert_array_equal(p["row_of"], c["row_of"], err_msg=name)
+        np.testing.assert_array_equal(p["kept"], c["kept"], err_msg=name)
+        assert p["stats"]["dropped"] == c["dropped"] and p["stats"]["rerouted"] == c["rerouted"]
+        if "D" in c:
+            np.testing.assert_array_equal(p["D"], c["D"], err_msg=name)
+            np.testing.assert_array_equal(p["packed_row_of"], c["packed_row_of"], err_msg=name)
+            assert p["stats"]["cross_rows"] == c["cross_rows"]
+            assert p["stats"]["dedup_pairs"] == c["dedup_pairs"]
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_reroute_brute_force(orc, seed):
+    """Re-routing of overflowed assignments to the next-best non-full expert, both
+    priority orders, against an independent O((N*K)^2) restatement."""
+    rng = np.random.default_rng(100 + seed)
+    W = int(rng.choice([1, 2, 3]))
+    E = W * int(rng.integers(2, 5))
+    K = int(rng.integers(1, min(E, 4) + 1))
+    N = W * int(rng.integers(2, 9))
+    lg = rng.standard_normal((N, E)).astype(np.float32)
+    lg[:, : max(1, E // 3)] += 1.2  # a few hot experts
+    if seed % 3 == 0:
+        lg = np.round(lg * 2) / 2  # ties between candidates
+    idx, _, _ = orc.topk(lg, K)
+    for C in (1, 2, max(1, N * K // E)):
+        for order in (0, 1):
+            p = orc.positions(idx, E, W, C, order=order, reroute=True, logits=lg)
+            b = brute.dispatch(idx, E, W, C, order=order, reroute=True, logits=lg)
+            for key in ("counts", "kept", "offsets", "row_of", "packed_row_of", "expert_of"):
+                np.testing.assert_array_equal(p[key], b[key], err_msg=(C, order, key))
+            np.testing.assert_array_equal(p["D"], b["D"])
+            assert p["stats"]["dedup_pairs"] == b["dedup"]
+            assert p["stats"]["rerouted"] == b["rerouted"]
+            # invariants: no expert above capacity, no token twice at one expert,
+            # re-routing never drops more than the plain policy
+            assert p["kept"].max(initial=0) <= C
+            eo = p["expert_of"].reshape(N, K)
+            for t in range(N):
+                got = eo[t][eo[t] >= 0]
+                assert len(set(got.tolist())) == len(got)
+            plain = orc.positions(idx, E, W, C, order=order)
+            assert p["stats"]["dropped"] == plain["stats"]["dropped"] - p["stats"]["rerouted"]
