@@ -162,9 +162,9 @@ class ClockSampler:
 # profiles/grouped_gemm_up_mixtral_prefill_half_full.md (half-size case, scaled x2 to the
 # full layer). Valid only for the kernel source it was measured on.
 MEASURED_UP_TRAFFIC = {
-    "kernel_sha256": "22c554d22716c0ea182bc63623776b24295dea3d04bfdfc1d0550202fb7781a5",
+    "kernel_sha256": "54dfe99065095ff871fae763340a72a193664460a2c77a1c3ae16b43d8216790",
     "workload": "mixtral_prefill",
-    "bytes": 2287.6e6,
+    "bytes": 2206.8e6,
 }
 
 
@@ -212,13 +212,16 @@ def run_gpu(args, w) -> dict:
     layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
               for l in range(L)]
     inp = layers[0]
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=L > 1)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=L > 1,
+                         slot_major=w.slot_major, reroute=w.reroute)
     RA = m.moe_rows_alloc(shape)
     ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
     x = inp["x"]
     N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
     topk_idx = [torch.empty(N, K, dtype=torch.int32, device=dev) for _ in range(L)]
     topk_w = torch.empty(N, K, dtype=torch.float32, device=dev)
+    # the logits rank the candidates of re-routed assignments
+    logits = torch.empty(N, E, dtype=torch.float32, device=dev) if w.reroute else None
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     kept = torch.empty(E, dtype=torch.int32, device=dev)
     offsets = [torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
@@ -247,7 +250,8 @@ def run_gpu(args, w) -> dict:
     n_ev = len(stage_names) + 1
     # per layer: logits, top-K, histogram, scan, positions, scatter, up, down, combine
     # (+ offsets, shared up, shared down for the Residual-MoE layer); + affinity per layer pair
-    launches_per_step = L * (9 + (3 if shared else 0)) + (L - 1)
+    # (+ histogram, scan, positions of the first pass and the ranking kernel when re-routing)
+    launches_per_step = L * (9 + (3 if shared else 0) + (4 if w.reroute else 0)) + (L - 1)
 
     def step(ev=None):
         """One step; ev (optional) is [layer][n_ev] events around the stages."""
@@ -259,11 +263,17 @@ def run_gpu(args, w) -> dict:
             e = ev[l] if ev is not None else None
             if e is not None:
                 e[0].record(st)
-            m.moe_route(shape, xin, lw["w_router"], lw["bias"], topk_idx[l], topk_w, None, ws, st)
+            m.moe_route(shape, xin, lw["w_router"], lw["bias"], topk_idx[l], topk_w, logits, ws,
+                        st)
             if e is not None:
                 e[1].record(st)
-            m.moe_dispatch(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of, assign,
-                           x_sorted, x_packed, D, pk_off, None, ws, st)
+            if w.reroute:
+                m.moe_dispatch_reroute(shape, xin, logits, topk_idx[l], counts, kept, offsets[l],
+                                       row_of, assign, x_sorted, x_packed=x_packed, rank_matrix=D,
+                                       packed_offsets=pk_off, ws=ws, stream=st)
+            else:
+                m.moe_dispatch(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of, assign,
+                               x_sorted, x_packed, D, pk_off, None, ws, st)
             if e is not None:
                 e[2].record(st)
             m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
@@ -503,7 +513,7 @@ def oracle_time(w, inp_cpu, sample_tokens: int, shared_cpu=None) -> dict:
     oracle.build()
     t0 = time.perf_counter()
     r = oracle.route_and_dispatch(inp_cpu["x"], inp_cpu["w_router"], inp_cpu.get("bias"), w.K,
-                                  w.W, w.cf)
+                                  w.W, w.cf, order=int(w.slot_major), reroute=w.reroute)
     t_route = time.perf_counter() - t0
     rng = np.random.default_rng(0)
     toks = np.sort(rng.choice(w.N, size=min(sample_tokens, w.N), replace=False))

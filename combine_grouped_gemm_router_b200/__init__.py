@@ -37,7 +37,8 @@ class MoeShape(ctypes.Structure):
 class MoeStats(ctypes.Structure):
     _fields_ = [("rows", c_i64), ("dropped", c_i64), ("cross_rows", c_i64),
                 ("dedup_pairs", c_i64), ("nonfinite_tokens", c_i64), ("capacity", c_i32),
-                ("active_experts", c_i32), ("max_kept", c_i32), ("min_kept", c_i32)]
+                ("active_experts", c_i32), ("max_kept", c_i32), ("min_kept", c_i32),
+                ("rerouted", c_i64)]
 
 
 class MoeReport(ctypes.Structure):
@@ -60,6 +61,7 @@ _sigs = {
     "moe_route": ([_SP] + [c_p] * 7 + [c_size, c_p], c_i32),
     "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
     "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
+    "moe_dispatch_reroute": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
     "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
     "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
@@ -74,6 +76,9 @@ _sigs = {
     "moe_get_device_error": ([ctypes.c_int], c_i32),
     "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
 }
+
+
+ABI_VERSION = 2  # MOE_ABI_VERSION the structures below match
 
 
 class _Lib:
@@ -93,6 +98,9 @@ class _Lib:
             fn = getattr(cdll, name)
             fn.argtypes = args
             fn.restype = res
+        if cdll.moe_abi_version() != ABI_VERSION:
+            raise ImportError(f"{LIB_PATH} has ABI version {cdll.moe_abi_version()}, this binding "
+                              f"expects {ABI_VERSION}: rebuild it")
         self._cdll = cdll
 
     def __getattr__(self, name):
@@ -133,12 +141,16 @@ def _stream(stream) -> Optional[int]:
 
 
 MOE_FLAG_OUT_BF16 = 1
+MOE_FLAG_SLOT_MAJOR = 2
+MOE_FLAG_REROUTE = 4
 
 
 def make_shape(N: int, d: int, f: int, E: int, K: int, W: int, capacity_factor: float = 0.0,
-               out_bf16: bool = False) -> MoeShape:
-    return MoeShape(N, d, f, E, K, W, float(capacity_factor),
-                    MOE_FLAG_OUT_BF16 if out_bf16 else 0)
+               out_bf16: bool = False, slot_major: bool = False,
+               reroute: bool = False) -> MoeShape:
+    flags = ((MOE_FLAG_OUT_BF16 if out_bf16 else 0) | (MOE_FLAG_SLOT_MAJOR if slot_major else 0)
+             | (MOE_FLAG_REROUTE if reroute else 0))
+    return MoeShape(N, d, f, E, K, W, float(capacity_factor), flags)
 
 
 # ---------------------------------------------------------------- sizes
@@ -185,6 +197,20 @@ def moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_ro
                              _ptr(x_sorted), _ptr(x_packed), _ptr(rank_matrix),
                              _ptr(packed_offsets), _ptr(stats), _ptr(ws), ws_bytes,
                              _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_reroute(shape, x, logits, topk_idx, counts, kept, offsets, row_of,
+                         assign_of_row, x_sorted, expert_of=None, x_packed=None,
+                         rank_matrix=None, packed_offsets=None, stats=None, ws=None, stream=None):
+    """moe_dispatch with overflowed assignments moved to the next-best non-full expert
+    (shape made with reroute=True; logits as written by moe_route)."""
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_dispatch_reroute(ctypes.byref(shape), _ptr(x), _ptr(logits), _ptr(topk_idx),
+                                     _ptr(counts), _ptr(kept), _ptr(offsets), _ptr(row_of),
+                                     _ptr(assign_of_row), _ptr(expert_of), _ptr(x_sorted),
+                                     _ptr(x_packed), _ptr(rank_matrix), _ptr(packed_offsets),
+                                     _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_dispatch_reroute")
 
 
 MOE_STATIC_SCRATCH_BYTES = 1 << 20

@@ -9,10 +9,25 @@
 // instead of a one-hot einsum. [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All
 // 分发与回收的机制] rows are packed by destination card before the exchange.
 //
-// Positions are taken in token-major (t, k) order without global atomics: a
-// block's base per expert comes from the scan over blocks, ranks inside a block
-// from per-warp counts and __match_any_sync, so the result is deterministic and
-// equal to the sequential definition.
+// Positions follow a priority order over the N*K assignments: token-major
+// ((t, k), a = t*K + k ascending) or slot-major ((k, t): every token's first
+// choice before any second choice). The dispatch walks that order as "virtual
+// blocks": token-major block b covers the K slots of HB tokens; slot-major block
+// (k, b) covers slot k of the same HB tokens. Blocks never straddle a home shard,
+// so the order is cut into segments (one per home shard, or one per (slot,
+// shard)) whose starts are block boundaries. A block's base per expert comes
+// from the scan over blocks, ranks inside a block from per-warp counts and
+// __match_any_sync, so the result is deterministic and equal to the sequential
+// definition, with no global atomics.
+//
+// Re-routing of overflowed assignments ([MoE 推理服务工程真相 2026, §4.3] token
+// drop: move to the next-best expert; [§2.3] the remapping of the overflow mask)
+// runs the dispatch twice. The first pass walks round 0 (the routed experts) and
+// finds the assignments past capacity; reroute_kernel picks each one's next-best
+// expert that is outside the token's top-K and not full; the second pass walks
+// round 0 followed by round 1 (the moved assignments at their new experts) as one
+// priority sequence, so a moved assignment queues behind every first-round
+// assignment of its new expert.
 #pragma once
 
 #include "common.cuh"
@@ -21,27 +36,61 @@ namespace moe {
 
 constexpr int kDispatchHB = 64;  // tokens per dispatch block
 
-// blk[e][b] = number of assignments in block b routed to expert e.
+// The dispatch's priority order, cut into virtual blocks: rounds of nvb_round
+// blocks each (round 1 only when re-routing), each round in priority order.
+struct VBlocks {
+    BlockMap bm;
+    int nblk_tok;           // token blocks (W * bps)
+    int slot_major;         // 0: token-major (nblk_tok blocks a round); 1: slot-major (K * nblk_tok)
+    int K;
+    int nvb_round;          // virtual blocks per round
+    const int32_t *moved;   // round 1's expert per assignment (-1: not moved), or null
+    // tokens [t0, t1), slot k (slot-major), round of virtual block vb
+    __device__ __forceinline__ void range(int vb, int &t0, int &t1, int &k, int &round) const
+    {
+        round = vb / nvb_round;
+        vb -= round * nvb_round;
+        k = slot_major ? vb / nblk_tok : 0;
+        bm.range(slot_major ? vb - k * nblk_tok : vb, t0, t1);
+    }
+    __device__ __forceinline__ int count(int t0, int t1) const
+    {
+        return slot_major ? t1 - t0 : (t1 - t0) * K;
+    }
+    // the i-th assignment of the block
+    __device__ __forceinline__ int assign(int t0, int k, int i) const
+    {
+        return slot_major ? (t0 + i) * K + k : t0 * K + i;
+    }
+    __device__ __forceinline__ const int32_t *experts(const int32_t *topk_idx, int round) const
+    {
+        return round ? moved : topk_idx;
+    }
+};
+
+// blk[e][vb] = number of assignments in virtual block vb routed to expert e.
 __global__ void __launch_bounds__(256)
-    block_hist_kernel(const int32_t *__restrict__ topk_idx, int K, int E, BlockMap bm, int nblk,
+    block_hist_kernel(const int32_t *__restrict__ topk_idx, int E, VBlocks vbm, int nvb,
                       int32_t *__restrict__ blk)
 {
     extern __shared__ int s_hist[];
     for (int e = threadIdx.x; e < E; e += blockDim.x)
         s_hist[e] = 0;
     __syncthreads();
-    int t0, t1;
-    bm.range(blockIdx.x, t0, t1);
-    for (int a = t0 * K + threadIdx.x; a < t1 * K; a += blockDim.x) {
-        const int e = topk_idx[a];
+    int t0, t1, k, round;
+    vbm.range(blockIdx.x, t0, t1, k, round);
+    const int32_t *src = vbm.experts(topk_idx, round);
+    const int n = vbm.count(t0, t1);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int e = src[vbm.assign(t0, k, i)];
         if ((unsigned)e < (unsigned)E)
             atomicAdd(&s_hist[e], 1);
-        else
-            set_dev_error(MOE_ERR_DEVICE_BOUNDS);
+        else if (round == 0)
+            set_dev_error(MOE_ERR_DEVICE_BOUNDS);  // round 1 marks "not moved" with -1
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x)
-        blk[(size_t)e * nblk + blockIdx.x] = s_hist[e];
+        blk[(size_t)e * nvb + blockIdx.x] = s_hist[e];
 }
 
 // In-place exclusive scan of a[0..n) in shared memory by the whole block;
@@ -80,44 +129,53 @@ __device__ void block_excl_scan_i64(int64_t *a, int n, int64_t *s_warp)
 }
 
 struct ScanArgs {
-    int32_t *blk;  // [E][nblk] counts in, exclusive bases out
-    int nblk;
-    BlockMap bm;
+    int32_t *blk;  // [E][nvb] counts in, exclusive bases out
+    int nvb;
+    int bps;       // virtual blocks per segment
+    int nseg;      // segments in priority order: W (token-major) or K*W (slot-major) a round
+    int nseg_round;
     int N, E, K, W;
     int C;
+    int32_t *cum_global;  // [E][nseg+1] when it does not fit in shared memory, else null
     int32_t *counts, *kept, *offsets;
     int64_t *D;        // [W][W]
     int64_t *pk_off;   // [W*W+1]
-    int64_t *pk_base;  // [E][W]
+    int64_t *pk_base;  // [E][nseg]
     moe_stats_t *stats;
 };
 
 // One CTA of 1024 threads.
-// Shared: s_cum [E][W+1] int32 (assignments of e before shard i; [W] = total),
-//         s_a   [max(E, W*W) + 1] int64 scan buffer, s_D [W*W] int64, s_warp[32].
+// Shared: s_a [max(E, W*W) + 1] int64 scan buffer, s_D [W*W] int64, s_warp [32],
+//         s_kh [E][W] int32 (kept rows of expert e from home shard i), then
+//         cum [E][nseg+1] int32 unless it lives in global memory: cum[e][g] =
+//         assignments to e before segment g in priority order, cum[e][nseg] = total.
+// Segment g belongs to home shard g % W; within one home shard its segments
+// come in priority order, so the kept rows of expert e from that shard are a
+// prefix of the shard's own sequence of assignments to e.
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
 {
     constexpr int NT = 1024;
     extern __shared__ __align__(16) unsigned char scan_smem[];
-    const int E = p.E, W = p.W, nblk = p.nblk, bps = p.bm.bps;
+    const int E = p.E, W = p.W, nvb = p.nvb, bps = p.bps, G = p.nseg;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t C = p.C;
     const int scan_len = max(E, W * W) + 1;
     int64_t *s_a = reinterpret_cast<int64_t *>(scan_smem);
     int64_t *s_D = s_a + scan_len;
     int64_t *s_warp = s_D + W * W;
-    int32_t *s_cum = reinterpret_cast<int32_t *>(s_warp + 32);
+    int32_t *s_kh = reinterpret_cast<int32_t *>(s_warp + 32);
+    int32_t *cum = p.cum_global ? p.cum_global : s_kh + E * W;
 
-    // 1. per expert: exclusive scan over blocks; record shard starts
+    // 1. per expert: exclusive scan over virtual blocks; record segment starts
     for (int e = warp; e < E; e += NT / 32) {
-        int32_t *row = p.blk + (size_t)e * nblk;
+        int32_t *row = p.blk + (size_t)e * nvb;
         int carry = 0;
-        for (int base = 0; base < nblk; base += 128) {
+        for (int base = 0; base < nvb; base += 128) {
             int v[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int idx = base + lane * 4 + q;
-                v[q] = idx < nblk ? row[idx] : 0;
+                v[q] = idx < nvb ? row[idx] : 0;
             }
             const int lsum = v[0] + v[1] + v[2] + v[3];
             const int incl = warp_incl_scan(lsum);
@@ -125,27 +183,36 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int idx = base + lane * 4 + q;
-                if (idx < nblk) {
+                if (idx < nvb) {
                     row[idx] = run;
                     if (idx % bps == 0)
-                        s_cum[e * (W + 1) + idx / bps] = run;
+                        cum[e * (G + 1) + idx / bps] = run;
                 }
                 run += v[q];
             }
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0)
-            s_cum[e * (W + 1) + W] = carry;
+            cum[e * (G + 1) + G] = carry;
     }
     __syncthreads();
 
-    // 2. counts, kept, offsets
+    // 2. counts (round 0: the routed demand), kept, offsets; kept rows per
+    //    (expert, home shard)
     for (int e = threadIdx.x; e < E; e += NT) {
-        const int c = s_cum[e * (W + 1) + W];
-        const int kp = (int)min((int64_t)c, C);
+        const int c = cum[e * (G + 1) + p.nseg_round];
+        const int kp = (int)min((int64_t)cum[e * (G + 1) + G], C);
         p.counts[e] = c;
         p.kept[e] = kp;
         s_a[e] = kp;
+    }
+    for (int ei = threadIdx.x; ei < E * W; ei += NT) {
+        const int e = ei / W, i = ei % W;
+        const int32_t *ce = cum + e * (G + 1);
+        int64_t s = 0;
+        for (int g = i; g < G; g += W)
+            s += min((int64_t)ce[g + 1], C) - min((int64_t)ce[g], C);
+        s_kh[ei] = (int32_t)s;
     }
     __syncthreads();
     block_excl_scan_i64<NT>(s_a, E, s_warp);
@@ -158,11 +225,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
     for (int ij = threadIdx.x; ij < W * W; ij += NT) {
         const int i = ij / W, j = ij % W;
         int64_t s = 0;
-        for (int e = j * e_per; e < (j + 1) * e_per; ++e) {
-            const int64_t lo = min((int64_t)s_cum[e * (W + 1) + i], C);
-            const int64_t hi = min((int64_t)s_cum[e * (W + 1) + i + 1], C);
-            s += hi - lo;
-        }
+        for (int e = j * e_per; e < (j + 1) * e_per; ++e)
+            s += s_kh[e * W + i];
         s_D[ij] = s;
         if (p.D)
             p.D[ij] = s;
@@ -176,30 +240,36 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
         for (int ij = threadIdx.x; ij <= W * W; ij += NT)
             p.pk_off[ij] = s_a[ij];
 
-    // 4. pack bases: packed row of expert e's row at position pos from shard i
-    //    = pk_base[e][i] + pos
+    // 4. pack bases: a kept assignment to expert e at position pos (in e's rows)
+    //    from segment g lands on packed row pk_base[e][g] + pos. Block (i, j)
+    //    holds its experts in order, each expert's rows from shard i in the
+    //    shard's own order: the earlier segments of shard i come first.
     for (int ei = threadIdx.x; ei < E * W; ei += NT) {
         const int e = ei / W, i = ei % W;
         const int j = e / e_per;
         int64_t base = s_a[i * W + j];
-        for (int e2 = j * e_per; e2 < e; ++e2) {
-            const int64_t lo = min((int64_t)s_cum[e2 * (W + 1) + i], C);
-            const int64_t hi = min((int64_t)s_cum[e2 * (W + 1) + i + 1], C);
-            base += hi - lo;
+        for (int e2 = j * e_per; e2 < e; ++e2)
+            base += s_kh[e2 * W + i];
+        const int32_t *ce = cum + e * (G + 1);
+        int64_t run = 0;
+        for (int g = i; g < G; g += W) {
+            p.pk_base[(size_t)e * G + g] = base + run - ce[g];
+            run += ce[g + 1] - ce[g];
         }
-        base -= min((int64_t)s_cum[e * (W + 1) + i], C);
-        p.pk_base[ei] = base;
     }
 
-    // 5. counters
+    // 5. counters (dedup_pairs is added by the scatter kernel)
     if (p.stats && warp == 0) {
         int mx = 0, mn = 0x7fffffff, act = 0;
+        int64_t first = 0;  // rows from round 0
         for (int e = lane; e < E; e += 32) {
-            const int kp = (int)min((int64_t)s_cum[e * (W + 1) + W], C);
+            const int kp = (int)min((int64_t)cum[e * (G + 1) + G], C);
             mx = max(mx, kp);
             mn = min(mn, kp);
             act += kp > 0;
+            first += min((int64_t)cum[e * (G + 1) + p.nseg_round], C);
         }
+        first = warp_sum(first);
 #pragma unroll
         for (int off = 16; off; off >>= 1) {
             mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -220,37 +290,38 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
             p.stats->active_experts = act;
             p.stats->max_kept = mx;
             p.stats->min_kept = mn;
+            p.stats->rerouted = R - first;
         }
     }
 }
 
 struct PosArgs {
     const int32_t *topk_idx;
-    const int32_t *blk;  // [E][nblk] exclusive bases
-    int nblk;
-    BlockMap bm;
-    int N, E, K, W;
+    const int32_t *blk;  // [E][nvb] exclusive bases
+    int nvb;
+    VBlocks vbm;
+    int E;
     int C;
     const int32_t *offsets;
     int32_t *row_of;
     int32_t *assign_of_row;
-    moe_stats_t *stats;
 };
 
-// One CTA (8 warps) per dispatch block. Shared: wcnt [8][E] int32,
-// s_off [E] int32, krank [HB*K] int8 (destination rank of a kept slot, else -1).
+// One CTA (8 warps) per virtual block. Shared: wcnt [8][E] int32, s_off [E] int32.
+// Each assignment's row_of is written by exactly one block: its round-0 block,
+// unless it was moved, then its round-1 block.
 __global__ void __launch_bounds__(256) dispatch_positions_kernel(PosArgs p)
 {
     extern __shared__ __align__(16) int pos_smem[];
-    const int E = p.E, K = p.K;
+    const int E = p.E;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int *wcnt = pos_smem;
     int *s_off = wcnt + 8 * E;
-    signed char *krank = reinterpret_cast<signed char *>(s_off + E);
 
-    int t0, t1;
-    p.bm.range(blockIdx.x, t0, t1);
-    const int a0 = t0 * K, na = (t1 - t0) * K;
+    int t0, t1, k, round;
+    p.vbm.range(blockIdx.x, t0, t1, k, round);
+    const int32_t *src = p.vbm.experts(p.topk_idx, round);
+    const int na = p.vbm.count(t0, t1);
     const int per = (na + 7) / 8;
     const int wb = min(na, warp * per), we = min(na, wb + per);
 
@@ -260,13 +331,13 @@ __global__ void __launch_bounds__(256) dispatch_positions_kernel(PosArgs p)
         s_off[e] = p.offsets[e];
     __syncthreads();
     for (int i = wb + lane; i < we; i += 32) {
-        const int e = p.topk_idx[a0 + i];
+        const int e = src[p.vbm.assign(t0, k, i)];
         if ((unsigned)e < (unsigned)E)
             atomicAdd(&wcnt[warp * E + e], 1);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = p.blk[(size_t)e * p.nblk + blockIdx.x];
+        int run = p.blk[(size_t)e * p.nvb + blockIdx.x];
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
             const int c = wcnt[w * E + e];
@@ -278,11 +349,11 @@ __global__ void __launch_bounds__(256) dispatch_positions_kernel(PosArgs p)
 
     unsigned lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
-    const int e_per = E / p.W;
     for (int g = wb; g < we; g += 32) {
         const int i = g + lane;
         const bool act = i < we;
-        int e = act ? p.topk_idx[a0 + i] : -1;
+        const int a = act ? p.vbm.assign(t0, k, i) : 0;
+        int e = act ? src[a] : -1;
         if ((unsigned)e >= (unsigned)E)
             e = -1;
         const unsigned peers = __match_any_sync(0xffffffffu, e);
@@ -295,30 +366,95 @@ __global__ void __launch_bounds__(256) dispatch_positions_kernel(PosArgs p)
         if (act) {
             const int pos = base + rank;
             const int row = (e >= 0 && pos < p.C) ? s_off[e] + pos : -1;
-            p.row_of[a0 + i] = row;
+            const bool owner = round ? e >= 0
+                                     : (row >= 0 || p.vbm.moved == nullptr || p.vbm.moved[a] < 0);
+            if (owner)
+                p.row_of[a] = row;
             if (row >= 0)
-                p.assign_of_row[row] = a0 + i;
-            krank[i] = row >= 0 ? (signed char)(e / e_per) : (signed char)-1;
+                p.assign_of_row[row] = a;
         }
     }
-    if (p.stats == nullptr)
-        return;
-    __syncthreads();
-    const int S = p.bm.S;
-    unsigned long long pairs = 0;
-    for (int tt = threadIdx.x; tt < t1 - t0; tt += blockDim.x) {
-        const int home = (t0 + tt) / S;
-        unsigned long long m = 0;
-        for (int k = 0; k < K; ++k) {
-            const int j = krank[tt * K + k];
-            if (j >= 0 && j != home)
-                m |= 1ull << j;
+}
+
+struct RerouteArgs {
+    const float *logits;     // [N][E]
+    const int32_t *topk_idx;
+    const int32_t *row_of;   // after round 0: -1 = past capacity (or invalid expert)
+    const int32_t *counts;   // round-0 demand per expert
+    int N, E, K, C;
+    int32_t *moved;          // [N*K] out: new expert of a moved assignment, else -1
+};
+
+// One warp per token. An expert is full when its demand reached C. The token's
+// overflowed slots, in slot order, take its best remaining experts (larger logit
+// first, ties to the lower index; NaN ranks as -inf) that are neither routed to by
+// the token, nor full, nor taken by an earlier slot.
+__global__ void __launch_bounds__(256) reroute_kernel(RerouteArgs p)
+{
+    constexpr int MAXJ = 8;  // E <= 256
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
+        int mine = -1;
+        bool over = false;
+        if (lane < p.K) {
+            mine = p.topk_idx[t * p.K + lane];
+            over = (unsigned)mine < (unsigned)p.E && p.row_of[t * p.K + lane] < 0;
         }
-        pairs += __popcll(m);
+        unsigned om = __ballot_sync(0xffffffffu, over);
+        int res = -1;
+        if (om) {
+            float v[MAXJ];
+            bool avail[MAXJ];
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                const int e = lane + 32 * j;
+                avail[j] = false;
+                v[j] = -INFINITY;
+                if (e < p.E) {
+                    const float l = p.logits[(size_t)t * p.E + e];
+                    v[j] = isnan(l) ? -INFINITY : l;
+                    avail[j] = p.counts[e] < p.C;
+                }
+            }
+            for (int k = 0; k < p.K; ++k) {
+                const int ek = __shfl_sync(0xffffffffu, mine, k);
+#pragma unroll
+                for (int j = 0; j < MAXJ; ++j)
+                    if (ek == lane + 32 * j)
+                        avail[j] = false;
+            }
+            while (om) {
+                const int k = __ffs(om) - 1;
+                om &= om - 1;
+                float bv = -INFINITY;
+                int be = -1;
+#pragma unroll
+                for (int j = 0; j < MAXJ; ++j)
+                    if (avail[j] && (be < 0 || v[j] > bv)) {  // j ascending: ties keep the lower
+                        bv = v[j];
+                        be = lane + 32 * j;
+                    }
+#pragma unroll
+                for (int off = 16; off; off >>= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) {
+                        bv = ov;
+                        be = oe;
+                    }
+                }
+                if (lane == k)
+                    res = be;
+#pragma unroll
+                for (int j = 0; j < MAXJ; ++j)
+                    if (be == lane + 32 * j)
+                        avail[j] = false;
+            }
+        }
+        if (lane < p.K)
+            p.moved[t * p.K + lane] = res;
     }
-    pairs = warp_sum(pairs);
-    if (lane == 0 && pairs)
-        atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
 }
 
 struct ScatterArgs {
@@ -326,31 +462,62 @@ struct ScatterArgs {
     const int32_t *topk_idx;
     const int32_t *row_of;
     const int32_t *offsets;
-    const int64_t *pk_base;  // [E][W]
+    const int64_t *pk_base;  // [E][nseg]
+    const int32_t *moved;    // round-1 expert per assignment, or null
     int N, d, K, W, E;
-    int S;  // N / W
+    int S;           // N / W
+    int slot_major;  // segment of (t, k) in its round: k*W + t/S, else t/S
+    int nseg;        // all rounds
+    int nseg_round;
+    int32_t *expert_of;  // nullable out: the expert whose row each assignment uses, or -1
     uint16_t *x_sorted;
     uint16_t *x_packed;  // nullable
+    moe_stats_t *stats;  // nullable: dedup_pairs is accumulated here
 };
 
 // One warp per token: read the token's row once (16-byte loads), write it to
 // each kept slot's expert-sorted row and, when requested, to its packed row.
+// The token's distinct destination ranks other than its home (over kept slots)
+// are counted into stats->dedup_pairs.
 __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
 {
     constexpr int U = 4;
     const int lane = threadIdx.x & 31;
     const int nvec = p.d >> 3;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int e_per = p.E / p.W;
+    unsigned lt_mask;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
+    unsigned long long pairs = 0;
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
         int r = -1;
         long long pk = -1;
+        int dest = -1;
+        const int home = t / p.S;
         if (lane < p.K) {
             const int a = t * p.K + lane;
             r = p.row_of[a];
-            if (r >= 0 && p.x_packed) {
-                const int e = p.topk_idx[a];
-                pk = p.pk_base[(size_t)e * p.W + t / p.S] + (r - p.offsets[e]);
+            int ef = -1;
+            if (r >= 0) {
+                const int em = p.moved ? p.moved[a] : -1;
+                const int e = em >= 0 ? em : p.topk_idx[a];
+                ef = e;
+                dest = e / e_per;
+                if (p.x_packed) {
+                    const int g = (em >= 0 ? p.nseg_round : 0) +
+                                  (p.slot_major ? lane * p.W + home : home);
+                    pk = p.pk_base[(size_t)e * p.nseg + g] + (r - p.offsets[e]);
+                }
             }
+            if (p.expert_of)
+                p.expert_of[a] = ef;
+        }
+        if (p.stats) {
+            // distinct non-home destinations: count the lowest lane of each group
+            const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
+            const unsigned grp = __match_any_sync(0xffffffffu, key);
+            const unsigned first = __ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0);
+            pairs += __popc(first);
         }
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
         uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
@@ -379,6 +546,8 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
             }
         }
     }
+    if (p.stats && lane == 0 && pairs)
+        atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
 }
 
 }  // namespace moe

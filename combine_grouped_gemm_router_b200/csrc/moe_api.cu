@@ -29,8 +29,25 @@ inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3
 struct Geometry {
     int64_t C;           // capacity as used by the kernels (<= N*K)
     int64_t rows_alloc;  // min(N*K, E*C) + 128
-    int S, bps, nblk;    // dispatch blocks
+    int S, bps, nblk;    // dispatch token blocks
+    int slot_major;      // priority order of the positions
+    int rounds;          // 2 when overflowed assignments are re-routed
+    int nvb_round, nseg_round;  // virtual blocks and segments of one round
+    int nvb, nseg;       // ... of all rounds
+    bool cum_in_smem;    // the scan's per-segment starts fit in shared memory
 };
+
+constexpr size_t kScanSmemLimit = 200 * 1024;
+
+// Shared memory of dispatch_scan_kernel without / with the per-segment starts.
+size_t scan_smem_base(const moe_shape_t *s)
+{
+    const int E = s->E, W = s->W;
+    const int scan_len = (E > W * W ? E : W * W) + 1;
+    return (size_t)scan_len * 8 + (size_t)W * W * 8 + 32 * 8 + (size_t)E * W * 4;
+}
+
+size_t scan_cum_bytes(const moe_shape_t *s, int nseg) { return (size_t)s->E * (nseg + 1) * 4; }
 
 int64_t capacity_of(const moe_shape_t *s)
 {
@@ -44,7 +61,7 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
 {
     if (!s)
         return MOE_ERR_INVALID_ARG;
-    if ((s->flags & ~(uint32_t)MOE_FLAG_OUT_BF16) != 0)
+    if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE)) != 0)
         return MOE_ERR_INVALID_ARG;
     if (s->N < 1 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
         return MOE_ERR_INVALID_ARG;
@@ -66,14 +83,43 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
         g->S = s->N / s->W;
         g->bps = (g->S + kDispatchHB - 1) / kDispatchHB;
         g->nblk = s->W * g->bps;
+        g->slot_major = (s->flags & MOE_FLAG_SLOT_MAJOR) ? 1 : 0;
+        g->rounds = (s->flags & MOE_FLAG_REROUTE) ? 2 : 1;
+        g->nvb_round = g->slot_major ? s->K * g->nblk : g->nblk;
+        g->nseg_round = g->slot_major ? s->K * s->W : s->W;
+        g->nvb = g->rounds * g->nvb_round;
+        g->nseg = g->rounds * g->nseg_round;
+        g->cum_in_smem = scan_smem_base(s) + scan_cum_bytes(s, g->nseg) <= kScanSmemLimit;
     }
     return MOE_OK;
 }
 
 // Route/dispatch scratch, carved in this order from the workspace.
 struct ScratchLayout {
-    size_t logits, blk, pk_base, D, pk_off, total;
+    size_t logits, blk, pk_base, cum, moved, D, pk_off, total;
 };
+
+// The dispatch's own scratch (block bases, pack bases, segment starts when they
+// do not fit in shared memory, traffic matrix, pack offsets), from offset o.
+template <typename Layout>
+size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layout &L)
+{
+    L.blk = o;
+    o = align_up(o + (size_t)s->E * g.nvb * 4);
+    L.pk_base = o;
+    o = align_up(o + (size_t)s->E * g.nseg * 8);
+    L.cum = o;
+    if (!g.cum_in_smem)
+        o = align_up(o + scan_cum_bytes(s, g.nseg));
+    L.moved = o;
+    if (g.rounds > 1)
+        o = align_up(o + (size_t)s->N * s->K * 4);
+    L.D = o;
+    o = align_up(o + (size_t)s->W * s->W * 8);
+    L.pk_off = o;
+    o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
+    return o;
+}
 
 ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
 {
@@ -81,15 +127,7 @@ ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
     size_t o = 0;
     L.logits = o;
     o = align_up(o + (size_t)s->N * s->E * 4);
-    L.blk = o;
-    o = align_up(o + (size_t)s->E * g.nblk * 4);
-    L.pk_base = o;
-    o = align_up(o + (size_t)s->E * s->W * 8);
-    L.D = o;
-    o = align_up(o + (size_t)s->W * s->W * 8);
-    L.pk_off = o;
-    o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
-    L.total = o;
+    L.total = dispatch_scratch(s, g, o, L);
     return L;
 }
 
@@ -194,31 +232,36 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
 
 // ---------------------------------------------------------------- dispatch
 
-size_t scan_smem_bytes(const moe_shape_t *s)
+// Histogram, scan and positions over `rounds` rounds of virtual blocks.
+void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const int32_t *moved,
+                   const int32_t *topk_idx, int32_t *counts, int32_t *kept, int32_t *offsets,
+                   int32_t *row_of, int32_t *assign_of_row, int64_t *D, int64_t *pk_off,
+                   moe_stats_t *stats, int32_t *blk, int64_t *pk_base, int32_t *cum,
+                   cudaStream_t st)
 {
-    const int E = s->E, W = s->W;
-    const int scan_len = (E > W * W ? E : W * W) + 1;
-    return (size_t)scan_len * 8 + (size_t)W * W * 8 + 32 * 8 + (size_t)E * (W + 1) * 4;
-}
+    VBlocks vbm;
+    vbm.bm = BlockMap{g.S, g.bps, kDispatchHB};
+    vbm.nblk_tok = g.nblk;
+    vbm.slot_major = g.slot_major;
+    vbm.K = s->K;
+    vbm.nvb_round = g.nvb_round;
+    vbm.moved = moved;
+    const int nvb = rounds * g.nvb_round, nseg = rounds * g.nseg_round;
+    block_hist_kernel<<<nvb, 256, s->E * 4, st>>>(topk_idx, s->E, vbm, nvb, blk);
 
-moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x,
-                           const int32_t *topk_idx, int32_t *counts, int32_t *kept,
-                           int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
-                           uint16_t *x_sorted, uint16_t *x_packed, int64_t *D, int64_t *pk_off,
-                           moe_stats_t *stats, int32_t *blk, int64_t *pk_base, cudaStream_t st)
-{
-    BlockMap bm{g.S, g.bps, kDispatchHB};
-    block_hist_kernel<<<g.nblk, 256, s->E * 4, st>>>(topk_idx, s->K, s->E, bm, g.nblk, blk);
-
+    const bool cum_in_smem = scan_smem_base(s) + scan_cum_bytes(s, nseg) <= kScanSmemLimit;
     ScanArgs sa;
     sa.blk = blk;
-    sa.nblk = g.nblk;
-    sa.bm = bm;
+    sa.nvb = nvb;
+    sa.bps = g.bps;
+    sa.nseg = nseg;
+    sa.nseg_round = g.nseg_round;
     sa.N = s->N;
     sa.E = s->E;
     sa.K = s->K;
     sa.W = s->W;
     sa.C = (int)g.C;
+    sa.cum_global = cum_in_smem ? nullptr : cum;
     sa.counts = counts;
     sa.kept = kept;
     sa.offsets = offsets;
@@ -226,30 +269,57 @@ moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16
     sa.pk_off = pk_off;
     sa.pk_base = pk_base;
     sa.stats = stats;
-    const size_t scan_smem = scan_smem_bytes(s);
+    const size_t scan_smem = scan_smem_base(s) + (cum_in_smem ? scan_cum_bytes(s, nseg) : 0);
     static std::once_flag scan_attr;
     std::call_once(scan_attr, [] {
         cudaFuncSetAttribute(dispatch_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024);
+                             (int)kScanSmemLimit);
     });
     dispatch_scan_kernel<<<1, 1024, scan_smem, st>>>(sa);
 
     PosArgs pa;
     pa.topk_idx = topk_idx;
     pa.blk = blk;
-    pa.nblk = g.nblk;
-    pa.bm = bm;
-    pa.N = s->N;
+    pa.nvb = nvb;
+    pa.vbm = vbm;
     pa.E = s->E;
-    pa.K = s->K;
-    pa.W = s->W;
     pa.C = (int)g.C;
     pa.offsets = offsets;
     pa.row_of = row_of;
     pa.assign_of_row = assign_of_row;
-    pa.stats = stats;
-    const size_t pos_smem = (size_t)9 * s->E * 4 + (size_t)kDispatchHB * s->K;
-    dispatch_positions_kernel<<<g.nblk, 256, pos_smem, st>>>(pa);
+    const size_t pos_smem = (size_t)9 * s->E * 4;
+    dispatch_positions_kernel<<<nvb, 256, pos_smem, st>>>(pa);
+}
+
+// logits: needed when g.rounds == 2 (re-routing); moved: N*K int32 scratch then.
+moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x,
+                           const float *logits, const int32_t *topk_idx, int32_t *counts,
+                           int32_t *kept, int32_t *offsets, int32_t *row_of,
+                           int32_t *assign_of_row, int32_t *expert_of, uint16_t *x_sorted,
+                           uint16_t *x_packed, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
+                           int32_t *blk, int64_t *pk_base, int32_t *cum, int32_t *moved,
+                           cudaStream_t st)
+{
+    const int32_t *round1 = nullptr;
+    if (g.rounds > 1) {
+        // round 0 alone: which assignments are past capacity
+        dispatch_pass(s, g, 1, nullptr, topk_idx, counts, kept, offsets, row_of, assign_of_row,
+                      nullptr, nullptr, nullptr, blk, pk_base, cum, st);
+        RerouteArgs ra;
+        ra.logits = logits;
+        ra.topk_idx = topk_idx;
+        ra.row_of = row_of;
+        ra.counts = counts;
+        ra.N = s->N;
+        ra.E = s->E;
+        ra.K = s->K;
+        ra.C = (int)g.C;
+        ra.moved = moved;
+        reroute_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ra);
+        round1 = moved;
+    }
+    dispatch_pass(s, g, g.rounds, round1, topk_idx, counts, kept, offsets, row_of, assign_of_row,
+                  D, pk_off, stats, blk, pk_base, cum, st);
 
     ScatterArgs ca;
     ca.x = x;
@@ -257,14 +327,20 @@ moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16
     ca.row_of = row_of;
     ca.offsets = offsets;
     ca.pk_base = pk_base;
+    ca.moved = round1;
     ca.N = s->N;
     ca.d = s->d;
     ca.K = s->K;
     ca.W = s->W;
     ca.E = s->E;
     ca.S = g.S;
+    ca.slot_major = g.slot_major;
+    ca.nseg = g.nseg;
+    ca.nseg_round = g.nseg_round;
+    ca.expert_of = expert_of;
     ca.x_sorted = x_sorted;
     ca.x_packed = x_packed;
+    ca.stats = stats;
     scatter_rows_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
     return launch_status();
 }
@@ -580,12 +656,14 @@ moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
-__attribute__((visibility("default"))) moe_status_t
-moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx, int32_t *counts,
-             int32_t *kept, int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
-             uint16_t *x_sorted, uint16_t *x_packed, int64_t *rank_matrix,
-             int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
-             moe_stream_t stream)
+namespace {
+
+moe_status_t dispatch_entry(const moe_shape_t *shape, const uint16_t *x, const float *logits,
+                            const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                            int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                            int32_t *expert_of, uint16_t *x_sorted, uint16_t *x_packed,
+                            int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
+                            void *ws, size_t ws_bytes, moe_stream_t stream)
 {
     Geometry g;
     moe_status_t rc = check_shape(shape, false, &g);
@@ -593,9 +671,12 @@ moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_id
         return rc;
     if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)
         return MOE_ERR_INVALID_ARG;
+    if ((g.rounds > 1) != (logits != nullptr))
+        return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(x_sorted) || (x_packed && !aligned16(x_packed)) ||
         !aligned4(topk_idx) || !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) ||
-        !aligned4(row_of) || !aligned4(assign_of_row) ||
+        !aligned4(row_of) || !aligned4(assign_of_row) || (logits && !aligned4(logits)) ||
+        (expert_of && !aligned4(expert_of)) ||
         (rank_matrix && (reinterpret_cast<uintptr_t>(rank_matrix) & 7u)) ||
         (packed_offsets && (reinterpret_cast<uintptr_t>(packed_offsets) & 7u)) ||
         (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
@@ -608,10 +689,45 @@ moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_id
     char *w = static_cast<char *>(ws);
     int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
     int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
-    return dispatch_impl(shape, g, x, topk_idx, counts, kept, offsets, row_of, assign_of_row,
-                         x_sorted, x_packed, D, pk, stats, reinterpret_cast<int32_t *>(w + L.blk),
+    return dispatch_impl(shape, g, x, logits, topk_idx, counts, kept, offsets, row_of,
+                         assign_of_row, expert_of, x_sorted, x_packed, D, pk, stats,
+                         reinterpret_cast<int32_t *>(w + L.blk),
                          reinterpret_cast<int64_t *>(w + L.pk_base),
+                         reinterpret_cast<int32_t *>(w + L.cum),
+                         reinterpret_cast<int32_t *>(w + L.moved),
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+__attribute__((visibility("default"))) moe_status_t
+moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx, int32_t *counts,
+             int32_t *kept, int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+             uint16_t *x_sorted, uint16_t *x_packed, int64_t *rank_matrix,
+             int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
+             moe_stream_t stream)
+{
+    // re-routing ranks candidates by the logits, which this entry point does not take
+    if (shape && (shape->flags & MOE_FLAG_REROUTE))
+        return MOE_ERR_INVALID_ARG;
+    return dispatch_entry(shape, x, nullptr, topk_idx, counts, kept, offsets, row_of,
+                          assign_of_row, nullptr, x_sorted, x_packed, rank_matrix,
+                          packed_offsets, stats, ws, ws_bytes, stream);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, const float *logits,
+                     const int32_t *topk_idx, int32_t *counts, int32_t *kept, int32_t *offsets,
+                     int32_t *row_of, int32_t *assign_of_row, int32_t *expert_of,
+                     uint16_t *x_sorted, uint16_t *x_packed, int64_t *rank_matrix,
+                     int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
+                     moe_stream_t stream)
+{
+    if (!shape || !(shape->flags & MOE_FLAG_REROUTE) || !logits)
+        return MOE_ERR_INVALID_ARG;
+    return dispatch_entry(shape, x, logits, topk_idx, counts, kept, offsets, row_of,
+                          assign_of_row, expert_of, x_sorted, x_packed, rank_matrix,
+                          packed_offsets, stats, ws, ws_bytes, stream);
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -723,13 +839,16 @@ moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
     uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
     uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
     float *y = reinterpret_cast<float *>(w + L.y);
-    rc = dispatch_impl(shape, g, x, topk_idx, reinterpret_cast<int32_t *>(w + L.counts),
+    rc = dispatch_impl(shape, g, x, reinterpret_cast<const float *>(w + S.logits), topk_idx,
+                       reinterpret_cast<int32_t *>(w + L.counts),
                        reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
-                       reinterpret_cast<int32_t *>(w + L.assign), x_sorted,
+                       reinterpret_cast<int32_t *>(w + L.assign), nullptr, x_sorted,
                        reinterpret_cast<uint16_t *>(w + L.x_packed),
                        reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
                        stats, reinterpret_cast<int32_t *>(w + S.blk),
-                       reinterpret_cast<int64_t *>(w + S.pk_base), st);
+                       reinterpret_cast<int64_t *>(w + S.pk_base),
+                       reinterpret_cast<int32_t *>(w + S.cum),
+                       reinterpret_cast<int32_t *>(w + S.moved), st);
     if (rc != MOE_OK)
         return rc;
     rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
@@ -821,13 +940,16 @@ moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
     uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
     uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
     float *y = reinterpret_cast<float *>(w + L.y);
-    rc = dispatch_impl(shape, g, x, topk_idx, reinterpret_cast<int32_t *>(w + L.counts),
+    rc = dispatch_impl(shape, g, x, reinterpret_cast<const float *>(w + S.logits), topk_idx,
+                       reinterpret_cast<int32_t *>(w + L.counts),
                        reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
-                       reinterpret_cast<int32_t *>(w + L.assign), x_sorted,
+                       reinterpret_cast<int32_t *>(w + L.assign), nullptr, x_sorted,
                        reinterpret_cast<uint16_t *>(w + L.x_packed),
                        reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
                        stats, reinterpret_cast<int32_t *>(w + S.blk),
-                       reinterpret_cast<int64_t *>(w + S.pk_base), st);
+                       reinterpret_cast<int64_t *>(w + S.pk_base),
+                       reinterpret_cast<int32_t *>(w + S.cum),
+                       reinterpret_cast<int32_t *>(w + S.moved), st);
     if (rc != MOE_OK)
         return rc;
     rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
@@ -974,22 +1096,13 @@ moe_status_t static_scratch_address(void **out)
 }
 
 struct StaticLayout {
-    size_t blk, pk_base, D, pk_off, total;
+    size_t blk, pk_base, cum, moved, D, pk_off, total;
 };
 
 StaticLayout static_layout(const moe_shape_t *s, const Geometry &g)
 {
     StaticLayout L;
-    size_t o = 0;
-    L.blk = o;
-    o = align_up(o + (size_t)s->E * g.nblk * 4);
-    L.pk_base = o;
-    o = align_up(o + (size_t)s->E * s->W * 8);
-    L.D = o;
-    o = align_up(o + (size_t)s->W * s->W * 8);
-    L.pk_off = o;
-    o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
-    L.total = o;
+    L.total = dispatch_scratch(s, g, 0, L);
     return L;
 }
 
@@ -1006,6 +1119,8 @@ moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *
     moe_status_t rc = check_shape(shape, false, &g);
     if (rc != MOE_OK)
         return rc;
+    if (g.rounds > 1)  // re-routing needs the logits
+        return MOE_ERR_INVALID_ARG;
     if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(x_sorted) || (x_packed && !aligned16(x_packed)) ||
@@ -1025,8 +1140,10 @@ moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *
     char *w = static_cast<char *>(base);
     int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
     int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
-    return dispatch_impl(shape, g, x, topk_idx, counts, kept, offsets, row_of, assign_of_row,
-                         x_sorted, x_packed, D, pk, stats, reinterpret_cast<int32_t *>(w + L.blk),
+    return dispatch_impl(shape, g, x, nullptr, topk_idx, counts, kept, offsets, row_of,
+                         assign_of_row, nullptr, x_sorted, x_packed, D, pk, stats,
+                         reinterpret_cast<int32_t *>(w + L.blk),
                          reinterpret_cast<int64_t *>(w + L.pk_base),
+                         reinterpret_cast<int32_t *>(w + L.cum), nullptr,
                          reinterpret_cast<cudaStream_t>(stream));
 }

@@ -42,7 +42,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st *moe_stream_t; /* identical to cudaStream_t */
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -63,12 +63,37 @@ typedef enum moe_status {
 typedef struct moe_shape {
     int32_t N, d, f, E, K, W;
     float capacity_factor;
-    uint32_t flags; /* 0 or MOE_FLAG_OUT_BF16; other bits must be 0 */
+    uint32_t flags; /* MOE_FLAG_* bits below; other bits must be 0 */
 } moe_shape_t;
 
 /* moe_combine / moe_layer write `out` as bf16 (one rounding of the fp32 sum) instead of the
  * default fp32. Meant for a stack of layers whose next input is bf16. */
 #define MOE_FLAG_OUT_BF16 1u
+
+/* Which assignments claim an expert's capacity first ("MoE 推理服务工程真相 2026", §2.2:
+ * assignments beyond the capacity are dropped; the page leaves the order open).
+ * Default (flag clear): token-major, assignment a = t*K + k in increasing a, so an earlier
+ * token's second choice beats a later token's first choice. With MOE_FLAG_SLOT_MAJOR:
+ * slot-major, every token's slot 0 (tokens ascending), then every token's slot 1, ..., so
+ * first choices are served before any second choice. Positions, row_of, the expert-sorted
+ * rows and the packed buffer follow the chosen order (inside a packed block (i, j): expert
+ * by expert, each expert's rows in their expert-sorted order). Slot-major dispatch scans
+ * K times as many blocks. */
+#define MOE_FLAG_SLOT_MAJOR 2u
+
+/* Re-route overflowed assignments instead of dropping them ("MoE 推理服务工程真相 2026",
+ * §4.3, token drop: move the excess to the next-best expert; §2.3, the remapping of the
+ * overflow mask). Reading, one round: an expert is full when the assignments routed to it
+ * number at least C. Every assignment past capacity moves to its token's best-ranked expert
+ * (larger logit first, ties to the lower index) that the token did not route to, that is not
+ * full, and that no earlier overflowed slot of the same token (in k order) took; if there is
+ * none it is dropped. The moved assignments then queue at their new experts behind all the
+ * routed assignments there, in the same priority order (token- or slot-major), and the ones
+ * still past C are dropped. A moved assignment keeps its gate weight. The candidates are
+ * ranked by the router logits, so the flag is taken by moe_layer, moe_layer_shared and
+ * moe_dispatch_reroute, and refused (MOE_ERR_INVALID_ARG) by moe_dispatch and
+ * moe_dispatch_static. The dispatch then runs two passes plus a ranking kernel. */
+#define MOE_FLAG_REROUTE 4u
 
 /* Per-call dispatch counters, written (not accumulated) by moe_dispatch / moe_layer into
  * DEVICE memory when a non-null pointer is given. Observability signals of
@@ -85,6 +110,8 @@ typedef struct moe_stats {
     int32_t active_experts;   /* experts with at least one kept row */
     int32_t max_kept;         /* max_e kept[e] */
     int32_t min_kept;         /* min_e kept[e] */
+    int64_t rerouted;         /* rows held by an expert the token did not route to (moved there
+                                 by MOE_FLAG_REROUTE); 0 without re-routing */
 } moe_stats_t;
 
 /* Host-side report derived from moe_stats_t, the traffic matrix D and kept[]. */
@@ -160,6 +187,24 @@ moe_status_t moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int
                           int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
                           void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_dispatch with overflowed assignments re-routed (MOE_FLAG_REROUTE must be set in
+ * shape->flags; see there for the rule). Extra arguments:
+ *  logits    [N][E] fp32, DEVICE: the router logits the candidates are ranked by (as written
+ *            by moe_route).
+ *  expert_of [N*K] int32, DEVICE, nullable: the expert whose row each assignment uses, -1 if
+ *            it was dropped (equal to topk_idx where it was not moved).
+ * counts[e] stays the routed demand; kept, offsets, row_of, assign_of_row, the scatter, the
+ * traffic matrix and the packed layout describe the rows after re-routing (a moved row is
+ * packed by its new expert's rank). The workspace is moe_workspace_size(shape) with the flag
+ * set. */
+moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, const float *logits,
+                                  const int32_t *topk_idx, int32_t *counts, int32_t *kept,
+                                  int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                                  int32_t *expert_of, uint16_t *x_sorted, uint16_t *x_packed,
+                                  int64_t *rank_matrix, int64_t *packed_offsets,
+                                  moe_stats_t *stats, void *ws, size_t ws_bytes,
+                                  moe_stream_t stream);
+
 /* Size of the library's fixed device scratch array used by moe_dispatch_static. */
 #define MOE_STATIC_SCRATCH_BYTES (1u << 20)
 
@@ -174,7 +219,8 @@ moe_status_t moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int
  * inside the library. Every GPU that loads the library holds that array until the process
  * exits. The call allocates and frees nothing.
  *  - Shapes whose scratch does not fit (about E * W * ceil(N / (64 W)) * 4 bytes plus
- *    E * W * 8 + 2 * W * W * 8) return MOE_ERR_WORKSPACE_TOO_SMALL before any launch.
+ *    E * W * 8 + 2 * W * W * 8, the first two terms K times larger with MOE_FLAG_SLOT_MAJOR)
+ *    return MOE_ERR_WORKSPACE_TOO_SMALL before any launch. MOE_FLAG_REROUTE is refused.
  *  - The first call on a device looks up the array's device address on that device (the
  *    device must be current); make that first call before any stream capture.
  *  - All calls share the one array, and it keeps the last call's contents; every scratch byte

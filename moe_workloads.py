@@ -52,6 +52,8 @@ class Workload:
     router: str = "normal"   # "normal" (N(0,1/d)) or "uniform" (U(+-1/sqrt d))
     layers: int = 1
     shared_f: int = 0        # width of the shared dense MLP (Residual-MoE); 0 = none
+    slot_major: bool = False  # drop priority: first choices before second choices
+    reroute: bool = False     # move overflowed assignments to the next-best non-full expert
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -68,6 +70,12 @@ WORKLOADS = {
     # Residual-MoE: top-1 routed experts plus a shared dense MLP of the same width
     "residual_top1": Workload("residual_top1", N=4096, d=4096, f=14336, E=8, K=1, W=8,
                               router="uniform", shared_f=14336),
+    # the 128-expert skewed layer with slot-major drop priority (first choices first)
+    "e128_skew_slot_major": Workload("e128_skew_slot_major", N=8192, d=2048, f=768, E=128, K=8,
+                                     W=8, cf=1.25, s=1.1, slot_major=True),
+    # the same with overflowed assignments re-routed to the next-best non-full expert
+    "e128_skew_reroute": Workload("e128_skew_reroute", N=8192, d=2048, f=768, E=128, K=8, W=8,
+                                  cf=1.25, s=1.1, reroute=True),
     # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
     # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
     "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,

@@ -16,7 +16,8 @@ def lib():
 def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
     """route -> dispatch -> expert GEMMs -> combine, each through its C entry point."""
     m = lib()
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
+                         reroute=w.reroute)
     dev = torch.device(device)
     x = inp["x"].to(dev)
     wr = inp["w_router"].to(dev)
@@ -39,11 +40,19 @@ def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
     D = torch.empty(W * W, dtype=torch.int64, device=dev)
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
     stats = m.stats_buffer(dev)
-    m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted, x_packed,
-                   D, pk_off, stats, ws)
+    expert_of = None
+    if w.reroute:
+        expert_of = torch.full((N * K,), -7, dtype=torch.int32, device=dev)
+        m.moe_dispatch_reroute(shape, x, logits, topk_idx, counts, kept, offsets, row_of, assign,
+                               x_sorted, expert_of=expert_of, x_packed=x_packed, rank_matrix=D,
+                               packed_offsets=pk_off, stats=stats, ws=ws)
+    else:
+        m.moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign, x_sorted,
+                       x_packed, D, pk_off, stats, ws)
     res = dict(shape=shape, logits=logits, topk_idx=topk_idx, topk_w=topk_w, counts=counts,
                kept=kept, offsets=offsets, row_of=row_of, assign=assign, x_sorted=x_sorted,
-               x_packed=x_packed, D=D, pk_off=pk_off, stats_buf=stats, rows_alloc=RA)
+               x_packed=x_packed, D=D, pk_off=pk_off, stats_buf=stats, rows_alloc=RA,
+               expert_of=expert_of)
     if w.d % 128 == 0 and w.f % 128 == 0:
         h = torch.zeros(RA, f, dtype=torch.bfloat16, device=dev)
         y = torch.zeros(RA, d, dtype=torch.float32, device=dev)
@@ -60,7 +69,8 @@ def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
 
 def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True) -> dict:
     m = lib()
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
+                         reroute=w.reroute)
     dev = torch.device(device)
     ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
     out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)

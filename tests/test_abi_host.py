@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_abi_version_and_status_strings(m):
-    assert m.moe_abi_version() == 1
+    assert m.moe_abi_version() == 2
     for code, name in m.STATUS_NAMES.items():
         assert m.moe_status_string(code) == name
     assert m.moe_status_string(99) == "MOE_ERR_UNKNOWN"
@@ -68,9 +68,13 @@ def test_shape_validation(m):
         assert m.moe_rows_alloc(s) == -1
         assert m.moe_workspace_size(s) == 0
     flags = m.make_shape(64, 128, 256, 8, 2, 4)
-    flags.flags = 2
+    flags.flags = 8  # no such flag
     assert m.moe_workspace_size(flags) == 0
     assert m.moe_workspace_size(m.make_shape(64, 128, 256, 8, 2, 4, out_bf16=True)) > 0
+    # slot-major priority scans K blocks per token block: a larger scratch, never smaller
+    tm = m.moe_workspace_size(m.make_shape(4096, 128, 256, 256, 32, 64, 1.0))
+    sm = m.moe_workspace_size(m.make_shape(4096, 128, 256, 256, 32, 64, 1.0, slot_major=True))
+    assert 0 < tm < sm
     # GEMM shapes: d % 128, f % 128
     assert m.moe_layer_workspace_size(m.make_shape(64, 136, 256, 8, 2, 4)) == 0
     assert m.moe_layer_workspace_size(m.make_shape(64, 128, 200, 8, 2, 4)) == 0
@@ -108,6 +112,22 @@ def test_argument_errors_return_before_launch(m):
     assert lib.moe_route(by(bad), P, P, None, P, P, P, None, 0, None) == 1
     assert lib.moe_expert_gemm(by(m.make_shape(64, 192, 256, 8, 2, 4)), P, P, P, P, P, P, P,
                                None) == 2
+    # re-routing needs the logits: refused by the entry points that do not take them
+    rr = m.make_shape(64, 128, 256, 8, 2, 4, 1.0, reroute=True)
+    need_rr = m.moe_workspace_size(rr)
+    assert need_rr > need  # the moved-expert array
+    assert lib.moe_dispatch(by(rr), P, P, P, P, P, P, P, P, None, None, None, None, P, need_rr,
+                            None) == 1
+    assert lib.moe_dispatch_static(by(rr), P, P, P, P, P, P, P, P, None, None, None, None,
+                                   None) == 1
+    assert lib.moe_dispatch_reroute(by(rr), P, None, P, P, P, P, P, P, None, P, None, None, None,
+                                    None, P, need_rr, None) == 1  # no logits
+    assert lib.moe_dispatch_reroute(by(s), P, P, P, P, P, P, P, P, None, P, None, None, None,
+                                    None, P, need, None) == 1  # flag not set
+    assert lib.moe_dispatch_reroute(by(rr), P, P + 2, P, P, P, P, P, P, None, P, None, None, None,
+                                    None, P, need_rr, None) == 4  # misaligned logits
+    assert lib.moe_dispatch_reroute(by(rr), P, P, P, P, P, P, P, P, None, P, None, None, None,
+                                    None, P, need_rr - 1, None) == 3
     assert lib.moe_affinity_accumulate(10, 8, 9, P, P, P, None) == 1
     assert lib.moe_affinity_accumulate(10, 300, 2, P, P, P, None) == 2
     assert lib.moe_debug_bounded_wait(0, None) == 1

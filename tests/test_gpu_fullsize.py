@@ -39,7 +39,8 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     got = run_stages(inp, w)
     assert got["dev_error"] == 0
     hx = host_inputs(inp, experts=[])  # routing needs no expert weights
-    r = orc.route_and_dispatch(hx["x"], hx["w_router"], hx["bias"], w.K, w.W, w.cf)
+    r = orc.route_and_dispatch(hx["x"], hx["w_router"], hx["bias"], w.K, w.W, w.cf,
+                               order=int(w.slot_major), reroute=w.reroute)
 
     # routing and bookkeeping, in full
     np.testing.assert_array_equal(got["logits"].cpu().numpy().view(np.uint32),
@@ -54,9 +55,11 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     np.testing.assert_array_equal(got["pk_off"].cpu().numpy(), r["pk_off"])
     st, rs = got["stats"], r["stats"]
     assert (st["rows"], st["dropped"], st["cross_rows"], st["dedup_pairs"], st["active_experts"],
-            st["max_kept"], st["min_kept"]) == (rs["R"], rs["dropped"], rs["cross_rows"],
-                                                 rs["dedup_pairs"], rs["active_experts"],
-                                                 rs["max_kept"], rs["min_kept"])
+            st["max_kept"], st["min_kept"], st["rerouted"]) == (
+                rs["R"], rs["dropped"], rs["cross_rows"], rs["dedup_pairs"], rs["active_experts"],
+                rs["max_kept"], rs["min_kept"], rs["rerouted"])
+    if w.reroute:
+        np.testing.assert_array_equal(got["expert_of"].cpu().numpy(), r["expert_of"])
 
     # both scatter layouts, every row (indices verified above)
     aor = torch.from_numpy(r["assign_of_row"]).cuda().long()
@@ -68,12 +71,14 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     # sampled tokens through the experts: the oracle computes them one by one
     toks = sample_tokens(w.N, n_sample, seed)
     slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
-    used = np.unique(r["topk_idx"].reshape(-1)[slots])
+    eo = r["expert_of"][slots]
+    used = np.unique(eo[eo >= 0])
     remap = np.full(w.E, -1, np.int64)
     remap[used] = np.arange(len(used))
     hx = host_inputs(inp, experts=torch.from_numpy(used).cuda())
     rr = dict(r)
-    rr["topk_idx"] = remap[r["topk_idx"]].astype(np.int32)  # compact weight numbering
+    # compact weight numbering for the experts the sampled rows use
+    rr["expert_of"] = np.where(r["expert_of"] >= 0, remap[r["expert_of"]], -1).astype(np.int32)
     smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr, want_h=True)
     rows = torch.from_numpy(smp["sample_rows"]).cuda().long()
     rep_h = tolerance_report(got["h"][rows], smp["sample_h"])
@@ -92,6 +97,23 @@ def check_full_size(orc, w, seed=0, n_sample=24):
 def test_full_size_workload(orc, name):
     rep = check_full_size(orc, WORKLOADS[name])
     print(name, rep)
+
+
+@pytest.mark.parametrize("name", ["e128_skew", "stack4"])
+def test_full_size_slot_major(orc, name):
+    """Slot-major drop priority at full size, with capacity binding under the Zipf skew."""
+    w = WORKLOADS[name].with_(slot_major=True, s=1.2, cf=1.0)
+    rep = check_full_size(orc, w, n_sample=16)
+    print(name, "slot-major", rep)
+
+
+@pytest.mark.parametrize("slot_major", [False, True])
+@pytest.mark.parametrize("name", ["e128_skew", "stack4"])
+def test_full_size_reroute(orc, name, slot_major):
+    """Re-routing of overflowed assignments at full size, capacity binding under the skew."""
+    w = WORKLOADS[name].with_(reroute=True, slot_major=slot_major, s=1.2, cf=1.0)
+    rep = check_full_size(orc, w, n_sample=16)
+    print(name, "reroute", "slot-major" if slot_major else "token-major", rep)
 
 
 @pytest.mark.parametrize("cf", STACK_GRID_CF)
@@ -183,12 +205,13 @@ def test_full_size_residual_moe(orc):
     np.testing.assert_array_equal(topk.cpu().numpy(), r["topk_idx"])
     toks = sample_tokens(w.N, 16, 0)
     slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
-    used = np.unique(r["topk_idx"].reshape(-1)[slots])
+    eo = r["expert_of"][slots]
+    used = np.unique(eo[eo >= 0])
     remap = np.full(w.E, -1, np.int64)
     remap[used] = np.arange(len(used))
     hx = host_inputs(inp, experts=torch.from_numpy(used).cuda())
     rr = dict(r)
-    rr["topk_idx"] = remap[r["topk_idx"]].astype(np.int32)
+    rr["expert_of"] = np.where(r["expert_of"] >= 0, remap[r["expert_of"]], -1).astype(np.int32)
     smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr)
     dense = orc.shared_expert(hx["x"][torch.from_numpy(toks)], sh["ws1"].cpu(), sh["ws3"].cpu(),
                               sh["ws2"].cpu())

@@ -33,6 +33,29 @@ CASES = [
     # skewed rows (Zipf bias): large experts on the pair kernel, small ones on the
     # single-CTA kernel, in the same GEMM
     Workload("pair_split", N=3200, d=256, f=256, E=4, K=1, W=4, s=1.6),
+    # slot-major drop priority (first choices before second choices)
+    Workload("slot_major_drop", N=384, d=384, f=256, E=6, K=3, W=3, cf=1.0, s=1.1,
+             slot_major=True),
+    Workload("slot_major_ragged", N=1040, d=256, f=384, E=8, K=2, W=4, cf=0.8, s=0.8,
+             slot_major=True),
+    Workload("slot_major_wide_k", N=96, d=128, f=128, E=48, K=32, W=4, cf=0.75, s=1.0,
+             slot_major=True),
+    # 256 experts, K = 32, 64 ranks: the scan's 2048 segment starts per expert live in
+    # global memory instead of shared memory (no Zipf skew: with it, most assignments drop
+    # and the output tail alone takes bf16 rounding of h to the max-abs bar)
+    Workload("slot_major_many_segments", N=128, d=128, f=128, E=256, K=32, W=64, cf=1.0,
+             slot_major=True),
+    Workload("slot_major_dropless", N=200, d=128, f=128, E=10, K=3, W=5, slot_major=True),
+    # overflowed assignments re-routed to the next-best non-full expert
+    Workload("reroute_drop", N=384, d=384, f=256, E=6, K=3, W=3, cf=1.0, s=1.1, reroute=True),
+    Workload("reroute_slot_major", N=1040, d=256, f=384, E=8, K=2, W=4, cf=0.8, s=0.8,
+             slot_major=True, reroute=True),
+    Workload("reroute_many_experts", N=256, d=128, f=128, E=64, K=6, W=8, cf=1.0, s=0.6,
+             reroute=True),
+    # 256 experts: eight logits per lane in the ranking warp
+    Workload("reroute_e256", N=128, d=128, f=128, E=256, K=8, W=8, cf=0.5, reroute=True),
+    # K = E: every expert is routed to by every token, so there is no candidate
+    Workload("reroute_all_full", N=64, d=128, f=128, E=4, K=4, W=2, cf=0.5, reroute=True),
 ]
 
 
@@ -51,7 +74,8 @@ def _u16(t):
 @pytest.mark.parametrize("seed", [0, 1])
 def test_layer_stages_match_oracle(orc, w, seed):
     inp = make_layer_inputs(w, seed=seed)
-    ref = orc.layer(inp, w.K, w.W, w.cf, want_h=True)
+    ref = orc.layer(inp, w.K, w.W, w.cf, want_h=True, order=int(w.slot_major),
+                    reroute=w.reroute)
     got = run_stages(inp, w)
     assert got["dev_error"] == 0
 
@@ -76,6 +100,9 @@ def test_layer_stages_match_oracle(orc, w, seed):
         rs["R"], rs["dropped"], rs["cross_rows"], rs["dedup_pairs"])
     assert (st["active_experts"], st["max_kept"], st["min_kept"]) == (
         rs["active_experts"], rs["max_kept"], rs["min_kept"])
+    assert st["rerouted"] == rs["rerouted"]
+    if w.reroute:
+        np.testing.assert_array_equal(got["expert_of"].cpu().numpy(), ref["expert_of"])
     assert st["capacity"] == min(ref["C"], w.N * w.K)
 
     # a4: scatter is an exact copy, in both layouts
@@ -89,7 +116,7 @@ def test_layer_stages_match_oracle(orc, w, seed):
     # a5/a6: expert GEMMs; a7: combine
     assert_rounded_bf16(got["h"][:R], ref["h_rows"], "h")
     w2 = inp["w2"].double().numpy()
-    row_expert = ref["topk_idx"].reshape(-1)[ref["assign_of_row"]]
+    row_expert = ref["expert_of"][ref["assign_of_row"]]
     ybound = bf16_h_bound_rows(ref["h_rows"], w2, row_expert)
     assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
     obound = np.zeros((w.N, w.d))
