@@ -65,6 +65,14 @@ def _load():
         lib.orc_combine.restype = None
         lib.orc_affinity.argtypes = [_i64, _i64, _i64, _p, _p, _p]
         lib.orc_affinity.restype = None
+        lib.orc_e4m3_encode.argtypes = [_i64, _p, _p]
+        lib.orc_e4m3_encode.restype = None
+        lib.orc_e4m3_decode.argtypes = [_i64, _p, _p]
+        lib.orc_e4m3_decode.restype = None
+        lib.orc_e4m3_scale_exponent.argtypes = [ctypes.c_double]
+        lib.orc_e4m3_scale_exponent.restype = _i64
+        lib.orc_quantize_rows_e4m3.argtypes = [_i64, _i64, _p, _p, _p]
+        lib.orc_quantize_rows_e4m3.restype = None
         _lib = lib
     return _lib
 
@@ -282,6 +290,88 @@ def layer_shared(inp: dict, shared: dict, K: int, W: int, cf: float, want_h: boo
     r["shared_y"] = shared_expert(inp["x"], shared["ws1"], shared["ws3"], shared["ws2"])
     r["out_routed"] = r["out"]
     r["out"] = r["out_routed"] + r["shared_y"]
+    return r
+
+
+# --------------------------------------------------------------------------- FP8 payload
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest e4m3 code of each value (ties to even, saturating at +-448)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, np.uint8)
+    _load().orc_e4m3_encode(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, np.float64)
+    _load().orc_e4m3_decode(codes.size, _ptr(codes), _ptr(out))
+    return out
+
+
+def e4m3_scale_exponent(amax: float) -> int:
+    return int(_load().orc_e4m3_scale_exponent(float(amax)))
+
+
+def quantize_rows_e4m3(a) -> tuple:
+    """Row-wise e4m3 quantisation of a bf16 matrix (torch bf16 or uint16 bits, any
+    leading shape; rows are the last axis): (codes uint8, scale float32 per row)."""
+    u = as_u16(a)
+    shape = u.shape
+    cols = shape[-1]
+    rows = u.size // cols
+    codes = np.empty(shape, np.uint8)
+    scale = np.empty(shape[:-1], np.float32)
+    _load().orc_quantize_rows_e4m3(rows, cols, _ptr(u), _ptr(codes), _ptr(scale))
+    return codes, scale
+
+
+def dequantize_rows_bf16(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """code value * row scale, as bf16 bits. Exact: an e4m3 value has 4 significant
+    bits, bf16 has 8, and the scale is a power of two (asserted)."""
+    v = e4m3_decode(codes) * scale.astype(np.float64)[..., None]
+    f = v.astype(np.float32)
+    bits = f.view(np.uint32)
+    assert np.all((bits & 0xFFFF) == 0) and np.array_equal(f.astype(np.float64), v), \
+        "dequantised value not exact in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+def fp8_operands(inp: dict) -> dict:
+    """The e4m3 operands of the FP8 gate/up GEMM: x rows per token, W1 and W3 rows
+    per output channel, each with its power-of-two scale, and their exact bf16
+    dequantisations."""
+    xq, sx = quantize_rows_e4m3(inp["x"])
+    w1q, s1 = quantize_rows_e4m3(inp["w1"])
+    w3q, s3 = quantize_rows_e4m3(inp["w3"])
+    return dict(xq=xq, sx=sx, w1q=w1q, s1=s1, w3q=w3q, s3=s3,
+                x_deq=dequantize_rows_bf16(xq, sx), w1_deq=dequantize_rows_bf16(w1q, s1),
+                w3_deq=dequantize_rows_bf16(w3q, s3))
+
+
+def layer_fp8(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0,
+              reroute: bool = False) -> dict:
+    """The layer with the FP8 payload: routing on the bf16 x; the experts' gate/up
+    projections on e4m3 rows of x (one scale per token) and e4m3 rows of W1, W3 (one
+    scale per output channel), i.e. on their dequantised values; the down projection
+    and the combine as in ``layer``."""
+    q = fp8_operands(inp)
+    r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order, reroute)
+    N = r["logits"].shape[0]
+    aor = r["assign_of_row"]
+    row_token = (aor // K).astype(np.int32)
+    row_expert = r["expert_of"][aor].astype(np.int32)
+    h, y = expert_rows(row_token, row_expert, q["x_deq"], q["w1_deq"], q["w3_deq"], inp["w2"],
+                       want_h)
+    d = y.shape[1]
+    y_of_slot = np.zeros((N * K, d), np.float64)
+    kept = r["row_of"] >= 0
+    y_of_slot[kept] = y[r["row_of"][kept]]
+    r["out"] = combine(r["row_of"], r["topk_w"], y_of_slot)
+    r["y_rows"] = y
+    r["h_rows"] = h
+    r["fp8"] = q
     return r
 
 

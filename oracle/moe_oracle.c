@@ -20,6 +20,7 @@
  *       cumsum, scatter; dense token->expert mapping table), §ExFlow 跨层专家
  *       亲和性 (conditional routing between consecutive layers), §Aurora 定理
  *       4.2 (traffic matrix D).
+ *  [P2] §6.3 通信压缩 (the token payload of the all-to-all in FP8 instead of BF16).
  * Readings where the pages are silent (all fixed by the workload statement):
  *  softmax over the K selected logits; ties to the lowest expert index; logits
  *  accumulated in fp32 by one fused multiply-add per input element, i
@@ -430,4 +431,99 @@ EXPORT void orc_affinity(int64_t N, int64_t E, int64_t K, const int32_t *topk_j,
         for (int64_t k = 0; k < K; ++k)
             for (int64_t q = 0; q < K; ++q)
                 cnt[(int64_t)topk_j[t * K + k] * E + topk_j1[t * K + q]] += 1;
+}
+
+/* FP8 payload [P2 §6.3 通信压缩: the token rows that cross the all-to-all are sent as
+ * FP8 instead of BF16]. Format: e4m3 ("E4M3" of the OCP 8-bit floating-point formats):
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ * subnormals m * 2^-9; no infinities; code 0x7F/0xFF is NaN, so 448 = 1.75 * 2^8 is the
+ * largest finite value.
+ *
+ * Readings (the page names no scheme): one scale per row, a power of two, so that
+ * dividing by it is exact; the scale is the smallest 2^j with amax(row) * 2^-j <= 448,
+ * j clamped to [-126, 127] (a row of zeros, or a non-finite amax, takes j = 0); each
+ * element is x * 2^-j rounded to the nearest e4m3 value, ties to the even code, values
+ * beyond 448 saturated to 448. */
+
+/* e4m3 value of a code. */
+static double e4m3_value(uint8_t c)
+{
+    double s = (c & 0x80) ? -1.0 : 1.0;
+    int ef = (c >> 3) & 15, m = c & 7;
+    if (ef == 15 && m == 7)
+        return NAN;
+    if (ef == 0)
+        return s * ldexp((double)m, -9);
+    return s * ldexp(1.0 + m / 8.0, ef - 7);
+}
+
+/* Nearest e4m3 code to v (ties to even), saturating at +-448. */
+static uint8_t e4m3_code(double v)
+{
+    if (isnan(v))
+        return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs(v);
+    if (a > 448.0)
+        return sign | 0x7E;
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e); /* a = f * 2^e, f in [0.5, 1): the binade is [2^(e-1), 2^e) */
+    int E = e - 1 < -6 ? -6 : e - 1;
+    double quantum = ldexp(1.0, E - 3);       /* spacing of e4m3 values in this binade */
+    double val = nearbyint(a / quantum) * quantum; /* exact quotient; ties to even */
+    if (val > 448.0)
+        val = 448.0;
+    if (val == 0.0)
+        return sign;
+    frexp(val, &e);
+    E = e - 1;
+    if (E < -6)
+        return sign | (uint8_t)(val / ldexp(1.0, -9)); /* subnormal: exponent field 0 */
+    return sign | (uint8_t)((E + 7) << 3) | (uint8_t)(val / ldexp(1.0, E - 3) - 8.0);
+}
+
+EXPORT void orc_e4m3_encode(int64_t n, const double *v, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i)
+        codes[i] = e4m3_code(v[i]);
+}
+
+EXPORT void orc_e4m3_decode(int64_t n, const uint8_t *codes, double *v)
+{
+    for (int64_t i = 0; i < n; ++i)
+        v[i] = e4m3_value(codes[i]);
+}
+
+/* Scale exponent j of a row with largest magnitude amax. */
+EXPORT int64_t orc_e4m3_scale_exponent(double amax)
+{
+    if (!(amax > 0.0) || !isfinite(amax))
+        return 0;
+    int64_t j = -126;
+    while (j < 127 && ldexp(amax, (int)-j) > 448.0)
+        j += 1;
+    return j;
+}
+
+/* Row-wise quantisation of a bf16 matrix [rows][cols]: codes [rows][cols] and the
+ * scale 2^j of each row (value = code value * scale). */
+EXPORT void orc_quantize_rows_e4m3(int64_t rows, int64_t cols, const uint16_t *src,
+                                   uint8_t *codes, float *scale)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double amax = 0.0;
+        for (int64_t c = 0; c < cols; ++c) {
+            double a = fabs((double)bf16_to_float(src[r * cols + c]));
+            if (a > amax || isnan(a))
+                amax = a;
+        }
+        int64_t j = orc_e4m3_scale_exponent(amax);
+        scale[r] = (float)ldexp(1.0, (int)j);
+        for (int64_t c = 0; c < cols; ++c)
+            codes[r * cols + c] =
+                e4m3_code(ldexp((double)bf16_to_float(src[r * cols + c]), (int)-j));
+    }
 }

@@ -453,3 +453,112 @@ def test_reroute_brute_force(orc, seed):
                 assert len(set(got.tolist())) == len(got)
             plain = orc.positions(idx, E, W, C, order=order)
             assert p["stats"]["dropped"] == plain["stats"]["dropped"] - p["stats"]["rerouted"]
+
+
+# --------------------------------------------------------------------------- FP8 payload
+# e4m3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no infinities, 448 the largest.
+
+E4M3_HAND = [  # (value, code): format corners and round-to-nearest-even ties, worked by hand
+    (0.0, 0x00), (-0.0, 0x80), (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (-448.0, 0xFE),
+    (500.0, 0x7E),  # saturates
+    (2.0 ** -9, 0x01), (7 * 2.0 ** -9, 0x07), (2.0 ** -6, 0x08),  # subnormals, smallest normal
+    (2.0 ** -10, 0x00),  # half the smallest subnormal: tie to the even code 0
+    (3 * 2.0 ** -10, 0x02),  # 1.5 subnormal quanta: tie to 2
+    (1.0625, 0x38),  # halfway 1.0 / 1.125: even mantissa 0
+    (1.1875, 0x3A),  # halfway 1.125 / 1.25: even mantissa 2
+    (240.0, 0x77), (256.0, 0x78), (416.0, 0x7D), (432.0, 0x7E),  # 432 halfway 416 / 448 -> 448
+]
+
+
+def test_e4m3_hand_values(orc):
+    v = np.array([a for a, _ in E4M3_HAND])
+    np.testing.assert_array_equal(orc.e4m3_encode(v), [c for _, c in E4M3_HAND])
+    assert np.isnan(orc.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+    assert orc.e4m3_encode(np.array([np.nan]))[0] == 0x7F
+
+
+def test_e4m3_round_trip_every_code(orc):
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    np.testing.assert_array_equal(orc.e4m3_encode(orc.e4m3_decode(codes)), codes)
+    vals = orc.e4m3_decode(codes[codes < 0x80])
+    assert np.all(np.diff(vals) > 0) and vals.max() == 448.0  # monotone codes, largest 448
+
+
+def test_e4m3_matches_torch_float8(orc):
+    """torch's float8_e4m3fn conversion is an independent implementation of the same
+    rounding: agree on random values and on every tie."""
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.standard_normal(100000) * 30,
+                        rng.uniform(-448, 448, 50000),
+                        np.exp(rng.uniform(-16, 6, 50000)) * rng.choice([-1, 1], 50000)])
+    codes = np.arange(0x7F, dtype=np.uint8)
+    grid = orc.e4m3_decode(codes[codes != 0x7F])
+    v = np.concatenate([v, (grid[1:] + grid[:-1]) / 2, -(grid[1:] + grid[:-1]) / 2])
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(orc.e4m3_encode(v), ref)
+
+
+def test_e4m3_scale_exponent(orc):
+    assert orc.e4m3_scale_exponent(0.0) == 0
+    assert orc.e4m3_scale_exponent(448.0) == 0 and orc.e4m3_scale_exponent(449.0) == 1
+    assert orc.e4m3_scale_exponent(1.0) == -8  # 1 * 2^8 = 256 <= 448 < 512
+    assert orc.e4m3_scale_exponent(float("inf")) == 0
+    rng = np.random.default_rng(1)
+    for amax in np.exp(rng.uniform(-80, 80, 2000)):
+        j = orc.e4m3_scale_exponent(amax)
+        assert 224.0 < math.ldexp(amax, -j) <= 448.0  # the smallest power of two that fits
+
+
+def test_quantize_rows(orc):
+    """Row quantisation = per-row power-of-two scale + e4m3 rounding, checked against
+    torch's float8 conversion of the scaled rows; the scaled row maximum lies in (224, 448],
+    so its code lies in [224, 448] (224.x may round down to 224)."""
+    rng = np.random.default_rng(2)
+    a = torch.from_numpy(rng.standard_normal((64, 96)) * np.exp(rng.uniform(-20, 20, (64, 1))))
+    a = a.to(torch.bfloat16)
+    a[3] = 0.0
+    codes, scale = orc.quantize_rows_e4m3(a)
+    af = a.double().numpy()
+    for r in range(a.shape[0]):
+        j = orc.e4m3_scale_exponent(np.abs(af[r]).max())
+        assert scale[r] == math.ldexp(1.0, j)
+        ref = torch.from_numpy(af[r] / scale[r]).to(torch.float8_e4m3fn).view(torch.uint8)
+        np.testing.assert_array_equal(codes[r], ref.numpy())
+        if r != 3:
+            assert 224.0 <= np.abs(orc.e4m3_decode(codes[r])).max() <= 448.0
+    assert np.all(codes[3] == 0) and scale[3] == 1.0
+    # dequantised values are exact bf16 and within half an e4m3 step of the input
+    deq = orc.dequantize_rows_bf16(codes, scale)
+    back = (deq.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    rel = np.abs(back - af) / np.maximum(np.abs(af), 2.0 ** -6 * scale[:, None])
+    assert rel.max() <= 2.0 ** -4
+
+
+def test_layer_fp8_reduces_to_bf16_layer_on_e4m3_inputs(orc):
+    """With x, W1, W3 already e4m3 values whose rows reach the top binade, quantisation is
+    the identity and the FP8 layer equals the bf16 layer exactly; on ordinary inputs it
+    stays within the e4m3 rounding bar (three mantissa bits on x and on W1, W3: relative
+    error <= 2^-4 per element, so the relative Frobenius deviation of the output is a few
+    times 2^-4 / sqrt(3) at most; bar 0.1)."""
+    w = WORKLOADS["tiny"]
+    inp = make_layer_inputs(w, seed=3)
+    rng = np.random.default_rng(3)
+    grid = orc.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+
+    def e4m3_like(shape, scale_exp):
+        v = rng.choice(grid[1:], size=shape) * rng.choice([-1.0, 1.0], size=shape)
+        v[..., 0] = 448.0  # every row's maximum in the top binade: scale exactly 2^scale_exp
+        return torch.from_numpy(v * 2.0 ** scale_exp).to(torch.bfloat16)
+
+    exact = dict(inp, x=e4m3_like(tuple(inp["x"].shape), -12),
+                 w1=e4m3_like(tuple(inp["w1"].shape), -14),
+                 w3=e4m3_like(tuple(inp["w3"].shape), -14))
+    a = orc.layer_fp8(exact, w.K, w.W, w.cf)
+    b = orc.layer(exact, w.K, w.W, w.cf)
+    assert np.all(a["fp8"]["sx"] == 2.0 ** -12) and np.all(a["fp8"]["s1"] == 2.0 ** -14)
+    np.testing.assert_array_equal(a["out"], b["out"])
+    r8 = orc.layer_fp8(inp, w.K, w.W, w.cf)
+    r16 = orc.layer(inp, w.K, w.W, w.cf)
+    np.testing.assert_array_equal(r8["row_of"], r16["row_of"])  # routing is on the bf16 x
+    dev = np.linalg.norm(r8["out"] - r16["out"]) / np.linalg.norm(r16["out"])
+    assert 1e-3 < dev <= 0.1, dev
