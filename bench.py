@@ -188,7 +188,9 @@ def algorithmic_work(w, R: int) -> dict:
         down_flops=2.0 * d * f * R,
         logits_bytes=N * d * 2 + E * d * 4 + N * E * 4,
         # scatter: read each token row once, write every kept row twice (sorted + packed)
-        scatter_bytes=N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3,
+        # (the FP8 payload writes one byte per element and a 4-byte scale per row)
+        scatter_bytes=(N * d * 2 + 2 * R * (d + 4) + N * K * 4 * 3 if w.fp8
+                       else N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3),
         # combine: read every kept fp32 expert row, the routing, write fp32 out
         combine_bytes=R * d * 4 + N * K * 8 + N * d * 4,
     )
@@ -209,6 +211,8 @@ def run_gpu(args, w) -> dict:
     # one step = the whole stack of w.layers layers (one layer unless the workload is a stack)
     L = w.layers
     shared = w.shared_f > 0
+    if w.fp8 and (w.reroute or shared or w.layers > 1):
+        raise ValueError("the FP8 payload is benchmarked on single plain layers")
     layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
               for l in range(L)]
     inp = layers[0]
@@ -227,8 +231,20 @@ def run_gpu(args, w) -> dict:
     offsets = [torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
     row_of = torch.empty(N * K, dtype=torch.int32, device=dev)
     assign = torch.empty(RA, dtype=torch.int32, device=dev)
-    x_sorted = torch.empty(RA, d, dtype=torch.bfloat16, device=dev)
-    x_packed = torch.empty(RA, d, dtype=torch.bfloat16, device=dev)
+    pay_dt = torch.uint8 if w.fp8 else torch.bfloat16  # e4m3 codes or bf16 rows
+    x_sorted = torch.empty(RA, d, dtype=pay_dt, device=dev)
+    x_packed = torch.empty(RA, d, dtype=pay_dt, device=dev)
+    if w.fp8:
+        # the FP8 payload's row scales; the experts' W1, W3 quantised once (weights are static)
+        sorted_scale = torch.empty(RA, dtype=torch.float32, device=dev)
+        packed_scale = torch.empty(RA, dtype=torch.float32, device=dev)
+        for lw in layers:
+            for k in ("w1", "w3"):
+                q = torch.empty(E, f, d, dtype=torch.uint8, device=dev)
+                sc = torch.empty(E, f, dtype=torch.float32, device=dev)
+                m.moe_quantize_rows_e4m3(lw[k], q, sc)
+                lw[k + "q"], lw[k + "s"] = q, sc
+        torch.cuda.synchronize(dev)
     D = torch.empty(W * W, dtype=torch.int64, device=dev)
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
     h = torch.empty(RA, f, dtype=torch.bfloat16, device=dev)
@@ -267,7 +283,12 @@ def run_gpu(args, w) -> dict:
                         st)
             if e is not None:
                 e[1].record(st)
-            if w.reroute:
+            if w.fp8:
+                m.moe_dispatch_fp8(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of,
+                                   assign, x_sorted, sorted_scale, x_packed=x_packed,
+                                   packed_scale=packed_scale, rank_matrix=D,
+                                   packed_offsets=pk_off, ws=ws, stream=st)
+            elif w.reroute:
                 m.moe_dispatch_reroute(shape, xin, logits, topk_idx[l], counts, kept, offsets[l],
                                        row_of, assign, x_sorted, x_packed=x_packed, rank_matrix=D,
                                        packed_offsets=pk_off, ws=ws, stream=st)
@@ -276,7 +297,11 @@ def run_gpu(args, w) -> dict:
                                x_sorted, x_packed, D, pk_off, None, ws, st)
             if e is not None:
                 e[2].record(st)
-            m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
+            if w.fp8:
+                m.moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets[l], lw["w1q"],
+                                    lw["w1s"], lw["w3q"], lw["w3s"], h, st)
+            else:
+                m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
             if e is not None:
                 e[3].record(st)
             m.moe_expert_down(shape, h, offsets[l], lw["w2"], y, st)
@@ -385,6 +410,10 @@ def run_gpu(args, w) -> dict:
                 m.moe_layer_shared(shape, w.shared_f, x_dev[b], l0["w_router"], l0["bias"],
                                    l0["w1"], l0["w3"], l0["w2"], sh["ws1"], sh["ws3"], sh["ws2"],
                                    out_dev[b], ws=lws, stream=stream)
+            elif w.fp8:
+                m.moe_layer_fp8(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1q"],
+                                l0["w1s"], l0["w3q"], l0["w3s"], l0["w2"], out_dev[b], ws=lws,
+                                stream=stream)
             elif L == 1:
                 m.moe_layer(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1"], l0["w3"],
                             l0["w2"], out_dev[b], ws=lws, stream=stream)
@@ -430,6 +459,8 @@ def run_gpu(args, w) -> dict:
         for k, v in algorithmic_work(w, Rl).items():
             work[k] = work.get(k, 0.0) + v
     peaks = load_peaks()
+    up_ratio = 2.0 if w.fp8 else 1.0  # e4m3 tensor throughput is twice bf16's (nominal)
+    up_peak = peaks["bf16_tflops"] * up_ratio
     up_s = stage_ms["expert_up"] / 1e3
     down_s = stage_ms["expert_down"] / 1e3
     up_tflops = work["up_flops"] / up_s / 1e12
@@ -449,7 +480,8 @@ def run_gpu(args, w) -> dict:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": ("e4m3 gate/up operands and dispatch payload, bf16 down, fp32 accumulate"
+                  if w.fp8 else "bf16"),
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",
         "config": {"workload": w.name, "N": N, "d": d, "f": f, "E": E, "K": K, "W": W,
@@ -459,12 +491,15 @@ def run_gpu(args, w) -> dict:
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step"},
-        "roofline": {"kernel": "grouped GEMM gate/up (moe_expert_up, CTA-pair tcgen05 kernel)",
+        "roofline": {"kernel": ("grouped GEMM gate/up on e4m3 (moe_expert_up_fp8, tcgen05 "
+                                "kind::f8f6f4)" if w.fp8 else
+                                "grouped GEMM gate/up (moe_expert_up, CTA-pair tcgen05 kernel)"),
                      "bound": "tensor",
-                     "achieved": up_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": up_tflops / peaks["bf16_tflops"],
-                     "peak_source": peaks["source"] + " bf16 burst",
-                     "frac_of_sustained": up_tflops / peaks["bf16_tflops_sustained"],
+                     "achieved": up_tflops, "peak": up_peak, "unit": "TFLOP/s",
+                     "frac": up_tflops / up_peak,
+                     "peak_source": (peaks["source"] + " bf16 burst x 2 (the nominal e4m3/bf16 "
+                                     "dense ratio)" if w.fp8 else peaks["source"] + " bf16 burst"),
+                     "frac_of_sustained": up_tflops / (peaks["bf16_tflops_sustained"] * up_ratio),
                      "traffic": up_traffic(w.name),
                      "algorithmic_flops_per_launch": work["up_flops"] / L},
         "stages_ms": stages,
@@ -511,14 +546,25 @@ def oracle_time(w, inp_cpu, sample_tokens: int, shared_cpu=None) -> dict:
 
     import oracle
     oracle.build()
+    exp_inp = inp_cpu
+    if w.fp8:  # the experts' W1, W3 quantised once, outside the timing (static weights)
+        import torch
+        as_bf16 = lambda u: torch.from_numpy(u.view(np.int16)).view(torch.bfloat16)
+        q1, s1 = oracle.quantize_rows_e4m3(inp_cpu["w1"])
+        q3, s3 = oracle.quantize_rows_e4m3(inp_cpu["w3"])
+        exp_inp = dict(inp_cpu, w1=as_bf16(oracle.dequantize_rows_bf16(q1, s1)),
+                       w3=as_bf16(oracle.dequantize_rows_bf16(q3, s3)))
     t0 = time.perf_counter()
     r = oracle.route_and_dispatch(inp_cpu["x"], inp_cpu["w_router"], inp_cpu.get("bias"), w.K,
                                   w.W, w.cf, order=int(w.slot_major), reroute=w.reroute)
+    if w.fp8:  # the FP8 payload: every token row quantised
+        xq, sx = oracle.quantize_rows_e4m3(inp_cpu["x"])
+        exp_inp = dict(exp_inp, x=as_bf16(oracle.dequantize_rows_bf16(xq, sx)))
     t_route = time.perf_counter() - t0
     rng = np.random.default_rng(0)
     toks = np.sort(rng.choice(w.N, size=min(sample_tokens, w.N), replace=False))
     t1 = time.perf_counter()
-    oracle.layer_sampled(inp_cpu, w.K, w.W, w.cf, toks, routing=r)
+    oracle.layer_sampled(exp_inp, w.K, w.W, w.cf, toks, routing=r)
     if shared_cpu is not None:
         oracle.shared_expert(inp_cpu["x"][torch_index(toks)], shared_cpu["ws1"], shared_cpu["ws3"],
                              shared_cpu["ws2"])

@@ -62,6 +62,10 @@ _sigs = {
     "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
     "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
     "moe_dispatch_reroute": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
+    "moe_dispatch_fp8": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
+    "moe_quantize_rows_e4m3": ([c_p, c_i64, c_i32, c_p, c_p, c_p], c_i32),
+    "moe_expert_up_fp8": ([_SP] + [c_p] * 9, c_i32),
+    "moe_layer_fp8": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
     "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
     "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
     "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
@@ -213,6 +217,34 @@ def moe_dispatch_reroute(shape, x, logits, topk_idx, counts, kept, offsets, row_
            "moe_dispatch_reroute")
 
 
+def moe_dispatch_fp8(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_row, x_sorted,
+                     sorted_scale, x_packed=None, packed_scale=None, rank_matrix=None,
+                     packed_offsets=None, stats=None, ws=None, stream=None):
+    """moe_dispatch writing the FP8 payload: e4m3 rows (uint8) with one scale per row."""
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_dispatch_fp8(ctypes.byref(shape), _ptr(x), _ptr(topk_idx), _ptr(counts),
+                                 _ptr(kept), _ptr(offsets), _ptr(row_of), _ptr(assign_of_row),
+                                 _ptr(x_sorted), _ptr(sorted_scale), _ptr(x_packed),
+                                 _ptr(packed_scale), _ptr(rank_matrix), _ptr(packed_offsets),
+                                 _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_dispatch_fp8")
+
+
+def moe_quantize_rows_e4m3(src, codes, scale, stream=None):
+    """Row-wise e4m3 quantisation of a bf16 matrix (rows = all leading dims)."""
+    cols = src.shape[-1]
+    rows = src.numel() // cols
+    _check(_lib.moe_quantize_rows_e4m3(_ptr(src), rows, cols, _ptr(codes), _ptr(scale),
+                                       _stream(stream)), "moe_quantize_rows_e4m3")
+
+
+def moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q, w3_scale, h,
+                      stream=None):
+    _check(_lib.moe_expert_up_fp8(ctypes.byref(shape), _ptr(x_sorted), _ptr(sorted_scale),
+                                  _ptr(offsets), _ptr(w1q), _ptr(w1_scale), _ptr(w3q),
+                                  _ptr(w3_scale), _ptr(h), _stream(stream)), "moe_expert_up_fp8")
+
+
 MOE_STATIC_SCRATCH_BYTES = 1 << 20
 
 
@@ -277,6 +309,17 @@ def moe_layer(shape, x, w_router, bias, w1, w3, w2, out, residual=None, topk_idx
     _check(_lib.moe_layer(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1),
                           _ptr(w3), _ptr(w2), _ptr(residual), _ptr(out), _ptr(topk_idx_out),
                           _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)), "moe_layer")
+
+
+def moe_layer_fp8(shape, x, w_router, bias, w1q, w1_scale, w3q, w3_scale, w2, out, residual=None,
+                  topk_idx_out=None, stats=None, ws=None, stream=None):
+    """moe_layer with the FP8 payload and the e4m3 gate/up GEMM (weights from
+    moe_quantize_rows_e4m3)."""
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_layer_fp8(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias),
+                              _ptr(w1q), _ptr(w1_scale), _ptr(w3q), _ptr(w3_scale), _ptr(w2),
+                              _ptr(residual), _ptr(out), _ptr(topk_idx_out), _ptr(stats),
+                              _ptr(ws), ws_bytes, _stream(stream)), "moe_layer_fp8")
 
 
 def moe_affinity_accumulate(N, E, K, topk_j, topk_j1, counts, stream=None):

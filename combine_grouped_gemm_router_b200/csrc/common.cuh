@@ -58,6 +58,40 @@ __device__ __forceinline__ T warp_sum(T v)
     return v;
 }
 
+// e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448):
+// two fp32 values -> two codes, round to nearest even, saturating; lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Exponent j of a row's power-of-two scale: the smallest j with amax * 2^-j <= 448,
+// clamped to [-126, 127]; 0 for a zero or non-finite amax. From the bits of amax
+// (amax = m * 2^k, m in [1, 2)): j = k - 8 when m <= 1.75, else k - 7.
+__device__ __forceinline__ int e4m3_scale_exp(float amax)
+{
+    if (!(amax > 0.0f) || !isfinite(amax))
+        return 0;
+    const uint32_t b = __float_as_uint(amax);
+    int k;
+    uint32_t frac;
+    if (b >= 0x00800000u) {
+        k = (int)(b >> 23) - 127;
+        frac = b & 0x007FFFFFu;
+    } else {  // subnormal: normalise the significand
+        const int lz = __clz(b) - 8;
+        k = -126 - lz;
+        frac = (b << lz) & 0x007FFFFFu;
+    }
+    const int j = frac <= 0x00600000u ? k - 8 : k - 7;
+    return max(-126, min(127, j));
+}
+
+// 2^j for j in [-126, 127] (a normal float).
+__device__ __forceinline__ float pow2f(int j) { return __uint_as_float((uint32_t)(j + 127) << 23); }
+
 // Token block b of the dispatch: blocks never straddle a home-rank shard, so
 // per-shard prefix counts are available at block boundaries.
 // shard = b / bps, tokens [shard*S + (b%bps)*HB, min(... + HB, (shard+1)*S)).

@@ -470,10 +470,50 @@ struct ScatterArgs {
     int nseg;        // all rounds
     int nseg_round;
     int32_t *expert_of;  // nullable out: the expert whose row each assignment uses, or -1
-    uint16_t *x_sorted;
-    uint16_t *x_packed;  // nullable
+    void *x_sorted;      // bf16 rows, or e4m3 rows with fp8 payload
+    void *x_packed;      // nullable, same element type
+    float *sorted_scale;  // e4m3 payload: scale of each x_sorted row
+    float *packed_scale;  // e4m3 payload: scale of each x_packed row (nullable)
     moe_stats_t *stats;  // nullable: dedup_pairs is accumulated here
 };
+
+// Targets of slot `lane` (lanes < K) of token t: its expert-sorted row r (-1 if
+// dropped) and packed row pk (-1 if dropped or not packing); also writes
+// expert_of and returns the number of distinct non-home destination ranks of the
+// token (the same value in every lane), when counting.
+__device__ __forceinline__ int slot_targets(const ScatterArgs &p, int t, int lane,
+                                            unsigned lt_mask, int &r, long long &pk)
+{
+    const int e_per = p.E / p.W;
+    const int home = t / p.S;
+    int dest = -1;
+    r = -1;
+    pk = -1;
+    if (lane < p.K) {
+        const int a = t * p.K + lane;
+        r = p.row_of[a];
+        int ef = -1;
+        if (r >= 0) {
+            const int em = p.moved ? p.moved[a] : -1;
+            const int e = em >= 0 ? em : p.topk_idx[a];
+            ef = e;
+            dest = e / e_per;
+            if (p.x_packed) {
+                const int g = (em >= 0 ? p.nseg_round : 0) +
+                              (p.slot_major ? lane * p.W + home : home);
+                pk = p.pk_base[(size_t)e * p.nseg + g] + (r - p.offsets[e]);
+            }
+        }
+        if (p.expert_of)
+            p.expert_of[a] = ef;
+    }
+    if (!p.stats)
+        return 0;
+    // distinct non-home destinations: count the lowest lane of each group
+    const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
+    const unsigned grp = __match_any_sync(0xffffffffu, key);
+    return __popc(__ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0));
+}
 
 // One warp per token: read the token's row once (16-byte loads), write it to
 // each kept slot's expert-sorted row and, when requested, to its packed row.
@@ -485,40 +525,13 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
     const int lane = threadIdx.x & 31;
     const int nvec = p.d >> 3;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
-    const int e_per = p.E / p.W;
     unsigned lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     unsigned long long pairs = 0;
     for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
-        int r = -1;
-        long long pk = -1;
-        int dest = -1;
-        const int home = t / p.S;
-        if (lane < p.K) {
-            const int a = t * p.K + lane;
-            r = p.row_of[a];
-            int ef = -1;
-            if (r >= 0) {
-                const int em = p.moved ? p.moved[a] : -1;
-                const int e = em >= 0 ? em : p.topk_idx[a];
-                ef = e;
-                dest = e / e_per;
-                if (p.x_packed) {
-                    const int g = (em >= 0 ? p.nseg_round : 0) +
-                                  (p.slot_major ? lane * p.W + home : home);
-                    pk = p.pk_base[(size_t)e * p.nseg + g] + (r - p.offsets[e]);
-                }
-            }
-            if (p.expert_of)
-                p.expert_of[a] = ef;
-        }
-        if (p.stats) {
-            // distinct non-home destinations: count the lowest lane of each group
-            const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
-            const unsigned grp = __match_any_sync(0xffffffffu, key);
-            const unsigned first = __ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0);
-            pairs += __popc(first);
-        }
+        int r;
+        long long pk;
+        pairs += slot_targets(p, t, lane, lt_mask, r, pk);
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
         uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
         uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
@@ -548,6 +561,127 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
     }
     if (p.stats && lane == 0 && pairs)
         atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
+}
+
+// FP8 payload ([MoE 推理服务工程真相 2026, §6.3]: the token rows that cross the
+// all-to-all travel as FP8): one warp per token reads its bf16 row twice (the
+// second pass hits L1/L2), first for the largest magnitude, then to write e4m3
+// codes (row scaled by 2^-j, the row's power-of-two scale) to every kept slot's
+// sorted and packed row, with the scale 2^j beside each row. d % 16 == 0.
+__global__ void __launch_bounds__(256) scatter_rows_e4m3_kernel(ScatterArgs p)
+{
+    const int lane = threadIdx.x & 31;
+    const int n16 = p.d >> 4;  // 16-element chunks: two 16-byte loads, one 16-byte store
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    unsigned lt_mask;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
+    unsigned long long pairs = 0;
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
+        int r;
+        long long pk;
+        pairs += slot_targets(p, t, lane, lt_mask, r, pk);
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
+        // pass 1: largest magnitude of the row (bf16 bits with the sign cleared
+        // order like the magnitudes; a NaN marks the row non-finite)
+        uint32_t mx = 0;
+        for (int c = lane; c < 2 * n16; c += 32) {
+            const uint4 v = src[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mx = max(mx, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float amax = __uint_as_float(mx << 16);  // NaN bits sort above Inf
+        const int j = e4m3_scale_exp(amax);
+        const float inv = pow2f(-j), scale = pow2f(j);
+        for (int k = 0; k < p.K; ++k) {
+            const int rk = __shfl_sync(0xffffffffu, r, k);
+            const long long pkk = __shfl_sync(0xffffffffu, pk, k);
+            if (lane == 0 && rk >= 0) {
+                p.sorted_scale[rk] = scale;
+                if (pkk >= 0)
+                    p.packed_scale[pkk] = scale;
+            }
+        }
+        uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
+        uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
+        // pass 2: every lane runs every iteration (the shuffles read lanes 0..K-1)
+        for (int c0 = 0; c0 < n16; c0 += 32) {
+            const int c = c0 + lane;
+            uint4 q = make_uint4(0, 0, 0, 0);
+            if (c < n16) {
+                const uint4 a = src[2 * c], b = src[2 * c + 1];
+                const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = pack_e4m3x2(bf16_lo(w[2 * i]) * inv, bf16_hi(w[2 * i]) * inv);
+                    const uint32_t hi =
+                        pack_e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv);
+                    o[i] = lo | (hi << 16);
+                }
+                q = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            for (int k = 0; k < p.K; ++k) {
+                const int rk = __shfl_sync(0xffffffffu, r, k);
+                const long long pkk = __shfl_sync(0xffffffffu, pk, k);
+                if (rk < 0 || c >= n16)
+                    continue;
+                dst_s[(size_t)rk * n16 + c] = q;
+                if (pkk >= 0)
+                    dst_p[(size_t)pkk * n16 + c] = q;
+            }
+        }
+    }
+    if (p.stats && lane == 0 && pairs)
+        atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
+}
+
+// Row-wise e4m3 quantisation of a bf16 matrix (for the experts' W1 and W3): one
+// warp per row, the same two passes and rounding as the FP8 scatter. cols % 16 == 0.
+__global__ void __launch_bounds__(256)
+    quantize_rows_e4m3_kernel(const uint16_t *__restrict__ src, int64_t rows, int cols,
+                              uint8_t *__restrict__ codes, float *__restrict__ scale)
+{
+    const int lane = threadIdx.x & 31;
+    const int n16 = cols >> 4;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+         row += nwarps) {
+        const uint4 *s = reinterpret_cast<const uint4 *>(src + row * cols);
+        uint32_t mx = 0;
+        for (int c = lane; c < 2 * n16; c += 32) {
+            const uint4 v = s[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mx = max(mx, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const int j = e4m3_scale_exp(__uint_as_float(mx << 16));
+        const float inv = pow2f(-j);
+        if (lane == 0)
+            scale[row] = pow2f(j);
+        uint4 *d = reinterpret_cast<uint4 *>(codes + row * cols);
+        for (int c = lane; c < n16; c += 32) {
+            const uint4 a = s[2 * c], b = s[2 * c + 1];
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t lo = pack_e4m3x2(bf16_lo(w[2 * i]) * inv, bf16_hi(w[2 * i]) * inv);
+                const uint32_t hi =
+                    pack_e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv);
+                o[i] = lo | (hi << 16);
+            }
+            d[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
 }
 
 }  // namespace moe

@@ -23,6 +23,11 @@
 // N=256 MMA per K-step; the epilogue reads gate column c and up column 128+c
 // and writes h = silu(g) * u as bf16 (the next GEMM's operand). Mode 1 (down):
 // fp32 output straight from TMEM, so the combine sums unrounded expert outputs.
+// Mode 2 (gate/up on the FP8 payload, [MoE 推理服务工程真相 2026, §6.3]): as mode 0
+// with e4m3 A and B (tcgen05 kind::f8f6f4). A 128-byte swizzle atom then holds
+// 128 K elements instead of 64, so tiles, stages and descriptors keep their byte
+// layout; the epilogue multiplies the accumulator by the row's scale and the
+// output channel's scale (both powers of two, so the products are exact).
 //
 // Every mbarrier wait is bounded (globaltimer); a wait that runs out records
 // MOE_ERR_DEVICE_TIMEOUT, raises a CTA-wide abort flag, and every role drains
@@ -42,16 +47,22 @@ constexpr int B_HALF_BYTES = 128 * BK * 2;  // 16 KB per 128-row B box
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int THREADS = 192;
 
+// K elements in one 128-byte swizzle atom: 64 bf16 or 128 e4m3.
+__host__ __device__ constexpr int atom_k(int MODE) { return MODE == 2 ? 128 : 64; }
+
 struct Args {
     const int32_t *offsets;  // [E+1]
     int E;
     int n_tiles;         // N-slabs per expert
-    int k_blocks;        // K / 64
+    int k_blocks;        // K / atom_k(MODE)
     int b_rows;          // rows of one expert's B matrix (f for mode 0, d for mode 1)
     int rows_alloc;      // rows of the A buffer
     int select;          // which experts this launch takes: 0 all, 1 pair-tile experts, 2 the rest
-    void *out;           // mode 0: bf16 h [rows_alloc][ldo]; mode 1: fp32 y [rows_alloc][ldo]
+    void *out;           // modes 0, 2: bf16 h [rows_alloc][ldo]; mode 1: fp32 y [rows_alloc][ldo]
     int ldo;
+    const float *row_scale;  // mode 2: scale of each A row [rows_alloc]
+    const float *b_scale0;   // mode 2: scale of each W1 row [E * b_rows]
+    const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
     uint64_t timeout_ns;
 };
 
@@ -158,14 +169,37 @@ __host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N)
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
-__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate)
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), fp32 accumulate.
+__host__ __device__ constexpr uint32_t instr_desc_e4m3(int M, int N)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    return (1u << 4)                          // D format: f32
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+template <int MODE>
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N)
+{
+    return MODE == 2 ? instr_desc_e4m3(M, N) : instr_desc_bf16(M, N);
+}
+
+// One MMA of 32 bytes of K (16 bf16 or 32 e4m3 elements).
+template <int MODE>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    if constexpr (MODE == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
@@ -223,16 +257,74 @@ __device__ __forceinline__ void decode_tile(int tile, const int *tile_start, con
     m = local - n * mt;
 }
 
+// Gate/up epilogue of one thread: accumulator row `row` (TMEM lane of this thread),
+// gate columns [0, 128) and up columns [128, 256) of N-slab n of expert e ->
+// 128 bf16 values of h. Mode 2 first scales the accumulators by the row scale and
+// the W1 / W3 output-channel scales.
+template <int MODE>
+__device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr, int e, int n,
+                                                int row, bool store)
+{
+    uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.ldo;
+    uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
+    float sx = 1.0f;
+    const float *s1 = nullptr, *s3 = nullptr;
+    if constexpr (MODE == 2) {
+        sx = store ? args.row_scale[row] : 0.0f;
+        s1 = args.b_scale0 + (size_t)e * args.b_rows + n * 128;
+        s3 = args.b_scale1 + (size_t)e * args.b_rows + n * 128;
+    }
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 16) {
+        uint32_t g[16], u[16];
+        tmem_ld16(taddr + c, g);
+        tmem_ld16(taddr + 128 + c, u);
+        tmem_ld_wait();
+        if (store) {
+            float gf[16], uf[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                gf[j] = __uint_as_float(g[j]);
+                uf[j] = __uint_as_float(u[j]);
+            }
+            if constexpr (MODE == 2) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(s1 + c + j);
+                    const float4 b = *reinterpret_cast<const float4 *>(s3 + c + j);
+                    gf[j] *= sx * a.x;
+                    gf[j + 1] *= sx * a.y;
+                    gf[j + 2] *= sx * a.z;
+                    gf[j + 3] *= sx * a.w;
+                    uf[j] *= sx * b.x;
+                    uf[j + 1] *= sx * b.y;
+                    uf[j + 2] *= sx * b.z;
+                    uf[j + 3] *= sx * b.w;
+                }
+            }
+            uint32_t p[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                p[j] = pack_bf16x2(silu_mul(gf[2 * j], uf[2 * j]),
+                                   silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
+            dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
+            dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
+        }
+    }
+}
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Args args)
 {
-    static_assert(MODE == 0 ? BN == 256 : (BN == 128 || BN == 256), "tile shape");
+    static_assert(MODE != 1 ? BN == 256 : (BN == 128 || BN == 256), "tile shape");
+    constexpr bool GATE = MODE != 1;  // gate/up: W1 and W3 halves, SwiGLU epilogue
+    constexpr int KX = atom_k(MODE);
     constexpr int B_BYTES = BN * BK * 2;
     constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    constexpr uint32_t IDESC = instr_desc_bf16(BM, BN);
+    constexpr uint32_t IDESC = instr_desc<MODE>(BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -322,15 +414,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t a_dst = smem_base + stage * STAGE_BYTES;
                     const uint32_t b_dst = a_dst + A_BYTES;
                     mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-                    tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
-                    if (MODE == 0) {
+                    tma_load_2d(a_dst, &tmA, kb * KX, row0, full_bar(stage));
+                    if (GATE) {
                         const int brow = e * args.b_rows + n * 128;
-                        tma_load_2d(b_dst, &tmB0, kb * BK, brow, full_bar(stage));
-                        tma_load_2d(b_dst + B_HALF_BYTES, &tmB1, kb * BK, brow, full_bar(stage));
+                        tma_load_2d(b_dst, &tmB0, kb * KX, brow, full_bar(stage));
+                        tma_load_2d(b_dst + B_HALF_BYTES, &tmB1, kb * KX, brow, full_bar(stage));
                     } else {
 #pragma unroll
                         for (int h = 0; h < BN / 128; ++h)
-                            tma_load_2d(b_dst + h * B_HALF_BYTES, &tmB0, kb * BK,
+                            tma_load_2d(b_dst + h * B_HALF_BYTES, &tmB0, kb * KX,
                                         e * args.b_rows + n * BN + h * 128, full_bar(stage));
                     }
                     issued[stage] = true;
@@ -368,10 +460,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t a_addr = smem_base + stage * STAGE_BYTES;
                     const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k)
-                        tc_mma_bf16(d_tmem, smem_desc_sw128(a_addr + k * 32),
-                                    smem_desc_sw128(b_addr + k * 32), IDESC,
-                                    (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)  // four 32-byte K slices per atom
+                        tc_mma<MODE>(d_tmem, smem_desc_sw128(a_addr + k * 32),
+                                     smem_desc_sw128(b_addr + k * 32), IDESC,
+                                     (kb > 0 || k > 0) ? 1u : 0u);
                     tc_commit(empty_bar(stage));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -409,27 +501,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            if (MODE == 0) {
-                uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)(row0 + r) * args.ldo;
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
-#pragma unroll 1
-                for (int c = 0; c < 128; c += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld16(taddr + c, g);
-                    tmem_ld16(taddr + 128 + c, u);
-                    tmem_ld_wait();
-                    if (r < valid) {
-                        uint32_t p[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            p[j] = pack_bf16x2(
-                                silu_mul(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j])),
-                                silu_mul(__uint_as_float(g[2 * j + 1]),
-                                         __uint_as_float(u[2 * j + 1])));
-                        dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
-                        dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
-                    }
-                }
+            if (GATE) {
+                swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
             } else {
                 // fp32 output: the down projection is not rounded before the combine
                 float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
@@ -528,14 +601,22 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr)
                  : "memory");
 }
 
-__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                                 uint32_t idesc, uint32_t accumulate)
+template <int MODE>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    if constexpr (MODE == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr)
@@ -553,7 +634,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 {
     constexpr int BMP = 256;  // rows per pair tile
     constexpr int BN = 256;
-    constexpr uint32_t IDESC = instr_desc_bf16(BMP, BN);
+    constexpr bool GATE = MODE != 1;
+    constexpr int KX = atom_k(MODE);
+    constexpr uint32_t IDESC = instr_desc<MODE>(BMP, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -632,13 +715,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int st = 0; st < STAGES2; ++st)
                 issued[st] = false;
             bool ok = true;
-            const CUtensorMap *bmap = (MODE == 0 && rank == 1) ? &tmB1 : &tmB0;
+            const CUtensorMap *bmap = (GATE && rank == 1) ? &tmB1 : &tmB0;
             for (int tile = pair; tile < total && ok; tile += npairs) {
                 int e, n, m;
                 decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
                 const int row0 = args.offsets[e] + m * BMP + (int)rank * 128;
-                const int brow = MODE == 0 ? e * args.b_rows + n * 128
-                                           : e * args.b_rows + n * BN + (int)rank * 128;
+                const int brow = GATE ? e * args.b_rows + n * 128
+                                      : e * args.b_rows + n * BN + (int)rank * 128;
                 for (int kb = 0; kb < args.k_blocks / KA2; ++kb) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, args.timeout_ns)) {
                         ok = false;
@@ -650,7 +733,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE2_BYTES);
 #pragma unroll
                     for (int at = 0; at < KA2; ++at) {
-                        const int kx = (kb * KA2 + at) * BK;
+                        const int kx = (kb * KA2 + at) * KX;
                         tma_load_2d_pair(a_dst + at * A_BYTES, &tmA, kx, row0, full_leader);
                         tma_load_2d_pair(a_dst + KA2 * A_BYTES + at * B_HALF_BYTES, bmap, kx, brow,
                                          full_leader);
@@ -691,11 +774,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t a_addr = smem_base + stage * STAGE2_BYTES;
                     const uint32_t b_addr = a_addr + KA2 * A_BYTES;
 #pragma unroll
-                    for (int k = 0; k < KA2 * BK / 16; ++k) {
+                    for (int k = 0; k < KA2 * 4; ++k) {  // four 32-byte K slices per atom
                         const uint32_t off = (uint32_t)((k / 4) * A_BYTES + (k % 4) * 32);
-                        tc_mma_bf16_pair(d_tmem, smem_desc_sw128(a_addr + off),
-                                         smem_desc_sw128(b_addr + off), IDESC,
-                                         (kb > 0 || k > 0) ? 1u : 0u);
+                        tc_mma_pair<MODE>(d_tmem, smem_desc_sw128(a_addr + off),
+                                          smem_desc_sw128(b_addr + off), IDESC,
+                                          (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(map_to_rank(empty_bar(stage), 0));
                     tc_commit_pair(map_to_rank(empty_bar(stage), 1));
@@ -735,27 +818,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-            if (MODE == 0) {
-                uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)(row0 + r) * args.ldo;
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
-#pragma unroll 1
-                for (int c = 0; c < 128; c += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld16(taddr + c, g);
-                    tmem_ld16(taddr + 128 + c, u);
-                    tmem_ld_wait();
-                    if (r < valid) {
-                        uint32_t p[8];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            p[j] = pack_bf16x2(
-                                silu_mul(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j])),
-                                silu_mul(__uint_as_float(g[2 * j + 1]),
-                                         __uint_as_float(u[2 * j + 1])));
-                        dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
-                        dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
-                    }
-                }
+            if (GATE) {
+                swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
             } else {
                 float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
                 uint4 *dst = reinterpret_cast<uint4 *>(frow + n * BN);

@@ -133,8 +133,8 @@ ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
 
 // moe_layer: every intermediate, after the scratch.
 struct LayerLayout {
-    size_t topk_idx, topk_w, counts, kept, offsets, row_of, assign, x_sorted, x_packed, h, y,
-        nonfinite, total;
+    size_t topk_idx, topk_w, counts, kept, offsets, row_of, assign, x_sorted, x_packed,
+        sorted_scale, packed_scale, h, y, nonfinite, total;
 };
 
 LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
@@ -160,6 +160,10 @@ LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
     o = align_up(o + RA * s->d * 2);
     L.x_packed = o;
     o = align_up(o + RA * s->d * 2);
+    L.sorted_scale = o;  // FP8 payload only
+    o = align_up(o + RA * 4);
+    L.packed_scale = o;
+    o = align_up(o + RA * 4);
     L.h = o;
     o = align_up(o + RA * (size_t)s->f * 2);
     L.y = o;
@@ -292,11 +296,20 @@ void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const in
 }
 
 // logits: needed when g.rounds == 2 (re-routing); moved: N*K int32 scratch then.
+// Row payload of the scatter: bf16 rows, or e4m3 rows with a scale per row.
+struct Payload {
+    void *x_sorted;
+    void *x_packed;       // nullable
+    bool e4m3;
+    float *sorted_scale;  // e4m3 only
+    float *packed_scale;  // e4m3 with x_packed only
+};
+
 moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x,
                            const float *logits, const int32_t *topk_idx, int32_t *counts,
                            int32_t *kept, int32_t *offsets, int32_t *row_of,
-                           int32_t *assign_of_row, int32_t *expert_of, uint16_t *x_sorted,
-                           uint16_t *x_packed, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
+                           int32_t *assign_of_row, int32_t *expert_of, const Payload &pay,
+                           int64_t *D, int64_t *pk_off, moe_stats_t *stats,
                            int32_t *blk, int64_t *pk_base, int32_t *cum, int32_t *moved,
                            cudaStream_t st)
 {
@@ -338,10 +351,15 @@ moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16
     ca.nseg = g.nseg;
     ca.nseg_round = g.nseg_round;
     ca.expert_of = expert_of;
-    ca.x_sorted = x_sorted;
-    ca.x_packed = x_packed;
+    ca.x_sorted = pay.x_sorted;
+    ca.x_packed = pay.x_packed;
+    ca.sorted_scale = pay.sorted_scale;
+    ca.packed_scale = pay.packed_scale;
     ca.stats = stats;
-    scatter_rows_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
+    if (pay.e4m3)
+        scatter_rows_e4m3_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
+    else
+        scatter_rows_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
     return launch_status();
 }
 
@@ -362,18 +380,21 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 2-D bf16 tensor [rows][inner], box 128 rows x 64 elements, 128-byte swizzle.
-bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows)
+// 2-D tensor [rows][inner] of bf16 (or e4m3 bytes), box 128 rows x one 128-byte swizzle
+// atom (64 bf16 or 128 e4m3 elements), 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, bool e4m3 = false)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
+    const uint64_t esize = e4m3 ? 1 : 2;
     cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {(cuuint32_t)gg::BK, 128};
+    cuuint64_t strides[1] = {inner * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 128};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -466,7 +487,7 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
     if (!make_tmap(&tA, a, d, (uint64_t)a_rows) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
         !make_tmap(&tW3, w3, d, (uint64_t)E * f))
         return MOE_ERR_CUDA;
-    gg::Args args;
+    gg::Args args = {};
     args.offsets = offsets;
     args.E = E;
     args.n_tiles = f / 128;
@@ -493,7 +514,7 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     CUtensorMap tA, tW2;
     if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
         return MOE_ERR_CUDA;
-    gg::Args args;
+    gg::Args args = {};
     args.offsets = offsets;
     args.E = E;
     args.k_blocks = f / gg::BK;
@@ -516,6 +537,43 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     }
     args.n_tiles = d / 128;
     return launch_gemm<1, 128>(tA, tW2, tW2, args, st);
+}
+
+// Gate/up on the FP8 payload: e4m3 rows of x (scale per row) and e4m3 rows of W1, W3
+// (scale per output channel). The pair kernel's stages hold two atoms, so it needs
+// d % 256 == 0; otherwise every expert takes the single-CTA kernel.
+moe_status_t gemm_up_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const uint8_t *a,
+                          const float *a_scale, const int32_t *offsets, const uint8_t *w1,
+                          const float *s1, const uint8_t *w3, const float *s3, uint16_t *h,
+                          cudaStream_t st)
+{
+    CUtensorMap tA, tW1, tW3;
+    if (!make_tmap(&tA, a, d, (uint64_t)a_rows, true) ||
+        !make_tmap(&tW1, w1, d, (uint64_t)E * f, true) ||
+        !make_tmap(&tW3, w3, d, (uint64_t)E * f, true))
+        return MOE_ERR_CUDA;
+    gg::Args args = {};
+    args.offsets = offsets;
+    args.E = E;
+    args.n_tiles = f / 128;
+    args.k_blocks = d / gg::atom_k(2);
+    args.b_rows = f;
+    args.rows_alloc = (int)a_rows;
+    args.out = h;
+    args.ldo = f;
+    args.row_scale = a_scale;
+    args.b_scale0 = s1;
+    args.b_scale1 = s3;
+    args.timeout_ns = kWaitTimeoutNs;
+    args.select = 0;
+    if (pair && args.k_blocks % gg::KA2 == 0) {
+        args.select = 1;
+        moe_status_t rc = launch_gemm_pair<2>(tA, tW1, tW3, args, st);
+        if (rc != MOE_OK)
+            return rc;
+        args.select = 2;
+    }
+    return launch_gemm<2, 256>(tA, tW1, tW3, args, st);
 }
 
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
@@ -661,19 +719,26 @@ namespace {
 moe_status_t dispatch_entry(const moe_shape_t *shape, const uint16_t *x, const float *logits,
                             const int32_t *topk_idx, int32_t *counts, int32_t *kept,
                             int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
-                            int32_t *expert_of, uint16_t *x_sorted, uint16_t *x_packed,
-                            int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
-                            void *ws, size_t ws_bytes, moe_stream_t stream)
+                            int32_t *expert_of, const Payload &pay, int64_t *rank_matrix,
+                            int64_t *packed_offsets, moe_stats_t *stats, void *ws,
+                            size_t ws_bytes, moe_stream_t stream)
 {
     Geometry g;
     moe_status_t rc = check_shape(shape, false, &g);
     if (rc != MOE_OK)
         return rc;
-    if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)
+    if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row ||
+        !pay.x_sorted)
         return MOE_ERR_INVALID_ARG;
     if ((g.rounds > 1) != (logits != nullptr))
         return MOE_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(x_sorted) || (x_packed && !aligned16(x_packed)) ||
+    if (pay.e4m3 && (shape->d % 16 != 0 || !pay.sorted_scale ||
+                     (pay.x_packed != nullptr) != (pay.packed_scale != nullptr)))
+        return pay.e4m3 && shape->d % 16 != 0 ? MOE_ERR_UNSUPPORTED_SHAPE : MOE_ERR_INVALID_ARG;
+    if (pay.e4m3 && (!aligned4(pay.sorted_scale) ||
+                     (pay.packed_scale && !aligned4(pay.packed_scale))))
+        return MOE_ERR_MISALIGNED;
+    if (!aligned16(x) || !aligned16(pay.x_sorted) || (pay.x_packed && !aligned16(pay.x_packed)) ||
         !aligned4(topk_idx) || !aligned4(counts) || !aligned4(kept) || !aligned4(offsets) ||
         !aligned4(row_of) || !aligned4(assign_of_row) || (logits && !aligned4(logits)) ||
         (expert_of && !aligned4(expert_of)) ||
@@ -690,7 +755,7 @@ moe_status_t dispatch_entry(const moe_shape_t *shape, const uint16_t *x, const f
     int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
     int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
     return dispatch_impl(shape, g, x, logits, topk_idx, counts, kept, offsets, row_of,
-                         assign_of_row, expert_of, x_sorted, x_packed, D, pk, stats,
+                         assign_of_row, expert_of, pay, D, pk, stats,
                          reinterpret_cast<int32_t *>(w + L.blk),
                          reinterpret_cast<int64_t *>(w + L.pk_base),
                          reinterpret_cast<int32_t *>(w + L.cum),
@@ -711,8 +776,8 @@ moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_id
     if (shape && (shape->flags & MOE_FLAG_REROUTE))
         return MOE_ERR_INVALID_ARG;
     return dispatch_entry(shape, x, nullptr, topk_idx, counts, kept, offsets, row_of,
-                          assign_of_row, nullptr, x_sorted, x_packed, rank_matrix,
-                          packed_offsets, stats, ws, ws_bytes, stream);
+                          assign_of_row, nullptr, Payload{x_sorted, x_packed, false, nullptr, nullptr},
+                          rank_matrix, packed_offsets, stats, ws, ws_bytes, stream);
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -726,8 +791,63 @@ moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, const float *l
     if (!shape || !(shape->flags & MOE_FLAG_REROUTE) || !logits)
         return MOE_ERR_INVALID_ARG;
     return dispatch_entry(shape, x, logits, topk_idx, counts, kept, offsets, row_of,
-                          assign_of_row, expert_of, x_sorted, x_packed, rank_matrix,
+                          assign_of_row, expert_of,
+                          Payload{x_sorted, x_packed, false, nullptr, nullptr}, rank_matrix,
                           packed_offsets, stats, ws, ws_bytes, stream);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_dispatch_fp8(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx,
+                 int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of,
+                 int32_t *assign_of_row, uint8_t *x_sorted, float *sorted_scale,
+                 uint8_t *x_packed, float *packed_scale, int64_t *rank_matrix,
+                 int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
+                 moe_stream_t stream)
+{
+    if (shape && (shape->flags & MOE_FLAG_REROUTE))
+        return MOE_ERR_INVALID_ARG;
+    return dispatch_entry(shape, x, nullptr, topk_idx, counts, kept, offsets, row_of,
+                          assign_of_row, nullptr,
+                          Payload{x_sorted, x_packed, true, sorted_scale, packed_scale},
+                          rank_matrix, packed_offsets, stats, ws, ws_bytes, stream);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int32_t cols, uint8_t *codes,
+                       float *scale, moe_stream_t stream)
+{
+    if (rows < 0 || cols < 16 || !src || !codes || !scale)
+        return MOE_ERR_INVALID_ARG;
+    if (cols % 16 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(src) || !aligned16(codes) || !aligned4(scale))
+        return MOE_ERR_MISALIGNED;
+    if (rows == 0)
+        return MOE_OK;
+    const int64_t blocks64 = (rows + 7) / 8;
+    const int blocks = (int)(blocks64 < 148 * 64 ? blocks64 : 148 * 64);
+    quantize_rows_e4m3_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        src, rows, cols, codes, scale);
+    return launch_status();
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted, const float *sorted_scale,
+                  const int32_t *offsets, const uint8_t *w1q, const float *w1_scale,
+                  const uint8_t *w3q, const float *w3_scale, uint16_t *h, moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!x_sorted || !sorted_scale || !offsets || !w1q || !w1_scale || !w3q || !w3_scale || !h)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_sorted) || !aligned16(w1q) || !aligned16(w3q) || !aligned16(w1_scale) ||
+        !aligned16(w3_scale) || !aligned16(h) || !aligned4(offsets) || !aligned4(sorted_scale))
+        return MOE_ERR_MISALIGNED;
+    return gemm_up_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
+                        x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q, w3_scale, h,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -797,6 +917,85 @@ moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+
+// Gate/up weights of a layer: bf16 W1, W3, or their e4m3 rows with per-row scales (then
+// the dispatch writes the FP8 payload).
+struct UpWeights {
+    const uint16_t *w1, *w3;
+    const uint8_t *w1q, *w3q;
+    const float *s1, *s3;
+    bool e4m3() const { return w1q != nullptr; }
+};
+
+// The layer: route -> dispatch -> gate/up -> down -> (shared MLP) -> combine, every
+// intermediate in the workspace. Arguments validated by the caller; f_shared == 0: no
+// shared MLP.
+moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16_t *x,
+                       const float *w_router, const float *bias, const UpWeights &up,
+                       const uint16_t *w2, int32_t f_shared, const uint16_t *ws1,
+                       const uint16_t *ws3, const uint16_t *ws2, const uint16_t *residual,
+                       void *out, int32_t *topk_idx_out, moe_stats_t *stats, char *w,
+                       size_t ws_need, cudaStream_t st)
+{
+    const ScratchLayout S = scratch_layout(shape, g);
+    const LayerLayout L = layer_layout(shape, g, S.total);
+    int32_t *topk_idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(w + L.topk_idx);
+    float *topk_w = reinterpret_cast<float *>(w + L.topk_w);
+    unsigned long long *nonfinite = nullptr;
+    if (stats) {
+        nonfinite = reinterpret_cast<unsigned long long *>(&stats->nonfinite_tokens);
+        if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    moe_status_t rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
+                                 reinterpret_cast<float *>(w + S.logits), nonfinite, st);
+    if (rc != MOE_OK)
+        return rc;
+    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+    int32_t *row_of = reinterpret_cast<int32_t *>(w + L.row_of);
+    uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
+    float *y = reinterpret_cast<float *>(w + L.y);
+    Payload pay{w + L.x_sorted, w + L.x_packed, up.e4m3(),
+                reinterpret_cast<float *>(w + L.sorted_scale),
+                reinterpret_cast<float *>(w + L.packed_scale)};
+    rc = dispatch_impl(shape, g, x, reinterpret_cast<const float *>(w + S.logits), topk_idx,
+                       reinterpret_cast<int32_t *>(w + L.counts),
+                       reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
+                       reinterpret_cast<int32_t *>(w + L.assign), nullptr, pay,
+                       reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
+                       stats, reinterpret_cast<int32_t *>(w + S.blk),
+                       reinterpret_cast<int64_t *>(w + S.pk_base),
+                       reinterpret_cast<int32_t *>(w + S.cum),
+                       reinterpret_cast<int32_t *>(w + S.moved), st);
+    if (rc != MOE_OK)
+        return rc;
+    if (up.e4m3())
+        rc = gemm_up_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
+                          static_cast<const uint8_t *>(pay.x_sorted), pay.sorted_scale, offsets,
+                          up.w1q, up.s1, up.w3q, up.s3, h, st);
+    else
+        rc = expert_up_impl(shape, g, static_cast<const uint16_t *>(pay.x_sorted), offsets, up.w1,
+                            up.w3, h, st);
+    if (rc != MOE_OK)
+        return rc;
+    rc = expert_down_impl(shape, g, h, offsets, w2, y, st);
+    if (rc != MOE_OK)
+        return rc;
+    float *y_s = nullptr;
+    if (f_shared > 0) {
+        uint16_t *h_s = reinterpret_cast<uint16_t *>(w + L.total);
+        y_s = reinterpret_cast<float *>(w + L.total + align_up((size_t)shape->N * f_shared * 2));
+        int32_t *off2 = reinterpret_cast<int32_t *>(w + ws_need - kAlign);
+        rc = shared_expert_impl(shape, f_shared, x, ws1, ws3, ws2, h_s, y_s, off2, st);
+        if (rc != MOE_OK)
+            return rc;
+    }
+    return combine_impl(shape, y, row_of, topk_w, y_s, residual, out, st);
+}
+
+}  // namespace
+
 __attribute__((visibility("default"))) moe_status_t
 moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, const float *bias,
           const uint16_t *w1, const uint16_t *w3, const uint16_t *w2, const uint16_t *residual,
@@ -814,47 +1013,44 @@ moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
         (residual && !aligned16(residual)) || (topk_idx_out && !aligned4(topk_idx_out)) ||
         (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
         return MOE_ERR_MISALIGNED;
-    const ScratchLayout S = scratch_layout(shape, g);
-    const LayerLayout L = layer_layout(shape, g, S.total);
-    if (!ws || ws_bytes < L.total)
+    const size_t need = moe_layer_workspace_size(shape);
+    if (!ws || ws_bytes < need)
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(ws))
         return MOE_ERR_MISALIGNED;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    char *w = static_cast<char *>(ws);
-    int32_t *topk_idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(w + L.topk_idx);
-    float *topk_w = reinterpret_cast<float *>(w + L.topk_w);
-    unsigned long long *nonfinite = nullptr;
-    if (stats) {
-        nonfinite = reinterpret_cast<unsigned long long *>(&stats->nonfinite_tokens);
-        if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
-            return MOE_ERR_CUDA;
-    }
-    rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
-                    reinterpret_cast<float *>(w + S.logits), nonfinite, st);
+    return layer_run(shape, g, x, w_router, bias, UpWeights{w1, w3, nullptr, nullptr, nullptr, nullptr},
+                     w2, 0, nullptr, nullptr, nullptr, residual, out, topk_idx_out, stats,
+                     static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
+              const float *bias, const uint8_t *w1q, const float *w1_scale, const uint8_t *w3q,
+              const float *w3_scale, const uint16_t *w2, const uint16_t *residual, void *out,
+              int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
+              moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
-    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
-    int32_t *row_of = reinterpret_cast<int32_t *>(w + L.row_of);
-    uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
-    uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
-    float *y = reinterpret_cast<float *>(w + L.y);
-    rc = dispatch_impl(shape, g, x, reinterpret_cast<const float *>(w + S.logits), topk_idx,
-                       reinterpret_cast<int32_t *>(w + L.counts),
-                       reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
-                       reinterpret_cast<int32_t *>(w + L.assign), nullptr, x_sorted,
-                       reinterpret_cast<uint16_t *>(w + L.x_packed),
-                       reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
-                       stats, reinterpret_cast<int32_t *>(w + S.blk),
-                       reinterpret_cast<int64_t *>(w + S.pk_base),
-                       reinterpret_cast<int32_t *>(w + S.cum),
-                       reinterpret_cast<int32_t *>(w + S.moved), st);
-    if (rc != MOE_OK)
-        return rc;
-    rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
-    if (rc != MOE_OK)
-        return rc;
-    return combine_impl(shape, y, row_of, topk_w, nullptr, residual, out, st);
+    if (!x || !w_router || !w1q || !w1_scale || !w3q || !w3_scale || !w2 || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1q) ||
+        !aligned16(w3q) || !aligned16(w1_scale) || !aligned16(w3_scale) || !aligned16(w2) ||
+        !aligned16(out) || (residual && !aligned16(residual)) ||
+        (topk_idx_out && !aligned4(topk_idx_out)) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const size_t need = moe_layer_workspace_size(shape);
+    if (!ws || ws_bytes < need)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    return layer_run(shape, g, x, w_router, bias,
+                     UpWeights{nullptr, nullptr, w1q, w3q, w1_scale, w3_scale}, w2, 0, nullptr,
+                     nullptr, nullptr, residual, out, topk_idx_out, stats,
+                     static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -916,49 +1112,9 @@ moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(ws))
         return MOE_ERR_MISALIGNED;
-    const ScratchLayout S = scratch_layout(shape, g);
-    const LayerLayout L = layer_layout(shape, g, S.total);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    char *w = static_cast<char *>(ws);
-    uint16_t *h_s = reinterpret_cast<uint16_t *>(w + L.total);
-    float *y_s = reinterpret_cast<float *>(w + L.total + align_up((size_t)shape->N * f_shared * 2));
-    int32_t *off2 = reinterpret_cast<int32_t *>(w + need - kAlign);
-    int32_t *topk_idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t *>(w + L.topk_idx);
-    float *topk_w = reinterpret_cast<float *>(w + L.topk_w);
-    unsigned long long *nonfinite = nullptr;
-    if (stats) {
-        nonfinite = reinterpret_cast<unsigned long long *>(&stats->nonfinite_tokens);
-        if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
-            return MOE_ERR_CUDA;
-    }
-    rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
-                    reinterpret_cast<float *>(w + S.logits), nonfinite, st);
-    if (rc != MOE_OK)
-        return rc;
-    int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
-    int32_t *row_of = reinterpret_cast<int32_t *>(w + L.row_of);
-    uint16_t *x_sorted = reinterpret_cast<uint16_t *>(w + L.x_sorted);
-    uint16_t *h = reinterpret_cast<uint16_t *>(w + L.h);
-    float *y = reinterpret_cast<float *>(w + L.y);
-    rc = dispatch_impl(shape, g, x, reinterpret_cast<const float *>(w + S.logits), topk_idx,
-                       reinterpret_cast<int32_t *>(w + L.counts),
-                       reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
-                       reinterpret_cast<int32_t *>(w + L.assign), nullptr, x_sorted,
-                       reinterpret_cast<uint16_t *>(w + L.x_packed),
-                       reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
-                       stats, reinterpret_cast<int32_t *>(w + S.blk),
-                       reinterpret_cast<int64_t *>(w + S.pk_base),
-                       reinterpret_cast<int32_t *>(w + S.cum),
-                       reinterpret_cast<int32_t *>(w + S.moved), st);
-    if (rc != MOE_OK)
-        return rc;
-    rc = expert_gemm_impl(shape, g, x_sorted, offsets, w1, w3, w2, h, y, st);
-    if (rc != MOE_OK)
-        return rc;
-    rc = shared_expert_impl(shape, f_shared, x, ws1, ws3, ws2, h_s, y_s, off2, st);
-    if (rc != MOE_OK)
-        return rc;
-    return combine_impl(shape, y, row_of, topk_w, y_s, residual, out, st);
+    return layer_run(shape, g, x, w_router, bias, UpWeights{w1, w3, nullptr, nullptr, nullptr, nullptr},
+                     w2, f_shared, ws1, ws3, ws2, residual, out, topk_idx_out, stats,
+                     static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -1141,7 +1297,8 @@ moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *
     int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
     int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
     return dispatch_impl(shape, g, x, nullptr, topk_idx, counts, kept, offsets, row_of,
-                         assign_of_row, nullptr, x_sorted, x_packed, D, pk, stats,
+                         assign_of_row, nullptr,
+                         Payload{x_sorted, x_packed, false, nullptr, nullptr}, D, pk, stats,
                          reinterpret_cast<int32_t *>(w + L.blk),
                          reinterpret_cast<int64_t *>(w + L.pk_base),
                          reinterpret_cast<int32_t *>(w + L.cum), nullptr,

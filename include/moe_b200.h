@@ -260,6 +260,43 @@ moe_status_t moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted,
 moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
                              const uint16_t *w2, float *y, moe_stream_t stream);
 
+/* ---- FP8 payload ("MoE 推理服务工程真相 2026", §6.3: send the token data of the all-to-all
+ * as FP8 instead of BF16, half the bytes, at the cost of quantisation noise).
+ * Format e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, largest finite 448, no
+ * infinities). Readings: one power-of-two scale per row, the smallest 2^j (j in [-126, 127])
+ * with max|row| * 2^-j <= 448 (j = 0 for a zero or non-finite row); each element is
+ * x * 2^-j rounded to nearest-even e4m3, saturating; value = code * 2^j. Routing stays on
+ * the bf16 x; the experts' gate/up projections consume the e4m3 rows of x together with
+ * e4m3 rows of W1 and W3 (one scale per output channel) on tcgen05 kind::f8f6f4; h, the
+ * down projection and the combine are as in the bf16 path. */
+
+/* Row-wise e4m3 quantisation of a bf16 matrix src [rows][cols] (DEVICE): codes [rows][cols]
+ * uint8 and scale [rows] fp32 (DEVICE, caller-owned). For the experts' W1 and W3 pass
+ * rows = E*f, cols = d. cols % 16 == 0; src, codes 16-byte aligned. */
+moe_status_t moe_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int32_t cols,
+                                    uint8_t *codes, float *scale, moe_stream_t stream);
+
+/* moe_dispatch with the FP8 payload: x_sorted and x_packed hold e4m3 rows ([rows_alloc][d]
+ * uint8) and sorted_scale / packed_scale [rows_alloc] fp32 the scale of each row (packed_scale
+ * is required with x_packed and ignored without it). The bookkeeping outputs are identical to
+ * moe_dispatch's. d % 16 == 0. MOE_FLAG_REROUTE is refused (no logits here; moe_layer_fp8
+ * takes it). Same workspace as moe_dispatch. */
+moe_status_t moe_dispatch_fp8(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_idx,
+                              int32_t *counts, int32_t *kept, int32_t *offsets, int32_t *row_of,
+                              int32_t *assign_of_row, uint8_t *x_sorted, float *sorted_scale,
+                              uint8_t *x_packed, float *packed_scale, int64_t *rank_matrix,
+                              int64_t *packed_offsets, moe_stats_t *stats, void *ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/* Gate/up GEMM on the FP8 payload: h = silu(sx * s1 * (xq W1q^T)) * (sx * s3 * (xq W3q^T)),
+ * bf16 h [rows_alloc][f]; x_sorted e4m3 [rows_alloc][d] with sorted_scale per row (from
+ * moe_dispatch_fp8); w1q, w3q e4m3 [E][f][d] with w1_scale, w3_scale [E][f] (from
+ * moe_quantize_rows_e4m3; 16-byte aligned). d % 128 == 0, f % 128 == 0. */
+moe_status_t moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted,
+                               const float *sorted_scale, const int32_t *offsets,
+                               const uint8_t *w1q, const float *w1_scale, const uint8_t *w3q,
+                               const float *w3_scale, uint16_t *h, moe_stream_t stream);
+
 /* Weighted combine back to token order.
  * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (weighted merge into the
  *  original token order, then on to the next layer); MoE 推理服务工程真相 2026, §2.2 (a
@@ -305,6 +342,16 @@ moe_status_t moe_layer(const moe_shape_t *shape, const uint16_t *x, const float 
                        const uint16_t *w2, const uint16_t *residual, void *out,
                        int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
+
+/* moe_layer with the FP8 payload: the dispatch writes e4m3 rows and the gate/up GEMM runs on
+ * them with the e4m3 weights w1q, w3q [E][f][d] and their scales w1_scale, w3_scale [E][f]
+ * (moe_quantize_rows_e4m3). W2 stays bf16. Every flag of moe_layer applies; the workspace is
+ * moe_layer_workspace_size(shape). */
+moe_status_t moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
+                           const float *bias, const uint8_t *w1q, const float *w1_scale,
+                           const uint8_t *w3q, const float *w3_scale, const uint16_t *w2,
+                           const uint16_t *residual, void *out, int32_t *topk_idx_out,
+                           moe_stats_t *stats, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Inter-layer expert affinity counts, accumulated into counts [E][E] int64:
  * for every token t, i in topk_j[t], p in topk_j1[t]: counts[i][p] += 1.

@@ -54,6 +54,7 @@ class Workload:
     shared_f: int = 0        # width of the shared dense MLP (Residual-MoE); 0 = none
     slot_major: bool = False  # drop priority: first choices before second choices
     reroute: bool = False     # move overflowed assignments to the next-best non-full expert
+    fp8: bool = False         # e4m3 dispatch payload and gate/up GEMM
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -76,6 +77,11 @@ WORKLOADS = {
     # the same with overflowed assignments re-routed to the next-best non-full expert
     "e128_skew_reroute": Workload("e128_skew_reroute", N=8192, d=2048, f=768, E=128, K=8, W=8,
                                   cf=1.25, s=1.1, reroute=True),
+    # the FP8 payload (e4m3 rows, e4m3 gate/up GEMM) on the Mixtral-shaped and 128-expert layers
+    "mixtral_prefill_fp8": Workload("mixtral_prefill_fp8", N=4096, d=4096, f=14336, E=8, K=2,
+                                    W=8, router="uniform", fp8=True),
+    "e128_skew_fp8": Workload("e128_skew_fp8", N=8192, d=2048, f=768, E=128, K=8, W=8, cf=1.25,
+                              s=1.1, fp8=True),
     # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
     # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
     "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,
