@@ -73,6 +73,10 @@ def _load():
         lib.orc_e4m3_scale_exponent.restype = _i64
         lib.orc_quantize_rows_e4m3.argtypes = [_i64, _i64, _p, _p, _p]
         lib.orc_quantize_rows_e4m3.restype = None
+        lib.orc_round_bf16.argtypes = [_i64, _p, _p]
+        lib.orc_round_bf16.restype = None
+        lib.orc_down_rows.argtypes = [_i64, _p, _i64, _i64, _p, _p, _p]
+        lib.orc_down_rows.restype = None
         _lib = lib
     return _lib
 
@@ -338,32 +342,63 @@ def dequantize_rows_bf16(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return (bits >> 16).astype(np.uint16)
 
 
+def round_bf16(v: np.ndarray) -> np.ndarray:
+    """Nearest bf16 of each float64 value (ties to even), as uint16 bits."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, np.uint16)
+    _load().orc_round_bf16(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def down_rows(row_expert: np.ndarray, h_u16: np.ndarray, w2) -> np.ndarray:
+    """y = W2[e] h for bf16 rows h [n][f] (uint16 bits), fp64."""
+    row_expert = np.ascontiguousarray(row_expert, dtype=np.int32)
+    h = np.ascontiguousarray(h_u16, dtype=np.uint16)
+    c = as_u16(w2)
+    n, f = h.shape
+    d = c.shape[1]
+    y = np.empty((n, d), np.float64)
+    _load().orc_down_rows(n, _ptr(row_expert), d, f, _ptr(h), _ptr(c), _ptr(y))
+    return y
+
+
 def fp8_operands(inp: dict) -> dict:
-    """The e4m3 operands of the FP8 gate/up GEMM: x rows per token, W1 and W3 rows
-    per output channel, each with its power-of-two scale, and their exact bf16
-    dequantisations."""
+    """The e4m3 operands of the FP8 expert GEMMs: x rows per token, W1, W3 and W2 rows per
+    output channel, each with its power-of-two scale, and their exact bf16 dequantisations."""
     xq, sx = quantize_rows_e4m3(inp["x"])
     w1q, s1 = quantize_rows_e4m3(inp["w1"])
     w3q, s3 = quantize_rows_e4m3(inp["w3"])
-    return dict(xq=xq, sx=sx, w1q=w1q, s1=s1, w3q=w3q, s3=s3,
+    w2q, s2 = quantize_rows_e4m3(inp["w2"])
+    return dict(xq=xq, sx=sx, w1q=w1q, s1=s1, w3q=w3q, s3=s3, w2q=w2q, s2=s2,
                 x_deq=dequantize_rows_bf16(xq, sx), w1_deq=dequantize_rows_bf16(w1q, s1),
-                w3_deq=dequantize_rows_bf16(w3q, s3))
+                w3_deq=dequantize_rows_bf16(w3q, s3), w2_deq=dequantize_rows_bf16(w2q, s2))
+
+
+def fp8_down(h: np.ndarray, row_expert: np.ndarray, q: dict) -> dict:
+    """The FP8 down projection: h rounded to bf16 (the precision it is stored in), its rows
+    quantised to e4m3 with a power-of-two scale each, times the e4m3 W2 rows."""
+    hb = round_bf16(h)
+    hq, hs = quantize_rows_e4m3(hb)
+    y = down_rows(row_expert, dequantize_rows_bf16(hq, hs), q["w2_deq"])
+    return dict(h_bf16=hb, hq=hq, hs=hs, y=y)
 
 
 def layer_fp8(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0,
               reroute: bool = False) -> dict:
-    """The layer with the FP8 payload: routing on the bf16 x; the experts' gate/up
-    projections on e4m3 rows of x (one scale per token) and e4m3 rows of W1, W3 (one
-    scale per output channel), i.e. on their dequantised values; the down projection
-    and the combine as in ``layer``."""
+    """The layer with the FP8 payload and FP8 expert GEMMs: routing on the bf16 x; the
+    gate/up projections on e4m3 rows of x (one scale per token) and e4m3 rows of W1, W3
+    (one scale per output channel); h rounded to bf16, then its rows quantised to e4m3
+    for the down projection with e4m3 rows of W2; the combine as in ``layer``."""
     q = fp8_operands(inp)
     r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order, reroute)
     N = r["logits"].shape[0]
     aor = r["assign_of_row"]
     row_token = (aor // K).astype(np.int32)
     row_expert = r["expert_of"][aor].astype(np.int32)
-    h, y = expert_rows(row_token, row_expert, q["x_deq"], q["w1_deq"], q["w3_deq"], inp["w2"],
-                       want_h)
+    h, _ = expert_rows(row_token, row_expert, q["x_deq"], q["w1_deq"], q["w3_deq"], inp["w2"],
+                       True)
+    dn = fp8_down(h, row_expert, q)
+    y = dn["y"]
     d = y.shape[1]
     y_of_slot = np.zeros((N * K, d), np.float64)
     kept = r["row_of"] >= 0
@@ -371,6 +406,7 @@ def layer_fp8(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order:
     r["out"] = combine(r["row_of"], r["topk_w"], y_of_slot)
     r["y_rows"] = y
     r["h_rows"] = h
+    q.update(hq=dn["hq"], hs=dn["hs"], h_bf16=dn["h_bf16"])
     r["fp8"] = q
     return r
 

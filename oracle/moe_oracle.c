@@ -527,3 +527,59 @@ EXPORT void orc_quantize_rows_e4m3(int64_t rows, int64_t cols, const uint16_t *s
                 e4m3_code(ldexp((double)bf16_to_float(src[r * cols + c]), (int)-j));
     }
 }
+
+/* Nearest bf16 value (1 sign, 8 exponent bits, 7 mantissa bits: binary32's range with 8
+ * significant bits) to a double, ties to even, as bf16 bits; beyond the largest finite value
+ * (2 - 2^-7) * 2^127 rounds to infinity. */
+static uint16_t bf16_nearest(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e); /* binade [2^(e-1), 2^e) */
+    int E = e - 1 < -126 ? -126 : e - 1;
+    double quantum = ldexp(1.0, E - 7);
+    double val = nearbyint(a / quantum) * quantum;
+    if (val > ldexp(2.0 - ldexp(1.0, -7), 127))
+        return sign | 0x7F80;
+    float f = (float)val; /* exact: 8 significant bits within binary32's range */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return sign | (uint16_t)(u >> 16);
+}
+
+EXPORT void orc_round_bf16(int64_t n, const double *v, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = bf16_nearest(v[i]);
+}
+
+/* Down projection alone, from bf16 activation rows: y[r][i] = sum_j h[r][j] * W2[e][i][j]
+ * in fp64, e = row_expert[r]; W2 [E][d][f]. (The FP8 path's down projection runs on the
+ * e4m3 rows of h, given here by their exact bf16 dequantisation.) */
+EXPORT void orc_down_rows(int64_t nrows, const int32_t *row_expert, int64_t d, int64_t f,
+                          const uint16_t *h, const uint16_t *w2, double *y_out)
+{
+#pragma omp parallel
+    {
+        double *hr = (double *)malloc((size_t)f * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t e = row_expert[r];
+            for (int64_t j = 0; j < f; ++j)
+                hr[j] = (double)bf16_to_float(h[r * f + j]);
+            for (int64_t i = 0; i < d; ++i) {
+                const uint16_t *c = w2 + (e * d + i) * f;
+                double y = 0.0;
+                for (int64_t j = 0; j < f; ++j)
+                    y += hr[j] * (double)bf16_to_float(c[j]);
+                y_out[r * d + i] = y;
+            }
+        }
+        free(hr);
+    }
+}

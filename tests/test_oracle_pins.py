@@ -535,11 +535,12 @@ def test_quantize_rows(orc):
 
 
 def test_layer_fp8_reduces_to_bf16_layer_on_e4m3_inputs(orc):
-    """With x, W1, W3 already e4m3 values whose rows reach the top binade, quantisation is
-    the identity and the FP8 layer equals the bf16 layer exactly; on ordinary inputs it
-    stays within the e4m3 rounding bar (three mantissa bits on x and on W1, W3: relative
-    error <= 2^-4 per element, so the relative Frobenius deviation of the output is a few
-    times 2^-4 / sqrt(3) at most; bar 0.1)."""
+    """With x, W1, W3, W2 already e4m3 values whose rows reach the top binade, quantising
+    them is the identity: the FP8 layer's h equals the bf16 layer's h exactly, and its
+    expert outputs differ only by h's roundings (to bf16, then to e4m3: within
+    (2^-4 + 2^-8) relative per element), element by element within
+    (2^-4 + 2^-8 + 2^-40) * sum_j |W2_ij h_j|; on ordinary inputs the output stays within the
+    FP8 bar (three mantissa bits per operand: <= 2^-4 relative per element; bar 0.1)."""
     w = WORKLOADS["tiny"]
     inp = make_layer_inputs(w, seed=3)
     rng = np.random.default_rng(3)
@@ -552,13 +553,85 @@ def test_layer_fp8_reduces_to_bf16_layer_on_e4m3_inputs(orc):
 
     exact = dict(inp, x=e4m3_like(tuple(inp["x"].shape), -12),
                  w1=e4m3_like(tuple(inp["w1"].shape), -14),
-                 w3=e4m3_like(tuple(inp["w3"].shape), -14))
-    a = orc.layer_fp8(exact, w.K, w.W, w.cf)
-    b = orc.layer(exact, w.K, w.W, w.cf)
+                 w3=e4m3_like(tuple(inp["w3"].shape), -14),
+                 w2=e4m3_like(tuple(inp["w2"].shape), -14))
+    a = orc.layer_fp8(exact, w.K, w.W, w.cf, want_h=True)
+    b = orc.layer(exact, w.K, w.W, w.cf, want_h=True)
     assert np.all(a["fp8"]["sx"] == 2.0 ** -12) and np.all(a["fp8"]["s1"] == 2.0 ** -14)
-    np.testing.assert_array_equal(a["out"], b["out"])
+    assert np.all(a["fp8"]["s2"] == 2.0 ** -14)
+    np.testing.assert_array_equal(a["h_rows"], b["h_rows"])
+    w2 = exact["w2"].double().numpy()
+    row_expert = a["expert_of"][a["assign_of_row"]]
+    mag = np.stack([np.abs(w2[e]) @ np.abs(a["h_rows"][i]) for i, e in enumerate(row_expert)])
+    assert np.all(np.abs(a["y_rows"] - b["y_rows"]) <= (2.0 ** -4 + 2.0 ** -8 + 2.0 ** -40) * mag)
+    assert np.abs(a["y_rows"] - b["y_rows"]).max() > 0  # h really was rounded
     r8 = orc.layer_fp8(inp, w.K, w.W, w.cf)
     r16 = orc.layer(inp, w.K, w.W, w.cf)
     np.testing.assert_array_equal(r8["row_of"], r16["row_of"])  # routing is on the bf16 x
     dev = np.linalg.norm(r8["out"] - r16["out"]) / np.linalg.norm(r16["out"])
     assert 1e-3 < dev <= 0.1, dev
+
+
+BF16_HAND = [  # (value, bits), worked by hand: 1 sign, 8 exponent, 7 mantissa bits
+    (1.0, 0x3F80), (-2.0, 0xC000), (0.0, 0x0000), (-0.0, 0x8000),
+    (1.0 + 2.0 ** -8, 0x3F80),  # halfway 1 / 1 + 2^-7: even mantissa 0
+    (1.0 + 3 * 2.0 ** -8, 0x3F82),  # halfway 1 + 2^-7 / 1 + 2^-6: even mantissa 2
+    (1.0 + 2.0 ** -8 + 2.0 ** -40, 0x3F81),  # just above halfway
+    ((2.0 - 2.0 ** -7) * 2.0 ** 127, 0x7F7F),  # largest finite
+    ((2.0 - 2.0 ** -8) * 2.0 ** 127, 0x7F80),  # halfway to 2^128: even -> infinity
+    (2.0 ** -133, 0x0001), (2.0 ** -134, 0x0000), (3 * 2.0 ** -134, 0x0002),  # subnormals
+]
+
+
+def test_round_bf16_hand_values_and_exact_nearest(orc):
+    v = np.array([a for a, _ in BF16_HAND])
+    np.testing.assert_array_equal(orc.round_bf16(v), [b for _, b in BF16_HAND])
+    # random doubles: the result is the nearer of the two bf16 neighbours (exact rationals),
+    # ties to the even code
+    from fractions import Fraction
+    rng = np.random.default_rng(9)
+    vals = rng.standard_normal(3000) * np.exp(rng.uniform(-30, 30, 3000))
+    got = orc.round_bf16(vals)
+    for x, b in zip(vals, got):
+        g = float(np.array([int(b) << 16], np.uint32).view(np.float32)[0])
+        lo_bits = int(np.array([g], np.float32).view(np.uint32)[0]) >> 16
+        nb = [((lo_bits + s) & 0xFFFF) for s in (-1, 1)]
+        for n in nb:
+            o = float(np.array([n << 16], np.uint32).view(np.float32)[0])
+            if np.isfinite(o) and np.sign(o) == np.sign(g):
+                dg, do = abs(Fraction(g) - Fraction(x)), abs(Fraction(o) - Fraction(x))
+                assert dg < do or (dg == do and (int(b) & 1) == 0), (x, hex(int(b)), hex(n))
+    # float32-exact inputs: torch's float32 -> bf16 rounding is a second implementation
+    f32 = (rng.standard_normal(20000) * 50).astype(np.float32)
+    ref = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(orc.round_bf16(f32.astype(np.float64)), ref)
+
+
+def test_down_rows_matches_matmul(orc):
+    rng = np.random.default_rng(10)
+    E, d, f, n = 3, 24, 40, 17
+    w2 = torch.from_numpy(rng.standard_normal((E, d, f)) * 0.1).to(torch.bfloat16)
+    h = torch.from_numpy(rng.standard_normal((n, f))).to(torch.bfloat16)
+    re = rng.integers(0, E, n).astype(np.int32)
+    y = orc.down_rows(re, orc.as_u16(h), w2)
+    ref = np.stack([w2[e].double().numpy() @ h[i].double().numpy() for i, e in enumerate(re)])
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_layer_fp8_down_noise_bounded(orc):
+    """The all-FP8 expert path (e4m3 x, W1, W3, then e4m3 h and W2) against the bf16 layer:
+    routing identical, deviation of the output above zero and within the FP8 bar 0.1; the
+    e4m3 h rows dequantise to within 2^-4 of the bf16 h."""
+    w = WORKLOADS["tiny"]
+    inp = make_layer_inputs(w, seed=4)
+    r8 = orc.layer_fp8(inp, w.K, w.W, w.cf)
+    r16 = orc.layer(inp, w.K, w.W, w.cf)
+    np.testing.assert_array_equal(r8["row_of"], r16["row_of"])
+    dev = np.linalg.norm(r8["out"] - r16["out"]) / np.linalg.norm(r16["out"])
+    assert 1e-3 < dev <= 0.1, dev
+    q = r8["fp8"]
+    hb = (q["h_bf16"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    hd = (orc.dequantize_rows_bf16(q["hq"], q["hs"]).astype(np.uint32) << 16).view(
+        np.float32).astype(np.float64)
+    rel = np.abs(hd - hb) / np.maximum(np.abs(hb), 2.0 ** -6 * q["hs"][:, None])
+    assert rel.max() <= 2.0 ** -4
