@@ -239,11 +239,13 @@ def run_gpu(args, w) -> dict:
         sorted_scale = torch.empty(RA, dtype=torch.float32, device=dev)
         packed_scale = torch.empty(RA, dtype=torch.float32, device=dev)
         for lw in layers:
-            for k in ("w1", "w3"):
-                q = torch.empty(E, f, d, dtype=torch.uint8, device=dev)
-                sc = torch.empty(E, f, dtype=torch.float32, device=dev)
+            for k in ("w1", "w3", "w2"):
+                q = torch.empty(lw[k].shape, dtype=torch.uint8, device=dev)
+                sc = torch.empty(lw[k].shape[:-1], dtype=torch.float32, device=dev)
                 m.moe_quantize_rows_e4m3(lw[k], q, sc)
                 lw[k + "q"], lw[k + "s"] = q, sc
+        h_q = torch.empty(RA, f, dtype=torch.uint8, device=dev)
+        h_scale = torch.empty(RA, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
     D = torch.empty(W * W, dtype=torch.int64, device=dev)
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
@@ -267,7 +269,9 @@ def run_gpu(args, w) -> dict:
     # per layer: logits, top-K, histogram, scan, positions, scatter, up, down, combine
     # (+ offsets, shared up, shared down for the Residual-MoE layer); + affinity per layer pair
     # (+ histogram, scan, positions of the first pass and the ranking kernel when re-routing)
-    launches_per_step = L * (9 + (3 if shared else 0) + (4 if w.reroute else 0)) + (L - 1)
+    # (+ the quantisation of h for the FP8 down projection)
+    launches_per_step = (L * (9 + (3 if shared else 0) + (4 if w.reroute else 0) +
+                              (1 if w.fp8 else 0)) + (L - 1))
 
     def step(ev=None):
         """One step; ev (optional) is [layer][n_ev] events around the stages."""
@@ -304,7 +308,12 @@ def run_gpu(args, w) -> dict:
                 m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
             if e is not None:
                 e[3].record(st)
-            m.moe_expert_down(shape, h, offsets[l], lw["w2"], y, st)
+            if w.fp8:  # the kept rows of h to e4m3, then the e4m3 down GEMM
+                m.moe_quantize_rows_e4m3(h, h_q, h_scale, rows_dev=offsets[l][E:], stream=st)
+                m.moe_expert_down_fp8(shape, h_q, h_scale, offsets[l], lw["w2q"], lw["w2s"], y,
+                                      st)
+            else:
+                m.moe_expert_down(shape, h, offsets[l], lw["w2"], y, st)
             j = 4
             if e is not None:
                 e[j].record(st)
@@ -412,8 +421,8 @@ def run_gpu(args, w) -> dict:
                                    out_dev[b], ws=lws, stream=stream)
             elif w.fp8:
                 m.moe_layer_fp8(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1q"],
-                                l0["w1s"], l0["w3q"], l0["w3s"], l0["w2"], out_dev[b], ws=lws,
-                                stream=stream)
+                                l0["w1s"], l0["w3q"], l0["w3s"], l0["w2q"], l0["w2s"], out_dev[b],
+                                ws=lws, stream=stream)
             elif L == 1:
                 m.moe_layer(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1"], l0["w3"],
                             l0["w2"], out_dev[b], ws=lws, stream=stream)
@@ -480,7 +489,7 @@ def run_gpu(args, w) -> dict:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("e4m3 gate/up operands and dispatch payload, bf16 down, fp32 accumulate"
+        "dtype": ("e4m3 (dispatch payload and both expert GEMMs' operands), fp32 accumulate"
                   if w.fp8 else "bf16"),
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",
@@ -552,8 +561,10 @@ def oracle_time(w, inp_cpu, sample_tokens: int, shared_cpu=None) -> dict:
         as_bf16 = lambda u: torch.from_numpy(u.view(np.int16)).view(torch.bfloat16)
         q1, s1 = oracle.quantize_rows_e4m3(inp_cpu["w1"])
         q3, s3 = oracle.quantize_rows_e4m3(inp_cpu["w3"])
+        q2, s2 = oracle.quantize_rows_e4m3(inp_cpu["w2"])
         exp_inp = dict(inp_cpu, w1=as_bf16(oracle.dequantize_rows_bf16(q1, s1)),
-                       w3=as_bf16(oracle.dequantize_rows_bf16(q3, s3)))
+                       w3=as_bf16(oracle.dequantize_rows_bf16(q3, s3)),
+                       w2=as_bf16(oracle.dequantize_rows_bf16(q2, s2)))
     t0 = time.perf_counter()
     r = oracle.route_and_dispatch(inp_cpu["x"], inp_cpu["w_router"], inp_cpu.get("bias"), w.K,
                                   w.W, w.cf, order=int(w.slot_major), reroute=w.reroute)

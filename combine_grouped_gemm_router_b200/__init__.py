@@ -63,9 +63,10 @@ _sigs = {
     "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
     "moe_dispatch_reroute": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_dispatch_fp8": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
-    "moe_quantize_rows_e4m3": ([c_p, c_i64, c_i32, c_p, c_p, c_p], c_i32),
+    "moe_quantize_rows_e4m3": ([c_p, c_i64, c_i32, c_p, c_p, c_p, c_p], c_i32),
     "moe_expert_up_fp8": ([_SP] + [c_p] * 9, c_i32),
-    "moe_layer_fp8": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
+    "moe_expert_down_fp8": ([_SP] + [c_p] * 7, c_i32),
+    "moe_layer_fp8": ([_SP] + [c_p] * 14 + [c_size, c_p], c_i32),
     "moe_expert_gemm": ([_SP] + [c_p] * 8, c_i32),
     "moe_expert_up": ([_SP] + [c_p] * 6, c_i32),
     "moe_expert_down": ([_SP] + [c_p] * 5, c_i32),
@@ -230,12 +231,13 @@ def moe_dispatch_fp8(shape, x, topk_idx, counts, kept, offsets, row_of, assign_o
            "moe_dispatch_fp8")
 
 
-def moe_quantize_rows_e4m3(src, codes, scale, stream=None):
-    """Row-wise e4m3 quantisation of a bf16 matrix (rows = all leading dims)."""
+def moe_quantize_rows_e4m3(src, codes, scale, rows_dev=None, stream=None):
+    """Row-wise e4m3 quantisation of a bf16 matrix (rows = all leading dims); rows_dev
+    (optional device int32 tensor) caps the row count on the device."""
     cols = src.shape[-1]
     rows = src.numel() // cols
     _check(_lib.moe_quantize_rows_e4m3(_ptr(src), rows, cols, _ptr(codes), _ptr(scale),
-                                       _stream(stream)), "moe_quantize_rows_e4m3")
+                                       _ptr(rows_dev), _stream(stream)), "moe_quantize_rows_e4m3")
 
 
 def moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q, w3_scale, h,
@@ -243,6 +245,12 @@ def moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q
     _check(_lib.moe_expert_up_fp8(ctypes.byref(shape), _ptr(x_sorted), _ptr(sorted_scale),
                                   _ptr(offsets), _ptr(w1q), _ptr(w1_scale), _ptr(w3q),
                                   _ptr(w3_scale), _ptr(h), _stream(stream)), "moe_expert_up_fp8")
+
+
+def moe_expert_down_fp8(shape, hq, h_scale, offsets, w2q, w2_scale, y, stream=None):
+    _check(_lib.moe_expert_down_fp8(ctypes.byref(shape), _ptr(hq), _ptr(h_scale), _ptr(offsets),
+                                    _ptr(w2q), _ptr(w2_scale), _ptr(y), _stream(stream)),
+           "moe_expert_down_fp8")
 
 
 MOE_STATIC_SCRATCH_BYTES = 1 << 20
@@ -311,15 +319,15 @@ def moe_layer(shape, x, w_router, bias, w1, w3, w2, out, residual=None, topk_idx
                           _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)), "moe_layer")
 
 
-def moe_layer_fp8(shape, x, w_router, bias, w1q, w1_scale, w3q, w3_scale, w2, out, residual=None,
-                  topk_idx_out=None, stats=None, ws=None, stream=None):
-    """moe_layer with the FP8 payload and the e4m3 gate/up GEMM (weights from
+def moe_layer_fp8(shape, x, w_router, bias, w1q, w1_scale, w3q, w3_scale, w2q, w2_scale, out,
+                  residual=None, topk_idx_out=None, stats=None, ws=None, stream=None):
+    """moe_layer with the FP8 payload and e4m3 expert GEMMs (weights from
     moe_quantize_rows_e4m3)."""
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.moe_layer_fp8(ctypes.byref(shape), _ptr(x), _ptr(w_router), _ptr(bias),
-                              _ptr(w1q), _ptr(w1_scale), _ptr(w3q), _ptr(w3_scale), _ptr(w2),
-                              _ptr(residual), _ptr(out), _ptr(topk_idx_out), _ptr(stats),
-                              _ptr(ws), ws_bytes, _stream(stream)), "moe_layer_fp8")
+                              _ptr(w1q), _ptr(w1_scale), _ptr(w3q), _ptr(w3_scale), _ptr(w2q),
+                              _ptr(w2_scale), _ptr(residual), _ptr(out), _ptr(topk_idx_out),
+                              _ptr(stats), _ptr(ws), ws_bytes, _stream(stream)), "moe_layer_fp8")
 
 
 def moe_affinity_accumulate(N, E, K, topk_j, topk_j1, counts, stream=None):

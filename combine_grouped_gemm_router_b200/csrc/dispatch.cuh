@@ -642,10 +642,15 @@ __global__ void __launch_bounds__(256) scatter_rows_e4m3_kernel(ScatterArgs p)
 
 // Row-wise e4m3 quantisation of a bf16 matrix (for the experts' W1 and W3): one
 // warp per row, the same two passes and rounding as the FP8 scatter. cols % 16 == 0.
+// rows_dev (nullable, device): rows beyond *rows_dev are skipped (the FP8 down projection
+// quantises only the rows the dispatch kept).
 __global__ void __launch_bounds__(256)
     quantize_rows_e4m3_kernel(const uint16_t *__restrict__ src, int64_t rows, int cols,
-                              uint8_t *__restrict__ codes, float *__restrict__ scale)
+                              uint8_t *__restrict__ codes, float *__restrict__ scale,
+                              const int32_t *__restrict__ rows_dev)
 {
+    if (rows_dev && *rows_dev < rows)
+        rows = *rows_dev;
     const int lane = threadIdx.x & 31;
     const int n16 = cols >> 4;
     const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);

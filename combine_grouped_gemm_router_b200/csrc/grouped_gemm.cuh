@@ -23,7 +23,7 @@
 // N=256 MMA per K-step; the epilogue reads gate column c and up column 128+c
 // and writes h = silu(g) * u as bf16 (the next GEMM's operand). Mode 1 (down):
 // fp32 output straight from TMEM, so the combine sums unrounded expert outputs.
-// Mode 2 (gate/up on the FP8 payload, [MoE 推理服务工程真相 2026, §6.3]): as mode 0
+// Modes 2 and 3 (the FP8 path, [MoE 推理服务工程真相 2026, §6.3]): modes 0 and 1
 // with e4m3 A and B (tcgen05 kind::f8f6f4). A 128-byte swizzle atom then holds
 // 128 K elements instead of 64, so tiles, stages and descriptors keep their byte
 // layout; the epilogue multiplies the accumulator by the row's scale and the
@@ -48,7 +48,9 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int THREADS = 192;
 
 // K elements in one 128-byte swizzle atom: 64 bf16 or 128 e4m3.
-__host__ __device__ constexpr int atom_k(int MODE) { return MODE == 2 ? 128 : 64; }
+__host__ __device__ constexpr bool is_e4m3(int MODE) { return MODE >= 2; }
+__host__ __device__ constexpr bool is_gate(int MODE) { return MODE == 0 || MODE == 2; }
+__host__ __device__ constexpr int atom_k(int MODE) { return is_e4m3(MODE) ? 128 : 64; }
 
 struct Args {
     const int32_t *offsets;  // [E+1]
@@ -58,10 +60,10 @@ struct Args {
     int b_rows;          // rows of one expert's B matrix (f for mode 0, d for mode 1)
     int rows_alloc;      // rows of the A buffer
     int select;          // which experts this launch takes: 0 all, 1 pair-tile experts, 2 the rest
-    void *out;           // modes 0, 2: bf16 h [rows_alloc][ldo]; mode 1: fp32 y [rows_alloc][ldo]
+    void *out;           // modes 0, 2: bf16 h [rows_alloc][ldo]; 1, 3: fp32 y [rows_alloc][ldo]
     int ldo;
-    const float *row_scale;  // mode 2: scale of each A row [rows_alloc]
-    const float *b_scale0;   // mode 2: scale of each W1 row [E * b_rows]
+    const float *row_scale;  // modes 2, 3: scale of each A row [rows_alloc]
+    const float *b_scale0;   // mode 2: scale of each W1 row; mode 3: of each W2 row [E * b_rows]
     const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
     uint64_t timeout_ns;
 };
@@ -180,7 +182,7 @@ __host__ __device__ constexpr uint32_t instr_desc_e4m3(int M, int N)
 template <int MODE>
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N)
 {
-    return MODE == 2 ? instr_desc_e4m3(M, N) : instr_desc_bf16(M, N);
+    return is_e4m3(MODE) ? instr_desc_e4m3(M, N) : instr_desc_bf16(M, N);
 }
 
 // One MMA of 32 bytes of K (16 bf16 or 32 e4m3 elements).
@@ -188,7 +190,7 @@ template <int MODE>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate)
 {
-    if constexpr (MODE == 2)
+    if constexpr (is_e4m3(MODE))
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
@@ -313,14 +315,53 @@ __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr
     }
 }
 
+// Down-projection epilogue of one thread: accumulator row `row`, columns [0, BN) of
+// N-slab n -> fp32 y (not rounded before the combine). Mode 3 scales by the row scale
+// and the W2 output-channel scales.
+template <int MODE, int BN>
+__device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int e, int n,
+                                              int row, bool store)
+{
+    float *frow = reinterpret_cast<float *>(args.out) + (size_t)row * args.ldo;
+    float4 *dst = reinterpret_cast<float4 *>(frow + n * BN);
+    float sx = 1.0f;
+    const float *s2 = nullptr;
+    if constexpr (MODE == 3) {
+        sx = store ? args.row_scale[row] : 0.0f;
+        s2 = args.b_scale0 + (size_t)e * args.b_rows + n * BN;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(v));
+        tmem_ld16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+        tmem_ld_wait();
+        if (store) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                       __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                if constexpr (MODE == 3) {
+                    const float4 sc = *reinterpret_cast<const float4 *>(s2 + c + j);
+                    o.x *= sx * sc.x;
+                    o.y *= sx * sc.y;
+                    o.z *= sx * sc.z;
+                    o.w *= sx * sc.w;
+                }
+                dst[(c + j) / 4] = o;
+            }
+        }
+    }
+}
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Args args)
 {
-    static_assert(MODE != 1 ? BN == 256 : (BN == 128 || BN == 256), "tile shape");
-    constexpr bool GATE = MODE != 1;  // gate/up: W1 and W3 halves, SwiGLU epilogue
+    static_assert(is_gate(MODE) ? BN == 256 : (BN == 128 || BN == 256), "tile shape");
+    constexpr bool GATE = is_gate(MODE);  // gate/up: W1 and W3 halves, SwiGLU epilogue
     constexpr int KX = atom_k(MODE);
     constexpr int B_BYTES = BN * BK * 2;
     constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -504,25 +545,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (GATE) {
                 swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
             } else {
-                // fp32 output: the down projection is not rounded before the combine
-                float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
-                uint4 *dst = reinterpret_cast<uint4 *>(frow + n * BN);
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16(taddr + c, v0);
-                    tmem_ld16(taddr + c + 16, v1);
-                    tmem_ld_wait();
-                    if (r < valid) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            dst[c / 4 + j] = make_uint4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2],
-                                                        v0[4 * j + 3]);
-                            dst[c / 4 + 4 + j] = make_uint4(v1[4 * j], v1[4 * j + 1],
-                                                            v1[4 * j + 2], v1[4 * j + 3]);
-                        }
-                    }
-                }
+                down_epilogue<MODE, BN>(args, taddr, e, n, row0 + r, r < valid);
             }
             tc_fence_before();
             __syncwarp();
@@ -605,7 +628,7 @@ template <int MODE>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate)
 {
-    if constexpr (MODE == 2)
+    if constexpr (is_e4m3(MODE))
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
@@ -634,7 +657,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 {
     constexpr int BMP = 256;  // rows per pair tile
     constexpr int BN = 256;
-    constexpr bool GATE = MODE != 1;
+    constexpr bool GATE = is_gate(MODE);
     constexpr int KX = atom_k(MODE);
     constexpr uint32_t IDESC = instr_desc<MODE>(BMP, BN);
 
@@ -821,24 +844,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (GATE) {
                 swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
             } else {
-                float *frow = reinterpret_cast<float *>(args.out) + (size_t)(row0 + r) * args.ldo;
-                uint4 *dst = reinterpret_cast<uint4 *>(frow + n * BN);
-#pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16(taddr + c, v0);
-                    tmem_ld16(taddr + c + 16, v1);
-                    tmem_ld_wait();
-                    if (r < valid) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            dst[c / 4 + j] = make_uint4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2],
-                                                        v0[4 * j + 3]);
-                            dst[c / 4 + 4 + j] = make_uint4(v1[4 * j], v1[4 * j + 1],
-                                                            v1[4 * j + 2], v1[4 * j + 3]);
-                        }
-                    }
-                }
+                down_epilogue<MODE, BN>(args, taddr, e, n, row0 + r, r < valid);
             }
             tc_fence_before();
             __syncwarp();

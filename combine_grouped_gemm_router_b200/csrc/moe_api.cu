@@ -134,7 +134,7 @@ ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
 // moe_layer: every intermediate, after the scratch.
 struct LayerLayout {
     size_t topk_idx, topk_w, counts, kept, offsets, row_of, assign, x_sorted, x_packed,
-        sorted_scale, packed_scale, h, y, nonfinite, total;
+        sorted_scale, packed_scale, h, hq, h_scale, y, nonfinite, total;
 };
 
 LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
@@ -166,6 +166,10 @@ LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
     o = align_up(o + RA * 4);
     L.h = o;
     o = align_up(o + RA * (size_t)s->f * 2);
+    L.hq = o;  // FP8 path: e4m3 rows of h and their scales
+    o = align_up(o + RA * (size_t)s->f);
+    L.h_scale = o;
+    o = align_up(o + RA * 4);
     L.y = o;
     o = align_up(o + RA * s->d * 4);
     L.nonfinite = o;
@@ -576,6 +580,53 @@ moe_status_t gemm_up_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const 
     return launch_gemm<2, 256>(tA, tW1, tW3, args, st);
 }
 
+// Down projection on e4m3 rows of h (scale per row) and e4m3 rows of W2 (scale per output
+// channel), fp32 y. The pair kernel needs f % 256 == 0 (two atoms per stage).
+moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const uint8_t *hq,
+                            const float *h_scale, const int32_t *offsets, const uint8_t *w2,
+                            const float *s2, float *y, cudaStream_t st)
+{
+    CUtensorMap tA, tW2;
+    if (!make_tmap(&tA, hq, f, (uint64_t)a_rows, true) ||
+        !make_tmap(&tW2, w2, f, (uint64_t)E * d, true))
+        return MOE_ERR_CUDA;
+    gg::Args args = {};
+    args.offsets = offsets;
+    args.E = E;
+    args.k_blocks = f / gg::atom_k(3);
+    args.b_rows = d;
+    args.rows_alloc = (int)a_rows;
+    args.out = y;
+    args.ldo = d;
+    args.row_scale = h_scale;
+    args.b_scale0 = s2;
+    args.timeout_ns = kWaitTimeoutNs;
+    args.select = 0;
+    if (d % 256 == 0) {
+        args.n_tiles = d / 256;
+        if (pair && args.k_blocks % gg::KA2 == 0) {
+            args.select = 1;
+            moe_status_t rc = launch_gemm_pair<3>(tA, tW2, tW2, args, st);
+            if (rc != MOE_OK)
+                return rc;
+            args.select = 2;
+        }
+        return launch_gemm<3, 256>(tA, tW2, tW2, args, st);
+    }
+    args.n_tiles = d / 128;
+    return launch_gemm<3, 128>(tA, tW2, tW2, args, st);
+}
+
+// Row-wise e4m3 quantisation launch; rows_dev (nullable, device) caps the row count.
+moe_status_t quantize_rows_launch(const uint16_t *src, int64_t rows, int cols, uint8_t *codes,
+                                  float *scale, const int32_t *rows_dev, cudaStream_t st)
+{
+    const int64_t blocks64 = (rows + 7) / 8;
+    const int blocks = (int)(blocks64 < 148 * 64 ? blocks64 : 148 * 64);
+    quantize_rows_e4m3_kernel<<<blocks, 256, 0, st>>>(src, rows, cols, codes, scale, rows_dev);
+    return launch_status();
+}
+
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                             uint16_t *h, cudaStream_t st)
@@ -814,21 +865,19 @@ moe_dispatch_fp8(const moe_shape_t *shape, const uint16_t *x, const int32_t *top
 
 __attribute__((visibility("default"))) moe_status_t
 moe_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int32_t cols, uint8_t *codes,
-                       float *scale, moe_stream_t stream)
+                       float *scale, const int32_t *rows_dev, moe_stream_t stream)
 {
     if (rows < 0 || cols < 16 || !src || !codes || !scale)
         return MOE_ERR_INVALID_ARG;
     if (cols % 16 != 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(src) || !aligned16(codes) || !aligned4(scale))
+    if (!aligned16(src) || !aligned16(codes) || !aligned4(scale) ||
+        (rows_dev && !aligned4(rows_dev)))
         return MOE_ERR_MISALIGNED;
     if (rows == 0)
         return MOE_OK;
-    const int64_t blocks64 = (rows + 7) / 8;
-    const int blocks = (int)(blocks64 < 148 * 64 ? blocks64 : 148 * 64);
-    quantize_rows_e4m3_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        src, rows, cols, codes, scale);
-    return launch_status();
+    return quantize_rows_launch(src, rows, cols, codes, scale, rows_dev,
+                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -848,6 +897,25 @@ moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted, const float
     return gemm_up_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
                         x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q, w3_scale, h,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_scale,
+                    const int32_t *offsets, const uint8_t *w2q, const float *w2_scale, float *y,
+                    moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, true, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (!hq || !h_scale || !offsets || !w2q || !w2_scale || !y)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(hq) || !aligned16(w2q) || !aligned16(w2_scale) || !aligned16(y) ||
+        !aligned4(offsets) || !aligned4(h_scale))
+        return MOE_ERR_MISALIGNED;
+    return gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
+                          hq, h_scale, offsets, w2q, w2_scale, y,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -919,12 +987,12 @@ moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
 
 namespace {
 
-// Gate/up weights of a layer: bf16 W1, W3, or their e4m3 rows with per-row scales (then
-// the dispatch writes the FP8 payload).
-struct UpWeights {
-    const uint16_t *w1, *w3;
-    const uint8_t *w1q, *w3q;
-    const float *s1, *s3;
+// Expert weights of a layer: bf16 W1, W3, W2, or their e4m3 rows with per-row scales
+// (then the dispatch writes the FP8 payload and both expert GEMMs run on e4m3).
+struct ExpertWeights {
+    const uint16_t *w1, *w3, *w2;
+    const uint8_t *w1q, *w3q, *w2q;
+    const float *s1, *s3, *s2;
     bool e4m3() const { return w1q != nullptr; }
 };
 
@@ -932,8 +1000,8 @@ struct UpWeights {
 // intermediate in the workspace. Arguments validated by the caller; f_shared == 0: no
 // shared MLP.
 moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16_t *x,
-                       const float *w_router, const float *bias, const UpWeights &up,
-                       const uint16_t *w2, int32_t f_shared, const uint16_t *ws1,
+                       const float *w_router, const float *bias, const ExpertWeights &up,
+                       int32_t f_shared, const uint16_t *ws1,
                        const uint16_t *ws3, const uint16_t *ws2, const uint16_t *residual,
                        void *out, int32_t *topk_idx_out, moe_stats_t *stats, char *w,
                        size_t ws_need, cudaStream_t st)
@@ -979,7 +1047,18 @@ moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16
                             up.w3, h, st);
     if (rc != MOE_OK)
         return rc;
-    rc = expert_down_impl(shape, g, h, offsets, w2, y, st);
+    if (up.e4m3()) {
+        // h -> e4m3 rows (only the offsets[E] kept rows), then the e4m3 down projection
+        uint8_t *hq = reinterpret_cast<uint8_t *>(w + L.hq);
+        float *hs = reinterpret_cast<float *>(w + L.h_scale);
+        rc = quantize_rows_launch(h, g.rows_alloc, shape->f, hq, hs, offsets + shape->E, st);
+        if (rc != MOE_OK)
+            return rc;
+        rc = gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc,
+                            use_pair_tiles(shape, g), hq, hs, offsets, up.w2q, up.s2, y, st);
+    } else {
+        rc = expert_down_impl(shape, g, h, offsets, up.w2, y, st);
+    }
     if (rc != MOE_OK)
         return rc;
     float *y_s = nullptr;
@@ -1018,26 +1097,28 @@ moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(ws))
         return MOE_ERR_MISALIGNED;
-    return layer_run(shape, g, x, w_router, bias, UpWeights{w1, w3, nullptr, nullptr, nullptr, nullptr},
-                     w2, 0, nullptr, nullptr, nullptr, residual, out, topk_idx_out, stats,
+    return layer_run(shape, g, x, w_router, bias,
+                     ExpertWeights{w1, w3, w2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr},
+                     0, nullptr, nullptr, nullptr, residual, out, topk_idx_out, stats,
                      static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
 moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
               const float *bias, const uint8_t *w1q, const float *w1_scale, const uint8_t *w3q,
-              const float *w3_scale, const uint16_t *w2, const uint16_t *residual, void *out,
-              int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
-              moe_stream_t stream)
+              const float *w3_scale, const uint8_t *w2q, const float *w2_scale,
+              const uint16_t *residual, void *out, int32_t *topk_idx_out, moe_stats_t *stats,
+              void *ws, size_t ws_bytes, moe_stream_t stream)
 {
     Geometry g;
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
-    if (!x || !w_router || !w1q || !w1_scale || !w3q || !w3_scale || !w2 || !out)
+    if (!x || !w_router || !w1q || !w1_scale || !w3q || !w3_scale || !w2q || !w2_scale || !out)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1q) ||
-        !aligned16(w3q) || !aligned16(w1_scale) || !aligned16(w3_scale) || !aligned16(w2) ||
+        !aligned16(w3q) || !aligned16(w1_scale) || !aligned16(w3_scale) || !aligned16(w2q) ||
+        !aligned16(w2_scale) ||
         !aligned16(out) || (residual && !aligned16(residual)) ||
         (topk_idx_out && !aligned4(topk_idx_out)) ||
         (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
@@ -1048,8 +1129,9 @@ moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router
     if (!aligned16(ws))
         return MOE_ERR_MISALIGNED;
     return layer_run(shape, g, x, w_router, bias,
-                     UpWeights{nullptr, nullptr, w1q, w3q, w1_scale, w3_scale}, w2, 0, nullptr,
-                     nullptr, nullptr, residual, out, topk_idx_out, stats,
+                     ExpertWeights{nullptr, nullptr, nullptr, w1q, w3q, w2q, w1_scale, w3_scale,
+                                   w2_scale},
+                     0, nullptr, nullptr, nullptr, residual, out, topk_idx_out, stats,
                      static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1112,8 +1194,9 @@ moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
         return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(ws))
         return MOE_ERR_MISALIGNED;
-    return layer_run(shape, g, x, w_router, bias, UpWeights{w1, w3, nullptr, nullptr, nullptr, nullptr},
-                     w2, f_shared, ws1, ws3, ws2, residual, out, topk_idx_out, stats,
+    return layer_run(shape, g, x, w_router, bias,
+                     ExpertWeights{w1, w3, w2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr},
+                     f_shared, ws1, ws3, ws2, residual, out, topk_idx_out, stats,
                      static_cast<char *>(ws), need, reinterpret_cast<cudaStream_t>(stream));
 }
 

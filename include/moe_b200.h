@@ -267,14 +267,20 @@ moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const 
  * with max|row| * 2^-j <= 448 (j = 0 for a zero or non-finite row); each element is
  * x * 2^-j rounded to nearest-even e4m3, saturating; value = code * 2^j. Routing stays on
  * the bf16 x; the experts' gate/up projections consume the e4m3 rows of x together with
- * e4m3 rows of W1 and W3 (one scale per output channel) on tcgen05 kind::f8f6f4; h, the
- * down projection and the combine are as in the bf16 path. */
+ * e4m3 rows of W1 and W3 (one scale per output channel) on tcgen05 kind::f8f6f4; h is
+ * written as bf16, its kept rows are then quantised to e4m3 the same way (one scale per
+ * row), and the down projection runs on them and on e4m3 rows of W2 (one scale per output
+ * channel); y and the combine stay fp32. */
 
 /* Row-wise e4m3 quantisation of a bf16 matrix src [rows][cols] (DEVICE): codes [rows][cols]
- * uint8 and scale [rows] fp32 (DEVICE, caller-owned). For the experts' W1 and W3 pass
- * rows = E*f, cols = d. cols % 16 == 0; src, codes 16-byte aligned. */
+ * uint8 and scale [rows] fp32 (DEVICE, caller-owned). For the experts' W1, W3 pass rows = E*f,
+ * cols = d; for W2 rows = E*d, cols = f; for the activations h of the FP8 down projection
+ * rows = rows_alloc, cols = f and rows_dev = offsets + E (nullable, DEVICE int32: only the
+ * first min(rows, *rows_dev) rows are quantised, a count known only on the device).
+ * cols % 16 == 0; src, codes 16-byte aligned. */
 moe_status_t moe_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int32_t cols,
-                                    uint8_t *codes, float *scale, moe_stream_t stream);
+                                    uint8_t *codes, float *scale, const int32_t *rows_dev,
+                                    moe_stream_t stream);
 
 /* moe_dispatch with the FP8 payload: x_sorted and x_packed hold e4m3 rows ([rows_alloc][d]
  * uint8) and sorted_scale / packed_scale [rows_alloc] fp32 the scale of each row (packed_scale
@@ -296,6 +302,14 @@ moe_status_t moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted
                                const float *sorted_scale, const int32_t *offsets,
                                const uint8_t *w1q, const float *w1_scale, const uint8_t *w3q,
                                const float *w3_scale, uint16_t *h, moe_stream_t stream);
+
+/* Down projection on e4m3 rows: y = sh * s2 * (hq W2q^T), fp32 y [rows_alloc][d]; hq e4m3
+ * [rows_alloc][f] with h_scale per row (moe_quantize_rows_e4m3 of the bf16 h, rows =
+ * offsets[E]); w2q e4m3 [E][d][f] with w2_scale [E][d] (16-byte aligned). d % 128 == 0,
+ * f % 128 == 0. */
+moe_status_t moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_scale,
+                                 const int32_t *offsets, const uint8_t *w2q, const float *w2_scale,
+                                 float *y, moe_stream_t stream);
 
 /* Weighted combine back to token order.
  * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (weighted merge into the
@@ -343,15 +357,17 @@ moe_status_t moe_layer(const moe_shape_t *shape, const uint16_t *x, const float 
                        int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
 
-/* moe_layer with the FP8 payload: the dispatch writes e4m3 rows and the gate/up GEMM runs on
- * them with the e4m3 weights w1q, w3q [E][f][d] and their scales w1_scale, w3_scale [E][f]
- * (moe_quantize_rows_e4m3). W2 stays bf16. Every flag of moe_layer applies; the workspace is
- * moe_layer_workspace_size(shape). */
+/* moe_layer with the FP8 payload and FP8 expert GEMMs: the dispatch writes e4m3 rows, the
+ * gate/up GEMM runs on them with the e4m3 weights w1q, w3q [E][f][d] (scales w1_scale,
+ * w3_scale [E][f]), h's kept rows are quantised to e4m3 and the down GEMM runs on them with
+ * w2q [E][d][f] (scales w2_scale [E][d]); all weights from moe_quantize_rows_e4m3. Every
+ * flag of moe_layer applies; the workspace is moe_layer_workspace_size(shape). */
 moe_status_t moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
                            const float *bias, const uint8_t *w1q, const float *w1_scale,
-                           const uint8_t *w3q, const float *w3_scale, const uint16_t *w2,
-                           const uint16_t *residual, void *out, int32_t *topk_idx_out,
-                           moe_stats_t *stats, void *ws, size_t ws_bytes, moe_stream_t stream);
+                           const uint8_t *w3q, const float *w3_scale, const uint8_t *w2q,
+                           const float *w2_scale, const uint16_t *residual, void *out,
+                           int32_t *topk_idx_out, moe_stats_t *stats, void *ws, size_t ws_bytes,
+                           moe_stream_t stream);
 
 /* Inter-layer expert affinity counts, accumulated into counts [E][E] int64:
  * for every token t, i in topk_j[t], p in topk_j1[t]: counts[i][p] += 1.

@@ -137,14 +137,19 @@ def test_argument_errors_return_before_launch(m):
                                 None, P, need, None) == 4  # misaligned scale
     assert lib.moe_dispatch_fp8(by(rr), P, P, P, P, P, P, P, P, P, None, None, None, None, None,
                                 P, need_rr, None) == 1  # re-routing needs the logits
-    assert lib.moe_quantize_rows_e4m3(P, 4, 24, P, P, None) == 2  # cols % 16
-    assert lib.moe_quantize_rows_e4m3(P, 4, 32, P + 8, P, None) == 4
-    assert lib.moe_quantize_rows_e4m3(None, 4, 32, P, P, None) == 1
-    assert lib.moe_quantize_rows_e4m3(P, 0, 32, P, P, None) == 0  # nothing to do
+    assert lib.moe_quantize_rows_e4m3(P, 4, 24, P, P, None, None) == 2  # cols % 16
+    assert lib.moe_quantize_rows_e4m3(P, 4, 32, P + 8, P, None, None) == 4
+    assert lib.moe_quantize_rows_e4m3(P, 4, 32, P, P, P + 2, None) == 4  # row count alignment
+    assert lib.moe_quantize_rows_e4m3(None, 4, 32, P, P, None, None) == 1
+    assert lib.moe_quantize_rows_e4m3(P, 0, 32, P, P, None, None) == 0  # nothing to do
+    assert lib.moe_expert_down_fp8(by(s), P, None, P, P, P, P, None) == 1
+    assert lib.moe_expert_down_fp8(by(s), P, P, P, P, P + 4, P, None) == 4
     assert lib.moe_expert_up_fp8(by(s), P, P, P, P, P + 4, P, P, P, None) == 4  # scale alignment
     assert lib.moe_expert_up_fp8(by(s), P, None, P, P, P, P, P, P, None) == 1
-    assert lib.moe_layer_fp8(by(s), P, P, None, P, P, P, P, P, None, P, None, None, P, 1024,
+    assert lib.moe_layer_fp8(by(s), P, P, None, P, P, P, P, P, P, None, P, None, None, P, 1024,
                              None) == 3
+    assert lib.moe_layer_fp8(by(s), P, P, None, P, P, P, P, P, None, None, P, None, None, P,
+                             1 << 30, None) == 1  # no W2 scales
     assert lib.moe_affinity_accumulate(10, 8, 9, P, P, P, None) == 1
     assert lib.moe_affinity_accumulate(10, 300, 2, P, P, P, None) == 2
     assert lib.moe_debug_bounded_wait(0, None) == 1
