@@ -259,41 +259,88 @@ __device__ __forceinline__ void decode_tile(int tile, const int *tile_start, con
     m = local - n * mt;
 }
 
-// Gate/up epilogue of one thread: accumulator row `row` (TMEM lane of this thread),
-// gate columns [0, 128) and up columns [128, 256) of N-slab n of expert e ->
-// 128 bf16 values of h. Mode 2 first scales the accumulators by the row scale and
-// the W1 / W3 output-channel scales.
-template <int MODE>
-__device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr, int e, int n,
-                                                int row, bool store)
+// The four epilogue warps (threads 64..191) of the FP8 modes meet at named barrier 1 once
+// per tile (after staging the tile's scales); every one of them passes it on every tile,
+// and all of them learn whether all of them are to go on, so none is left waiting there.
+__device__ __forceinline__ bool epilogue_all(bool v)
 {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.cta.red.and.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
+// Shared memory holding one tile's output-channel scales (FP8 modes), two tiles deep.
+constexpr int SCALE_STAGE_FLOATS = 2 * 256;
+constexpr int SCALE_STAGE_BYTES = SCALE_STAGE_FLOATS * 4 + 16;
+
+// Before a tile's accumulator is ready: its channel scales into ss (FP8 modes; the 128
+// epilogue threads copy them) and this thread's row scale into sx.
+template <int MODE, int BN>
+__device__ __forceinline__ void stage_scales(const Args &args, int e, int n, int row, bool valid,
+                                             float *ss, float &sx)
+{
+    if constexpr (is_e4m3(MODE)) {
+        const int t = (int)threadIdx.x - 64;
+        if constexpr (is_gate(MODE)) {  // 128 W1 then 128 W3 channels
+            const size_t base = (size_t)e * args.b_rows + n * 128;
+            ss[t] = args.b_scale0[base + t];
+            ss[128 + t] = args.b_scale1[base + t];
+        } else {  // BN W2 channels
+            const size_t base = (size_t)e * args.b_rows + n * BN;
+            for (int c = t; c < BN; c += 128)
+                ss[c] = args.b_scale0[base + c];
+        }
+        sx = valid ? args.row_scale[row] : 0.0f;
+    }
+}
+
+// Columns per TMEM round trip of the epilogue: the FP8 modes' shorter K loop leaves
+// the epilogue exposed, so they batch more loads per wait (measured: the bf16 modes are
+// fastest with the smaller batches).
+__host__ __device__ constexpr int epilogue_cols(int MODE)
+{
+    return MODE == 0 ? 16 : MODE == 1 ? 32 : MODE == 2 ? 32 : 64;
+}
+
+// Gate/up epilogue of one thread: accumulator row `row` (TMEM lane of this thread),
+// gate columns [0, 128) and up columns [128, 256) of N-slab n -> 128 bf16 values of h.
+// The FP8 mode first scales the accumulators by the row scale sx and the staged W1 / W3
+// channel scales ss.
+template <int MODE>
+__device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr, int n, int row,
+                                                bool store, float sx, const float *ss)
+{
+    constexpr int CB = epilogue_cols(MODE);
     uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.ldo;
     uint4 *dst = reinterpret_cast<uint4 *>(orow + n * 128);
-    float sx = 1.0f;
-    const float *s1 = nullptr, *s3 = nullptr;
-    if constexpr (MODE == 2) {
-        sx = store ? args.row_scale[row] : 0.0f;
-        s1 = args.b_scale0 + (size_t)e * args.b_rows + n * 128;
-        s3 = args.b_scale1 + (size_t)e * args.b_rows + n * 128;
-    }
 #pragma unroll 1
-    for (int c = 0; c < 128; c += 16) {
-        uint32_t g[16], u[16];
-        tmem_ld16(taddr + c, g);
-        tmem_ld16(taddr + 128 + c, u);
+    for (int c = 0; c < 128; c += CB) {
+        uint32_t g[CB], u[CB];
+#pragma unroll
+        for (int q = 0; q < CB / 16; ++q) {
+            tmem_ld16(taddr + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(g + 16 * q));
+            tmem_ld16(taddr + 128 + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(u + 16 * q));
+        }
         tmem_ld_wait();
         if (store) {
-            float gf[16], uf[16];
+            float gf[CB], uf[CB];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < CB; ++j) {
                 gf[j] = __uint_as_float(g[j]);
                 uf[j] = __uint_as_float(u[j]);
             }
             if constexpr (MODE == 2) {
 #pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 a = *reinterpret_cast<const float4 *>(s1 + c + j);
-                    const float4 b = *reinterpret_cast<const float4 *>(s3 + c + j);
+                for (int j = 0; j < CB; j += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(ss + c + j);
+                    const float4 b = *reinterpret_cast<const float4 *>(ss + 128 + c + j);
                     gf[j] *= sx * a.x;
                     gf[j + 1] *= sx * a.y;
                     gf[j + 2] *= sx * a.z;
@@ -304,45 +351,42 @@ __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr
                     uf[j + 3] *= sx * b.w;
                 }
             }
-            uint32_t p[8];
+            uint32_t p[CB / 2];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < CB / 2; ++j)
                 p[j] = pack_bf16x2(silu_mul(gf[2 * j], uf[2 * j]),
                                    silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
-            dst[c / 8] = make_uint4(p[0], p[1], p[2], p[3]);
-            dst[c / 8 + 1] = make_uint4(p[4], p[5], p[6], p[7]);
+#pragma unroll
+            for (int j = 0; j < CB / 8; ++j)
+                dst[c / 8 + j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
         }
     }
 }
 
 // Down-projection epilogue of one thread: accumulator row `row`, columns [0, BN) of
-// N-slab n -> fp32 y (not rounded before the combine). Mode 3 scales by the row scale
-// and the W2 output-channel scales.
+// N-slab n -> fp32 y (not rounded before the combine). The FP8 mode scales by the row
+// scale sx and the staged W2 channel scales ss.
 template <int MODE, int BN>
-__device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int e, int n,
-                                              int row, bool store)
+__device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int n, int row,
+                                              bool store, float sx, const float *ss)
 {
+    constexpr int CB = epilogue_cols(MODE);
     float *frow = reinterpret_cast<float *>(args.out) + (size_t)row * args.ldo;
     float4 *dst = reinterpret_cast<float4 *>(frow + n * BN);
-    float sx = 1.0f;
-    const float *s2 = nullptr;
-    if constexpr (MODE == 3) {
-        sx = store ? args.row_scale[row] : 0.0f;
-        s2 = args.b_scale0 + (size_t)e * args.b_rows + n * BN;
-    }
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-        uint32_t v[32];
-        tmem_ld16(taddr + c, *reinterpret_cast<uint32_t(*)[16]>(v));
-        tmem_ld16(taddr + c + 16, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+    for (int c = 0; c < BN; c += CB) {
+        uint32_t v[CB];
+#pragma unroll
+        for (int q = 0; q < CB / 16; ++q)
+            tmem_ld16(taddr + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * q));
         tmem_ld_wait();
         if (store) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int j = 0; j < CB; j += 4) {
                 float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
                                        __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
                 if constexpr (MODE == 3) {
-                    const float4 sc = *reinterpret_cast<const float4 *>(s2 + c + j);
+                    const float4 sc = *reinterpret_cast<const float4 *>(ss + c + j);
                     o.x *= sx * sc.x;
                     o.y *= sx * sc.y;
                     o.z *= sx * sc.z;
@@ -376,6 +420,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *tile_start = reinterpret_cast<int *>(tmem_slot + 4);
     int *mtiles = tile_start + (args.E + 1);
+    float *scale_stage = reinterpret_cast<float *>(
+        (reinterpret_cast<uintptr_t>(mtiles + args.E) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t smem_base = smem_u32(smem);
@@ -528,24 +574,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             int e, n, m;
             decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
             const int rows_e = args.offsets[e + 1] - args.offsets[e];
             const int valid = min(BM, rows_e - m * BM);
             const int row0 = args.offsets[e] + m * BM;
+            float *ss = scale_stage + (it & 1) * 256;
+            float sx = 1.0f;
+            stage_scales<MODE, BN>(args, e, n, row0 + r, r < valid, ss, sx);
             int ok = 0;
             if (lane == 0)
                 ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.timeout_ns) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok)
+            if constexpr (is_e4m3(MODE)) {
+                if (!epilogue_all(ok != 0))  // also publishes the staged scales
+                    break;
+            } else if (!ok) {
                 break;
+            }
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             if (GATE) {
-                swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
+                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
             } else {
-                down_epilogue<MODE, BN>(args, taddr, e, n, row0 + r, r < valid);
+                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss);
             }
             tc_fence_before();
             __syncwarp();
@@ -669,6 +723,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *tile_start = reinterpret_cast<int *>(tmem_slot + 4);
     int *mtiles = tile_start + (args.E + 1);
+    float *scale_stage = reinterpret_cast<float *>(
+        (reinterpret_cast<uintptr_t>(mtiles + args.E) + 15) & ~uintptr_t(15));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -827,24 +883,32 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int r = q * 32 + lane;
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = pair; tile < total; tile += npairs) {
+        int it = 0;
+        for (int tile = pair; tile < total; tile += npairs, ++it) {
             int e, n, m;
             decode_tile(tile, tile_start, mtiles, E, args.n_tiles, e, n, m);
             const int rows_e = args.offsets[e + 1] - args.offsets[e];
             const int valid = min(128, rows_e - m * BMP - (int)rank * 128);
             const int row0 = args.offsets[e] + m * BMP + (int)rank * 128;
+            float *ss = scale_stage + (it & 1) * 256;
+            float sx = 1.0f;
+            stage_scales<MODE, BN>(args, e, n, row0 + r, r < valid, ss, sx);
             int ok = 0;
             if (lane == 0)
                 ok = mbar_wait(tfull_bar(acc), acc_phase, abort_flag, args.timeout_ns) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok)
+            if constexpr (is_e4m3(MODE)) {
+                if (!epilogue_all(ok != 0))  // also publishes the staged scales
+                    break;
+            } else if (!ok) {
                 break;
+            }
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             if (GATE) {
-                swiglu_epilogue<MODE>(args, taddr, e, n, row0 + r, r < valid);
+                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
             } else {
-                down_epilogue<MODE, BN>(args, taddr, e, n, row0 + r, r < valid);
+                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss);
             }
             tc_fence_before();
             __syncwarp();
@@ -875,14 +939,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 constexpr int smem_bytes_pair(int E)
 {
-    return STAGES2 * STAGE2_BYTES + 1024 + 8 * (2 * STAGES2 + 5) + 16 + 8 * (E + 1) + 64;
+    return STAGES2 * STAGE2_BYTES + 1024 + 8 * (2 * STAGES2 + 5) + 16 + 8 * (E + 1) + 64 +
+           SCALE_STAGE_BYTES;
 }
 
 template <int MODE, int BN>
 constexpr int smem_bytes(int E)
 {
     return STAGES * (A_BYTES + BN * BK * 2) + 1024 /* alignment */ + 8 * (2 * STAGES + 5) +
-           16 + 8 * (E + 1) + 64;
+           16 + 8 * (E + 1) + 64 + SCALE_STAGE_BYTES;
 }
 
 }  // namespace gg

@@ -86,6 +86,8 @@ WORKLOADS = {
     # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
     "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,
                                      W=4, router="uniform"),
+    "mixtral_prefill_half_fp8": Workload("mixtral_prefill_half_fp8", N=2048, d=4096, f=14336,
+                                         E=4, K=2, W=4, router="uniform", fp8=True),
 }
 
 STACK_GRID_CF = (1.0, 1.25, 2.0)
