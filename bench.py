@@ -93,29 +93,74 @@ def aggregate(tokens_per_rank: float, elapsed_s: float, device=None) -> dict:
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks, power and throttle reasons while running: through NVML every
+    10 ms in a thread (read-only queries), else with nvidia-smi every 100 ms."""
 
+    # NVML clock-event reason bits
+    REASON_BITS = (("sw_power_cap", 0x4), ("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+                   ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80))
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
+        self.rows = []
         self.proc = None
-        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+        self.thread = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        try:  # the CUDA device by its PCI address (CUDA and NVML may number GPUs differently)
+            p = torch.cuda.get_device_properties(self.gpu_index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu_index)
+
+    def _poll(self, nv, h):
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.rows.append(dict(sm=float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                      smax=float(smax),
+                                      power=nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                      reasons={n for n, bit in self.REASON_BITS if reasons & bit}))
+            except Exception:
+                pass
+            self.stop.wait(0.01)
 
     def __enter__(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            return self
+        except Exception:
+            self.thread = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
                  "-i", str(self.gpu_index), "-lms", "100"], stdout=self.fh,
                 stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi, 100 ms"
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -123,61 +168,69 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.fh.close()
+            self._read_smi()
 
-    def summary(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
+    def _read_smi(self):
         with open(self.path) as fh:
             for line in fh:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
-                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
-                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
-                                     hw=parts[5], hwt=parts[6], swt=parts[7], cap=parts[8]))
+                    flags = {name for name, v in (("hw_slowdown", parts[5]),
+                                                  ("hw_thermal_slowdown", parts[6]),
+                                                  ("sw_thermal_slowdown", parts[7]),
+                                                  ("sw_power_cap", parts[8]))
+                             if v.lower() == "active"}
+                    self.rows.append(dict(sm=float(parts[1]), smax=float(parts[2]),
+                                          power=float(parts[3]) if parts[3] not in ("[N/A]", "")
+                                          else 0.0, reasons=flags))
                 except ValueError:
                     continue
         try:
             os.remove(self.path)
         except OSError:
             pass
+
+    def summary(self) -> dict:
+        rows = self.rows
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
+                    "source": self.source}
         load = [r for r in rows if r["power"] > 300.0] or rows
-        reasons = []
-        for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
-                          ("swt", "sw_thermal_slowdown"), ("cap", "sw_power_cap")):
-            if any(r[key].lower() == "active" for r in load):
-                reasons.append(name)
+        reasons = sorted(set().union(*(r["reasons"] for r in load)))
         return {"sm_mhz": statistics.median(r["sm"] for r in load),
                 "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
-                "samples": len(rows), "samples_under_load": len(load)}
+                "samples": len(rows), "samples_under_load": len(load), "source": self.source}
 
 
 # --------------------------------------------------------------------------- GPU arm
 
-# DRAM bytes per launch of the gate/up grouped GEMM, from the ncu capture summarised in
-# profiles/grouped_gemm_up_mixtral_prefill_half_full.md (half-size case, scaled x2 to the
-# full layer). Valid only for the kernel source it was measured on.
+# DRAM bytes per launch of the gate/up grouped GEMM at full size, from ncu captures of the
+# half-size cases (scaled x2: weights, rows and h all double), summarised in profiles/.
+# A figure holds only for the kernel source it was measured on (sha256 of grouped_gemm.cuh).
 MEASURED_UP_TRAFFIC = {
-    "kernel_sha256": "54dfe99065095ff871fae763340a72a193664460a2c77a1c3ae16b43d8216790",
-    "workload": "mixtral_prefill",
-    "bytes": 2206.8e6,
+    # workload: (kernel source sha256, bytes per launch)
+    "mixtral_prefill": ("d2ac64b6aad83395de3cdc67273b75efa558f213bed65c11a72745ad27e8530d",
+                        2 * (1015.3e6 + 117.4e6)),
+    "mixtral_prefill_fp8": ("d2ac64b6aad83395de3cdc67273b75efa558f213bed65c11a72745ad27e8530d",
+                            2 * (487.7e6 + 106.1e6)),
 }
 
 
 def up_traffic(workload: str):
+    sha_ref, nbytes = MEASURED_UP_TRAFFIC.get(workload, (None, None))
+    if sha_ref is None:
+        return None
     path = os.path.join(ROOT, "combine_grouped_gemm_router_b200", "csrc", "grouped_gemm.cuh")
     try:
         with open(path, "rb") as fh:
             sha = hashlib.sha256(fh.read()).hexdigest()
     except OSError:
         return None
-    if sha == MEASURED_UP_TRAFFIC["kernel_sha256"] and workload == MEASURED_UP_TRAFFIC["workload"]:
-        return MEASURED_UP_TRAFFIC["bytes"]
-    return None
+    return nbytes if sha == sha_ref else None
 
 
 def algorithmic_work(w, R: int) -> dict:
