@@ -264,8 +264,8 @@ def run_gpu(args, w) -> dict:
     # one step = the whole stack of w.layers layers (one layer unless the workload is a stack)
     L = w.layers
     shared = w.shared_f > 0
-    if w.fp8 and (w.reroute or shared or w.layers > 1):
-        raise ValueError("the FP8 payload is benchmarked on single plain layers")
+    if w.fp8 and (w.reroute or shared):
+        raise ValueError("the FP8 path is benchmarked without re-routing or a shared MLP")
     layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
               for l in range(L)]
     inp = layers[0]
@@ -472,7 +472,7 @@ def run_gpu(args, w) -> dict:
                 m.moe_layer_shared(shape, w.shared_f, x_dev[b], l0["w_router"], l0["bias"],
                                    l0["w1"], l0["w3"], l0["w2"], sh["ws1"], sh["ws3"], sh["ws2"],
                                    out_dev[b], ws=lws, stream=stream)
-            elif w.fp8:
+            elif w.fp8 and L == 1:
                 m.moe_layer_fp8(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1q"],
                                 l0["w1s"], l0["w3q"], l0["w3s"], l0["w2q"], l0["w2s"], out_dev[b],
                                 ws=lws, stream=stream)
@@ -484,8 +484,13 @@ def run_gpu(args, w) -> dict:
                 for l in range(L):
                     lw = layers[l]
                     dst = out_dev[b] if l == L - 1 else mid[l % 2]
-                    m.moe_layer(shape, xin, lw["w_router"], lw["bias"], lw["w1"], lw["w3"],
-                                lw["w2"], dst, residual=xin, ws=lws, stream=stream)
+                    if w.fp8:
+                        m.moe_layer_fp8(shape, xin, lw["w_router"], lw["bias"], lw["w1q"],
+                                        lw["w1s"], lw["w3q"], lw["w3s"], lw["w2q"], lw["w2s"], dst,
+                                        residual=xin, ws=lws, stream=stream)
+                    else:
+                        m.moe_layer(shape, xin, lw["w_router"], lw["bias"], lw["w1"], lw["w3"],
+                                    lw["w2"], dst, residual=xin, ws=lws, stream=stream)
                     xin = dst
             ev_comp[b].record(stream)
             s_out.wait_event(ev_comp[b])

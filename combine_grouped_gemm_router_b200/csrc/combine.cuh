@@ -15,19 +15,26 @@ namespace moe {
 // the shared MLP's and the routed experts' outputs) and a bf16 residual row (the
 // inter-layer step of a stack of MoE layers, x_{j+1} = x_j + MoE_j(x_j)). The
 // result is stored as fp32, or rounded once to bf16 (OUT_BF16).
+// A warp's work item is one token and `seg` 8-column chunks of its row (the whole
+// row for large N; a slice when there are too few tokens to fill the GPU).
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(256)
     combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ row_of,
                    const float *__restrict__ topk_w, const float *__restrict__ shared_y,
-                   const uint16_t *__restrict__ residual, int N, int d, int K,
+                   const uint16_t *__restrict__ residual, int N, int d, int K, int seg,
                    void *__restrict__ out)
 {
     constexpr int U = 2;
     const int lane = threadIdx.x & 31;
     const int nvec = d >> 3;  // 8-column chunks
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int nseg = (nvec + seg - 1) / seg;
+    const int64_t items = (int64_t)N * nseg;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     const float4 *ysrc = reinterpret_cast<const float4 *>(y);
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < N; t += nwarps) {
+    for (int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         item < items; item += nwarps) {
+        const int t = (int)(item / nseg);
+        const int cbeg = (int)(item % nseg) * seg, cend = min(nvec, cbeg + seg);
         int r = -1;
         float w = 0.0f;
         if (lane < K) {
@@ -35,7 +42,7 @@ __global__ void __launch_bounds__(256)
             w = topk_w[(size_t)t * K + lane];
         }
         // every lane runs every iteration: the shuffles below read lanes 0..K-1
-        for (int c0 = 0; c0 < nvec; c0 += 32 * U) {
+        for (int c0 = cbeg; c0 < cend; c0 += 32 * U) {
             const int c = c0 + lane;
             float acc[U][8];
 #pragma unroll
@@ -51,13 +58,13 @@ __global__ void __launch_bounds__(256)
                 float4 v[U][2];
 #pragma unroll
                 for (int u = 0; u < U; ++u)
-                    if (c + 32 * u < nvec) {
+                    if (c + 32 * u < cend) {
                         v[u][0] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2];
                         v[u][1] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2 + 1];
                     }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < nvec) {
+                    if (c + 32 * u < cend) {
                         const float f8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
                                              v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
 #pragma unroll
@@ -70,7 +77,7 @@ __global__ void __launch_bounds__(256)
                 const float4 *ssrc = reinterpret_cast<const float4 *>(shared_y);
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < nvec) {
+                    if (c + 32 * u < cend) {
                         const size_t chunk = (size_t)t * nvec + c + 32 * u;
                         const float4 a = ssrc[chunk * 2], b = ssrc[chunk * 2 + 1];
                         const float f8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -84,7 +91,7 @@ __global__ void __launch_bounds__(256)
                 const uint4 *rsrc = reinterpret_cast<const uint4 *>(residual);
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < nvec) {
+                    if (c + 32 * u < cend) {
                         const uint4 rv = rsrc[(size_t)t * nvec + c + 32 * u];
                         const uint32_t q4[4] = {rv.x, rv.y, rv.z, rv.w};
 #pragma unroll
@@ -97,7 +104,7 @@ __global__ void __launch_bounds__(256)
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (c + 32 * u < nvec) {
+                if (c + 32 * u < cend) {
                     const size_t chunk = (size_t)t * nvec + c + 32 * u;
                     if (OUT_BF16) {
                         uint4 o;

@@ -470,6 +470,7 @@ struct ScatterArgs {
     int nseg;        // all rounds
     int nseg_round;
     int32_t *expert_of;  // nullable out: the expert whose row each assignment uses, or -1
+    int seg;             // bf16 scatter: 16-byte chunks per work item (whole row for large N)
     void *x_sorted;      // bf16 rows, or e4m3 rows with fp8 payload
     void *x_packed;      // nullable, same element type
     float *sorted_scale;  // e4m3 payload: scale of each x_sorted row
@@ -478,11 +479,13 @@ struct ScatterArgs {
 };
 
 // Targets of slot `lane` (lanes < K) of token t: its expert-sorted row r (-1 if
-// dropped) and packed row pk (-1 if dropped or not packing); also writes
-// expert_of and returns the number of distinct non-home destination ranks of the
-// token (the same value in every lane), when counting.
+// dropped) and packed row pk (-1 if dropped or not packing). When `first` (the
+// token's first work item): also writes expert_of and returns the number of
+// distinct non-home destination ranks of the token (the same value in every lane),
+// when counting.
 __device__ __forceinline__ int slot_targets(const ScatterArgs &p, int t, int lane,
-                                            unsigned lt_mask, int &r, long long &pk)
+                                            unsigned lt_mask, int &r, long long &pk,
+                                            bool first = true)
 {
     const int e_per = p.E / p.W;
     const int home = t / p.S;
@@ -504,10 +507,10 @@ __device__ __forceinline__ int slot_targets(const ScatterArgs &p, int t, int lan
                 pk = p.pk_base[(size_t)e * p.nseg + g] + (r - p.offsets[e]);
             }
         }
-        if (p.expert_of)
+        if (p.expert_of && first)
             p.expert_of[a] = ef;
     }
-    if (!p.stats)
+    if (!p.stats || !first)
         return 0;
     // distinct non-home destinations: count the lowest lane of each group
     const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
@@ -515,33 +518,40 @@ __device__ __forceinline__ int slot_targets(const ScatterArgs &p, int t, int lan
     return __popc(__ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0));
 }
 
-// One warp per token: read the token's row once (16-byte loads), write it to
-// each kept slot's expert-sorted row and, when requested, to its packed row.
-// The token's distinct destination ranks other than its home (over kept slots)
-// are counted into stats->dedup_pairs.
+// One warp per work item (a token and `seg` 16-byte chunks of its row: the whole
+// row unless there are too few tokens to fill the GPU): read the token's row once
+// (16-byte loads), write it to each kept slot's expert-sorted row and, when
+// requested, to its packed row. The token's distinct destination ranks other than
+// its home (over kept slots) are counted into stats->dedup_pairs.
 __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
 {
     constexpr int U = 4;
     const int lane = threadIdx.x & 31;
     const int nvec = p.d >> 3;
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const int nseg = (nvec + p.seg - 1) / p.seg;
+    const int64_t items = (int64_t)p.N * nseg;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
     unsigned lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     unsigned long long pairs = 0;
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
+    for (int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+         item < items; item += nwarps) {
+        const int t = (int)(item / nseg);
+        const int sidx = (int)(item % nseg);
+        const int cbeg = sidx * p.seg, cend = min(nvec, cbeg + p.seg);
         int r;
         long long pk;
-        pairs += slot_targets(p, t, lane, lt_mask, r, pk);
+        pairs += slot_targets(p, t, lane, lt_mask, r, pk, sidx == 0);
         const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
         uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
         uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
         // every lane runs every iteration: the shuffles below read lanes 0..K-1
-        for (int c0 = 0; c0 < nvec; c0 += 32 * U) {
+        for (int c0 = cbeg; c0 < cend; c0 += 32 * U) {
             const int c = c0 + lane;
             uint4 v[U];
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (c + 32 * u < nvec)
+                if (c + 32 * u < cend)
                     v[u] = __ldcs(src + c + 32 * u);
             for (int k = 0; k < p.K; ++k) {
                 const int rk = __shfl_sync(0xffffffffu, r, k);
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
                     continue;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < nvec) {
+                    if (c + 32 * u < cend) {
                         dst_s[(size_t)rk * nvec + c + 32 * u] = v[u];
                         if (pkk >= 0)
                             dst_p[(size_t)pkk * nvec + c + 32 * u] = v[u];

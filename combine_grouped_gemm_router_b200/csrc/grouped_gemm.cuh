@@ -133,6 +133,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// 2-D tiled bulk store shared -> global (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// This thread's bulk stores have finished reading shared memory / have completed.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before()
 {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -363,14 +380,24 @@ __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr
     }
 }
 
+// Per epilogue warp of the down-projection modes: a 32-row x 32-column fp32 tile in
+// shared memory (4 KB, 128-byte swizzled as the y tensor map expects), stored by TMA.
+constexpr int Y_STAGE_BYTES = 4 * 4096 + 1024;
+
 // Down-projection epilogue of one thread: accumulator row `row`, columns [0, BN) of
 // N-slab n -> fp32 y (not rounded before the combine). The FP8 mode scales by the row
-// scale sx and the staged W2 channel scales ss.
+// scale sx and the staged W2 channel scales ss. When all 32 rows of this warp belong to
+// the expert (wfull), each 32-column piece goes through the warp's shared-memory tile
+// (ystage) and one TMA store of 32 x 32 at (x = column, y = wrow0); otherwise every
+// thread stores its own row's values directly (no row past the expert is written).
 template <int MODE, int BN>
 __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int n, int row,
-                                              bool store, float sx, const float *ss)
+                                              bool store, float sx, const float *ss,
+                                              const CUtensorMap *ymap, uint32_t ystage,
+                                              int wrow0, bool wfull)
 {
     constexpr int CB = epilogue_cols(MODE);
+    const int lane = threadIdx.x & 31;
     float *frow = reinterpret_cast<float *>(args.out) + (size_t)row * args.ldo;
     float4 *dst = reinterpret_cast<float4 *>(frow + n * BN);
 #pragma unroll 1
@@ -380,7 +407,35 @@ __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, 
         for (int q = 0; q < CB / 16; ++q)
             tmem_ld16(taddr + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * q));
         tmem_ld_wait();
-        if (store) {
+        if (wfull) {
+#pragma unroll
+            for (int h = 0; h < CB / 32; ++h) {
+                if (lane == 0)
+                    bulk_wait_read();  // the previous piece has left the tile
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int k = 32 * h + 4 * j;
+                    float4 o = make_float4(__uint_as_float(v[k]), __uint_as_float(v[k + 1]),
+                                           __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+                    if constexpr (MODE == 3) {
+                        const float4 sc = *reinterpret_cast<const float4 *>(ss + c + k);
+                        o.x *= sx * sc.x;
+                        o.y *= sx * sc.y;
+                        o.z *= sx * sc.z;
+                        o.w *= sx * sc.w;
+                    }
+                    const uint32_t addr = ystage + lane * 128 + ((j ^ (lane & 7)) << 4);
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(o.x),
+                                 "f"(o.y), "f"(o.z), "f"(o.w)
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    tma_store_2d(ymap, ystage, n * BN + c + 32 * h, wrow0);
+            }
+        } else if (store) {
 #pragma unroll
             for (int j = 0; j < CB; j += 4) {
                 float4 o = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
@@ -422,6 +477,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     int *mtiles = tile_start + (args.E + 1);
     float *scale_stage = reinterpret_cast<float *>(
         (reinterpret_cast<uintptr_t>(mtiles + args.E) + 15) & ~uintptr_t(15));
+    // down-projection modes: 4 warp tiles of 4 KB, 1024-byte aligned (128-byte swizzle)
+    const uint32_t y_stage = (smem_u32(scale_stage + SCALE_STAGE_FLOATS) + 1023u) & ~1023u;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t smem_base = smem_u32(smem);
@@ -599,7 +656,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (GATE) {
                 swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
             } else {
-                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss);
+                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss, &tmB1,
+                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32);
             }
             tc_fence_before();
             __syncwarp();
@@ -611,6 +669,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
 
+    if (!is_gate(MODE) && warp >= 2 && lane == 0)
+        bulk_wait_all();  // this warp's y stores are complete before its shared memory goes
     __syncwarp();
     tc_fence_before();
     __syncthreads();
@@ -725,6 +785,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     int *mtiles = tile_start + (args.E + 1);
     float *scale_stage = reinterpret_cast<float *>(
         (reinterpret_cast<uintptr_t>(mtiles + args.E) + 15) & ~uintptr_t(15));
+    // down-projection modes: 4 warp tiles of 4 KB, 1024-byte aligned (128-byte swizzle)
+    const uint32_t y_stage = (smem_u32(scale_stage + SCALE_STAGE_FLOATS) + 1023u) & ~1023u;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -908,7 +970,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (GATE) {
                 swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
             } else {
-                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss);
+                down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss, &tmB1,
+                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32);
             }
             tc_fence_before();
             __syncwarp();
@@ -920,6 +983,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
 
+    if (!is_gate(MODE) && warp >= 2 && lane == 0)
+        bulk_wait_all();  // this warp's y stores are complete before its shared memory goes
     __syncwarp();
     tc_fence_before();
     if (*abort_flag) {
@@ -937,17 +1002,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                      : "memory");
 }
 
+template <int MODE>
 constexpr int smem_bytes_pair(int E)
 {
     return STAGES2 * STAGE2_BYTES + 1024 + 8 * (2 * STAGES2 + 5) + 16 + 8 * (E + 1) + 64 +
-           SCALE_STAGE_BYTES;
+           SCALE_STAGE_BYTES + (is_gate(MODE) ? 0 : Y_STAGE_BYTES);
 }
 
 template <int MODE, int BN>
 constexpr int smem_bytes(int E)
 {
     return STAGES * (A_BYTES + BN * BK * 2) + 1024 /* alignment */ + 8 * (2 * STAGES + 5) +
-           16 + 8 * (E + 1) + 64 + SCALE_STAGE_BYTES;
+           16 + 8 * (E + 1) + 64 + SCALE_STAGE_BYTES + (is_gate(MODE) ? 0 : Y_STAGE_BYTES);
 }
 
 }  // namespace gg

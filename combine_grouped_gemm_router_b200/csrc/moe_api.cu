@@ -188,6 +188,22 @@ int num_sms()
     return n;
 }
 
+// Warp work items of the row kernels (combine, bf16 scatter): a whole token row each
+// when there are enough tokens to fill the GPU, else slices of `slice` chunks, so that a
+// decode batch of a few tokens still spreads over every SM.
+int row_slice(int N, int nchunks, int slice)
+{
+    return N >= 8 * num_sms() ? nchunks : slice;
+}
+
+int row_blocks(int N, int nchunks, int seg)
+{
+    const int64_t items = (int64_t)N * ((nchunks + seg - 1) / seg);
+    const int64_t blocks = (items + 7) / 8;
+    return (int)(blocks < 64 * num_sms() ? blocks : 64 * num_sms());
+}
+
+
 inline moe_status_t launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -360,10 +376,13 @@ moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16
     ca.sorted_scale = pay.sorted_scale;
     ca.packed_scale = pay.packed_scale;
     ca.stats = stats;
-    if (pay.e4m3)
+    if (pay.e4m3) {
+        ca.seg = s->d / 8;  // one token row per warp (its maximum is taken over the row)
         scatter_rows_e4m3_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
-    else
-        scatter_rows_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
+    } else {
+        ca.seg = row_slice(s->N, s->d / 8, 128);
+        scatter_rows_kernel<<<row_blocks(s->N, s->d / 8, ca.seg), 256, 0, st>>>(ca);
+    }
     return launch_status();
 }
 
@@ -403,6 +422,23 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, b
     return r == CUDA_SUCCESS;
 }
 
+// The down projection's output y [rows][inner] fp32 as a store target: box 32 rows x 32
+// columns (128 bytes), 128-byte swizzle (the epilogue's shared-memory tile layout).
+bool make_tmap_y(CUtensorMap *m, float *ptr, uint64_t inner, uint64_t rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int MODE, int BN>
 moe_status_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1,
                          const gg::Args &args, cudaStream_t st)
@@ -426,7 +462,7 @@ template <int MODE>
 moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1,
                               const gg::Args &args, cudaStream_t st)
 {
-    const int smem = gg::smem_bytes_pair(kMaxE);
+    const int smem = gg::smem_bytes_pair<MODE>(kMaxE);
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     static int pairs = 0;
@@ -515,8 +551,9 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
 moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
                        const int32_t *offsets, const uint16_t *w2, float *y, cudaStream_t st)
 {
-    CUtensorMap tA, tW2;
-    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
+    CUtensorMap tA, tW2, tY;
+    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d) ||
+        !make_tmap_y(&tY, y, d, (uint64_t)a_rows))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -532,15 +569,15 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
         args.n_tiles = d / 256;
         if (pair) {
             args.select = 1;
-            moe_status_t rc = launch_gemm_pair<1>(tA, tW2, tW2, args, st);
+            moe_status_t rc = launch_gemm_pair<1>(tA, tW2, tY, args, st);
             if (rc != MOE_OK)
                 return rc;
             args.select = 2;
         }
-        return launch_gemm<1, 256>(tA, tW2, tW2, args, st);
+        return launch_gemm<1, 256>(tA, tW2, tY, args, st);
     }
     args.n_tiles = d / 128;
-    return launch_gemm<1, 128>(tA, tW2, tW2, args, st);
+    return launch_gemm<1, 128>(tA, tW2, tY, args, st);
 }
 
 // Gate/up on the FP8 payload: e4m3 rows of x (scale per row) and e4m3 rows of W1, W3
@@ -586,9 +623,9 @@ moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, cons
                             const float *h_scale, const int32_t *offsets, const uint8_t *w2,
                             const float *s2, float *y, cudaStream_t st)
 {
-    CUtensorMap tA, tW2;
+    CUtensorMap tA, tW2, tY;
     if (!make_tmap(&tA, hq, f, (uint64_t)a_rows, true) ||
-        !make_tmap(&tW2, w2, f, (uint64_t)E * d, true))
+        !make_tmap(&tW2, w2, f, (uint64_t)E * d, true) || !make_tmap_y(&tY, y, d, (uint64_t)a_rows))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -606,15 +643,15 @@ moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, cons
         args.n_tiles = d / 256;
         if (pair && args.k_blocks % gg::KA2 == 0) {
             args.select = 1;
-            moe_status_t rc = launch_gemm_pair<3>(tA, tW2, tW2, args, st);
+            moe_status_t rc = launch_gemm_pair<3>(tA, tW2, tY, args, st);
             if (rc != MOE_OK)
                 return rc;
             args.select = 2;
         }
-        return launch_gemm<3, 256>(tA, tW2, tW2, args, st);
+        return launch_gemm<3, 256>(tA, tW2, tY, args, st);
     }
     args.n_tiles = d / 128;
-    return launch_gemm<3, 128>(tA, tW2, tW2, args, st);
+    return launch_gemm<3, 128>(tA, tW2, tY, args, st);
 }
 
 // Row-wise e4m3 quantisation launch; rows_dev (nullable, device) caps the row count.
@@ -675,12 +712,15 @@ moe_status_t combine_impl(const moe_shape_t *s, const float *y, const int32_t *r
                           const float *topk_w, const float *shared_y, const uint16_t *residual,
                           void *out, cudaStream_t st)
 {
+    const int nvec = s->d / 8;
+    const int seg = row_slice(s->N, nvec, 64);
+    const int blocks = row_blocks(s->N, nvec, seg);
     if (s->flags & MOE_FLAG_OUT_BF16)
-        combine_kernel<true><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, shared_y,
-                                                              residual, s->N, s->d, s->K, out);
+        combine_kernel<true><<<blocks, 256, 0, st>>>(y, row_of, topk_w, shared_y, residual, s->N,
+                                                      s->d, s->K, seg, out);
     else
-        combine_kernel<false><<<(s->N + 7) / 8, 256, 0, st>>>(y, row_of, topk_w, shared_y,
-                                                               residual, s->N, s->d, s->K, out);
+        combine_kernel<false><<<blocks, 256, 0, st>>>(y, row_of, topk_w, shared_y, residual, s->N,
+                                                       s->d, s->K, seg, out);
     return launch_status();
 }
 

@@ -82,6 +82,10 @@ WORKLOADS = {
                                     W=8, router="uniform", fp8=True),
     "e128_skew_fp8": Workload("e128_skew_fp8", N=8192, d=2048, f=768, E=128, K=8, W=8, cf=1.25,
                               s=1.1, fp8=True),
+    # the weight-bound decode layer and the 4-layer stack on the FP8 path
+    "decode_fp8": Workload("decode_fp8", N=16, d=7168, f=2048, E=256, K=8, W=8, fp8=True),
+    "stack4_fp8": Workload("stack4_fp8", N=32768, d=4096, f=1536, E=64, K=6, W=8, cf=1.25,
+                           layers=4, fp8=True),
     # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
     # same GEMM tiles): a smaller case of the same kernels, for hardware-counter captures
     "mixtral_prefill_half": Workload("mixtral_prefill_half", N=2048, d=4096, f=14336, E=4, K=2,
