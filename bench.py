@@ -233,12 +233,16 @@ def up_traffic(workload: str):
     return nbytes if sha == sha_ref else None
 
 
-def algorithmic_work(w, R: int) -> dict:
-    """Algorithmic flops and bytes per launch of each stage (see the design notes)."""
+def algorithmic_work(w, R: int, E_act: int) -> dict:
+    """Algorithmic flops and bytes per launch of each stage (see the design notes);
+    E_act = experts with at least one kept row (only their weights are read)."""
     N, d, f, E, K = w.N, w.d, w.f, w.E, w.K
+    eb = 1 if w.fp8 else 2  # bytes per GEMM operand element
     return dict(
         up_flops=4.0 * d * f * R,
         down_flops=2.0 * d * f * R,
+        # gate/up: W1 and W3 of the active experts, the x_sorted rows, h written (bf16)
+        up_bytes=2.0 * E_act * f * d * eb + R * d * eb + R * f * 2,
         logits_bytes=N * d * 2 + E * d * 4 + N * E * 4,
         # scatter: read each token row once, write every kept row twice (sorted + packed)
         # (the FP8 payload writes one byte per element and a 4-byte scale per row)
@@ -436,6 +440,7 @@ def run_gpu(args, w) -> dict:
         del graph
     err = m.moe_get_device_error(True)
     R_layers = [int(o[E].item()) for o in offsets]
+    act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
     R = R_layers[0]
     agg = aggregate(float(N * args.steps), elapsed_s, dev)
 
@@ -522,8 +527,8 @@ def run_gpu(args, w) -> dict:
 
     # algorithmic work of one step (all layers of a stack)
     work = {}
-    for Rl in R_layers:
-        for k, v in algorithmic_work(w, Rl).items():
+    for Rl, Al in zip(R_layers, act_layers):
+        for k, v in algorithmic_work(w, Rl, Al).items():
             work[k] = work.get(k, 0.0) + v
     peaks = load_peaks()
     up_ratio = 2.0 if w.fp8 else 1.0  # e4m3 tensor throughput is twice bf16's (nominal)
@@ -536,6 +541,31 @@ def run_gpu(args, w) -> dict:
     stages = {k: round(v, 4) for k, v in stage_ms.items()}
     hbm = peaks["hbm_gbs"]
     comb_gbs = work["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
+    # the dominant kernel's roofline: tensor-bound when its flops per algorithmic byte exceed
+    # the machine balance (peak flops / copy bandwidth), else HBM-bound (decode, and layers
+    # with few rows per expert, stream weights)
+    up_gbs = work["up_bytes"] / up_s / 1e9
+    intensity = work["up_flops"] / work["up_bytes"]
+    balance = up_peak * 1e12 / (hbm * 1e9)
+    kernel_name = ("grouped GEMM gate/up on e4m3 (moe_expert_up_fp8, tcgen05 kind::f8f6f4)"
+                   if w.fp8 else "grouped GEMM gate/up (moe_expert_up, tcgen05)")
+    tensor_line = {"achieved": up_tflops, "peak": up_peak, "unit": "TFLOP/s",
+                   "frac": up_tflops / up_peak,
+                   "peak_source": (peaks["source"] + " bf16 burst x 2 (the nominal e4m3/bf16 "
+                                   "dense ratio)" if w.fp8 else peaks["source"] + " bf16 burst"),
+                   "frac_of_sustained": up_tflops / (peaks["bf16_tflops_sustained"] * up_ratio)}
+    hbm_line = {"achieved": up_gbs, "peak": hbm, "unit": "GB/s", "frac": up_gbs / hbm,
+                "peak_source": peaks["source"] + " copy bandwidth"}
+    roofline = {"kernel": kernel_name, "bound": "tensor" if intensity >= balance else "hbm"}
+    roofline.update(tensor_line if intensity >= balance else hbm_line)
+    roofline.update({"traffic": up_traffic(w.name),
+                     "algorithmic_flops_per_launch": work["up_flops"] / L,
+                     "algorithmic_bytes_per_launch": work["up_bytes"] / L,
+                     "flops_per_byte": intensity, "machine_balance": balance,
+                     "other_bound": ({"unit": "GB/s", "achieved": up_gbs, "frac": up_gbs / hbm}
+                                     if intensity >= balance else
+                                     {"unit": "TFLOP/s", "achieved": up_tflops,
+                                      "frac": up_tflops / up_peak})})
     res = {
         "metric": METRIC,
         "value": agg["value"],
@@ -558,17 +588,7 @@ def run_gpu(args, w) -> dict:
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step"},
-        "roofline": {"kernel": ("grouped GEMM gate/up on e4m3 (moe_expert_up_fp8, tcgen05 "
-                                "kind::f8f6f4)" if w.fp8 else
-                                "grouped GEMM gate/up (moe_expert_up, CTA-pair tcgen05 kernel)"),
-                     "bound": "tensor",
-                     "achieved": up_tflops, "peak": up_peak, "unit": "TFLOP/s",
-                     "frac": up_tflops / up_peak,
-                     "peak_source": (peaks["source"] + " bf16 burst x 2 (the nominal e4m3/bf16 "
-                                     "dense ratio)" if w.fp8 else peaks["source"] + " bf16 burst"),
-                     "frac_of_sustained": up_tflops / (peaks["bf16_tflops_sustained"] * up_ratio),
-                     "traffic": up_traffic(w.name),
-                     "algorithmic_flops_per_launch": work["up_flops"] / L},
+        "roofline": roofline,
         "stages_ms": stages,
         "grouped_gemm": {"tflops": gemm_tflops, "frac_of_bf16_peak": gemm_tflops / peaks["bf16_tflops"],
                          "frac_of_bf16_sustained": gemm_tflops / peaks["bf16_tflops_sustained"]},
