@@ -211,12 +211,15 @@ class ClockSampler:
 # DRAM bytes per launch of the gate/up grouped GEMM at full size, from ncu captures of the
 # half-size cases (scaled x2: weights, rows and h all double), summarised in profiles/.
 # A figure holds only for the kernel source it was measured on (sha256 of grouped_gemm.cuh).
+_UP_SHA = "f61e56b8c311a8cfe4f71397b2cde337d17dda240cc229f238719f05b7eab2d7"
 MEASURED_UP_TRAFFIC = {
     # workload: (kernel source sha256, bytes per launch)
-    "mixtral_prefill": ("d2ac64b6aad83395de3cdc67273b75efa558f213bed65c11a72745ad27e8530d",
-                        2 * (1015.3e6 + 117.4e6)),
-    "mixtral_prefill_fp8": ("d2ac64b6aad83395de3cdc67273b75efa558f213bed65c11a72745ad27e8530d",
-                            2 * (487.7e6 + 106.1e6)),
+    "mixtral_prefill": (_UP_SHA, 2 * (996.6e6 + 113.1e6)),      # half-size capture x 2
+    "mixtral_prefill_fp8": (_UP_SHA, 2 * (488.0e6 + 105.0e6)),  # half-size capture x 2
+    "e128_skew": (_UP_SHA, 886.9e6 + 36.5e6),
+    "e128_skew_fp8": (_UP_SHA, 444.1e6 + 36.3e6),
+    "decode": (_UP_SHA, 6071.7e6 + 4.4e6),
+    "decode_fp8": (_UP_SHA, 3037.1e6 + 4.5e6),
 }
 
 
