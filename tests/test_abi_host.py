@@ -196,3 +196,10 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(ImportError):
         fresh.moe_abi_version()
     importlib.reload(mod)
+
+
+def test_graft_build_entry():
+    """The build entry point compiles (or finds current) the library and the oracle and checks
+    the library's ABI version against the binding's."""
+    import __graft_entry__
+    __graft_entry__.build()
