@@ -128,6 +128,45 @@ __device__ void block_excl_scan_i64(int64_t *a, int n, int64_t *s_warp)
     __syncthreads();
 }
 
+// Many blocks (slot-major priority, re-routing): one CTA per expert turns its row of
+// block counts into exclusive bases and records the expert's count at every segment start
+// (cum [E][nseg+1], cum[e][nseg] = total); dispatch_scan_kernel then skips that step.
+__global__ void __launch_bounds__(256)
+    expert_block_scan_kernel(int32_t *__restrict__ blk, int nvb, int bps, int nseg,
+                             int32_t *__restrict__ cum)
+{
+    __shared__ int s_warp[8];
+    const int e = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t *row = blk + (size_t)e * nvb;
+    const int per = (nvb + 255) / 256;
+    const int beg = min(nvb, (int)threadIdx.x * per), end = min(nvb, beg + per);
+    int local = 0;
+    for (int i = beg; i < end; ++i)
+        local += row[i];
+    const int incl = warp_incl_scan(local);
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < 8 ? s_warp[lane] : 0;
+        const int vi = warp_incl_scan(v);
+        if (lane < 8)
+            s_warp[lane] = vi - v;
+    }
+    __syncthreads();
+    int run = s_warp[warp] + incl - local;
+    for (int i = beg; i < end; ++i) {
+        const int v = row[i];
+        row[i] = run;
+        if (i % bps == 0)
+            cum[(size_t)e * (nseg + 1) + i / bps] = run;
+        run += v;
+    }
+    if (threadIdx.x == 255)
+        cum[(size_t)e * (nseg + 1) + nseg] = run;  // the last thread ends at the total
+}
+
 struct ScanArgs {
     int32_t *blk;  // [E][nvb] counts in, exclusive bases out
     int nvb;
@@ -137,6 +176,7 @@ struct ScanArgs {
     int N, E, K, W;
     int C;
     int32_t *cum_global;  // [E][nseg+1] when it does not fit in shared memory, else null
+    int prescanned;       // expert_block_scan_kernel has done step 1 into cum_global
     int32_t *counts, *kept, *offsets;
     int64_t *D;        // [W][W]
     int64_t *pk_off;   // [W*W+1]
@@ -167,7 +207,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
     int32_t *cum = p.cum_global ? p.cum_global : s_kh + E * W;
 
     // 1. per expert: exclusive scan over virtual blocks; record segment starts
-    for (int e = warp; e < E; e += NT / 32) {
+    for (int e = warp; e < E && !p.prescanned; e += NT / 32) {
         int32_t *row = p.blk + (size_t)e * nvb;
         int carry = 0;
         for (int base = 0; base < nvb; base += 128) {

@@ -108,9 +108,8 @@ size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layou
     o = align_up(o + (size_t)s->E * g.nvb * 4);
     L.pk_base = o;
     o = align_up(o + (size_t)s->E * g.nseg * 8);
-    L.cum = o;
-    if (!g.cum_in_smem)
-        o = align_up(o + scan_cum_bytes(s, g.nseg));
+    L.cum = o;  // the scan's segment starts, when not in shared memory or pre-scanned
+    o = align_up(o + scan_cum_bytes(s, g.nseg));
     L.moved = o;
     if (g.rounds > 1)
         o = align_up(o + (size_t)s->N * s->K * 4);
@@ -273,7 +272,12 @@ void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const in
     const int nvb = rounds * g.nvb_round, nseg = rounds * g.nseg_round;
     block_hist_kernel<<<nvb, 256, s->E * 4, st>>>(topk_idx, s->E, vbm, nvb, blk);
 
-    const bool cum_in_smem = scan_smem_base(s) + scan_cum_bytes(s, nseg) <= kScanSmemLimit;
+    // many blocks per expert: scan each expert's row in its own CTA first
+    const bool prescan = nvb > 128;
+    if (prescan)
+        expert_block_scan_kernel<<<s->E, 256, 0, st>>>(blk, nvb, g.bps, nseg, cum);
+    const bool cum_in_smem =
+        !prescan && scan_smem_base(s) + scan_cum_bytes(s, nseg) <= kScanSmemLimit;
     ScanArgs sa;
     sa.blk = blk;
     sa.nvb = nvb;
@@ -286,6 +290,7 @@ void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const in
     sa.W = s->W;
     sa.C = (int)g.C;
     sa.cum_global = cum_in_smem ? nullptr : cum;
+    sa.prescanned = prescan ? 1 : 0;
     sa.counts = counts;
     sa.kept = kept;
     sa.offsets = offsets;

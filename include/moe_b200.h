@@ -219,7 +219,7 @@ moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, c
  * inside the library. Every GPU that loads the library holds that array until the process
  * exits. The call allocates and frees nothing.
  *  - Shapes whose scratch does not fit (about E * W * ceil(N / (64 W)) * 4 bytes plus
- *    E * W * 8 + 2 * W * W * 8, the first two terms K times larger with MOE_FLAG_SLOT_MAJOR)
+ *    E * W * 12 + 2 * W * W * 8, the first two terms K times larger with MOE_FLAG_SLOT_MAJOR)
  *    return MOE_ERR_WORKSPACE_TOO_SMALL before any launch. MOE_FLAG_REROUTE is refused.
  *  - The first call on a device looks up the array's device address on that device (the
  *    device must be current); make that first call before any stream capture.
