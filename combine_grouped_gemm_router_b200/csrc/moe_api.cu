@@ -63,7 +63,7 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
         return MOE_ERR_INVALID_ARG;
     if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE)) != 0)
         return MOE_ERR_INVALID_ARG;
-    if (s->N < 1 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
+    if (s->N < 0 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
         return MOE_ERR_INVALID_ARG;
     if (s->K > s->E || s->E % s->W != 0 || s->N % s->W != 0)
         return MOE_ERR_INVALID_ARG;
@@ -729,6 +729,34 @@ moe_status_t combine_impl(const moe_shape_t *s, const float *y, const int32_t *r
     return launch_status();
 }
 
+// An empty batch (N = 0) is a valid call: nothing is launched, and the outputs indexed by
+// expert or rank (counts, kept, offsets, traffic matrix, pack offsets, counters) are zeroed.
+moe_status_t empty_dispatch(const moe_shape_t *s, int32_t *counts, int32_t *kept,
+                            int32_t *offsets, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
+                            cudaStream_t st)
+{
+    if (!counts || !kept || !offsets)
+        return MOE_ERR_INVALID_ARG;
+    const size_t E = (size_t)s->E, WW = (size_t)s->W * s->W;
+    bool ok = cudaMemsetAsync(counts, 0, E * 4, st) == cudaSuccess &&
+              cudaMemsetAsync(kept, 0, E * 4, st) == cudaSuccess &&
+              cudaMemsetAsync(offsets, 0, (E + 1) * 4, st) == cudaSuccess;
+    if (ok && D)
+        ok = cudaMemsetAsync(D, 0, WW * 8, st) == cudaSuccess;
+    if (ok && pk_off)
+        ok = cudaMemsetAsync(pk_off, 0, (WW + 1) * 8, st) == cudaSuccess;
+    if (ok && stats)
+        ok = cudaMemsetAsync(stats, 0, sizeof(moe_stats_t), st) == cudaSuccess;
+    return ok ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t empty_layer(moe_stats_t *stats, cudaStream_t st)
+{
+    if (stats && cudaMemsetAsync(stats, 0, sizeof(moe_stats_t), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -793,6 +821,8 @@ moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
     moe_status_t rc = check_shape(shape, false, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!x || !w_router || !topk_idx || !topk_w)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) ||
@@ -823,6 +853,9 @@ moe_status_t dispatch_entry(const moe_shape_t *shape, const uint16_t *x, const f
     moe_status_t rc = check_shape(shape, false, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return empty_dispatch(shape, counts, kept, offsets, rank_matrix, packed_offsets, stats,
+                              reinterpret_cast<cudaStream_t>(stream));
     if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row ||
         !pay.x_sorted)
         return MOE_ERR_INVALID_ARG;
@@ -884,7 +917,7 @@ moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, const float *l
                      int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
                      moe_stream_t stream)
 {
-    if (!shape || !(shape->flags & MOE_FLAG_REROUTE) || !logits)
+    if (!shape || !(shape->flags & MOE_FLAG_REROUTE) || (!logits && shape->N != 0))
         return MOE_ERR_INVALID_ARG;
     return dispatch_entry(shape, x, logits, topk_idx, counts, kept, offsets, row_of,
                           assign_of_row, expert_of,
@@ -934,6 +967,8 @@ moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted, const float
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!x_sorted || !sorted_scale || !offsets || !w1q || !w1_scale || !w3q || !w3_scale || !h)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x_sorted) || !aligned16(w1q) || !aligned16(w3q) || !aligned16(w1_scale) ||
@@ -953,6 +988,8 @@ moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!hq || !h_scale || !offsets || !w2q || !w2_scale || !y)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(hq) || !aligned16(w2q) || !aligned16(w2_scale) || !aligned16(y) ||
@@ -972,6 +1009,8 @@ moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!x_sorted || !offsets || !w1 || !w3 || !w2 || !h || !y)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x_sorted) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
@@ -989,6 +1028,8 @@ moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_t 
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!x_sorted || !offsets || !w1 || !w3 || !h)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x_sorted) || !aligned16(w1) || !aligned16(w3) || !aligned16(h) ||
@@ -1006,6 +1047,8 @@ moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offs
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!h || !offsets || !w2 || !y)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(w2) || !aligned16(y) || !aligned4(offsets))
@@ -1021,6 +1064,8 @@ moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
     moe_status_t rc = check_shape(shape, false, nullptr);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (!y || !row_of || !topk_w || !out)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(y) || !aligned16(out) || !aligned4(row_of) || !aligned4(topk_w) ||
@@ -1130,6 +1175,8 @@ moe_layer(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return empty_layer(stats, reinterpret_cast<cudaStream_t>(stream));
     if (!x || !w_router || !w1 || !w3 || !w2 || !out)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1) ||
@@ -1159,6 +1206,8 @@ moe_layer_fp8(const moe_shape_t *shape, const uint16_t *x, const float *w_router
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return empty_layer(stats, reinterpret_cast<cudaStream_t>(stream));
     if (!x || !w_router || !w1q || !w1_scale || !w3q || !w3_scale || !w2q || !w2_scale || !out)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) || !aligned16(w1q) ||
@@ -1188,6 +1237,8 @@ moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
     moe_status_t rc = check_shape(shape, true, nullptr);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return MOE_OK;  // empty batch: nothing to do
     if (f_shared < 128 || f_shared % 128 != 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!x || !ws1 || !ws3 || !ws2 || !h_s || !y_s)
@@ -1224,6 +1275,8 @@ moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
     moe_status_t rc = check_shape(shape, true, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return empty_layer(stats, reinterpret_cast<cudaStream_t>(stream));
     if (f_shared < 128 || f_shared % 128 != 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (!x || !w_router || !w1 || !w3 || !w2 || !ws1 || !ws3 || !ws2 || !out)
@@ -1249,7 +1302,11 @@ __attribute__((visibility("default"))) moe_status_t
 moe_affinity_accumulate(int32_t N, int32_t E, int32_t K, const int32_t *topk_j,
                         const int32_t *topk_j1, int64_t *counts, moe_stream_t stream)
 {
-    if (N < 1 || E < 1 || K < 1 || K > E || !topk_j || !topk_j1 || !counts)
+    if (N < 0 || E < 1 || K < 1 || K > E || !counts)
+        return MOE_ERR_INVALID_ARG;
+    if (N == 0)
+        return MOE_OK;  // no tokens: nothing to count
+    if (!topk_j || !topk_j1)
         return MOE_ERR_INVALID_ARG;
     if (E > kMaxE || K > kMaxK)
         return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -1308,12 +1365,12 @@ moe_derive_report(const moe_shape_t *shape, const moe_stats_t *st, const int64_t
     int32_t kmax = 0;
     for (int e = 0; e < E; ++e)
         kmax = kept[e] > kmax ? kept[e] : kmax;
-    out->drop_rate = (double)st->dropped / NK;
+    out->drop_rate = NK > 0 ? (double)st->dropped / NK : 0.0;
     out->send_max_over_min = smin > 0 ? (double)smax / (double)smin : INFINITY;
     out->recv_max_over_min = rmin > 0 ? (double)rmax / (double)rmin : INFINITY;
     out->cross_rank_fraction = st->rows > 0 ? (double)st->cross_rows / (double)st->rows : 0.0;
     out->load_std_over_mean = mean > 0 ? sqrt(var) / mean : 0.0;
-    out->capacity_factor_effective = (double)kmax / (NK / (double)E);
+    out->capacity_factor_effective = NK > 0 ? (double)kmax / (NK / (double)E) : 0.0;
     out->tau_min_tokens = off_row > off_col ? off_row : off_col;
     out->dispatch_bytes = st->rows * (int64_t)shape->d * 2;
     out->send_max = smax;
@@ -1403,6 +1460,9 @@ moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *
     moe_status_t rc = check_shape(shape, false, &g);
     if (rc != MOE_OK)
         return rc;
+    if (shape->N == 0)
+        return empty_dispatch(shape, counts, kept, offsets, rank_matrix, packed_offsets, stats,
+                              reinterpret_cast<cudaStream_t>(stream));
     if (g.rounds > 1)  // re-routing needs the logits
         return MOE_ERR_INVALID_ARG;
     if (!x || !topk_idx || !counts || !kept || !offsets || !row_of || !assign_of_row || !x_sorted)

@@ -60,7 +60,7 @@ def test_shape_validation(m):
     bad = [m.make_shape(64, 128, 256, 8, 9, 4),      # K > E
            m.make_shape(64, 128, 256, 8, 2, 3),      # E % W
            m.make_shape(66, 128, 256, 8, 2, 4),      # N % W
-           m.make_shape(0, 128, 256, 8, 2, 4),       # N
+           m.make_shape(-4, 128, 256, 8, 2, 4),      # N < 0
            m.make_shape(64, 100, 256, 8, 2, 4),      # d % 8
            m.make_shape(64, 128, 256, 512, 2, 4),    # E > 256
            m.make_shape(64, 128, 256, 64, 33, 4)]    # K > 32
@@ -70,6 +70,9 @@ def test_shape_validation(m):
     flags = m.make_shape(64, 128, 256, 8, 2, 4)
     flags.flags = 8  # no such flag
     assert m.moe_workspace_size(flags) == 0
+    # an empty batch is a valid shape
+    assert m.moe_workspace_size(m.make_shape(0, 128, 256, 8, 2, 4)) > 0
+    assert m.moe_rows_alloc(m.make_shape(0, 128, 256, 8, 2, 4)) == 128
     assert m.moe_workspace_size(m.make_shape(64, 128, 256, 8, 2, 4, out_bf16=True)) > 0
     # slot-major priority scans K blocks per token block: a larger scratch, never smaller
     tm = m.moe_workspace_size(m.make_shape(4096, 128, 256, 256, 32, 64, 1.0))

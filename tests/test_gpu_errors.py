@@ -62,3 +62,55 @@ def test_nonfinite_logits_are_flagged(m):
                 inp["w2"].cuda(), out, stats=stats, ws=ws)
     assert m.moe_get_device_error(True) == 7  # MOE_ERR_NONFINITE
     assert m.read_stats(stats).nonfinite_tokens == 1
+
+
+def test_empty_batch_every_entry_point():
+    """N = 0 (an empty batch) is a valid call: every entry point returns OK, launches nothing,
+    and the outputs indexed by expert or rank come back zero."""
+    import combine_grouped_gemm_router_b200 as m
+    dev = torch.device("cuda")
+    E, K, W, d, f = 8, 2, 4, 128, 256
+    for flags in ({}, {"slot_major": True}, {"reroute": True, "capacity_factor": 1.0}):
+        shape = m.make_shape(0, d, f, E, K, W, **flags)
+        ws = torch.empty(max(m.moe_layer_workspace_size(shape), 256), dtype=torch.uint8,
+                         device=dev)
+        empty = lambda *sz, dt=torch.float32: torch.empty(*sz, dtype=dt, device=dev)
+        x = empty(0, d, dt=torch.bfloat16)
+        topk = empty(0, K, dt=torch.int32)
+        tw = empty(0, K)
+        logits = empty(0, E)
+        m.moe_route(shape, x, torch.randn(E, d, device=dev), None, topk, tw, logits, ws)
+        counts = torch.full((E,), 7, dtype=torch.int32, device=dev)
+        kept = torch.full((E,), 7, dtype=torch.int32, device=dev)
+        offsets = torch.full((E + 1,), 7, dtype=torch.int32, device=dev)
+        D = torch.full((W * W,), 7, dtype=torch.int64, device=dev)
+        pk = torch.full((W * W + 1,), 7, dtype=torch.int64, device=dev)
+        stats = torch.full_like(m.stats_buffer(dev), 7)
+        RA = m.moe_rows_alloc(shape)
+        xs = empty(RA, d, dt=torch.bfloat16)
+        row_of = empty(0, dt=torch.int32)
+        assign = empty(RA, dt=torch.int32)
+        if flags.get("reroute"):
+            m.moe_dispatch_reroute(shape, x, logits, topk, counts, kept, offsets, row_of, assign, xs,
+                                   rank_matrix=D, packed_offsets=pk, stats=stats, ws=ws)
+        else:
+            m.moe_dispatch(shape, x, topk, counts, kept, offsets, row_of, assign, xs, None, D, pk,
+                           stats, ws)
+        torch.cuda.synchronize()
+        for t in (counts, kept, offsets, D, pk, stats):
+            assert int(t.abs().sum().item()) == 0
+        w1 = torch.zeros(E, f, d, dtype=torch.bfloat16, device=dev)
+        w2 = torch.zeros(E, d, f, dtype=torch.bfloat16, device=dev)
+        h = empty(RA, f, dt=torch.bfloat16)
+        y = empty(RA, d)
+        m.moe_expert_gemm(shape, xs, offsets, w1, w1, w2, h, y)
+        out = empty(0, d)
+        m.moe_combine(shape, y, row_of, tw, out)
+        stats2 = torch.full_like(m.stats_buffer(dev), 7)
+        m.moe_layer(shape, x, torch.randn(E, d, device=dev), None, w1, w1, w2, out, stats=stats2,
+                    ws=ws)
+        torch.cuda.synchronize()
+        assert int(stats2.abs().sum().item()) == 0
+        m.moe_affinity_accumulate(0, E, K, topk, topk, torch.zeros(E, E, dtype=torch.int64,
+                                                                  device=dev))
+    assert m.moe_get_device_error(True) == 0

@@ -239,3 +239,30 @@ def test_residual_moe_layer(orc):
         assert m.moe_get_device_error(True) == 0
         assert torch.equal(out, out_st)
         assert_within_tolerance(out, ref["out"], w.name)
+
+
+@pytest.mark.parametrize("d", [8, 24])
+@pytest.mark.parametrize("slot_major", [False, True])
+def test_route_dispatch_small_hidden(orc, d, slot_major):
+    """Routing and dispatch at the smallest hidden sizes the boundary accepts (d % 8 == 0;
+    the GEMMs need d % 128): logits, selection, bookkeeping and both scatter layouts, exact."""
+    w = Workload(f"small_d{d}", N=96, d=d, f=128, E=6, K=2, W=3, cf=1.0, s=1.0,
+                 slot_major=slot_major)
+    inp = make_layer_inputs(w, seed=4)
+    ref = orc.route_and_dispatch(inp["x"], inp["w_router"], inp["bias"], w.K, w.W, w.cf,
+                                 order=int(slot_major))
+    got = run_stages(inp, w)
+    assert got["dev_error"] == 0 and "h" not in got
+    np.testing.assert_array_equal(got["logits"].cpu().numpy().view(np.uint32),
+                                  ref["logits"].view(np.uint32))
+    np.testing.assert_array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
+    for key in ("counts", "kept", "offsets", "row_of"):
+        np.testing.assert_array_equal(got[key].cpu().numpy(), ref[key], err_msg=key)
+    R = ref["R"]
+    xu = _u16(inp["x"])
+    np.testing.assert_array_equal(_u16(got["x_sorted"][:R]), xu[ref["assign_of_row"] // w.K])
+    kept_slots = np.nonzero(ref["row_of"] >= 0)[0]
+    packed = np.empty((R, w.d), np.uint16)
+    packed[ref["packed_row_of"][kept_slots]] = xu[kept_slots // w.K]
+    np.testing.assert_array_equal(_u16(got["x_packed"][:R]), packed)
+    np.testing.assert_array_equal(got["D"].cpu().numpy().reshape(w.W, w.W), ref["D"])
