@@ -56,10 +56,13 @@ typedef enum moe_status {
     MOE_ERR_DEVICE_BOUNDS = 8        /* an expert id outside [0, E) reached a kernel */
 } moe_status_t;
 
-/* Problem description. Limits: 1 <= N, N*K < 2^31; d % 8 == 0 (d % 128 == 0 for
+/* Problem description. Limits: 0 <= N, N*K < 2^31; d % 8 == 0 (d % 128 == 0 for
  * moe_expert_gemm / moe_layer); f % 128 == 0 for the GEMMs; 1 <= E <= 256;
  * 1 <= K <= min(E, 32); 1 <= W <= 64, E % W == 0, N % W == 0.
- * capacity_factor <= 0 selects dropless routing. */
+ * capacity_factor <= 0 selects dropless routing.
+ * N = 0 (an empty batch) is valid everywhere: nothing is launched, the token-indexed
+ * arguments may be NULL, and the outputs indexed by expert or rank (counts, kept, offsets,
+ * rank_matrix, packed_offsets, stats) are set to zero. */
 typedef struct moe_shape {
     int32_t N, d, f, E, K, W;
     float capacity_factor;
