@@ -441,6 +441,31 @@ def run_gpu(args, w) -> dict:
         graph_res = {"value": g_agg["value"], "unit": UNIT,
                      "ms_per_step": g_agg["elapsed_max_s"] / args.steps * 1e3}
         del graph
+    # the routing report of layer 0 (untimed): one more route + dispatch with the counters on,
+    # then the derived figures (drop rate, per-rank send/receive balance, cross-rank fraction,
+    # expert-load spread, effective capacity factor, the exchange-time bound tau_min)
+    stats_buf = m.stats_buffer(dev)
+    l0 = layers[0]
+    m.moe_route(shape, x, l0["w_router"], l0["bias"], topk_idx[0], topk_w, logits, ws, stream)
+    if w.reroute:
+        m.moe_dispatch_reroute(shape, x, logits, topk_idx[0], counts, kept, offsets[0], row_of,
+                               assign, x_sorted, x_packed=x_packed, rank_matrix=D,
+                               packed_offsets=pk_off, stats=stats_buf, ws=ws, stream=stream)
+    elif w.fp8:
+        m.moe_dispatch_fp8(shape, x, topk_idx[0], counts, kept, offsets[0], row_of, assign,
+                           x_sorted, sorted_scale, x_packed=x_packed, packed_scale=packed_scale,
+                           rank_matrix=D, packed_offsets=pk_off, stats=stats_buf, ws=ws,
+                           stream=stream)
+    else:
+        m.moe_dispatch(shape, x, topk_idx[0], counts, kept, offsets[0], row_of, assign, x_sorted,
+                       x_packed, D, pk_off, stats_buf, ws, stream)
+    st0 = m.read_stats(stats_buf, stream)
+    rep0 = m.report_dict(m.moe_derive_report(shape, st0, D.cpu().numpy(), kept.cpu().numpy()))
+    routing = {"rows_kept": st0.rows, "dropped": st0.dropped, "active_experts": st0.active_experts,
+               "dedup_pairs": st0.dedup_pairs, "rerouted": st0.rerouted,
+               **{k: rep0[k] for k in ("drop_rate", "send_max_over_min", "recv_max_over_min",
+                                       "cross_rank_fraction", "load_std_over_mean",
+                                       "capacity_factor_effective", "tau_min_tokens")}}
     err = m.moe_get_device_error(True)
     R_layers = [int(o[E].item()) for o in offsets]
     act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
@@ -600,7 +625,13 @@ def run_gpu(args, w) -> dict:
                            "tflops": 6.0 * d * w.shared_f * N / (stage_ms["shared_expert"] / 1e3) / 1e12}
                           if shared else None),
         "dispatch": {"ms": stage_ms["dispatch"],
-                     "scatter_bytes": work["scatter_bytes"]},
+                     "scatter_bytes": work["scatter_bytes"],
+                     # the whole dispatch stage (histogram, scans, positions, scatter) against
+                     # the scatter's bytes alone: a lower bound on the scatter kernel's rate
+                     "gbs": work["scatter_bytes"] / (stage_ms["dispatch"] / 1e3) / 1e9,
+                     "frac_of_hbm": work["scatter_bytes"] / (stage_ms["dispatch"] / 1e3) / 1e9
+                     / hbm},
+        "routing": routing,
         "clocks": clocks.summary(),
         "gpu_launches": launches_per_step * args.steps,
         "graph": graph_res,

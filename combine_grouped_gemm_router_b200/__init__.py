@@ -79,6 +79,7 @@ _sigs = {
     "moe_derive_report": ([_SP, ctypes.POINTER(MoeStats), c_p, c_p, ctypes.POINTER(MoeReport)],
                           c_i32),
     "moe_get_device_error": ([ctypes.c_int], c_i32),
+    "moe_read_stats": ([c_p, ctypes.POINTER(MoeStats), c_p], c_i32),
     "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
 }
 
@@ -364,8 +365,11 @@ def stats_buffer(device="cuda"):
     return torch.zeros(ctypes.sizeof(MoeStats), dtype=torch.uint8, device=device)
 
 
-def read_stats(buf) -> MoeStats:
-    return MoeStats.from_buffer_copy(bytes(buf.to("cpu").numpy().tobytes()))
+def read_stats(buf, stream=None) -> MoeStats:
+    """The counters in a device stats buffer, through moe_read_stats (waits for the stream)."""
+    st = MoeStats()
+    _check(_lib.moe_read_stats(_ptr(buf), ctypes.byref(st), _stream(stream)), "moe_read_stats")
+    return st
 
 
 def report_dict(rep: MoeReport) -> dict:

@@ -1380,6 +1380,21 @@ moe_derive_report(const moe_shape_t *shape, const moe_stats_t *st, const int64_t
     return MOE_OK;
 }
 
+__attribute__((visibility("default"))) moe_status_t
+moe_read_stats(const moe_stats_t *stats_dev, moe_stats_t *out, moe_stream_t stream)
+{
+    if (!stats_dev || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(stats_dev) & 7u)
+        return MOE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(out, stats_dev, sizeof(moe_stats_t), cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 __attribute__((visibility("default"))) moe_status_t moe_get_device_error(int clear)
 {
     if (cudaDeviceSynchronize() != cudaSuccess)

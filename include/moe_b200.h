@@ -395,6 +395,11 @@ moe_status_t moe_derive_report(const moe_shape_t *shape, const moe_stats_t *stat
  * the device. Returns MOE_OK when no kernel has recorded an error. */
 moe_status_t moe_get_device_error(int clear);
 
+/* Copies the counters a dispatch or layer call wrote to DEVICE memory (stats_dev) into HOST
+ * memory (out, caller-owned), in order on `stream`, and waits for that stream: the one call
+ * here that synchronises on purpose, for observability outside the timed path. */
+moe_status_t moe_read_stats(const moe_stats_t *stats_dev, moe_stats_t *out, moe_stream_t stream);
+
 /* Launches one kernel whose only work is a bounded wait on a flag that nothing sets; it gives
  * up after timeout_ns nanoseconds and records MOE_ERR_DEVICE_TIMEOUT. Lets a test see the
  * bounded-wait path end with an error status while the context stays usable. */
