@@ -3,6 +3,8 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 
+#include <functional>
+#include <map>
 #include <mutex>
 
 #include "combine.cuh"
@@ -187,6 +189,37 @@ int num_sms()
     return n;
 }
 
+// Per-device, per-kernel one-time setup (function attributes belong to a device's context,
+// so a process that drives several GPUs sets them on each). `init` runs once per
+// (device, key) under a lock; its result is cached, as is the integer it returns in *value.
+cudaError_t once_per_device(const void *key, const std::function<cudaError_t(int *)> &init,
+                            int *value = nullptr)
+{
+    static std::mutex mu;
+    static std::map<std::pair<int, const void *>, std::pair<cudaError_t, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find({dev, key});
+    if (it == done.end()) {
+        int v = 0;
+        const cudaError_t e = init(&v);
+        it = done.emplace(std::make_pair(dev, key), std::make_pair(e, v)).first;
+    }
+    if (value)
+        *value = it->second.second;
+    return it->second.first;
+}
+
+template <typename Kernel>
+cudaError_t smem_attr_once(Kernel kernel, int bytes)
+{
+    return once_per_device(reinterpret_cast<const void *>(kernel), [&](int *) {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    });
+}
+
 // Warp work items of the row kernels (combine, bf16 scatter): a whole token row each
 // when there are enough tokens to fill the GPU, else slices of `slice` chunks, so that a
 // decode batch of a few tokens still spreads over every SM.
@@ -215,11 +248,7 @@ void launch_logits(const uint16_t *x, const float *wr, const float *bias, float 
                    int d, int E, cudaStream_t st)
 {
     using L = LogitTile<TY, TX, TT, TE, KC, S>;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(router_logits_kernel<TY, TX, TT, TE, KC, S>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
-    });
+    smem_attr_once(router_logits_kernel<TY, TX, TT, TE, KC, S>, L::SMEM_BYTES);
     dim3 grid((N + L::BT - 1) / L::BT, (E + L::BE - 1) / L::BE);
     router_logits_kernel<TY, TX, TT, TE, KC, S>
         <<<grid, L::NT, L::SMEM_BYTES, st>>>(x, wr, bias, logits, N, d, E);
@@ -299,11 +328,7 @@ void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const in
     sa.pk_base = pk_base;
     sa.stats = stats;
     const size_t scan_smem = scan_smem_base(s) + (cum_in_smem ? scan_cum_bytes(s, nseg) : 0);
-    static std::once_flag scan_attr;
-    std::call_once(scan_attr, [] {
-        cudaFuncSetAttribute(dispatch_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kScanSmemLimit);
-    });
+    smem_attr_once(dispatch_scan_kernel, (int)kScanSmemLimit);
     dispatch_scan_kernel<<<1, 1024, scan_smem, st>>>(sa);
 
     PosArgs pa;
@@ -449,13 +474,7 @@ moe_status_t launch_gemm(const CUtensorMap &a, const CUtensorMap &b0, const CUte
                          const gg::Args &args, cudaStream_t st)
 {
     const int smem = gg::smem_bytes<MODE, BN>(kMaxE);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(gg::grouped_gemm_kernel<MODE, BN>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    });
-    if (attr_err != cudaSuccess)
+    if (smem_attr_once(gg::grouped_gemm_kernel<MODE, BN>, smem) != cudaSuccess)
         return MOE_ERR_CUDA;
     gg::grouped_gemm_kernel<MODE, BN><<<num_sms(), gg::THREADS, smem, st>>>(a, b0, b1, args);
     return launch_status();
@@ -468,14 +487,13 @@ moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const
                               const gg::Args &args, cudaStream_t st)
 {
     const int smem = gg::smem_bytes_pair<MODE>(kMaxE);
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    static int pairs = 0;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(gg::grouped_gemm_pair_kernel<MODE>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (attr_err != cudaSuccess)
-            return;
+    int pairs = 0;
+    const cudaError_t attr_err = once_per_device(
+        reinterpret_cast<const void *>(gg::grouped_gemm_pair_kernel<MODE>), [&](int *n_pairs) {
+        cudaError_t e = cudaFuncSetAttribute(gg::grouped_gemm_pair_kernel<MODE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -487,10 +505,8 @@ moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const
         cfg.dynamicSmemBytes = smem;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        int n = 0;
-        attr_err = cudaOccupancyMaxActiveClusters(&n, gg::grouped_gemm_pair_kernel<MODE>, &cfg);
-        pairs = n;
-    });
+        return cudaOccupancyMaxActiveClusters(n_pairs, gg::grouped_gemm_pair_kernel<MODE>, &cfg);
+    }, &pairs);
     if (attr_err != cudaSuccess || pairs <= 0)
         return MOE_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};

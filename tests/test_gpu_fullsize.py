@@ -10,7 +10,8 @@ import numpy as np
 import pytest
 import torch
 
-from layer_runner import assert_within_tolerance, run_stages, tolerance_report
+from layer_runner import (assert_within_bound, assert_within_tolerance, bf16_h_bound_rows,
+                          run_stages, tolerance_report)
 from moe_workloads import STACK_GRID_CF, STACK_GRID_S, WORKLOADS, make_layer_inputs
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -83,9 +84,32 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     rows = torch.from_numpy(smp["sample_rows"]).cuda().long()
     rep_h = tolerance_report(got["h"][rows], smp["sample_h"])
     assert rep_h["rel_frob"] <= 5e-3, rep_h
-    rep_y = assert_within_tolerance(got["y"][rows], smp["sample_y"], "y sample")
-    rep_o = assert_within_tolerance(got["out"][torch.from_numpy(toks).cuda()], smp["out_tokens"],
-                                    "out sample")
+    # y and out: the per-element bound of one bf16 rounding of h (the down projection's
+    # operand) plus fp32 accumulation, and the relative Frobenius bar; the max-abs bar is
+    # asserted when nothing is dropped and reported otherwise (with heavy drops many
+    # sampled tokens have zero output, which deflates the RMS the bar is relative to)
+    w2 = hx["w2"].double().numpy()
+    sample_expert = rr["expert_of"][smp["sample_slots"]]
+    ybound = bf16_h_bound_rows(smp["sample_h"], w2, sample_expert)
+    assert_within_bound(got["y"][rows], smp["sample_y"], ybound, "y sample")
+    obound = np.zeros_like(smp["out_tokens"])
+    pos = {int(a): i for i, a in enumerate(smp["sample_slots"])}
+    for li, t in enumerate(toks):
+        for k in range(w.K):
+            a = int(t) * w.K + k
+            if a in pos:
+                wa = abs(float(r["topk_w"].reshape(-1)[a]))
+                yi = pos[a]
+                obound[li] += wa * ybound[yi] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(
+                    smp["sample_y"][yi])
+    got_out = got["out"][torch.from_numpy(toks).cuda()]
+    assert_within_bound(got_out, smp["out_tokens"], obound, "out sample")
+    rep_y = tolerance_report(got["y"][rows], smp["sample_y"])
+    rep_o = tolerance_report(got_out, smp["out_tokens"])
+    assert rep_y["rel_frob"] <= 5e-3 and rep_o["rel_frob"] <= 5e-3, (rep_y, rep_o)
+    if r["stats"]["dropped"] == 0:
+        assert_within_tolerance(got["y"][rows], smp["sample_y"], "y sample")
+        assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
     # routing margins (reported; the logits are bit-exact, so no seed is rejected)
     lg = np.sort(r["logits"], axis=1)[:, ::-1]
     margin = lg[:, w.K - 1] - lg[:, w.K] if w.K < w.E else np.full(w.N, np.inf)
@@ -93,10 +117,11 @@ def check_full_size(orc, w, seed=0, n_sample=24):
                 tokens_margin_below_1e5=int((margin < 1e-5).sum()))
 
 
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
 @pytest.mark.parametrize("name", ["mixtral_prefill", "e128_skew", "decode"])
-def test_full_size_workload(orc, name):
-    rep = check_full_size(orc, WORKLOADS[name])
-    print(name, rep)
+def test_full_size_workload(orc, name, seed):
+    rep = check_full_size(orc, WORKLOADS[name], seed=seed)
+    print(name, seed, rep)
 
 
 @pytest.mark.parametrize("name", ["e128_skew", "stack4"])
