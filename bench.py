@@ -199,11 +199,12 @@ class ClockSampler:
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"],
                     "source": self.source}
-        load = [r for r in rows if r["power"] > 300.0] or rows
-        reasons = sorted(set().union(*(r["reasons"] for r in load)))
-        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+        # every sample falls inside the timed region (the sampler runs only there); NVML's
+        # power reading is averaged, so it does not tell busy samples from idle ones
+        reasons = sorted(set().union(*(r["reasons"] for r in rows)))
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
                 "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
-                "samples": len(rows), "samples_under_load": len(load), "source": self.source}
+                "samples": len(rows), "source": self.source}
 
 
 # --------------------------------------------------------------------------- GPU arm
