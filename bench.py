@@ -237,6 +237,36 @@ def up_traffic(workload: str):
     return nbytes if sha == sha_ref else None
 
 
+def kernel_launches(w) -> int:
+    """Kernels the library launches for one layer of workload w, by the same rules as its
+    host code: routing 2; per dispatch pass a histogram, a per-expert scan when there are
+    more than 128 blocks, the scan and the positions; the ranking kernel between the two
+    passes of re-routing; the scatter; each grouped GEMM once, or twice (CTA-pair tiles, then
+    single-CTA tiles) when the experts average at least 768 rows and the K extent allows pair
+    stages; the quantisation of h on the FP8 path; the shared MLP's offsets and GEMMs; the
+    combine."""
+    N, d, f, E, K, W = w.N, w.d, w.f, w.E, w.K, w.W
+    NK = N * K
+    C = NK if not w.cf > 0 else min(NK, math.ceil(w.cf * N * K / E))
+    pair = min(NK // E, C) >= 768
+    nvb_round = (K if w.slot_major else 1) * W * (-(-(N // W) // 64))
+    def dispatch_pass(nvb):
+        return 3 + (1 if nvb > 128 else 0)
+    n = 2
+    n += dispatch_pass(nvb_round) + 1 + dispatch_pass(2 * nvb_round) if w.reroute \
+        else dispatch_pass(nvb_round)
+    n += 1  # scatter
+    atom = 128 if w.fp8 else 64
+    n += 2 if pair and (d // atom) % 2 == 0 else 1                     # gate/up
+    n += 1 if w.fp8 else 0                                              # h -> e4m3
+    n += (2 if pair and (f // atom) % 2 == 0 else 1) if d % 256 == 0 else 1   # down
+    if w.shared_f > 0:
+        sp = N >= 768
+        n += 1 + (2 if sp else 1) + ((2 if sp else 1) if d % 256 == 0 else 1)
+    n += 1  # combine
+    return n
+
+
 def algorithmic_work(w, R: int, E_act: int) -> dict:
     """Algorithmic flops and bytes per launch of each stage (see the design notes);
     E_act = experts with at least one kept row (only their weights are read)."""
@@ -327,12 +357,8 @@ def run_gpu(args, w) -> dict:
     stage_names = ["route", "dispatch", "expert_up", "expert_down"] + (
         ["shared_expert"] if shared else []) + ["combine"]
     n_ev = len(stage_names) + 1
-    # per layer: logits, top-K, histogram, scan, positions, scatter, up, down, combine
-    # (+ offsets, shared up, shared down for the Residual-MoE layer); + affinity per layer pair
-    # (+ histogram, scan, positions of the first pass and the ranking kernel when re-routing)
-    # (+ the quantisation of h for the FP8 down projection)
-    launches_per_step = (L * (9 + (3 if shared else 0) + (4 if w.reroute else 0) +
-                              (1 if w.fp8 else 0)) + (L - 1))
+    # the library's kernels per step: every layer's, plus one affinity count per layer pair
+    launches_per_step = L * kernel_launches(w) + (L - 1)
 
     def step(ev=None):
         """One step; ev (optional) is [layer][n_ev] events around the stages."""
