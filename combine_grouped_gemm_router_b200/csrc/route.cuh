@@ -43,6 +43,36 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// Stages chunk c of d (x rows of the CTA's tokens, Wr rows of its experts) into ring
+// slot c % S with cp.async; always commits a group (possibly empty) so that every
+// thread's group count stays uniform.
+template <class L, int KC, int S>
+__device__ __forceinline__ void stage_logit_chunk(unsigned char *smem, int c, int nchunks,
+                                                  const uint16_t *__restrict__ x,
+                                                  const float *__restrict__ wr, int t0, int e0,
+                                                  int N, int d, int E)
+{
+    const int tid = threadIdx.x;
+    if (c < nchunks) {
+        unsigned char *st = smem + (c % S) * L::STAGE_BYTES;
+        uint16_t *xs = reinterpret_cast<uint16_t *>(st);
+        float *ws = reinterpret_cast<float *>(st + L::X_BYTES);
+        const int k0 = c * KC;
+        const int kc = min(KC, d - k0);  // a multiple of 8 (d % 8 == 0)
+        for (int idx = tid; idx < L::BT * (KC / 8); idx += L::NT) {
+            const int row = idx / (KC / 8), v = idx % (KC / 8);
+            if (t0 + row < N && v * 8 < kc)
+                cp_async16(xs + row * L::XROW + v * 8, x + (size_t)(t0 + row) * d + k0 + v * 8);
+        }
+        for (int idx = tid; idx < L::BE * (KC / 4); idx += L::NT) {
+            const int row = idx / (KC / 4), v = idx % (KC / 4);
+            if (e0 + row < E && v * 4 < kc)
+                cp_async16(ws + row * L::WROW + v * 4, wr + (size_t)(e0 + row) * d + k0 + v * 4);
+        }
+    }
+    cp_async_commit();
+}
+
 template <int TY, int TX, int TT, int TE, int KC, int S>
 __global__ void __launch_bounds__(TY *TX)
     router_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
@@ -57,26 +87,8 @@ __global__ void __launch_bounds__(TY *TX)
     const int t0 = blockIdx.x * L::BT;
     const int e0 = blockIdx.y * L::BE;
     const int nchunks = (d + KC - 1) / KC;
-
     auto issue = [&](int c) {
-        if (c < nchunks) {
-            unsigned char *st = logit_smem + (c % S) * L::STAGE_BYTES;
-            uint16_t *xs = reinterpret_cast<uint16_t *>(st);
-            float *ws = reinterpret_cast<float *>(st + L::X_BYTES);
-            const int k0 = c * KC;
-            const int kc = min(KC, d - k0);  // a multiple of 8 (d % 8 == 0)
-            for (int idx = tid; idx < L::BT * (KC / 8); idx += L::NT) {
-                const int row = idx / (KC / 8), v = idx % (KC / 8);
-                if (t0 + row < N && v * 8 < kc)
-                    cp_async16(xs + row * L::XROW + v * 8, x + (size_t)(t0 + row) * d + k0 + v * 8);
-            }
-            for (int idx = tid; idx < L::BE * (KC / 4); idx += L::NT) {
-                const int row = idx / (KC / 4), v = idx % (KC / 4);
-                if (e0 + row < E && v * 4 < kc)
-                    cp_async16(ws + row * L::WROW + v * 4, wr + (size_t)(e0 + row) * d + k0 + v * 4);
-            }
-        }
-        cp_async_commit();  // possibly empty: keeps the group count uniform
+        stage_logit_chunk<L, KC, S>(logit_smem, c, nchunks, x, wr, t0, e0, N, d, E);
     };
 
     float acc[TT][TE];
@@ -139,6 +151,95 @@ __global__ void __launch_bounds__(TY *TX)
             }
         }
     }
+}
+
+// The same tile with two tokens per instruction: the accumulators of tokens (2p, 2p+1)
+// for one expert form a pair, updated by one packed fp32 FMA (`__ffma2_rn`). Each half of
+// a packed FMA is rounded exactly like one fmaf, and every chain still walks d in order,
+// so the logits are the same bits as router_logits_kernel's. Halving the FMA instructions
+// frees issue slots where a thread owns many outputs (large N, E > 32).
+template <int TY, int TX, int TT, int TE, int KC, int S>
+__global__ void __launch_bounds__(TY *TX)
+    router_logits_pairs_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
+                               const float *__restrict__ bias, float *__restrict__ logits, int N,
+                               int d, int E)
+{
+    using L = LogitTile<TY, TX, TT, TE, KC, S>;
+    static_assert(KC % 8 == 0 && TT % 2 == 0, "whole 16-byte vectors, token pairs");
+    extern __shared__ __align__(16) unsigned char logit_smem[];
+    const int tid = threadIdx.x;
+    const int ty = tid / TX, tx = tid % TX;
+    const int t0 = blockIdx.x * L::BT;
+    const int e0 = blockIdx.y * L::BE;
+    const int nchunks = (d + KC - 1) / KC;
+
+    float2 acc[TT / 2][TE];
+#pragma unroll
+    for (int i = 0; i < TT / 2; ++i)
+#pragma unroll
+        for (int j = 0; j < TE; ++j)
+            acc[i][j] = make_float2(0.0f, 0.0f);
+
+#pragma unroll
+    for (int c = 0; c < S - 1; ++c)
+        stage_logit_chunk<L, KC, S>(logit_smem, c, nchunks, x, wr, t0, e0, N, d, E);
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<S - 2>();
+        __syncthreads();
+        stage_logit_chunk<L, KC, S>(logit_smem, c + S - 1, nchunks, x, wr, t0, e0, N, d, E);
+        const unsigned char *st = logit_smem + (c % S) * L::STAGE_BYTES;
+        const uint16_t *xs = reinterpret_cast<const uint16_t *>(st);
+        const float *ws = reinterpret_cast<const float *>(st + L::X_BYTES);
+        const int kc = min(KC, d - c * KC);
+        for (int kk = 0; kk < kc; kk += 8) {
+            float2 xv[TT / 2][8];
+#pragma unroll
+            for (int p = 0; p < TT / 2; ++p) {
+                const uint4 a =
+                    *reinterpret_cast<const uint4 *>(xs + (ty * TT + 2 * p) * L::XROW + kk);
+                const uint4 b =
+                    *reinterpret_cast<const uint4 *>(xs + (ty * TT + 2 * p + 1) * L::XROW + kk);
+                xv[p][0] = make_float2(bf16_lo(a.x), bf16_lo(b.x));
+                xv[p][1] = make_float2(bf16_hi(a.x), bf16_hi(b.x));
+                xv[p][2] = make_float2(bf16_lo(a.y), bf16_lo(b.y));
+                xv[p][3] = make_float2(bf16_hi(a.y), bf16_hi(b.y));
+                xv[p][4] = make_float2(bf16_lo(a.z), bf16_lo(b.z));
+                xv[p][5] = make_float2(bf16_hi(a.z), bf16_hi(b.z));
+                xv[p][6] = make_float2(bf16_lo(a.w), bf16_lo(b.w));
+                xv[p][7] = make_float2(bf16_hi(a.w), bf16_hi(b.w));
+            }
+#pragma unroll
+            for (int j = 0; j < TE; ++j) {
+                const float *wrow = ws + (tx + TX * j) * L::WROW + kk;
+                const float4 a = *reinterpret_cast<const float4 *>(wrow);
+                const float4 b = *reinterpret_cast<const float4 *>(wrow + 4);
+                const float wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float2 w2 = make_float2(wv[q], wv[q]);
+#pragma unroll
+                    for (int p = 0; p < TT / 2; ++p)
+                        acc[p][j] = __ffma2_rn(xv[p][q], w2, acc[p][j]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < TT / 2; ++p)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int t = t0 + ty * TT + 2 * p + h;
+#pragma unroll
+            for (int j = 0; j < TE; ++j) {
+                const int e = e0 + tx + TX * j;
+                if (t < N && e < E) {
+                    float v = h ? acc[p][j].y : acc[p][j].x;
+                    if (bias)
+                        v = __fadd_rn(v, bias[e]);
+                    logits[(size_t)t * E + e] = v;
+                }
+            }
+        }
 }
 
 // One warp per token. Lane l holds logits of experts l + 32*j (E <= 256).
