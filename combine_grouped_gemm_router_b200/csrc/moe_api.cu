@@ -179,28 +179,18 @@ LayerLayout layer_layout(const moe_shape_t *s, const Geometry &g, size_t base)
     return L;
 }
 
-int num_sms()
-{
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return 148;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-        return 148;
-    return n;
-}
-
 // Per-device, per-kernel one-time setup (function attributes belong to a device's context,
 // so a process that drives several GPUs sets them on each). `init` runs once per
 // (device, key) under a lock; its result is cached, as is the integer it returns in *value.
 cudaError_t once_per_device(const void *key, const std::function<cudaError_t(int *)> &init,
                             int *value = nullptr)
 {
-    static std::mutex mu;
+    static std::recursive_mutex mu;  // an init may itself ask for a per-device value
     static std::map<std::pair<int, const void *>, std::pair<cudaError_t, int>> done;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
+    std::lock_guard<std::recursive_mutex> lock(mu);
     auto it = done.find({dev, key});
     if (it == done.end()) {
         int v = 0;
@@ -210,6 +200,21 @@ cudaError_t once_per_device(const void *key, const std::function<cudaError_t(int
     if (value)
         *value = it->second.second;
     return it->second.first;
+}
+
+// Streaming multiprocessors of the current device (queried once per device).
+int num_sms()
+{
+    static const char key = 0;
+    int n = 0;
+    const cudaError_t e = once_per_device(&key, [](int *v) {
+        int dev = 0;
+        cudaError_t r = cudaGetDevice(&dev);
+        if (r == cudaSuccess)
+            r = cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+        return r;
+    }, &n);
+    return (e == cudaSuccess && n > 0) ? n : 148;
 }
 
 template <typename Kernel>
@@ -502,6 +507,7 @@ moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const
                               const gg::Args &args, cudaStream_t st)
 {
     const int smem = gg::smem_bytes_pair<MODE>(kMaxE);
+    const int sms = num_sms();
     int pairs = 0;
     const cudaError_t attr_err = once_per_device(
         reinterpret_cast<const void *>(gg::grouped_gemm_pair_kernel<MODE>), [&](int *n_pairs) {
@@ -515,7 +521,7 @@ moe_status_t launch_gemm_pair(const CUtensorMap &a, const CUtensorMap &b0, const
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+        cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
         cfg.blockDim = dim3(gg::THREADS, 1, 1);
         cfg.dynamicSmemBytes = smem;
         cfg.attrs = attr;
