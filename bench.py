@@ -237,6 +237,36 @@ def up_traffic(workload: str):
     return nbytes if sha == sha_ref else None
 
 
+PEER_COPY_GBS = 770.0  # measured NVLink peer copy per direction per GPU on this GPU type
+
+
+def exchange_report(m, D, row_bytes: int) -> dict:
+    """The exchange of layer 0's packed rows as W ranks would run it (host planning only; nothing
+    crosses a link here): the contention-free order from moe_exchange_schedule, its length in
+    rows (equal to tau_min), and, for contrast, the plain rotation order in which, in round s,
+    rank i sends to rank (i + s) mod W and a round lasts as long as its largest block."""
+    W = D.shape[0]
+    dst, ln, span = m.moe_exchange_schedule(D)
+    rotation = sum(int(max(D[i, (i + s) % W] for i in range(W))) for s in range(1, W))
+    return {"phases": int(len(ln)), "makespan_rows": span, "rotation_rows": rotation,
+            "makespan_us_at_peer_copy": span * row_bytes / (PEER_COPY_GBS * 1e3),
+            "rotation_us_at_peer_copy": rotation * row_bytes / (PEER_COPY_GBS * 1e3)}
+
+
+def placement_report(m, counts, L: int, E: int, P: int) -> dict:
+    """Expert placement over P GPUs from the affinity counts the timed steps accumulated:
+    the fraction of inter-layer token hops that cross GPUs with contiguous placement and with
+    moe_place_experts' placement, and the host time the placement took."""
+    t0 = time.perf_counter()
+    _, cost, base = m.moe_place_experts(counts, L, E, P, starts=16)
+    host_s = time.perf_counter() - t0
+    hops = int(counts.sum())
+    return {"gpus": P, "hops": hops,
+            "cross_fraction_contiguous": base / hops if hops else 0.0,
+            "cross_fraction_placed": cost / hops if hops else 0.0,
+            "host_s": host_s}
+
+
 def kernel_launches(w) -> int:
     """Kernels the library launches for one layer of workload w, by the same rules as its
     host code: routing 2; per dispatch pass a histogram, a per-expert scan when there are
@@ -493,6 +523,10 @@ def run_gpu(args, w) -> dict:
                **{k: rep0[k] for k in ("drop_rate", "send_max_over_min", "recv_max_over_min",
                                        "cross_rank_fraction", "load_std_over_mean",
                                        "capacity_factor_effective", "tau_min_tokens")}}
+    routing["exchange"] = exchange_report(m, D.cpu().numpy().reshape(W, W),
+                                          row_bytes=(d + 4) if w.fp8 else 2 * d)
+    if L > 1:
+        routing["placement"] = placement_report(m, affinity.cpu().numpy(), L, E, W)
     err = m.moe_get_device_error(True)
     R_layers = [int(o[E].item()) for o in offsets]
     act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]

@@ -78,6 +78,8 @@ _sigs = {
     "moe_affinity_accumulate": ([c_i32, c_i32, c_i32, c_p, c_p, c_p, c_p], c_i32),
     "moe_derive_report": ([_SP, ctypes.POINTER(MoeStats), c_p, c_p, ctypes.POINTER(MoeReport)],
                           c_i32),
+    "moe_exchange_schedule": ([c_i32, c_p, c_i32, c_p, c_p, c_p, c_p], c_i32),
+    "moe_place_experts": ([c_i32, c_i32, c_i32, c_p, c_i32, c_p, c_p, c_p], c_i32),
     "moe_get_device_error": ([ctypes.c_int], c_i32),
     "moe_read_stats": ([c_p, ctypes.POINTER(MoeStats), c_p], c_i32),
     "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
@@ -348,6 +350,46 @@ def moe_derive_report(shape, stats: MoeStats, rank_matrix, kept) -> MoeReport:
                                   D.ctypes.data_as(c_p), k.ctypes.data_as(c_p),
                                   ctypes.byref(rep)), "moe_derive_report")
     return rep
+
+
+def moe_exchange_schedule(rank_matrix, max_phases: Optional[int] = None):
+    """Contention-free transmission order of one exchange (host arrays in, host arrays out).
+
+    rank_matrix: int64 [W, W]. Returns (phase_dst int32 [n, W], phase_len int64 [n], makespan).
+    """
+    import numpy as np
+    D = np.ascontiguousarray(rank_matrix, dtype=np.int64)
+    W = int(round(D.size ** 0.5))
+    if D.size != W * W:
+        raise MoeError(1, "moe_exchange_schedule: rank_matrix is not square")
+    cap = 2 * W * W if max_phases is None else int(max_phases)
+    dst = np.empty((max(cap, 1), W), np.int32)
+    ln = np.empty(max(cap, 1), np.int64)
+    n = ctypes.c_int32(0)
+    span = ctypes.c_int64(0)
+    _check(_lib.moe_exchange_schedule(W, D.ctypes.data_as(c_p), cap, dst.ctypes.data_as(c_p),
+                                      ln.ctypes.data_as(c_p), ctypes.byref(n),
+                                      ctypes.byref(span)), "moe_exchange_schedule")
+    return dst[:n.value].copy(), ln[:n.value].copy(), int(span.value)
+
+
+def moe_place_experts(counts, L: int, E: int, P: int, starts: int = 16):
+    """Expert placement from affinity counts int64 [L-1, E, E] (host).
+
+    Returns (gpu_of int32 [L, E], cost, contiguous_cost).
+    """
+    import numpy as np
+    c = np.ascontiguousarray(counts, dtype=np.int64).reshape(-1)
+    if c.size != max(L - 1, 0) * E * E:
+        raise MoeError(1, "moe_place_experts: counts must hold (L-1)*E*E entries")
+    g = np.empty((L, E), np.int32)
+    cost = ctypes.c_int64(0)
+    base = ctypes.c_int64(0)
+    _check(_lib.moe_place_experts(int(L), int(E), int(P),
+                                  c.ctypes.data_as(c_p) if c.size else None, int(starts),
+                                  g.ctypes.data_as(c_p), ctypes.byref(cost), ctypes.byref(base)),
+           "moe_place_experts")
+    return g, int(cost.value), int(base.value)
 
 
 def moe_get_device_error(clear: bool = True) -> int:

@@ -1,0 +1,357 @@
+// Host-side planning of the expert-parallel exchange (no device code, no CUDA calls).
+//
+//  * exchange_schedule: a transmission order for one exchange with traffic matrix D in which no
+//    two senders feed the same receiver at once, and whose length is the lower bound of
+//    "MoE Inference Communication", §Aurora 定理 4.2: max over ranks of the tokens a rank sends
+//    or receives over links. The pages' own procedure (Aurora, Algorithm 1: bottleneck rank
+//    first, the others by volume, no receiver shared) only states the rule and the bound; here
+//    the bound is reached by construction: D is embedded in a 2W x 2W matrix whose every row and
+//    column sums to the bound, and that matrix is peeled into weighted permutations (Birkhoff's
+//    decomposition; each permutation found by augmenting paths, Kuhn's method). Each
+//    permutation restricted to the real block is one phase.
+//
+//  * place_experts: which E/P experts of every layer each of P GPUs holds, so that few token
+//    hops between consecutive layers cross GPUs ("MoE Inference Communication", §ExFlow
+//    形式化：整数线性规划建模: the objective, the equal-share and one-GPU-per-expert
+//    constraints). The pages solve it as an ILP; here it is solved by block coordinate descent:
+//    the placement of one layer, given both neighbours, is an assignment problem (experts to GPU
+//    slots, each GPU E/P slots) solved exactly with the Hungarian method, so every accepted move
+//    lowers the cost; sweeps run forward and backward over the layers from several starts, and
+//    each start's result is perturbed and descended again a few times (iterated local search).
+#pragma once
+
+#include <stdint.h>
+
+#include <algorithm>
+#include <vector>
+
+namespace moe_plan {
+
+// ------------------------------------------------------------------ exchange schedule
+
+// Perfect matching on the positive entries of an n x n matrix, repaired row by row.
+struct SupportMatching {
+    int n;
+    const std::vector<int64_t> &m;
+    std::vector<int> row_to, col_to, seen;
+    int stamp = 0;
+
+    SupportMatching(int n_, const std::vector<int64_t> &m_)
+        : n(n_), m(m_), row_to(n_, -1), col_to(n_, -1), seen(n_, -1) {}
+
+    bool augment_from(int r)
+    {
+        for (int c = 0; c < n; ++c) {
+            if (m[(size_t)r * n + c] <= 0 || seen[c] == stamp)
+                continue;
+            seen[c] = stamp;
+            if (col_to[c] < 0 || augment_from(col_to[c])) {
+                row_to[r] = c;
+                col_to[c] = r;
+                return true;
+            }
+        }
+        return false;
+    }
+
+    bool match_row(int r)
+    {
+        ++stamp;
+        return augment_from(r);
+    }
+};
+
+// Off-diagonal line sums of D and their maximum (the bound, in tokens).
+inline int64_t exchange_bound(int W, const int64_t *D, std::vector<int64_t> *row,
+                              std::vector<int64_t> *col)
+{
+    row->assign(W, 0);
+    col->assign(W, 0);
+    for (int i = 0; i < W; ++i)
+        for (int j = 0; j < W; ++j)
+            if (i != j) {
+                (*row)[i] += D[i * W + j];
+                (*col)[j] += D[i * W + j];
+            }
+    int64_t b = 0;
+    for (int i = 0; i < W; ++i)
+        b = std::max(b, std::max((*row)[i], (*col)[i]));
+    return b;
+}
+
+// Returns false when the phases do not fit in max_phases (cannot happen for
+// max_phases >= 2*W*W) or when a matching cannot be repaired (cannot happen for D >= 0).
+inline bool exchange_schedule(int W, const int64_t *D, int max_phases, int32_t *phase_dst,
+                              int64_t *phase_len, int *n_phases, int64_t *makespan)
+{
+    std::vector<int64_t> row, col;
+    const int64_t bound = exchange_bound(W, D, &row, &col);
+    *n_phases = 0;
+    *makespan = 0;
+    if (bound == 0)
+        return true;
+    // [ D_off            diag(bound - row) ]   every row and column of this 2W x 2W
+    // [ diag(bound - col)     D_off^T       ]   matrix sums to `bound`.
+    const int n = 2 * W;
+    std::vector<int64_t> m((size_t)n * n, 0);
+    for (int i = 0; i < W; ++i) {
+        for (int j = 0; j < W; ++j)
+            if (i != j) {
+                m[(size_t)i * n + j] = D[i * W + j];
+                m[(size_t)(W + j) * n + (W + i)] = D[i * W + j];
+            }
+        m[(size_t)i * n + (W + i)] = bound - row[i];
+        m[(size_t)(W + i) * n + i] = bound - col[i];
+    }
+    SupportMatching pm(n, m);
+    for (int r = 0; r < n; ++r)
+        if (!pm.match_row(r))
+            return false;
+    int64_t left = bound;
+    std::vector<int> broken;
+    while (left > 0) {
+        int64_t step = left;
+        for (int r = 0; r < n; ++r)
+            step = std::min(step, m[(size_t)r * n + pm.row_to[r]]);
+        // The phase: sender i -> receiver row_to[i] when that entry lies in the real block.
+        bool same = *n_phases > 0;
+        for (int i = 0; i < W && same; ++i) {
+            const int dst = pm.row_to[i] < W ? pm.row_to[i] : -1;
+            same = phase_dst[(size_t)(*n_phases - 1) * W + i] == dst;
+        }
+        if (same) {
+            phase_len[*n_phases - 1] += step;
+        } else {
+            if (*n_phases >= max_phases)
+                return false;
+            for (int i = 0; i < W; ++i)
+                phase_dst[(size_t)*n_phases * W + i] = pm.row_to[i] < W ? pm.row_to[i] : -1;
+            phase_len[*n_phases] = step;
+            ++*n_phases;
+        }
+        broken.clear();
+        for (int r = 0; r < n; ++r) {
+            const int c = pm.row_to[r];
+            m[(size_t)r * n + c] -= step;
+            if (m[(size_t)r * n + c] == 0)
+                broken.push_back(r);
+        }
+        left -= step;
+        *makespan += step;
+        if (left == 0)
+            break;
+        for (int r : broken) {
+            pm.col_to[pm.row_to[r]] = -1;
+            pm.row_to[r] = -1;
+        }
+        for (int r : broken)
+            if (!pm.match_row(r))
+                return false;
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ expert placement
+
+// Minimum-cost perfect assignment of n rows to n columns (Hungarian method with row and
+// column potentials, O(n^3)). cost is n x n, row-major. Writes col_of_row.
+inline void min_cost_assignment(int n, const std::vector<int64_t> &cost,
+                                std::vector<int> *col_of_row)
+{
+    const int64_t INF = INT64_MAX / 4;
+    std::vector<int64_t> u(n + 1, 0), v(n + 1, 0), minv(n + 1);
+    std::vector<int> row_of_col(n + 1, 0), way(n + 1, 0);
+    std::vector<char> used(n + 1);
+    for (int r = 1; r <= n; ++r) {
+        row_of_col[0] = r;
+        int c0 = 0;
+        std::fill(minv.begin(), minv.end(), INF);
+        std::fill(used.begin(), used.end(), 0);
+        do {
+            used[c0] = 1;
+            const int r0 = row_of_col[c0];
+            int64_t delta = INF;
+            int c1 = 0;
+            for (int c = 1; c <= n; ++c) {
+                if (used[c])
+                    continue;
+                const int64_t cur = cost[(size_t)(r0 - 1) * n + (c - 1)] - u[r0] - v[c];
+                if (cur < minv[c]) {
+                    minv[c] = cur;
+                    way[c] = c0;
+                }
+                if (minv[c] < delta) {
+                    delta = minv[c];
+                    c1 = c;
+                }
+            }
+            for (int c = 0; c <= n; ++c) {
+                if (used[c]) {
+                    u[row_of_col[c]] += delta;
+                    v[c] -= delta;
+                } else {
+                    minv[c] -= delta;
+                }
+            }
+            c0 = c1;
+        } while (row_of_col[c0] != 0);
+        do {
+            const int c1 = way[c0];
+            row_of_col[c0] = row_of_col[c1];
+            c0 = c1;
+        } while (c0);
+    }
+    col_of_row->assign(n, -1);
+    for (int c = 1; c <= n; ++c)
+        (*col_of_row)[row_of_col[c] - 1] = c - 1;
+}
+
+struct Placement {
+    int L, E, P;
+    const int64_t *counts;  // [L-1][E][E]
+
+    int64_t cnt(int j, int i, int p) const { return counts[((size_t)j * E + i) * E + p]; }
+
+    // Hops between consecutive layers whose experts sit on different GPUs.
+    int64_t cost(const std::vector<int32_t> &g) const
+    {
+        int64_t c = 0;
+        for (int j = 0; j + 1 < L; ++j)
+            for (int i = 0; i < E; ++i)
+                for (int p = 0; p < E; ++p)
+                    if (g[(size_t)j * E + i] != g[(size_t)(j + 1) * E + p])
+                        c += cnt(j, i, p);
+        return c;
+    }
+
+    // Re-places layer l given its neighbours (only the previous layer when !right, and then
+    // the result is taken even when it is not better); returns true if it changed the layer.
+    bool improve_layer(int l, std::vector<int32_t> *g, bool right = true) const
+    {
+        const int share = E / P;
+        std::vector<int64_t> score((size_t)E * P, 0);
+        if (l > 0)
+            for (int i = 0; i < E; ++i) {
+                const int q = (*g)[(size_t)(l - 1) * E + i];
+                for (int e = 0; e < E; ++e)
+                    score[(size_t)e * P + q] += cnt(l - 1, i, e);
+            }
+        if (right && l + 1 < L)
+            for (int e = 0; e < E; ++e)
+                for (int p = 0; p < E; ++p)
+                    score[(size_t)e * P + (*g)[(size_t)(l + 1) * E + p]] += cnt(l, e, p);
+        int64_t current = 0;
+        for (int e = 0; e < E; ++e)
+            current += score[(size_t)e * P + (*g)[(size_t)l * E + e]];
+        // GPU q owns columns [q*share, (q+1)*share) of the square assignment.
+        std::vector<int64_t> cost((size_t)E * E);
+        for (int e = 0; e < E; ++e)
+            for (int c = 0; c < E; ++c)
+                cost[(size_t)e * E + c] = -score[(size_t)e * P + c / share];
+        std::vector<int> col;
+        min_cost_assignment(E, cost, &col);
+        int64_t best = 0;
+        for (int e = 0; e < E; ++e)
+            best += score[(size_t)e * P + col[e] / share];
+        if (right && best <= current)
+            return false;
+        bool changed = false;
+        for (int e = 0; e < E; ++e) {
+            changed |= (*g)[(size_t)l * E + e] != col[e] / share;
+            (*g)[(size_t)l * E + e] = col[e] / share;
+        }
+        return changed;
+    }
+};
+
+// splitmix64 (Steele, Lea and Flood, "Fast splittable pseudorandom number generators", 2014).
+inline uint64_t splitmix64(uint64_t *state)
+{
+    uint64_t z = (*state += 0x9E3779B97F4A7C15ull);
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// Start 0: every layer contiguous (expert e on GPU e / (E/P)), so the result is never worse
+// than that placement. Start 1: layer 0 contiguous. Start s >= 2: layer 0 a shuffle of the
+// contiguous assignment (Fisher-Yates driven by splitmix64 seeded with s); for odd s every
+// other layer is shuffled the same way. Returns true when the later layers are still to be
+// built from layer 0 (each placed best given the one before it).
+inline bool initial_placement(int L, int E, int P, int start, std::vector<int32_t> *g)
+{
+    const int share = E / P;
+    g->assign((size_t)L * E, 0);
+    uint64_t state = (uint64_t)start;
+    for (int l = 0; l < L; ++l) {
+        int32_t *row = g->data() + (size_t)l * E;
+        for (int e = 0; e < E; ++e)
+            row[e] = e / share;
+        if (start >= 2 && (l == 0 || start % 2 == 1))
+            for (int e = E - 1; e > 0; --e) {
+                const int k = (int)(splitmix64(&state) % (uint64_t)(e + 1));
+                std::swap(row[e], row[k]);
+            }
+    }
+    return start == 1 || (start >= 2 && start % 2 == 0);
+}
+
+// Block coordinate descent: each layer re-placed best given its neighbours, forward then
+// backward, until a sweep changes nothing (at most 64 sweeps).
+inline void descend(const Placement &pl, std::vector<int32_t> *g)
+{
+    for (int sweep = 0; sweep < 64 && pl.L > 1; ++sweep) {
+        bool moved = false;
+        for (int l = 0; l < pl.L; ++l)
+            moved |= pl.improve_layer(l, g);
+        for (int l = pl.L - 2; l > 0; --l)
+            moved |= pl.improve_layer(l, g);
+        if (!moved)
+            break;
+    }
+}
+
+inline void place_experts(int L, int E, int P, const int64_t *counts, int starts,
+                          int32_t *gpu_of, int64_t *cost_out, int64_t *contiguous_out)
+{
+    const Placement pl{L, E, P, counts};
+    std::vector<int32_t> best, g, h;
+    int64_t best_cost = INT64_MAX;
+    for (int s = 0; s < starts; ++s) {
+        const bool build = initial_placement(L, E, P, s, &g);
+        if (s == 0 && contiguous_out)
+            *contiguous_out = pl.cost(g);
+        if (build)
+            for (int l = 1; l < L; ++l)
+                pl.improve_layer(l, &g, false);
+        descend(pl, &g);
+        int64_t c = pl.cost(g);
+        // Kicks: swap two pairs of experts (on different GPUs) in one layer, descend again,
+        // keep the result if it is cheaper.
+        uint64_t state = 0x5eedull + (uint64_t)s;
+        for (int kick = 0; kick < 4 * L && L > 1 && P > 1; ++kick) {
+            h = g;
+            const int l = (int)(splitmix64(&state) % (uint64_t)L);
+            for (int t = 0; t < 2; ++t) {
+                const int a = (int)(splitmix64(&state) % (uint64_t)E);
+                const int b = (int)(splitmix64(&state) % (uint64_t)E);
+                std::swap(h[(size_t)l * E + a], h[(size_t)l * E + b]);
+            }
+            descend(pl, &h);
+            const int64_t ch = pl.cost(h);
+            if (ch < c) {
+                c = ch;
+                g.swap(h);
+            }
+        }
+        if (c < best_cost) {
+            best_cost = c;
+            best = g;
+        }
+    }
+    std::copy(best.begin(), best.end(), gpu_of);
+    if (cost_out)
+        *cost_out = best_cost;
+}
+
+}  // namespace moe_plan

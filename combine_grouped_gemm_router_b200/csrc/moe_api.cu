@@ -10,6 +10,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "dispatch.cuh"
+#include "exchange_plan.cuh"
 #include "grouped_gemm.cuh"
 #include "route.cuh"
 
@@ -1429,6 +1430,41 @@ moe_read_stats(const moe_stats_t *stats_dev, moe_stats_t *out, moe_stream_t stre
             cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_exchange_schedule(int32_t W, const int64_t *D, int32_t max_phases, int32_t *phase_dst,
+                      int64_t *phase_len, int32_t *n_phases, int64_t *makespan)
+{
+    if (!D || !n_phases || !makespan || W < 1 || W > kMaxW || max_phases < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (max_phases > 0 && (!phase_dst || !phase_len))
+        return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < W * W; ++i)
+        if (D[i] < 0)
+            return MOE_ERR_INVALID_ARG;
+    int np = 0;
+    int64_t span = 0;
+    if (!moe_plan::exchange_schedule(W, D, max_phases, phase_dst, phase_len, &np, &span))
+        return MOE_ERR_INVALID_ARG;
+    *n_phases = np;
+    *makespan = span;
+    return MOE_OK;
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts, int32_t starts,
+                  int32_t *gpu_of, int64_t *cost, int64_t *contiguous_cost)
+{
+    if (!gpu_of || (L > 1 && !counts) || L < 1 || E < 1 || E > kMaxE || P < 1 || E % P != 0 ||
+        starts < 1 || starts > 64)
+        return MOE_ERR_INVALID_ARG;
+    if (L > 1)
+        for (size_t i = 0; i < (size_t)(L - 1) * E * E; ++i)
+            if (counts[i] < 0)
+                return MOE_ERR_INVALID_ARG;
+    moe_plan::place_experts(L, E, P, counts, starts, gpu_of, cost, contiguous_cost);
     return MOE_OK;
 }
 

@@ -391,6 +391,51 @@ moe_status_t moe_derive_report(const moe_shape_t *shape, const moe_stats_t *stat
                                const int64_t *rank_matrix, const int32_t *kept,
                                moe_report_t *out);
 
+/* Receiver-contention-free transmission order of one exchange of the packed rows.
+ * [MoE Inference Communication, §Aurora 场景 1: 定理 4.2 (the bound) and the scheduling rule
+ *  that follows it (no receiver is fed by two senders at once)]
+ * rank_matrix: HOST [W][W] int64, D[i][j] = rows rank i sends to rank j (moe_dispatch's
+ *   rank_matrix); the diagonal stays on its rank and is not scheduled. Entries must be >= 0.
+ * Output, HOST, caller-owned: phases s = 0 .. *n_phases - 1. During phase s, which lasts
+ *   phase_len[s] rows (> 0), rank i sends to rank phase_dst[s*W + i], or nothing when that is
+ *   -1; within a phase no receiver appears twice and no rank sends to itself. Summed over the
+ *   phases, rank i sends D[i][j] rows to every j != i. *makespan = the sum of phase_len =
+ *   max(max_i sum_{j!=i} D[i][j], max_j sum_{i!=j} D[i][j]) (tau_min of moe_derive_report):
+ *   the order reaches the theorem's lower bound. Phases with the same destinations follow
+ *   each other only once merged. At most 2*W*W phases: max_phases >= 2*W*W always suffices;
+ *   a smaller max_phases that the order does not fit returns MOE_ERR_INVALID_ARG.
+ * phase_dst holds max_phases*W int32, phase_len max_phases int64. Pure host computation,
+ * needs no GPU. Errors: null pointers, W outside [1, 64], a negative entry, max_phases < 0. */
+moe_status_t moe_exchange_schedule(int32_t W, const int64_t *rank_matrix, int32_t max_phases,
+                                   int32_t *phase_dst, int64_t *phase_len, int32_t *n_phases,
+                                   int64_t *makespan);
+
+/* Expert placement across GPUs from inter-layer expert affinity.
+ * [MoE Inference Communication, §ExFlow 形式化：整数线性规划建模: minimise the token hops
+ *  between consecutive layers whose experts sit on different GPUs, every GPU holding E/P
+ *  experts of every layer and every expert on one GPU]
+ * counts: HOST [L-1][E][E] int64, counts[j][i][p] = token hops from expert i of layer j to
+ *   expert p of layer j+1 (moe_affinity_accumulate of layers j and j+1), entries >= 0.
+ * gpu_of: HOST out [L][E] int32: the GPU (0 .. P-1) of expert e of layer l; each GPU gets
+ *   exactly E/P experts per layer. Deploying it means storing layer l's experts GPU by GPU.
+ * cost (nullable): sum over j, i, p of counts[j][i][p] where gpu_of[j][i] != gpu_of[j+1][p],
+ *   for the returned placement; contiguous_cost (nullable): the same for the contiguous
+ *   placement (expert e on GPU e / (E/P)), the default of moe_dispatch's rank emulation.
+ * Method: a heuristic, not the pages' exact ILP. From `starts` initial placements (all layers
+ *   contiguous; layer 0 contiguous or shuffled with the later layers built one by one, each
+ *   best given the one before; all layers shuffled), each layer in turn is re-placed optimally
+ *   given its two neighbours (an assignment problem, Hungarian method), forward and backward,
+ *   until nothing improves (at most 64 sweeps); then, 4*L times, two pairs of experts of one layer
+ *   are swapped and the descent repeated, keeping the result when it is cheaper. The cheapest
+ *   placement over the starts is returned; start 0 makes it never worse than contiguous.
+ *   Deterministic. Cost grows as starts * L^2 * E^3 (E = 64, L = 4, 16 starts: about 0.4 s;
+ *   E = 256: about 15 s).
+ * Errors: null counts (L > 1) or gpu_of; L < 1; E outside [1, 256]; P < 1 or E % P != 0;
+ *   starts outside [1, 64]; a negative count. Pure host computation, needs no GPU. */
+moe_status_t moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts,
+                               int32_t starts, int32_t *gpu_of, int64_t *cost,
+                               int64_t *contiguous_cost);
+
 /* Reads (and, if clear != 0, resets) the calling device's sticky error word. Synchronises
  * the device. Returns MOE_OK when no kernel has recorded an error. */
 moe_status_t moe_get_device_error(int clear);

@@ -27,7 +27,10 @@ and skips x):
 * expert weights W1, W3 [E][f][d] and W2 [E][d][f] ~ N(0, 0.02^2) (std 0.02),
   rounded to bf16;
 * Zipf(s) bias: bias[e] = -s * ln(e + 1), computed in float64, stored fp32
-  (expert 0 hottest); s = 0 means no bias (None).
+  (expert 0 hottest); s = 0 means no bias (None);
+* ``stack4_affinity`` replaces each layer's router by one that leans on the
+  previous layer's with its experts permuted (``affine_router``), so that the
+  inter-layer expert affinity a trained model shows is present.
 """
 from __future__ import annotations
 
@@ -55,6 +58,7 @@ class Workload:
     slot_major: bool = False  # drop priority: first choices before second choices
     reroute: bool = False     # move overflowed assignments to the next-best non-full expert
     fp8: bool = False         # e4m3 dispatch payload and gate/up GEMM
+    affinity: float = 0.0     # stacks: correlation of a layer's router with the previous one's
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -84,6 +88,10 @@ WORKLOADS = {
                               s=1.1, fp8=True),
     # the weight-bound decode layer and the 4-layer stack on the FP8 path
     "decode_fp8": Workload("decode_fp8", N=16, d=7168, f=2048, E=256, K=8, W=8, fp8=True),
+    # the stack with inter-layer expert affinity planted in the routers (rho = 0.9): the routing
+    # structure a trained model shows, for the placement report
+    "stack4_affinity": Workload("stack4_affinity", N=32768, d=4096, f=1536, E=64, K=6, W=8,
+                                cf=1.25, layers=4, affinity=0.9),
     "stack4_fp8": Workload("stack4_fp8", N=32768, d=4096, f=1536, E=64, K=6, W=8, cf=1.25,
                            layers=4, fp8=True),
     # the Mixtral-shaped layer with half the experts and tokens (same rows per expert,
@@ -106,6 +114,28 @@ def zipf_bias(E: int, s: float) -> Optional[torch.Tensor]:
         torch.float32)
 
 
+def affine_router(w: Workload, seed: int, layer: int, device: str = "cpu") -> torch.Tensor:
+    """Router [E][d] fp32 of layer ``layer`` of a stack with planted inter-layer affinity
+    (``w.affinity`` = rho > 0): R_0 = Z_0 and R_l = rho * R_{l-1}[pi_l] + sqrt(1 - rho^2) * Z_l,
+    where Z_l ~ N(0, 1/d) and pi_l is a permutation of the experts, both drawn from a generator
+    seeded ``seed + 1000*l + 7``. Row e of layer l leans on row pi_l[e] of layer l-1, so tokens
+    that chose expert pi_l[e] tend to choose expert e next (the residual stream changes little
+    from one layer to the next). Every entry keeps variance 1/d."""
+    rho = w.affinity
+    r = None
+    for j in range(layer + 1):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed + 1000 * j + 7)
+        z = torch.randn(w.E, w.d, generator=g, device=device,
+                        dtype=torch.float32) * (1.0 / math.sqrt(w.d))
+        if j == 0:
+            r = z
+        else:
+            perm = torch.randperm(w.E, generator=g, device=device)
+            r = rho * r[perm] + math.sqrt(1.0 - rho * rho) * z
+    return r
+
+
 def make_layer_inputs(w: Workload, seed: int = 0, device: str = "cpu", layer: int = 0,
                       with_x: bool = True) -> dict:
     """Draw one layer's inputs. Returns a dict of tensors on ``device``.
@@ -126,6 +156,8 @@ def make_layer_inputs(w: Workload, seed: int = 0, device: str = "cpu", layer: in
     else:
         out["w_router"] = torch.randn(w.E, w.d, generator=g, device=device,
                                       dtype=torch.float32) * (1.0 / math.sqrt(w.d))
+    if w.affinity > 0.0:  # drawn above to keep the draw order; replaced by the planted router
+        out["w_router"] = affine_router(w, seed, layer, device)
     b = zipf_bias(w.E, w.s)
     out["bias"] = None if b is None else b.to(device)
     for name, shape in (("w1", (w.E, w.f, w.d)), ("w3", (w.E, w.f, w.d)), ("w2", (w.E, w.d, w.f))):

@@ -145,3 +145,89 @@ def swiglu_rows(x_u16, w1_u16, w3_u16, w2_u16, row_token, row_expert):
         H = G / (1.0 + np.exp(-G)) * U
         y[sel] = H @ w2[e].T
     return y
+
+
+def min_unit_slots(D) -> int:
+    """Fewest unit time slots that carry the off-diagonal traffic of a small integer matrix D
+    when, in one slot, every sender sends one row to at most one receiver and every receiver
+    takes at most one row: breadth-first search over the remaining traffic."""
+    D = np.array(D, dtype=np.int64)
+    W = D.shape[0]
+    np.fill_diagonal(D, 0)
+    cells = [(i, j) for i in range(W) for j in range(W) if i != j]
+
+    def matchings(rem):
+        out = []
+
+        def grow(k, used_r, used_c, chosen):
+            if k == len(cells):
+                if chosen:
+                    out.append(tuple(chosen))
+                return
+            grow(k + 1, used_r, used_c, chosen)
+            i, j = cells[k]
+            if rem[i][j] > 0 and i not in used_r and j not in used_c:
+                grow(k + 1, used_r | {i}, used_c | {j}, chosen + [(i, j)])
+
+        grow(0, frozenset(), frozenset(), [])
+        return out
+
+    start = tuple(tuple(int(v) for v in r) for r in D)
+    if not any(any(r) for r in start):
+        return 0
+    frontier, seen, depth = {start}, {start}, 0
+    while frontier:
+        depth += 1
+        nxt = set()
+        for s in frontier:
+            for mt in matchings(s):
+                rem = [list(r) for r in s]
+                for i, j in mt:
+                    rem[i][j] -= 1
+                t = tuple(tuple(r) for r in rem)
+                if not any(any(r) for r in t):
+                    return depth
+                if t not in seen:
+                    seen.add(t)
+                    nxt.add(t)
+        frontier = nxt
+    raise AssertionError("unreachable")
+
+
+def balanced_placements(E: int, P: int):
+    """Every assignment of E experts to P GPUs with E/P experts each."""
+    share = E // P
+    out = []
+
+    def rec(e, load, cur):
+        if e == E:
+            out.append(tuple(cur))
+            return
+        for g in range(P):
+            if load[g] < share:
+                load[g] += 1
+                cur.append(g)
+                rec(e + 1, load, cur)
+                cur.pop()
+                load[g] -= 1
+
+    rec(0, [0] * P, [])
+    return out
+
+
+def best_placement_cost(counts, P: int) -> int:
+    """Exhaustive minimum over all balanced placements of every layer of the crossing hops."""
+    import itertools
+    counts = np.asarray(counts, dtype=np.int64)
+    Lm1, E, _ = counts.shape
+    opts = balanced_placements(E, P)
+    best = None
+    for combo in itertools.product(opts, repeat=Lm1 + 1):
+        c = 0
+        for j in range(Lm1):
+            for i in range(E):
+                for p in range(E):
+                    if combo[j][i] != combo[j + 1][p]:
+                        c += int(counts[j, i, p])
+        best = c if best is None else min(best, c)
+    return best

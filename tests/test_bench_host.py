@@ -21,6 +21,7 @@ sys.path.insert(0, ROOT)
     ("e128_skew_slot_major", 10),  # 1024 blocks per expert: the per-expert scan
     ("e128_skew_reroute", 14),     # two dispatch passes and the ranking kernel
     ("stack4", 12),                # 512 blocks per expert, pair GEMMs
+    ("stack4_affinity", 12),
     ("residual_top1", 14),         # shared MLP: offsets, pair + single GEMMs twice
 ])
 def test_kernel_launch_count(name, count):
@@ -43,3 +44,45 @@ def test_reference_arm_json_line():
     assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "tiny"
+
+
+def test_exchange_and_placement_reports():
+    import numpy as np
+
+    import bench
+    import combine_grouped_gemm_router_b200 as m
+    from oracle import exchange_plan as xp
+    rng = np.random.default_rng(5)
+    D = rng.integers(0, 500, (8, 8)) * (np.arange(8) + 1)
+    rep = bench.exchange_report(m, D, row_bytes=8192)
+    assert rep["makespan_rows"] == xp.exchange_bound(D)
+    assert rep["rotation_rows"] >= rep["makespan_rows"]
+    assert rep["makespan_us_at_peer_copy"] == pytest.approx(
+        rep["makespan_rows"] * 8192 / (bench.PEER_COPY_GBS * 1e3))
+    counts = rng.integers(0, 9, (3, 16, 16))
+    rep = bench.placement_report(m, counts, 4, 16, 4)
+    assert rep["hops"] == int(counts.sum())
+    assert 0.0 <= rep["cross_fraction_placed"] <= rep["cross_fraction_contiguous"] <= 1.0
+
+
+def test_affine_router_leans_on_the_previous_layer():
+    """Layer l's router row e is rho times the previous layer's row pi_l[e] plus independent
+    noise: the correlation of matched rows is rho, and every entry keeps variance 1/d."""
+    import math
+
+    import torch
+
+    from moe_workloads import WORKLOADS, affine_router, make_layer_inputs
+    w = WORKLOADS["stack4_affinity"].with_(N=64, d=1024, f=128)
+    r0, r1 = affine_router(w, 0, 0), affine_router(w, 0, 1)
+    assert float(r1.var()) * w.d == pytest.approx(1.0, rel=0.05)
+    corr = (r1 @ r0.T) / (r1.norm(dim=1, keepdim=True) * r0.norm(dim=1)[None, :])
+    best = corr.max(dim=1).values
+    assert float(best.mean()) == pytest.approx(w.affinity, abs=0.02)
+    assert sorted(corr.argmax(dim=1).tolist()) == list(range(w.E))   # a permutation
+    # the expert weights are the plain stack's: the draw order is unchanged
+    plain = make_layer_inputs(w.with_(affinity=0.0), seed=0, layer=1, with_x=False)
+    planted = make_layer_inputs(w, seed=0, layer=1, with_x=False)
+    assert torch.equal(plain["w2"], planted["w2"])
+    assert torch.equal(planted["w_router"], r1)
+    assert not math.isclose(float((plain["w_router"] - r1).abs().max()), 0.0)

@@ -1,0 +1,201 @@
+"""Exchange planning on the host: the contention-free transmission order and the expert
+placement of the C library against the oracle (CPU only; the functions need no GPU).
+
+Pins of the oracle itself: the exchange bound against a breadth-first search for the fewest
+unit slots (König's theorem says they agree), and the placement ILP against exhaustive search
+over every balanced placement.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import brute
+from oracle import exchange_plan as xp
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+@pytest.fixture(scope="module")
+def m():
+    import combine_grouped_gemm_router_b200 as mod
+    return mod
+
+
+# ------------------------------------------------------------------ pins of the oracle
+
+@pytest.mark.parametrize("seed", range(12))
+def test_exchange_bound_is_the_fewest_unit_slots(seed):
+    rng = np.random.default_rng(seed)
+    W = 2 + seed % 2
+    D = rng.integers(0, 3, (W, W))
+    assert xp.exchange_bound(D) == brute.min_unit_slots(D)
+
+
+def test_exchange_bound_hand_example():
+    # off-diagonal row sums 2, 4, 8; column sums 5, 6, 3 -> the busiest rank sends 8 rows
+    D = [[5, 2, 0], [1, 0, 3], [4, 4, 9]]
+    assert xp.exchange_bound(D) == 8
+    assert xp.exchange_bound([[7]]) == 0
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_placement_ilp_is_the_exhaustive_optimum(seed):
+    rng = np.random.default_rng(100 + seed)
+    L, E, P = [(2, 4, 2), (3, 4, 2), (2, 6, 3), (3, 6, 2), (2, 6, 2), (4, 4, 2)][seed]
+    counts = rng.integers(0, 6, (L - 1, E, E))
+    opt, g = xp.ilp_placement(counts, P)
+    assert opt == brute.best_placement_cost(counts, P)
+    assert xp.placement_cost(counts, g) == opt
+    for layer in g:
+        assert np.bincount(layer, minlength=P).tolist() == [E // P] * P
+
+
+def test_placement_cost_hand_example():
+    # two layers of 4 experts on 2 GPUs; expert 0 -> 2 (3 hops), 1 -> 3 (2 hops), 0 -> 0 (1 hop)
+    counts = np.zeros((1, 4, 4), np.int64)
+    counts[0, 0, 2], counts[0, 1, 3], counts[0, 0, 0] = 3, 2, 1
+    contiguous = xp.contiguous_placement(2, 4, 2)        # {0,1} on GPU 0, {2,3} on GPU 1
+    assert xp.placement_cost(counts, contiguous) == 5    # 0 -> 2 and 1 -> 3 cross
+    swapped = np.array([[0, 0, 1, 1], [1, 1, 0, 0]])      # layer 1 mirrored
+    assert xp.placement_cost(counts, swapped) == 1       # only 0 -> 0 crosses
+
+
+# ------------------------------------------------------------------ the library
+
+def check_schedule(D, dst, ln, span):
+    D = np.asarray(D, dtype=np.int64)
+    W = D.shape[0]
+    assert dst.shape == (len(ln), W)
+    assert (ln > 0).all()
+    assert len(ln) <= 2 * W * W
+    sent = np.zeros_like(D)
+    for s in range(len(ln)):
+        d = dst[s]
+        busy = d[d >= 0]
+        assert len(set(busy.tolist())) == len(busy), "a receiver fed by two senders"
+        assert all(d[i] != i for i in range(W))
+        assert ((d >= -1) & (d < W)).all()
+        for i in range(W):
+            if d[i] >= 0:
+                sent[i, d[i]] += ln[s]
+        if s > 0:
+            assert (dst[s] != dst[s - 1]).any(), "equal neighbouring phases are merged"
+    off = D.copy()
+    np.fill_diagonal(off, 0)
+    assert (sent == off).all()
+    assert int(ln.sum()) == span
+
+
+SCHEDULE_CASES = [
+    ("one_rank", lambda r: np.array([[9]])),
+    ("zeros", lambda r: np.zeros((8, 8), np.int64)),
+    ("diagonal_only", lambda r: np.diag(r.integers(1, 50, 8))),
+    ("uniform_8", lambda r: r.integers(0, 1000, (8, 8))),
+    ("skewed_8", lambda r: (r.integers(0, 100, (8, 8)) * (np.arange(8) + 1) ** 2)),
+    ("one_hot_receiver", lambda r: np.outer(r.integers(1, 9, 8), np.eye(8)[3]).astype(np.int64)),
+    ("sparse_16", lambda r: r.integers(0, 50, (16, 16)) * (r.random((16, 16)) < 0.2)),
+    ("dense_64", lambda r: r.integers(0, 10000, (64, 64))),
+    ("two_ranks", lambda r: np.array([[3, 11], [4, 0]])),
+]
+
+
+@pytest.mark.parametrize("name,make", SCHEDULE_CASES, ids=[c[0] for c in SCHEDULE_CASES])
+def test_exchange_schedule_reaches_the_bound(m, name, make):
+    D = make(np.random.default_rng(7))
+    dst, ln, span = m.moe_exchange_schedule(D)
+    assert span == xp.exchange_bound(D)
+    check_schedule(D, dst, ln, span)
+
+
+def test_exchange_schedule_on_dispatch_traffic(m):
+    """The traffic matrix of a real routing (oracle positions of a skewed top-8 routing)."""
+    import oracle
+    rng = np.random.default_rng(3)
+    N, E, K, W = 512, 32, 4, 8
+    logits = rng.standard_normal((N, E)) - 0.8 * np.log1p(np.arange(E))
+    idx = np.argsort(-logits, axis=1, kind="stable")[:, :K].astype(np.int32)
+    for C in (N * K, 40):
+        D = oracle.positions(idx, E, W, C)["D"].reshape(W, W)
+        dst, ln, span = m.moe_exchange_schedule(D)
+        assert span == xp.exchange_bound(D)
+        check_schedule(D, dst, ln, span)
+
+
+def test_exchange_schedule_errors(m):
+    D = np.random.default_rng(0).integers(1, 9, (8, 8))
+    with pytest.raises(m.MoeError):
+        m.moe_exchange_schedule(D, max_phases=1)     # the order needs more phases
+    bad = D.copy()
+    bad[1, 2] = -1
+    with pytest.raises(m.MoeError):
+        m.moe_exchange_schedule(bad)
+    with pytest.raises(m.MoeError):
+        m.moe_exchange_schedule(np.zeros((65, 65), np.int64))
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_placement_valid_and_costed(m, seed):
+    rng = np.random.default_rng(200 + seed)
+    L, E, P = [(2, 8, 2), (3, 8, 4), (4, 16, 4), (2, 64, 8), (4, 64, 8), (3, 32, 8),
+               (2, 8, 8), (3, 12, 3)][seed]
+    counts = rng.integers(0, 20, (L - 1, E, E))
+    g, cost, base = m.moe_place_experts(counts, L, E, P, starts=4)
+    for layer in g:
+        assert np.bincount(layer, minlength=P).tolist() == [E // P] * P
+    assert cost == xp.placement_cost(counts, g)
+    assert base == xp.placement_cost(counts, xp.contiguous_placement(L, E, P))
+    assert cost <= base
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_placement_matches_the_ilp_on_small_layers(m, seed):
+    """The local search never beats the ILP's optimum (a check of both), and with 8 starts it
+    reaches that optimum on each of these seeded random stacks. That is a property of these
+    instances, not a guarantee of the method (one start can stop well above it)."""
+    rng = np.random.default_rng(300 + seed)
+    L, E, P = [(2, 4, 2), (3, 4, 2), (2, 6, 2), (3, 6, 3), (2, 8, 2), (3, 8, 2), (2, 8, 4),
+               (4, 6, 2), (3, 8, 4), (2, 9, 3)][seed]
+    counts = rng.integers(0, 10, (L - 1, E, E))
+    opt, _ = xp.ilp_placement(counts, P)
+    _, one, _ = m.moe_place_experts(counts, L, E, P, starts=1)
+    assert opt <= one
+    _, cost, _ = m.moe_place_experts(counts, L, E, P, starts=8)
+    assert cost == opt
+
+
+def test_placement_recovers_planted_affinity(m):
+    """Layers whose experts hand tokens on to one partner expert each (a permutation per layer
+    pair, with a little noise): the best placement keeps every partner pair on one GPU."""
+    rng = np.random.default_rng(11)
+    L, E, P = 4, 64, 8
+    counts = rng.integers(0, 2, (L - 1, E, E))
+    planted = 0
+    for j in range(L - 1):
+        perm = rng.permutation(E)
+        counts[j, np.arange(E), perm] += 500
+        planted += 500 * E
+    g, cost, base = m.moe_place_experts(counts, L, E, P, starts=4)
+    noise = int(counts.sum()) - planted
+    assert cost <= noise                    # no planted hop crosses GPUs
+    assert base > 0.8 * planted * (1 - 1 / P)
+
+
+def test_placement_degenerate_shapes(m):
+    g, cost, base = m.moe_place_experts(np.zeros(0, np.int64), 1, 8, 2)
+    assert g.tolist() == [[0, 0, 0, 0, 1, 1, 1, 1]] and cost == 0 and base == 0
+    g, cost, base = m.moe_place_experts(np.ones((1, 4, 4), np.int64), 2, 4, 1)
+    assert (g == 0).all() and cost == 0 and base == 0
+    g, cost, base = m.moe_place_experts(np.ones((1, 4, 4), np.int64), 2, 4, 4)
+    assert cost == base == 12          # one expert per GPU: 4 of the 16 hops stay
+
+
+def test_placement_errors(m):
+    c = np.ones((1, 8, 8), np.int64)
+    for args in [(c, 2, 8, 3), (c, 2, 8, 0), (-c, 2, 8, 2)]:
+        with pytest.raises(m.MoeError):
+            m.moe_place_experts(*args)
+    with pytest.raises(m.MoeError):
+        m.moe_place_experts(c, 2, 8, 2, starts=0)
+    with pytest.raises(m.MoeError):
+        m.moe_place_experts(np.ones((1, 300, 300), np.int64), 2, 300, 2)
