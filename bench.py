@@ -621,7 +621,9 @@ def run_gpu(args, w) -> dict:
             work[k] = work.get(k, 0.0) + v
     peaks = load_peaks()
     up_ratio = 2.0 if w.fp8 else 1.0  # e4m3 tensor throughput is twice bf16's (nominal)
-    up_peak = peaks["bf16_tflops"] * up_ratio
+    # the GEMM is timed inside a long run of steps at the power cap, so its peak is the
+    # sustained cuBLAS figure; the burst figure (a GEMM timed alone) is reported beside it
+    up_peak = peaks["bf16_tflops_sustained"] * up_ratio
     up_s = stage_ms["expert_up"] / 1e3
     down_s = stage_ms["expert_down"] / 1e3
     up_tflops = work["up_flops"] / up_s / 1e12
@@ -640,9 +642,10 @@ def run_gpu(args, w) -> dict:
                    if w.fp8 else "grouped GEMM gate/up (moe_expert_up, tcgen05)")
     tensor_line = {"achieved": up_tflops, "peak": up_peak, "unit": "TFLOP/s",
                    "frac": up_tflops / up_peak,
-                   "peak_source": (peaks["source"] + " bf16 burst x 2 (the nominal e4m3/bf16 "
-                                   "dense ratio)" if w.fp8 else peaks["source"] + " bf16 burst"),
-                   "frac_of_sustained": up_tflops / (peaks["bf16_tflops_sustained"] * up_ratio)}
+                   "peak_source": (peaks["source"] + " bf16 sustained x 2 (the nominal "
+                                   "e4m3/bf16 dense ratio)" if w.fp8
+                                   else peaks["source"] + " bf16 sustained"),
+                   "frac_of_burst": up_tflops / (peaks["bf16_tflops"] * up_ratio)}
     hbm_line = {"achieved": up_gbs, "peak": hbm, "unit": "GB/s", "frac": up_gbs / hbm,
                 "peak_source": peaks["source"] + " copy bandwidth"}
     roofline = {"kernel": kernel_name, "bound": "tensor" if intensity >= balance else "hbm"}
