@@ -312,8 +312,9 @@ def algorithmic_work(w, R: int, E_act: int) -> dict:
         # (the FP8 payload writes one byte per element and a 4-byte scale per row)
         scatter_bytes=(N * d * 2 + 2 * R * (d + 4) + N * K * 4 * 3 if w.fp8
                        else N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3),
-        # combine: read every kept fp32 expert row, the routing, write fp32 out
-        combine_bytes=R * d * 4 + N * K * 8 + N * d * 4,
+        # combine: read every kept expert row (fp32, or the FP8 return payload: e4m3 codes and
+        # one exponent byte per 32 columns), the routing, write fp32 out
+        combine_bytes=(R * (d + d // 32) if w.fp8_return else R * d * 4) + N * K * 8 + N * d * 4,
     )
 
 
@@ -338,7 +339,7 @@ def run_gpu(args, w) -> dict:
               for l in range(L)]
     inp = layers[0]
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=L > 1,
-                         slot_major=w.slot_major, reroute=w.reroute)
+                         slot_major=w.slot_major, reroute=w.reroute, fp8_return=w.fp8_return)
     RA = m.moe_rows_alloc(shape)
     ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
     x = inp["x"]
@@ -371,7 +372,8 @@ def run_gpu(args, w) -> dict:
     D = torch.empty(W * W, dtype=torch.int64, device=dev)
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
     h = torch.empty(RA, f, dtype=torch.bfloat16, device=dev)
-    y = torch.empty(RA, d, dtype=torch.float32, device=dev)
+    # fp32 expert outputs, or the FP8 return payload (e4m3 codes + block exponents)
+    y = torch.empty(m.moe_y_bytes(shape), dtype=torch.uint8, device=dev)
     if L > 1:  # x_{l+1} = bf16(x_l + MoE_l(x_l)), ping-pong buffers
         xbuf = [torch.empty(N, d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
         affinity = torch.zeros(L - 1, E, E, dtype=torch.int64, device=dev)
@@ -669,7 +671,9 @@ def run_gpu(args, w) -> dict:
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": ("e4m3 (dispatch payload and both expert GEMMs' operands), fp32 accumulate"
+        "dtype": (("e4m3 (dispatch payload, both expert GEMMs' operands and the return "
+                   "payload), fp32 accumulate" if w.fp8_return else
+                   "e4m3 (dispatch payload and both expert GEMMs' operands), fp32 accumulate")
                   if w.fp8 else "bf16"),
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",

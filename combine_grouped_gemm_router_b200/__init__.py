@@ -58,6 +58,7 @@ _sigs = {
     "moe_rows_alloc": ([_SP], c_i64),
     "moe_workspace_size": ([_SP], c_size),
     "moe_layer_workspace_size": ([_SP], c_size),
+    "moe_y_bytes": ([_SP], c_size),
     "moe_route": ([_SP] + [c_p] * 7 + [c_size, c_p], c_i32),
     "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
     "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
@@ -151,13 +152,14 @@ def _stream(stream) -> Optional[int]:
 MOE_FLAG_OUT_BF16 = 1
 MOE_FLAG_SLOT_MAJOR = 2
 MOE_FLAG_REROUTE = 4
+MOE_FLAG_FP8_RETURN = 8
 
 
 def make_shape(N: int, d: int, f: int, E: int, K: int, W: int, capacity_factor: float = 0.0,
                out_bf16: bool = False, slot_major: bool = False,
-               reroute: bool = False) -> MoeShape:
+               reroute: bool = False, fp8_return: bool = False) -> MoeShape:
     flags = ((MOE_FLAG_OUT_BF16 if out_bf16 else 0) | (MOE_FLAG_SLOT_MAJOR if slot_major else 0)
-             | (MOE_FLAG_REROUTE if reroute else 0))
+             | (MOE_FLAG_REROUTE if reroute else 0) | (MOE_FLAG_FP8_RETURN if fp8_return else 0))
     return MoeShape(N, d, f, E, K, W, float(capacity_factor), flags)
 
 
@@ -173,6 +175,16 @@ def moe_status_string(status: int) -> str:
 
 def moe_capacity(shape: MoeShape) -> int:
     return _lib.moe_capacity(ctypes.byref(shape))
+
+
+def moe_y_bytes(shape: MoeShape) -> int:
+    """Bytes of the expert-output buffer y (fp32 rows, or the FP8 return payload)."""
+    return _lib.moe_y_bytes(ctypes.byref(shape))
+
+
+def y_payload_stride(shape: MoeShape) -> int:
+    """Row stride in bytes of the FP8 return payload: d codes + d/32 exponents, padded to 16."""
+    return shape.d + ((shape.d // 32 + 15) // 16) * 16
 
 
 def moe_rows_alloc(shape: MoeShape) -> int:

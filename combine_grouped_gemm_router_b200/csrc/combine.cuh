@@ -17,9 +17,35 @@ namespace moe {
 // result is stored as fp32, or rounded once to bf16 (OUT_BF16).
 // A warp's work item is one token and `seg` 8-column chunks of its row (the whole
 // row for large N; a slice when there are too few tokens to fill the GPU).
-template <bool OUT_BF16>
+// Y8: the expert outputs arrive as the FP8 return payload (rows of y_stride bytes: d e4m3
+// codes, then one exponent byte j + 127 per 32 columns); each value is decoded exactly
+// (e4m3 -> f16 -> f32, times 2^j) before the same fp32 accumulation.
+__device__ __forceinline__ float f16_to_f32(uint32_t h)
+{
+    float f;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"((unsigned short)h));
+    return f;
+}
+
+// Eight e4m3 codes (bytes of lo, then hi) -> eight floats scaled by sc (a power of two).
+__device__ __forceinline__ void decode_e4m3x8(uint32_t lo, uint32_t hi, float sc, float o[8])
+{
+    const uint32_t w[2] = {lo, hi};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        uint32_t a, b;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"((unsigned short)(w[i] & 0xFFFFu)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"((unsigned short)(w[i] >> 16)));
+        o[4 * i] = f16_to_f32(a & 0xFFFFu) * sc;
+        o[4 * i + 1] = f16_to_f32(a >> 16) * sc;
+        o[4 * i + 2] = f16_to_f32(b & 0xFFFFu) * sc;
+        o[4 * i + 3] = f16_to_f32(b >> 16) * sc;
+    }
+}
+
+template <bool OUT_BF16, bool Y8>
 __global__ void __launch_bounds__(256)
-    combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ row_of,
+    combine_kernel(const void *__restrict__ y, int y_stride, const int32_t *__restrict__ row_of,
                    const float *__restrict__ topk_w, const float *__restrict__ shared_y,
                    const uint16_t *__restrict__ residual, int N, int d, int K, int seg,
                    void *__restrict__ out)
@@ -55,21 +81,44 @@ __global__ void __launch_bounds__(256)
                 const float wk = __shfl_sync(0xffffffffu, w, k);
                 if (rk < 0)
                     continue;
-                float4 v[U][2];
+                if constexpr (Y8) {
+                    const uint8_t *prow = reinterpret_cast<const uint8_t *>(y) +
+                                          (size_t)rk * y_stride;
+                    uint2 v[U];
+                    uint32_t ex[U];
 #pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (c + 32 * u < cend) {
-                        v[u][0] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2];
-                        v[u][1] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2 + 1];
+                    for (int u = 0; u < U; ++u)
+                        if (c + 32 * u < cend) {
+                            v[u] = reinterpret_cast<const uint2 *>(prow)[c + 32 * u];
+                            ex[u] = prow[d + (c + 32 * u) / 4];
+                        }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (c + 32 * u < cend) {
+                            float f8[8];
+                            decode_e4m3x8(v[u].x, v[u].y, pow2f((int)ex[u] - 127), f8);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                acc[u][q] = __fmaf_rn(wk, f8[q], acc[u][q]);
+                        }
                     }
+                } else {
+                    float4 v[U][2];
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < cend) {
-                        const float f8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
-                                             v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+                    for (int u = 0; u < U; ++u)
+                        if (c + 32 * u < cend) {
+                            v[u][0] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2];
+                            v[u][1] = ysrc[((size_t)rk * nvec + c + 32 * u) * 2 + 1];
+                        }
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            acc[u][q] = __fmaf_rn(wk, f8[q], acc[u][q]);
+                    for (int u = 0; u < U; ++u) {
+                        if (c + 32 * u < cend) {
+                            const float f8[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                                                 v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                acc[u][q] = __fmaf_rn(wk, f8[q], acc[u][q]);
+                        }
                     }
                 }
             }

@@ -60,8 +60,11 @@ struct Args {
     int b_rows;          // rows of one expert's B matrix (f for mode 0, d for mode 1)
     int rows_alloc;      // rows of the A buffer
     int select;          // which experts this launch takes: 0 all, 1 pair-tile experts, 2 the rest
-    void *out;           // modes 0, 2: bf16 h [rows_alloc][ldo]; 1, 3: fp32 y [rows_alloc][ldo]
+    void *out;           // modes 0, 2: bf16 h [rows_alloc][ldo]; 1, 3: fp32 y [rows_alloc][ldo],
+                         // or the FP8 return payload when y_stride > 0
     int ldo;
+    int y_stride;        // modes 1, 3: 0, or the payload's row stride in bytes (ldo e4m3 codes,
+                         // then ldo / 32 exponent bytes, padded to 16 bytes)
     const float *row_scale;  // modes 2, 3: scale of each A row [rows_alloc]
     const float *b_scale0;   // mode 2: scale of each W1 row; mode 3: of each W2 row [E * b_rows]
     const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
@@ -390,12 +393,73 @@ constexpr int Y_STAGE_BYTES = 4 * 4096 + 1024;
 // the expert (wfull), each 32-column piece goes through the warp's shared-memory tile
 // (ystage) and one TMA store of 32 x 32 at (x = column, y = wrow0); otherwise every
 // thread stores its own row's values directly (no row past the expert is written).
+// FP8 return payload ("MoE 推理服务工程真相 2026", §6.3: the exchange's token data in FP8):
+// every 32-column block of a y row becomes 32 e4m3 codes and one exponent j (stored as the
+// byte j + 127), the smallest power of two with max|block| * 2^-j <= 448, as for the
+// dispatch payload. Row `row` of the payload: codes at [0, ldo), exponents at
+// [ldo, ldo + ldo / 32). The values quantised are the fp32 y values the plain mode stores.
+template <int MODE, int BN>
+__device__ __forceinline__ void down_epilogue_fp8_return(const Args &args, uint32_t taddr, int n,
+                                                         int row, bool store, float sx,
+                                                         const float *ss)
+{
+    constexpr int CB = epilogue_cols(MODE);
+    uint8_t *prow = reinterpret_cast<uint8_t *>(args.out) + (size_t)row * args.y_stride;
+    uint64_t exps = 0;  // BN / 32 <= 8 exponent bytes of this tile's row piece
+#pragma unroll 1
+    for (int c = 0; c < BN; c += CB) {
+        uint32_t v[CB];
+#pragma unroll
+        for (int q = 0; q < CB / 16; ++q)
+            tmem_ld16(taddr + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * q));
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < CB / 32; ++h) {
+            float f[32];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                float o = __uint_as_float(v[32 * h + k]);
+                if constexpr (MODE == 3)
+                    o *= sx * ss[c + 32 * h + k];
+                f[k] = o;
+                mx = max(mx, __float_as_uint(o) & 0x7FFFFFFFu);
+            }
+            const int j = e4m3_scale_exp(__uint_as_float(mx));
+            const float inv = pow2f(-j);
+            uint32_t p[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                p[k] = pack_e4m3x2(f[4 * k] * inv, f[4 * k + 1] * inv) |
+                       (pack_e4m3x2(f[4 * k + 2] * inv, f[4 * k + 3] * inv) << 16);
+            const int col = c + 32 * h;
+            if (store) {
+                uint4 *dst = reinterpret_cast<uint4 *>(prow + n * BN + col);
+                dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+                dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+            }
+            exps |= (uint64_t)(uint32_t)(j + 127) << (8 * (col / 32));
+        }
+    }
+    if (store) {
+        uint8_t *eb = prow + args.ldo + n * (BN / 32);
+        if constexpr (BN == 256)
+            *reinterpret_cast<uint2 *>(eb) = make_uint2((uint32_t)exps, (uint32_t)(exps >> 32));
+        else
+            *reinterpret_cast<uint32_t *>(eb) = (uint32_t)exps;
+    }
+}
+
 template <int MODE, int BN>
 __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int n, int row,
                                               bool store, float sx, const float *ss,
                                               const CUtensorMap *ymap, uint32_t ystage,
                                               int wrow0, bool wfull)
 {
+    if (args.y_stride > 0) {
+        down_epilogue_fp8_return<MODE, BN>(args, taddr, n, row, store, sx, ss);
+        return;
+    }
     constexpr int CB = epilogue_cols(MODE);
     const int lane = threadIdx.x & 31;
     float *frow = reinterpret_cast<float *>(args.out) + (size_t)row * args.ldo;

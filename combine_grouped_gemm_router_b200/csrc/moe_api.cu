@@ -60,11 +60,21 @@ int64_t capacity_of(const moe_shape_t *s)
     return (int64_t)ceil((double)s->capacity_factor * (double)s->N * (double)s->K / (double)s->E);
 }
 
+// Row stride in bytes of the FP8 return payload (d codes, d/32 exponent bytes padded to 16),
+// or 0 when y is fp32.
+int y_payload_stride(const moe_shape_t *s)
+{
+    if (!(s->flags & MOE_FLAG_FP8_RETURN))
+        return 0;
+    return s->d + ((s->d / 32 + 15) & ~15);
+}
+
 moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
 {
     if (!s)
         return MOE_ERR_INVALID_ARG;
-    if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE)) != 0)
+    if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE |
+                                MOE_FLAG_FP8_RETURN)) != 0)
         return MOE_ERR_INVALID_ARG;
     if (s->N < 0 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
         return MOE_ERR_INVALID_ARG;
@@ -75,6 +85,8 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
     if ((int64_t)s->N * s->K >= (int64_t)1 << 31)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (gemm && (s->d % 128 != 0 || s->f < 128 || s->f % 128 != 0))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((s->flags & MOE_FLAG_FP8_RETURN) && s->d % 128 != 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (g) {
         const int64_t NK = (int64_t)s->N * s->K;
@@ -591,12 +603,18 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
     return launch_gemm<0, 256>(tA, tW1, tW3, args, st);
 }
 
+// y_stride > 0: y is the FP8 return payload with that row stride (written by plain stores;
+// the y tensor map, unused then, is a copy of the W2 map).
 moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
-                       const int32_t *offsets, const uint16_t *w2, float *y, cudaStream_t st)
+                       const int32_t *offsets, const uint16_t *w2, void *y, int y_stride,
+                       cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
-    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d) ||
-        !make_tmap_y(&tY, y, d, (uint64_t)a_rows))
+    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
+        return MOE_ERR_CUDA;
+    if (y_stride > 0)
+        tY = tW2;
+    else if (!make_tmap_y(&tY, static_cast<float *>(y), d, (uint64_t)a_rows))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -606,6 +624,7 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     args.rows_alloc = (int)a_rows;
     args.out = y;
     args.ldo = d;
+    args.y_stride = y_stride;
     args.timeout_ns = kWaitTimeoutNs;
     args.select = 0;
     if (d % 256 == 0) {
@@ -664,11 +683,15 @@ moe_status_t gemm_up_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const 
 // channel), fp32 y. The pair kernel needs f % 256 == 0 (two atoms per stage).
 moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const uint8_t *hq,
                             const float *h_scale, const int32_t *offsets, const uint8_t *w2,
-                            const float *s2, float *y, cudaStream_t st)
+                            const float *s2, void *y, int y_stride, cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
     if (!make_tmap(&tA, hq, f, (uint64_t)a_rows, true) ||
-        !make_tmap(&tW2, w2, f, (uint64_t)E * d, true) || !make_tmap_y(&tY, y, d, (uint64_t)a_rows))
+        !make_tmap(&tW2, w2, f, (uint64_t)E * d, true))
+        return MOE_ERR_CUDA;
+    if (y_stride > 0)
+        tY = tW2;
+    else if (!make_tmap_y(&tY, static_cast<float *>(y), d, (uint64_t)a_rows))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -678,6 +701,7 @@ moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, cons
     args.rows_alloc = (int)a_rows;
     args.out = y;
     args.ldo = d;
+    args.y_stride = y_stride;
     args.row_scale = h_scale;
     args.b_scale0 = s2;
     args.timeout_ns = kWaitTimeoutNs;
@@ -716,15 +740,16 @@ moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint1
 }
 
 moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *h,
-                              const int32_t *offsets, const uint16_t *w2, float *y,
+                              const int32_t *offsets, const uint16_t *w2, void *y,
                               cudaStream_t st)
 {
-    return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y, st);
+    return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y,
+                     y_payload_stride(s), st);
 }
 
 moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                               const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
-                              const uint16_t *w2, uint16_t *h, float *y, cudaStream_t st)
+                              const uint16_t *w2, uint16_t *h, void *y, cudaStream_t st)
 {
     moe_status_t rc = expert_up_impl(s, g, x_sorted, offsets, w1, w3, h, st);
     if (rc != MOE_OK)
@@ -748,22 +773,31 @@ moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x
     moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, st);
     if (rc != MOE_OK)
         return rc;
-    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, st);
+    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, st);
 }
 
-moe_status_t combine_impl(const moe_shape_t *s, const float *y, const int32_t *row_of,
+moe_status_t combine_impl(const moe_shape_t *s, const void *y, const int32_t *row_of,
                           const float *topk_w, const float *shared_y, const uint16_t *residual,
                           void *out, cudaStream_t st)
 {
     const int nvec = s->d / 8;
     const int seg = row_slice(s->N, nvec, 64);
     const int blocks = row_blocks(s->N, nvec, seg);
-    if (s->flags & MOE_FLAG_OUT_BF16)
-        combine_kernel<true><<<blocks, 256, 0, st>>>(y, row_of, topk_w, shared_y, residual, s->N,
-                                                      s->d, s->K, seg, out);
+    const int ys = y_payload_stride(s);
+    const bool ob = (s->flags & MOE_FLAG_OUT_BF16) != 0;
+    if (ob && ys)
+        combine_kernel<true, true><<<blocks, 256, 0, st>>>(y, ys, row_of, topk_w, shared_y,
+                                                            residual, s->N, s->d, s->K, seg, out);
+    else if (ob)
+        combine_kernel<true, false><<<blocks, 256, 0, st>>>(y, 0, row_of, topk_w, shared_y,
+                                                             residual, s->N, s->d, s->K, seg, out);
+    else if (ys)
+        combine_kernel<false, true><<<blocks, 256, 0, st>>>(y, ys, row_of, topk_w, shared_y,
+                                                             residual, s->N, s->d, s->K, seg, out);
     else
-        combine_kernel<false><<<blocks, 256, 0, st>>>(y, row_of, topk_w, shared_y, residual, s->N,
-                                                       s->d, s->K, seg, out);
+        combine_kernel<false, false><<<blocks, 256, 0, st>>>(y, 0, row_of, topk_w, shared_y,
+                                                              residual, s->N, s->d, s->K, seg,
+                                                              out);
     return launch_status();
 }
 
@@ -848,6 +882,15 @@ __attribute__((visibility("default"))) size_t moe_layer_workspace_size(const moe
     if (check_shape(shape, true, &g) != MOE_OK)
         return 0;
     return layer_layout(shape, g, scratch_layout(shape, g).total).total;
+}
+
+__attribute__((visibility("default"))) size_t moe_y_bytes(const moe_shape_t *shape)
+{
+    Geometry g;
+    if (check_shape(shape, false, &g) != MOE_OK)
+        return 0;
+    const int ys = y_payload_stride(shape);
+    return (size_t)g.rows_alloc * (ys > 0 ? (size_t)ys : (size_t)shape->d * 4);
 }
 
 __attribute__((visibility("default"))) moe_status_t
@@ -1019,7 +1062,7 @@ moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted, const float
 
 __attribute__((visibility("default"))) moe_status_t
 moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_scale,
-                    const int32_t *offsets, const uint8_t *w2q, const float *w2_scale, float *y,
+                    const int32_t *offsets, const uint8_t *w2q, const float *w2_scale, void *y,
                     moe_stream_t stream)
 {
     Geometry g;
@@ -1034,14 +1077,14 @@ moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_
         !aligned4(offsets) || !aligned4(h_scale))
         return MOE_ERR_MISALIGNED;
     return gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
-                          hq, h_scale, offsets, w2q, w2_scale, y,
+                          hq, h_scale, offsets, w2q, w2_scale, y, y_payload_stride(shape),
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 __attribute__((visibility("default"))) moe_status_t
 moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_t *offsets,
                 const uint16_t *w1, const uint16_t *w3, const uint16_t *w2, uint16_t *h,
-                float *y, moe_stream_t stream)
+                void *y, moe_stream_t stream)
 {
     Geometry g;
     moe_status_t rc = check_shape(shape, true, &g);
@@ -1079,7 +1122,7 @@ moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted, const int32_t 
 
 __attribute__((visibility("default"))) moe_status_t
 moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
-                const uint16_t *w2, float *y, moe_stream_t stream)
+                const uint16_t *w2, void *y, moe_stream_t stream)
 {
     Geometry g;
     moe_status_t rc = check_shape(shape, true, &g);
@@ -1095,7 +1138,7 @@ moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offs
 }
 
 __attribute__((visibility("default"))) moe_status_t
-moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
+moe_combine(const moe_shape_t *shape, const void *y, const int32_t *row_of,
             const float *topk_w, const float *shared_y, const uint16_t *residual, void *out,
             moe_stream_t stream)
 {
@@ -1183,7 +1226,8 @@ moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16
         if (rc != MOE_OK)
             return rc;
         rc = gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc,
-                            use_pair_tiles(shape, g), hq, hs, offsets, up.w2q, up.s2, y, st);
+                            use_pair_tiles(shape, g), hq, hs, offsets, up.w2q, up.s2, y,
+                            y_payload_stride(shape), st);
     } else {
         rc = expert_down_impl(shape, g, h, offsets, up.w2, y, st);
     }

@@ -98,6 +98,20 @@ typedef struct moe_shape {
  * moe_dispatch_static. The dispatch then runs two passes plus a ranking kernel. */
 #define MOE_FLAG_REROUTE 4u
 
+/* FP8 return payload ("MoE 推理服务工程真相 2026", §6.3: the exchange's token data in FP8,
+ * here the expert outputs y that travel back to the tokens' ranks). With this flag the `y`
+ * buffer of moe_expert_down, moe_expert_down_fp8, moe_expert_gemm and moe_combine (and the
+ * layer's internal y) holds, per row, d e4m3 codes, then one exponent byte per 32 columns,
+ * zero-padded to a multiple of 16 bytes: row stride d + roundup16(d / 32) bytes,
+ * moe_y_bytes(shape) bytes in all. Block b of row r (columns [32b, 32b + 32)) with exponent
+ * byte j + 127 holds the values code * 2^j, where j is the smallest power of two with
+ * max|block| * 2^-j <= 448 (j in [-126, 127]; 0 for a zero or non-finite block) and each code
+ * is the value * 2^-j rounded to nearest-even e4m3, saturating: the dispatch payload's rule
+ * with a 32-column block in place of a row (a row of y spans several GEMM tiles, a block
+ * does not). The values quantised are the fp32 y the plain down GEMM writes; the combine
+ * decodes them exactly and accumulates in fp32 as before. Needs d % 128 == 0. */
+#define MOE_FLAG_FP8_RETURN 8u
+
 /* Per-call dispatch counters, written (not accumulated) by moe_dispatch / moe_layer into
  * DEVICE memory when a non-null pointer is given. Observability signals of
  * "MoE 专家并行的 All-to-All 通信瓶颈", §可观测指标与故障定位, and
@@ -147,6 +161,11 @@ size_t moe_workspace_size(const moe_shape_t *shape);
 
 /* Workspace bytes for moe_layer: every intermediate of the layer plus the scratch above. */
 size_t moe_layer_workspace_size(const moe_shape_t *shape);
+
+/* Bytes of the y buffer of moe_expert_down / moe_expert_gemm / moe_combine: rows_alloc * d * 4
+ * (fp32 y), or rows_alloc * (d + roundup16(d / 32)) with MOE_FLAG_FP8_RETURN. 0 on an invalid
+ * shape. */
+size_t moe_y_bytes(const moe_shape_t *shape);
 
 /* ---------------------------------------------------------------- stages */
 
@@ -245,23 +264,24 @@ moe_status_t moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x,
  *   h[r] = silu(x_sorted[r] W1[e]^T) * (x_sorted[r] W3[e]^T)   (bf16 out, fp32 accumulate)
  *   y[r] = h[r] W2[e]^T                                         (fp32 out, fp32 accumulate)
  * x_sorted [rows_alloc][d], w1, w3 [E][f][d], w2 [E][d][f], h [rows_alloc][f] bf16;
- * y [rows_alloc][d] fp32; offsets [E+1] device int32 (as written by moe_dispatch).
+ * y [rows_alloc][d] fp32 (the FP8 return payload with MOE_FLAG_FP8_RETURN, moe_y_bytes);
+ * offsets [E+1] device int32 (as written by moe_dispatch).
  * h is bf16 because it is the second GEMM's tensor-core operand; y stays fp32 so the
- * combine adds unrounded expert outputs.
+ * combine adds unrounded expert outputs (unless the flag asks for the FP8 payload).
  * Rows past offsets[E] are neither read for output nor written. Experts with no rows cost
  * nothing (their weights are not read). Needs d % 128 == 0, f % 128 == 0. */
 moe_status_t moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted,
                              const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
-                             const uint16_t *w2, uint16_t *h, float *y, moe_stream_t stream);
+                             const uint16_t *w2, uint16_t *h, void *y, moe_stream_t stream);
 
 /* The two halves of moe_expert_gemm as separate launches (same contracts as above):
  * moe_expert_up:   h = silu(x_sorted W1^T) * (x_sorted W3^T)   (gate/up GEMM, bf16 h)
- * moe_expert_down: y = h W2^T                                  (down GEMM, fp32 y) */
+ * moe_expert_down: y = h W2^T                     (down GEMM, fp32 y or the FP8 payload) */
 moe_status_t moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted,
                            const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                            uint16_t *h, moe_stream_t stream);
 moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
-                             const uint16_t *w2, float *y, moe_stream_t stream);
+                             const uint16_t *w2, void *y, moe_stream_t stream);
 
 /* ---- FP8 payload ("MoE 推理服务工程真相 2026", §6.3: send the token data of the all-to-all
  * as FP8 instead of BF16, half the bytes, at the cost of quantisation noise).
@@ -273,7 +293,7 @@ moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const 
  * e4m3 rows of W1 and W3 (one scale per output channel) on tcgen05 kind::f8f6f4; h is
  * written as bf16, its kept rows are then quantised to e4m3 the same way (one scale per
  * row), and the down projection runs on them and on e4m3 rows of W2 (one scale per output
- * channel); y and the combine stay fp32. */
+ * channel); y and the combine stay fp32 unless MOE_FLAG_FP8_RETURN is set. */
 
 /* Row-wise e4m3 quantisation of a bf16 matrix src [rows][cols] (DEVICE): codes [rows][cols]
  * uint8 and scale [rows] fp32 (DEVICE, caller-owned). For the experts' W1, W3 pass rows = E*f,
@@ -306,13 +326,14 @@ moe_status_t moe_expert_up_fp8(const moe_shape_t *shape, const uint8_t *x_sorted
                                const uint8_t *w1q, const float *w1_scale, const uint8_t *w3q,
                                const float *w3_scale, uint16_t *h, moe_stream_t stream);
 
-/* Down projection on e4m3 rows: y = sh * s2 * (hq W2q^T), fp32 y [rows_alloc][d]; hq e4m3
+/* Down projection on e4m3 rows: y = sh * s2 * (hq W2q^T), fp32 y [rows_alloc][d] (or the FP8
+ * return payload with MOE_FLAG_FP8_RETURN); hq e4m3
  * [rows_alloc][f] with h_scale per row (moe_quantize_rows_e4m3 of the bf16 h, rows =
  * offsets[E]); w2q e4m3 [E][d][f] with w2_scale [E][d] (16-byte aligned). d % 128 == 0,
  * f % 128 == 0. */
 moe_status_t moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_scale,
                                  const int32_t *offsets, const uint8_t *w2q, const float *w2_scale,
-                                 float *y, moe_stream_t stream);
+                                 void *y, moe_stream_t stream);
 
 /* Weighted combine back to token order.
  * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制 (weighted merge into the
@@ -321,9 +342,10 @@ moe_status_t moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, co
  * out[t] = (sum over k = 0..K-1 with row_of[t*K+k] >= 0 of topk_w[t][k] * y[row])
  *          + shared_y[t] + residual[t], accumulated in fp32 in k order, then the shared dense
  * MLP's output (nullable, fp32 [N][d], see moe_shared_expert), then the residual (nullable,
- * bf16 [N][d]). y [rows_alloc][d] fp32. out [N][d] is fp32, or bf16 (rounded once) when
- * shape->flags has MOE_FLAG_OUT_BF16; a bf16 out may alias residual. */
-moe_status_t moe_combine(const moe_shape_t *shape, const float *y, const int32_t *row_of,
+ * bf16 [N][d]). y [rows_alloc][d] fp32, or the FP8 return payload with MOE_FLAG_FP8_RETURN
+ * (each value decoded exactly before it is accumulated). out [N][d] is fp32, or bf16
+ * (rounded once) when shape->flags has MOE_FLAG_OUT_BF16; a bf16 out may alias residual. */
+moe_status_t moe_combine(const moe_shape_t *shape, const void *y, const int32_t *row_of,
                          const float *topk_w, const float *shared_y, const uint16_t *residual,
                          void *out, moe_stream_t stream);
 

@@ -59,6 +59,7 @@ class Workload:
     reroute: bool = False     # move overflowed assignments to the next-best non-full expert
     fp8: bool = False         # e4m3 dispatch payload and gate/up GEMM
     affinity: float = 0.0     # stacks: correlation of a layer's router with the previous one's
+    fp8_return: bool = False  # FP8 path: expert outputs travel back as e4m3 + block exponents
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -86,6 +87,13 @@ WORKLOADS = {
                                     W=8, router="uniform", fp8=True),
     "e128_skew_fp8": Workload("e128_skew_fp8", N=8192, d=2048, f=768, E=128, K=8, W=8, cf=1.25,
                               s=1.1, fp8=True),
+    # the FP8 path with the FP8 return payload as well (expert outputs as e4m3 codes with one
+    # power-of-two exponent per 32 columns)
+    "mixtral_prefill_fp8_return": Workload("mixtral_prefill_fp8_return", N=4096, d=4096, f=14336,
+                                           E=8, K=2, W=8, router="uniform", fp8=True,
+                                           fp8_return=True),
+    "e128_skew_fp8_return": Workload("e128_skew_fp8_return", N=8192, d=2048, f=768, E=128, K=8,
+                                     W=8, cf=1.25, s=1.1, fp8=True, fp8_return=True),
     # the weight-bound decode layer and the 4-layer stack on the FP8 path
     "decode_fp8": Workload("decode_fp8", N=16, d=7168, f=2048, E=256, K=8, W=8, fp8=True),
     # the stack with inter-layer expert affinity planted in the routers (rho = 0.9): the routing

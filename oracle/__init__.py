@@ -73,6 +73,8 @@ def _load():
         lib.orc_e4m3_scale_exponent.restype = _i64
         lib.orc_quantize_rows_e4m3.argtypes = [_i64, _i64, _p, _p, _p]
         lib.orc_quantize_rows_e4m3.restype = None
+        lib.orc_quantize_blocks_e4m3.argtypes = [_i64, _i64, _i64, _p, _p, _p]
+        lib.orc_quantize_blocks_e4m3.restype = None
         lib.orc_round_bf16.argtypes = [_i64, _p, _p]
         lib.orc_round_bf16.restype = None
         lib.orc_down_rows.argtypes = [_i64, _p, _i64, _i64, _p, _p, _p]
@@ -342,6 +344,26 @@ def dequantize_rows_bf16(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return (bits >> 16).astype(np.uint16)
 
 
+def quantize_blocks_e4m3(v, block: int = 32) -> tuple:
+    """Block-wise e4m3 quantisation of a float matrix [rows][cols] (fp32 or fp64 values, taken
+    exactly): the row rule on every `block` consecutive columns. Returns (codes uint8
+    [rows][cols], exps int32 [rows][cols / block]); value = code value * 2^exp."""
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    rows, cols = a.shape
+    assert cols % block == 0
+    codes = np.empty((rows, cols), np.uint8)
+    exps = np.empty((rows, cols // block), np.int32)
+    _load().orc_quantize_blocks_e4m3(rows, cols, block, _ptr(a), _ptr(codes), _ptr(exps))
+    return codes, exps
+
+
+def dequantize_blocks_e4m3(codes: np.ndarray, exps: np.ndarray, block: int = 32) -> np.ndarray:
+    """code value * 2^exp of every element, float64 (exact)."""
+    v = e4m3_decode(codes)
+    scale = np.ldexp(1.0, np.repeat(np.asarray(exps, dtype=np.int64), block, axis=-1))
+    return v * scale
+
+
 def round_bf16(v: np.ndarray) -> np.ndarray:
     """Nearest bf16 of each float64 value (ties to even), as uint16 bits."""
     v = np.ascontiguousarray(v, dtype=np.float64)
@@ -384,11 +406,14 @@ def fp8_down(h: np.ndarray, row_expert: np.ndarray, q: dict) -> dict:
 
 
 def layer_fp8(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order: int = 0,
-              reroute: bool = False) -> dict:
+              reroute: bool = False, fp8_return: bool = False) -> dict:
     """The layer with the FP8 payload and FP8 expert GEMMs: routing on the bf16 x; the
     gate/up projections on e4m3 rows of x (one scale per token) and e4m3 rows of W1, W3
     (one scale per output channel); h rounded to bf16, then its rows quantised to e4m3
-    for the down projection with e4m3 rows of W2; the combine as in ``layer``."""
+    for the down projection with e4m3 rows of W2; the combine as in ``layer``. With
+    ``fp8_return`` the expert outputs y travel back as e4m3 codes with one power-of-two
+    exponent per 32-column block (``quantize_blocks_e4m3``) and the combine weighs their
+    exact values."""
     q = fp8_operands(inp)
     r = route_and_dispatch(inp["x"], inp["w_router"], inp.get("bias"), K, W, cf, order, reroute)
     N = r["logits"].shape[0]
@@ -400,6 +425,11 @@ def layer_fp8(inp: dict, K: int, W: int, cf: float, want_h: bool = False, order:
     dn = fp8_down(h, row_expert, q)
     y = dn["y"]
     d = y.shape[1]
+    if fp8_return:
+        yq, ye = quantize_blocks_e4m3(y)
+        r["y_payload"] = (yq, ye)
+        r["y_exact"] = y
+        y = dequantize_blocks_e4m3(yq, ye)
     y_of_slot = np.zeros((N * K, d), np.float64)
     kept = r["row_of"] >= 0
     y_of_slot[kept] = y[r["row_of"][kept]]

@@ -528,6 +528,32 @@ EXPORT void orc_quantize_rows_e4m3(int64_t rows, int64_t cols, const uint16_t *s
     }
 }
 
+/* Block-wise quantisation of the return payload [MoE 推理服务工程真相 2026, §6.3]: the rule of
+ * orc_quantize_rows_e4m3 applied to every run of `block` consecutive columns of a row
+ * instead of the whole row (reading: a row of expert outputs is produced in column tiles, a
+ * block is not split across them). src [rows][cols] double; codes [rows][cols]; exps
+ * [rows][cols / block] the exponent j of each block (value = code value * 2^j). */
+EXPORT void orc_quantize_blocks_e4m3(int64_t rows, int64_t cols, int64_t block,
+                                     const double *src, uint8_t *codes, int32_t *exps)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < cols / block; ++b) {
+            const double *v = src + r * cols + b * block;
+            double amax = 0.0;
+            for (int64_t c = 0; c < block; ++c) {
+                double a = fabs(v[c]);
+                if (a > amax || isnan(a))
+                    amax = a;
+            }
+            int64_t j = orc_e4m3_scale_exponent(amax);
+            exps[r * (cols / block) + b] = (int32_t)j;
+            for (int64_t c = 0; c < block; ++c)
+                codes[r * cols + b * block + c] = e4m3_code(ldexp(v[c], (int)-j));
+        }
+    }
+}
+
 /* Nearest bf16 value (1 sign, 8 exponent bits, 7 mantissa bits: binary32's range with 8
  * significant bits) to a double, ties to even, as bf16 bits; beyond the largest finite value
  * (2 - 2^-7) * 2^127 rounds to infinity. */

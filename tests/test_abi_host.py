@@ -68,7 +68,7 @@ def test_shape_validation(m):
         assert m.moe_rows_alloc(s) == -1
         assert m.moe_workspace_size(s) == 0
     flags = m.make_shape(64, 128, 256, 8, 2, 4)
-    flags.flags = 8  # no such flag
+    flags.flags = 16  # no such flag
     assert m.moe_workspace_size(flags) == 0
     # an empty batch is a valid shape
     assert m.moe_workspace_size(m.make_shape(0, 128, 256, 8, 2, 4)) > 0
@@ -206,3 +206,20 @@ def test_graft_build_entry():
     the library's ABI version against the binding's."""
     import __graft_entry__
     __graft_entry__.build()
+
+
+def test_y_buffer_sizes(m):
+    """fp32 y: rows_alloc * d * 4 bytes; the FP8 return payload: rows_alloc rows of d codes
+    plus d/32 exponent bytes padded to 16 (d = 128: 4 -> 16; 2048: 64; 7168: 224)."""
+    for d, pad in ((128, 16), (384, 16), (2048, 64), (7168, 224)):
+        s = m.make_shape(64, d, 256, 8, 2, 4)
+        s8 = m.make_shape(64, d, 256, 8, 2, 4, fp8_return=True)
+        RA = m.moe_rows_alloc(s)
+        assert m.moe_y_bytes(s) == RA * d * 4
+        assert m.y_payload_stride(s8) == d + pad and (d + pad) % 16 == 0
+        assert m.moe_y_bytes(s8) == RA * (d + pad)
+    # the payload needs d % 128 == 0 (the down GEMM's tiles), also for the combine alone
+    assert m.moe_y_bytes(m.make_shape(64, 136, 256, 8, 2, 4, fp8_return=True)) == 0
+    P = 0x100000  # a fake, 16-byte aligned address: never dereferenced
+    s8 = m.make_shape(64, 136, 256, 8, 2, 4, fp8_return=True)
+    assert _raw(m).moe_combine(ctypes.byref(s8), P, P, P, None, None, P, None) == 2

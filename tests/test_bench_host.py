@@ -22,6 +22,8 @@ sys.path.insert(0, ROOT)
     ("e128_skew_reroute", 14),     # two dispatch passes and the ranking kernel
     ("stack4", 12),                # 512 blocks per expert, pair GEMMs
     ("stack4_affinity", 12),
+    ("mixtral_prefill_fp8_return", 12),
+    ("e128_skew_fp8_return", 10),
     ("residual_top1", 14),         # shared MLP: offsets, pair + single GEMMs twice
 ])
 def test_kernel_launch_count(name, count):

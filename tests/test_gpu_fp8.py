@@ -41,9 +41,10 @@ def deq(codes, scale, orc):
     return orc.e4m3_decode(codes) * np.asarray(scale, np.float64)[..., None]
 
 
-def run_fp8_stages(inp, w, dev="cuda"):
+def run_fp8_stages(inp, w, dev="cuda", fp8_return=False):
     m = lib()
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
+                         fp8_return=fp8_return)
     N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
     RA = m.moe_rows_alloc(shape)
     ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
@@ -70,7 +71,8 @@ def run_fp8_stages(inp, w, dev="cuda"):
     h = torch.zeros(RA, f, dtype=torch.bfloat16, device=dev)
     hq = torch.zeros(RA, f, dtype=torch.uint8, device=dev)
     hs = torch.zeros(RA, dtype=torch.float32, device=dev)
-    y = torch.zeros(RA, d, dtype=torch.float32, device=dev)
+    y = (torch.zeros(m.moe_y_bytes(shape), dtype=torch.uint8, device=dev) if fp8_return
+         else torch.zeros(RA, d, dtype=torch.float32, device=dev))
     m.moe_expert_up_fp8(shape, xs, ss, offsets, w1q, s1, w3q, s3, h)
     m.moe_quantize_rows_e4m3(h, hq, hs, rows_dev=offsets[E:])  # the kept rows of h
     m.moe_expert_down_fp8(shape, hq, hs, offsets, w2q, s2, y)
@@ -227,9 +229,10 @@ def test_fp8_down_gemm_on_oracle_rows(orc):
         assert_within_bound(y[:R], ref["y_rows"], 2.0 ** -16 * mag + 1e-30, w.name)
 
 
-def sampled_fp8_layer(orc, hx, K, toks, r, used):
+def sampled_fp8_layer(orc, hx, K, toks, r, used, fp8_return=False):
     """The oracle's FP8 layer on sampled tokens: the quantised operands of the used experts,
-    h and the e4m3 down projection for their kept rows, and the combine."""
+    h and the e4m3 down projection for their kept rows (then, with fp8_return, the block
+    quantisation of those rows of y), and the combine."""
     q = orc.fp8_operands(hx)
     remap = np.full(max(int(r["expert_of"].max()) + 1, 1), -1, np.int64)
     remap[used] = np.arange(len(used))
@@ -240,6 +243,8 @@ def sampled_fp8_layer(orc, hx, K, toks, r, used):
     h, _ = orc.expert_rows(row_token, row_expert, q["x_deq"], q["w1_deq"], q["w3_deq"], hx["w2"],
                            True)
     y = orc.fp8_down(h, row_expert, q)["y"]
+    if fp8_return:
+        y = orc.dequantize_blocks_e4m3(*orc.quantize_blocks_e4m3(y))
     out = np.zeros((len(toks), y.shape[1]))
     pos = {int(a): i for i, a in enumerate(kept)}
     for li, t in enumerate(toks):
@@ -250,17 +255,18 @@ def sampled_fp8_layer(orc, hx, K, toks, r, used):
     return out, q
 
 
-def test_fp8_layer_full_size_mixtral(orc):
+@pytest.mark.parametrize("fp8_return", [False, True], ids=["fp32_return", "fp8_return"])
+def test_fp8_layer_full_size_mixtral(orc, fp8_return):
     """The Mixtral-shaped layer (N=4096, d=4096, f=14336, E=8, K=2) through moe_layer_fp8:
     routing in full, the weight codes of the used experts bit for bit, the output on sampled
     tokens against the oracle's FP8 layer (relative Frobenius bar) and against the bf16 layer
-    (the FP8 bar)."""
+    (the FP8 bar); with and without the FP8 return payload."""
     from test_gpu_fullsize import host_inputs, sample_tokens
     m = lib()
     w = WORKLOADS["mixtral_prefill"]
     torch.cuda.empty_cache()
     inp = make_layer_inputs(w, seed=0, device="cuda")
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, fp8_return=fp8_return)
     w1q, s1 = quantize_weights(m, inp["w1"])
     w3q, s3 = quantize_weights(m, inp["w3"])
     w2q, s2 = quantize_weights(m, inp["w2"])
@@ -281,7 +287,7 @@ def test_fp8_layer_full_size_mixtral(orc):
     ut = torch.from_numpy(used).cuda()
     hx = host_inputs(inp, experts=ut)
     got = out[torch.from_numpy(toks).cuda()]
-    ref8, q = sampled_fp8_layer(orc, hx, w.K, toks, r, used)
+    ref8, q = sampled_fp8_layer(orc, hx, w.K, toks, r, used, fp8_return)
     for name, qg, sg in (("w1q", w1q, s1), ("w3q", w3q, s3), ("w2q", w2q, s2)):
         np.testing.assert_array_equal(_u8(qg[ut]), q[name])
         np.testing.assert_array_equal(sg[ut].cpu().numpy(), q["s" + name[1]])
@@ -294,4 +300,4 @@ def test_fp8_layer_full_size_mixtral(orc):
     smp16 = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr)
     dev = tolerance_report(got, smp16["out_tokens"])
     assert dev["rel_frob"] <= FP8_VS_BF16_REL_FROB, dev
-    print("mixtral fp8", rep, "vs bf16", dev)
+    print("mixtral fp8", "fp8 return" if fp8_return else "", rep, "vs bf16", dev)

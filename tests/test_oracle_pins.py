@@ -534,6 +534,49 @@ def test_quantize_rows(orc):
     assert rel.max() <= 2.0 ** -4
 
 
+def test_quantize_blocks_is_the_row_rule_per_block(orc):
+    """Block quantisation of the return payload = the (pinned) row quantisation applied to
+    each 32-column block as a row of its own, on bf16-representable values; and the same
+    rule checked directly against torch's float8 conversion on fp32 values."""
+    rng = np.random.default_rng(5)
+    a = torch.from_numpy(rng.standard_normal((24, 128)) *
+                         np.exp(rng.uniform(-30, 30, (24, 4))).repeat(32, axis=1))
+    a = a.to(torch.bfloat16)
+    a[2, 32:64] = 0.0
+    codes, exps = orc.quantize_blocks_e4m3(a.double().numpy())
+    rc, rs = orc.quantize_rows_e4m3(a.reshape(-1, 32))
+    np.testing.assert_array_equal(codes.reshape(-1, 32), rc)
+    np.testing.assert_array_equal(np.ldexp(1.0, exps.reshape(-1)), rs.astype(np.float64))
+    assert exps[2, 1] == 0 and np.all(codes[2, 32:64] == 0)
+    # fp32 values (not bf16): torch's conversion of each block scaled by 2^-j
+    v = (rng.standard_normal((16, 96)) * np.exp(rng.uniform(-10, 10, (16, 3))).repeat(32, axis=1)
+         ).astype(np.float32).astype(np.float64)
+    codes, exps = orc.quantize_blocks_e4m3(v)
+    for b in range(3):
+        blk = v[:, 32 * b:32 * b + 32]
+        for r in range(16):
+            j = orc.e4m3_scale_exponent(np.abs(blk[r]).max())
+            assert exps[r, b] == j
+            ref = torch.from_numpy(np.ldexp(blk[r], -j)).to(torch.float8_e4m3fn).view(torch.uint8)
+            np.testing.assert_array_equal(codes[r, 32 * b:32 * b + 32], ref.numpy())
+    back = orc.dequantize_blocks_e4m3(codes, exps)
+    floor = np.ldexp(2.0 ** -6, np.repeat(exps, 32, axis=1))   # below: e4m3 subnormals
+    assert (np.abs(back - v) / np.maximum(np.abs(v), floor)).max() <= 2.0 ** -4
+
+
+def test_quantize_blocks_hand_values(orc):
+    """One row, two blocks: block 0 has largest magnitude 448 (j = 0: the codes are the values'
+    own e4m3 codes), block 1 has 449 (j = 1: every value halved first)."""
+    row = np.zeros((1, 64))
+    row[0, 0], row[0, 1], row[0, 2] = 448.0, -1.0, 0.3
+    row[0, 32], row[0, 33] = 449.0, 3.0
+    codes, exps = orc.quantize_blocks_e4m3(row)
+    assert exps.tolist() == [[0, 1]]
+    assert codes[0, 0] == 0x7E and codes[0, 1] == 0xB8   # 448; -1.0 = sign, exponent 7
+    assert orc.e4m3_decode(codes[0, 2:3])[0] == 0.3125    # 0.3 -> nearest e4m3 (0.3125)
+    assert orc.e4m3_decode(codes[0, 32:34]).tolist() == [224.0, 1.5]  # 224.5 -> 224; 1.5
+
+
 def test_layer_fp8_reduces_to_bf16_layer_on_e4m3_inputs(orc):
     """With x, W1, W3, W2 already e4m3 values whose rows reach the top binade, quantising
     them is the identity: the FP8 layer's h equals the bf16 layer's h exactly, and its
