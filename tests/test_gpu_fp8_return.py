@@ -78,11 +78,14 @@ def test_payload_is_the_block_code_of_y(orc, case, fp8_gemm):
     assert np.all(pad == 0xAB) and np.all(tail == 0xAB), "bytes outside the kept rows written"
 
 
-def test_combine_weighs_the_payload_exactly(orc):
-    """moe_combine on a payload: out = sum_k w_k * (code * 2^j), fp32 accumulation in k order;
-    the oracle's combine of the decoded payload (fp64) bounds the difference per element."""
+@pytest.mark.parametrize("N", [96, 2048])
+def test_combine_weighs_the_payload_exactly(orc, N):
+    """moe_combine on a payload: out = sum_k w_k * (code * 2^j), fp32 accumulation in k order,
+    then the shared MLP's output and the residual when given; the oracle's combine of the
+    decoded payload (fp64) bounds the difference per element. N = 96 takes the sliced-row
+    path (few tokens per SM), N = 2048 the whole-row path."""
     m = lib()
-    N, K, d, E = 96, 3, 256, 4
+    K, d, E = 3, 256, 4
     shape = m.make_shape(N, d, 128, E, K, 1, 0.0, fp8_return=True)
     RA = m.moe_rows_alloc(shape)
     rng = np.random.default_rng(9)
@@ -99,15 +102,25 @@ def test_combine_weighs_the_payload_exactly(orc):
     y_of_slot = np.where(row_of[:, None] >= 0, deq_all[np.maximum(row_of, 0)], 0.0)
     ref = orc.combine(row_of, topk_w, y_of_slot)
     mag = orc.combine(row_of, np.abs(topk_w), np.abs(y_of_slot))
+    # the extras a Residual-MoE layer and a stack add after the routed sum
+    shared_y = (rng.standard_normal((N, d)) * 3).astype(np.float32)
+    residual = torch.from_numpy(rng.standard_normal((N, d))).to(torch.bfloat16)
+    res64 = residual.double().numpy()
     for out_bf16 in (False, True):
-        sh = m.make_shape(N, d, 128, E, K, 1, 0.0, out_bf16=out_bf16, fp8_return=True)
-        out = torch.empty(N, d, dtype=torch.bfloat16 if out_bf16 else torch.float32,
-                          device="cuda")
-        m.moe_combine(sh, torch.from_numpy(buf.reshape(-1)).cuda(),
-                      torch.from_numpy(row_of).cuda(), torch.from_numpy(topk_w).cuda(), out)
-        torch.cuda.synchronize()
-        bound = (K + 2) * 2.0 ** -24 * mag + (2.0 ** -8 * np.abs(ref) if out_bf16 else 0) + 1e-37
-        assert_within_bound(out.float(), ref, bound, f"out_bf16={out_bf16}")
+        for extras in (False, True):
+            sh = m.make_shape(N, d, 128, E, K, 1, 0.0, out_bf16=out_bf16, fp8_return=True)
+            out = torch.empty(N, d, dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                              device="cuda")
+            m.moe_combine(sh, torch.from_numpy(buf.reshape(-1)).cuda(),
+                          torch.from_numpy(row_of).cuda(), torch.from_numpy(topk_w).cuda(), out,
+                          residual=residual.cuda() if extras else None,
+                          shared_y=torch.from_numpy(shared_y).cuda() if extras else None)
+            torch.cuda.synchronize()
+            want = ref + (shared_y.astype(np.float64) + res64 if extras else 0.0)
+            size = mag + (np.abs(shared_y) + np.abs(res64) if extras else 0.0)
+            bound = ((K + 4) * 2.0 ** -24 * size + (2.0 ** -8 * np.abs(want) if out_bf16 else 0)
+                     + 1e-37)
+            assert_within_bound(out.float(), want, bound, f"out_bf16={out_bf16} extras={extras}")
 
 
 CASES = [
