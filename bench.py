@@ -316,8 +316,8 @@ def algorithmic_work(w, R: int, E_act: int) -> dict:
         scatter_bytes=(N * d * 2 + 2 * R * (d + 4) + N * K * 4 * 3 if w.fp8
                        else N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3),
         # combine: read every kept expert row (fp32, or the FP8 return payload: e4m3 codes and
-        # one exponent byte per 32 columns), the routing, write fp32 out
-        combine_bytes=(R * (d + d // 32) if w.fp8_return else R * d * 4) + N * K * 8 + N * d * 4,
+        # one exponent byte per 32 columns), the routing, write the bf16 out
+        combine_bytes=(R * (d + d // 32) if w.fp8_return else R * d * 4) + N * K * 8 + N * d * 2,
     )
 
 
@@ -341,7 +341,8 @@ def run_gpu(args, w) -> dict:
     layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
               for l in range(L)]
     inp = layers[0]
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=L > 1,
+    # the layer's output is bf16, as the hidden states it replaces (a stack's next input)
+    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=True,
                          slot_major=w.slot_major, reroute=w.reroute, fp8_return=w.fp8_return)
     RA = m.moe_rows_alloc(shape)
     ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
@@ -382,7 +383,7 @@ def run_gpu(args, w) -> dict:
         affinity = torch.zeros(L - 1, E, E, dtype=torch.int64, device=dev)
         out = xbuf[(L - 1) % 2]
     else:
-        out = torch.empty(N, d, dtype=torch.float32, device=dev)
+        out = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
     if shared:  # Residual-MoE: the shared dense MLP on every token
         sh = make_shared_inputs(w, seed=args.seed + rank, device=str(dev))
         h_s = torch.empty(N, w.shared_f, dtype=torch.bfloat16, device=dev)
@@ -548,7 +549,7 @@ def run_gpu(args, w) -> dict:
                      else m.moe_layer_workspace_size(shape))
         lws = torch.empty(lws_bytes, dtype=torch.uint8, device=dev)
         x_host = x.cpu().pin_memory()
-        out_dt = torch.bfloat16 if L > 1 else torch.float32
+        out_dt = torch.bfloat16
         out_host = [torch.empty(N, d, dtype=out_dt).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]
         out_dev = [torch.empty(N, d, dtype=out_dt, device=dev) for _ in range(2)]
@@ -615,7 +616,7 @@ def run_gpu(args, w) -> dict:
         barrier()
         e2e_agg = aggregate(float(N * args.steps), e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": e2e_agg["value"], "unit": UNIT, "h2d_bytes_per_step": N * d * 2,
-               "d2h_bytes_per_step": N * d * (2 if L > 1 else 4),
+               "d2h_bytes_per_step": N * d * 2,
                "note": "pinned host input and output; copies overlap the previous step's layer"}
         del lws
 
@@ -684,6 +685,7 @@ def run_gpu(args, w) -> dict:
                    "shared_f": w.shared_f,
                    "capacity_factor": w.cf if w.cf > 0 else "dropless", "zipf_s": w.s,
                    "rows_kept": R_layers if L > 1 else R, "layers": L,
+                   "output": "bf16 [N][d], the fp32 sum rounded once",
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step"},
