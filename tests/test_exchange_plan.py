@@ -199,3 +199,37 @@ def test_placement_errors(m):
         m.moe_place_experts(c, 2, 8, 2, starts=0)
     with pytest.raises(m.MoeError):
         m.moe_place_experts(np.ones((1, 300, 300), np.int64), 2, 300, 2)
+
+
+def test_placement_deployed_by_relabelling_experts(m):
+    """Deploying a placement = storing each layer's experts GPU by GPU (router rows permuted
+    with them). The routing is the same up to the relabelling, and the relabelled stack's
+    affinity counts under the contiguous placement cost exactly what moe_place_experts
+    reported: the placement's cost is the crossing count the deployed layers will show."""
+    import torch
+
+    import oracle
+    from moe_workloads import WORKLOADS, affine_router
+    w = WORKLOADS["stack4_affinity"].with_(N=256, d=64, f=128, E=16, K=2, W=4, layers=3)
+    L, E, K, P = w.layers, w.E, w.K, w.W
+    g = torch.Generator().manual_seed(4)
+    x0 = torch.randn(w.N, w.d, generator=g)
+    xs = [(x0 + 0.3 * torch.randn(w.N, w.d, generator=g)).to(torch.bfloat16) for _ in range(L)]
+    routers = [affine_router(w, 0, l) for l in range(L)]
+    topk = [oracle.topk(oracle.router_logits(xs[l], routers[l]), K)[0] for l in range(L)]
+    counts = np.stack([oracle.affinity(topk[j], topk[j + 1], E) for j in range(L - 1)])
+    gpu_of, cost, base = m.moe_place_experts(counts, L, E, P)
+    assert cost < base
+    topk2, new_ids = [], []
+    for l in range(L):
+        order = np.lexsort((np.arange(E), gpu_of[l]))      # GPU by GPU, experts ascending
+        new_id = np.empty(E, np.int64)
+        new_id[order] = np.arange(E)
+        new_ids.append(new_id)
+        t2 = oracle.topk(oracle.router_logits(xs[l], routers[l][torch.from_numpy(order)]), K)[0]
+        np.testing.assert_array_equal(t2, new_id[topk[l]])  # same choices, new names
+        topk2.append(t2)
+    counts2 = np.stack([oracle.affinity(topk2[j], topk2[j + 1], E) for j in range(L - 1)])
+    for j in range(L - 1):
+        np.testing.assert_array_equal(counts2[j][np.ix_(new_ids[j], new_ids[j + 1])], counts[j])
+    assert xp.placement_cost(counts2, xp.contiguous_placement(L, E, P)) == cost

@@ -28,6 +28,8 @@ CASES = [
     Workload("odd_e", N=100, d=128, f=128, E=5, K=2, W=5, cf=0.9),
     Workload("one_token_per_rank", N=8, d=128, f=128, E=16, K=3, W=8, cf=0.5),
     Workload("wide_k", N=96, d=128, f=128, E=48, K=32, W=4),
+    # every limit at once, token-major: 256 experts, K = 32, 64 ranks, capacity drops
+    Workload("max_limits", N=128, d=128, f=128, E=256, K=32, W=64, cf=1.0),
     # >= 768 rows per expert on average: the CTA-pair GEMM kernel (256-row tiles)
     Workload("pair_tiles", N=1600, d=256, f=256, E=2, K=1, W=2),
     # skewed rows (Zipf bias): large experts on the pair kernel, small ones on the
