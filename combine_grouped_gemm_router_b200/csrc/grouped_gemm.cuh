@@ -260,7 +260,20 @@ __device__ __forceinline__ bool expert_selected(int select, int rows)
     return select == 0 || (select == 1) == prefer_pair_tiles(rows);
 }
 
-// Tile index -> (expert, N-slab, M-tile). tile_start[e] = first tile of expert e.
+// The order in which experts take their tiles: alternately from the two ends of the expert
+// range (0, E-1, 1, E-2, ...). With skewed routing the heavy experts crowd one end (a Zipf
+// bias makes the low indices hot), and their tiles after the first of each N slab find the
+// weight tile in L2 and run at tensor-core speed, while a light expert's tiles stream weights
+// from DRAM; alternating the ends keeps both kinds in every wave of tiles, so DRAM stays busy
+// throughout instead of idling through the heavy experts and then saturating. Uniform
+// routing is unaffected. Position i of the order -> expert.
+__device__ __forceinline__ int visit_expert(int i, int E)
+{
+    return (i & 1) ? E - 1 - (i >> 1) : (i >> 1);
+}
+
+// Tile index -> (expert, N-slab, M-tile). tile_start[i] = first tile of the expert at
+// position i of the visit order, mtiles[i] its M-tile count.
 __device__ __forceinline__ void decode_tile(int tile, const int *tile_start, const int *mtiles,
                                             int E, int n_tiles, int &e, int &n, int &m)
 {
@@ -272,9 +285,9 @@ __device__ __forceinline__ void decode_tile(int tile, const int *tile_start, con
         else
             hi = mid - 1;
     }
-    e = lo;
-    const int local = tile - tile_start[e];
-    const int mt = mtiles[e];
+    e = visit_expert(lo, E);
+    const int local = tile - tile_start[lo];
+    const int mt = mtiles[lo];
     n = local / mt;
     m = local - n * mt;
 }
@@ -578,17 +591,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         // per-expert M-tile counts and their prefix (in tiles, times n_tiles)
         int carry = 0;
         for (int base = 0; base < E; base += 32) {
-            const int e = base + lane;
+            const int i = base + lane;  // position in the visit order
             int mt = 0;
-            if (e < E) {
+            if (i < E) {
+                const int e = visit_expert(i, E);
                 int rows = args.offsets[e + 1] - args.offsets[e];
                 rows = max(0, min(rows, args.rows_alloc));
                 mt = expert_selected(args.select, rows) ? (rows + BM - 1) / BM : 0;
-                mtiles[e] = mt;
+                mtiles[i] = mt;
             }
             const int incl = warp_incl_scan(mt);
-            if (e < E)
-                tile_start[e] = (carry + incl - mt) * args.n_tiles;
+            if (i < E)
+                tile_start[i] = (carry + incl - mt) * args.n_tiles;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0)
@@ -888,17 +902,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         int carry = 0;
         for (int base = 0; base < E; base += 32) {
-            const int e = base + lane;
+            const int i = base + lane;  // position in the visit order
             int mt = 0;
-            if (e < E) {
+            if (i < E) {
+                const int e = visit_expert(i, E);
                 int rows = args.offsets[e + 1] - args.offsets[e];
                 rows = max(0, min(rows, args.rows_alloc));
                 mt = expert_selected(args.select, rows) ? (rows + BMP - 1) / BMP : 0;
-                mtiles[e] = mt;
+                mtiles[i] = mt;
             }
             const int incl = warp_incl_scan(mt);
-            if (e < E)
-                tile_start[e] = (carry + incl - mt) * args.n_tiles;
+            if (i < E)
+                tile_start[i] = (carry + incl - mt) * args.n_tiles;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
         if (lane == 0)
