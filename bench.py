@@ -212,18 +212,18 @@ class ClockSampler:
 # DRAM bytes per launch of the gate/up grouped GEMM at full size, from ncu captures of the
 # half-size cases (scaled x2: weights, rows and h all double), summarised in profiles/.
 # A figure holds only for the kernel source it was measured on (sha256 of grouped_gemm.cuh).
-_UP_SHA = "1bf2bf1450364aa5aaa06a231a28be39b41791ca98e3d8cc11f6aa8e6a9e9bb1"
+_UP_SHA = "f434a3866c6d2c34f80a08e718b0f424a9f9ca1cf11ed545f0cebe319035a775"
 MEASURED_UP_TRAFFIC = {
     # workload: (kernel source sha256, bytes per launch)
-    "mixtral_prefill": (_UP_SHA, 2 * (1003.3e6 + 113.4e6)),     # half-size capture x 2
-    "mixtral_prefill_fp8": (_UP_SHA, 2 * (487.8e6 + 105.5e6)),  # half-size capture x 2
-    "e128_skew": (_UP_SHA, 886.7e6 + 35.7e6),
-    "e128_skew_fp8": (_UP_SHA, 444.1e6 + 35.2e6),
+    "mixtral_prefill": (_UP_SHA, 2 * (994.2e6 + 112.2e6)),      # half-size capture x 2
+    "mixtral_prefill_fp8": (_UP_SHA, 2 * (487.8e6 + 104.4e6)),  # half-size capture x 2
+    "e128_skew": (_UP_SHA, 894.0e6 + 34.4e6),
+    "e128_skew_fp8": (_UP_SHA, 444.1e6 + 32.5e6),
     # the return payload changes the down GEMM and the combine, not the gate/up GEMM
-    "mixtral_prefill_fp8_return": (_UP_SHA, 2 * (487.8e6 + 105.5e6)),
-    "e128_skew_fp8_return": (_UP_SHA, 444.1e6 + 35.2e6),
-    "decode": (_UP_SHA, 6072.1e6 + 3.8e6),
-    "decode_fp8": (_UP_SHA, 3037.4e6 + 4.2e6),
+    "mixtral_prefill_fp8_return": (_UP_SHA, 2 * (487.8e6 + 104.4e6)),
+    "e128_skew_fp8_return": (_UP_SHA, 444.1e6 + 32.5e6),
+    "decode": (_UP_SHA, 6081.7e6 + 3.9e6),
+    "decode_fp8": (_UP_SHA, 3042.0e6 + 3.6e6),
 }
 
 
