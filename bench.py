@@ -211,8 +211,9 @@ class ClockSampler:
 
 # DRAM bytes per launch of the gate/up grouped GEMM at full size, from ncu captures of the
 # half-size cases (scaled x2: weights, rows and h all double), summarised in profiles/.
-# A figure holds only for the kernel source it was measured on (sha256 of grouped_gemm.cuh).
-_UP_SHA = "f434a3866c6d2c34f80a08e718b0f424a9f9ca1cf11ed545f0cebe319035a775"
+# A figure holds only for the kernel code it was measured on (kernel_source_hash of
+# grouped_gemm.cuh: comments and whitespace do not count).
+_UP_SHA = "677f9b61402ef3adcb881fae89c4b2c3e66732c2611b4496b9bb8e93c6b1a331"
 MEASURED_UP_TRAFFIC = {
     # workload: (kernel source sha256, bytes per launch)
     "mixtral_prefill": (_UP_SHA, 2 * (994.2e6 + 112.2e6)),      # half-size capture x 2
@@ -227,14 +228,25 @@ MEASURED_UP_TRAFFIC = {
 }
 
 
+def kernel_source_hash(path: str) -> str:
+    """sha256 of a source file with its comments and whitespace removed: the code the
+    traffic figures were measured on, unaffected by edits to comments."""
+    import re
+    with open(path, "r", encoding="utf-8") as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = " ".join(text.split())
+    return hashlib.sha256(text.encode()).hexdigest()
+
+
 def up_traffic(workload: str):
     sha_ref, nbytes = MEASURED_UP_TRAFFIC.get(workload, (None, None))
     if sha_ref is None:
         return None
     path = os.path.join(ROOT, "combine_grouped_gemm_router_b200", "csrc", "grouped_gemm.cuh")
     try:
-        with open(path, "rb") as fh:
-            sha = hashlib.sha256(fh.read()).hexdigest()
+        sha = kernel_source_hash(path)
     except OSError:
         return None
     return nbytes if sha == sha_ref else None

@@ -15,14 +15,17 @@
 //    the epilogue of one tile overlaps the MMAs of the next;
 //  - the tile list is derived on device from the expert offsets: experts with
 //    no rows have no tiles, so their weights are never read;
-//  - tiles are ordered expert-major, then N-slab, then M (fastest): CTAs that
-//    run at the same time share one weight slab and one expert's rows in L2;
+//  - tiles are ordered expert by expert (visiting the experts alternately from
+//    both ends of the range, see visit_expert), then N-slab, then M (fastest):
+//    CTAs that run at the same time share one weight slab and one expert's rows
+//    in L2;
 //  - rows of a tile past the expert's end are computed (they are the next
 //    expert's rows or zero fill) but never stored.
 // Mode 0 (gate/up): the B tile stacks 128 rows of W1 and 128 rows of W3, one
 // N=256 MMA per K-step; the epilogue reads gate column c and up column 128+c
 // and writes h = silu(g) * u as bf16 (the next GEMM's operand). Mode 1 (down):
-// fp32 output straight from TMEM, so the combine sums unrounded expert outputs.
+// fp32 output straight from TMEM, so the combine sums unrounded expert outputs
+// (or the FP8 return payload: e4m3 codes with one exponent per 32 columns).
 // Modes 2 and 3 (the FP8 path, [MoE 推理服务工程真相 2026, §6.3]): modes 0 and 1
 // with e4m3 A and B (tcgen05 kind::f8f6f4). A 128-byte swizzle atom then holds
 // 128 K elements instead of 64, so tiles, stages and descriptors keep their byte

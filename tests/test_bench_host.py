@@ -88,3 +88,17 @@ def test_affine_router_leans_on_the_previous_layer():
     assert torch.equal(plain["w2"], planted["w2"])
     assert torch.equal(planted["w_router"], r1)
     assert not math.isclose(float((plain["w_router"] - r1).abs().max()), 0.0)
+
+
+def test_traffic_gate_ignores_comments_only(tmp_path):
+    """The bench reports measured DRAM traffic only for the kernel code it was measured on:
+    an edit to comments or whitespace keeps the figure, an edit to code drops it."""
+    import bench
+    src = tmp_path / "k.cuh"
+    src.write_text("// header\nint f(int a) { return a + 1; }  /* note */\n")
+    h0 = bench.kernel_source_hash(str(src))
+    src.write_text("// header, reworded\n\nint f(int a)   { return a + 1; }\n")
+    assert bench.kernel_source_hash(str(src)) == h0
+    src.write_text("// header\nint f(int a) { return a + 2; }\n")
+    assert bench.kernel_source_hash(str(src)) != h0
+    assert bench.up_traffic("mixtral_prefill") is not None   # the captured code is current
