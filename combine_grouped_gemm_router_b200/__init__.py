@@ -81,6 +81,7 @@ _sigs = {
                           c_i32),
     "moe_exchange_schedule": ([c_i32, c_p, c_i32, c_p, c_p, c_p, c_p], c_i32),
     "moe_place_experts": ([c_i32, c_i32, c_i32, c_p, c_i32, c_p, c_p, c_p], c_i32),
+    "moe_place_experts_staged": ([c_i32] * 4 + [c_p, c_i32] + [c_p] * 5, c_i32),
     "moe_get_device_error": ([ctypes.c_int], c_i32),
     "moe_read_stats": ([c_p, ctypes.POINTER(MoeStats), c_p], c_i32),
     "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
@@ -402,6 +403,26 @@ def moe_place_experts(counts, L: int, E: int, P: int, starts: int = 16):
                                   g.ctypes.data_as(c_p), ctypes.byref(cost), ctypes.byref(base)),
            "moe_place_experts")
     return g, int(cost.value), int(base.value)
+
+
+def moe_place_experts_staged(counts, L: int, E: int, nodes: int, gpus_per_node: int,
+                             starts: int = 16):
+    """Two-stage placement (nodes, then GPUs inside each node) from affinity counts
+    int64 [L-1, E, E]. Returns (gpu_of int32 [L, E], dict of node/GPU hop counts, placed and
+    contiguous)."""
+    import numpy as np
+    c = np.ascontiguousarray(counts, dtype=np.int64).reshape(-1)
+    if c.size != max(L - 1, 0) * E * E:
+        raise MoeError(1, "moe_place_experts_staged: counts must hold (L-1)*E*E entries")
+    g = np.empty((L, E), np.int32)
+    out = [ctypes.c_int64(0) for _ in range(4)]
+    _check(_lib.moe_place_experts_staged(int(L), int(E), int(nodes), int(gpus_per_node),
+                                         c.ctypes.data_as(c_p) if c.size else None, int(starts),
+                                         g.ctypes.data_as(c_p),
+                                         *[ctypes.byref(v) for v in out]),
+           "moe_place_experts_staged")
+    keys = ("node_hops", "gpu_hops", "contiguous_node_hops", "contiguous_gpu_hops")
+    return g, {k: int(v.value) for k, v in zip(keys, out)}
 
 
 def moe_get_device_error(clear: bool = True) -> int:

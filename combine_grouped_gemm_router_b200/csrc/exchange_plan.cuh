@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cmath>
 #include <vector>
 
 namespace moe_plan {
@@ -296,27 +297,104 @@ inline uint64_t splitmix64(uint64_t *state)
     return z ^ (z >> 31);
 }
 
+// Layer 0's experts in P groups of E/P whose hops go to similar experts of layer 1 (cosine
+// similarity of their rows of the affinity counts): P seeds taken farthest-first, then every
+// other expert, most decided first, joins the group with room whose members it resembles
+// most on average. Experts that feed the same experts next belong on the same GPU, and no
+// single-layer move of the local search can gather them once they are spread.
+inline void similarity_groups(int E, int P, const int64_t *c0, int32_t *group)
+{
+    const int share = E / P;
+    std::vector<double> norm(E, 0.0), sim((size_t)E * E, 0.0);
+    for (int i = 0; i < E; ++i) {
+        double q = 0.0;
+        for (int p = 0; p < E; ++p)
+            q += (double)c0[(size_t)i * E + p] * (double)c0[(size_t)i * E + p];
+        norm[i] = q > 0.0 ? std::sqrt(q) : 1.0;
+    }
+    for (int i = 0; i < E; ++i)
+        for (int k = i; k < E; ++k) {
+            double dot = 0.0;
+            for (int p = 0; p < E; ++p)
+                dot += (double)c0[(size_t)i * E + p] * (double)c0[(size_t)k * E + p];
+            sim[(size_t)i * E + k] = sim[(size_t)k * E + i] = dot / (norm[i] * norm[k]);
+        }
+    std::vector<int> size(P, 0);
+    std::vector<double> gsum((size_t)E * P, 0.0);  // expert x group: summed similarity
+    for (int e = 0; e < E; ++e)
+        group[e] = -1;
+    auto join = [&](int e, int q) {
+        group[e] = q;
+        ++size[q];
+        for (int k = 0; k < E; ++k)
+            gsum[(size_t)k * P + q] += sim[(size_t)k * E + e];
+    };
+    // seeds: the expert with the most hops, then each time the one least like any seed
+    int first = 0;
+    for (int e = 1; e < E; ++e)
+        if (norm[e] > norm[first])
+            first = e;
+    join(first, 0);
+    for (int q = 1; q < P; ++q) {
+        int pick = -1;
+        double best = 0.0;
+        for (int e = 0; e < E; ++e) {
+            if (group[e] >= 0)
+                continue;
+            double closest = -1.0;
+            for (int r = 0; r < q; ++r)
+                closest = std::max(closest, gsum[(size_t)e * P + r]);
+            if (pick < 0 || closest < best) {
+                pick = e;
+                best = closest;
+            }
+        }
+        join(pick, q);
+    }
+    for (int left = E - P; left > 0; --left) {
+        int pe = -1, pq = -1;
+        double pv = 0.0;
+        for (int e = 0; e < E; ++e) {
+            if (group[e] >= 0)
+                continue;
+            for (int q = 0; q < P; ++q) {
+                if (size[q] >= share)
+                    continue;
+                const double v = gsum[(size_t)e * P + q] / size[q];
+                if (pe < 0 || v > pv) {
+                    pe = e;
+                    pq = q;
+                    pv = v;
+                }
+            }
+        }
+        join(pe, pq);
+    }
+}
+
 // Start 0: every layer contiguous (expert e on GPU e / (E/P)), so the result is never worse
-// than that placement. Start 1: layer 0 contiguous. Start s >= 2: layer 0 a shuffle of the
-// contiguous assignment (Fisher-Yates driven by splitmix64 seeded with s); for odd s every
+// than that placement. Start 1: layer 0 contiguous. Start 2: layer 0 grouped by
+// similarity_groups (set by the caller). Start s >= 3, with k = s - 1: layer 0 a shuffle of the
+// contiguous assignment (Fisher-Yates driven by splitmix64 seeded with k); for odd k every
 // other layer is shuffled the same way. Returns true when the later layers are still to be
 // built from layer 0 (each placed best given the one before it).
 inline bool initial_placement(int L, int E, int P, int start, std::vector<int32_t> *g)
 {
     const int share = E / P;
     g->assign((size_t)L * E, 0);
-    uint64_t state = (uint64_t)start;
+    const int k = start - 1;  // the shuffle's seed and kind for start >= 3
+    uint64_t state = (uint64_t)k;
     for (int l = 0; l < L; ++l) {
         int32_t *row = g->data() + (size_t)l * E;
         for (int e = 0; e < E; ++e)
             row[e] = e / share;
-        if (start >= 2 && (l == 0 || start % 2 == 1))
+        if (start >= 3 && (l == 0 || k % 2 == 1))
             for (int e = E - 1; e > 0; --e) {
-                const int k = (int)(splitmix64(&state) % (uint64_t)(e + 1));
-                std::swap(row[e], row[k]);
+                const int r = (int)(splitmix64(&state) % (uint64_t)(e + 1));
+                std::swap(row[e], row[r]);
             }
     }
-    return start == 1 || (start >= 2 && start % 2 == 0);
+    return start == 1 || start == 2 || (start >= 3 && k % 2 == 0);
 }
 
 // Block coordinate descent: each layer re-placed best given its neighbours, forward then
@@ -344,12 +422,14 @@ inline void place_experts(int L, int E, int P, const int64_t *counts, int starts
         const bool build = initial_placement(L, E, P, s, &g);
         if (s == 0 && contiguous_out)
             *contiguous_out = pl.cost(g);
+        if (s == 2 && L > 1 && P > 1)
+            similarity_groups(E, P, counts, g.data());
         if (build)
             for (int l = 1; l < L; ++l)
                 pl.improve_layer(l, &g, false);
         descend(pl, &g);
         int64_t c = pl.cost(g);
-        // Kicks: swap two pairs of experts (on different GPUs) in one layer, descend again,
+        // Kicks: swap the GPUs of two random pairs of experts in one layer, descend again,
         // keep the result if it is cheaper.
         uint64_t state = 0x5eedull + (uint64_t)s;
         for (int kick = 0; kick < 4 * L && L > 1 && P > 1; ++kick) {
@@ -375,6 +455,52 @@ inline void place_experts(int L, int E, int P, const int64_t *counts, int starts
     std::copy(best.begin(), best.end(), gpu_of);
     if (cost_out)
         *cost_out = best_cost;
+}
+
+// Hops between consecutive layers whose experts' groups differ, a group being g / per
+// (per = 1: GPUs; per = GPUs per node: nodes).
+inline int64_t crossing_hops(int L, int E, const int64_t *counts, const int32_t *g, int per)
+{
+    int64_t c = 0;
+    for (int j = 0; j + 1 < L; ++j)
+        for (int i = 0; i < E; ++i)
+            for (int p = 0; p < E; ++p)
+                if (g[(size_t)j * E + i] / per != g[(size_t)(j + 1) * E + p] / per)
+                    c += counts[((size_t)j * E + i) * E + p];
+    return c;
+}
+
+// Two stages, as ExFlow's staged expert affinity: first the experts of every layer are placed
+// on nodes (E / nodes each), minimising the hops that cross nodes; then, node by node, that
+// node's experts are placed on its GPUs, minimising the hops inside the node that cross GPUs
+// (the affinity counts restricted to the node's experts of consecutive layers).
+inline void place_experts_staged(int L, int E, int nodes, int gpn, const int64_t *counts,
+                                 int starts, int32_t *gpu_of)
+{
+    std::vector<int32_t> node_of((size_t)L * E);
+    place_experts(L, E, nodes, counts, starts, node_of.data(), nullptr, nullptr);
+    const int Ep = E / nodes;
+    std::vector<int32_t> members((size_t)L * Ep), local((size_t)L * Ep);
+    std::vector<int64_t> sub((size_t)(L > 1 ? L - 1 : 0) * Ep * Ep);
+    for (int n = 0; n < nodes; ++n) {
+        for (int l = 0; l < L; ++l) {
+            int k = 0;
+            for (int e = 0; e < E; ++e)
+                if (node_of[(size_t)l * E + e] == n)
+                    members[(size_t)l * Ep + k++] = e;
+        }
+        for (int j = 0; j + 1 < L; ++j)
+            for (int a = 0; a < Ep; ++a)
+                for (int b = 0; b < Ep; ++b)
+                    sub[((size_t)j * Ep + a) * Ep + b] =
+                        counts[((size_t)j * E + members[(size_t)j * Ep + a]) * E +
+                               members[(size_t)(j + 1) * Ep + b]];
+        place_experts(L, Ep, gpn, sub.data(), starts, local.data(), nullptr, nullptr);
+        for (int l = 0; l < L; ++l)
+            for (int a = 0; a < Ep; ++a)
+                gpu_of[(size_t)l * E + members[(size_t)l * Ep + a]] =
+                    n * gpn + local[(size_t)l * Ep + a];
+    }
 }
 
 }  // namespace moe_plan

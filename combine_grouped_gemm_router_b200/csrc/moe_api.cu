@@ -1512,6 +1512,37 @@ moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts, int32_
     return MOE_OK;
 }
 
+__attribute__((visibility("default"))) moe_status_t
+moe_place_experts_staged(int32_t L, int32_t E, int32_t nodes, int32_t gpus_per_node,
+                         const int64_t *counts, int32_t starts, int32_t *gpu_of,
+                         int64_t *node_hops, int64_t *gpu_hops, int64_t *contiguous_node_hops,
+                         int64_t *contiguous_gpu_hops)
+{
+    if (!gpu_of || (L > 1 && !counts) || L < 1 || E < 1 || E > kMaxE || nodes < 1 ||
+        gpus_per_node < 1 || E % (nodes * gpus_per_node) != 0 || starts < 1 || starts > 64)
+        return MOE_ERR_INVALID_ARG;
+    if (L > 1)
+        for (size_t i = 0; i < (size_t)(L - 1) * E * E; ++i)
+            if (counts[i] < 0)
+                return MOE_ERR_INVALID_ARG;
+    moe_plan::place_experts_staged(L, E, nodes, gpus_per_node, counts, starts, gpu_of);
+    std::vector<int32_t> contiguous((size_t)L * E);
+    const int share = E / (nodes * gpus_per_node);
+    for (int l = 0; l < L; ++l)
+        for (int e = 0; e < E; ++e)
+            contiguous[(size_t)l * E + e] = e / share;
+    if (node_hops)
+        *node_hops = moe_plan::crossing_hops(L, E, counts, gpu_of, gpus_per_node);
+    if (gpu_hops)
+        *gpu_hops = moe_plan::crossing_hops(L, E, counts, gpu_of, 1);
+    if (contiguous_node_hops)
+        *contiguous_node_hops =
+            moe_plan::crossing_hops(L, E, counts, contiguous.data(), gpus_per_node);
+    if (contiguous_gpu_hops)
+        *contiguous_gpu_hops = moe_plan::crossing_hops(L, E, counts, contiguous.data(), 1);
+    return MOE_OK;
+}
+
 __attribute__((visibility("default"))) moe_status_t moe_get_device_error(int clear)
 {
     if (cudaDeviceSynchronize() != cudaSuccess)

@@ -446,8 +446,9 @@ moe_status_t moe_exchange_schedule(int32_t W, const int64_t *rank_matrix, int32_
  *   for the returned placement; contiguous_cost (nullable): the same for the contiguous
  *   placement (expert e on GPU e / (E/P)), the default of moe_dispatch's rank emulation.
  * Method: a heuristic, not the pages' exact ILP. From `starts` initial placements (all layers
- *   contiguous; layer 0 contiguous or shuffled with the later layers built one by one, each
- *   best given the one before; all layers shuffled), each layer in turn is re-placed optimally
+ *   contiguous; layer 0 contiguous, grouped by the similarity of its experts' affinity rows, or
+ *   shuffled, with the later layers built one by one, each best given the one before; all
+ *   layers shuffled), each layer in turn is re-placed optimally
  *   given its two neighbours (an assignment problem, Hungarian method), forward and backward,
  *   until nothing improves (at most 64 sweeps); then, 4*L times, two pairs of experts of one layer
  *   are swapped and the descent repeated, keeping the result when it is cheaper. The cheapest
@@ -459,6 +460,24 @@ moe_status_t moe_exchange_schedule(int32_t W, const int64_t *rank_matrix, int32_
 moe_status_t moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts,
                                int32_t starts, int32_t *gpu_of, int64_t *cost,
                                int64_t *contiguous_cost);
+
+/* Staged expert placement over nodes of GPUs.
+ * [MoE Inference Communication, §ExFlow 形式化：整数线性规划建模, the staged expert affinity:
+ *  first minimise the hops that cross nodes, then, inside each node, the hops that cross GPUs]
+ * GPUs are numbered node by node (GPU g is on node g / gpus_per_node). Stage 1 places every
+ * layer's experts on the nodes (E / nodes each) by the method of moe_place_experts; stage 2, for
+ * each node, places that node's experts on its GPUs by the same method, on the affinity counts
+ * restricted to the node's experts of consecutive layers. Each GPU gets E / (nodes *
+ * gpus_per_node) experts per layer. Outputs (HOST): gpu_of [L][E]; node_hops / gpu_hops (nullable):
+ * the hops between consecutive layers whose experts sit on different nodes / GPUs; and the same
+ * two for the contiguous placement (expert e on GPU e / (E / (nodes * gpus_per_node))).
+ * counts as for moe_place_experts. Errors: as moe_place_experts, with E % (nodes *
+ * gpus_per_node) != 0. Pure host computation, needs no GPU. */
+moe_status_t moe_place_experts_staged(int32_t L, int32_t E, int32_t nodes, int32_t gpus_per_node,
+                                      const int64_t *counts, int32_t starts, int32_t *gpu_of,
+                                      int64_t *node_hops, int64_t *gpu_hops,
+                                      int64_t *contiguous_node_hops,
+                                      int64_t *contiguous_gpu_hops);
 
 /* Reads (and, if clear != 0, resets) the calling device's sticky error word. Synchronises
  * the device. Returns MOE_OK when no kernel has recorded an error. */

@@ -243,3 +243,59 @@ def test_placement_deployed_by_relabelling_experts(m):
     for j in range(L - 1):
         np.testing.assert_array_equal(counts2[j][np.ix_(new_ids[j], new_ids[j + 1])], counts[j])
     assert xp.placement_cost(counts2, xp.contiguous_placement(L, E, P)) == cost
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_staged_placement_costs_and_shape(m, seed):
+    """Nodes first, then GPUs inside each node: every GPU holds E / (nodes * gpus) experts of
+    every layer; the reported node and GPU hop counts are the oracle's costs of the placement
+    seen at node and at GPU granularity; stage 1 is moe_place_experts on the nodes."""
+    rng = np.random.default_rng(400 + seed)
+    L, E, nodes, gpn = [(3, 16, 2, 4), (4, 32, 4, 2), (2, 64, 2, 4), (3, 24, 3, 2)][seed]
+    counts = rng.integers(0, 12, (L - 1, E, E))
+    g, hops = m.moe_place_experts_staged(counts, L, E, nodes, gpn, starts=4)
+    P = nodes * gpn
+    for layer in g:
+        assert np.bincount(layer, minlength=P).tolist() == [E // P] * P
+    assert hops["gpu_hops"] == xp.placement_cost(counts, g)
+    assert hops["node_hops"] == xp.placement_cost(counts, g // gpn)
+    contiguous = xp.contiguous_placement(L, E, P)
+    assert hops["contiguous_gpu_hops"] == xp.placement_cost(counts, contiguous)
+    assert hops["contiguous_node_hops"] == xp.placement_cost(counts, contiguous // gpn)
+    _, node_cost, _ = m.moe_place_experts(counts, L, E, nodes, starts=4)
+    assert hops["node_hops"] == node_cost
+    assert hops["node_hops"] <= hops["contiguous_node_hops"]
+
+
+def test_staged_placement_keeps_planted_groups_on_nodes(m):
+    """Tokens that stay inside groups of 8 experts across layers (a permutation of the groups
+    per layer, plus noise): the staged placement keeps every group on one node, so the only
+    node crossings are the noise; inside the node the hops between the group's experts also
+    follow a partner permutation, which stage 2 keeps on one GPU."""
+    rng = np.random.default_rng(12)
+    L, E, nodes, gpn = 3, 32, 4, 2
+    counts = rng.integers(0, 2, (L - 1, E, E))
+    planted = 0
+    groups = rng.permutation(E).reshape(nodes, E // nodes)   # layer 0's groups
+    for j in range(L - 1):
+        perm = rng.permutation(E)        # expert i hands on to perm[i] ...
+        for grp in groups:               # ... and to the rest of its group's image, less so
+            nxt = perm[grp]
+            for a in grp:
+                counts[j, a, nxt] += 20
+                planted += 20 * len(nxt)
+            counts[j, grp, nxt] += 200
+            planted += 200 * len(grp)
+        groups = perm[groups]            # the groups of layer j + 1
+    g, hops = m.moe_place_experts_staged(counts, L, E, nodes, gpn, starts=8)
+    noise = int(counts.sum()) - planted
+    assert hops["node_hops"] <= noise
+    assert hops["gpu_hops"] < 0.5 * hops["contiguous_gpu_hops"]
+
+
+def test_staged_placement_errors(m):
+    c = np.ones((1, 12, 12), np.int64)
+    with pytest.raises(m.MoeError):
+        m.moe_place_experts_staged(c, 2, 12, 5, 2)    # 12 experts do not split over 10 GPUs
+    with pytest.raises(m.MoeError):
+        m.moe_place_experts_staged(-c, 2, 12, 2, 3)
