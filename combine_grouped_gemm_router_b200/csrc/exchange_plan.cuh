@@ -15,9 +15,9 @@
 //    hops between consecutive layers cross GPUs ("MoE Inference Communication", §ExFlow
 //    形式化：整数线性规划建模: the objective, the equal-share and one-GPU-per-expert
 //    constraints). The pages solve it as an ILP; here it is solved by block coordinate descent:
-//    the placement of one layer, given both neighbours, is an assignment problem (experts to GPU
-//    slots, each GPU E/P slots) solved exactly with the Hungarian method, so every accepted move
-//    lowers the cost; sweeps run forward and backward over the layers from several starts, and
+//    the placement of one layer, given both neighbours, is a transportation problem (experts to
+//    GPUs, E/P each) solved exactly by successive shortest paths, so every accepted move lowers
+//    the cost; sweeps run forward and backward over the layers from several starts, and
 //    each start's result is perturbed and descended again a few times (iterated local search).
 #pragma once
 
@@ -177,57 +177,78 @@ inline bool exchange_schedule(int W, const int64_t *D, int max_phases, int32_t *
 
 // ------------------------------------------------------------------ expert placement
 
-// Minimum-cost perfect assignment of n rows to n columns (Hungarian method with row and
-// column potentials, O(n^3)). cost is n x n, row-major. Writes col_of_row.
-inline void min_cost_assignment(int n, const std::vector<int64_t> &cost,
-                                std::vector<int> *col_of_row)
+// Experts to P GPUs, E / P each, maximising the summed score[e][q] (E x P, row-major): a
+// transportation problem, solved exactly by successive shortest paths over the GPUs with
+// potentials (the Hungarian method with capacitated columns). Experts enter one at a time; a
+// Dijkstra over GPUs, reduced costs cost - u[e] - v[q] >= 0 (cost = -score), finds the cheapest
+// way to seat the newcomer, possibly moving seated experts to other GPUs along the path; the
+// potentials then keep every seated pair at reduced cost 0. O(E^2 P) in all, against O(E^3)
+// for the square assignment with E/P copies of each GPU.
+inline void balanced_assignment(int E, int P, const std::vector<int64_t> &score,
+                                std::vector<int> *bin_of)
 {
-    const int64_t INF = INT64_MAX / 4;
-    std::vector<int64_t> u(n + 1, 0), v(n + 1, 0), minv(n + 1);
-    std::vector<int> row_of_col(n + 1, 0), way(n + 1, 0);
-    std::vector<char> used(n + 1);
-    for (int r = 1; r <= n; ++r) {
-        row_of_col[0] = r;
-        int c0 = 0;
-        std::fill(minv.begin(), minv.end(), INF);
-        std::fill(used.begin(), used.end(), 0);
-        do {
-            used[c0] = 1;
-            const int r0 = row_of_col[c0];
-            int64_t delta = INF;
-            int c1 = 0;
-            for (int c = 1; c <= n; ++c) {
-                if (used[c])
-                    continue;
-                const int64_t cur = cost[(size_t)(r0 - 1) * n + (c - 1)] - u[r0] - v[c];
-                if (cur < minv[c]) {
-                    minv[c] = cur;
-                    way[c] = c0;
-                }
-                if (minv[c] < delta) {
-                    delta = minv[c];
-                    c1 = c;
-                }
+    const int share = E / P;
+    std::vector<int64_t> u(E, 0), v(P, 0), dist(P);
+    std::vector<int> prev_row(P), prev_bin(P), count(P, 0);
+    std::vector<char> done(P);
+    std::vector<std::vector<int>> members(P);
+    bin_of->assign(E, -1);
+    auto rc = [&](int e, int q) { return -score[(size_t)e * P + q] - u[e] - v[q]; };
+    for (int s = 0; s < E; ++s) {
+        for (int q = 0; q < P; ++q) {
+            dist[q] = rc(s, q);
+            prev_row[q] = s;
+            prev_bin[q] = -1;
+            done[q] = 0;
+        }
+        int t = -1;
+        for (;;) {
+            int q = -1;
+            for (int k = 0; k < P; ++k)
+                if (!done[k] && (q < 0 || dist[k] < dist[q]))
+                    q = k;
+            done[q] = 1;
+            if (count[q] < share) {
+                t = q;
+                break;
             }
-            for (int c = 0; c <= n; ++c) {
-                if (used[c]) {
-                    u[row_of_col[c]] += delta;
-                    v[c] -= delta;
-                } else {
-                    minv[c] -= delta;
+            for (int r : members[q])
+                for (int k = 0; k < P; ++k) {
+                    if (done[k])
+                        continue;
+                    const int64_t nd = dist[q] + rc(r, k);
+                    if (nd < dist[k]) {
+                        dist[k] = nd;
+                        prev_row[k] = r;
+                        prev_bin[k] = q;
+                    }
                 }
+        }
+        const int64_t delta = dist[t];
+        for (int q = 0; q < P; ++q)
+            if (done[q]) {
+                v[q] -= delta - dist[q];
+                for (int r : members[q])
+                    u[r] += delta - dist[q];
             }
-            c0 = c1;
-        } while (row_of_col[c0] != 0);
-        do {
-            const int c1 = way[c0];
-            row_of_col[c0] = row_of_col[c1];
-            c0 = c1;
-        } while (c0);
+        u[s] += delta;
+        // seat along the path: the row that reached t moves into t, and so on back to s
+        for (int q = t;;) {
+            const int r = prev_row[q];
+            const int from = prev_bin[q];
+            if (from >= 0) {
+                auto &m = members[from];
+                m.erase(std::find(m.begin(), m.end(), r));
+                --count[from];
+            }
+            members[q].push_back(r);
+            ++count[q];
+            (*bin_of)[r] = q;
+            if (r == s)
+                break;
+            q = from;
+        }
     }
-    col_of_row->assign(n, -1);
-    for (int c = 1; c <= n; ++c)
-        (*col_of_row)[row_of_col[c] - 1] = c - 1;
 }
 
 struct Placement {
@@ -252,7 +273,6 @@ struct Placement {
     // the result is taken even when it is not better); returns true if it changed the layer.
     bool improve_layer(int l, std::vector<int32_t> *g, bool right = true) const
     {
-        const int share = E / P;
         std::vector<int64_t> score((size_t)E * P, 0);
         if (l > 0)
             for (int i = 0; i < E; ++i) {
@@ -267,22 +287,17 @@ struct Placement {
         int64_t current = 0;
         for (int e = 0; e < E; ++e)
             current += score[(size_t)e * P + (*g)[(size_t)l * E + e]];
-        // GPU q owns columns [q*share, (q+1)*share) of the square assignment.
-        std::vector<int64_t> cost((size_t)E * E);
-        for (int e = 0; e < E; ++e)
-            for (int c = 0; c < E; ++c)
-                cost[(size_t)e * E + c] = -score[(size_t)e * P + c / share];
-        std::vector<int> col;
-        min_cost_assignment(E, cost, &col);
+        std::vector<int> bin;
+        balanced_assignment(E, P, score, &bin);
         int64_t best = 0;
         for (int e = 0; e < E; ++e)
-            best += score[(size_t)e * P + col[e] / share];
+            best += score[(size_t)e * P + bin[e]];
         if (right && best <= current)
             return false;
         bool changed = false;
         for (int e = 0; e < E; ++e) {
-            changed |= (*g)[(size_t)l * E + e] != col[e] / share;
-            (*g)[(size_t)l * E + e] = col[e] / share;
+            changed |= (*g)[(size_t)l * E + e] != bin[e];
+            (*g)[(size_t)l * E + e] = bin[e];
         }
         return changed;
     }

@@ -449,12 +449,12 @@ moe_status_t moe_exchange_schedule(int32_t W, const int64_t *rank_matrix, int32_
  *   contiguous; layer 0 contiguous, grouped by the similarity of its experts' affinity rows, or
  *   shuffled, with the later layers built one by one, each best given the one before; all
  *   layers shuffled), each layer in turn is re-placed optimally
- *   given its two neighbours (an assignment problem, Hungarian method), forward and backward,
+ *   given its two neighbours (a transportation problem, solved exactly), forward and backward,
  *   until nothing improves (at most 64 sweeps); then, 4*L times, two pairs of experts of one layer
  *   are swapped and the descent repeated, keeping the result when it is cheaper. The cheapest
  *   placement over the starts is returned; start 0 makes it never worse than contiguous.
- *   Deterministic. Cost grows as starts * L^2 * E^3 (E = 64, L = 4, 16 starts: about 0.4 s;
- *   E = 256: about 15 s).
+ *   Deterministic. Cost grows as starts * L^2 * E^2 * P (E = 64, L = 4, 16 starts: 0.05 s;
+ *   E = 256: 0.5 s; 58 layers of 256 experts on 32 GPUs, one start: 20 s).
  * Errors: null counts (L > 1) or gpu_of; L < 1; E outside [1, 256]; P < 1 or E % P != 0;
  *   starts outside [1, 64]; a negative count. Pure host computation, needs no GPU. */
 moe_status_t moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts,
