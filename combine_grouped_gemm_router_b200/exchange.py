@@ -81,6 +81,9 @@ def exchange_rows_ordered(send: torch.Tensor, D: torch.Tensor, group=None,
         raise ValueError("send holds sum(D[rank]) rows")
     send = send.contiguous()
     recv = send.new_empty((recv_off[-1],) + tuple(send.shape[1:]))
+    # NCCL needs every rank of the group in its first collective before point-to-point batches
+    # that leave some ranks out (a phase may): a barrier makes that true whatever came before
+    dist.barrier(group=group)
     # rows that stay on this rank
     recv[recv_off[r]:recv_off[r + 1]] = send[send_off[r]:send_off[r + 1]]
     sent = [0] * W  # rows of each destination block already sent
