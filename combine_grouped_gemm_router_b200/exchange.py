@@ -20,7 +20,7 @@ collectives; it launches no kernel of its own.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Sequence
+from typing import List, Sequence
 
 import torch
 import torch.distributed as dist
@@ -75,6 +75,18 @@ def exchange_rows_ordered(send: torch.Tensor, D: torch.Tensor, group=None,
         dst, ln, _ = moe_exchange_schedule(D.numpy())
     else:
         dst, ln = schedule
+    # every rank checks the whole schedule before any transfer, so all raise together
+    total = [[0] * W for _ in range(W)]
+    for s in range(len(ln)):
+        busy = [int(dst[s][i]) for i in range(W) if int(dst[s][i]) >= 0]
+        if len(set(busy)) != len(busy) or any(int(dst[s][i]) == i for i in range(W)) or \
+                int(ln[s]) <= 0:
+            raise ValueError(f"schedule phase {s} is not a matching of distinct receivers")
+        for i in range(W):
+            if int(dst[s][i]) >= 0:
+                total[i][int(dst[s][i])] += int(ln[s])
+    if any(total[i][j] != int(D[i, j]) for i in range(W) for j in range(W) if i != j):
+        raise ValueError("the schedule does not deliver D")
     send_off = _offsets(D[r].tolist())
     recv_off = _offsets(D[:, r].tolist())
     if send.shape[0] != send_off[-1]:
@@ -96,17 +108,11 @@ def exchange_rows_ordered(send: torch.Tensor, D: torch.Tensor, group=None,
             a = send_off[j] + sent[j]
             ops.append(dist.P2POp(dist.isend, send[a:a + n], j, group))
             sent[j] += n
-        srcs = [i for i in range(W) if int(dst[s][i]) == r]
-        if len(srcs) > 1:
-            raise ValueError("a schedule phase feeds one receiver from two senders")
-        for i in srcs:
+        for i in (i for i in range(W) if int(dst[s][i]) == r):
             b = recv_off[i] + got[i]
             ops.append(dist.P2POp(dist.irecv, recv[b:b + n], i, group))
             got[i] += n
         if ops:
             for work in dist.batch_isend_irecv(ops):
                 work.wait()
-    if any(sent[j] != int(D[r, j]) for j in range(W) if j != r) or \
-            any(got[i] != int(D[i, r]) for i in range(W) if i != r):
-        raise ValueError("the schedule does not deliver D")
     return recv

@@ -78,3 +78,21 @@ def test_exchange_delivers_every_block(world, seed):
         np.testing.assert_array_equal(plain, expect)
         np.testing.assert_array_equal(ordered, expect)
         np.testing.assert_array_equal(ordered2, expect)
+
+
+def test_ordered_exchange_rejects_a_bad_schedule_before_sending(monkeypatch):
+    """A schedule that is not a matching, or does not deliver D, is refused by every rank before
+    any transfer (checked here in one process as rank 0 of 2: the check needs no peers)."""
+    import torch
+    import torch.distributed as dist
+
+    from combine_grouped_gemm_router_b200 import exchange as ex
+    monkeypatch.setattr(dist, "get_rank", lambda group=None: 0)
+    monkeypatch.setattr(dist, "get_world_size", lambda group=None: 2)
+    D = torch.tensor([[0, 3], [2, 0]])
+    with pytest.raises(ValueError):      # receiver 1 fed by both ranks (one to itself)
+        ex.exchange_rows_ordered(torch.zeros(3, 1), D, schedule=(np.array([[1, 1]]),
+                                                                 np.array([3])))
+    with pytest.raises(ValueError):      # a matching, but it delivers too little
+        ex.exchange_rows_ordered(torch.zeros(3, 1), D, schedule=(np.array([[1, 0]]),
+                                                                 np.array([2])))
