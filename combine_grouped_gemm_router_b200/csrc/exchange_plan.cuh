@@ -17,8 +17,12 @@
 //    constraints). The pages solve it as an ILP; here it is solved by block coordinate descent:
 //    the placement of one layer, given both neighbours, is a transportation problem (experts to
 //    GPUs, E/P each) solved exactly by successive shortest paths, so every accepted move lowers
-//    the cost; sweeps run forward and backward over the layers from several starts, and
+//    the cost; sweeps run forward and backward over the layers from several starts (one of
+//    them groups the first layer's experts by the similarity of their affinity rows), and
 //    each start's result is perturbed and descended again a few times (iterated local search).
+//
+//  * place_experts_staged: the staged form of the same page — experts on nodes first, then, node
+//    by node, on that node's GPUs.
 #pragma once
 
 #include <stdint.h>
