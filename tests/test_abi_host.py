@@ -223,3 +223,27 @@ def test_y_buffer_sizes(m):
     P = 0x100000  # a fake, 16-byte aligned address: never dereferenced
     s8 = m.make_shape(64, 136, 256, 8, 2, 4, fp8_return=True)
     assert _raw(m).moe_combine(ctypes.byref(s8), P, P, P, None, None, P, None) == 2
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/moe_b200.h is a C header: it compiles as strict C11 (no C++ or CUDA types in the
+    signatures), and a C program can call a host entry point through it and link."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use.c"
+    src.write_text(
+        '#include "moe_b200.h"\n'
+        "int main(void) {\n"
+        "    moe_shape_t s = {64, 128, 256, 8, 2, 4, 0.0f, 0u};\n"
+        "    return moe_capacity(&s) == 128 && moe_abi_version() == MOE_ABI_VERSION ? 0 : 1;\n"
+        "}\n")
+    lib_dir = os.path.join(root, "combine_grouped_gemm_router_b200")
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                    "-L", lib_dir, "-l:libmoe_b200.so", "-Wl,-rpath," + lib_dir],
+                   check=True, capture_output=True)
+    assert subprocess.run([str(exe)]).returncode == 0
