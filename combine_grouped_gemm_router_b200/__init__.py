@@ -405,6 +405,17 @@ def moe_place_experts(counts, L: int, E: int, P: int, starts: int = 16):
     return g, int(cost.value), int(base.value)
 
 
+def placement_order(gpu_of):
+    """Storage order that deploys a placement: order[l][s] = the expert of layer l stored at
+    slot s, GPU by GPU (experts ascending within a GPU), so that slot s sits on GPU
+    s // (E / P) as the contiguous rank layout of the dispatch expects. Permute a layer's
+    router rows and expert weights with it (offline, when the weights are loaded)."""
+    import numpy as np
+    g = np.asarray(gpu_of)
+    E = g.shape[-1]
+    return np.stack([np.lexsort((np.arange(E), row)) for row in g.reshape(-1, E)]).reshape(g.shape)
+
+
 def moe_place_experts_staged(counts, L: int, E: int, nodes: int, gpus_per_node: int,
                              starts: int = 16):
     """Two-stage placement (nodes, then GPUs inside each node) from affinity counts

@@ -231,8 +231,10 @@ def test_placement_deployed_by_relabelling_experts(m):
     gpu_of, cost, base = m.moe_place_experts(counts, L, E, P)
     assert cost < base
     topk2, new_ids = [], []
+    orders = m.placement_order(gpu_of)
     for l in range(L):
-        order = np.lexsort((np.arange(E), gpu_of[l]))      # GPU by GPU, experts ascending
+        order = orders[l]                                   # GPU by GPU, experts ascending
+        assert (gpu_of[l][order] == np.arange(E) // (E // P)).all()
         new_id = np.empty(E, np.int64)
         new_id[order] = np.arange(E)
         new_ids.append(new_id)
