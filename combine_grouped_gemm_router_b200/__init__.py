@@ -82,6 +82,7 @@ _sigs = {
     "moe_exchange_schedule": ([c_i32, c_p, c_i32, c_p, c_p, c_p, c_p], c_i32),
     "moe_place_experts": ([c_i32, c_i32, c_i32, c_p, c_i32, c_p, c_p, c_p], c_i32),
     "moe_place_experts_staged": ([c_i32] * 4 + [c_p, c_i32] + [c_p] * 5, c_i32),
+    "moe_placement_order": ([c_i32] * 3 + [c_p] * 2, c_i32),
     "moe_get_device_error": ([ctypes.c_int], c_i32),
     "moe_read_stats": ([c_p, ctypes.POINTER(MoeStats), c_p], c_i32),
     "moe_debug_bounded_wait": ([c_u64, c_p], c_i32),
@@ -405,15 +406,16 @@ def moe_place_experts(counts, L: int, E: int, P: int, starts: int = 16):
     return g, int(cost.value), int(base.value)
 
 
-def placement_order(gpu_of):
-    """Storage order that deploys a placement: order[l][s] = the expert of layer l stored at
-    slot s, GPU by GPU (experts ascending within a GPU), so that slot s sits on GPU
-    s // (E / P) as the contiguous rank layout of the dispatch expects. Permute a layer's
-    router rows and expert weights with it (offline, when the weights are loaded)."""
+def placement_order(gpu_of, P: int):
+    """Storage order that deploys a placement (moe_placement_order): order[l][s] = the expert of
+    layer l to store at slot s, GPU by GPU; permute the router rows and expert weights with it."""
     import numpy as np
-    g = np.asarray(gpu_of)
-    E = g.shape[-1]
-    return np.stack([np.lexsort((np.arange(E), row)) for row in g.reshape(-1, E)]).reshape(g.shape)
+    g = np.ascontiguousarray(gpu_of, dtype=np.int32)
+    L, E = g.shape
+    order = np.empty((L, E), np.int32)
+    _check(_lib.moe_placement_order(L, E, int(P), g.ctypes.data_as(c_p),
+                                    order.ctypes.data_as(c_p)), "moe_placement_order")
+    return order
 
 
 def moe_place_experts_staged(counts, L: int, E: int, nodes: int, gpus_per_node: int,

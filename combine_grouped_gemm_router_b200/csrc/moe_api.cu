@@ -1513,6 +1513,28 @@ moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *counts, int32_
 }
 
 __attribute__((visibility("default"))) moe_status_t
+moe_placement_order(int32_t L, int32_t E, int32_t P, const int32_t *gpu_of, int32_t *order)
+{
+    if (!gpu_of || !order || L < 1 || E < 1 || P < 1 || E % P != 0)
+        return MOE_ERR_INVALID_ARG;
+    const int share = E / P;
+    std::vector<int> fill(P);
+    for (int l = 0; l < L; ++l) {
+        const int32_t *g = gpu_of + (size_t)l * E;
+        std::fill(fill.begin(), fill.end(), 0);
+        for (int e = 0; e < E; ++e) {
+            if (g[e] < 0 || g[e] >= P || fill[g[e]] >= share)
+                return MOE_ERR_INVALID_ARG;  // not a placement with E / P experts per GPU
+            ++fill[g[e]];
+        }
+        std::fill(fill.begin(), fill.end(), 0);
+        for (int e = 0; e < E; ++e)  // experts ascending within each GPU
+            order[(size_t)l * E + (size_t)g[e] * share + fill[g[e]]++] = e;
+    }
+    return MOE_OK;
+}
+
+__attribute__((visibility("default"))) moe_status_t
 moe_place_experts_staged(int32_t L, int32_t E, int32_t nodes, int32_t gpus_per_node,
                          const int64_t *counts, int32_t starts, int32_t *gpu_of,
                          int64_t *node_hops, int64_t *gpu_hops, int64_t *contiguous_node_hops,

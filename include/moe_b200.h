@@ -461,6 +461,15 @@ moe_status_t moe_place_experts(int32_t L, int32_t E, int32_t P, const int64_t *c
                                int32_t starts, int32_t *gpu_of, int64_t *cost,
                                int64_t *contiguous_cost);
 
+/* Storage order that deploys a placement: gpu_of [L][E] (HOST, from moe_place_experts or
+ * moe_place_experts_staged) -> order [L][E] (HOST, out): order[l][s] = the expert of layer l to
+ * store at slot s, GPU by GPU and experts ascending within a GPU, so that slot s sits on GPU
+ * s / (E / P), the contiguous rank layout of the dispatch. Permuting a layer's router rows and
+ * expert weights by it deploys the placement. MOE_ERR_INVALID_ARG unless every GPU holds
+ * exactly E / P experts of every layer. Pure host computation. */
+moe_status_t moe_placement_order(int32_t L, int32_t E, int32_t P, const int32_t *gpu_of,
+                                 int32_t *order);
+
 /* Staged expert placement over nodes of GPUs.
  * [MoE Inference Communication, §ExFlow 形式化：整数线性规划建模, the staged expert affinity:
  *  first minimise the hops that cross nodes, then, inside each node, the hops that cross GPUs]

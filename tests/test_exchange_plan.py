@@ -231,7 +231,7 @@ def test_placement_deployed_by_relabelling_experts(m):
     gpu_of, cost, base = m.moe_place_experts(counts, L, E, P)
     assert cost < base
     topk2, new_ids = [], []
-    orders = m.placement_order(gpu_of)
+    orders = m.placement_order(gpu_of, P)
     for l in range(L):
         order = orders[l]                                   # GPU by GPU, experts ascending
         assert (gpu_of[l][order] == np.arange(E) // (E // P)).all()
@@ -301,3 +301,11 @@ def test_staged_placement_errors(m):
         m.moe_place_experts_staged(c, 2, 12, 5, 2)    # 12 experts do not split over 10 GPUs
     with pytest.raises(m.MoeError):
         m.moe_place_experts_staged(-c, 2, 12, 2, 3)
+
+
+def test_placement_order_errors(m):
+    with pytest.raises(m.MoeError):
+        m.placement_order(np.array([[0, 0, 0, 1]]), 2)   # GPU 0 holds 3 of 4 experts
+    with pytest.raises(m.MoeError):
+        m.placement_order(np.array([[0, 2, 1, 1]]), 2)   # no GPU 2
+    assert m.placement_order(np.array([[1, 0, 0, 1]]), 2).tolist() == [[1, 2, 0, 3]]
