@@ -1,9 +1,12 @@
 """Python binding of the B200 MoE layer library (``libmoe_b200.so``).
 
 Argument marshalling only: every step of the layer runs in the library's CUDA
-kernels. Torch tensors supply device memory and the current stream. The
-functions keep the C names of ``include/moe_b200.h``; each raises
-``MoeError`` on a non-OK status. There is no fallback: the first call raises
+kernels, and the exchange planning (moe_exchange_schedule, moe_place_experts,
+moe_place_experts_staged, moe_placement_order) in its host code. Torch tensors
+supply device memory and the current stream; the planning functions take and
+return numpy arrays. The functions keep the C names of ``include/moe_b200.h``;
+each raises ``MoeError`` on a non-OK status. ``exchange`` (a submodule) moves
+packed rows between ranks with torch.distributed. There is no fallback: the first call raises
 ``ImportError`` when the library has not been built
 (``python -m combine_grouped_gemm_router_b200.build``).
 """
