@@ -309,3 +309,52 @@ def test_placement_order_errors(m):
     with pytest.raises(m.MoeError):
         m.placement_order(np.array([[0, 2, 1, 1]]), 2)   # no GPU 2
     assert m.placement_order(np.array([[1, 0, 0, 1]]), 2).tolist() == [[1, 2, 0, 3]]
+
+
+def test_schedule_on_random_and_degenerate_matrices(m):
+    """Seeded sweep: tiny entries (many ties), huge sparse entries (2^40), one non-zero block,
+    rank-one traffic, dense traffic, 1 to 19 ranks; every order a valid contention-free
+    delivery of D of length tau_min."""
+    rng = np.random.default_rng(123)
+    for it in range(120):
+        W = int(rng.integers(1, 20))
+        kind = it % 5
+        if kind == 0:
+            D = rng.integers(0, 3, (W, W))
+        elif kind == 1:
+            D = (rng.integers(0, 2 ** 40, (W, W)) * (rng.random((W, W)) < 0.3)).astype(np.int64)
+        elif kind == 2:
+            D = np.zeros((W, W), np.int64)
+            D[rng.integers(0, W), rng.integers(0, W)] = int(rng.integers(1, 100))
+        elif kind == 3:
+            D = np.outer(rng.integers(0, 5, W), rng.integers(0, 5, W)).astype(np.int64)
+        else:
+            D = rng.integers(0, 1000, (W, W))
+        dst, ln, span = m.moe_exchange_schedule(D)
+        assert span == xp.exchange_bound(D)
+        if len(ln):
+            check_schedule(D, dst, ln, span)
+
+
+def test_placements_on_random_and_degenerate_counts(m):
+    """Seeded sweep of one-level and staged placements: no hops at all, 0/1 counts, counts up
+    to 1e9; shapes, costs (oracle), never worse than contiguous, and the storage order."""
+    rng = np.random.default_rng(7)
+    for it in range(60):
+        P, share, L = int(rng.integers(1, 6)), int(rng.integers(1, 5)), int(rng.integers(1, 5))
+        E = P * share
+        hi = (1, 2, 10 ** 9)[it % 3]
+        c = rng.integers(0, hi, (L - 1, E, E)) if L > 1 else np.zeros(0, np.int64)
+        g, cost, base = m.moe_place_experts(c, L, E, P, starts=3)
+        for row in g:
+            assert np.bincount(row, minlength=P).tolist() == [share] * P
+        if L > 1:
+            assert cost == xp.placement_cost(c, g) <= base
+            assert base == xp.placement_cost(c, xp.contiguous_placement(L, E, P))
+        order = m.placement_order(g, P)
+        assert all((g[l][order[l]] == np.arange(E) // share).all() for l in range(L))
+        if P > 1 and P % 2 == 0:
+            gs, hops = m.moe_place_experts_staged(c, L, E, 2, P // 2, starts=2)
+            if L > 1:
+                assert hops["gpu_hops"] == xp.placement_cost(c, gs)
+                assert hops["node_hops"] == xp.placement_cost(c, gs // (P // 2))
