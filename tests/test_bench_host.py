@@ -102,3 +102,19 @@ def test_traffic_gate_ignores_comments_only(tmp_path):
     src.write_text("// header\nint f(int a) { return a + 2; }\n")
     assert bench.kernel_source_hash(str(src)) != h0
     assert bench.up_traffic("mixtral_prefill") is not None   # the captured code is current
+
+
+def test_algorithmic_work_counts_the_payload_and_output_bytes():
+    """The combine's algorithmic bytes follow what it reads and writes: fp32 expert rows or the
+    FP8 return payload (d codes + d/32 exponent bytes per row), and the bf16 layer output."""
+    import bench
+    from moe_workloads import WORKLOADS
+    w = WORKLOADS["e128_skew_fp8"]
+    R, N, d, K = 21185, w.N, w.d, w.K
+    plain = bench.algorithmic_work(w, R, 128)["combine_bytes"]
+    ret = bench.algorithmic_work(w.with_(fp8_return=True), R, 128)["combine_bytes"]
+    assert plain == R * d * 4 + N * K * 8 + N * d * 2
+    assert ret == R * (d + d // 32) + N * K * 8 + N * d * 2
+    up = bench.algorithmic_work(WORKLOADS["mixtral_prefill"], 8192, 8)
+    assert up["up_flops"] == 4.0 * 4096 * 14336 * 8192
+    assert up["up_bytes"] == 2.0 * 8 * 14336 * 4096 * 2 + 8192 * 4096 * 2 + 8192 * 14336 * 2
