@@ -103,3 +103,34 @@ def ilp_placement(counts, P: int):
     x = np.round(res.x[:nx]).astype(np.int64).reshape(L, E, P)
     gpu_of = x.argmax(axis=2).astype(np.int32)
     return int(round(res.fun)), gpu_of
+
+
+def greedy_order_makespan(D) -> int:
+    """The page's transmission-order procedure (§Aurora 场景 1, the steps after 定理 4.2) read as
+    a list schedule, for comparison with the bound: the bottleneck rank (largest send or receive
+    volume) first, the other ranks by send volume, largest first; each rank sends its blocks one
+    after another (largest first), each block whole, starting at the earliest time at which both
+    the rank and the block's receiver are free, so that no receiver is fed by two senders at
+    once. Returns the time the last block ends, in rows (ties to the lower rank index)."""
+    D = np.array(D, dtype=np.int64, copy=True)
+    np.fill_diagonal(D, 0)
+    W = D.shape[0]
+    send, recv = D.sum(axis=1), D.sum(axis=0)
+    load = np.maximum(send, recv)
+    first = int(np.argmax(load))
+    order = [first] + sorted((i for i in range(W) if i != first), key=lambda i: (-send[i], i))
+    busy = [[] for _ in range(W)]   # per receiver: (start, end) intervals taken
+    end_all = 0
+    for i in order:
+        t = 0
+        for j in sorted((j for j in range(W) if D[i, j] > 0), key=lambda j: (-D[i, j], j)):
+            n = int(D[i, j])
+            start = t
+            for a, b in sorted(busy[j]):   # first gap of length n at or after `start`
+                if start + n <= a:
+                    break
+                start = max(start, b)
+            busy[j].append((start, start + n))
+            t = start + n
+            end_all = max(end_all, t)
+    return end_all

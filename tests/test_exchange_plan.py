@@ -358,3 +358,25 @@ def test_placements_on_random_and_degenerate_counts(m):
             if L > 1:
                 assert hops["gpu_hops"] == xp.placement_cost(c, gs)
                 assert hops["node_hops"] == xp.placement_cost(c, gs // (P // 2))
+
+
+def test_literal_greedy_reading_misses_the_bound():
+    """The page's steps read literally as a list schedule of whole blocks (bottleneck rank
+    first, the rest by volume, each block at the earliest time its receiver is free) never beat
+    tau_min and on random 8-rank traffic end well above it, which is why the library builds
+    its order by a matching decomposition that meets the bound exactly."""
+    rng = np.random.default_rng(0)
+    gaps = []
+    for _ in range(100):
+        D = rng.integers(0, 1000, (8, 8)) * (rng.random((8, 8)) < 0.8)
+        bound = xp.exchange_bound(D)
+        g = xp.greedy_order_makespan(D)
+        assert g >= bound
+        gaps.append(g / bound - 1)
+    assert np.mean(gaps) > 0.2
+    # a hand-checked case: 0 -> 1 (2 rows), 0 -> 2 (1), 1 -> 2 (2), 2 -> 0 (1). tau_min = 3
+    # (rank 0 sends 3, rank 2 receives 3); whole blocks, largest first: 0 sends to 1 over [0, 2)
+    # then to 2 over [2, 3); rank 1 (next by volume) sends to 2 over [0, 2); rank 2 to 0 over
+    # [0, 1): makespan 3, the bound.
+    D = np.array([[0, 2, 1], [0, 0, 2], [1, 0, 0]])
+    assert xp.exchange_bound(D) == 3 and xp.greedy_order_makespan(D) == 3
