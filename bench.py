@@ -3,8 +3,11 @@
 One step = one pass of the whole layer over one batch of synthetic tokens:
 router logits -> top-K -> dispatch (histogram, scan, positions, scatter into
 the expert-sorted and the rank-packed buffers) -> gate/up grouped GEMM -> down
-grouped GEMM -> combine. Default workload: the Mixtral-shaped prefill layer
-(N=4096 tokens, d=4096, f=14336, E=8, K=2, W=8 virtual ranks, dropless).
+grouped GEMM -> combine; for a stack of layers, every layer in turn with
+x_(l+1) = bf16(x_l + MoE_l(x_l)). Default workload: the stack of four MoE layers
+(N=32768 tokens, d=4096, f=1536, E=64, K=6, W=8 virtual ranks, capacity factor
+1.25), the largest single-GPU configuration, with every point of its capacity
+factor {1.0, 1.25, 2.0} x Zipf skew {0, 1.2} grid timed as well.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
@@ -333,11 +336,24 @@ def algorithmic_work(w, R: int, E_act: int) -> dict:
     )
 
 
+def gemm_peak_choice(peaks: dict, timed_s: float, clocks: dict) -> tuple:
+    """The bf16 peak the GEMM roofline divides by: the burst cuBLAS figure (a GEMM timed
+    alone), unless the timed region lasted at least a second and the clock record shows the
+    power cap holding the SM clock below its maximum, the condition the sustained figure (a
+    seconds-long GEMM loop under the power cap) was measured in."""
+    capped = ("sw_power_cap" in (clocks.get("reasons") or []) and clocks.get("sm_mhz")
+              and clocks.get("sm_max_mhz") and clocks["sm_mhz"] < 0.95 * clocks["sm_max_mhz"])
+    if timed_s >= 1.0 and capped:
+        return peaks["bf16_tflops_sustained"], "bf16 sustained (timed region >= 1 s, power-capped)"
+    return peaks["bf16_tflops"], "bf16 burst"
+
+
 def run_gpu(args, w) -> dict:
     import torch
 
     import combine_grouped_gemm_router_b200 as m
-    from moe_workloads import make_layer_inputs, make_shared_inputs
+    from moe_workloads import STACK_GRID_CF, STACK_GRID_S, make_layer_inputs, make_shared_inputs
+    from moe_workloads import zipf_bias
 
     world, rank = init_dist("nccl")
     _, _, local = dist_env()
@@ -353,11 +369,21 @@ def run_gpu(args, w) -> dict:
     layers = [make_layer_inputs(w, seed=args.seed + rank, device=str(dev), layer=l, with_x=(l == 0))
               for l in range(L)]
     inp = layers[0]
-    # the layer's output is bf16, as the hidden states it replaces (a stack's next input)
-    shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=True,
-                         slot_major=w.slot_major, reroute=w.reroute, fp8_return=w.fp8_return)
-    RA = m.moe_rows_alloc(shape)
-    ws = torch.empty(m.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
+
+    def make(wl):
+        # the layer's output is bf16, as the hidden states it replaces (a stack's next input)
+        return m.make_shape(wl.N, wl.d, wl.f, wl.E, wl.K, wl.W, wl.cf, out_bf16=True,
+                            slot_major=wl.slot_major, reroute=wl.reroute,
+                            fp8_return=wl.fp8_return)
+
+    shape = make(w)
+    # a stack also times every point of its capacity-factor x Zipf-skew grid (same weights)
+    grid = [w.with_(cf=cf, s=s) for cf in STACK_GRID_CF for s in STACK_GRID_S] \
+        if (L > 1 and not args.no_grid and w.affinity == 0.0) else []
+    shapes = [shape] + [make(g) for g in grid]
+    RA = max(m.moe_rows_alloc(s_) for s_ in shapes)
+    ws = torch.empty(max(m.moe_workspace_size(s_) for s_ in shapes), dtype=torch.uint8,
+                     device=dev)
     x = inp["x"]
     N, K, E, W, d, f = w.N, w.K, w.E, w.W, w.d, w.f
     topk_idx = [torch.empty(N, K, dtype=torch.int32, device=dev) for _ in range(L)]
@@ -384,12 +410,16 @@ def run_gpu(args, w) -> dict:
                 lw[k + "q"], lw[k + "s"] = q, sc
         h_q = torch.empty(RA, f, dtype=torch.uint8, device=dev)
         h_scale = torch.empty(RA, dtype=torch.float32, device=dev)
-        torch.cuda.synchronize(dev)
+    else:
+        # the down projection reads fp16 h and an fp16 copy of W2, made once (static weights)
+        for lw in layers:
+            lw["w2h"] = m.w2_for(shape, lw["w2"])
+    torch.cuda.synchronize(dev)
     D = torch.empty(W * W, dtype=torch.int64, device=dev)
     pk_off = torch.empty(W * W + 1, dtype=torch.int64, device=dev)
-    h = torch.empty(RA, f, dtype=torch.bfloat16, device=dev)
+    h = torch.empty(RA, f, dtype=torch.bfloat16 if w.fp8 else torch.float16, device=dev)
     # fp32 expert outputs, or the FP8 return payload (e4m3 codes + block exponents)
-    y = torch.empty(m.moe_y_bytes(shape), dtype=torch.uint8, device=dev)
+    y = torch.empty(max(m.moe_y_bytes(s_) for s_ in shapes), dtype=torch.uint8, device=dev)
     if L > 1:  # x_{l+1} = bf16(x_l + MoE_l(x_l)), ping-pong buffers
         xbuf = [torch.empty(N, d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
         affinity = torch.zeros(L - 1, E, E, dtype=torch.int64, device=dev)
@@ -398,67 +428,67 @@ def run_gpu(args, w) -> dict:
         out = torch.empty(N, d, dtype=torch.bfloat16, device=dev)
     if shared:  # Residual-MoE: the shared dense MLP on every token
         sh = make_shared_inputs(w, seed=args.seed + rank, device=str(dev))
-        h_s = torch.empty(N, w.shared_f, dtype=torch.bfloat16, device=dev)
+        sh["ws2h"] = m.w2_for(shape, sh["ws2"])
+        h_s = torch.empty(N, w.shared_f, dtype=torch.float16, device=dev)
         y_s = torch.empty(N, d, dtype=torch.float32, device=dev)
         ws_s = torch.empty(256, dtype=torch.uint8, device=dev)
 
     stage_names = ["route", "dispatch", "expert_up", "expert_down"] + (
         ["shared_expert"] if shared else []) + ["combine"]
     n_ev = len(stage_names) + 1
-    # the library's kernels per step: every layer's, plus one affinity count per layer pair
-    launches_per_step = L * kernel_launches(w) + (L - 1)
 
-    def step(ev=None):
-        """One step; ev (optional) is [layer][n_ev] events around the stages."""
+    def step(ev=None, shp=shape, biases=None):
+        """One step; ev (optional) is [layer][n_ev] events around the stages; biases
+        (optional) replaces each layer's router bias (the grid's Zipf skew)."""
         st = torch.cuda.current_stream(dev)
         for l in range(L):
             lw = layers[l]
+            bias = lw["bias"] if biases is None else biases
             xin = x if l == 0 else xbuf[(l - 1) % 2]
             dst = xbuf[l % 2] if L > 1 else out
             e = ev[l] if ev is not None else None
             if e is not None:
                 e[0].record(st)
-            m.moe_route(shape, xin, lw["w_router"], lw["bias"], topk_idx[l], topk_w, logits, ws,
-                        st)
+            m.moe_route(shp, xin, lw["w_router"], bias, topk_idx[l], topk_w, logits, ws, st)
             if e is not None:
                 e[1].record(st)
             if w.fp8:
-                m.moe_dispatch_fp8(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of,
+                m.moe_dispatch_fp8(shp, xin, topk_idx[l], counts, kept, offsets[l], row_of,
                                    assign, x_sorted, sorted_scale, x_packed=x_packed,
                                    packed_scale=packed_scale, rank_matrix=D,
                                    packed_offsets=pk_off, ws=ws, stream=st)
             elif w.reroute:
-                m.moe_dispatch_reroute(shape, xin, logits, topk_idx[l], counts, kept, offsets[l],
+                m.moe_dispatch_reroute(shp, xin, logits, topk_idx[l], counts, kept, offsets[l],
                                        row_of, assign, x_sorted, x_packed=x_packed, rank_matrix=D,
                                        packed_offsets=pk_off, ws=ws, stream=st)
             else:
-                m.moe_dispatch(shape, xin, topk_idx[l], counts, kept, offsets[l], row_of, assign,
+                m.moe_dispatch(shp, xin, topk_idx[l], counts, kept, offsets[l], row_of, assign,
                                x_sorted, x_packed, D, pk_off, None, ws, st)
             if e is not None:
                 e[2].record(st)
             if w.fp8:
-                m.moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets[l], lw["w1q"],
+                m.moe_expert_up_fp8(shp, x_sorted, sorted_scale, offsets[l], lw["w1q"],
                                     lw["w1s"], lw["w3q"], lw["w3s"], h, st)
             else:
-                m.moe_expert_up(shape, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
+                m.moe_expert_up(shp, x_sorted, offsets[l], lw["w1"], lw["w3"], h, st)
             if e is not None:
                 e[3].record(st)
             if w.fp8:  # the kept rows of h to e4m3, then the e4m3 down GEMM
                 m.moe_quantize_rows_e4m3(h, h_q, h_scale, rows_dev=offsets[l][E:], stream=st)
-                m.moe_expert_down_fp8(shape, h_q, h_scale, offsets[l], lw["w2q"], lw["w2s"], y,
+                m.moe_expert_down_fp8(shp, h_q, h_scale, offsets[l], lw["w2q"], lw["w2s"], y,
                                       st)
             else:
-                m.moe_expert_down(shape, h, offsets[l], lw["w2"], y, st)
+                m.moe_expert_down(shp, h, offsets[l], lw["w2h"], y, st)
             j = 4
             if e is not None:
                 e[j].record(st)
             if shared:
-                m.moe_shared_expert(shape, w.shared_f, xin, sh["ws1"], sh["ws3"], sh["ws2"], h_s,
+                m.moe_shared_expert(shp, w.shared_f, xin, sh["ws1"], sh["ws3"], sh["ws2h"], h_s,
                                     y_s, ws_s, st)
                 j += 1
                 if e is not None:
                     e[j].record(st)
-            m.moe_combine(shape, y, row_of, topk_w, dst, residual=xin if L > 1 else None,
+            m.moe_combine(shp, y, row_of, topk_w, dst, residual=xin if L > 1 else None,
                           shared_y=y_s if shared else None, stream=st)
             if e is not None:
                 e[j + 1].record(st)
@@ -466,35 +496,47 @@ def run_gpu(args, w) -> dict:
                 m.moe_affinity_accumulate(N, E, K, topk_idx[l - 1], topk_idx[l], affinity[l - 1],
                                           st)
 
+    def timed(n_steps, shp=shape, biases=None, with_clocks=False):
+        """n_steps eager steps between a barrier and a synchronize on each side, CUDA events
+        around the whole run and between the stages of every step (on the stream the kernels
+        run on). Returns (elapsed s, per-stage ms: mean over steps of the sum over the
+        stack's layers, clock summary or None)."""
+        events = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(L)]
+                  for _ in range(n_steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        sampler = ClockSampler(local) if with_clocks else None
+        if sampler is not None:
+            sampler.__enter__()
+        t0.record(stream)
+        for i in range(n_steps):
+            step(events[i], shp, biases)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        if sampler is not None:
+            sampler.__exit__(None, None, None)
+        barrier()
+        stage = {name: statistics.mean(sum(ev[l][j].elapsed_time(ev[l][j + 1]) for l in range(L))
+                                       for ev in events)
+                 for j, name in enumerate(stage_names)}
+        return t0.elapsed_time(t1) / 1e3, stage, (sampler.summary() if sampler else None)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     if m.moe_get_device_error(True) != 0:
         raise RuntimeError("device error during warm-up")
 
-    # the timed run: K eager steps, CUDA events between the stages of every step (on the
-    # stream the kernels run on), barrier + synchronize on both sides
-    events = [[[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(L)]
-              for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_stop = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        t_start.record(stream)
-        for i in range(args.steps):
-            step(events[i])
-        t_stop.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier()
-    elapsed_s = t_start.elapsed_time(t_stop) / 1e3
-    # per stage: mean over steps of the sum over the stack's layers
-    stage_ms = {name: statistics.mean(sum(ev[l][j].elapsed_time(ev[l][j + 1]) for l in range(L))
-                                      for ev in events)
-                for j, name in enumerate(stage_names)}
+    elapsed_s, stage_ms, clock_summary = timed(args.steps, with_clocks=True)
+    R_layers = [int(o[E].item()) for o in offsets]
+    act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
+    R = R_layers[0]
+    agg = aggregate(float(N * args.steps), elapsed_s, dev)
 
-    # the same step captured once in a CUDA graph (its 9 kernels) and replayed K times: the
-    # host launch overhead disappears, which matters for small (decode) steps
+    # the same step captured once in a CUDA graph and replayed K times: the host launch
+    # overhead disappears, which matters for small (decode) steps
     graph_res = None
     if not args.no_graph:
         graph = torch.cuda.CUDAGraph()
@@ -516,6 +558,44 @@ def run_gpu(args, w) -> dict:
         graph_res = {"value": g_agg["value"], "unit": UNIT,
                      "ms_per_step": g_agg["elapsed_max_s"] / args.steps * 1e3}
         del graph
+
+    peaks = load_peaks()
+    up_peak_bf16, up_peak_name = gemm_peak_choice(peaks, elapsed_s, clock_summary or {})
+
+    def work_of(R_list, A_list, wl):
+        tot = {}
+        for Rl, Al in zip(R_list, A_list):
+            for k, v in algorithmic_work(wl, Rl, Al).items():
+                tot[k] = tot.get(k, 0.0) + v
+        return tot
+
+    # the grid of a stack: every (capacity factor, Zipf skew) point, timed the same way on the
+    # same weights (the bias carries the skew; the capacity factor is in the shape)
+    grid_res = []
+    for gw, gshape in zip(grid, shapes[1:]):
+        gb = zipf_bias(E, gw.s)
+        gb = None if gb is None else gb.to(dev)
+        for _ in range(3):
+            step(None, gshape, gb)
+        torch.cuda.synchronize(dev)
+        gs, gstage, _ = timed(args.grid_steps, gshape, gb)
+        gR = [int(o[E].item()) for o in offsets]
+        gA = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
+        gwk = work_of(gR, gA, gw)
+        up_s, down_s = gstage["expert_up"] / 1e3, gstage["expert_down"] / 1e3
+        g_agg = aggregate(float(N * args.grid_steps), gs, dev)
+        gemm_tf = (gwk["up_flops"] + gwk["down_flops"]) / (up_s + down_s) / 1e12
+        grid_res.append({
+            "capacity_factor": gw.cf, "zipf_s": gw.s, "tokens_per_s": g_agg["value"],
+            "ms_per_step": g_agg["elapsed_max_s"] / args.grid_steps * 1e3,
+            "layer_tokens_per_s": g_agg["value"] * L, "rows_kept": gR,
+            "drop_rate": 1.0 - sum(gR) / float(L * N * K),
+            "stages_ms": {k: round(v, 4) for k, v in gstage.items()},
+            "gate_up_tflops": gwk["up_flops"] / up_s / 1e12,
+            "gemm_tflops": gemm_tf, "gemm_frac_of_bf16_burst": gemm_tf / peaks["bf16_tflops"]})
+    if m.moe_get_device_error(True) != 0:
+        raise RuntimeError("device error during the timed runs")
+
     # the routing report of layer 0 (untimed): one more route + dispatch with the counters on,
     # then the derived figures (drop rate, per-rank send/receive balance, cross-rank fraction,
     # expert-load spread, effective capacity factor, the exchange-time bound tau_min)
@@ -546,25 +626,19 @@ def run_gpu(args, w) -> dict:
     if L > 1:
         routing["placement"] = placement_report(m, affinity.cpu().numpy(), L, E, W)
     err = m.moe_get_device_error(True)
-    R_layers = [int(o[E].item()) for o in offsets]
-    act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
-    R = R_layers[0]
-    agg = aggregate(float(N * args.steps), elapsed_s, dev)
 
-    # end to end through the public API: pinned host input -> moe_layer -> host output
     # end to end through the public API: every step copies its input from pinned host memory,
-    # runs moe_layer and copies the fp32 result back; the copies of one step overlap the layer
-    # of the previous one (two buffers, one copy stream each way)
+    # runs moe_layer (each layer of a stack in turn) and copies the bf16 result back; the copies
+    # of one step overlap the layers of the previous one (two buffers, one copy stream each way)
     e2e = None
     if not args.no_e2e:
         lws_bytes = (m.moe_layer_shared_workspace_size(shape, w.shared_f) if shared
                      else m.moe_layer_workspace_size(shape))
         lws = torch.empty(lws_bytes, dtype=torch.uint8, device=dev)
         x_host = x.cpu().pin_memory()
-        out_dt = torch.bfloat16
-        out_host = [torch.empty(N, d, dtype=out_dt).pin_memory() for _ in range(2)]
+        out_host = [torch.empty(N, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]
-        out_dev = [torch.empty(N, d, dtype=out_dt, device=dev) for _ in range(2)]
+        out_dev = [torch.empty(N, d, dtype=torch.bfloat16, device=dev) for _ in range(2)]
         mid = [torch.empty_like(x) for _ in range(2)] if L > 1 else None
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(2)]
@@ -579,31 +653,23 @@ def run_gpu(args, w) -> dict:
             ev_in[b].record(s_in)
             stream.wait_event(ev_in[b])
             stream.wait_event(ev_out[b])  # buffer b's previous result has left the device
-            l0 = layers[0]
-            if shared:
-                m.moe_layer_shared(shape, w.shared_f, x_dev[b], l0["w_router"], l0["bias"],
-                                   l0["w1"], l0["w3"], l0["w2"], sh["ws1"], sh["ws3"], sh["ws2"],
-                                   out_dev[b], ws=lws, stream=stream)
-            elif w.fp8 and L == 1:
-                m.moe_layer_fp8(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1q"],
-                                l0["w1s"], l0["w3q"], l0["w3s"], l0["w2q"], l0["w2s"], out_dev[b],
-                                ws=lws, stream=stream)
-            elif L == 1:
-                m.moe_layer(shape, x_dev[b], l0["w_router"], l0["bias"], l0["w1"], l0["w3"],
-                            l0["w2"], out_dev[b], ws=lws, stream=stream)
-            else:  # the stack: each layer adds its MoE output to its input, bf16 in between
-                xin = x_dev[b]
-                for l in range(L):
-                    lw = layers[l]
-                    dst = out_dev[b] if l == L - 1 else mid[l % 2]
-                    if w.fp8:
-                        m.moe_layer_fp8(shape, xin, lw["w_router"], lw["bias"], lw["w1q"],
-                                        lw["w1s"], lw["w3q"], lw["w3s"], lw["w2q"], lw["w2s"], dst,
-                                        residual=xin, ws=lws, stream=stream)
-                    else:
-                        m.moe_layer(shape, xin, lw["w_router"], lw["bias"], lw["w1"], lw["w3"],
-                                    lw["w2"], dst, residual=xin, ws=lws, stream=stream)
-                    xin = dst
+            xin = x_dev[b]
+            for l in range(L):
+                lw = layers[l]
+                dst = out_dev[b] if l == L - 1 else mid[l % 2]
+                res = xin if L > 1 else None
+                if shared:
+                    m.moe_layer_shared(shape, w.shared_f, xin, lw["w_router"], lw["bias"],
+                                       lw["w1"], lw["w3"], lw["w2h"], sh["ws1"], sh["ws3"],
+                                       sh["ws2h"], dst, residual=res, ws=lws, stream=stream)
+                elif w.fp8:
+                    m.moe_layer_fp8(shape, xin, lw["w_router"], lw["bias"], lw["w1q"], lw["w1s"],
+                                    lw["w3q"], lw["w3s"], lw["w2q"], lw["w2s"], dst, residual=res,
+                                    ws=lws, stream=stream)
+                else:
+                    m.moe_layer(shape, xin, lw["w_router"], lw["bias"], lw["w1"], lw["w3"],
+                                lw["w2h"], dst, residual=res, ws=lws, stream=stream)
+                xin = dst
             ev_comp[b].record(stream)
             s_out.wait_event(ev_comp[b])
             with torch.cuda.stream(s_out):
@@ -629,24 +695,18 @@ def run_gpu(args, w) -> dict:
         e2e_agg = aggregate(float(N * args.steps), e0.elapsed_time(e1) / 1e3, dev)
         e2e = {"value": e2e_agg["value"], "unit": UNIT, "h2d_bytes_per_step": N * d * 2,
                "d2h_bytes_per_step": N * d * 2,
-               "note": "pinned host input and output; copies overlap the previous step's layer"}
+               "note": "pinned host input and output; copies overlap the previous step's layers"}
         del lws
 
     # algorithmic work of one step (all layers of a stack)
-    work = {}
-    for Rl, Al in zip(R_layers, act_layers):
-        for k, v in algorithmic_work(w, Rl, Al).items():
-            work[k] = work.get(k, 0.0) + v
-    peaks = load_peaks()
+    work = work_of(R_layers, act_layers, w)
     up_ratio = 2.0 if w.fp8 else 1.0  # e4m3 tensor throughput is twice bf16's (nominal)
-    # the GEMM is timed inside a long run of steps at the power cap, so its peak is the
-    # sustained cuBLAS figure; the burst figure (a GEMM timed alone) is reported beside it
-    up_peak = peaks["bf16_tflops_sustained"] * up_ratio
+    up_peak = up_peak_bf16 * up_ratio
     up_s = stage_ms["expert_up"] / 1e3
     down_s = stage_ms["expert_down"] / 1e3
     up_tflops = work["up_flops"] / up_s / 1e12
+    down_tflops = work["down_flops"] / down_s / 1e12
     gemm_tflops = (work["up_flops"] + work["down_flops"]) / (up_s + down_s) / 1e12
-    scat_gbs = None
     stages = {k: round(v, 4) for k, v in stage_ms.items()}
     hbm = peaks["hbm_gbs"]
     comb_gbs = work["combine_bytes"] / (stage_ms["combine"] / 1e3) / 1e9
@@ -660,22 +720,25 @@ def run_gpu(args, w) -> dict:
                    if w.fp8 else "grouped GEMM gate/up (moe_expert_up, tcgen05)")
     tensor_line = {"achieved": up_tflops, "peak": up_peak, "unit": "TFLOP/s",
                    "frac": up_tflops / up_peak,
-                   "peak_source": (peaks["source"] + " bf16 sustained x 2 (the nominal "
-                                   "e4m3/bf16 dense ratio)" if w.fp8
-                                   else peaks["source"] + " bf16 sustained"),
-                   "frac_of_burst": up_tflops / (peaks["bf16_tflops"] * up_ratio)}
+                   "peak_source": (peaks["source"] + " " + up_peak_name +
+                                   (" x 2 (the nominal e4m3/bf16 dense ratio)" if w.fp8 else "")),
+                   "frac_of_burst": up_tflops / (peaks["bf16_tflops"] * up_ratio),
+                   "frac_of_sustained": up_tflops / (peaks["bf16_tflops_sustained"] * up_ratio)}
     hbm_line = {"achieved": up_gbs, "peak": hbm, "unit": "GB/s", "frac": up_gbs / hbm,
                 "peak_source": peaks["source"] + " copy bandwidth"}
     roofline = {"kernel": kernel_name, "bound": "tensor" if intensity >= balance else "hbm"}
     roofline.update(tensor_line if intensity >= balance else hbm_line)
     roofline.update({"traffic": up_traffic(w.name),
+                     "launches_per_step": L,
                      "algorithmic_flops_per_launch": work["up_flops"] / L,
                      "algorithmic_bytes_per_launch": work["up_bytes"] / L,
+                     "mean_launch_ms": stage_ms["expert_up"] / L,
                      "flops_per_byte": intensity, "machine_balance": balance,
                      "other_bound": ({"unit": "GB/s", "achieved": up_gbs, "frac": up_gbs / hbm}
                                      if intensity >= balance else
                                      {"unit": "TFLOP/s", "achieved": up_tflops,
                                       "frac": up_tflops / up_peak})})
+    ms_step = agg["elapsed_max_s"] / args.steps * 1e3
     res = {
         "metric": METRIC,
         "value": agg["value"],
@@ -683,27 +746,32 @@ def run_gpu(args, w) -> dict:
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": agg["elapsed_max_s"] / args.steps * 1e3,
+        "ms_per_step": ms_step,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": (("e4m3 (dispatch payload, both expert GEMMs' operands and the return "
                    "payload), fp32 accumulate" if w.fp8_return else
                    "e4m3 (dispatch payload and both expert GEMMs' operands), fp32 accumulate")
-                  if w.fp8 else "bf16"),
+                  if w.fp8 else "bf16 (x, W1, W3), fp16 (h, W2), fp32 accumulate"),
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",
         "config": {"workload": w.name, "N": N, "d": d, "f": f, "E": E, "K": K, "W": W,
                    "shared_f": w.shared_f,
                    "capacity_factor": w.cf if w.cf > 0 else "dropless", "zipf_s": w.s,
                    "rows_kept": R_layers if L > 1 else R, "layers": L,
+                   "step": (f"the {L}-layer stack, x_(l+1) = bf16(x_l + MoE_l(x_l))" if L > 1
+                            else "one layer"),
                    "output": "bf16 [N][d], the fp32 sum rounded once",
                    "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {3 * E * d * f * 2 / 1e9:.2f} GB of expert "
-                         "weights streamed per step"},
+                   "l2": f"inputs larger than L2: {L * 3 * E * d * f * 2 / 1e9:.2f} GB of expert "
+                         "weights streamed per step, no flush"},
+        "per_layer": {"layer_tokens_per_s": agg["value"] * L, "ms_per_layer": ms_step / L},
         "roofline": roofline,
         "stages_ms": stages,
-        "grouped_gemm": {"tflops": gemm_tflops, "frac_of_bf16_peak": gemm_tflops / peaks["bf16_tflops"],
+        "grouped_gemm": {"tflops": gemm_tflops, "gate_up_tflops": up_tflops,
+                         "down_tflops": down_tflops,
+                         "frac_of_bf16_burst": gemm_tflops / peaks["bf16_tflops"],
                          "frac_of_bf16_sustained": gemm_tflops / peaks["bf16_tflops_sustained"]},
         "combine": {"gbs": comb_gbs, "frac_of_hbm": comb_gbs / hbm, "frac_of_8tbs": comb_gbs / 8000.0},
         "shared_expert": ({"ms": stage_ms["shared_expert"],
@@ -716,15 +784,18 @@ def run_gpu(args, w) -> dict:
                      "gbs": work["scatter_bytes"] / (stage_ms["dispatch"] / 1e3) / 1e9,
                      "frac_of_hbm": work["scatter_bytes"] / (stage_ms["dispatch"] / 1e3) / 1e9
                      / hbm},
+        "route": {"ms": stage_ms["route"],
+                  "tflops_fp32": 2.0 * N * d * E * L / (stage_ms["route"] / 1e3) / 1e12},
+        "grid": grid_res or None,
         "routing": routing,
-        "clocks": clocks.summary(),
-        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clock_summary,
+        "gpu_launches": (L * kernel_launches(w) + (L - 1)) * args.steps,
         "graph": graph_res,
         "device_error": err,
         "e2e": e2e,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_sample_tokens,
+        res["cpu_baseline"] = cpu_baseline(w, layers, args.cpu_sample_tokens,
                                            sh if shared else None)
     return res if rank == 0 else None
 
@@ -744,47 +815,70 @@ def load_peaks() -> dict:
 
 # --------------------------------------------------------------------------- CPU oracle legs
 
-def oracle_time(w, inp_cpu, sample_tokens: int, shared_cpu=None) -> dict:
-    """Times the oracle on a bounded sample: routing + dispatch for every token,
-    expert FFN + combine (and the shared dense MLP, for a Residual-MoE layer) for
-    `sample_tokens` tokens; extrapolates to the layer."""
+def sample_size(w, seconds: float, cores: int) -> int:
+    """Tokens of a sample the oracle finishes in about `seconds` on `cores` host cores, from
+    its work per token (the router's 2*d*E fp32 multiply-adds at about 0.7 GFLOP/s and the
+    experts' K*6*d*f fp64 flops at about 2 GFLOP/s per core, measured on this oracle), every
+    layer of a stack; a multiple of W, at least W, at most N."""
+    per_core_s = w.layers * (2.0 * w.d * w.E / 0.7e9 + w.K * 6.0 * w.d * (w.f + w.shared_f)
+                             / 2.0e9)
+    S = int(seconds * max(cores, 1) / per_core_s)
+    return max(w.W, min(w.N, (S // w.W) * w.W))
+
+
+def slice_inputs(w, layers_cpu: list, S: int) -> tuple:
+    """The first S tokens of the workload's batch (S a multiple of W) and its weights: the
+    bounded sample the oracle is timed on. The capacity is the same factor of the smaller
+    batch (C = ceil(cf * S * K / E))."""
+    S = max(w.W, (min(S, w.N) // w.W) * w.W)
+    return w.with_(N=S), layers_cpu[0]["x"][:S].contiguous()
+
+
+def oracle_step(ws, layers_cpu: list, x, shared_cpu=None):
+    """One step of the oracle on the sample: the whole layer (route, dispatch, the experts,
+    combine) for every token of the sample, every layer of a stack in turn with
+    x_(l+1) = bf16(x_l + out_l). The FP8 workloads run on the operands quantised once outside
+    the timing (static weights), the token rows quantised inside it."""
     import numpy as np
+    import torch
+
+    import oracle
+    for l, lw in enumerate(layers_cpu):
+        inp = dict(lw, x=x)
+        if ws.fp8:
+            xq, sx = oracle.quantize_rows_e4m3(x)
+            as_bf16 = lambda u: torch.from_numpy(u.view(np.int16)).view(torch.bfloat16)
+            inp = dict(lw["deq"], x=as_bf16(oracle.dequantize_rows_bf16(xq, sx)),
+                       w_router=lw["w_router"], bias=lw["bias"])
+        r = oracle.layer(inp, ws.K, ws.W, ws.cf, order=int(ws.slot_major), reroute=ws.reroute)
+        out = r["out"]
+        if shared_cpu is not None:
+            out = out + oracle.shared_expert(x, shared_cpu["ws1"], shared_cpu["ws3"],
+                                             shared_cpu["ws2"])
+        if len(layers_cpu) > 1:
+            xf = oracle.bf16_bits_to_f64(oracle.as_u16(x))
+            x = torch.from_numpy(oracle.round_bf16(xf + out).view(np.int16)).view(torch.bfloat16)
+    return x
+
+
+def prepare_oracle_layers(w, layers: list) -> list:
+    """Host copies of every layer's inputs for the oracle; for the FP8 workloads also the
+    dequantised e4m3 weights (made once: the weights are static)."""
+    import numpy as np
+    import torch
 
     import oracle
     oracle.build()
-    exp_inp = inp_cpu
-    if w.fp8:  # the experts' W1, W3 quantised once, outside the timing (static weights)
-        import torch
-        as_bf16 = lambda u: torch.from_numpy(u.view(np.int16)).view(torch.bfloat16)
-        q1, s1 = oracle.quantize_rows_e4m3(inp_cpu["w1"])
-        q3, s3 = oracle.quantize_rows_e4m3(inp_cpu["w3"])
-        q2, s2 = oracle.quantize_rows_e4m3(inp_cpu["w2"])
-        exp_inp = dict(inp_cpu, w1=as_bf16(oracle.dequantize_rows_bf16(q1, s1)),
-                       w3=as_bf16(oracle.dequantize_rows_bf16(q3, s3)),
-                       w2=as_bf16(oracle.dequantize_rows_bf16(q2, s2)))
-    t0 = time.perf_counter()
-    r = oracle.route_and_dispatch(inp_cpu["x"], inp_cpu["w_router"], inp_cpu.get("bias"), w.K,
-                                  w.W, w.cf, order=int(w.slot_major), reroute=w.reroute)
-    if w.fp8:  # the FP8 payload: every token row quantised
-        xq, sx = oracle.quantize_rows_e4m3(inp_cpu["x"])
-        exp_inp = dict(exp_inp, x=as_bf16(oracle.dequantize_rows_bf16(xq, sx)))
-    t_route = time.perf_counter() - t0
-    rng = np.random.default_rng(0)
-    toks = np.sort(rng.choice(w.N, size=min(sample_tokens, w.N), replace=False))
-    t1 = time.perf_counter()
-    oracle.layer_sampled(exp_inp, w.K, w.W, w.cf, toks, routing=r)
-    if shared_cpu is not None:
-        oracle.shared_expert(inp_cpu["x"][torch_index(toks)], shared_cpu["ws1"], shared_cpu["ws3"],
-                             shared_cpu["ws2"])
-    t_exp = time.perf_counter() - t1
-    t_full = t_route + t_exp * (w.N / len(toks))
-    return dict(value=w.N / t_full, t_route_s=t_route, t_expert_sample_s=t_exp,
-                sample_tokens=int(len(toks)), extrapolated_layer_s=t_full)
-
-
-def torch_index(toks):
-    import torch
-    return torch.from_numpy(toks)
+    out = []
+    for lw in layers:
+        c = {k: (None if v is None else v.cpu()) for k, v in lw.items()
+             if k in ("x", "w_router", "bias", "w1", "w3", "w2")}
+        if w.fp8:
+            as_bf16 = lambda u: torch.from_numpy(u.view(np.int16)).view(torch.bfloat16)
+            c["deq"] = {k: as_bf16(oracle.dequantize_rows_bf16(*oracle.quantize_rows_e4m3(c[k])))
+                        for k in ("w1", "w3", "w2")}
+        out.append(c)
+    return out
 
 
 def cpu_threads() -> int:
@@ -792,52 +886,62 @@ def cpu_threads() -> int:
     return int(n) if n else (os.cpu_count() or 1)
 
 
-def cpu_baseline(w, inp, sample_tokens: int, shared=None) -> dict:
-    inp_cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
-    sh_cpu = None if shared is None else {k: v.cpu() for k, v in shared.items()}
-    t = oracle_time(w, inp_cpu, sample_tokens, sh_cpu)
-    stack = f"; one layer timed, x{w.layers} for the stack" if w.layers > 1 else ""
-    return {"value": t["value"] / w.layers, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"routing + dispatch for all {w.N} tokens; expert FFN + combine for "
-                      f"{t['sample_tokens']} tokens, extrapolated to {w.N} "
-                      f"(route {t['t_route_s']:.2f} s, experts {t['t_expert_sample_s']:.2f} s)"
-                      + stack}
+def cpu_baseline(w, layers, sample_tokens: int, shared=None) -> dict:
+    """The oracle as it stands, timed on the host cores on a bounded sample of the workload:
+    the first `sample_tokens` tokens through the whole layer (or stack); measured, not
+    extrapolated."""
+    lc = prepare_oracle_layers(w, layers)
+    sh = None if shared is None else {k: v.cpu() for k, v in shared.items()}
+    ws, x = slice_inputs(w, lc, sample_tokens or sample_size(w, 15.0, cpu_threads()))
+    t0 = time.perf_counter()
+    oracle_step(ws, lc, x, sh)
+    t = time.perf_counter() - t0
+    return {"value": ws.N / t, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "seconds": t,
+            "sample": f"the first {ws.N} of the {w.N} tokens through the whole "
+                      + (f"{w.layers}-layer stack" if w.layers > 1 else "layer")
+                      + " (route, dispatch, experts, combine; capacity ceil(cf*S*K/E)), "
+                        "measured"}
 
 
 def run_reference(args, w) -> dict:
-    import torch
-
     from moe_workloads import make_layer_inputs
     world, rank, _ = dist_env()
     if rank != 0:
         return None
-    inp = make_layer_inputs(w, seed=args.seed, device="cpu")
+    layers = [make_layer_inputs(w, seed=args.seed, device="cpu", layer=l, with_x=(l == 0))
+              for l in range(w.layers)]
     sh = None
     if w.shared_f > 0:
         from moe_workloads import make_shared_inputs
         sh = make_shared_inputs(w, seed=args.seed, device="cpu")
-    times, values = [], []
+    lc = prepare_oracle_layers(w, layers)
+    ws, x = slice_inputs(w, lc, args.ref_sample_tokens or sample_size(w, 1.0, cpu_threads()))
+    times = []
+    wall0 = time.perf_counter()
     for i in range(args.warmup + args.steps):
-        t = oracle_time(w, inp, args.ref_sample_tokens, sh)
+        t0 = time.perf_counter()
+        oracle_step(ws, lc, x, sh)
         if i >= args.warmup:
-            times.append(t["extrapolated_layer_s"] * w.layers)  # one layer timed, x layers
-            values.append(t["value"] / w.layers)
+            times.append(time.perf_counter() - t0)
     total = sum(times)
-    value = w.N * len(times) / total
+    value = ws.N * len(times) / total
+    sample = (f"each step: the first {ws.N} of the {w.N} tokens through the whole "
+              + (f"{w.layers}-layer stack" if w.layers > 1 else "layer")
+              + " (route, dispatch, experts, combine; capacity ceil(cf*S*K/E)), measured")
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "impl": "reference",
         "config": {"workload": w.name, "N": w.N, "d": w.d, "f": w.f, "E": w.E, "K": w.K,
-                   "W": w.W, "capacity_factor": w.cf if w.cf > 0 else "dropless"},
+                   "W": w.W, "capacity_factor": w.cf if w.cf > 0 else "dropless",
+                   "zipf_s": w.s, "layers": w.layers, "tokens_per_step": ws.N},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": f"each step: routing + dispatch for all {w.N} tokens, expert "
-                                   f"FFN + combine for {args.ref_sample_tokens} tokens, "
-                                   f"extrapolated to {w.N}"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - wall0,
     }
-    del torch
     return res
 
 
@@ -848,11 +952,16 @@ def parse(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mixtral_prefill")
+    ap.add_argument("--workload", default="stack4")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-sample-tokens", type=int, default=32)
-    ap.add_argument("--ref-sample-tokens", type=int, default=4)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=0,
+                    help="tokens of the cpu_baseline sample (0: about 15 s of oracle work)")
+    ap.add_argument("--ref-sample-tokens", type=int, default=0,
+                    help="tokens per step of the reference arm (0: about 1 s of oracle work)")
+    ap.add_argument("--grid-steps", type=int, default=10,
+                    help="timed steps per point of a stack's capacity-factor x skew grid")
+    ap.add_argument("--no-grid", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of replaying the step's CUDA graph")

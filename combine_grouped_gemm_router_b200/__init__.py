@@ -29,6 +29,7 @@ STATUS_NAMES = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_MISALIGNED", 5: "MOE_ERR_CUDA",
     6: "MOE_ERR_DEVICE_TIMEOUT", 7: "MOE_ERR_NONFINITE", 8: "MOE_ERR_DEVICE_BOUNDS",
+    9: "MOE_ERR_F16_RANGE",
 }
 
 
@@ -68,6 +69,7 @@ _sigs = {
     "moe_dispatch_reroute": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_dispatch_fp8": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_quantize_rows_e4m3": ([c_p, c_i64, c_i32, c_p, c_p, c_p, c_p], c_i32),
+    "moe_convert_bf16_to_f16": ([c_p, c_i64, c_p, c_p, c_p], c_i32),
     "moe_expert_up_fp8": ([_SP] + [c_p] * 9, c_i32),
     "moe_expert_down_fp8": ([_SP] + [c_p] * 7, c_i32),
     "moe_layer_fp8": ([_SP] + [c_p] * 14 + [c_size, c_p], c_i32),
@@ -92,7 +94,7 @@ _sigs = {
 }
 
 
-ABI_VERSION = 2  # MOE_ABI_VERSION the structures below match
+ABI_VERSION = 3  # MOE_ABI_VERSION the structures below match
 
 
 class _Lib:
@@ -158,13 +160,17 @@ MOE_FLAG_OUT_BF16 = 1
 MOE_FLAG_SLOT_MAJOR = 2
 MOE_FLAG_REROUTE = 4
 MOE_FLAG_FP8_RETURN = 8
+MOE_FLAG_H_BF16 = 16
 
 
 def make_shape(N: int, d: int, f: int, E: int, K: int, W: int, capacity_factor: float = 0.0,
                out_bf16: bool = False, slot_major: bool = False,
-               reroute: bool = False, fp8_return: bool = False) -> MoeShape:
+               reroute: bool = False, fp8_return: bool = False, h_bf16: bool = False) -> MoeShape:
+    """h_bf16: the SwiGLU activation h and the down-projection weights in bf16 instead of the
+    default fp16 (then W2 is passed as the bf16 weights, not their fp16 copy)."""
     flags = ((MOE_FLAG_OUT_BF16 if out_bf16 else 0) | (MOE_FLAG_SLOT_MAJOR if slot_major else 0)
-             | (MOE_FLAG_REROUTE if reroute else 0) | (MOE_FLAG_FP8_RETURN if fp8_return else 0))
+             | (MOE_FLAG_REROUTE if reroute else 0) | (MOE_FLAG_FP8_RETURN if fp8_return else 0)
+             | (MOE_FLAG_H_BF16 if h_bf16 else 0))
     return MoeShape(N, d, f, E, K, W, float(capacity_factor), flags)
 
 
@@ -258,6 +264,28 @@ def moe_quantize_rows_e4m3(src, codes, scale, rows_dev=None, stream=None):
     rows = src.numel() // cols
     _check(_lib.moe_quantize_rows_e4m3(_ptr(src), rows, cols, _ptr(codes), _ptr(scale),
                                        _ptr(rows_dev), _stream(stream)), "moe_quantize_rows_e4m3")
+
+
+def moe_convert_bf16_to_f16(src, dst, changed=None, stream=None):
+    """fp16 copy of a bf16 weight array (all elements; the down projection's W2 / Ws2);
+    changed (optional device int64 tensor of one element) accumulates the count of elements
+    whose value changed."""
+    n = src.numel()
+    if dst.numel() != n:
+        raise MoeError(1, "moe_convert_bf16_to_f16: src and dst sizes differ")
+    _check(_lib.moe_convert_bf16_to_f16(_ptr(src), n, _ptr(dst), _ptr(changed), _stream(stream)),
+           "moe_convert_bf16_to_f16")
+
+
+def w2_for(shape, w2, stream=None):
+    """The down-projection weights in the form `shape` asks for: the bf16 tensor itself with
+    h_bf16, else a new fp16 copy made by moe_convert_bf16_to_f16."""
+    if shape.flags & MOE_FLAG_H_BF16:
+        return w2
+    import torch
+    out = torch.empty(w2.shape, dtype=torch.float16, device=w2.device)
+    moe_convert_bf16_to_f16(w2, out, stream=stream)
+    return out
 
 
 def moe_expert_up_fp8(shape, x_sorted, sorted_scale, offsets, w1q, w1_scale, w3q, w3_scale, h,

@@ -739,4 +739,45 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// bf16 -> fp16 conversion of a weight matrix (the experts' W2 and the shared MLP's Ws2, which
+// the down projection reads as fp16 beside the fp16 h), eight elements per 16-byte load. Every
+// bf16 value whose magnitude lies in [2^-17, 65504] converts exactly (fp16 keeps 11
+// significant bits and reaches down to 2^-24 in steps of 2^-24); smaller ones round to the
+// nearest fp16 step, larger ones become infinite and record MOE_ERR_F16_RANGE. The number of
+// elements whose value changed is added to *changed (nullable). n % 8 == 0.
+__global__ void __launch_bounds__(256)
+    convert_bf16_f16_kernel(const uint16_t *__restrict__ src, int64_t n, uint16_t *__restrict__ dst,
+                            unsigned long long *__restrict__ changed)
+{
+    const int64_t nvec = n >> 3;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    unsigned long long cnt = 0;
+    bool over = false;
+    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
+        const uint4 a = reinterpret_cast<const uint4 *>(src)[v];
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float lo = bf16_lo(w[i]), hi = bf16_hi(w[i]);
+            uint32_t r;
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+            float blo, bhi;
+            asm("cvt.f32.f16 %0, %1;" : "=f"(blo) : "h"((unsigned short)(r & 0xFFFFu)));
+            asm("cvt.f32.f16 %0, %1;" : "=f"(bhi) : "h"((unsigned short)(r >> 16)));
+            cnt += (blo != lo) + (bhi != hi);
+            over |= (isinf(blo) && !isinf(lo)) || (isinf(bhi) && !isinf(hi));
+            o[i] = r;
+        }
+        reinterpret_cast<uint4 *>(dst)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (over)
+        set_dev_error(MOE_ERR_F16_RANGE);
+    if (changed) {
+        cnt = warp_sum(cnt);
+        if ((threadIdx.x & 31) == 0 && cnt)
+            atomicAdd(changed, cnt);
+    }
+}
+
 }  // namespace moe

@@ -23,9 +23,13 @@
 //    expert's rows or zero fill) but never stored.
 // Mode 0 (gate/up): the B tile stacks 128 rows of W1 and 128 rows of W3, one
 // N=256 MMA per K-step; the epilogue reads gate column c and up column 128+c
-// and writes h = silu(g) * u as bf16 (the next GEMM's operand). Mode 1 (down):
-// fp32 output straight from TMEM, so the combine sums unrounded expert outputs
-// (or the FP8 return payload: e4m3 codes with one exponent per 32 columns).
+// and writes h = silu(g) * u, the next GEMM's operand, as fp16 (or bf16 when
+// Args::h_f16 is 0): fp16's 11 significant bits against bf16's 8 make h's one
+// rounding 8x smaller, and every value the epilogue produces is checked
+// against fp16's range (65504). Mode 1 (down): h times W2 with both operands
+// fp16 (or both bf16), fp32 output straight from TMEM, so the combine sums
+// unrounded expert outputs (or the FP8 return payload: e4m3 codes with one
+// exponent per 32 columns).
 // Modes 2 and 3 (the FP8 path, [MoE 推理服务工程真相 2026, §6.3]): modes 0 and 1
 // with e4m3 A and B (tcgen05 kind::f8f6f4). A 128-byte swizzle atom then holds
 // 128 K elements instead of 64, so tiles, stages and descriptors keep their byte
@@ -71,6 +75,8 @@ struct Args {
     const float *row_scale;  // modes 2, 3: scale of each A row [rows_alloc]
     const float *b_scale0;   // mode 2: scale of each W1 row; mode 3: of each W2 row [E * b_rows]
     const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
+    int h_f16;               // modes 0, 1: h (mode 0's output, mode 1's A) and W2 are fp16,
+                             // else bf16
     uint64_t timeout_ns;
 };
 
@@ -194,6 +200,14 @@ __host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N)
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// Instruction descriptor, kind::f16: fp16 A and B (format code 0), fp32 accumulate.
+__host__ __device__ constexpr uint32_t instr_desc_f16(int M, int N)
+{
+    return (1u << 4)                          // D format: f32
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
 // Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), fp32 accumulate.
 __host__ __device__ constexpr uint32_t instr_desc_e4m3(int M, int N)
 {
@@ -206,6 +220,28 @@ template <int MODE>
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N)
 {
     return is_e4m3(MODE) ? instr_desc_e4m3(M, N) : instr_desc_bf16(M, N);
+}
+
+// The descriptor a launch uses: the down projection (mode 1) reads fp16 h and W2 when the
+// launch says so; every other case is fixed by the mode.
+template <int MODE>
+__device__ __forceinline__ uint32_t launch_idesc(const Args &args, int M, int N)
+{
+    return (MODE == 1 && args.h_f16) ? instr_desc_f16(M, N) : instr_desc<MODE>(M, N);
+}
+
+// Two fp32 -> one f16x2 word (round to nearest even; beyond 65504 becomes infinity).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Nonzero when either half of an f16x2 word is infinite or NaN (all exponent bits set).
+__device__ __forceinline__ uint32_t f16x2_nonfinite(uint32_t p)
+{
+    return ((p & 0x7C00u) == 0x7C00u) | ((p & 0x7C000000u) == 0x7C000000u);
 }
 
 // One MMA of 32 bytes of K (16 bf16 or 32 e4m3 elements).
@@ -388,10 +424,22 @@ __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr
                 }
             }
             uint32_t p[CB / 2];
+            if (MODE == 0 && args.h_f16) {
+                uint32_t bad = 0;
 #pragma unroll
-            for (int j = 0; j < CB / 2; ++j)
-                p[j] = pack_bf16x2(silu_mul(gf[2 * j], uf[2 * j]),
-                                   silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
+                for (int j = 0; j < CB / 2; ++j) {
+                    p[j] = pack_f16x2(silu_mul(gf[2 * j], uf[2 * j]),
+                                      silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
+                    bad |= f16x2_nonfinite(p[j]);
+                }
+                if (bad)  // a value of h outside fp16's range (or not finite)
+                    set_dev_error(MOE_ERR_F16_RANGE);
+            } else {
+#pragma unroll
+                for (int j = 0; j < CB / 2; ++j)
+                    p[j] = pack_bf16x2(silu_mul(gf[2 * j], uf[2 * j]),
+                                       silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
+            }
 #pragma unroll
             for (int j = 0; j < CB / 8; ++j)
                 dst[c / 8 + j] = make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
@@ -544,7 +592,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int KX = atom_k(MODE);
     constexpr int B_BYTES = BN * BK * 2;
     constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    constexpr uint32_t IDESC = instr_desc<MODE>(BM, BN);
+    const uint32_t IDESC = launch_idesc<MODE>(args, BM, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -854,7 +902,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int BN = 256;
     constexpr bool GATE = is_gate(MODE);
     constexpr int KX = atom_k(MODE);
-    constexpr uint32_t IDESC = instr_desc<MODE>(BMP, BN);
+    const uint32_t IDESC = launch_idesc<MODE>(args, BMP, BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(

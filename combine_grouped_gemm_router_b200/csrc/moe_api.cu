@@ -74,7 +74,7 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
     if (!s)
         return MOE_ERR_INVALID_ARG;
     if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE |
-                                MOE_FLAG_FP8_RETURN)) != 0)
+                                MOE_FLAG_FP8_RETURN | MOE_FLAG_H_BF16)) != 0)
         return MOE_ERR_INVALID_ARG;
     if (s->N < 0 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
         return MOE_ERR_INVALID_ARG;
@@ -466,20 +466,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// 2-D tensor [rows][inner] of bf16 (or e4m3 bytes), box 128 rows x one 128-byte swizzle
-// atom (64 bf16 or 128 e4m3 elements), 128-byte swizzle.
-bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, bool e4m3 = false)
+// 2-D tensor [rows][inner] of bf16 (or fp16, or e4m3 bytes), box 128 rows x one 128-byte
+// swizzle atom (64 bf16 / fp16 or 128 e4m3 elements), 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, bool e4m3 = false,
+               bool f16 = false)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
     const uint64_t esize = e4m3 ? 1 : 2;
+    const CUtensorMapDataType dt = e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {inner * esize};
     cuuint32_t box[2] = {(cuuint32_t)(128 / esize), 128};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                     const_cast<void *>(ptr), dims, strides, box, estr,
+    CUresult r = enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -573,10 +576,11 @@ bool use_pair_tiles(const moe_shape_t *s, const Geometry &g)
 }
 
 // Grouped GEMM launches for E experts of width f over an A buffer of a_rows rows (the
-// tensor map's extent: rows past it read as zeros). `pair` selects the CTA-pair kernel.
+// tensor map's extent: rows past it read as zeros). `pair` selects the CTA-pair kernel;
+// `f16`: h is written (gate/up) or read together with fp16 W2 (down) as fp16, else bf16.
 moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *a,
                      const int32_t *offsets, const uint16_t *w1, const uint16_t *w3, uint16_t *h,
-                     cudaStream_t st)
+                     bool f16, cudaStream_t st)
 {
     CUtensorMap tA, tW1, tW3;
     if (!make_tmap(&tA, a, d, (uint64_t)a_rows) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
@@ -591,6 +595,7 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
     args.rows_alloc = (int)a_rows;
     args.out = h;
     args.ldo = f;
+    args.h_f16 = f16 ? 1 : 0;
     args.timeout_ns = kWaitTimeoutNs;
     args.select = 0;
     if (pair) {
@@ -607,10 +612,11 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
 // the y tensor map, unused then, is a copy of the W2 map).
 moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
                        const int32_t *offsets, const uint16_t *w2, void *y, int y_stride,
-                       cudaStream_t st)
+                       bool f16, cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
-    if (!make_tmap(&tA, h, f, (uint64_t)a_rows) || !make_tmap(&tW2, w2, f, (uint64_t)E * d))
+    if (!make_tmap(&tA, h, f, (uint64_t)a_rows, false, f16) ||
+        !make_tmap(&tW2, w2, f, (uint64_t)E * d, false, f16))
         return MOE_ERR_CUDA;
     if (y_stride > 0)
         tY = tW2;
@@ -625,6 +631,7 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     args.out = y;
     args.ldo = d;
     args.y_stride = y_stride;
+    args.h_f16 = f16 ? 1 : 0;
     args.timeout_ns = kWaitTimeoutNs;
     args.select = 0;
     if (d % 256 == 0) {
@@ -731,12 +738,15 @@ moe_status_t quantize_rows_launch(const uint16_t *src, int64_t rows, int cols, u
     return launch_status();
 }
 
+// h and the down-projection weights are fp16 unless the shape asks for bf16.
+inline bool h_is_f16(const moe_shape_t *s) { return !(s->flags & MOE_FLAG_H_BF16); }
+
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                             uint16_t *h, cudaStream_t st)
 {
     return gemm_up(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), x_sorted, offsets, w1,
-                   w3, h, st);
+                   w3, h, h_is_f16(s), st);
 }
 
 moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *h,
@@ -744,7 +754,7 @@ moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uin
                               cudaStream_t st)
 {
     return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y,
-                     y_payload_stride(s), st);
+                     y_payload_stride(s), h_is_f16(s), st);
 }
 
 moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
@@ -770,10 +780,11 @@ moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x
 {
     whole_range_offsets_kernel<<<1, 1, 0, st>>>(offsets2, s->N);
     const bool pair = s->N >= 768;
-    moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, st);
+    moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, h_is_f16(s),
+                              st);
     if (rc != MOE_OK)
         return rc;
-    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, st);
+    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, h_is_f16(s), st);
 }
 
 moe_status_t combine_impl(const moe_shape_t *s, const void *y, const int32_t *row_of,
@@ -849,6 +860,7 @@ __attribute__((visibility("default"))) const char *moe_status_string(moe_status_
     case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
     case MOE_ERR_NONFINITE: return "MOE_ERR_NONFINITE";
     case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS";
+    case MOE_ERR_F16_RANGE: return "MOE_ERR_F16_RANGE";
     }
     return "MOE_ERR_UNKNOWN";
 }
@@ -1037,6 +1049,27 @@ moe_quantize_rows_e4m3(const uint16_t *src, int64_t rows, int32_t cols, uint8_t 
         return MOE_OK;
     return quantize_rows_launch(src, rows, cols, codes, scale, rows_dev,
                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_convert_bf16_to_f16(const uint16_t *src, int64_t n, uint16_t *dst, int64_t *changed,
+                        moe_stream_t stream)
+{
+    if (n < 0 || (n > 0 && (!src || !dst)))
+        return MOE_ERR_INVALID_ARG;
+    if (n % 8 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if ((n > 0 && (!aligned16(src) || !aligned16(dst))) ||
+        (changed && (reinterpret_cast<uintptr_t>(changed) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    if (n == 0)
+        return MOE_OK;
+    const int64_t vec = n / 8;
+    const int64_t blocks64 = (vec + 255) / 256;
+    const int blocks = (int)(blocks64 < 64LL * num_sms() ? blocks64 : 64LL * num_sms());
+    convert_bf16_f16_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        src, n, dst, reinterpret_cast<unsigned long long *>(changed));
+    return launch_status();
 }
 
 __attribute__((visibility("default"))) moe_status_t

@@ -42,7 +42,7 @@ extern "C" {
 struct CUstream_st;
 typedef struct CUstream_st *moe_stream_t; /* identical to cudaStream_t */
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef enum moe_status {
     MOE_OK = 0,
@@ -53,7 +53,9 @@ typedef enum moe_status {
     MOE_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
     MOE_ERR_DEVICE_TIMEOUT = 6,      /* a bounded device-side wait gave up */
     MOE_ERR_NONFINITE = 7,           /* a router logit was NaN or infinite */
-    MOE_ERR_DEVICE_BOUNDS = 8        /* an expert id outside [0, E) reached a kernel */
+    MOE_ERR_DEVICE_BOUNDS = 8,       /* an expert id outside [0, E) reached a kernel */
+    MOE_ERR_F16_RANGE = 9            /* a value of h (or of a weight converted to fp16) beyond
+                                        fp16's largest finite value 65504, or not finite */
 } moe_status_t;
 
 /* Problem description. Limits: 0 <= N, N*K < 2^31; d % 8 == 0 (d % 128 == 0 for
@@ -111,6 +113,21 @@ typedef struct moe_shape {
  * does not). The values quantised are the fp32 y the plain down GEMM writes; the combine
  * decodes them exactly and accumulates in fp32 as before. Needs d % 128 == 0. */
 #define MOE_FLAG_FP8_RETURN 8u
+
+/* Precision of the SwiGLU activation h, the down projection's tensor-core operand.
+ * Default (flag clear): h is stored as fp16 and the down projection reads fp16 weights (W2 of
+ * moe_expert_down / moe_expert_gemm / moe_layer / moe_layer_shared, Ws2 of moe_shared_expert
+ * and moe_layer_shared), converted once from the bf16 weights by moe_convert_bf16_to_f16. One
+ * tensor-core MMA takes A and B of one type, so h and W2 share it. Why fp16: h is rounded once
+ * (after fp32 accumulation and the SwiGLU in fp32) and that rounding is the largest error of the
+ * layer; fp16 keeps 11 significant bits, bf16 8, so the error is 8 times smaller (on the
+ * 128-expert layer with drops, max |error| / RMS(output) 0.0045 instead of 0.031; the bound
+ * asked of the layer is 0.02). The price is fp16's range: a value of h beyond 65504 is stored
+ * as infinity and sets MOE_ERR_F16_RANGE in the device error word (rerun that layer with this
+ * flag). With MOE_FLAG_H_BF16: h is bf16 and W2 / Ws2 are the bf16 weights themselves.
+ * The FP8 path (moe_expert_up_fp8, moe_layer_fp8) keeps its bf16 h before the e4m3
+ * quantisation and ignores this flag. */
+#define MOE_FLAG_H_BF16 16u
 
 /* Per-call dispatch counters, written (not accumulated) by moe_dispatch / moe_layer into
  * DEVICE memory when a non-null pointer is given. Observability signals of
@@ -261,13 +278,14 @@ moe_status_t moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x,
  *  variable per-expert token counts) and §容量因子、专家复制与 dropless 的取舍 (dropless
  *  grouped GEMM in a single call)]
  * For every expert e and every row r in [offsets[e], offsets[e+1]):
- *   h[r] = silu(x_sorted[r] W1[e]^T) * (x_sorted[r] W3[e]^T)   (bf16 out, fp32 accumulate)
+ *   h[r] = silu(x_sorted[r] W1[e]^T) * (x_sorted[r] W3[e]^T)   (fp16 out, fp32 accumulate)
  *   y[r] = h[r] W2[e]^T                                         (fp32 out, fp32 accumulate)
- * x_sorted [rows_alloc][d], w1, w3 [E][f][d], w2 [E][d][f], h [rows_alloc][f] bf16;
- * y [rows_alloc][d] fp32 (the FP8 return payload with MOE_FLAG_FP8_RETURN, moe_y_bytes);
- * offsets [E+1] device int32 (as written by moe_dispatch).
- * h is bf16 because it is the second GEMM's tensor-core operand; y stays fp32 so the
- * combine adds unrounded expert outputs (unless the flag asks for the FP8 payload).
+ * x_sorted [rows_alloc][d], w1, w3 [E][f][d] bf16; w2 [E][d][f] and h [rows_alloc][f] fp16
+ * (both bf16 with MOE_FLAG_H_BF16; see there); y [rows_alloc][d] fp32 (the FP8 return payload
+ * with MOE_FLAG_FP8_RETURN, moe_y_bytes); offsets [E+1] device int32 (as written by
+ * moe_dispatch). h is rounded once because it is the second GEMM's tensor-core operand; y
+ * stays fp32 so the combine adds unrounded expert outputs (unless the flag asks for the FP8
+ * payload).
  * Rows past offsets[E] are neither read for output nor written. Experts with no rows cost
  * nothing (their weights are not read). Needs d % 128 == 0, f % 128 == 0. */
 moe_status_t moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted,
@@ -275,13 +293,23 @@ moe_status_t moe_expert_gemm(const moe_shape_t *shape, const uint16_t *x_sorted,
                              const uint16_t *w2, uint16_t *h, void *y, moe_stream_t stream);
 
 /* The two halves of moe_expert_gemm as separate launches (same contracts as above):
- * moe_expert_up:   h = silu(x_sorted W1^T) * (x_sorted W3^T)   (gate/up GEMM, bf16 h)
+ * moe_expert_up:   h = silu(x_sorted W1^T) * (x_sorted W3^T)   (gate/up GEMM, fp16 h)
  * moe_expert_down: y = h W2^T                     (down GEMM, fp32 y or the FP8 payload) */
 moe_status_t moe_expert_up(const moe_shape_t *shape, const uint16_t *x_sorted,
                            const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                            uint16_t *h, moe_stream_t stream);
 moe_status_t moe_expert_down(const moe_shape_t *shape, const uint16_t *h, const int32_t *offsets,
                              const uint16_t *w2, void *y, moe_stream_t stream);
+
+/* bf16 -> fp16 copy of a weight array for the down projection (W2 [E][d][f], Ws2 [d][f_shared]),
+ * made once when the weights are loaded. src, dst: DEVICE, n elements each, 16-byte aligned,
+ * n % 8 == 0; dst may not overlap src. Each value is converted to the nearest fp16 (ties to
+ * even): exact for magnitudes in [2^-17, 65504] (all but ~0.03 % of N(0, 0.02) weights, the
+ * rest move by less than 2^-25); a magnitude above 65504 becomes infinite and sets
+ * MOE_ERR_F16_RANGE. changed (DEVICE int64, nullable): the number of elements whose value
+ * changed is ADDED to it. Not a step of the pages' method: a storage format of the weights. */
+moe_status_t moe_convert_bf16_to_f16(const uint16_t *src, int64_t n, uint16_t *dst,
+                                     int64_t *changed, moe_stream_t stream);
 
 /* ---- FP8 payload ("MoE 推理服务工程真相 2026", §6.3: send the token data of the all-to-all
  * as FP8 instead of BF16, half the bytes, at the cost of quantisation noise).
@@ -353,8 +381,9 @@ moe_status_t moe_combine(const moe_shape_t *shape, const void *y, const int32_t 
  * (one "expert" that owns all N rows of x).
  * [MoE Inference Communication, §DeepSpeed-MoE › PR-MoE, 现象二 / Residual: a dense MLP every
  *  token passes through, added to the output of the routed expert(s)]
- * Same SwiGLU form as the experts: h_s = silu(x Ws1^T) * (x Ws3^T) (bf16), y_s = h_s Ws2^T (fp32).
- * x [N][d]; ws1, ws3 [f_shared][d]; ws2 [d][f_shared]; h_s [N][f_shared]; y_s [N][d] fp32.
+ * Same SwiGLU form as the experts: h_s = silu(x Ws1^T) * (x Ws3^T), y_s = h_s Ws2^T (fp32).
+ * x [N][d], ws1, ws3 [f_shared][d] bf16; ws2 [d][f_shared] and h_s [N][f_shared] fp16 (bf16
+ * with MOE_FLAG_H_BF16); y_s [N][d] fp32.
  * f_shared % 128 == 0. ws: at least 256 bytes of device scratch. */
 moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
                                const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2,
@@ -362,7 +391,9 @@ moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const
                                moe_stream_t stream);
 
 /* Residual-MoE layer: moe_layer's routed path plus the shared dense MLP, the two outputs
- * added in the combine (then the optional residual). Workspace: moe_layer_shared_workspace_size. */
+ * added in the combine (then the optional residual). Workspace: moe_layer_shared_workspace_size.
+ * w2 and ws2 fp16 (bf16 with MOE_FLAG_H_BF16), the other weights bf16.
+ * [MoE Inference Communication, §DeepSpeed-MoE › PR-MoE, Residual-MoE] */
 size_t moe_layer_shared_workspace_size(const moe_shape_t *shape, int32_t f_shared);
 moe_status_t moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
                               const float *w_router, const float *bias, const uint16_t *w1,
@@ -373,6 +404,10 @@ moe_status_t moe_layer_shared(const moe_shape_t *shape, int32_t f_shared, const 
 
 /* The whole layer: moe_route -> moe_dispatch (with the packed buffer) -> moe_expert_gemm ->
  * moe_combine, every intermediate in the workspace (moe_layer_workspace_size bytes).
+ * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制: its flowchart (route
+ *  Top-K, pack by destination, group by expert, grouped GEMM, weighted merge into the original
+ *  token order), the two exchanges emulated for W ranks inside this GPU's memory]
+ * w1, w3 bf16 [E][f][d]; w2 fp16 [E][d][f] (bf16 with MOE_FLAG_H_BF16).
  * residual (nullable) is added in the combine (pass x for x + MoE(x)); out [N][d] is fp32,
  * or bf16 with MOE_FLAG_OUT_BF16, and must not alias x. topk_idx_out [N][K] (nullable)
  * receives the routing; stats (nullable, DEVICE) the counters. */

@@ -13,11 +13,12 @@ def lib():
     return m
 
 
-def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
-    """route -> dispatch -> expert GEMMs -> combine, each through its C entry point."""
+def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda", h_bf16: bool = False) -> dict:
+    """route -> dispatch -> expert GEMMs -> combine, each through its C entry point. h and the
+    down-projection weights are fp16 (the library's default) unless h_bf16."""
     m = lib()
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
-                         reroute=w.reroute)
+                         reroute=w.reroute, h_bf16=h_bf16)
     dev = torch.device(device)
     x = inp["x"].to(dev)
     wr = inp["w_router"].to(dev)
@@ -54,23 +55,25 @@ def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda") -> dict:
                x_packed=x_packed, D=D, pk_off=pk_off, stats_buf=stats, rows_alloc=RA,
                expert_of=expert_of)
     if w.d % 128 == 0 and w.f % 128 == 0:
-        h = torch.zeros(RA, f, dtype=torch.bfloat16, device=dev)
+        h = torch.zeros(RA, f, dtype=torch.bfloat16 if h_bf16 else torch.float16, device=dev)
         y = torch.zeros(RA, d, dtype=torch.float32, device=dev)
+        w2 = m.w2_for(shape, inp["w2"].to(dev))
         m.moe_expert_gemm(shape, x_sorted, offsets, inp["w1"].to(dev), inp["w3"].to(dev),
-                          inp["w2"].to(dev), h, y)
+                          w2, h, y)
         out = torch.empty(N, d, dtype=torch.float32, device=dev)
         m.moe_combine(shape, y, row_of, topk_w, out)
-        res.update(h=h, y=y, out=out)
+        res.update(h=h, y=y, out=out, w2_used=w2)
     torch.cuda.synchronize()
     res["stats"] = m.stats_dict(m.read_stats(stats))
     res["dev_error"] = m.moe_get_device_error(True)
     return res
 
 
-def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True) -> dict:
+def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True,
+              h_bf16: bool = False) -> dict:
     m = lib()
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
-                         reroute=w.reroute)
+                         reroute=w.reroute, h_bf16=h_bf16)
     dev = torch.device(device)
     ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
     out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
@@ -78,7 +81,8 @@ def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True) -> di
     stats = m.stats_buffer(dev) if with_stats else None
     bias = None if inp["bias"] is None else inp["bias"].to(dev)
     m.moe_layer(shape, inp["x"].to(dev), inp["w_router"].to(dev), bias, inp["w1"].to(dev),
-                inp["w3"].to(dev), inp["w2"].to(dev), out, topk_idx_out=topk, stats=stats, ws=ws)
+                inp["w3"].to(dev), m.w2_for(shape, inp["w2"].to(dev)), out, topk_idx_out=topk,
+                stats=stats, ws=ws)
     torch.cuda.synchronize()
     res = dict(out=out, topk_idx=topk, ws=ws)
     if with_stats:
@@ -120,6 +124,26 @@ def assert_rounded_bf16(got, ref, what: str = ""):
     assert tolerance_report(g, r)["rel_frob"] <= REL_FROB, what
 
 
+def assert_rounded_f16(got, ref, what: str = ""):
+    """An intermediate stored as fp16: each element within twice fp16's rounding (2^-10
+    relative; 11 significant bits) of the reference, plus half the subnormal step (2^-25) and
+    a slack of 1e-5 * RMS for the fp32 accumulation and the SwiGLU's fp32 arithmetic."""
+    g = f64(got)
+    r = f64(ref)
+    rms = np.sqrt(np.mean(r * r))
+    excess = np.abs(g - r) - (2.0 ** -10 * np.abs(r) + 2.0 ** -25 + 1e-5 * rms)
+    assert excess.max() <= 0, (what, float(excess.max() / rms))
+    assert tolerance_report(g, r)["rel_frob"] <= REL_FROB, what
+
+
+def assert_rounded_h(got, ref, what: str = ""):
+    """h as the GPU stores it: fp16 by default, bf16 with the h_bf16 flag."""
+    if got.dtype == torch.float16:
+        assert_rounded_f16(got, ref, what)
+    else:
+        assert_rounded_bf16(got, ref, what)
+
+
 def bf16_h_bound_rows(h_ref: np.ndarray, w2_f64: np.ndarray, row_expert: np.ndarray) -> np.ndarray:
     """Per-element bound on |y_gpu - y_ref| implied by the arithmetic: h is rounded once
     to bf16 (relative error <= 2^-8) before the down projection, which accumulates in
@@ -130,6 +154,33 @@ def bf16_h_bound_rows(h_ref: np.ndarray, w2_f64: np.ndarray, row_expert: np.ndar
         sel = row_expert == e
         bound[sel] = np.abs(h_ref[sel]) @ np.abs(w2_f64[e]).T
     return bound * (2.0 ** -8 + f * 2.0 ** -23) + 1e-30
+
+
+def f16_h_bound_rows(h_ref: np.ndarray, w2_f64: np.ndarray, w2_used_f64: np.ndarray,
+                     row_expert: np.ndarray) -> np.ndarray:
+    """The same bound for the default precision: h rounded once to fp16 (relative error
+    <= 2^-11, bounded by 2^-10; absolute error <= 2^-25 where h is subnormal) and the fp16 copy
+    of W2 (w2_used_f64, the weights the GPU multiplied; it differs from W2 only where a bf16
+    weight is not an fp16 value): |dy_i| <= (2^-10 + f*2^-23) * sum_j |h_j W2[i][j]|
+    + 2^-25 * sum_j |W2[i][j]| + sum_j |h_j| |W2_used[i][j] - W2[i][j]| (+ tiny)."""
+    f = h_ref.shape[1]
+    bound = np.empty((h_ref.shape[0], w2_f64.shape[1]))
+    for e in np.unique(row_expert):
+        sel = row_expert == e
+        ah = np.abs(h_ref[sel])
+        a2 = np.abs(w2_f64[e])
+        bound[sel] = ((2.0 ** -10 + f * 2.0 ** -23) * (ah @ a2.T) + 2.0 ** -25 * a2.sum(1)[None]
+                      + ah @ np.abs(w2_used_f64[e] - w2_f64[e]).T)
+    return bound + 1e-30
+
+
+def h_bound_rows(h_ref, inp_w2, got_w2_used, row_expert) -> np.ndarray:
+    """The per-element y bound for the precision the run used (fp16 h unless the run kept W2
+    in bf16)."""
+    w2 = f64(inp_w2)
+    if got_w2_used is None or got_w2_used.dtype == torch.bfloat16:
+        return bf16_h_bound_rows(h_ref, w2, row_expert)
+    return f16_h_bound_rows(h_ref, w2, f64(got_w2_used), row_expert)
 
 
 def assert_within_bound(got, ref, bound, what: str = ""):

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(m):
 
 
 def test_abi_version_and_status_strings(m):
-    assert m.moe_abi_version() == 2
+    assert m.moe_abi_version() == 3
     for code, name in m.STATUS_NAMES.items():
         assert m.moe_status_string(code) == name
     assert m.moe_status_string(99) == "MOE_ERR_UNKNOWN"
@@ -68,7 +68,7 @@ def test_shape_validation(m):
         assert m.moe_rows_alloc(s) == -1
         assert m.moe_workspace_size(s) == 0
     flags = m.make_shape(64, 128, 256, 8, 2, 4)
-    flags.flags = 16  # no such flag
+    flags.flags = 1 << 10  # no such flag
     assert m.moe_workspace_size(flags) == 0
     # an empty batch is a valid shape
     assert m.moe_workspace_size(m.make_shape(0, 128, 256, 8, 2, 4)) > 0
@@ -156,6 +156,17 @@ def test_argument_errors_return_before_launch(m):
     assert lib.moe_affinity_accumulate(10, 8, 9, P, P, P, None) == 1
     assert lib.moe_affinity_accumulate(10, 300, 2, P, P, P, None) == 2
     assert lib.moe_debug_bounded_wait(0, None) == 1
+    # the fp16 copy of the down-projection weights
+    assert lib.moe_convert_bf16_to_f16(P, 12, P, None, None) == 2   # n % 8
+    assert lib.moe_convert_bf16_to_f16(None, 16, P, None, None) == 1
+    assert lib.moe_convert_bf16_to_f16(P, -8, P, None, None) == 1
+    assert lib.moe_convert_bf16_to_f16(P + 2, 16, P, None, None) == 4
+    assert lib.moe_convert_bf16_to_f16(P, 16, P, P + 4, None) == 4   # counter alignment
+    assert lib.moe_convert_bf16_to_f16(None, 0, None, None, None) == 0  # nothing to do
+    assert m.moe_status_string(9) == "MOE_ERR_F16_RANGE"
+    # every flag bit the header defines is accepted; the bf16 h flag among them
+    assert m.moe_layer_workspace_size(m.make_shape(64, 128, 256, 8, 2, 4, h_bf16=True)) == \
+        m.moe_layer_workspace_size(s)
 
 
 def test_derive_report_matches_oracle(m, orc):

@@ -101,7 +101,11 @@ def test_traffic_gate_ignores_comments_only(tmp_path):
     assert bench.kernel_source_hash(str(src)) == h0
     src.write_text("// header\nint f(int a) { return a + 2; }\n")
     assert bench.kernel_source_hash(str(src)) != h0
-    assert bench.up_traffic("mixtral_prefill") is not None   # the captured code is current
+    # a figure is reported only while the kernel source hashes to the captured one
+    for name, (sha, nbytes) in bench.MEASURED_UP_TRAFFIC.items():
+        cur = bench.kernel_source_hash(os.path.join(bench.ROOT, "combine_grouped_gemm_router_b200",
+                                                    "csrc", "grouped_gemm.cuh"))
+        assert bench.up_traffic(name) == (nbytes if sha == cur else None)
 
 
 def test_algorithmic_work_counts_the_payload_and_output_bytes():

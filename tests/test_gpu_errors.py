@@ -59,7 +59,7 @@ def test_nonfinite_logits_are_flagged(m):
     out = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
     stats = m.stats_buffer()
     m.moe_layer(shape, x.cuda(), inp["w_router"].cuda(), None, inp["w1"].cuda(), inp["w3"].cuda(),
-                inp["w2"].cuda(), out, stats=stats, ws=ws)
+                m.w2_for(shape, inp["w2"].cuda()), out, stats=stats, ws=ws)
     assert m.moe_get_device_error(True) == 7  # MOE_ERR_NONFINITE
     assert m.read_stats(stats).nonfinite_tokens == 1
 

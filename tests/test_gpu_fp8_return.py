@@ -44,8 +44,9 @@ def test_payload_is_the_block_code_of_y(orc, case, fp8_gemm):
     name, E, rows, d, f = case
     R = sum(rows)
     N = -(-max(R, E) // E) * E
-    shape32 = m.make_shape(N, d, f, E, 1, 1, 0.0)
-    shape8 = m.make_shape(N, d, f, E, 1, 1, 0.0, fp8_return=True)
+    # h and W2 in bf16 (the payload is quantised from whatever fp32 y the down GEMM forms)
+    shape32 = m.make_shape(N, d, f, E, 1, 1, 0.0, h_bf16=True)
+    shape8 = m.make_shape(N, d, f, E, 1, 1, 0.0, fp8_return=True, h_bf16=True)
     RA = m.moe_rows_alloc(shape32)
     assert RA >= R + 128
     g = torch.Generator().manual_seed(sum(map(ord, name)))

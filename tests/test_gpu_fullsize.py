@@ -4,14 +4,18 @@ Inputs are drawn on the GPU with a seeded generator and copied to the host for
 the oracle. Routing, counts, positions, the mapping table, the traffic matrix,
 the pack offsets and the counters are compared in full, bit for bit; both
 scatter layouts are checked row for row; expert outputs and the layer output
-are checked on a sample of tokens (first, last and seeded-random ones) that the
-oracle computes one by one, against the stated tolerance."""
+are checked against the stated tolerance (relative Frobenius 5e-3, max-abs
+2e-2 * RMS) on a sample of tokens (first, last and seeded-random ones) that the
+oracle computes one by one, and on the whole output of the 128-expert, decode and
+Mixtral-shaped layers. The stack of four layers is checked layer by layer with
+the oracle fed the GPU's own input to each layer (teacher forcing): routing and
+the inter-layer affinity counts bit for bit, each layer's output at the bar."""
 import numpy as np
 import pytest
 import torch
 
-from layer_runner import (assert_within_bound, assert_within_tolerance, bf16_h_bound_rows,
-                          run_stages, tolerance_report)
+from layer_runner import (assert_rounded_h, assert_within_bound, assert_within_tolerance,
+                          h_bound_rows, run_stages, tolerance_report)
 from moe_workloads import STACK_GRID_CF, STACK_GRID_S, WORKLOADS, make_layer_inputs
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -82,15 +86,13 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     rr["expert_of"] = np.where(r["expert_of"] >= 0, remap[r["expert_of"]], -1).astype(np.int32)
     smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr, want_h=True)
     rows = torch.from_numpy(smp["sample_rows"]).cuda().long()
+    assert_rounded_h(got["h"][rows], smp["sample_h"], "h sample")
     rep_h = tolerance_report(got["h"][rows], smp["sample_h"])
-    assert rep_h["rel_frob"] <= 5e-3, rep_h
-    # y and out: the per-element bound of one bf16 rounding of h (the down projection's
-    # operand) plus fp32 accumulation, and the relative Frobenius bar; the max-abs bar is
-    # asserted when nothing is dropped and reported otherwise (with heavy drops many
-    # sampled tokens have zero output, which deflates the RMS the bar is relative to)
-    w2 = hx["w2"].double().numpy()
+    # y and out: the per-element bound of one rounding of h (the down projection's operand,
+    # fp16) plus fp32 accumulation, the relative Frobenius bar and the max-abs bar
     sample_expert = rr["expert_of"][smp["sample_slots"]]
-    ybound = bf16_h_bound_rows(smp["sample_h"], w2, sample_expert)
+    ybound = h_bound_rows(smp["sample_h"], hx["w2"], got["w2_used"][torch.from_numpy(used).cuda()],
+                          sample_expert)
     assert_within_bound(got["y"][rows], smp["sample_y"], ybound, "y sample")
     obound = np.zeros_like(smp["out_tokens"])
     pos = {int(a): i for i, a in enumerate(smp["sample_slots"])}
@@ -104,12 +106,8 @@ def check_full_size(orc, w, seed=0, n_sample=24):
                     smp["sample_y"][yi])
     got_out = got["out"][torch.from_numpy(toks).cuda()]
     assert_within_bound(got_out, smp["out_tokens"], obound, "out sample")
-    rep_y = tolerance_report(got["y"][rows], smp["sample_y"])
-    rep_o = tolerance_report(got_out, smp["out_tokens"])
-    assert rep_y["rel_frob"] <= 5e-3 and rep_o["rel_frob"] <= 5e-3, (rep_y, rep_o)
-    if r["stats"]["dropped"] == 0:
-        assert_within_tolerance(got["y"][rows], smp["sample_y"], "y sample")
-        assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
+    rep_y = assert_within_tolerance(got["y"][rows], smp["sample_y"], "y sample")
+    rep_o = assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
     # routing margins (reported; the logits are bit-exact, so no seed is rejected)
     lg = np.sort(r["logits"], axis=1)[:, ::-1]
     margin = lg[:, w.K - 1] - lg[:, w.K] if w.K < w.E else np.full(w.N, np.inf)
@@ -149,61 +147,158 @@ def test_full_size_stack_layer(orc, cf, s):
     print("stack4 layer 0", cf, s, rep)
 
 
-def test_stack_affinity_full_size(orc):
-    """The affinity counts of the 4-layer stack at full size (N=32768, E=64, K=6).
+def full_output_check(orc, w, seed=0):
+    """The whole output of one layer (every token, every column) against the oracle's layer
+    computed in full: routing bit for bit, h within its rounding, y and the output per element
+    within the bound the arithmetic implies and within the stated bar."""
+    torch.cuda.empty_cache()
+    inp = make_layer_inputs(w, seed=seed, device="cuda")
+    got = run_stages(inp, w)
+    assert got["dev_error"] == 0
+    hx = host_inputs(inp)
+    ref = orc.layer(hx, w.K, w.W, w.cf, want_h=True, order=int(w.slot_major), reroute=w.reroute)
+    np.testing.assert_array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
+    np.testing.assert_array_equal(got["row_of"].cpu().numpy(), ref["row_of"])
+    R = ref["R"]
+    assert_rounded_h(got["h"][:R], ref["h_rows"], "h")
+    row_expert = ref["expert_of"][ref["assign_of_row"]]
+    ybound = h_bound_rows(ref["h_rows"], hx["w2"], got["w2_used"].cpu(), row_expert)
+    assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
+    kept = np.nonzero(ref["row_of"] >= 0)[0]
+    wa = np.abs(ref["topk_w"].reshape(-1)[kept].astype(np.float64))[:, None]
+    rows = ref["row_of"][kept]
+    per_slot = wa * ybound[rows] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(ref["y_rows"][rows])
+    obound = np.zeros((w.N, w.d))
+    np.add.at(obound, kept // w.K, per_slot)
+    assert_within_bound(got["out"], ref["out"], obound + 1e-30, "out")
+    rep_y = assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
+    rep_o = assert_within_tolerance(got["out"], ref["out"], "out")
+    return dict(R=R, dropped=ref["stats"]["dropped"], y=rep_y, out=rep_o)
 
-    Exactness of the count: each layer pair is counted by the GPU kernel from routing
-    that the oracle produced for seeded inputs of those two layers, and compared bit
-    for bit with the oracle's count. Then the stack itself runs on the GPU (each layer
-    fed the previous layer's output x + MoE(x), rounded to bf16) and its affinity
-    counts satisfy the invariants exactly: row sums are K times the tokens routed to
-    the row's expert, the total is K^2 N, and they equal a recount of its own routing."""
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_full_output_e128_skew(orc, seed):
+    """The 128-expert layer with Zipf skew and capacity drops (two thirds of the assignments
+    dropped): every element of the output, four seeds."""
+    rep = full_output_check(orc, WORKLOADS["e128_skew"], seed)
+    assert rep["dropped"] > 0
+    print("e128_skew full output", seed, rep)
+
+
+def test_full_output_decode(orc):
+    rep = full_output_check(orc, WORKLOADS["decode"], 0)
+    print("decode full output", rep)
+
+
+def test_full_output_mixtral_prefill(orc):
+    """The Mixtral-shaped layer in full: 2.9 TFLOP for the oracle (about a minute on 16 host
+    cores)."""
+    rep = full_output_check(orc, WORKLOADS["mixtral_prefill"], 0)
+    print("mixtral_prefill full output", rep)
+
+
+def sampled_output_check(orc, inp, w, r, toks, got_out, w2_used):
+    """The layer output of the tokens `toks` (got_out, fp32 rows in the order of toks) against
+    the oracle's expert FFN and combine of those tokens under the routing r: per element within
+    the propagated bound, and the stated bar."""
+    slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
+    eo = r["expert_of"][slots]
+    used = np.unique(eo[eo >= 0])
+    remap = np.full(w.E, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    ut = torch.from_numpy(used).to(inp["w1"].device)
+    hx = host_inputs(inp, experts=ut)
+    rr = dict(r)
+    rr["expert_of"] = np.where(r["expert_of"] >= 0, remap[r["expert_of"]], -1).astype(np.int32)
+    smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr, want_h=True)
+    sample_expert = rr["expert_of"][smp["sample_slots"]]
+    ybound = h_bound_rows(smp["sample_h"], hx["w2"], w2_used[ut].cpu(), sample_expert)
+    obound = np.zeros_like(smp["out_tokens"])
+    pos = {int(a): i for i, a in enumerate(smp["sample_slots"])}
+    for li, t in enumerate(toks):
+        for k in range(w.K):
+            a = int(t) * w.K + k
+            if a in pos:
+                wa = abs(float(r["topk_w"].reshape(-1)[a]))
+                yi = pos[a]
+                obound[li] += wa * ybound[yi] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(
+                    smp["sample_y"][yi])
+    assert_within_bound(got_out, smp["out_tokens"], obound, "out sample")
+    return assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
+
+
+def stack_teacher_forced(orc, w, n_sample=16):
+    """The stack of w.layers layers on the GPU, x_{j+1} = bf16(x_j + MoE_j(x_j)), checked layer by
+    layer against the oracle fed the GPU's own x_j (teacher forcing, so that the routing
+    contract holds per layer):
+     * the stack's step equals the layer's fp32 output plus x_j, rounded once to bf16;
+     * topk_idx and the dispatch counters of layer j equal the oracle's on x_j, bit for bit;
+     * the output of layer j on sampled tokens is within the stated bar of the oracle's;
+     * the inter-layer affinity counts moe_affinity_accumulate forms from the GPU's routing
+       equal the oracle's counts from its own routing, bit for bit."""
     import combine_grouped_gemm_router_b200 as m
-    w = WORKLOADS["stack4"].with_(cf=1.25, s=1.2)
-    N, E, K = w.N, w.E, w.K
-    routes = []
-    for layer in range(2):
-        inp = make_layer_inputs(w, seed=layer, device="cuda")
-        hx = host_inputs(inp, experts=[])
-        lg = orc.router_logits(hx["x"], hx["w_router"], hx["bias"])
-        routes.append(orc.topk(lg, K)[0])
-        del inp
-    cnt = torch.zeros(E, E, dtype=torch.int64, device="cuda")
-    m.moe_affinity_accumulate(N, E, K, torch.from_numpy(routes[0]).cuda(),
-                              torch.from_numpy(routes[1]).cuda(), cnt)
-    np.testing.assert_array_equal(cnt.cpu().numpy(), orc.affinity(routes[0], routes[1], E))
-
-    # the stack on the GPU
-    shape = m.make_shape(N, w.d, w.f, E, K, w.W, w.cf, out_bf16=True)
-    ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device="cuda")
-    x = make_layer_inputs(w, seed=0, device="cuda")["x"]
-    topks = []
+    N, d, E, K = w.N, w.d, w.E, w.K
+    torch.cuda.empty_cache()
+    shape32 = m.make_shape(N, d, w.f, E, K, w.W, w.cf)
+    shape16 = m.make_shape(N, d, w.f, E, K, w.W, w.cf, out_bf16=True)
+    ws = torch.empty(m.moe_layer_workspace_size(shape16), dtype=torch.uint8, device="cuda")
+    x = make_layer_inputs(w, seed=0, device="cuda", with_x=True)["x"]
+    gpu_routes, orc_routes, reports = [], [], []
     for layer in range(w.layers):
         lin = make_layer_inputs(w, seed=0, device="cuda", layer=layer, with_x=False)
+        w2h = m.w2_for(shape32, lin["w2"])
+        moe = torch.empty(N, d, dtype=torch.float32, device="cuda")
         topk = torch.empty(N, K, dtype=torch.int32, device="cuda")
+        stats = m.stats_buffer()
+        m.moe_layer(shape32, x, lin["w_router"], lin["bias"], lin["w1"], lin["w3"], w2h, moe,
+                    topk_idx_out=topk, stats=stats, ws=ws)
         nxt = torch.empty_like(x)
-        m.moe_layer(shape, x, lin["w_router"], lin["bias"], lin["w1"], lin["w3"], lin["w2"], nxt,
-                    residual=x, topk_idx_out=topk, ws=ws)
-        topks.append(topk)
+        topk2 = torch.empty_like(topk)
+        m.moe_layer(shape16, x, lin["w_router"], lin["bias"], lin["w1"], lin["w3"], w2h, nxt,
+                    residual=x, topk_idx_out=topk2, ws=ws)
+        torch.cuda.synchronize()
+        assert m.moe_get_device_error(True) == 0
+        assert torch.equal(topk, topk2)
+        assert torch.equal(nxt, (moe + x.float()).to(torch.bfloat16)), "stack step"
+        inp = dict(lin, x=x)
+        hx = host_inputs(inp, experts=[])
+        r = orc.route_and_dispatch(hx["x"], hx["w_router"], hx["bias"], K, w.W, w.cf)
+        np.testing.assert_array_equal(topk.cpu().numpy(), r["topk_idx"])
+        st, rs = m.stats_dict(m.read_stats(stats)), r["stats"]
+        assert (st["rows"], st["dropped"], st["cross_rows"], st["dedup_pairs"],
+                st["active_experts"], st["max_kept"], st["min_kept"]) == (
+                    rs["R"], rs["dropped"], rs["cross_rows"], rs["dedup_pairs"],
+                    rs["active_experts"], rs["max_kept"], rs["min_kept"])
+        toks = sample_tokens(N, n_sample, seed=layer)
+        rep = sampled_output_check(orc, inp, w, r, toks, moe[torch.from_numpy(toks).cuda()], w2h)
+        reports.append(dict(layer=layer, dropped=rs["dropped"], **rep))
+        gpu_routes.append(topk)
+        orc_routes.append(r["topk_idx"])
+        del lin, w2h
         x = nxt
-        del lin
-    torch.cuda.synchronize()
-    assert m.moe_get_device_error(True) == 0
     for j in range(w.layers - 1):
         c = torch.zeros(E, E, dtype=torch.int64, device="cuda")
-        m.moe_affinity_accumulate(N, E, K, topks[j], topks[j + 1], c)
-        c = c.cpu().numpy()
-        a = topks[j].cpu().numpy()
-        b = topks[j + 1].cpu().numpy()
-        n_i = np.bincount(a.reshape(-1), minlength=E)
-        np.testing.assert_array_equal(c.sum(1), K * n_i)
-        assert c.sum() == K * K * N
-        recount = np.zeros((E, E), np.int64)
-        np.add.at(recount, (np.repeat(a, K, axis=1).reshape(-1), np.tile(b, (1, K)).reshape(-1)), 1)
-        np.testing.assert_array_equal(c, recount)
-        P = c / np.maximum(n_i[:, None], 1)
-        print(f"layer pair {j}->{j + 1}: max P(p|i) = {P.max():.3f}, diag mass "
-              f"{np.trace(c) / c.sum():.4f}")
+        m.moe_affinity_accumulate(N, E, K, gpu_routes[j], gpu_routes[j + 1], c)
+        ref = orc.affinity(orc_routes[j], orc_routes[j + 1], E)
+        np.testing.assert_array_equal(c.cpu().numpy(), ref)
+        assert int(ref.sum()) == K * K * N
+    return reports
+
+
+@pytest.mark.parametrize("cf", STACK_GRID_CF)
+@pytest.mark.parametrize("s", STACK_GRID_S)
+def test_stack_teacher_forced(orc, cf, s):
+    """The 4-layer stack (N=32768, d=4096, f=1536, E=64, K=6) at every capacity factor and Zipf
+    skew of its grid, each layer against the oracle on the GPU's own input."""
+    reps = stack_teacher_forced(orc, WORKLOADS["stack4"].with_(cf=cf, s=s))
+    print("stack4", cf, s, reps)
+
+
+def test_stack_teacher_forced_planted_affinity(orc):
+    """The stack whose routers carry planted inter-layer affinity: the affinity counts (sparse,
+    concentrated rows) bit for bit against the oracle's."""
+    reps = stack_teacher_forced(orc, WORKLOADS["stack4_affinity"], n_sample=8)
+    print("stack4_affinity", reps)
 
 
 def test_full_size_residual_moe(orc):
@@ -216,12 +311,13 @@ def test_full_size_residual_moe(orc):
     inp = make_layer_inputs(w, seed=0, device="cuda")
     sh = make_shared_inputs(w, seed=0, device="cuda")
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
+    w2h, ws2h = m.w2_for(shape, inp["w2"]), m.w2_for(shape, sh["ws2"])
     ws = torch.empty(m.moe_layer_shared_workspace_size(shape, w.shared_f), dtype=torch.uint8,
                      device="cuda")
     out = torch.empty(w.N, w.d, dtype=torch.float32, device="cuda")
     topk = torch.empty(w.N, w.K, dtype=torch.int32, device="cuda")
     m.moe_layer_shared(shape, w.shared_f, inp["x"], inp["w_router"], inp["bias"], inp["w1"],
-                       inp["w3"], inp["w2"], sh["ws1"], sh["ws3"], sh["ws2"], out,
+                       inp["w3"], w2h, sh["ws1"], sh["ws3"], ws2h, out,
                        topk_idx_out=topk, ws=ws)
     torch.cuda.synchronize()
     assert m.moe_get_device_error(True) == 0

@@ -1,13 +1,14 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle on shapes the
 oracle finishes in seconds: several tiles per expert, ragged tails, drops,
 empty experts, K = E, E = 1. Integer outputs bit-exact; floating-point outputs
-within relative Frobenius 5e-3 and max-abs 2e-2 * RMS of the oracle."""
+within relative Frobenius 5e-3 and max-abs 2e-2 * RMS of the oracle, on every case,
+and within the per-element bound the arithmetic implies."""
 import numpy as np
 import pytest
 import torch
 
-from layer_runner import (assert_rounded_bf16, assert_within_bound, assert_within_tolerance,
-                          bf16_h_bound_rows, run_layer, run_stages, tolerance_report)
+from layer_runner import (assert_rounded_h, assert_within_bound, assert_within_tolerance,
+                          h_bound_rows, run_layer, run_stages, tolerance_report)
 from moe_workloads import WORKLOADS, Workload, make_layer_inputs
 
 pytestmark = pytest.mark.gpu
@@ -19,8 +20,8 @@ CASES = [
     # capacity drops under Zipf skew; d = 384 takes the 128-wide N tile of G2
     Workload("drop_bn128", N=384, d=384, f=256, E=6, K=3, W=3, cf=1.25, s=1.1),
     # many experts with few rows, some with none; heavy Zipf skew with drops gives a
-    # heavy-tailed output (a few elements near 7x its RMS), where one bf16 rounding of h
-    # moves the largest element by about 2.1% of the RMS: see HEAVY_TAIL below
+    # heavy-tailed output (a few elements near 7x its RMS): the case where a bf16 h would
+    # miss the max-abs bar (2.1% of the RMS) and the fp16 h meets it (0.3%)
     Workload("sparse_experts", N=256, d=128, f=128, E=64, K=6, W=8, cf=1.0, s=1.2),
     Workload("k_eq_e", N=64, d=128, f=128, E=4, K=4, W=2),
     Workload("dense_e1", N=300, d=256, f=256, E=1, K=1, W=1),
@@ -61,15 +62,32 @@ CASES = [
 ]
 
 
-# Cases whose max-abs error against the fp64 oracle is set by the bf16 rounding of the
-# SwiGLU activation h (the down projection's tensor-core operand) on a heavy-tailed
-# output; for them the stated max-abs bar is not claimed, the derived per-element bound
-# and the relative Frobenius bar are.
-HEAVY_TAIL = {"sparse_experts"}
-
-
 def _u16(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_float_outputs(ref, got, inp, w, stated_bar: bool = True):
+    """h, y and out against the oracle: per element within the bound the arithmetic implies
+    (one rounding of h in the precision the run stored it in, fp32 accumulation), relative
+    Frobenius 5e-3, and, when `stated_bar`, max-abs 2e-2 * RMS on y and on the output."""
+    R = ref["R"]
+    assert_rounded_h(got["h"][:R], ref["h_rows"], "h")
+    row_expert = ref["expert_of"][ref["assign_of_row"]]
+    ybound = h_bound_rows(ref["h_rows"], inp["w2"], got.get("w2_used"), row_expert)
+    assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
+    obound = np.zeros((w.N, w.d))
+    for a in np.nonzero(ref["row_of"] >= 0)[0]:
+        wa = abs(float(ref["topk_w"].reshape(-1)[a]))
+        r = ref["row_of"][a]
+        # propagated y bound, plus the fp32 weights and the fp32 sum over K slots
+        obound[a // w.K] += wa * ybound[r] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(ref["y_rows"][r])
+    assert_within_bound(got["out"], ref["out"], obound, "out")
+    if stated_bar:
+        assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
+        return assert_within_tolerance(got["out"], ref["out"], "out")
+    rep = tolerance_report(got["out"], ref["out"])
+    assert rep["rel_frob"] <= 5e-3, rep
+    return rep
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
@@ -115,25 +133,8 @@ def test_layer_stages_match_oracle(orc, w, seed):
     packed[ref["packed_row_of"][kept_slots]] = xu[kept_slots // w.K]
     np.testing.assert_array_equal(_u16(got["x_packed"][:R]), packed)
 
-    # a5/a6: expert GEMMs; a7: combine
-    assert_rounded_bf16(got["h"][:R], ref["h_rows"], "h")
-    w2 = inp["w2"].double().numpy()
-    row_expert = ref["expert_of"][ref["assign_of_row"]]
-    ybound = bf16_h_bound_rows(ref["h_rows"], w2, row_expert)
-    assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
-    obound = np.zeros((w.N, w.d))
-    for a in np.nonzero(ref["row_of"] >= 0)[0]:
-        wa = abs(float(ref["topk_w"].reshape(-1)[a]))
-        r = ref["row_of"][a]
-        # propagated y bound, plus the fp32 weights and the fp32 sum over K slots
-        obound[a // w.K] += wa * ybound[r] + (w.K + 8) * 2.0 ** -24 * wa * np.abs(ref["y_rows"][r])
-    assert_within_bound(got["out"], ref["out"], obound, "out")
-    if w.name in HEAVY_TAIL:
-        rep = tolerance_report(got["out"], ref["out"])
-        assert rep["rel_frob"] <= 5e-3 and rep["max_abs_over_rms"] <= 3e-2, rep
-    else:
-        assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
-        assert_within_tolerance(got["out"], ref["out"], "out")
+    # a5/a6: expert GEMMs; a7: combine (fp16 h: the stated bar on every case)
+    check_float_outputs(ref, got, inp, w)
 
     # the fused entry point runs the same kernels: identical bits
     lay = run_layer(inp, w)
@@ -142,6 +143,55 @@ def test_layer_stages_match_oracle(orc, w, seed):
                                   got["out"].cpu().numpy().view(np.uint32))
     np.testing.assert_array_equal(lay["topk_idx"].cpu().numpy(), ref["topk_idx"])
     assert lay["stats"]["dedup_pairs"] == rs["dedup_pairs"]
+
+
+BF16_H_CASES = ["tiny", "ragged", "drop_bn128", "sparse_experts", "pair_split", "max_limits"]
+
+
+@pytest.mark.parametrize("name", BF16_H_CASES)
+def test_layer_bf16_h_mode(orc, name):
+    """The bf16 precision of h (MOE_FLAG_H_BF16; W2 in bf16): every output within the
+    per-element bound of one bf16 rounding of h and the relative Frobenius bar. The max-abs bar
+    is not claimed for this mode: on a heavy-tailed output (sparse_experts) one bf16 rounding
+    of h moves the largest element by about 2 % of the output's RMS."""
+    w = next(c for c in CASES if c.name == name)
+    inp = make_layer_inputs(w, seed=0)
+    ref = orc.layer(inp, w.K, w.W, w.cf, want_h=True, order=int(w.slot_major),
+                    reroute=w.reroute)
+    got = run_stages(inp, w, h_bf16=True)
+    assert got["dev_error"] == 0
+    assert got["h"].dtype == torch.bfloat16
+    np.testing.assert_array_equal(got["row_of"].cpu().numpy(), ref["row_of"])
+    rep = check_float_outputs(ref, got, inp, w, stated_bar=False)
+    lay = run_layer(inp, w, h_bf16=True)
+    np.testing.assert_array_equal(lay["out"].cpu().numpy().view(np.uint32),
+                                  got["out"].cpu().numpy().view(np.uint32))
+    print(name, "bf16 h", rep)
+
+
+def test_convert_bf16_to_f16_matches_torch():
+    """The fp16 copy of the weights: bit for bit torch's own bf16 -> fp16 conversion (round to
+    nearest even), and the count of changed elements equal to the count of values that are
+    not fp16 numbers, on N(0, 0.02) weights plus hand-picked corners (tiny, subnormal in fp16,
+    the largest finite fp16, beyond it)."""
+    import combine_grouped_gemm_router_b200 as m
+    g = torch.Generator().manual_seed(3)
+    w = (torch.randn(1 << 20, generator=g) * 0.02).to(torch.bfloat16)
+    corners = torch.tensor([0.0, -0.0, 2.0 ** -17, -2.0 ** -18, 3.0 * 2.0 ** -20, 2.0 ** -24,
+                            2.0 ** -26, 1e-30, 65504.0, -65504.0, 1.0, -448.0, 3.0e38, -7e4,
+                            2.0 ** -14, 0.5], dtype=torch.float32).to(torch.bfloat16)
+    src = torch.cat([w, corners]).cuda()
+    dst = torch.empty(src.shape, dtype=torch.float16, device="cuda")
+    changed = torch.zeros(1, dtype=torch.int64, device="cuda")
+    m.moe_convert_bf16_to_f16(src, dst, changed)
+    torch.cuda.synchronize()
+    ref = src.cpu().to(torch.float16)
+    assert torch.equal(dst.cpu().view(torch.int16), ref.view(torch.int16))
+    n_changed = int((ref.float() != src.cpu().float()).sum())
+    assert int(changed.item()) == n_changed and n_changed > 0
+    # the two values beyond 65504 became infinite: recorded in the device error word
+    assert m.moe_get_device_error(True) == 9
+    assert m.moe_get_device_error(True) == 0
 
 
 def test_residual_combine(orc):
@@ -154,13 +204,14 @@ def test_residual_combine(orc):
     ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
     x = inp["x"].to(dev)
     out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
+    w2 = m.w2_for(shape, inp["w2"].to(dev))
     m.moe_layer(shape, x, inp["w_router"].to(dev), None, inp["w1"].to(dev), inp["w3"].to(dev),
-                inp["w2"].to(dev), out, residual=x, ws=ws)
+                w2, out, residual=x, ws=ws)
     # bf16 output mode (the next layer's input), out of place
     shape16 = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, out_bf16=True)
     out16 = torch.empty(w.N, w.d, dtype=torch.bfloat16, device=dev)
     m.moe_layer(shape16, x, inp["w_router"].to(dev), None, inp["w1"].to(dev), inp["w3"].to(dev),
-                inp["w2"].to(dev), out16, residual=x, ws=ws)
+                w2, out16, residual=x, ws=ws)
     torch.cuda.synchronize()
     xr = inp["x"].double().numpy()
     assert_within_tolerance(out, xr + ref["out"], "x + moe(x)")
@@ -220,7 +271,8 @@ def test_residual_moe_layer(orc):
         dev = torch.device("cuda")
         shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf)
         shd = {k: v.to(dev) for k, v in sh.items()}
-        h_s = torch.empty(w.N, w.shared_f, dtype=torch.bfloat16, device=dev)
+        shd["ws2"] = m.w2_for(shape, shd["ws2"])  # the down projection's weights in fp16
+        h_s = torch.empty(w.N, w.shared_f, dtype=torch.float16, device=dev)
         y_s = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
         ws_s = torch.empty(256, dtype=torch.uint8, device=dev)
         x = inp["x"].to(dev)
@@ -235,7 +287,7 @@ def test_residual_moe_layer(orc):
         out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
         bias = None if inp["bias"] is None else inp["bias"].to(dev)
         m.moe_layer_shared(shape, w.shared_f, x, inp["w_router"].to(dev), bias, inp["w1"].to(dev),
-                           inp["w3"].to(dev), inp["w2"].to(dev), shd["ws1"], shd["ws3"], shd["ws2"],
+                           inp["w3"].to(dev), got["w2_used"], shd["ws1"], shd["ws3"], shd["ws2"],
                            out, ws=ws)
         torch.cuda.synchronize()
         assert m.moe_get_device_error(True) == 0
