@@ -287,23 +287,19 @@ def placement_report(m, counts, L: int, E: int, P: int) -> dict:
 
 def kernel_launches(w) -> int:
     """Kernels the library launches for one layer of workload w, by the same rules as its
-    host code: routing 2; per dispatch pass a histogram, a per-expert scan when there are
-    more than 128 blocks, the scan and the positions; the ranking kernel between the two
-    passes of re-routing; the scatter; each grouped GEMM once, or twice (CTA-pair tiles, then
-    single-CTA tiles) when the experts average at least 768 rows and the K extent allows pair
-    stages; the quantisation of h on the FP8 path; the shared MLP's offsets and GEMMs; the
-    combine."""
+    host code: routing 1 (the fused projection + top-K kernel, E >= 32 and N >= 2048) or 2
+    (projection, then selection); per dispatch pass the histogram / look-back kernel and the
+    placement kernel (the pass's control words are cleared by a memset, not a kernel); with
+    re-routing a positions-only pass, the ranking kernel, then the full pass; each grouped GEMM
+    once, or twice (CTA-pair tiles, then single-CTA tiles) when the experts average at least
+    768 rows and the K extent allows pair stages; the quantisation of h on the FP8 path; the
+    shared MLP's offsets and GEMMs; the combine."""
     N, d, f, E, K, W = w.N, w.d, w.f, w.E, w.K, w.W
     NK = N * K
     C = NK if not w.cf > 0 else min(NK, math.ceil(w.cf * N * K / E))
     pair = min(NK // E, C) >= 768
-    nvb_round = (K if w.slot_major else 1) * W * (-(-(N // W) // 64))
-    def dispatch_pass(nvb):
-        return 3 + (1 if nvb > 128 else 0)
-    n = 2
-    n += dispatch_pass(nvb_round) + 1 + dispatch_pass(2 * nvb_round) if w.reroute \
-        else dispatch_pass(nvb_round)
-    n += 1  # scatter
+    n = 1 if (E >= 32 and N >= 2048) else 2
+    n += (2 + 1 + 2) if w.reroute else 2
     atom = 128 if w.fp8 else 64
     n += 2 if pair and (d // atom) % 2 == 0 else 1                     # gate/up
     n += 1 if w.fp8 else 0                                              # h -> e4m3

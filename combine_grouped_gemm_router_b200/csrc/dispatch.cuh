@@ -68,32 +68,55 @@ struct VBlocks {
     }
 };
 
-// blk[e][vb] = number of assignments in virtual block vb routed to expert e.
-__global__ void __launch_bounds__(256)
-    block_hist_kernel(const int32_t *__restrict__ topk_idx, int E, VBlocks vbm, int nvb,
-                      int32_t *__restrict__ blk)
+// Control words of one dispatch pass, zeroed before the pass: the ticket that hands out
+// virtual blocks in launch order, the count of blocks finished, then one status flag per
+// virtual block (0: nothing published; kFlagAgg: its histogram; kFlagIncl: its inclusive
+// prefix over every earlier block of the priority order).
+constexpr unsigned int kFlagAgg = 1;
+constexpr unsigned int kFlagIncl = 2;
+
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int *p)
 {
-    extern __shared__ int s_hist[];
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        s_hist[e] = 0;
-    __syncthreads();
-    int t0, t1, k, round;
-    vbm.range(blockIdx.x, t0, t1, k, round);
-    const int32_t *src = vbm.experts(topk_idx, round);
-    const int n = vbm.count(t0, t1);
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int e = src[vbm.assign(t0, k, i)];
-        if ((unsigned)e < (unsigned)E)
-            atomicAdd(&s_hist[e], 1);
-        else if (round == 0)
-            set_dev_error(MOE_ERR_DEVICE_BOUNDS);  // round 1 marks "not moved" with -1
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        blk[(size_t)e * nvb + blockIdx.x] = s_hist[e];
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
-// In-place exclusive scan of a[0..n) in shared memory by the whole block;
+__device__ __forceinline__ void st_release_u32(unsigned int *p, unsigned int v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+struct HistArgs {
+    const int32_t *topk_idx;
+    VBlocks vbm;
+    int nvb;         // virtual blocks of the pass (all its rounds)
+    int bps;         // virtual blocks per segment (segment g = blocks [g*bps, (g+1)*bps))
+    int nseg;        // segments of the pass
+    int nseg_round;  // segments of one round
+    int N, E, K, W, C;
+    unsigned int *ctl;  // [2 + nvb]: ticket, done, flags
+    int32_t *agg;       // [nvb][E] the blocks' histograms
+    int32_t *incl;      // [nvb][E] inclusive prefixes over the priority order
+    // the pass's totals, written by the block that finishes last:
+    int32_t *counts, *kept, *offsets;
+    int64_t *D;        // [W][W]
+    int64_t *pk_off;   // [W*W+1]
+    int64_t *pk_base;  // [nseg][E]
+    moe_stats_t *stats;
+    uint64_t timeout_ns;
+};
+
+// Assignments to expert e before segment g in priority order (g = nseg: the pass's total).
+__device__ __forceinline__ int seg_cum(const HistArgs &p, int e, int g)
+{
+    if (g >= p.nseg)
+        return __ldcg(p.incl + (size_t)(p.nvb - 1) * p.E + e);
+    const size_t o = (size_t)g * p.bps * p.E + e;
+    return __ldcg(p.incl + o) - __ldcg(p.agg + o);
+}
+
+// In-place exclusive scan of a[0..n) in shared memory by the whole block of NT threads;
 // a[n] receives the total. s_warp needs 32 entries.
 template <int NT>
 __device__ void block_excl_scan_i64(int64_t *a, int n, int64_t *s_warp)
@@ -128,130 +151,48 @@ __device__ void block_excl_scan_i64(int64_t *a, int n, int64_t *s_warp)
     __syncthreads();
 }
 
-// Many blocks (slot-major priority, re-routing): one CTA per expert turns its row of
-// block counts into exclusive bases and records the expert's count at every segment start
-// (cum [E][nseg+1], cum[e][nseg] = total); dispatch_scan_kernel then skips that step.
-__global__ void __launch_bounds__(256)
-    expert_block_scan_kernel(int32_t *__restrict__ blk, int nvb, int bps, int nseg,
-                             int32_t *__restrict__ cum)
+constexpr int kHistThreads = 256;
+
+// Shared memory of dispatch_hist_kernel: the block's histogram, then (for the block that
+// finishes last) s_a [max(E, W*W) + 1] int64, s_D [W*W] int64, s_warp [32] int64 and
+// s_kh [E][W] int32 (kept rows of expert e from home shard i).
+__host__ __device__ inline size_t hist_smem_bytes(int E, int W)
 {
-    __shared__ int s_warp[8];
-    const int e = blockIdx.x;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int32_t *row = blk + (size_t)e * nvb;
-    const int per = (nvb + 255) / 256;
-    const int beg = min(nvb, (int)threadIdx.x * per), end = min(nvb, beg + per);
-    int local = 0;
-    for (int i = beg; i < end; ++i)
-        local += row[i];
-    const int incl = warp_incl_scan(local);
-    if (lane == 31)
-        s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        const int v = lane < 8 ? s_warp[lane] : 0;
-        const int vi = warp_incl_scan(v);
-        if (lane < 8)
-            s_warp[lane] = vi - v;
-    }
-    __syncthreads();
-    int run = s_warp[warp] + incl - local;
-    for (int i = beg; i < end; ++i) {
-        const int v = row[i];
-        row[i] = run;
-        if (i % bps == 0)
-            cum[(size_t)e * (nseg + 1) + i / bps] = run;
-        run += v;
-    }
-    if (threadIdx.x == 255)
-        cum[(size_t)e * (nseg + 1) + nseg] = run;  // the last thread ends at the total
+    const size_t scan = ((size_t)(E > W * W ? E : W * W) + 1) * 8 + (size_t)W * W * 8 + 32 * 8 +
+                        (size_t)E * W * 4;
+    const size_t hist = (size_t)E * 4;
+    return scan > hist ? scan : hist;
 }
 
-struct ScanArgs {
-    int32_t *blk;  // [E][nvb] counts in, exclusive bases out
-    int nvb;
-    int bps;       // virtual blocks per segment
-    int nseg;      // segments in priority order: W (token-major) or K*W (slot-major) a round
-    int nseg_round;
-    int N, E, K, W;
-    int C;
-    int32_t *cum_global;  // [E][nseg+1] when it does not fit in shared memory, else null
-    int prescanned;       // expert_block_scan_kernel has done step 1 into cum_global
-    int32_t *counts, *kept, *offsets;
-    int64_t *D;        // [W][W]
-    int64_t *pk_off;   // [W*W+1]
-    int64_t *pk_base;  // [E][nseg]
-    moe_stats_t *stats;
-};
-
-// One CTA of 1024 threads.
-// Shared: s_a [max(E, W*W) + 1] int64 scan buffer, s_D [W*W] int64, s_warp [32],
-//         s_kh [E][W] int32 (kept rows of expert e from home shard i), then
-//         cum [E][nseg+1] int32 unless it lives in global memory: cum[e][g] =
-//         assignments to e before segment g in priority order, cum[e][nseg] = total.
-// Segment g belongs to home shard g % W; within one home shard its segments
-// come in priority order, so the kept rows of expert e from that shard are a
-// prefix of the shard's own sequence of assignments to e.
-__global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
+// The pass's totals, from the prefixes every block published (the block that finished last
+// runs this): counts (routed demand: round 0's total), kept = min(total, C), offsets (scan of
+// kept), the traffic matrix D, the pack offsets and the pack base of every (segment, expert),
+// and the counters. Segment g belongs to home shard g % W; within one home shard its
+// segments come in priority order, so the kept rows of expert e from that shard are a prefix
+// of the shard's own sequence of assignments to e.
+__device__ void pass_totals(const HistArgs &p, unsigned char *smem)
 {
-    constexpr int NT = 1024;
-    extern __shared__ __align__(16) unsigned char scan_smem[];
-    const int E = p.E, W = p.W, nvb = p.nvb, bps = p.bps, G = p.nseg;
+    constexpr int NT = kHistThreads;
+    const int E = p.E, W = p.W, G = p.nseg;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t C = p.C;
     const int scan_len = max(E, W * W) + 1;
-    int64_t *s_a = reinterpret_cast<int64_t *>(scan_smem);
+    int64_t *s_a = reinterpret_cast<int64_t *>(smem);
     int64_t *s_D = s_a + scan_len;
     int64_t *s_warp = s_D + W * W;
     int32_t *s_kh = reinterpret_cast<int32_t *>(s_warp + 32);
-    int32_t *cum = p.cum_global ? p.cum_global : s_kh + E * W;
 
-    // 1. per expert: exclusive scan over virtual blocks; record segment starts
-    for (int e = warp; e < E && !p.prescanned; e += NT / 32) {
-        int32_t *row = p.blk + (size_t)e * nvb;
-        int carry = 0;
-        for (int base = 0; base < nvb; base += 128) {
-            int v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int idx = base + lane * 4 + q;
-                v[q] = idx < nvb ? row[idx] : 0;
-            }
-            const int lsum = v[0] + v[1] + v[2] + v[3];
-            const int incl = warp_incl_scan(lsum);
-            int run = carry + incl - lsum;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int idx = base + lane * 4 + q;
-                if (idx < nvb) {
-                    row[idx] = run;
-                    if (idx % bps == 0)
-                        cum[e * (G + 1) + idx / bps] = run;
-                }
-                run += v[q];
-            }
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0)
-            cum[e * (G + 1) + G] = carry;
-    }
-    __syncthreads();
-
-    // 2. counts (round 0: the routed demand), kept, offsets; kept rows per
-    //    (expert, home shard)
     for (int e = threadIdx.x; e < E; e += NT) {
-        const int c = cum[e * (G + 1) + p.nseg_round];
-        const int kp = (int)min((int64_t)cum[e * (G + 1) + G], C);
-        p.counts[e] = c;
+        const int kp = (int)min((int64_t)seg_cum(p, e, G), C);
+        p.counts[e] = seg_cum(p, e, p.nseg_round);
         p.kept[e] = kp;
         s_a[e] = kp;
     }
     for (int ei = threadIdx.x; ei < E * W; ei += NT) {
         const int e = ei / W, i = ei % W;
-        const int32_t *ce = cum + e * (G + 1);
         int64_t s = 0;
         for (int g = i; g < G; g += W)
-            s += min((int64_t)ce[g + 1], C) - min((int64_t)ce[g], C);
+            s += min((int64_t)seg_cum(p, e, g + 1), C) - min((int64_t)seg_cum(p, e, g), C);
         s_kh[ei] = (int32_t)s;
     }
     __syncthreads();
@@ -260,7 +201,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
         p.offsets[e] = (int32_t)s_a[e];
     __syncthreads();
 
-    // 3. traffic matrix D[i][j] = kept rows of experts on rank j from shard i
+    // traffic matrix D[i][j] = kept rows of experts on rank j from shard i
     const int e_per = E / W;
     for (int ij = threadIdx.x; ij < W * W; ij += NT) {
         const int i = ij / W, j = ij % W;
@@ -268,46 +209,44 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
         for (int e = j * e_per; e < (j + 1) * e_per; ++e)
             s += s_kh[e * W + i];
         s_D[ij] = s;
-        if (p.D)
-            p.D[ij] = s;
+        p.D[ij] = s;
     }
     __syncthreads();
     for (int ij = threadIdx.x; ij < W * W; ij += NT)
         s_a[ij] = s_D[ij];
     __syncthreads();
     block_excl_scan_i64<NT>(s_a, W * W, s_warp);
-    if (p.pk_off)
-        for (int ij = threadIdx.x; ij <= W * W; ij += NT)
-            p.pk_off[ij] = s_a[ij];
+    for (int ij = threadIdx.x; ij <= W * W; ij += NT)
+        p.pk_off[ij] = s_a[ij];
 
-    // 4. pack bases: a kept assignment to expert e at position pos (in e's rows)
-    //    from segment g lands on packed row pk_base[e][g] + pos. Block (i, j)
-    //    holds its experts in order, each expert's rows from shard i in the
-    //    shard's own order: the earlier segments of shard i come first.
+    // pack bases: a kept assignment to expert e at position pos (in e's rows) from segment g
+    // lands on packed row pk_base[g][e] + pos. Block (i, j) holds its experts in order, each
+    // expert's rows from shard i in the shard's own order: the earlier segments of shard i
+    // come first.
     for (int ei = threadIdx.x; ei < E * W; ei += NT) {
         const int e = ei / W, i = ei % W;
         const int j = e / e_per;
         int64_t base = s_a[i * W + j];
         for (int e2 = j * e_per; e2 < e; ++e2)
             base += s_kh[e2 * W + i];
-        const int32_t *ce = cum + e * (G + 1);
         int64_t run = 0;
         for (int g = i; g < G; g += W) {
-            p.pk_base[(size_t)e * G + g] = base + run - ce[g];
-            run += ce[g + 1] - ce[g];
+            const int c0 = seg_cum(p, e, g);
+            p.pk_base[(size_t)g * E + e] = base + run - c0;
+            run += seg_cum(p, e, g + 1) - c0;
         }
     }
 
-    // 5. counters (dedup_pairs is added by the scatter kernel)
+    // counters (dedup_pairs is added by the placement kernel)
     if (p.stats && warp == 0) {
         int mx = 0, mn = 0x7fffffff, act = 0;
         int64_t first = 0;  // rows from round 0
         for (int e = lane; e < E; e += 32) {
-            const int kp = (int)min((int64_t)cum[e * (G + 1) + G], C);
+            const int kp = (int)min((int64_t)seg_cum(p, e, G), C);
             mx = max(mx, kp);
             mn = min(mn, kp);
             act += kp > 0;
-            first += min((int64_t)cum[e * (G + 1) + p.nseg_round], C);
+            first += min((int64_t)seg_cum(p, e, p.nseg_round), C);
         }
         first = warp_sum(first);
 #pragma unroll
@@ -335,83 +274,334 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(ScanArgs p)
     }
 }
 
-struct PosArgs {
-    const int32_t *topk_idx;
-    const int32_t *blk;  // [E][nvb] exclusive bases
-    int nvb;
-    VBlocks vbm;
-    int E;
-    int C;
-    const int32_t *offsets;
-    int32_t *row_of;
-    int32_t *assign_of_row;
-};
-
-// One CTA (8 warps) per virtual block. Shared: wcnt [8][E] int32, s_off [E] int32.
-// Each assignment's row_of is written by exactly one block: its round-0 block,
-// unless it was moved, then its round-1 block.
-__global__ void __launch_bounds__(256) dispatch_positions_kernel(PosArgs p)
+// One CTA per virtual block, taken in launch order from a ticket: the block's expert
+// histogram, published; its exclusive prefix over all earlier blocks of the priority order
+// by a decoupled look-back (each thread walks back over its expert's column: a predecessor
+// that published its inclusive prefix ends the walk, one that published only its histogram
+// adds it and the walk goes on), published as the inclusive prefix; the block that finishes
+// last then forms the pass's totals. A block only ever waits for blocks that took earlier
+// tickets, which are resident or done, so the waits end; each is bounded all the same
+// (MOE_ERR_DEVICE_TIMEOUT). The scan stays deterministic: positions are exact counts.
+__global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(HistArgs p)
 {
-    extern __shared__ __align__(16) int pos_smem[];
+    extern __shared__ __align__(16) unsigned char hist_smem[];
+    int *s_hist = reinterpret_cast<int *>(hist_smem);
+    __shared__ int s_vb, s_last;
     const int E = p.E;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int *wcnt = pos_smem;
-    int *s_off = wcnt + 8 * E;
-
-    int t0, t1, k, round;
-    p.vbm.range(blockIdx.x, t0, t1, k, round);
-    const int32_t *src = p.vbm.experts(p.topk_idx, round);
-    const int na = p.vbm.count(t0, t1);
-    const int per = (na + 7) / 8;
-    const int wb = min(na, warp * per), we = min(na, wb + per);
-
-    for (int i = threadIdx.x; i < 8 * E; i += blockDim.x)
-        wcnt[i] = 0;
-    for (int e = threadIdx.x; e < E; e += blockDim.x)
-        s_off[e] = p.offsets[e];
+    if (threadIdx.x == 0)
+        s_vb = (int)atomicAdd(&p.ctl[0], 1u);
+    for (int e = threadIdx.x; e < E; e += kHistThreads)
+        s_hist[e] = 0;
     __syncthreads();
-    for (int i = wb + lane; i < we; i += 32) {
+    const int vb = s_vb;
+    int t0, t1, k, round;
+    p.vbm.range(vb, t0, t1, k, round);
+    const int32_t *src = p.vbm.experts(p.topk_idx, round);
+    const int n = p.vbm.count(t0, t1);
+    for (int i = threadIdx.x; i < n; i += kHistThreads) {
         const int e = src[p.vbm.assign(t0, k, i)];
         if ((unsigned)e < (unsigned)E)
-            atomicAdd(&wcnt[warp * E + e], 1);
+            atomicAdd(&s_hist[e], 1);
+        else if (round == 0)
+            set_dev_error(MOE_ERR_DEVICE_BOUNDS);  // round 1 marks "not moved" with -1
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = p.blk[(size_t)e * p.nvb + blockIdx.x];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const int c = wcnt[w * E + e];
-            wcnt[w * E + e] = run;
-            run += c;
+    unsigned int *flags = p.ctl + 2;
+    for (int e = threadIdx.x; e < E; e += kHistThreads)
+        p.agg[(size_t)vb * E + e] = s_hist[e];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        st_release_u32(&flags[vb], kFlagAgg);
+    for (int e = threadIdx.x; e < E; e += kHistThreads) {
+        int excl = 0;
+        for (int q = vb - 1; q >= 0; --q) {
+            unsigned int f = ld_acquire_u32(&flags[q]);
+            if (f == 0) {
+                const uint64_t w0 = global_timer_ns();
+                while ((f = ld_acquire_u32(&flags[q])) == 0) {
+                    if (global_timer_ns() - w0 > p.timeout_ns) {
+                        set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+                        break;
+                    }
+                }
+                if (f == 0)
+                    break;  // gave up (the error is recorded)
+            }
+            if (f == kFlagIncl) {
+                excl += __ldcg(p.incl + (size_t)q * E + e);
+                break;
+            }
+            excl += __ldcg(p.agg + (size_t)q * E + e);
         }
+        p.incl[(size_t)vb * E + e] = excl + s_hist[e];
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        st_release_u32(&flags[vb], kFlagIncl);
+        __threadfence();
+        s_last = atomicAdd(&p.ctl[1], 1u) == (unsigned int)(p.nvb - 1);
     }
     __syncthreads();
+    if (!s_last)
+        return;
+    __threadfence();
+    pass_totals(p, hist_smem);
+}
 
+constexpr int kPlaceThreads = 256;
+
+struct PlaceArgs {
+    const int32_t *topk_idx;
+    VBlocks vbm;
+    int rounds;
+    int bps;          // virtual blocks per segment (a token block's segment: vb / bps)
+    int E, K, W, C;
+    const int32_t *agg, *incl;  // [nvb][E]
+    const int32_t *offsets;     // [E+1]
+    const int64_t *pk_base;     // [nseg][E]
+    int32_t *row_of, *assign_of_row;
+    int32_t *expert_of;         // nullable: the expert whose row each assignment uses, or -1
+    // the copy of the rows (copy != 0)
+    int copy;
+    int e4m3;
+    const uint16_t *x;
+    int d;
+    void *x_sorted, *x_packed;          // bf16 rows, or e4m3 rows with the FP8 payload
+    float *sorted_scale, *packed_scale;  // FP8 payload: one scale per row
+    moe_stats_t *stats;                  // nullable: dedup_pairs is accumulated here
+};
+
+// Shared memory of dispatch_place_kernel: per-warp counts [8][E] and offsets [E+1] (int32),
+// then the expert-sorted row, the packed row and the expert of each of the token block's
+// HB * K slots (int32 each).
+__host__ __device__ inline size_t place_smem_bytes(int E, int K)
+{
+    return ((size_t)9 * E + 1 + (size_t)3 * kDispatchHB * K) * 4;
+}
+
+// One CTA per (token block, part). Positions: for every virtual block of the token block (all
+// rounds; each slot k in slot-major order), warps count their sub-ranges per expert, take
+// their bases from the block's exclusive prefix (inclusive minus own), and rank equal experts
+// with __match_any_sync, which gives the sequential first-come position exactly; the
+// mapping table (row_of, assign_of_row, expert_of) is written by part 0. Each assignment's
+// row is decided by exactly one virtual block: its round-0 block unless it was moved, then
+// its round-1 block. Copy: part p of the token block's rows (a column slice of every bf16
+// row; whole rows of a share of the tokens for the FP8 payload, whose scale needs the row)
+// goes to every kept slot's expert-sorted row and, when requested, its packed row.
+__global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs p)
+{
+    extern __shared__ __align__(16) int place_smem[];
+    const int E = p.E, K = p.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int *wcnt = place_smem;
+    int *s_off = wcnt + 8 * E;
+    int *s_rk = s_off + E + 1;
+    int *s_pk = s_rk + kDispatchHB * K;
+    int *s_ex = s_pk + kDispatchHB * K;
+    const int tb = blockIdx.x, part = blockIdx.y, parts = gridDim.y;
+    int t0, t1;
+    p.vbm.bm.range(tb, t0, t1);
+    const int nt = t1 - t0;
+    for (int i = threadIdx.x; i < nt * K; i += kPlaceThreads) {
+        s_rk[i] = -1;
+        s_pk[i] = -1;
+        s_ex[i] = -1;
+    }
+    for (int e = threadIdx.x; e <= E; e += kPlaceThreads)
+        s_off[e] = p.offsets[e];
     unsigned lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
-    for (int g = wb; g < we; g += 32) {
-        const int i = g + lane;
-        const bool act = i < we;
-        const int a = act ? p.vbm.assign(t0, k, i) : 0;
-        int e = act ? src[a] : -1;
-        if ((unsigned)e >= (unsigned)E)
-            e = -1;
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const int rank = __popc(peers & lt_mask);
-        const int base = e >= 0 ? wcnt[warp * E + e] : 0;
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(peers) - 1)
-            wcnt[warp * E + e] = base + __popc(peers);
-        __syncwarp();
-        if (act) {
-            const int pos = base + rank;
-            const int row = (e >= 0 && pos < p.C) ? s_off[e] + pos : -1;
-            const bool owner = round ? e >= 0
-                                     : (row >= 0 || p.vbm.moved == nullptr || p.vbm.moved[a] < 0);
-            if (owner)
-                p.row_of[a] = row;
-            if (row >= 0)
-                p.assign_of_row[row] = a;
+    const int nsub = p.vbm.slot_major ? K : 1;
+    for (int round = 0; round < p.rounds; ++round) {
+        const int32_t *src = p.vbm.experts(p.topk_idx, round);
+        for (int kk = 0; kk < nsub; ++kk) {
+            const int vb = round * p.vbm.nvb_round + (p.vbm.slot_major ? kk * p.vbm.nblk_tok : 0) + tb;
+            const int g = vb / p.bps;
+            const int na = p.vbm.count(t0, t1);
+            const int per = (na + 7) / 8;
+            const int wb = min(na, warp * per), we = min(na, wb + per);
+            for (int i = threadIdx.x; i < 8 * E; i += kPlaceThreads)
+                wcnt[i] = 0;
+            __syncthreads();
+            for (int i = wb + lane; i < we; i += 32) {
+                const int e = src[p.vbm.assign(t0, kk, i)];
+                if ((unsigned)e < (unsigned)E)
+                    atomicAdd(&wcnt[warp * E + e], 1);
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < E; e += kPlaceThreads) {
+                const size_t o = (size_t)vb * E + e;
+                int run = __ldcg(p.incl + o) - __ldcg(p.agg + o);
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    const int c = wcnt[w * E + e];
+                    wcnt[w * E + e] = run;
+                    run += c;
+                }
+            }
+            __syncthreads();
+            for (int g0 = wb; g0 < we; g0 += 32) {
+                const int i = g0 + lane;
+                const bool act = i < we;
+                const int a = act ? p.vbm.assign(t0, kk, i) : 0;
+                int e = act ? src[a] : -1;
+                if ((unsigned)e >= (unsigned)E)
+                    e = -1;
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                const int rank = __popc(peers & lt_mask);
+                const int base = e >= 0 ? wcnt[warp * E + e] : 0;
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1)
+                    wcnt[warp * E + e] = base + __popc(peers);
+                __syncwarp();
+                if (act) {
+                    const int pos = base + rank;
+                    // kept iff pos < C; a kept position is always below the expert's kept
+                    // count, which the second test restates so that no row outside the
+                    // expert's range is ever written, whatever the prefixes held
+                    const int row = (e >= 0 && pos < p.C && s_off[e] + pos < s_off[e + 1])
+                                        ? s_off[e] + pos : -1;
+                    const bool owner = round ? e >= 0
+                                             : (row >= 0 || p.vbm.moved == nullptr ||
+                                                p.vbm.moved[a] < 0);
+                    if (owner) {
+                        const int ls = a - t0 * K;
+                        s_rk[ls] = row;
+                        s_ex[ls] = row >= 0 ? e : -1;
+                        const int64_t pk = p.pk_base[(size_t)g * E + e] + pos;
+                        s_pk[ls] = (row >= 0 && p.x_packed && pk >= 0 && pk < s_off[E])
+                                       ? (int)pk : -1;
+                        if (row >= 0 && part == 0)
+                            p.assign_of_row[row] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (part == 0) {
+        for (int i = threadIdx.x; i < nt * K; i += kPlaceThreads) {
+            p.row_of[t0 * K + i] = s_rk[i];
+            if (p.expert_of)
+                p.expert_of[t0 * K + i] = s_ex[i];
+        }
+        if (p.stats) {
+            // distinct destination ranks other than the token's home over its kept slots
+            const int e_per = E / p.W;
+            const int home = tb / p.vbm.bm.bps;
+            unsigned long long pairs = 0;
+            for (int lt = warp; lt < nt; lt += 8) {
+                const int ex = lane < K ? s_ex[lt * K + lane] : -1;
+                const int dest = ex >= 0 ? ex / e_per : -1;
+                const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
+                const unsigned grp = __match_any_sync(0xffffffffu, key);
+                pairs += __popc(__ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0));
+            }
+            if (lane == 0 && pairs)
+                atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
+        }
+    }
+    if (!p.copy)
+        return;
+
+    if (!p.e4m3) {
+        // a column slice of every row of the block: `cs` 16-byte chunks from cbeg
+        constexpr int U = 4;
+        const int nvec = p.d >> 3;
+        const int cs = (nvec + parts - 1) / parts;
+        const int cbeg = part * cs, cend = min(nvec, cbeg + cs);
+        uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
+        uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
+        for (int lt = warp; lt < nt; lt += 8) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + lt) * p.d);
+            const int *rk_l = s_rk + lt * K;
+            const int *pk_l = s_pk + lt * K;
+            for (int c0 = cbeg; c0 < cend; c0 += 32 * U) {
+                const int c = c0 + lane;
+                uint4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (c + 32 * u < cend)
+                        v[u] = __ldcs(src + c + 32 * u);
+                for (int k = 0; k < K; ++k) {
+                    const int rk = rk_l[k];
+                    if (rk < 0)
+                        continue;
+                    const int pk = pk_l[k];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (c + 32 * u < cend) {
+                            dst_s[(size_t)rk * nvec + c + 32 * u] = v[u];
+                            if (pk >= 0)
+                                dst_p[(size_t)pk * nvec + c + 32 * u] = v[u];
+                        }
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // FP8 payload ([MoE 推理服务工程真相 2026, §6.3]: the token rows that cross the
+    // all-to-all travel as FP8): one warp per token reads its bf16 row twice (the second pass
+    // hits L1/L2), first for the largest magnitude, then to write e4m3 codes (row scaled by
+    // 2^-j, the row's power-of-two scale) to every kept slot's sorted and packed row, with the
+    // scale 2^j beside each row. This part takes the tokens part, part + parts, ... of the block.
+    const int n16 = p.d >> 4;  // 16-element chunks: two 16-byte loads, one 16-byte store
+    uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
+    uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
+    for (int lt = part + parts * warp; lt < nt; lt += parts * 8) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + lt) * p.d);
+        const int *rk_l = s_rk + lt * K;
+        const int *pk_l = s_pk + lt * K;
+        // pass 1: largest magnitude of the row (bf16 bits with the sign cleared order like the
+        // magnitudes; a NaN marks the row non-finite)
+        uint32_t mx = 0;
+        for (int c = lane; c < 2 * n16; c += 32) {
+            const uint4 v = src[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                mx = max(mx, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        const float amax = __uint_as_float(mx << 16);  // NaN bits sort above Inf
+        const int j = e4m3_scale_exp(amax);
+        const float inv = pow2f(-j), scale = pow2f(j);
+        if (lane < K) {
+            const int rk = rk_l[lane], pk = pk_l[lane];
+            if (rk >= 0) {
+                p.sorted_scale[rk] = scale;
+                if (pk >= 0)
+                    p.packed_scale[pk] = scale;
+            }
+        }
+        // pass 2
+        for (int c = lane; c < n16; c += 32) {
+            const uint4 a = src[2 * c], b = src[2 * c + 1];
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t lo = pack_e4m3x2(bf16_lo(w[2 * i]) * inv, bf16_hi(w[2 * i]) * inv);
+                const uint32_t hi =
+                    pack_e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv);
+                o[i] = lo | (hi << 16);
+            }
+            const uint4 q = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int k = 0; k < K; ++k) {
+                const int rk = rk_l[k];
+                if (rk < 0)
+                    continue;
+                dst_s[(size_t)rk * n16 + c] = q;
+                const int pk = pk_l[k];
+                if (pk >= 0)
+                    dst_p[(size_t)pk * n16 + c] = q;
+            }
         }
     }
 }
@@ -495,199 +685,6 @@ __global__ void __launch_bounds__(256) reroute_kernel(RerouteArgs p)
         if (lane < p.K)
             p.moved[t * p.K + lane] = res;
     }
-}
-
-struct ScatterArgs {
-    const uint16_t *x;
-    const int32_t *topk_idx;
-    const int32_t *row_of;
-    const int32_t *offsets;
-    const int64_t *pk_base;  // [E][nseg]
-    const int32_t *moved;    // round-1 expert per assignment, or null
-    int N, d, K, W, E;
-    int S;           // N / W
-    int slot_major;  // segment of (t, k) in its round: k*W + t/S, else t/S
-    int nseg;        // all rounds
-    int nseg_round;
-    int32_t *expert_of;  // nullable out: the expert whose row each assignment uses, or -1
-    int seg;             // bf16 scatter: 16-byte chunks per work item (whole row for large N)
-    void *x_sorted;      // bf16 rows, or e4m3 rows with fp8 payload
-    void *x_packed;      // nullable, same element type
-    float *sorted_scale;  // e4m3 payload: scale of each x_sorted row
-    float *packed_scale;  // e4m3 payload: scale of each x_packed row (nullable)
-    moe_stats_t *stats;  // nullable: dedup_pairs is accumulated here
-};
-
-// Targets of slot `lane` (lanes < K) of token t: its expert-sorted row r (-1 if
-// dropped) and packed row pk (-1 if dropped or not packing). When `first` (the
-// token's first work item): also writes expert_of and returns the number of
-// distinct non-home destination ranks of the token (the same value in every lane),
-// when counting.
-__device__ __forceinline__ int slot_targets(const ScatterArgs &p, int t, int lane,
-                                            unsigned lt_mask, int &r, long long &pk,
-                                            bool first = true)
-{
-    const int e_per = p.E / p.W;
-    const int home = t / p.S;
-    int dest = -1;
-    r = -1;
-    pk = -1;
-    if (lane < p.K) {
-        const int a = t * p.K + lane;
-        r = p.row_of[a];
-        int ef = -1;
-        if (r >= 0) {
-            const int em = p.moved ? p.moved[a] : -1;
-            const int e = em >= 0 ? em : p.topk_idx[a];
-            ef = e;
-            dest = e / e_per;
-            if (p.x_packed) {
-                const int g = (em >= 0 ? p.nseg_round : 0) +
-                              (p.slot_major ? lane * p.W + home : home);
-                pk = p.pk_base[(size_t)e * p.nseg + g] + (r - p.offsets[e]);
-            }
-        }
-        if (p.expert_of && first)
-            p.expert_of[a] = ef;
-    }
-    if (!p.stats || !first)
-        return 0;
-    // distinct non-home destinations: count the lowest lane of each group
-    const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
-    const unsigned grp = __match_any_sync(0xffffffffu, key);
-    return __popc(__ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0));
-}
-
-// One warp per work item (a token and `seg` 16-byte chunks of its row: the whole
-// row unless there are too few tokens to fill the GPU): read the token's row once
-// (16-byte loads), write it to each kept slot's expert-sorted row and, when
-// requested, to its packed row. The token's distinct destination ranks other than
-// its home (over kept slots) are counted into stats->dedup_pairs.
-__global__ void __launch_bounds__(256) scatter_rows_kernel(ScatterArgs p)
-{
-    constexpr int U = 4;
-    const int lane = threadIdx.x & 31;
-    const int nvec = p.d >> 3;
-    const int nseg = (nvec + p.seg - 1) / p.seg;
-    const int64_t items = (int64_t)p.N * nseg;
-    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    unsigned lt_mask;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
-    unsigned long long pairs = 0;
-    for (int64_t item = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-         item < items; item += nwarps) {
-        const int t = (int)(item / nseg);
-        const int sidx = (int)(item % nseg);
-        const int cbeg = sidx * p.seg, cend = min(nvec, cbeg + p.seg);
-        int r;
-        long long pk;
-        pairs += slot_targets(p, t, lane, lt_mask, r, pk, sidx == 0);
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
-        uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
-        uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
-        // every lane runs every iteration: the shuffles below read lanes 0..K-1
-        for (int c0 = cbeg; c0 < cend; c0 += 32 * U) {
-            const int c = c0 + lane;
-            uint4 v[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (c + 32 * u < cend)
-                    v[u] = __ldcs(src + c + 32 * u);
-            for (int k = 0; k < p.K; ++k) {
-                const int rk = __shfl_sync(0xffffffffu, r, k);
-                const long long pkk = __shfl_sync(0xffffffffu, pk, k);
-                if (rk < 0)
-                    continue;
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    if (c + 32 * u < cend) {
-                        dst_s[(size_t)rk * nvec + c + 32 * u] = v[u];
-                        if (pkk >= 0)
-                            dst_p[(size_t)pkk * nvec + c + 32 * u] = v[u];
-                    }
-                }
-            }
-        }
-    }
-    if (p.stats && lane == 0 && pairs)
-        atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
-}
-
-// FP8 payload ([MoE 推理服务工程真相 2026, §6.3]: the token rows that cross the
-// all-to-all travel as FP8): one warp per token reads its bf16 row twice (the
-// second pass hits L1/L2), first for the largest magnitude, then to write e4m3
-// codes (row scaled by 2^-j, the row's power-of-two scale) to every kept slot's
-// sorted and packed row, with the scale 2^j beside each row. d % 16 == 0.
-__global__ void __launch_bounds__(256) scatter_rows_e4m3_kernel(ScatterArgs p)
-{
-    const int lane = threadIdx.x & 31;
-    const int n16 = p.d >> 4;  // 16-element chunks: two 16-byte loads, one 16-byte store
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
-    unsigned lt_mask;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
-    unsigned long long pairs = 0;
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < p.N; t += nwarps) {
-        int r;
-        long long pk;
-        pairs += slot_targets(p, t, lane, lt_mask, r, pk);
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)t * p.d);
-        // pass 1: largest magnitude of the row (bf16 bits with the sign cleared
-        // order like the magnitudes; a NaN marks the row non-finite)
-        uint32_t mx = 0;
-        for (int c = lane; c < 2 * n16; c += 32) {
-            const uint4 v = src[c];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                mx = max(mx, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1)
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float amax = __uint_as_float(mx << 16);  // NaN bits sort above Inf
-        const int j = e4m3_scale_exp(amax);
-        const float inv = pow2f(-j), scale = pow2f(j);
-        for (int k = 0; k < p.K; ++k) {
-            const int rk = __shfl_sync(0xffffffffu, r, k);
-            const long long pkk = __shfl_sync(0xffffffffu, pk, k);
-            if (lane == 0 && rk >= 0) {
-                p.sorted_scale[rk] = scale;
-                if (pkk >= 0)
-                    p.packed_scale[pkk] = scale;
-            }
-        }
-        uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
-        uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
-        // pass 2: every lane runs every iteration (the shuffles read lanes 0..K-1)
-        for (int c0 = 0; c0 < n16; c0 += 32) {
-            const int c = c0 + lane;
-            uint4 q = make_uint4(0, 0, 0, 0);
-            if (c < n16) {
-                const uint4 a = src[2 * c], b = src[2 * c + 1];
-                const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t lo = pack_e4m3x2(bf16_lo(w[2 * i]) * inv, bf16_hi(w[2 * i]) * inv);
-                    const uint32_t hi =
-                        pack_e4m3x2(bf16_lo(w[2 * i + 1]) * inv, bf16_hi(w[2 * i + 1]) * inv);
-                    o[i] = lo | (hi << 16);
-                }
-                q = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-            for (int k = 0; k < p.K; ++k) {
-                const int rk = __shfl_sync(0xffffffffu, r, k);
-                const long long pkk = __shfl_sync(0xffffffffu, pk, k);
-                if (rk < 0 || c >= n16)
-                    continue;
-                dst_s[(size_t)rk * n16 + c] = q;
-                if (pkk >= 0)
-                    dst_p[(size_t)pkk * n16 + c] = q;
-            }
-        }
-    }
-    if (p.stats && lane == 0 && pairs)
-        atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
 }
 
 // Row-wise e4m3 quantisation of a bf16 matrix (for the experts' W1 and W3): one

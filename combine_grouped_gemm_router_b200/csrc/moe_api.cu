@@ -37,20 +37,7 @@ struct Geometry {
     int rounds;          // 2 when overflowed assignments are re-routed
     int nvb_round, nseg_round;  // virtual blocks and segments of one round
     int nvb, nseg;       // ... of all rounds
-    bool cum_in_smem;    // the scan's per-segment starts fit in shared memory
 };
-
-constexpr size_t kScanSmemLimit = 200 * 1024;
-
-// Shared memory of dispatch_scan_kernel without / with the per-segment starts.
-size_t scan_smem_base(const moe_shape_t *s)
-{
-    const int E = s->E, W = s->W;
-    const int scan_len = (E > W * W ? E : W * W) + 1;
-    return (size_t)scan_len * 8 + (size_t)W * W * 8 + 32 * 8 + (size_t)E * W * 4;
-}
-
-size_t scan_cum_bytes(const moe_shape_t *s, int nseg) { return (size_t)s->E * (nseg + 1) * 4; }
 
 int64_t capacity_of(const moe_shape_t *s)
 {
@@ -104,27 +91,30 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
         g->nseg_round = g->slot_major ? s->K * s->W : s->W;
         g->nvb = g->rounds * g->nvb_round;
         g->nseg = g->rounds * g->nseg_round;
-        g->cum_in_smem = scan_smem_base(s) + scan_cum_bytes(s, g->nseg) <= kScanSmemLimit;
     }
     return MOE_OK;
 }
 
 // Route/dispatch scratch, carved in this order from the workspace.
 struct ScratchLayout {
-    size_t logits, blk, pk_base, cum, moved, D, pk_off, total;
+    size_t logits, ctl, agg, incl, pk_base, moved, D, pk_off, total;
 };
 
-// The dispatch's own scratch (block bases, pack bases, segment starts when they
-// do not fit in shared memory, traffic matrix, pack offsets), from offset o.
+// The dispatch's own scratch, from offset o: the pass's control words (ticket, finished
+// blocks, one flag per virtual block), the blocks' histograms and inclusive prefixes
+// [nvb][E], the pack bases [nseg][E], the moved-to expert of each assignment (re-routing),
+// the traffic matrix and the pack offsets (when the caller does not want them).
 template <typename Layout>
 size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layout &L)
 {
-    L.blk = o;
+    L.ctl = o;
+    o = align_up(o + ((size_t)g.nvb + 2) * 4);
+    L.agg = o;
+    o = align_up(o + (size_t)s->E * g.nvb * 4);
+    L.incl = o;
     o = align_up(o + (size_t)s->E * g.nvb * 4);
     L.pk_base = o;
     o = align_up(o + (size_t)s->E * g.nseg * 8);
-    L.cum = o;  // the scan's segment starts, when not in shared memory or pre-scanned
-    o = align_up(o + scan_cum_bytes(s, g.nseg));
     L.moved = o;
     if (g.rounds > 1)
         o = align_up(o + (size_t)s->N * s->K * 4);
@@ -283,11 +273,38 @@ void launch_logits_pairs(const uint16_t *x, const float *wr, const float *bias, 
         <<<grid, L::NT, L::SMEM_BYTES, st>>>(x, wr, bias, logits, N, d, E);
 }
 
-moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_router,
-                        const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+template <int NW>
+void launch_router_topk(const moe_shape_t *s, const uint16_t *x, const float *wr, const float *bias,
+                        int32_t *topk_idx, float *topk_w, float *logits,
                         unsigned long long *nonfinite, cudaStream_t st)
 {
+    using L = RouterTopkTile<NW>;
+    smem_attr_once(router_topk_kernel<NW>, L::SMEM_BYTES);
+    router_topk_kernel<NW><<<(s->N + kRtTokens - 1) / kRtTokens, L::NT, L::SMEM_BYTES, st>>>(
+        x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
+}
+
+// The router projection and the top-K selection. logits_out (nullable) receives the [N][E]
+// logits; scratch ([N][E] fp32) is used when the two steps run as separate kernels.
+moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_router,
+                        const float *bias, int32_t *topk_idx, float *topk_w, float *logits_out,
+                        float *scratch, unsigned long long *nonfinite, cudaStream_t st)
+{
     const int N = s->N, d = s->d, E = s->E;
+    // Many tokens and E >= 32: the projection and the selection in one kernel (64 tokens x
+    // every expert per CTA; the logits reach HBM only when asked for).
+    if (E >= 32 && N >= 2048) {
+        if (E <= 32)
+            launch_router_topk<2>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+        else if (E <= 64)
+            launch_router_topk<4>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+        else if (E <= 128)
+            launch_router_topk<8>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+        else
+            launch_router_topk<16>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+        return launch_status();
+    }
+    float *logits = logits_out ? logits_out : scratch;
     // Tile choice. Each output is one dependent chain of d fused multiply-adds, so
     // the floor is d x (fma latency). Few outputs (small N or small E): one chain per
     // thread and many warps per SM, so latency, not issue, is the limit. Many outputs
@@ -317,68 +334,6 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
 
 // ---------------------------------------------------------------- dispatch
 
-// Histogram, scan and positions over `rounds` rounds of virtual blocks.
-void dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds, const int32_t *moved,
-                   const int32_t *topk_idx, int32_t *counts, int32_t *kept, int32_t *offsets,
-                   int32_t *row_of, int32_t *assign_of_row, int64_t *D, int64_t *pk_off,
-                   moe_stats_t *stats, int32_t *blk, int64_t *pk_base, int32_t *cum,
-                   cudaStream_t st)
-{
-    VBlocks vbm;
-    vbm.bm = BlockMap{g.S, g.bps, kDispatchHB};
-    vbm.nblk_tok = g.nblk;
-    vbm.slot_major = g.slot_major;
-    vbm.K = s->K;
-    vbm.nvb_round = g.nvb_round;
-    vbm.moved = moved;
-    const int nvb = rounds * g.nvb_round, nseg = rounds * g.nseg_round;
-    block_hist_kernel<<<nvb, 256, s->E * 4, st>>>(topk_idx, s->E, vbm, nvb, blk);
-
-    // many blocks per expert: scan each expert's row in its own CTA first
-    const bool prescan = nvb > 128;
-    if (prescan)
-        expert_block_scan_kernel<<<s->E, 256, 0, st>>>(blk, nvb, g.bps, nseg, cum);
-    const bool cum_in_smem =
-        !prescan && scan_smem_base(s) + scan_cum_bytes(s, nseg) <= kScanSmemLimit;
-    ScanArgs sa;
-    sa.blk = blk;
-    sa.nvb = nvb;
-    sa.bps = g.bps;
-    sa.nseg = nseg;
-    sa.nseg_round = g.nseg_round;
-    sa.N = s->N;
-    sa.E = s->E;
-    sa.K = s->K;
-    sa.W = s->W;
-    sa.C = (int)g.C;
-    sa.cum_global = cum_in_smem ? nullptr : cum;
-    sa.prescanned = prescan ? 1 : 0;
-    sa.counts = counts;
-    sa.kept = kept;
-    sa.offsets = offsets;
-    sa.D = D;
-    sa.pk_off = pk_off;
-    sa.pk_base = pk_base;
-    sa.stats = stats;
-    const size_t scan_smem = scan_smem_base(s) + (cum_in_smem ? scan_cum_bytes(s, nseg) : 0);
-    smem_attr_once(dispatch_scan_kernel, (int)kScanSmemLimit);
-    dispatch_scan_kernel<<<1, 1024, scan_smem, st>>>(sa);
-
-    PosArgs pa;
-    pa.topk_idx = topk_idx;
-    pa.blk = blk;
-    pa.nvb = nvb;
-    pa.vbm = vbm;
-    pa.E = s->E;
-    pa.C = (int)g.C;
-    pa.offsets = offsets;
-    pa.row_of = row_of;
-    pa.assign_of_row = assign_of_row;
-    const size_t pos_smem = (size_t)9 * s->E * 4;
-    dispatch_positions_kernel<<<nvb, 256, pos_smem, st>>>(pa);
-}
-
-// logits: needed when g.rounds == 2 (re-routing); moved: N*K int32 scratch then.
 // Row payload of the scatter: bf16 rows, or e4m3 rows with a scale per row.
 struct Payload {
     void *x_sorted;
@@ -388,19 +343,134 @@ struct Payload {
     float *packed_scale;  // e4m3 with x_packed only
 };
 
+// The dispatch's scratch pointers (inside a workspace or the static array).
+struct DispatchScratch {
+    unsigned int *ctl;
+    int32_t *agg, *incl;
+    int64_t *pk_base;
+    int32_t *moved;
+};
+
+// Column (bf16) or token (FP8) parts per token block of the placement kernel: enough CTAs for
+// about two per SM, each part at least 64 16-byte chunks of a row (or one token per warp).
+int place_parts(const moe_shape_t *s, const Geometry &g, bool e4m3)
+{
+    const int want = (2 * num_sms() + g.nblk - 1) / g.nblk;
+    const int cap = e4m3 ? (kDispatchHB + 7) / 8 : ((s->d / 8) + 63) / 64;
+    const int parts = want < cap ? want : cap;
+    return parts < 1 ? 1 : parts;
+}
+
+// One dispatch pass over `rounds` rounds of virtual blocks: the control words zeroed, the
+// histogram / look-back / totals kernel, then the placement kernel (positions, the mapping
+// table and, when `pay` is given, the copy of the rows).
+moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
+                           const int32_t *moved, const int32_t *topk_idx, int32_t *counts,
+                           int32_t *kept, int32_t *offsets, int32_t *row_of,
+                           int32_t *assign_of_row, int32_t *expert_of, const Payload *pay,
+                           const uint16_t *x, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
+                           const DispatchScratch &sc, cudaStream_t st)
+{
+    VBlocks vbm;
+    vbm.bm = BlockMap{g.S, g.bps, kDispatchHB};
+    vbm.nblk_tok = g.nblk;
+    vbm.slot_major = g.slot_major;
+    vbm.K = s->K;
+    vbm.nvb_round = g.nvb_round;
+    vbm.moved = moved;
+    const int nvb = rounds * g.nvb_round, nseg = rounds * g.nseg_round;
+    if (cudaMemsetAsync(sc.ctl, 0, ((size_t)nvb + 2) * 4, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    HistArgs ha;
+    ha.topk_idx = topk_idx;
+    ha.vbm = vbm;
+    ha.nvb = nvb;
+    ha.bps = g.bps;
+    ha.nseg = nseg;
+    ha.nseg_round = g.nseg_round;
+    ha.N = s->N;
+    ha.E = s->E;
+    ha.K = s->K;
+    ha.W = s->W;
+    ha.C = (int)g.C;
+    ha.ctl = sc.ctl;
+    ha.agg = sc.agg;
+    ha.incl = sc.incl;
+    ha.counts = counts;
+    ha.kept = kept;
+    ha.offsets = offsets;
+    ha.D = D;
+    ha.pk_off = pk_off;
+    ha.pk_base = sc.pk_base;
+    ha.stats = stats;
+    ha.timeout_ns = kWaitTimeoutNs;
+    const size_t hsm = hist_smem_bytes(s->E, s->W);
+    if (smem_attr_once(dispatch_hist_kernel, (int)hist_smem_bytes(kMaxE, kMaxW)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dispatch_hist_kernel<<<nvb, kHistThreads, hsm, st>>>(ha);
+
+    PlaceArgs pa = {};
+    pa.topk_idx = topk_idx;
+    pa.vbm = vbm;
+    pa.rounds = rounds;
+    pa.bps = g.bps;
+    pa.E = s->E;
+    pa.K = s->K;
+    pa.W = s->W;
+    pa.C = (int)g.C;
+    pa.agg = sc.agg;
+    pa.incl = sc.incl;
+    pa.offsets = offsets;
+    pa.pk_base = sc.pk_base;
+    pa.row_of = row_of;
+    pa.assign_of_row = assign_of_row;
+    pa.expert_of = expert_of;
+    pa.stats = stats;
+    pa.x = x;
+    pa.d = s->d;
+    int parts = 1;
+    if (pay) {
+        pa.copy = 1;
+        pa.e4m3 = pay->e4m3 ? 1 : 0;
+        pa.x_sorted = pay->x_sorted;
+        pa.x_packed = pay->x_packed;
+        pa.sorted_scale = pay->sorted_scale;
+        pa.packed_scale = pay->packed_scale;
+        parts = place_parts(s, g, pay->e4m3);
+    }
+    const size_t psm = place_smem_bytes(s->E, s->K);
+    if (smem_attr_once(dispatch_place_kernel, (int)place_smem_bytes(kMaxE, kMaxK)) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    dispatch_place_kernel<<<dim3(g.nblk, parts), kPlaceThreads, psm, st>>>(pa);
+    return launch_status();
+}
+
+template <typename Layout>
+DispatchScratch scratch_at(char *w, const Layout &L)
+{
+    return DispatchScratch{reinterpret_cast<unsigned int *>(w + L.ctl),
+                           reinterpret_cast<int32_t *>(w + L.agg),
+                           reinterpret_cast<int32_t *>(w + L.incl),
+                           reinterpret_cast<int64_t *>(w + L.pk_base),
+                           reinterpret_cast<int32_t *>(w + L.moved)};
+}
+
+// logits: needed when g.rounds == 2 (re-routing); the moved-to experts then go to sc.moved.
 moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x,
                            const float *logits, const int32_t *topk_idx, int32_t *counts,
                            int32_t *kept, int32_t *offsets, int32_t *row_of,
                            int32_t *assign_of_row, int32_t *expert_of, const Payload &pay,
                            int64_t *D, int64_t *pk_off, moe_stats_t *stats,
-                           int32_t *blk, int64_t *pk_base, int32_t *cum, int32_t *moved,
-                           cudaStream_t st)
+                           const DispatchScratch &sc, cudaStream_t st)
 {
     const int32_t *round1 = nullptr;
     if (g.rounds > 1) {
-        // round 0 alone: which assignments are past capacity
-        dispatch_pass(s, g, 1, nullptr, topk_idx, counts, kept, offsets, row_of, assign_of_row,
-                      nullptr, nullptr, nullptr, blk, pk_base, cum, st);
+        // round 0 alone: which assignments are past capacity (positions only, no copy)
+        moe_status_t rc = dispatch_pass(s, g, 1, nullptr, topk_idx, counts, kept, offsets,
+                                        row_of, assign_of_row, nullptr, nullptr, x, D, pk_off,
+                                        nullptr, sc, st);
+        if (rc != MOE_OK)
+            return rc;
         RerouteArgs ra;
         ra.logits = logits;
         ra.topk_idx = topk_idx;
@@ -410,43 +480,12 @@ moe_status_t dispatch_impl(const moe_shape_t *s, const Geometry &g, const uint16
         ra.E = s->E;
         ra.K = s->K;
         ra.C = (int)g.C;
-        ra.moved = moved;
+        ra.moved = sc.moved;
         reroute_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ra);
-        round1 = moved;
+        round1 = sc.moved;
     }
-    dispatch_pass(s, g, g.rounds, round1, topk_idx, counts, kept, offsets, row_of, assign_of_row,
-                  D, pk_off, stats, blk, pk_base, cum, st);
-
-    ScatterArgs ca;
-    ca.x = x;
-    ca.topk_idx = topk_idx;
-    ca.row_of = row_of;
-    ca.offsets = offsets;
-    ca.pk_base = pk_base;
-    ca.moved = round1;
-    ca.N = s->N;
-    ca.d = s->d;
-    ca.K = s->K;
-    ca.W = s->W;
-    ca.E = s->E;
-    ca.S = g.S;
-    ca.slot_major = g.slot_major;
-    ca.nseg = g.nseg;
-    ca.nseg_round = g.nseg_round;
-    ca.expert_of = expert_of;
-    ca.x_sorted = pay.x_sorted;
-    ca.x_packed = pay.x_packed;
-    ca.sorted_scale = pay.sorted_scale;
-    ca.packed_scale = pay.packed_scale;
-    ca.stats = stats;
-    if (pay.e4m3) {
-        ca.seg = s->d / 8;  // one token row per warp (its maximum is taken over the row)
-        scatter_rows_e4m3_kernel<<<(s->N + 7) / 8, 256, 0, st>>>(ca);
-    } else {
-        ca.seg = row_slice(s->N, s->d / 8, 128);
-        scatter_rows_kernel<<<row_blocks(s->N, s->d / 8, ca.seg), 256, 0, st>>>(ca);
-    }
-    return launch_status();
+    return dispatch_pass(s, g, g.rounds, round1, topk_idx, counts, kept, offsets, row_of,
+                         assign_of_row, expert_of, &pay, x, D, pk_off, stats, sc, st);
 }
 
 // ---------------------------------------------------------------- expert GEMMs
@@ -921,15 +960,16 @@ moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
     if (!aligned16(x) || !aligned16(w_router) || (bias && !aligned4(bias)) ||
         !aligned4(topk_idx) || !aligned4(topk_w) || (logits && !aligned4(logits)))
         return MOE_ERR_MISALIGNED;
+    float *scratch = nullptr;
     if (!logits) {
         const ScratchLayout L = scratch_layout(shape, g);
         if (!ws || ws_bytes < L.total)
             return MOE_ERR_WORKSPACE_TOO_SMALL;
         if (!aligned16(ws))
             return MOE_ERR_MISALIGNED;
-        logits = reinterpret_cast<float *>(static_cast<char *>(ws) + L.logits);
+        scratch = reinterpret_cast<float *>(static_cast<char *>(ws) + L.logits);
     }
-    return route_impl(shape, x, w_router, bias, topk_idx, topk_w, logits, nullptr,
+    return route_impl(shape, x, w_router, bias, topk_idx, topk_w, logits, scratch, nullptr,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -977,11 +1017,7 @@ moe_status_t dispatch_entry(const moe_shape_t *shape, const uint16_t *x, const f
     int64_t *D = rank_matrix ? rank_matrix : reinterpret_cast<int64_t *>(w + L.D);
     int64_t *pk = packed_offsets ? packed_offsets : reinterpret_cast<int64_t *>(w + L.pk_off);
     return dispatch_impl(shape, g, x, logits, topk_idx, counts, kept, offsets, row_of,
-                         assign_of_row, expert_of, pay, D, pk, stats,
-                         reinterpret_cast<int32_t *>(w + L.blk),
-                         reinterpret_cast<int64_t *>(w + L.pk_base),
-                         reinterpret_cast<int32_t *>(w + L.cum),
-                         reinterpret_cast<int32_t *>(w + L.moved),
+                         assign_of_row, expert_of, pay, D, pk, stats, scratch_at(w, L),
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1220,8 +1256,10 @@ moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16
         if (cudaMemsetAsync(nonfinite, 0, sizeof(unsigned long long), st) != cudaSuccess)
             return MOE_ERR_CUDA;
     }
+    // the logits are kept (in the workspace) only when re-routing ranks candidates by them
+    float *lg = reinterpret_cast<float *>(w + S.logits);
     moe_status_t rc = route_impl(shape, x, w_router, bias, topk_idx, topk_w,
-                                 reinterpret_cast<float *>(w + S.logits), nonfinite, st);
+                                 g.rounds > 1 ? lg : nullptr, lg, nonfinite, st);
     if (rc != MOE_OK)
         return rc;
     int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
@@ -1236,10 +1274,7 @@ moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16
                        reinterpret_cast<int32_t *>(w + L.kept), offsets, row_of,
                        reinterpret_cast<int32_t *>(w + L.assign), nullptr, pay,
                        reinterpret_cast<int64_t *>(w + S.D), reinterpret_cast<int64_t *>(w + S.pk_off),
-                       stats, reinterpret_cast<int32_t *>(w + S.blk),
-                       reinterpret_cast<int64_t *>(w + S.pk_base),
-                       reinterpret_cast<int32_t *>(w + S.cum),
-                       reinterpret_cast<int32_t *>(w + S.moved), st);
+                       stats, scratch_at(w, S), st);
     if (rc != MOE_OK)
         return rc;
     if (up.e4m3())
@@ -1628,7 +1663,10 @@ __attribute__((visibility("default"))) moe_status_t moe_debug_bounded_wait(uint6
 //
 // Scratch of moe_dispatch_static: one fixed array per device. Host code never uses the
 // symbol itself as an address (on the host it is only a stand-in); the device address is
-// looked up once per device with cudaGetSymbolAddress while that device is current.
+// looked up with cudaGetSymbolAddress while that device is current, once per device and
+// context: the cache is keyed on the current context's unique id, so after a
+// cudaDeviceReset (which destroys the context and, with it, the module holding the array)
+// the next call looks the address up again instead of using a stale one.
 
 static __device__ __align__(256) unsigned char g_static_scratch[MOE_STATIC_SCRATCH_BYTES];
 
@@ -1637,6 +1675,33 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
 void *g_static_addr[kMaxDevices];
+unsigned long long g_static_ctx[kMaxDevices];  // context id the cached address belongs to
+
+// Unique id of the calling thread's current CUDA context (0 when none is current or the
+// driver does not provide ids).
+unsigned long long current_context_id()
+{
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+        get_id(ctx, &id) == CUDA_SUCCESS)
+        return id;
+    return 0;
+}
 
 moe_status_t static_scratch_address(void **out)
 {
@@ -1644,18 +1709,21 @@ moe_status_t static_scratch_address(void **out)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (!g_static_addr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_static_addr[dev] || ctx == 0 || ctx != g_static_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p)
             return MOE_ERR_CUDA;
         g_static_addr[dev] = p;
+        // the lookup made the device's primary context current if none was
+        g_static_ctx[dev] = current_context_id();
     }
     *out = g_static_addr[dev];
     return MOE_OK;
 }
 
 struct StaticLayout {
-    size_t blk, pk_base, cum, moved, D, pk_off, total;
+    size_t ctl, agg, incl, pk_base, moved, D, pk_off, total;
 };
 
 StaticLayout static_layout(const moe_shape_t *s, const Geometry &g)
@@ -1705,8 +1773,5 @@ moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x, const int32_t *
     return dispatch_impl(shape, g, x, nullptr, topk_idx, counts, kept, offsets, row_of,
                          assign_of_row, nullptr,
                          Payload{x_sorted, x_packed, false, nullptr, nullptr}, D, pk, stats,
-                         reinterpret_cast<int32_t *>(w + L.blk),
-                         reinterpret_cast<int64_t *>(w + L.pk_base),
-                         reinterpret_cast<int32_t *>(w + L.cum), nullptr,
-                         reinterpret_cast<cudaStream_t>(stream));
+                         scratch_at(w, L), reinterpret_cast<cudaStream_t>(stream));
 }

@@ -242,6 +242,240 @@ __global__ void __launch_bounds__(TY *TX)
         }
 }
 
+// ---------------------------------------------------------------------------
+// Router projection fused with the top-K selection, for many tokens and E >= 32.
+//
+// [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化] the gate's top-k runs
+// in the same kernel as the projection: the [N][E] logits need not go to HBM.
+//
+// A CTA takes 64 tokens and every expert. Lane l of every warp owns tokens l and l + 32 of the
+// tile, and warp w owns experts [16w, 16w + 16), so the W values a warp needs are the same
+// for all its lanes (broadcast shared-memory loads) and each lane's x values are its own. The
+// 8-element pieces of d are walked in order; per element i a lane forms (x_t[i], x_t[i]) and
+// multiplies it by two neighbouring experts' (W_e[i], W_e+1[i]) in one packed fp32 FMA
+// (`__ffma2_rn`: each half rounds like one fmaf), so every logit is still the single ascending
+// fmaf chain, bit for bit. W is staged transposed ([i][e]) so that one 16-byte load gives four
+// experts' weights of one element; the transposition happens on the way through registers,
+// one chunk ahead of its use. After the chain, the tile's logits go to shared memory and each
+// warp selects the top K of its tokens: K rounds of a warp-wide argmax on (value desc, expert
+// asc), then a softmax over the K picked logits, as topk_softmax_kernel does.
+constexpr int kRtTokens = 64;  // tokens per CTA (two per lane)
+constexpr int kRtKC = 32;      // elements of d per staged chunk
+constexpr int kRtXRow = kRtKC + 8;  // bf16 per staged x row (16-byte pad)
+
+template <int NW>
+struct RouterTopkTile {
+    static constexpr int NT = 32 * NW;
+    static constexpr int EP = 16 * NW + 4;  // fp32 per staged W^T row (16-byte pad)
+    static constexpr int X_BYTES = kRtTokens * kRtXRow * 2;
+    static constexpr int W_BYTES = kRtKC * EP * 4;
+    static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
+    static constexpr int LOGIT_BYTES = kRtTokens * (16 * NW + 1) * 4;  // epilogue tile
+    static constexpr int SMEM_BYTES =
+        2 * STAGE_BYTES > LOGIT_BYTES ? 2 * STAGE_BYTES : LOGIT_BYTES;
+    // W elements each thread carries from global memory to the next stage: E_pad x KC / NT
+    static constexpr int WV = (16 * NW * kRtKC) / (4 * NT);  // float4 per thread
+};
+
+template <int NW>
+__global__ void __launch_bounds__(32 * NW)
+    router_topk_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
+                       const float *__restrict__ bias, int N, int d, int E, int K,
+                       int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                       float *__restrict__ logits, unsigned long long *nonfinite_count)
+{
+    using L = RouterTopkTile<NW>;
+    extern __shared__ __align__(16) unsigned char rt_smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * kRtTokens;
+    const int nchunks = (d + kRtKC - 1) / kRtKC;
+    const int EW = 16 * NW;  // experts covered (E rounded up to 16 per warp)
+
+    // x chunk c -> stage s (cp.async, 16 bytes per copy; rows past N are left alone)
+    auto stage_x = [&](int c, int s) {
+        if (c < nchunks) {
+            uint16_t *xs = reinterpret_cast<uint16_t *>(rt_smem + s * L::STAGE_BYTES);
+            const int k0 = c * kRtKC, kc = min(kRtKC, d - k0);
+            for (int idx = tid; idx < kRtTokens * (kRtKC / 8); idx += L::NT) {
+                const int row = idx / (kRtKC / 8), v = idx % (kRtKC / 8);
+                if (t0 + row < N && v * 8 < kc)
+                    cp_async16(xs + row * kRtXRow + v * 8, x + (size_t)(t0 + row) * d + k0 + v * 8);
+            }
+        }
+        cp_async_commit();
+    };
+    // W chunk c -> registers: thread holds float4 pieces (expert e, elements 4q .. 4q+3)
+    float4 wreg[L::WV];
+    auto load_w = [&](int c) {
+        const int k0 = c * kRtKC, kc = c < nchunks ? min(kRtKC, d - k0) : 0;
+#pragma unroll
+        for (int j = 0; j < L::WV; ++j) {
+            const int idx = tid + j * L::NT;  // over EW x (KC / 4), element quad fastest
+            const int e = idx / (kRtKC / 4), q = idx % (kRtKC / 4);
+            wreg[j] = (e < E && q * 4 < kc)
+                          ? __ldg(reinterpret_cast<const float4 *>(wr + (size_t)e * d + k0) + q)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    // registers -> stage s, transposed to [i][e]
+    auto store_w = [&](int s) {
+        float *ws = reinterpret_cast<float *>(rt_smem + s * L::STAGE_BYTES + L::X_BYTES);
+#pragma unroll
+        for (int j = 0; j < L::WV; ++j) {
+            const int idx = tid + j * L::NT;
+            const int e = idx / (kRtKC / 4), q = idx % (kRtKC / 4);
+            ws[(4 * q + 0) * L::EP + e] = wreg[j].x;
+            ws[(4 * q + 1) * L::EP + e] = wreg[j].y;
+            ws[(4 * q + 2) * L::EP + e] = wreg[j].z;
+            ws[(4 * q + 3) * L::EP + e] = wreg[j].w;
+        }
+    };
+
+    float2 acc[2][8];  // [token of the lane][expert pair of the warp]
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+            acc[t][p] = make_float2(0.0f, 0.0f);
+
+    stage_x(0, 0);
+    load_w(0);
+    store_w(0);
+    load_w(1);
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        cp_async_wait<0>();
+        __syncthreads();  // stage s complete (x by cp.async, W by the stores); stage s^1 free
+        stage_x(c + 1, s ^ 1);
+        const uint16_t *xs = reinterpret_cast<const uint16_t *>(rt_smem + s * L::STAGE_BYTES);
+        const float *ws = reinterpret_cast<const float *>(rt_smem + s * L::STAGE_BYTES + L::X_BYTES);
+        const int kc = min(kRtKC, d - c * kRtKC);
+        for (int kk = 0; kk < kc; kk += 8) {
+            uint4 xq[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+                xq[t] = *reinterpret_cast<const uint4 *>(xs + (lane + 32 * t) * kRtXRow + kk);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float *wrow = ws + (kk + q) * L::EP + 16 * warp;
+                float2 wp[8];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float4 v = *reinterpret_cast<const float4 *>(wrow + 4 * h);
+                    wp[2 * h] = make_float2(v.x, v.y);
+                    wp[2 * h + 1] = make_float2(v.z, v.w);
+                }
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const uint32_t word = (q < 2) ? xq[t].x : (q < 4) ? xq[t].y : (q < 6) ? xq[t].z : xq[t].w;
+                    const float xv = (q & 1) ? bf16_hi(word) : bf16_lo(word);
+                    const float2 xx = make_float2(xv, xv);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p)
+                        acc[t][p] = __ffma2_rn(xx, wp[p], acc[t][p]);
+                }
+            }
+        }
+        store_w(s ^ 1);  // chunk c + 1 (loaded one iteration ago) into the free stage
+        load_w(c + 2);
+    }
+    cp_async_wait<0>();
+    __syncthreads();  // every warp is done with the stages: the logit tile may reuse them
+
+    // logits of the tile -> shared memory [token][expert] (row of EW + 1 floats)
+    float *lt = reinterpret_cast<float *>(rt_smem);
+    const int LR = EW + 1;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int tok = lane + 32 * t;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int e = 16 * warp + 2 * p;
+            float a = acc[t][p].x, b = acc[t][p].y;
+            if (bias) {
+                if (e < E)
+                    a = __fadd_rn(a, bias[e]);
+                if (e + 1 < E)
+                    b = __fadd_rn(b, bias[e + 1]);
+            }
+            lt[tok * LR + e] = a;
+            lt[tok * LR + e + 1] = b;
+        }
+    }
+    __syncthreads();
+
+    // top-K of each token: warp w takes tokens w, w + NW, ...; lane l holds experts l + 32j
+    constexpr int MAXJ = (16 * NW + 31) / 32;
+    for (int tok = warp; tok < kRtTokens; tok += NW) {
+        const int t = t0 + tok;
+        if (t >= N)
+            break;
+        const float *lrow = lt + tok * LR;
+        float v[MAXJ];
+        unsigned taken = 0;
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) {
+                float l = lrow[e];
+                if (logits)
+                    logits[(size_t)t * E + e] = l;
+                if (!isfinite(l)) {
+                    bad = true;
+                    if (isnan(l))
+                        l = -INFINITY;
+                }
+                v[j] = l;
+            } else {
+                v[j] = -INFINITY;
+                taken |= 1u << j;
+            }
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) {
+            set_dev_error(MOE_ERR_NONFINITE);
+            if (nonfinite_count)
+                atomicAdd(nonfinite_count, 1ull);
+        }
+        float my_v = 0.0f;
+        int my_e = 0;
+        for (int k = 0; k < K; ++k) {
+            float bv = -INFINITY;
+            int be = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                const int e = lane + 32 * j;
+                if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) {
+                    bv = v[j];
+                    be = e;
+                }
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (ov > bv || (ov == bv && oe < be)) {
+                    bv = ov;
+                    be = oe;
+                }
+            }
+            if ((be & 31) == lane)
+                taken |= 1u << (be >> 5);
+            if (lane == k) {
+                my_v = bv;
+                my_e = be;
+            }
+        }
+        const float top = __shfl_sync(0xffffffffu, my_v, 0);
+        const float ex = lane < K ? expf(my_v - top) : 0.0f;
+        const float ssum = warp_sum(ex);
+        if (lane < K) {
+            topk_idx[(size_t)t * K + lane] = my_e;
+            topk_w[(size_t)t * K + lane] = ex / ssum;
+        }
+    }
+}
+
 // One warp per token. Lane l holds logits of experts l + 32*j (E <= 256).
 // K rounds of a warp-wide argmax on (value desc, expert asc); then a softmax over
 // the K picked logits. NaN is treated as -inf for the choice; any non-finite

@@ -194,7 +194,8 @@ size_t moe_y_bytes(const moe_shape_t *shape);
  * starting from +0) + bias[e]: bit-identical to any IEEE implementation of that order.
  * topk_idx [N][K] int32: the K largest logits, larger first, equal logits to the lower
  * expert index. topk_w [N][K] fp32: softmax over the K selected logits.
- * logits [N][E] fp32 or NULL (then written to the workspace). A non-finite logit sets
+ * logits [N][E] fp32 or NULL (then not returned; the workspace holds them only where the two
+ * steps run as separate kernels: few tokens or E < 32). A non-finite logit sets
  * MOE_ERR_NONFINITE in the device error word; that token's result is unspecified. */
 moe_status_t moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
                        const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
@@ -257,15 +258,19 @@ moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, c
  * offsets when those are NULL) lives in one static device array of MOE_STATIC_SCRATCH_BYTES
  * inside the library. Every GPU that loads the library holds that array until the process
  * exits. The call allocates and frees nothing.
- *  - Shapes whose scratch does not fit (about E * W * ceil(N / (64 W)) * 4 bytes plus
- *    E * W * 12 + 2 * W * W * 8, the first two terms K times larger with MOE_FLAG_SLOT_MAJOR)
- *    return MOE_ERR_WORKSPACE_TOO_SMALL before any launch. MOE_FLAG_REROUTE is refused.
+ *  - Shapes whose scratch does not fit (about 8 * E * B + 8 * E * W + 16 * W * W bytes with
+ *    B = W * ceil(N / (64 W)) token blocks, the first two terms K times larger with
+ *    MOE_FLAG_SLOT_MAJOR) return MOE_ERR_WORKSPACE_TOO_SMALL before any launch.
+ *    MOE_FLAG_REROUTE is refused.
  *  - The first call on a device looks up the array's device address on that device (the
- *    device must be current); make that first call before any stream capture.
- *  - All calls share the one array, and it keeps the last call's contents; every scratch byte
- *    a call reads it has written first in the same call, so nothing needs clearing. Two calls
- *    that overlap on the GPU (other streams, other host threads) race on the array: serialise
- *    them. */
+ *    device must be current); make that first call before any stream capture. The address is
+ *    kept per device and per CUDA context: after cudaDeviceReset (which destroys the context
+ *    and the array with it) the next call looks it up again, so that call, too, must come
+ *    before any stream capture.
+ *  - All calls share the one array, and it keeps the last call's contents; each call clears
+ *    the control words it needs (one cudaMemsetAsync on `stream`, which allocates nothing) and
+ *    writes every other scratch byte before reading it. Two calls that overlap on the GPU
+ *    (other streams, other host threads) race on the array: serialise them. */
 moe_status_t moe_dispatch_static(const moe_shape_t *shape, const uint16_t *x,
                                  const int32_t *topk_idx, int32_t *counts, int32_t *kept,
                                  int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,

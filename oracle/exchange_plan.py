@@ -106,12 +106,16 @@ def ilp_placement(counts, P: int):
 
 
 def greedy_order_makespan(D) -> int:
-    """The page's transmission-order procedure (§Aurora 场景 1, the steps after 定理 4.2) read as
-    a list schedule, for comparison with the bound: the bottleneck rank (largest send or receive
-    volume) first, the other ranks by send volume, largest first; each rank sends its blocks one
-    after another (largest first), each block whole, starting at the earliest time at which both
-    the rank and the block's receiver are free, so that no receiver is fed by two senders at
-    once. Returns the time the last block ends, in rows (ties to the lower rank index)."""
+    """One list-schedule reading of the page's transmission-order steps (§Aurora 场景 1, the
+    steps after 定理 4.2), for comparison with the bound only; the page does not fix these
+    details, so other readings can end elsewhere. This reading: the bottleneck rank (largest
+    send or receive volume) is scheduled first as a sender, even when its load is on the
+    receive side (a rank that only receives then sends nothing and its own blocks are placed by
+    the other senders like anyone else's); the other ranks follow by send volume, largest
+    first; each rank sends its blocks one after another (largest first), each block whole (no
+    pre-emption), starting at the earliest time at which both the rank and the block's
+    receiver are free, so that no receiver is fed by two senders at once. Returns the time the
+    last block ends, in rows (ties to the lower rank index)."""
     D = np.array(D, dtype=np.int64, copy=True)
     np.fill_diagonal(D, 0)
     W = D.shape[0]

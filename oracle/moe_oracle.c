@@ -8,19 +8,20 @@
  * never does. It shares no code, header, table or helper with the CUDA path.
  *
  * Sources (page title, section):
- *  [P1] "MoE 专家并行的 All-to-All 通信瓶颈：专家越多推理延迟为何反而上升"
+ *  "MoE 专家并行的 All-to-All 通信瓶颈：专家越多推理延迟为何反而上升"
  *       §All-to-All 分发与回收的机制 (dataflow flowchart: route Top-K, pack by
  *       destination card, group by expert, grouped GEMM, weighted merge back to
  *       token order), §专家越多，通信为什么越重 (E/W experts per card, even
  *       placement, per-card send volume N*K*d*b/W).
- *  [P2] "MoE 推理服务工程真相 2026 ..." §2.2 Expert Capacity Factor (tokens above
+ *  "MoE 推理服务工程真相 2026 ..." §2.2 Expert Capacity Factor (tokens above
  *       an expert's capacity are dropped, router output set to zero) and the
  *       moe_dispatch pseudo-code of §2.3 (bincount of expert ids, overflow mask).
- *  [P3] "MoE Inference Communication" §DeepSpeed-MoE › MoE 计算核优化 (top-k,
+ *  "MoE Inference Communication" §DeepSpeed-MoE › MoE 计算核优化 (top-k,
  *       cumsum, scatter; dense token->expert mapping table), §ExFlow 跨层专家
  *       亲和性 (conditional routing between consecutive layers), §Aurora 定理
  *       4.2 (traffic matrix D).
- *  [P2] §6.3 通信压缩 (the token payload of the all-to-all in FP8 instead of BF16).
+ *  "MoE 推理服务工程真相 2026 ..." §6.3 通信压缩 (the token payload of the all-to-all in FP8
+ *       instead of BF16).
  * Readings where the pages are silent (all fixed by the workload statement):
  *  softmax over the K selected logits; ties to the lowest expert index; logits
  *  accumulated in fp32 by one fused multiply-add per input element, i
@@ -48,8 +49,8 @@ static float bf16_to_float(uint16_t h)
     return f;
 }
 
-/* Router projection [P1 §All-to-All 分发与回收的机制, node B; P3 §Aurora, gate
- * term G_i]. logits[t][e] = (sum_i x[t][i] * Wr[e][i]) + bias[e], the sum taken
+/* Router projection [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制,
+ * node B; MoE Inference Communication, §Aurora, gate term G_i]. logits[t][e] = (sum_i x[t][i] * Wr[e][i]) + bias[e], the sum taken
  * as one fmaf per i in ascending order starting from +0.0f. */
 EXPORT void orc_router_logits(int64_t N, int64_t d, int64_t E, const uint16_t *x,
                               const float *w_router, const float *bias, float *logits)
@@ -67,9 +68,9 @@ EXPORT void orc_router_logits(int64_t N, int64_t d, int64_t E, const uint16_t *x
     }
 }
 
-/* Top-K selection and gate weights [P1 §一个反直觉的扩容结果 (Top-K experts per
- * token); P3 §MoE 计算核优化 (top-k)]. The K largest logits, larger value first,
- * equal values ordered by lower expert index. Weights: softmax over the K
+/* Top-K selection and gate weights [MoE 专家并行的 All-to-All 通信瓶颈, §一个反直觉的
+ * 扩容结果 (Top-K experts per token); MoE Inference Communication, §MoE 计算核优化 (top-k)].
+ * The K largest logits, larger value first, equal values ordered by lower expert index. Weights: softmax over the K
  * selected logits, in fp64, stored as fp32. Returns the number of tokens that
  * have a non-finite logit (their result is unspecified). */
 EXPORT int64_t orc_topk(int64_t N, int64_t E, int64_t K, const float *logits,
@@ -112,8 +113,8 @@ EXPORT int64_t orc_topk(int64_t N, int64_t E, int64_t K, const float *logits,
     return nonfinite;
 }
 
-/* Expert capacity [P2 §2.2]: C = ceil(cf * N * K / E), in double. cf <= 0 means
- * dropless; then C = N * K, which no expert can exceed (each token picks K
+/* Expert capacity [MoE 推理服务工程真相 2026, §2.2]: C = ceil(cf * N * K / E), in double.
+ * cf <= 0 means dropless; then C = N * K, which no expert can exceed (each token picks K
  * distinct experts, so an expert receives at most N). */
 EXPORT int64_t orc_capacity(int64_t N, int64_t E, int64_t K, float cf)
 {
@@ -143,10 +144,11 @@ static void walk_positions(int64_t N, int64_t E, int64_t K, int64_t order,
     }
 }
 
-/* Dispatch bookkeeping [P2 §2.3 pseudo-code (bincount, overflow mask, remapping of
- * overflowed assignments); §2.2 (capacity, expert drop); §4.3 (token drop: re-route
- * to the next-best expert); P3 §MoE 计算核优化 (cumsum, scatter, mapping table);
- * P1 §All-to-All 分发与回收的机制 (pack by destination card)].
+/* Dispatch bookkeeping [MoE 推理服务工程真相 2026, §2.3 pseudo-code (bincount, overflow
+ * mask, remapping of overflowed assignments); §2.2 (capacity, expert drop); §4.3 (token
+ * drop: re-route to the next-best expert); MoE Inference Communication, §MoE 计算核优化
+ * (cumsum, scatter, mapping table); MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与
+ * 回收的机制 (pack by destination card)].
  *
  * First pass: pos0[a] = number of earlier assignments (in priority order) to the
  * same expert; the assignment is kept iff pos0 < C. demand counts[e] = all
@@ -353,8 +355,8 @@ EXPORT void orc_positions(int64_t N, int64_t E, int64_t K, int64_t W, int64_t C,
                           assign_of_row, D, pk_off, packed_row_of, stats);
 }
 
-/* Expert FFN for a list of rows [P1 §All-to-All 分发与回收的机制, node F: each
- * expert's tokens through its own FFN]. Row r holds the hidden state of token
+/* Expert FFN for a list of rows [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与
+ * 回收的机制, node F: each expert's tokens through its own FFN]. Row r holds the hidden state of token
  * row_token[r] for expert row_expert[r]:
  *   g = W1[e] x, u = W3[e] x, h = g * sigmoid(g) * u, y = W2[e] h,
  * all in fp64 from the bf16 inputs. W1, W3 are [E][f][d]; W2 is [E][d][f].
@@ -397,9 +399,9 @@ EXPORT void orc_expert_rows(int64_t nrows, const int32_t *row_token, const int32
     }
 }
 
-/* Weighted combine [P1 §All-to-All 分发与回收的机制, node I: weighted merge back
- * to the original token order; P2 §2.2: a dropped slot's router output is
- * zero]. out[t] = sum over kept slots k, in k order, of w[t][k] * y[row], where
+/* Weighted combine [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制,
+ * node I: weighted merge back to the original token order; MoE 推理服务工程真相 2026, §2.2:
+ * a dropped slot's router output is zero]. out[t] = sum over kept slots k, in k order, of w[t][k] * y[row], where
  * y_of_slot[(t*K+k)*d ...] holds the expert output of slot (t, k). */
 EXPORT void orc_combine(int64_t N, int64_t K, int64_t d, const int32_t *row_of,
                         const float *topk_w, const double *y_of_slot, double *out)
@@ -419,8 +421,8 @@ EXPORT void orc_combine(int64_t N, int64_t K, int64_t d, const int32_t *row_of,
     }
 }
 
-/* Inter-layer expert affinity counts [P3 §ExFlow 跨层专家亲和性]: for every
- * token t, every expert i in its top-K at layer j and every expert p in its
+/* Inter-layer expert affinity counts [MoE Inference Communication, §ExFlow 跨层专家
+ * 亲和性]: for every token t, every expert i in its top-K at layer j and every expert p in its
  * top-K at layer j+1, cnt[i][p] += 1 (pre-drop routing decisions). The
  * conditional P(p | i) is cnt[i][p] / (number of tokens with i in their top-K
  * at layer j); each row of cnt sums to K times that number. */
@@ -433,8 +435,8 @@ EXPORT void orc_affinity(int64_t N, int64_t E, int64_t K, const int32_t *topk_j,
                 cnt[(int64_t)topk_j[t * K + k] * E + topk_j1[t * K + q]] += 1;
 }
 
-/* FP8 payload [P2 §6.3 通信压缩: the token rows that cross the all-to-all are sent as
- * FP8 instead of BF16]. Format: e4m3 ("E4M3" of the OCP 8-bit floating-point formats):
+/* FP8 payload [MoE 推理服务工程真相 2026, §6.3 通信压缩: the token rows that cross the
+ * all-to-all are sent as FP8 instead of BF16]. Format: e4m3 ("E4M3" of the OCP 8-bit floating-point formats):
  * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
  * subnormals m * 2^-9; no infinities; code 0x7F/0xFF is NaN, so 448 = 1.75 * 2^8 is the
  * largest finite value.

@@ -13,18 +13,18 @@ sys.path.insert(0, ROOT)
 
 
 @pytest.mark.parametrize("name,count", [
-    ("mixtral_prefill", 11),       # pair + single-CTA launch for each GEMM
-    ("mixtral_prefill_fp8", 12),   # + quantisation of h
-    ("e128_skew", 9),              # ~165 rows per expert: single-CTA GEMMs only
-    ("e128_skew_fp8", 10),
-    ("decode", 9),
-    ("e128_skew_slot_major", 10),  # 1024 blocks per expert: the per-expert scan
-    ("e128_skew_reroute", 14),     # two dispatch passes and the ranking kernel
-    ("stack4", 12),                # 512 blocks per expert, pair GEMMs
-    ("stack4_affinity", 12),
-    ("mixtral_prefill_fp8_return", 12),
-    ("e128_skew_fp8_return", 10),
-    ("residual_top1", 14),         # shared MLP: offsets, pair + single GEMMs twice
+    ("mixtral_prefill", 9),        # E = 8: projection, then selection; pair + single GEMMs
+    ("mixtral_prefill_fp8", 10),   # + quantisation of h
+    ("e128_skew", 6),              # fused router; ~165 rows per expert: single-CTA GEMMs only
+    ("e128_skew_fp8", 7),
+    ("decode", 7),                 # 16 tokens: projection, then selection
+    ("e128_skew_slot_major", 6),   # the same two dispatch kernels over K times more blocks
+    ("e128_skew_reroute", 9),      # positions-only pass, the ranking kernel, the full pass
+    ("stack4", 8),                 # pair GEMMs
+    ("stack4_affinity", 8),
+    ("mixtral_prefill_fp8_return", 10),
+    ("e128_skew_fp8_return", 7),
+    ("residual_top1", 12),         # shared MLP: offsets, pair + single GEMMs twice
 ])
 def test_kernel_launch_count(name, count):
     import bench

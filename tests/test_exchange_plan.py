@@ -361,10 +361,11 @@ def test_placements_on_random_and_degenerate_counts(m):
 
 
 def test_literal_greedy_reading_misses_the_bound():
-    """The page's steps read literally as a list schedule of whole blocks (bottleneck rank
-    first, the rest by volume, each block at the earliest time its receiver is free) never beat
-    tau_min and on random 8-rank traffic end well above it, which is why the library builds
-    its order by a matching decomposition that meets the bound exactly."""
+    """One list-schedule reading of the page's steps (whole blocks, bottleneck rank first as a
+    sender, the rest by volume, each block at the earliest time its receiver is free) never
+    beats tau_min (no order can) and, in this reading, on random 8-rank traffic ends well above
+    it (the 0.2 mean-gap threshold belongs to this reading only); the library builds its order
+    by a matching decomposition that meets the bound exactly."""
     rng = np.random.default_rng(0)
     gaps = []
     for _ in range(100):

@@ -81,14 +81,18 @@ def test_static_scratch_dispatch_matches_workspace_dispatch(m, w):
                               got["D"], got["pk_off"], got["stats"])
         torch.cuda.synchronize()
         _same(ref, got, R)
-    # with the traffic matrix and pack offsets left to the scratch array as well
+    # with the traffic matrix and pack offsets left to the scratch array as well: every other
+    # output still bit for bit (a wrong pack-offset layout inside the array would show in
+    # x_packed, a wrong counter write in stats)
     got = _buffers(m, shape, w, dev)
     m.moe_dispatch_static(shape, x, topk, got["counts"], got["kept"], got["offsets"],
-                          got["row_of"], got["assign"], got["x_sorted"], got["x_packed"])
+                          got["row_of"], got["assign"], got["x_sorted"], got["x_packed"],
+                          stats=got["stats"])
     torch.cuda.synchronize()
-    for k in ("counts", "kept", "offsets", "row_of"):
+    for k in ("counts", "kept", "offsets", "row_of", "stats"):
         assert torch.equal(ref[k], got[k]), k
-    assert torch.equal(ref["x_packed"][:R], got["x_packed"][:R])
+    for k in ("assign", "x_sorted", "x_packed"):
+        assert torch.equal(ref[k][:R], got[k][:R]), k
     assert m.moe_get_device_error(True) == 0
 
 
