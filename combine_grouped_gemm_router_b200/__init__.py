@@ -66,6 +66,8 @@ _sigs = {
     "moe_route": ([_SP] + [c_p] * 7 + [c_size, c_p], c_i32),
     "moe_dispatch": ([_SP] + [c_p] * 13 + [c_size, c_p], c_i32),
     "moe_dispatch_static": ([_SP] + [c_p] * 13, c_i32),
+    "moe_dispatch_rank": ([_SP, c_i32] + [c_p] * 14 + [c_size, c_p], c_i32),
+    "moe_regroup_rows": ([_SP, c_i32, c_i32, c_i32] + [c_p] * 8, c_i32),
     "moe_dispatch_reroute": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_dispatch_fp8": ([_SP] + [c_p] * 15 + [c_size, c_p], c_i32),
     "moe_quantize_rows_e4m3": ([c_p, c_i64, c_i32, c_p, c_p, c_p, c_p], c_i32),
@@ -228,6 +230,31 @@ def moe_dispatch(shape, x, topk_idx, counts, kept, offsets, row_of, assign_of_ro
                              _ptr(x_sorted), _ptr(x_packed), _ptr(rank_matrix),
                              _ptr(packed_offsets), _ptr(stats), _ptr(ws), ws_bytes,
                              _stream(stream)), "moe_dispatch")
+
+
+def moe_dispatch_rank(shape, rank, x_local, topk_idx_all, counts, kept, offsets, row_of,
+                      assign_of_row, packed_row_of, send_row_of, x_send, rank_matrix,
+                      packed_offsets, stats=None, ws=None, stream=None):
+    """Rank `rank`'s dispatch with W real ranks (shape: the whole batch)."""
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.moe_dispatch_rank(ctypes.byref(shape), int(rank), _ptr(x_local),
+                                  _ptr(topk_idx_all), _ptr(counts), _ptr(kept), _ptr(offsets),
+                                  _ptr(row_of), _ptr(assign_of_row), _ptr(packed_row_of),
+                                  _ptr(send_row_of), _ptr(x_send), _ptr(rank_matrix),
+                                  _ptr(packed_offsets), _ptr(stats), _ptr(ws), ws_bytes,
+                                  _stream(stream)), "moe_dispatch_rank")
+
+
+def moe_regroup_rows(shape, rank, direction, src, dst, assign_of_row, packed_row_of, offsets,
+                     packed_offsets, offsets_local=None, row_bytes=None, stream=None):
+    """Rows of rank `rank` between the exchange's order (direction 0: src) and its experts'
+    order (direction 1: src). row_bytes defaults to the byte size of one row of src."""
+    if row_bytes is None:
+        row_bytes = src[0].numel() * src.element_size() if src.dim() > 1 else src.element_size()
+    _check(_lib.moe_regroup_rows(ctypes.byref(shape), int(rank), int(row_bytes), int(direction),
+                                 _ptr(src), _ptr(dst), _ptr(assign_of_row), _ptr(packed_row_of),
+                                 _ptr(offsets), _ptr(packed_offsets), _ptr(offsets_local),
+                                 _stream(stream)), "moe_regroup_rows")
 
 
 def moe_dispatch_reroute(shape, x, logits, topk_idx, counts, kept, offsets, row_of,

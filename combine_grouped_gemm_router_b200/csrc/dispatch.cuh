@@ -363,6 +363,16 @@ struct PlaceArgs {
     const int64_t *pk_base;     // [nseg][E]
     int32_t *row_of, *assign_of_row;
     int32_t *expert_of;         // nullable: the expert whose row each assignment uses, or -1
+    int32_t *packed_row_of;     // nullable: each assignment's packed row, or -1
+    // W real ranks: this process is rank `rank` (home shard `rank`), -1 for the whole batch on
+    // one GPU. Then only the home shard's rows are copied, x holds just those tokens (token t
+    // at row t - x_row0), and packed row p goes to x_packed row p - pk_off[rank W] (the start of
+    // its block row); send_row_of (nullable) receives, per slot of the home shard's tokens,
+    // that same row or -1.
+    int rank;
+    int x_row0;
+    const int64_t *pk_off;  // [W*W+1]: the pack offsets the totals kernel wrote
+    int32_t *send_row_of;
     // the copy of the rows (copy != 0)
     int copy;
     int e4m3;
@@ -471,8 +481,7 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
                         s_rk[ls] = row;
                         s_ex[ls] = row >= 0 ? e : -1;
                         const int64_t pk = p.pk_base[(size_t)g * E + e] + pos;
-                        s_pk[ls] = (row >= 0 && p.x_packed && pk >= 0 && pk < s_off[E])
-                                       ? (int)pk : -1;
+                        s_pk[ls] = (row >= 0 && pk >= 0 && pk < s_off[E]) ? (int)pk : -1;
                         if (row >= 0 && part == 0)
                             p.assign_of_row[row] = a;
                     }
@@ -481,11 +490,18 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
             __syncthreads();
         }
     }
+    const bool home_block = p.rank < 0 || tb / p.vbm.bm.bps == p.rank;
+    const int64_t pack_row0 = p.rank < 0 ? 0 : p.pk_off[(size_t)p.rank * p.W];
     if (part == 0) {
         for (int i = threadIdx.x; i < nt * K; i += kPlaceThreads) {
             p.row_of[t0 * K + i] = s_rk[i];
             if (p.expert_of)
                 p.expert_of[t0 * K + i] = s_ex[i];
+            if (p.packed_row_of)
+                p.packed_row_of[t0 * K + i] = s_pk[i];
+            if (p.send_row_of && home_block)
+                p.send_row_of[(t0 - p.x_row0) * K + i] =
+                    s_pk[i] >= 0 ? (int)(s_pk[i] - pack_row0) : -1;
         }
         if (p.stats) {
             // distinct destination ranks other than the token's home over its kept slots
@@ -503,41 +519,52 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
                 atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
         }
     }
-    if (!p.copy)
+    if (!p.copy || !home_block)
         return;
+    // rows of this block's tokens: x holds token t at row t - x_row0; the packed rows of a rank
+    // start at its block row (pack_row0); without a packed buffer no packed row is written
+    const uint16_t *xb = p.x + (size_t)(t0 - p.x_row0) * p.d;  // the block's first token
+    if (!p.x_packed)
+        for (int i = threadIdx.x; i < nt * K; i += kPlaceThreads)
+            s_pk[i] = -1;
+    else if (pack_row0 != 0)
+        for (int i = threadIdx.x; i < nt * K; i += kPlaceThreads)
+            s_pk[i] = s_pk[i] >= 0 ? (int)(s_pk[i] - pack_row0) : -1;
+    __syncthreads();
 
     if (!p.e4m3) {
-        // a column slice of every row of the block: `cs` 16-byte chunks from cbeg
-        constexpr int U = 4;
+        // a column slice of every row of the block (16-byte chunks [cbeg, cend)): lane l takes
+        // chunks cbeg + l, + 32, ...; warp w takes tokens w, w + 8, ... and loads one chunk of
+        // all of them before storing any (eight independent loads in flight per lane)
+        constexpr int TB = kDispatchHB / 8;  // tokens per warp
         const int nvec = p.d >> 3;
         const int cs = (nvec + parts - 1) / parts;
         const int cbeg = part * cs, cend = min(nvec, cbeg + cs);
         uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
         uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
-        for (int lt = warp; lt < nt; lt += 8) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + lt) * p.d);
-            const int *rk_l = s_rk + lt * K;
-            const int *pk_l = s_pk + lt * K;
-            for (int c0 = cbeg; c0 < cend; c0 += 32 * U) {
-                const int c = c0 + lane;
-                uint4 v[U];
+        const uint4 *src = reinterpret_cast<const uint4 *>(xb);
+        for (int c = cbeg + lane; c < cend; c += 32) {
+            uint4 v[TB];
 #pragma unroll
-                for (int u = 0; u < U; ++u)
-                    if (c + 32 * u < cend)
-                        v[u] = __ldcs(src + c + 32 * u);
+            for (int i = 0; i < TB; ++i) {
+                const int lt = warp + 8 * i;
+                if (lt < nt)
+                    v[i] = __ldcs(src + (size_t)lt * nvec + c);
+            }
+#pragma unroll
+            for (int i = 0; i < TB; ++i) {
+                const int lt = warp + 8 * i;
+                if (lt >= nt)
+                    break;
                 for (int k = 0; k < K; ++k) {
-                    const int rk = rk_l[k];
+                    const int rk = s_rk[lt * K + k];
                     if (rk < 0)
                         continue;
-                    const int pk = pk_l[k];
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        if (c + 32 * u < cend) {
-                            dst_s[(size_t)rk * nvec + c + 32 * u] = v[u];
-                            if (pk >= 0)
-                                dst_p[(size_t)pk * nvec + c + 32 * u] = v[u];
-                        }
-                    }
+                    const int pk = s_pk[lt * K + k];
+                    if (dst_s)
+                        dst_s[(size_t)rk * nvec + c] = v[i];
+                    if (pk >= 0)
+                        dst_p[(size_t)pk * nvec + c] = v[i];
                 }
             }
         }
@@ -553,7 +580,7 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
     uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
     uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
     for (int lt = part + parts * warp; lt < nt; lt += parts * 8) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.x + (size_t)(t0 + lt) * p.d);
+        const uint4 *src = reinterpret_cast<const uint4 *>(xb + (size_t)lt * p.d);
         const int *rk_l = s_rk + lt * K;
         const int *pk_l = s_pk + lt * K;
         // pass 1: largest magnitude of the row (bf16 bits with the sign cleared order like the
@@ -575,7 +602,8 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
         if (lane < K) {
             const int rk = rk_l[lane], pk = pk_l[lane];
             if (rk >= 0) {
-                p.sorted_scale[rk] = scale;
+                if (p.sorted_scale)
+                    p.sorted_scale[rk] = scale;
                 if (pk >= 0)
                     p.packed_scale[pk] = scale;
             }
@@ -597,12 +625,65 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
                 const int rk = rk_l[k];
                 if (rk < 0)
                     continue;
-                dst_s[(size_t)rk * n16 + c] = q;
+                if (dst_s)
+                    dst_s[(size_t)rk * n16 + c] = q;
                 const int pk = pk_l[k];
                 if (pk >= 0)
                     dst_p[(size_t)pk * n16 + c] = q;
             }
         }
+    }
+}
+
+// W real ranks: the rows that rank j receives in one exchange (the blocks (i, j) of every home
+// rank i, one after another, each in its (expert, token) order) <-> rank j's expert-sorted rows
+// (its experts [j E/W, (j+1) E/W), their rows in the one-GPU order: rows [offsets[e0],
+// offsets[e1]) of the whole batch's expert-sorted layout). Row r of that layout is assignment
+// a = assign_of_row[r], of a token whose home shard is i = (a / K) / S, at packed row
+// packed_row_of[a] inside block (i, j), which starts at pk_off[i W + j]; in the received buffer
+// block (i, j) starts after the blocks (i', j) of i' < i. dir 0 gathers received rows into
+// sorted order (the layer's way out to the experts), dir 1 scatters sorted rows back into the
+// received order (the way back). Block 0 also writes the rank's expert offsets (E/W + 1).
+struct RegroupArgs {
+    const int32_t *assign_of_row, *packed_row_of, *offsets;
+    const int64_t *pk_off;  // [W*W+1]
+    int E, K, W, S, rank;
+    int row_vec;            // 16-byte vectors per row
+    const uint4 *src;
+    uint4 *dst;
+    int dir;
+    int32_t *offsets_local;  // nullable
+};
+
+__global__ void __launch_bounds__(256) regroup_rows_kernel(RegroupArgs p)
+{
+    __shared__ int64_t s_base[64 + 1];  // per home rank i: received index - packed row
+    const int W = p.W, j = p.rank, e_per = p.E / W;
+    const int e0 = j * e_per;
+    if (threadIdx.x == 0) {
+        int64_t run = 0;
+        for (int i = 0; i < W; ++i) {
+            const int64_t b0 = p.pk_off[i * W + j], b1 = p.pk_off[i * W + j + 1];
+            s_base[i] = run - b0;
+            run += b1 - b0;
+        }
+    }
+    if (blockIdx.x == 0 && p.offsets_local)
+        for (int e = threadIdx.x; e <= e_per; e += blockDim.x)
+            p.offsets_local[e] = p.offsets[e0 + e] - p.offsets[e0];
+    __syncthreads();
+    const int r0 = p.offsets[e0], r1 = p.offsets[e0 + e_per];
+    const int lane = threadIdx.x & 31;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    for (int r = r0 + blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < r1; r += nwarps) {
+        const int a = p.assign_of_row[r];
+        const int i = (a / p.K) / p.S;
+        const int64_t recv = s_base[i] + p.packed_row_of[a];
+        const size_t sorted = (size_t)(r - r0);
+        const uint4 *from = p.src + (p.dir == 0 ? (size_t)recv : sorted) * p.row_vec;
+        uint4 *to = p.dst + (p.dir == 0 ? sorted : (size_t)recv) * p.row_vec;
+        for (int c = lane; c < p.row_vec; c += 32)
+            to[c] = from[c];
     }
 }
 

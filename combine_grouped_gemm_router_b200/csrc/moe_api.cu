@@ -343,6 +343,14 @@ struct Payload {
     float *packed_scale;  // e4m3 with x_packed only
 };
 
+// W real ranks: this process's rank and where its rows go (see PlaceArgs).
+struct RankPack {
+    int rank = -1;
+    int x_row0 = 0;
+    int32_t *packed_row_of = nullptr;
+    int32_t *send_row_of = nullptr;
+};
+
 // The dispatch's scratch pointers (inside a workspace or the static array).
 struct DispatchScratch {
     unsigned int *ctl;
@@ -352,11 +360,12 @@ struct DispatchScratch {
 };
 
 // Column (bf16) or token (FP8) parts per token block of the placement kernel: enough CTAs for
-// about two per SM, each part at least 64 16-byte chunks of a row (or one token per warp).
+// about eight per SM, each part at least 32 16-byte chunks of a row (one per lane; or one
+// token per warp for the FP8 payload).
 int place_parts(const moe_shape_t *s, const Geometry &g, bool e4m3)
 {
-    const int want = (2 * num_sms() + g.nblk - 1) / g.nblk;
-    const int cap = e4m3 ? (kDispatchHB + 7) / 8 : ((s->d / 8) + 63) / 64;
+    const int want = (8 * num_sms() + g.nblk - 1) / g.nblk;
+    const int cap = e4m3 ? (kDispatchHB + 7) / 8 : ((s->d / 8) + 31) / 32;
     const int parts = want < cap ? want : cap;
     return parts < 1 ? 1 : parts;
 }
@@ -369,7 +378,8 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
                            int32_t *kept, int32_t *offsets, int32_t *row_of,
                            int32_t *assign_of_row, int32_t *expert_of, const Payload *pay,
                            const uint16_t *x, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
-                           const DispatchScratch &sc, cudaStream_t st)
+                           const DispatchScratch &sc, cudaStream_t st,
+                           const RankPack &rk = RankPack())
 {
     VBlocks vbm;
     vbm.bm = BlockMap{g.S, g.bps, kDispatchHB};
@@ -425,6 +435,11 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
     pa.row_of = row_of;
     pa.assign_of_row = assign_of_row;
     pa.expert_of = expert_of;
+    pa.packed_row_of = rk.packed_row_of;
+    pa.rank = rk.rank;
+    pa.x_row0 = rk.x_row0;
+    pa.pk_off = pk_off;
+    pa.send_row_of = rk.send_row_of;
     pa.stats = stats;
     pa.x = x;
     pa.d = s->d;
@@ -1036,6 +1051,93 @@ moe_dispatch(const moe_shape_t *shape, const uint16_t *x, const int32_t *topk_id
     return dispatch_entry(shape, x, nullptr, topk_idx, counts, kept, offsets, row_of,
                           assign_of_row, nullptr, Payload{x_sorted, x_packed, false, nullptr, nullptr},
                           rank_matrix, packed_offsets, stats, ws, ws_bytes, stream);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_dispatch_rank(const moe_shape_t *shape, int32_t rank, const uint16_t *x_local,
+                  const int32_t *topk_idx_all, int32_t *counts, int32_t *kept, int32_t *offsets,
+                  int32_t *row_of, int32_t *assign_of_row, int32_t *packed_row_of,
+                  int32_t *send_row_of, uint16_t *x_send, int64_t *rank_matrix,
+                  int64_t *packed_offsets, moe_stats_t *stats, void *ws, size_t ws_bytes,
+                  moe_stream_t stream)
+{
+    Geometry g;
+    moe_status_t rc = check_shape(shape, false, &g);
+    if (rc != MOE_OK)
+        return rc;
+    if (shape->flags & MOE_FLAG_REROUTE)
+        return MOE_ERR_INVALID_ARG;  // candidates are ranked by every token's logits
+    if (rank < 0 || rank >= shape->W)
+        return MOE_ERR_INVALID_ARG;
+    if (shape->N == 0)
+        return empty_dispatch(shape, counts, kept, offsets, rank_matrix, packed_offsets, stats,
+                              reinterpret_cast<cudaStream_t>(stream));
+    if (!x_local || !topk_idx_all || !counts || !kept || !offsets || !row_of || !assign_of_row ||
+        !packed_row_of || !send_row_of || !x_send || !rank_matrix || !packed_offsets)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_local) || !aligned16(x_send) || !aligned4(topk_idx_all) || !aligned4(counts) ||
+        !aligned4(kept) || !aligned4(offsets) || !aligned4(row_of) || !aligned4(assign_of_row) ||
+        !aligned4(packed_row_of) || !aligned4(send_row_of) ||
+        (reinterpret_cast<uintptr_t>(rank_matrix) & 7u) ||
+        (reinterpret_cast<uintptr_t>(packed_offsets) & 7u) ||
+        (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)))
+        return MOE_ERR_MISALIGNED;
+    const ScratchLayout L = scratch_layout(shape, g);
+    if (!ws || ws_bytes < L.total)
+        return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return MOE_ERR_MISALIGNED;
+    RankPack rk;
+    rk.rank = rank;
+    rk.x_row0 = rank * g.S;
+    rk.packed_row_of = packed_row_of;
+    rk.send_row_of = send_row_of;
+    const Payload pay{nullptr, x_send, false, nullptr, nullptr};
+    return dispatch_pass(shape, g, 1, nullptr, topk_idx_all, counts, kept, offsets, row_of,
+                         assign_of_row, nullptr, &pay, x_local, rank_matrix, packed_offsets, stats,
+                         scratch_at(static_cast<char *>(ws), L),
+                         reinterpret_cast<cudaStream_t>(stream), rk);
+}
+
+__attribute__((visibility("default"))) moe_status_t
+moe_regroup_rows(const moe_shape_t *shape, int32_t rank, int32_t row_bytes, int32_t direction,
+                 const void *src, void *dst, const int32_t *assign_of_row,
+                 const int32_t *packed_row_of, const int32_t *offsets,
+                 const int64_t *packed_offsets, int32_t *offsets_local, moe_stream_t stream)
+{
+    moe_status_t rc = check_shape(shape, false, nullptr);
+    if (rc != MOE_OK)
+        return rc;
+    if (rank < 0 || rank >= shape->W || (direction != 0 && direction != 1) || row_bytes <= 0)
+        return MOE_ERR_INVALID_ARG;
+    if (row_bytes % 16 != 0)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (shape->N == 0)
+        return MOE_OK;  // no rows
+    if (!src || !dst || !assign_of_row || !packed_row_of || !offsets || !packed_offsets)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(dst) || !aligned4(assign_of_row) ||
+        !aligned4(packed_row_of) || !aligned4(offsets) ||
+        (reinterpret_cast<uintptr_t>(packed_offsets) & 7u) ||
+        (offsets_local && !aligned4(offsets_local)))
+        return MOE_ERR_MISALIGNED;
+    RegroupArgs ra;
+    ra.assign_of_row = assign_of_row;
+    ra.packed_row_of = packed_row_of;
+    ra.offsets = offsets;
+    ra.pk_off = packed_offsets;
+    ra.E = shape->E;
+    ra.K = shape->K;
+    ra.W = shape->W;
+    ra.S = shape->N / shape->W;
+    ra.rank = rank;
+    ra.row_vec = row_bytes / 16;
+    ra.src = static_cast<const uint4 *>(src);
+    ra.dst = static_cast<uint4 *>(dst);
+    ra.dir = direction;
+    ra.offsets_local = offsets_local;
+    regroup_rows_kernel<<<2 * num_sms(), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ra);
+    return launch_status();
 }
 
 __attribute__((visibility("default"))) moe_status_t

@@ -245,6 +245,51 @@ moe_status_t moe_dispatch_reroute(const moe_shape_t *shape, const uint16_t *x, c
                                   moe_stats_t *stats, void *ws, size_t ws_bytes,
                                   moe_stream_t stream);
 
+/* ---- W real ranks, one process per GPU (the exchange the one-GPU path emulates).
+ * [MoE 专家并行的 All-to-All 通信瓶颈, §All-to-All 分发与回收的机制: route Top-K, pack by
+ *  destination card, all-to-all, group by expert, grouped GEMM, pack by source, all-to-all,
+ *  weighted merge into the original token order]
+ * Rank r holds the tokens of home shard r (tokens [r N/W, (r+1) N/W)) and experts
+ * [r E/W, (r+1) E/W). After routing its own tokens (moe_route), every rank gathers every rank's
+ * topk_idx [N][K] and runs the whole batch's bookkeeping (cheap integer work over N*K), so the
+ * W ranks keep exactly the assignments one dispatch of the whole batch keeps (the capacity is
+ * per expert over all ranks' tokens, in the same priority order). */
+
+/* Rank `rank`'s dispatch. shape: the whole batch (N tokens over W ranks; MOE_FLAG_SLOT_MAJOR
+ * allowed, MOE_FLAG_REROUTE refused: its candidates are ranked by every token's logits).
+ * x_local [N/W][d] bf16: this rank's tokens. topk_idx_all [N][K]: every rank's routing.
+ * Outputs of the whole batch, the same on every rank: counts, kept, offsets, row_of,
+ * assign_of_row (as moe_dispatch), packed_row_of [N*K] (each kept assignment's row in the
+ * whole batch's packed layout, -1 if dropped), rank_matrix D [W][W] and packed_offsets
+ * [W*W+1] (required: the exchange's split sizes are D's row and column of this rank).
+ * Outputs of this rank: x_send [rows_alloc][d] bf16, the rows it sends, blocks (rank, j) for
+ * j = 0 .. W-1 (D[rank][j] rows each, rows inside a block by (expert, token)); send_row_of
+ * [N/W * K]: per slot of this rank's tokens, its row in x_send (and so in the buffer the
+ * return exchange brings back), -1 if dropped: the row_of of moe_combine after the return.
+ * Workspace: moe_workspace_size(shape). */
+moe_status_t moe_dispatch_rank(const moe_shape_t *shape, int32_t rank, const uint16_t *x_local,
+                               const int32_t *topk_idx_all, int32_t *counts, int32_t *kept,
+                               int32_t *offsets, int32_t *row_of, int32_t *assign_of_row,
+                               int32_t *packed_row_of, int32_t *send_row_of, uint16_t *x_send,
+                               int64_t *rank_matrix, int64_t *packed_offsets, moe_stats_t *stats,
+                               void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Rank `rank`'s rows between the exchange's order and its experts' order. The received
+ * buffer holds the blocks (i, rank) of i = 0 .. W-1 one after another (D[i][rank] rows each,
+ * as moe_dispatch_rank of rank i sent them); the sorted buffer holds this rank's experts' kept
+ * rows in the whole batch's expert-sorted order (rows offsets[r E/W] .. offsets[(r+1) E/W] - 1 of
+ * the one-GPU layout, shifted to 0). direction 0: src = received rows, dst = sorted rows (the
+ * way to the experts); direction 1: src = sorted rows, dst = rows in the received order (the
+ * way back, before the return exchange). row_bytes: bytes per row (a multiple of 16: d*2 for
+ * bf16 x, d*4 for fp32 y, the FP8 return payload's stride). offsets_local [E/W + 1] (nullable):
+ * this rank's experts' offsets into the sorted rows (the grouped GEMM's offsets). Inputs are
+ * moe_dispatch_rank's outputs (DEVICE). */
+moe_status_t moe_regroup_rows(const moe_shape_t *shape, int32_t rank, int32_t row_bytes,
+                              int32_t direction, const void *src, void *dst,
+                              const int32_t *assign_of_row, const int32_t *packed_row_of,
+                              const int32_t *offsets, const int64_t *packed_offsets,
+                              int32_t *offsets_local, moe_stream_t stream);
+
 /* Size of the library's fixed device scratch array used by moe_dispatch_static. */
 #define MOE_STATIC_SCRATCH_BYTES (1u << 20)
 

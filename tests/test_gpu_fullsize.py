@@ -86,7 +86,7 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     rr["expert_of"] = np.where(r["expert_of"] >= 0, remap[r["expert_of"]], -1).astype(np.int32)
     smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr, want_h=True)
     rows = torch.from_numpy(smp["sample_rows"]).cuda().long()
-    assert_rounded_h(got["h"][rows], smp["sample_h"], "h sample")
+    assert_rounded_h(got["h"][rows], smp["sample_h"], "h sample", w.d)
     rep_h = tolerance_report(got["h"][rows], smp["sample_h"])
     # y and out: the per-element bound of one rounding of h (the down projection's operand,
     # fp16) plus fp32 accumulation, the relative Frobenius bar and the max-abs bar
@@ -160,7 +160,7 @@ def full_output_check(orc, w, seed=0):
     np.testing.assert_array_equal(got["topk_idx"].cpu().numpy(), ref["topk_idx"])
     np.testing.assert_array_equal(got["row_of"].cpu().numpy(), ref["row_of"])
     R = ref["R"]
-    assert_rounded_h(got["h"][:R], ref["h_rows"], "h")
+    assert_rounded_h(got["h"][:R], ref["h_rows"], "h", w.d)
     row_expert = ref["expert_of"][ref["assign_of_row"]]
     ybound = h_bound_rows(ref["h_rows"], hx["w2"], got["w2_used"].cpu(), row_expert)
     assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")

@@ -71,7 +71,7 @@ def check_float_outputs(ref, got, inp, w, stated_bar: bool = True):
     (one rounding of h in the precision the run stored it in, fp32 accumulation), relative
     Frobenius 5e-3, and, when `stated_bar`, max-abs 2e-2 * RMS on y and on the output."""
     R = ref["R"]
-    assert_rounded_h(got["h"][:R], ref["h_rows"], "h")
+    assert_rounded_h(got["h"][:R], ref["h_rows"], "h", w.d)
     row_expert = ref["expert_of"][ref["assign_of_row"]]
     ybound = h_bound_rows(ref["h_rows"], inp["w2"], got.get("w2_used"), row_expert)
     assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
