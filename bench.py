@@ -292,8 +292,9 @@ def kernel_launches(w) -> int:
     placement kernel (the pass's control words are cleared by a memset, not a kernel); with
     re-routing a positions-only pass, the ranking kernel, then the full pass; each grouped GEMM
     once, or twice (CTA-pair tiles, then single-CTA tiles) when the experts average at least
-    768 rows and the K extent allows pair stages; the quantisation of h on the FP8 path; the
-    shared MLP's offsets and GEMMs; the combine."""
+    768 rows and the K extent allows pair stages, and for fp16 h one more gate/up launch (the
+    range pass, which does nothing while h is in fp16's range); the quantisation of h on the
+    FP8 path; the shared MLP's offsets and GEMMs; the combine."""
     N, d, f, E, K, W = w.N, w.d, w.f, w.E, w.K, w.W
     NK = N * K
     C = NK if not w.cf > 0 else min(NK, math.ceil(w.cf * N * K / E))
@@ -302,11 +303,12 @@ def kernel_launches(w) -> int:
     n += (2 + 1 + 2) if w.reroute else 2
     atom = 128 if w.fp8 else 64
     n += 2 if pair and (d // atom) % 2 == 0 else 1                     # gate/up
+    n += 0 if w.fp8 else 1                      # the fp16 range pass (does nothing in range)
     n += 1 if w.fp8 else 0                                              # h -> e4m3
     n += (2 if pair and (f // atom) % 2 == 0 else 1) if d % 256 == 0 else 1   # down
     if w.shared_f > 0:
         sp = N >= 768
-        n += 1 + (2 if sp else 1) + ((2 if sp else 1) if d % 256 == 0 else 1)
+        n += 1 + (2 if sp else 1) + 1 + ((2 if sp else 1) if d % 256 == 0 else 1)
     n += 1  # combine
     return n
 

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(HistArgs p)
 {
     extern __shared__ __align__(16) unsigned char hist_smem[];
     int *s_hist = reinterpret_cast<int *>(hist_smem);
-    __shared__ int s_vb, s_last;
+    __shared__ int s_vb, s_last, s_stop;
     const int E = p.E;
     if (threadIdx.x == 0)
         s_vb = (int)atomicAdd(&p.ctl[0], 1u);
@@ -313,28 +313,55 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(HistArgs p)
     __syncthreads();
     if (threadIdx.x == 0)
         st_release_u32(&flags[vb], kFlagAgg);
-    for (int e = threadIdx.x; e < E; e += kHistThreads) {
-        int excl = 0;
-        for (int q = vb - 1; q >= 0; --q) {
-            unsigned int f = ld_acquire_u32(&flags[q]);
-            if (f == 0) {
-                const uint64_t w0 = global_timer_ns();
-                while ((f = ld_acquire_u32(&flags[q])) == 0) {
-                    if (global_timer_ns() - w0 > p.timeout_ns) {
-                        set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
-                        break;
+    // look-back in windows of 32 predecessors: warp 0 reads their flags at once (waiting, with
+    // a bound, for any that has not published yet) and finds the nearest one whose inclusive
+    // prefix is out; every thread then adds its expert's histograms of the blocks after that
+    // one (and that prefix), or of the whole window and the walk goes on.
+    int excl[(256 + kHistThreads - 1) / kHistThreads] = {};  // one per expert of this thread
+    int cur = vb;
+    while (cur > 0) {
+        const int lo = max(0, cur - 32);
+        if (threadIdx.x < 32) {
+            const int q = cur - 1 - (int)threadIdx.x;
+            unsigned int f = kFlagIncl;
+            if (q >= lo) {
+                f = ld_acquire_u32(&flags[q]);
+                if (f == 0) {
+                    const uint64_t w0 = global_timer_ns();
+                    while ((f = ld_acquire_u32(&flags[q])) == 0) {
+                        if (global_timer_ns() - w0 > p.timeout_ns) {
+                            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+                            f = kFlagIncl;  // give up on it (the error is recorded)
+                            break;
+                        }
                     }
                 }
-                if (f == 0)
-                    break;  // gave up (the error is recorded)
             }
-            if (f == kFlagIncl) {
-                excl += __ldcg(p.incl + (size_t)q * E + e);
-                break;
-            }
-            excl += __ldcg(p.agg + (size_t)q * E + e);
+            const unsigned incl_mask = __ballot_sync(0xffffffffu, q >= lo && f == kFlagIncl);
+            if (threadIdx.x == 0)
+                s_stop = incl_mask ? cur - 1 - (__ffs(incl_mask) - 1) : -1;
         }
-        p.incl[(size_t)vb * E + e] = excl + s_hist[e];
+        __syncthreads();
+        const int stop = s_stop;  // the nearest block with its inclusive prefix out, or -1
+        const int from = stop >= 0 ? stop + 1 : lo;
+        int j = 0;
+        for (int e = threadIdx.x; e < E; e += kHistThreads, ++j) {
+            int acc = 0;
+            for (int q = from; q < cur; ++q)
+                acc += __ldcg(p.agg + (size_t)q * E + e);
+            if (stop >= 0)
+                acc += __ldcg(p.incl + (size_t)stop * E + e);
+            excl[j] += acc;
+        }
+        __syncthreads();  // s_stop is read by every thread before it is written again
+        if (stop >= 0)
+            break;
+        cur = lo;
+    }
+    {
+        int j = 0;
+        for (int e = threadIdx.x; e < E; e += kHistThreads, ++j)
+            p.incl[(size_t)vb * E + e] = excl[j] + s_hist[e];
     }
     __threadfence();
     __syncthreads();

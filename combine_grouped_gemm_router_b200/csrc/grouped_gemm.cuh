@@ -77,8 +77,33 @@ struct Args {
     const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
     int h_f16;               // modes 0, 1: h (mode 0's output, mode 1's A) and W2 are fp16,
                              // else bf16
+    // fp16 h's range (h_f16 only): *h_amax holds the largest |h| of the launch's first pass
+    // (fp32 bits; atomicMax). A second gate/up pass (h_pass 1) runs only when that exceeds
+    // fp16's largest finite value: it recomputes every tile with h scaled by 2^-k, k the
+    // smallest exponent that brings the largest |h| into range, and the down projection
+    // multiplies its accumulators by 2^k (powers of two: both exact).
+    uint32_t *h_amax;
+    int h_pass;
     uint64_t timeout_ns;
 };
+
+// fp16's largest finite value.
+constexpr float kF16Max = 65504.0f;
+
+// Exponent k of the scale 2^-k that brings a largest |h| (fp32 bits) into fp16's range: 0 when
+// it already is; -1 when it is not finite (nothing brings it into range).
+__device__ __forceinline__ int f16_range_exp(uint32_t amax_bits)
+{
+    if (amax_bits >= 0x7F800000u)
+        return -1;
+    float t = __uint_as_float(amax_bits);
+    int k = 0;
+    while (t > kF16Max) {  // halving a normal fp32 value is exact
+        t *= 0.5f;
+        ++k;
+    }
+    return k;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -385,9 +410,12 @@ __host__ __device__ constexpr int epilogue_cols(int MODE)
 // gate columns [0, 128) and up columns [128, 256) of N-slab n -> 128 bf16 values of h.
 // The FP8 mode first scales the accumulators by the row scale sx and the staged W1 / W3
 // channel scales ss.
+// hscale: the fp16 range scale 2^-k of a second pass (1 otherwise); hmax: the largest |h| bits
+// this thread stored (fp16 path).
 template <int MODE>
 __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr, int n, int row,
-                                                bool store, float sx, const float *ss)
+                                                bool store, float sx, const float *ss,
+                                                float hscale, uint32_t &hmax)
 {
     constexpr int CB = epilogue_cols(MODE);
     uint16_t *orow = reinterpret_cast<uint16_t *>(args.out) + (size_t)row * args.ldo;
@@ -425,15 +453,14 @@ __device__ __forceinline__ void swiglu_epilogue(const Args &args, uint32_t taddr
             }
             uint32_t p[CB / 2];
             if (MODE == 0 && args.h_f16) {
-                uint32_t bad = 0;
 #pragma unroll
                 for (int j = 0; j < CB / 2; ++j) {
-                    p[j] = pack_f16x2(silu_mul(gf[2 * j], uf[2 * j]),
-                                      silu_mul(gf[2 * j + 1], uf[2 * j + 1]));
-                    bad |= f16x2_nonfinite(p[j]);
+                    const float h0 = silu_mul(gf[2 * j], uf[2 * j]) * hscale;
+                    const float h1 = silu_mul(gf[2 * j + 1], uf[2 * j + 1]) * hscale;
+                    hmax = max(hmax, max(__float_as_uint(h0) & 0x7FFFFFFFu,
+                                         __float_as_uint(h1) & 0x7FFFFFFFu));
+                    p[j] = pack_f16x2(h0, h1);
                 }
-                if (bad)  // a value of h outside fp16's range (or not finite)
-                    set_dev_error(MOE_ERR_F16_RANGE);
             } else {
 #pragma unroll
                 for (int j = 0; j < CB / 2; ++j)
@@ -465,7 +492,7 @@ constexpr int Y_STAGE_BYTES = 4 * 4096 + 1024;
 template <int MODE, int BN>
 __device__ __forceinline__ void down_epilogue_fp8_return(const Args &args, uint32_t taddr, int n,
                                                          int row, bool store, float sx,
-                                                         const float *ss)
+                                                         const float *ss, float yscale)
 {
     constexpr int CB = epilogue_cols(MODE);
     uint8_t *prow = reinterpret_cast<uint8_t *>(args.out) + (size_t)row * args.y_stride;
@@ -486,6 +513,8 @@ __device__ __forceinline__ void down_epilogue_fp8_return(const Args &args, uint3
                 float o = __uint_as_float(v[32 * h + k]);
                 if constexpr (MODE == 3)
                     o *= sx * ss[c + 32 * h + k];
+                else
+                    o *= yscale;
                 f[k] = o;
                 mx = max(mx, __float_as_uint(o) & 0x7FFFFFFFu);
             }
@@ -514,14 +543,15 @@ __device__ __forceinline__ void down_epilogue_fp8_return(const Args &args, uint3
     }
 }
 
+// yscale: 2^k when h was stored scaled by 2^-k to stay in fp16's range (1 otherwise).
 template <int MODE, int BN>
 __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int n, int row,
                                               bool store, float sx, const float *ss,
                                               const CUtensorMap *ymap, uint32_t ystage,
-                                              int wrow0, bool wfull)
+                                              int wrow0, bool wfull, float yscale)
 {
     if (args.y_stride > 0) {
-        down_epilogue_fp8_return<MODE, BN>(args, taddr, n, row, store, sx, ss);
+        down_epilogue_fp8_return<MODE, BN>(args, taddr, n, row, store, sx, ss, yscale);
         return;
     }
     constexpr int CB = epilogue_cols(MODE);
@@ -552,6 +582,11 @@ __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, 
                         o.y *= sx * sc.y;
                         o.z *= sx * sc.z;
                         o.w *= sx * sc.w;
+                    } else {
+                        o.x *= yscale;
+                        o.y *= yscale;
+                        o.z *= yscale;
+                        o.w *= yscale;
                     }
                     const uint32_t addr = ystage + lane * 128 + ((j ^ (lane & 7)) << 4);
                     asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(o.x),
@@ -574,6 +609,11 @@ __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, 
                     o.y *= sx * sc.y;
                     o.z *= sx * sc.z;
                     o.w *= sx * sc.w;
+                } else {
+                    o.x *= yscale;
+                    o.y *= yscale;
+                    o.z *= yscale;
+                    o.w *= yscale;
                 }
                 dst[(c + j) / 4] = o;
             }
@@ -617,6 +657,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES + 2 + a); };
     const uint32_t done_bar = bar_base + 8u * (2 * STAGES + 4);
     const int E = args.E;
+    // fp16 range: the second gate/up pass runs only if the first one's largest |h| is beyond
+    // fp16's range; it stores h * 2^-k, and the down projection multiplies y by 2^k
+    int hk = 0;
+    if (args.h_f16 && (MODE == 1 || (MODE == 0 && args.h_pass == 1)))
+        hk = f16_range_exp(*reinterpret_cast<volatile uint32_t *>(args.h_amax));
+    const bool pass_needed = !(MODE == 0 && args.h_f16 && args.h_pass == 1) || hk > 0;
+    if (MODE == 0 && args.h_pass == 1 && hk < 0 && blockIdx.x == 0 && threadIdx.x == 0)
+        set_dev_error(MOE_ERR_F16_RANGE);  // a non-finite activation: no scale brings it in
+    const float hscale = (MODE == 0 && args.h_pass == 1 && hk > 0) ? pow2f(-hk) : 1.0f;
+    const float yscale = (MODE == 1 && hk > 0) ? pow2f(hk) : 1.0f;
+    uint32_t hmax = 0;  // largest |h| this thread stored (first gate/up pass)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -648,7 +699,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int e = visit_expert(i, E);
                 int rows = args.offsets[e + 1] - args.offsets[e];
                 rows = max(0, min(rows, args.rows_alloc));
-                mt = expert_selected(args.select, rows) ? (rows + BM - 1) / BM : 0;
+                mt = (expert_selected(args.select, rows) && pass_needed) ? (rows + BM - 1) / BM
+                                                                         : 0;
                 mtiles[i] = mt;
             }
             const int incl = warp_incl_scan(mt);
@@ -783,10 +835,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             if (GATE) {
-                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
+                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss, hscale, hmax);
             } else {
                 down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss, &tmB1,
-                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32);
+                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32,
+                                        yscale);
             }
             tc_fence_before();
             __syncwarp();
@@ -800,6 +853,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (!is_gate(MODE) && warp >= 2 && lane == 0)
         bulk_wait_all();  // this warp's y stores are complete before its shared memory goes
+    if (MODE == 0 && args.h_f16 && args.h_pass == 0 && warp >= 2) {
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, off));
+        if (lane == 0 && hmax)
+            atomicMax(args.h_amax, hmax);
+    }
     __syncwarp();
     tc_fence_before();
     __syncthreads();
@@ -929,6 +989,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * STAGES2 + 2 + a); };
     const uint32_t done_bar = bar_base + 8u * (2 * STAGES2 + 4);
     const int E = args.E;
+    // fp16 range (see grouped_gemm_kernel); the pair kernel runs first passes only
+    int hk = 0;
+    if (args.h_f16 && MODE == 1)
+        hk = f16_range_exp(*reinterpret_cast<volatile uint32_t *>(args.h_amax));
+    const bool pass_needed = true;
+    const float hscale = 1.0f;
+    const float yscale = (MODE == 1 && hk > 0) ? pow2f(hk) : 1.0f;
+    uint32_t hmax = 0;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < STAGES2; ++st) {
@@ -959,7 +1027,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int e = visit_expert(i, E);
                 int rows = args.offsets[e + 1] - args.offsets[e];
                 rows = max(0, min(rows, args.rows_alloc));
-                mt = expert_selected(args.select, rows) ? (rows + BMP - 1) / BMP : 0;
+                mt = (expert_selected(args.select, rows) && pass_needed) ? (rows + BMP - 1) / BMP
+                                                                         : 0;
                 mtiles[i] = mt;
             }
             const int incl = warp_incl_scan(mt);
@@ -1098,10 +1167,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             if (GATE) {
-                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss);
+                swiglu_epilogue<MODE>(args, taddr, n, row0 + r, r < valid, sx, ss, hscale, hmax);
             } else {
                 down_epilogue<MODE, BN>(args, taddr, n, row0 + r, r < valid, sx, ss, &tmB1,
-                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32);
+                                        y_stage + q * 4096, row0 + q * 32, valid - q * 32 >= 32,
+                                        yscale);
             }
             tc_fence_before();
             __syncwarp();
@@ -1115,6 +1185,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (!is_gate(MODE) && warp >= 2 && lane == 0)
         bulk_wait_all();  // this warp's y stores are complete before its shared memory goes
+    if (MODE == 0 && args.h_f16 && warp >= 2) {
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            hmax = max(hmax, __shfl_xor_sync(0xffffffffu, hmax, off));
+        if (lane == 0 && hmax)
+            atomicMax(args.h_amax, hmax);
+    }
     __syncwarp();
     tc_fence_before();
     if (*abort_flag) {

@@ -273,15 +273,28 @@ void launch_logits_pairs(const uint16_t *x, const float *wr, const float *bias, 
         <<<grid, L::NT, L::SMEM_BYTES, st>>>(x, wr, bias, logits, N, d, E);
 }
 
-template <int NW>
+template <int NW, int TT>
 void launch_router_topk(const moe_shape_t *s, const uint16_t *x, const float *wr, const float *bias,
                         int32_t *topk_idx, float *topk_w, float *logits,
                         unsigned long long *nonfinite, cudaStream_t st)
 {
-    using L = RouterTopkTile<NW>;
-    smem_attr_once(router_topk_kernel<NW>, L::SMEM_BYTES);
-    router_topk_kernel<NW><<<(s->N + kRtTokens - 1) / kRtTokens, L::NT, L::SMEM_BYTES, st>>>(
+    using L = RouterTopkTile<NW, TT>;
+    smem_attr_once(router_topk_kernel<NW, TT>, L::SMEM_BYTES);
+    router_topk_kernel<NW, TT><<<(s->N + L::TOK - 1) / L::TOK, L::NT, L::SMEM_BYTES, st>>>(
         x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
+}
+
+// Tokens per lane of the fused router: two (64-token CTAs) when that still gives every SM a
+// CTA, else one (32-token CTAs).
+template <int NW>
+void launch_router_topk_any(const moe_shape_t *s, const uint16_t *x, const float *wr,
+                            const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+                            unsigned long long *nonfinite, cudaStream_t st)
+{
+    if ((s->N + 63) / 64 >= num_sms())
+        launch_router_topk<NW, 2>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
+    else
+        launch_router_topk<NW, 1>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
 }
 
 // The router projection and the top-K selection. logits_out (nullable) receives the [N][E]
@@ -295,13 +308,17 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
     // every expert per CTA; the logits reach HBM only when asked for).
     if (E >= 32 && N >= 2048) {
         if (E <= 32)
-            launch_router_topk<2>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+            launch_router_topk_any<2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                      nonfinite, st);
         else if (E <= 64)
-            launch_router_topk<4>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+            launch_router_topk_any<4>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                      nonfinite, st);
         else if (E <= 128)
-            launch_router_topk<8>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+            launch_router_topk_any<8>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                      nonfinite, st);
         else
-            launch_router_topk<16>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite, st);
+            launch_router_topk_any<16>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                       nonfinite, st);
         return launch_status();
     }
     float *logits = logits_out ? logits_out : scratch;
@@ -631,10 +648,12 @@ bool use_pair_tiles(const moe_shape_t *s, const Geometry &g)
 
 // Grouped GEMM launches for E experts of width f over an A buffer of a_rows rows (the
 // tensor map's extent: rows past it read as zeros). `pair` selects the CTA-pair kernel;
-// `f16`: h is written (gate/up) or read together with fp16 W2 (down) as fp16, else bf16.
+// `f16`: h is written (gate/up) or read together with fp16 W2 (down) as fp16, else bf16;
+// h_amax (f16 only, DEVICE, one word): the largest |h| of the gate/up, which sizes the fp16
+// range scale (a second gate/up pass runs only when it is beyond fp16's range).
 moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *a,
                      const int32_t *offsets, const uint16_t *w1, const uint16_t *w3, uint16_t *h,
-                     bool f16, cudaStream_t st)
+                     bool f16, uint32_t *h_amax, cudaStream_t st)
 {
     CUtensorMap tA, tW1, tW3;
     if (!make_tmap(&tA, a, d, (uint64_t)a_rows) || !make_tmap(&tW1, w1, d, (uint64_t)E * f) ||
@@ -650,8 +669,11 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
     args.out = h;
     args.ldo = f;
     args.h_f16 = f16 ? 1 : 0;
+    args.h_amax = h_amax;
     args.timeout_ns = kWaitTimeoutNs;
     args.select = 0;
+    if (f16 && cudaMemsetAsync(h_amax, 0, sizeof(uint32_t), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
     if (pair) {
         args.select = 1;
         moe_status_t rc = launch_gemm_pair<0>(tA, tW1, tW3, args, st);
@@ -659,6 +681,12 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
             return rc;
         args.select = 2;
     }
+    moe_status_t rc = launch_gemm<0, 256>(tA, tW1, tW3, args, st);
+    if (rc != MOE_OK || !f16)
+        return rc;
+    // the fp16 range pass: every expert again with h scaled into range, only if it is needed
+    args.select = 0;
+    args.h_pass = 1;
     return launch_gemm<0, 256>(tA, tW1, tW3, args, st);
 }
 
@@ -666,7 +694,7 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
 // the y tensor map, unused then, is a copy of the W2 map).
 moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
                        const int32_t *offsets, const uint16_t *w2, void *y, int y_stride,
-                       bool f16, cudaStream_t st)
+                       bool f16, uint32_t *h_amax, cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
     if (!make_tmap(&tA, h, f, (uint64_t)a_rows, false, f16) ||
@@ -686,6 +714,7 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     args.ldo = d;
     args.y_stride = y_stride;
     args.h_f16 = f16 ? 1 : 0;
+    args.h_amax = h_amax;
     args.timeout_ns = kWaitTimeoutNs;
     args.select = 0;
     if (d % 256 == 0) {
@@ -795,12 +824,19 @@ moe_status_t quantize_rows_launch(const uint16_t *src, int64_t rows, int cols, u
 // h and the down-projection weights are fp16 unless the shape asks for bf16.
 inline bool h_is_f16(const moe_shape_t *s) { return !(s->flags & MOE_FLAG_H_BF16); }
 
+// The fp16 range word of an expert GEMM's h [rows_alloc][f]: the first 4 bytes of its last row,
+// which is never a kept row (rows_alloc >= R + 128).
+inline uint32_t *h_range_word(const uint16_t *h, const Geometry &g, int f)
+{
+    return reinterpret_cast<uint32_t *>(const_cast<uint16_t *>(h) + (size_t)(g.rows_alloc - 1) * f);
+}
+
 moe_status_t expert_up_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
                             const int32_t *offsets, const uint16_t *w1, const uint16_t *w3,
                             uint16_t *h, cudaStream_t st)
 {
     return gemm_up(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), x_sorted, offsets, w1,
-                   w3, h, h_is_f16(s), st);
+                   w3, h, h_is_f16(s), h_range_word(h, g, s->f), st);
 }
 
 moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *h,
@@ -808,7 +844,7 @@ moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uin
                               cudaStream_t st)
 {
     return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y,
-                     y_payload_stride(s), h_is_f16(s), st);
+                     y_payload_stride(s), h_is_f16(s), h_range_word(h, g, s->f), st);
 }
 
 moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
@@ -834,11 +870,13 @@ moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x
 {
     whole_range_offsets_kernel<<<1, 1, 0, st>>>(offsets2, s->N);
     const bool pair = s->N >= 768;
+    // the fp16 range word lives beside the offsets in the caller's scratch
+    uint32_t *amax = reinterpret_cast<uint32_t *>(offsets2 + 4);
     moe_status_t rc = gemm_up(1, s->d, f_s, s->N, pair, x, offsets2, ws1, ws3, h_s, h_is_f16(s),
-                              st);
+                              amax, st);
     if (rc != MOE_OK)
         return rc;
-    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, h_is_f16(s), st);
+    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, h_is_f16(s), amax, st);
 }
 
 moe_status_t combine_impl(const moe_shape_t *s, const void *y, const int32_t *row_of,

@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(TY *TX)
 // [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化] the gate's top-k runs
 // in the same kernel as the projection: the [N][E] logits need not go to HBM.
 //
-// A CTA takes 64 tokens and every expert. Lane l of every warp owns tokens l and l + 32 of the
-// tile, and warp w owns experts [16w, 16w + 16), so the W values a warp needs are the same
+// A CTA takes 32 TT tokens and every expert. Lane l of every warp owns tokens l, l + 32, ... of
+// the tile, and warp w owns experts [16w, 16w + 16), so the W values a warp needs are the same
 // for all its lanes (broadcast shared-memory loads) and each lane's x values are its own. The
 // 8-element pieces of d are walked in order; per element i a lane forms (x_t[i], x_t[i]) and
 // multiplies it by two neighbouring experts' (W_e[i], W_e+1[i]) in one packed fp32 FMA
@@ -259,32 +259,33 @@ __global__ void __launch_bounds__(TY *TX)
 // one chunk ahead of its use. After the chain, the tile's logits go to shared memory and each
 // warp selects the top K of its tokens: K rounds of a warp-wide argmax on (value desc, expert
 // asc), then a softmax over the K picked logits, as topk_softmax_kernel does.
-constexpr int kRtTokens = 64;  // tokens per CTA (two per lane)
 constexpr int kRtKC = 32;      // elements of d per staged chunk
 constexpr int kRtXRow = kRtKC + 8;  // bf16 per staged x row (16-byte pad)
 
-template <int NW>
+template <int NW, int TT>
 struct RouterTopkTile {
     static constexpr int NT = 32 * NW;
+    static constexpr int TOK = 32 * TT;     // tokens per CTA
     static constexpr int EP = 16 * NW + 4;  // fp32 per staged W^T row (16-byte pad)
-    static constexpr int X_BYTES = kRtTokens * kRtXRow * 2;
+    static constexpr int X_BYTES = TOK * kRtXRow * 2;
     static constexpr int W_BYTES = kRtKC * EP * 4;
     static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
-    static constexpr int LOGIT_BYTES = kRtTokens * (16 * NW + 1) * 4;  // epilogue tile
+    static constexpr int LOGIT_BYTES = TOK * (16 * NW + 1) * 4;  // epilogue tile
     static constexpr int SMEM_BYTES =
         2 * STAGE_BYTES > LOGIT_BYTES ? 2 * STAGE_BYTES : LOGIT_BYTES;
     // W elements each thread carries from global memory to the next stage: E_pad x KC / NT
     static constexpr int WV = (16 * NW * kRtKC) / (4 * NT);  // float4 per thread
 };
 
-template <int NW>
+template <int NW, int TT>
 __global__ void __launch_bounds__(32 * NW)
     router_topk_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
                        const float *__restrict__ bias, int N, int d, int E, int K,
                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                        float *__restrict__ logits, unsigned long long *nonfinite_count)
 {
-    using L = RouterTopkTile<NW>;
+    using L = RouterTopkTile<NW, TT>;
+    constexpr int kRtTokens = L::TOK;
     extern __shared__ __align__(16) unsigned char rt_smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * kRtTokens;
@@ -331,9 +332,9 @@ __global__ void __launch_bounds__(32 * NW)
         }
     };
 
-    float2 acc[2][8];  // [token of the lane][expert pair of the warp]
+    float2 acc[TT][8];  // [token of the lane][expert pair of the warp]
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < TT; ++t)
 #pragma unroll
         for (int p = 0; p < 8; ++p)
             acc[t][p] = make_float2(0.0f, 0.0f);
@@ -351,9 +352,9 @@ __global__ void __launch_bounds__(32 * NW)
         const float *ws = reinterpret_cast<const float *>(rt_smem + s * L::STAGE_BYTES + L::X_BYTES);
         const int kc = min(kRtKC, d - c * kRtKC);
         for (int kk = 0; kk < kc; kk += 8) {
-            uint4 xq[2];
+            uint4 xq[TT];
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+            for (int t = 0; t < TT; ++t)
                 xq[t] = *reinterpret_cast<const uint4 *>(xs + (lane + 32 * t) * kRtXRow + kk);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(32 * NW)
                     wp[2 * h + 1] = make_float2(v.z, v.w);
                 }
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
+                for (int t = 0; t < TT; ++t) {
                     const uint32_t word = (q < 2) ? xq[t].x : (q < 4) ? xq[t].y : (q < 6) ? xq[t].z : xq[t].w;
                     const float xv = (q & 1) ? bf16_hi(word) : bf16_lo(word);
                     const float2 xx = make_float2(xv, xv);
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(32 * NW)
     float *lt = reinterpret_cast<float *>(rt_smem);
     const int LR = EW + 1;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
+    for (int t = 0; t < TT; ++t) {
         const int tok = lane + 32 * t;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {

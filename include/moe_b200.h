@@ -122,9 +122,14 @@ typedef struct moe_shape {
  * (after fp32 accumulation and the SwiGLU in fp32) and that rounding is the largest error of the
  * layer; fp16 keeps 11 significant bits, bf16 8, so the error is 8 times smaller (on the
  * 128-expert layer with drops, max |error| / RMS(output) 0.0045 instead of 0.031; the bound
- * asked of the layer is 0.02). The price is fp16's range: a value of h beyond 65504 is stored
- * as infinity and sets MOE_ERR_F16_RANGE in the device error word (rerun that layer with this
- * flag). With MOE_FLAG_H_BF16: h is bf16 and W2 / Ws2 are the bf16 weights themselves.
+ * asked of the layer is 0.02). fp16's range is handled exactly: the gate/up GEMM records the
+ * largest |h|, and only when it exceeds 65504 a second gate/up pass (launched every time, it
+ * does nothing otherwise) stores h * 2^-k instead, k the smallest exponent that brings it into
+ * range, and the down GEMM multiplies its accumulators by 2^k (powers of two: no rounding). The
+ * record travels in the first 4 bytes of h's last row (row rows_alloc - 1, never a kept row), so
+ * moe_expert_down must get the h buffer moe_expert_up wrote (a caller that fills h by other
+ * means sets those 4 bytes to 0). A non-finite activation sets MOE_ERR_F16_RANGE.
+ * With MOE_FLAG_H_BF16: h is bf16 and W2 / Ws2 are the bf16 weights themselves.
  * The FP8 path (moe_expert_up_fp8, moe_layer_fp8) keeps its bf16 h before the e4m3
  * quantisation and ignores this flag. */
 #define MOE_FLAG_H_BF16 16u
@@ -433,7 +438,7 @@ moe_status_t moe_combine(const moe_shape_t *shape, const void *y, const int32_t 
  *  token passes through, added to the output of the routed expert(s)]
  * Same SwiGLU form as the experts: h_s = silu(x Ws1^T) * (x Ws3^T), y_s = h_s Ws2^T (fp32).
  * x [N][d], ws1, ws3 [f_shared][d] bf16; ws2 [d][f_shared] and h_s [N][f_shared] fp16 (bf16
- * with MOE_FLAG_H_BF16); y_s [N][d] fp32.
+ * with MOE_FLAG_H_BF16); y_s [N][d] fp32. The fp16 range record of h_s lives in ws.
  * f_shared % 128 == 0. ws: at least 256 bytes of device scratch. */
 moe_status_t moe_shared_expert(const moe_shape_t *shape, int32_t f_shared, const uint16_t *x,
                                const uint16_t *ws1, const uint16_t *ws3, const uint16_t *ws2,

@@ -320,3 +320,33 @@ def test_route_dispatch_small_hidden(orc, d, slot_major):
     packed[ref["packed_row_of"][kept_slots]] = xu[kept_slots // w.K]
     np.testing.assert_array_equal(_u16(got["x_packed"][:R]), packed)
     np.testing.assert_array_equal(got["D"].cpu().numpy().reshape(w.W, w.W), ref["D"])
+
+
+@pytest.mark.parametrize("scale", [1.0, 400.0])
+def test_fp16_range_pass(orc, scale):
+    """Activations beyond fp16's range (x scaled by 400: |h| far above 65504): the range pass
+    stores h * 2^-k and the down projection multiplies back by 2^k, so the layer stays within
+    the stated bar of the oracle and no error is recorded; in range (scale 1) the record stays
+    below 65504 and the second pass does nothing."""
+    import combine_grouped_gemm_router_b200 as m
+    w = Workload("range", N=256, d=256, f=256, E=8, K=2, W=4)
+    inp = make_layer_inputs(w, seed=6)
+    inp["x"] = (inp["x"].float() * scale).to(torch.bfloat16)
+    ref = orc.layer(inp, w.K, w.W, w.cf, want_h=True)
+    got = run_stages(inp, w)
+    assert got["dev_error"] == 0
+    R = ref["R"]
+    amax = got["h"][-1].view(torch.int32)[0:2].cpu().numpy().view(np.uint32)[0]
+    top = float(np.abs(ref["h_rows"]).max())
+    assert np.float32(amax.view(np.float32)) == pytest.approx(top, rel=2e-3)
+    assert (top > 65504) == (scale > 1)
+    if scale > 1:  # h was stored scaled into range: compare it scaled back
+        k = int(np.ceil(np.log2(top / 65504.0)))
+        hk = got["h"][:R].double() * 2.0 ** k
+        rel = float(((hk.cpu().numpy() - ref["h_rows"]) ** 2).sum() / (ref["h_rows"] ** 2).sum())
+        assert rel ** 0.5 <= 5e-3
+    assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
+    assert_within_tolerance(got["out"], ref["out"], "out")
+    lay = run_layer(inp, w)
+    assert lay["dev_error"] == 0
+    assert torch.equal(lay["out"], got["out"])
