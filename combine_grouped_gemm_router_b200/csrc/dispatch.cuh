@@ -282,7 +282,7 @@ __device__ void pass_totals(const HistArgs &p, unsigned char *smem)
 // last then forms the pass's totals. A block only ever waits for blocks that took earlier
 // tickets, which are resident or done, so the waits end; each is bounded all the same
 // (MOE_ERR_DEVICE_TIMEOUT). The scan stays deterministic: positions are exact counts.
-__global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(HistArgs p)
+__global__ void __launch_bounds__(kHistThreads, 4) dispatch_hist_kernel(HistArgs p)
 {
     extern __shared__ __align__(16) unsigned char hist_smem[];
     int *s_hist = reinterpret_cast<int *>(hist_smem);
@@ -346,11 +346,15 @@ __global__ void __launch_bounds__(kHistThreads) dispatch_hist_kernel(HistArgs p)
         const int from = stop >= 0 ? stop + 1 : lo;
         int j = 0;
         for (int e = threadIdx.x; e < E; e += kHistThreads, ++j) {
-            int acc = 0;
-            for (int q = from; q < cur; ++q)
-                acc += __ldcg(p.agg + (size_t)q * E + e);
-            if (stop >= 0)
-                acc += __ldcg(p.incl + (size_t)stop * E + e);
+            // the window's (at most 32) histograms: every load issued before the first add
+            int part[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                part[i] = from + i < cur ? __ldcg(p.agg + (size_t)(from + i) * E + e) : 0;
+            int acc = stop >= 0 ? __ldcg(p.incl + (size_t)stop * E + e) : 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                acc += part[i];
             excl[j] += acc;
         }
         __syncthreads();  // s_stop is read by every thread before it is written again
@@ -408,6 +412,8 @@ struct PlaceArgs {
     void *x_sorted, *x_packed;          // bf16 rows, or e4m3 rows with the FP8 payload
     float *sorted_scale, *packed_scale;  // FP8 payload: one scale per row
     moe_stats_t *stats;                  // nullable: dedup_pairs is accumulated here
+    int slots;                           // bf16 copy: ring slots per warp (1 to 3)
+    uint64_t timeout_ns;                 // bound of every wait of the bulk copy
 };
 
 // Shared memory of dispatch_place_kernel: per-warp counts [8][E] and offsets [E+1] (int32),
@@ -416,6 +422,53 @@ struct PlaceArgs {
 __host__ __device__ inline size_t place_smem_bytes(int E, int K)
 {
     return ((size_t)9 * E + 1 + (size_t)3 * kDispatchHB * K) * 4;
+}
+
+// The bf16 rows move by bulk copies (cp.async.bulk) in pieces of at most kPiece bytes: global
+// -> a shared-memory ring slot (one mbarrier per slot) -> every kept destination row. The ring
+// follows the tables above (128-byte aligned): per warp `slots` pieces, then the mbarriers.
+constexpr int kPiece = 4096;
+
+__host__ __device__ inline size_t place_ring_offset(int E, int K)
+{
+    return (place_smem_bytes(E, K) + 127) & ~(size_t)127;
+}
+
+__host__ __device__ inline size_t place_smem_total(int E, int K, int slots)
+{
+    return place_ring_offset(E, K) + (size_t)8 * slots * kPiece + (size_t)8 * slots * 8;
+}
+
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_store_s2g(void *dst, uint32_t src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Bounded wait on an mbarrier phase; false (and MOE_ERR_DEVICE_TIMEOUT) when it runs out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > timeout_ns) {
+            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
 }
 
 // One CTA per (token block, part). Positions: for every virtual block of the token block (all
@@ -560,41 +613,99 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
     __syncthreads();
 
     if (!p.e4m3) {
-        // a column slice of every row of the block (16-byte chunks [cbeg, cend)): lane l takes
-        // chunks cbeg + l, + 32, ...; warp w takes tokens w, w + 8, ... and loads one chunk of
-        // all of them before storing any (eight independent loads in flight per lane)
-        constexpr int TB = kDispatchHB / 8;  // tokens per warp
-        const int nvec = p.d >> 3;
-        const int cs = (nvec + parts - 1) / parts;
-        const int cbeg = part * cs, cend = min(nvec, cbeg + cs);
-        uint4 *dst_s = reinterpret_cast<uint4 *>(p.x_sorted);
-        uint4 *dst_p = reinterpret_cast<uint4 *>(p.x_packed);
-        const uint4 *src = reinterpret_cast<const uint4 *>(xb);
-        for (int c = cbeg + lane; c < cend; c += 32) {
-            uint4 v[TB];
-#pragma unroll
-            for (int i = 0; i < TB; ++i) {
-                const int lt = warp + 8 * i;
-                if (lt < nt)
-                    v[i] = __ldcs(src + (size_t)lt * nvec + c);
-            }
-#pragma unroll
-            for (int i = 0; i < TB; ++i) {
-                const int lt = warp + 8 * i;
-                if (lt >= nt)
+        // Bulk copies. The block's items are (token, piece) pairs, q = lt * npc + piece; part
+        // p's warp w takes q = p + parts * (w + 8 j) of the tokens that keep a slot. Per warp a
+        // pipeline over its items: the piece of item c + 1 is loaded into its ring slot while
+        // item c's stores go out (lane k < K stores slot k's expert-sorted and packed rows),
+        // with up to slots - 1 items' stores in flight; a slot is reloaded only once the stores
+        // that read it have read it.
+        const uint32_t rb = (uint32_t)p.d * 2u;
+        const int npc = (int)((rb + kPiece - 1) / kPiece);
+        const int nq = nt * npc, qstep = parts * 8, S = p.slots;
+        unsigned char *smem_b = reinterpret_cast<unsigned char *>(place_smem);
+        const uint32_t ring = smem_u32(smem_b + place_ring_offset(E, K)) + warp * S * kPiece;
+        const uint32_t bars = smem_u32(smem_b + place_ring_offset(E, K)) + 8 * S * kPiece +
+                              warp * S * 8;
+        if (lane == 0) {
+            for (int j = 0; j < S; ++j)
+                mbar_init(bars + 8 * j, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncwarp();
+        // the next item at or after q whose token keeps a slot (nq: none)
+        auto next_item = [&](int q) {
+            for (; q < nq; q += qstep) {
+                const int lt = q / npc;
+                if (__any_sync(0xffffffffu, lane < K && s_rk[lt * K + lane] >= 0))
                     break;
-                for (int k = 0; k < K; ++k) {
-                    const int rk = s_rk[lt * K + k];
-                    if (rk < 0)
-                        continue;
-                    const int pk = s_pk[lt * K + k];
+            }
+            return q < nq ? q : nq;
+        };
+        auto issue_load = [&](int q, int slot) {
+            if (lane == 0) {
+                const int lt = q / npc, pc = q - lt * npc;
+                const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
+                const unsigned char *src = reinterpret_cast<const unsigned char *>(xb) +
+                                           (size_t)lt * rb + (size_t)pc * kPiece;
+                mbar_arrive_expect_tx(bars + 8 * slot, bytes);
+                bulk_load_g2s(ring + slot * kPiece, src, bytes, bars + 8 * slot);
+            }
+        };
+        auto wait_read = [&](int pending) {  // this lane's store groups beyond `pending` read
+            if (pending <= 0)
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            else
+                asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        };
+        unsigned char *dst_s = reinterpret_cast<unsigned char *>(p.x_sorted);
+        unsigned char *dst_p = reinterpret_cast<unsigned char *>(p.x_packed);
+        int q_cur = next_item(part + parts * warp);
+        int c = 0;          // items whose stores have been issued
+        int loaded = -1;    // the last item index whose load was issued
+        if (q_cur < nq) {
+            issue_load(q_cur, 0);
+            loaded = 0;
+        }
+        while (q_cur < nq) {
+            const int q_nxt = next_item(q_cur + qstep);
+            if (S > 1 && q_nxt < nq) {  // load item c + 1 (its slot's earlier stores read)
+                wait_read(S - 2);
+                __syncwarp();
+                issue_load(q_nxt, (c + 1) % S);
+                loaded = c + 1;
+            }
+            const int slot = c % S;
+            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((c / S) & 1), p.timeout_ns))
+                break;
+            const int lt = q_cur / npc, pc = q_cur - lt * npc;
+            const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
+            const size_t off = (size_t)pc * kPiece;
+            if (lane < K) {  // x_sorted is null for a rank's dispatch (send rows only)
+                const int rk = s_rk[lt * K + lane];
+                if (rk >= 0) {
                     if (dst_s)
-                        dst_s[(size_t)rk * nvec + c] = v[i];
+                        bulk_store_s2g(dst_s + (size_t)rk * rb + off, ring + slot * kPiece, bytes);
+                    const int pk = s_pk[lt * K + lane];
                     if (pk >= 0)
-                        dst_p[(size_t)pk * nvec + c] = v[i];
+                        bulk_store_s2g(dst_p + (size_t)pk * rb + off, ring + slot * kPiece, bytes);
                 }
             }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            ++c;
+            if (S == 1 && q_nxt < nq) {  // one slot: reload it once this item's stores read it
+                wait_read(0);
+                __syncwarp();
+                issue_load(q_nxt, 0);
+                loaded = c;
+            }
+            q_cur = q_nxt;
         }
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        // loads issued and not consumed (only after a wait that ran out): let them land first
+        if (lane == 0)
+            for (int j = c; j <= loaded; ++j)
+                mbar_wait_bounded(bars + 8 * (j % S), (uint32_t)((j / S) & 1), p.timeout_ns);
+        __syncwarp();
         return;
     }
 

@@ -284,17 +284,15 @@ void launch_router_topk(const moe_shape_t *s, const uint16_t *x, const float *wr
         x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
 }
 
-// Tokens per lane of the fused router: two (64-token CTAs) when that still gives every SM a
-// CTA, else one (32-token CTAs).
+// The fused router with two tokens per lane (64-token CTAs): measured faster than one token per
+// lane (32-token CTAs) even where 64-token CTAs leave SMs idle (155 against 204 us at N = 8192,
+// E = 128), since one token per lane is bound by the broadcast W loads.
 template <int NW>
 void launch_router_topk_any(const moe_shape_t *s, const uint16_t *x, const float *wr,
                             const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
                             unsigned long long *nonfinite, cudaStream_t st)
 {
-    if ((s->N + 63) / 64 >= num_sms())
-        launch_router_topk<NW, 2>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
-    else
-        launch_router_topk<NW, 1>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
+    launch_router_topk<NW, 2>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
 }
 
 // The router projection and the top-K selection. logits_out (nullable) receives the [N][E]
@@ -376,15 +374,36 @@ struct DispatchScratch {
     int32_t *moved;
 };
 
-// Column (bf16) or token (FP8) parts per token block of the placement kernel: enough CTAs for
-// about eight per SM, each part at least 32 16-byte chunks of a row (one per lane; or one
-// token per warp for the FP8 payload).
+// Row pieces of a token block (an upper bound: the block's tokens times pieces per row).
+int place_items(const moe_shape_t *s, const Geometry &g)
+{
+    const int tokens = g.S < kDispatchHB ? g.S : kDispatchHB;
+    const int npc = (int)(((size_t)s->d * 2 + kPiece - 1) / kPiece);
+    return tokens * npc;
+}
+
+// Parts per token block of the placement kernel. FP8 payload: token parts, enough CTAs for
+// about eight per SM, at least one token per warp. bf16 rows (bulk copies of pieces): about
+// four CTAs per SM, at least four pieces per part.
 int place_parts(const moe_shape_t *s, const Geometry &g, bool e4m3)
 {
-    const int want = (8 * num_sms() + g.nblk - 1) / g.nblk;
-    const int cap = e4m3 ? (kDispatchHB + 7) / 8 : ((s->d / 8) + 31) / 32;
+    int want, cap;
+    if (e4m3) {
+        want = (8 * num_sms() + g.nblk - 1) / g.nblk;
+        cap = (kDispatchHB + 7) / 8;
+    } else {
+        want = (4 * num_sms() + g.nblk - 1) / g.nblk;
+        cap = (place_items(s, g) + 3) / 4;
+    }
     const int parts = want < cap ? want : cap;
     return parts < 1 ? 1 : parts;
+}
+
+// Ring slots per warp of the bf16 bulk copy: the pieces a warp takes, 1 to 3.
+int place_slots(const moe_shape_t *s, const Geometry &g, int parts)
+{
+    const int per_warp = (place_items(s, g) + 8 * parts - 1) / (8 * parts);
+    return per_warp < 1 ? 1 : per_warp > 3 ? 3 : per_warp;
 }
 
 // One dispatch pass over `rounds` rounds of virtual blocks: the control words zeroed, the
@@ -460,7 +479,9 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
     pa.stats = stats;
     pa.x = x;
     pa.d = s->d;
+    pa.timeout_ns = kWaitTimeoutNs;
     int parts = 1;
+    size_t psm = place_smem_bytes(s->E, s->K);
     if (pay) {
         pa.copy = 1;
         pa.e4m3 = pay->e4m3 ? 1 : 0;
@@ -469,9 +490,13 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
         pa.sorted_scale = pay->sorted_scale;
         pa.packed_scale = pay->packed_scale;
         parts = place_parts(s, g, pay->e4m3);
+        if (!pay->e4m3) {
+            pa.slots = place_slots(s, g, parts);
+            psm = place_smem_total(s->E, s->K, pa.slots);
+        }
     }
-    const size_t psm = place_smem_bytes(s->E, s->K);
-    if (smem_attr_once(dispatch_place_kernel, (int)place_smem_bytes(kMaxE, kMaxK)) != cudaSuccess)
+    if (smem_attr_once(dispatch_place_kernel, (int)place_smem_total(kMaxE, kMaxK, 3)) !=
+        cudaSuccess)
         return MOE_ERR_CUDA;
     dispatch_place_kernel<<<dim3(g.nblk, parts), kPlaceThreads, psm, st>>>(pa);
     return launch_status();

@@ -243,6 +243,83 @@ __global__ void __launch_bounds__(TY *TX)
 }
 
 // ---------------------------------------------------------------------------
+// Top-K selection of one token by one warp: lane l holds the logits of experts l + 32 j
+// (j < MAXJ, E <= 32 MAXJ). K rounds of a warp-wide argmax on (value desc, expert asc), then a
+// softmax over the K picked logits. NaN counts as -inf for the choice; any non-finite logit
+// flags MOE_ERR_NONFINITE (the token's result is then unspecified). lrow: the token's logits
+// (shared or global memory); logits_out (nullable): where to copy them.
+template <int MAXJ>
+__device__ __forceinline__ void topk_select_warp(const float *lrow, int E, int K, size_t t,
+                                                 float *logits_out, int32_t *__restrict__ topk_idx,
+                                                 float *__restrict__ topk_w,
+                                                 unsigned long long *nonfinite_count)
+{
+    const int lane = threadIdx.x & 31;
+    float v[MAXJ];
+    unsigned taken = 0;  // bit j: entry j unavailable (chosen or absent)
+    bool bad = false;
+#pragma unroll
+    for (int j = 0; j < MAXJ; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) {
+            float l = lrow[e];
+            if (logits_out)
+                logits_out[t * E + e] = l;
+            if (!isfinite(l)) {
+                bad = true;
+                if (isnan(l))
+                    l = -INFINITY;
+            }
+            v[j] = l;
+        } else {
+            v[j] = -INFINITY;
+            taken |= 1u << j;
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) {
+        set_dev_error(MOE_ERR_NONFINITE);
+        if (nonfinite_count)
+            atomicAdd(nonfinite_count, 1ull);
+    }
+    float my_v = 0.0f;
+    int my_e = 0;
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int be = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < MAXJ; ++j) {
+            const int e = lane + 32 * j;
+            if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) {
+                bv = v[j];
+                be = e;
+            }
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+            if (ov > bv || (ov == bv && oe < be)) {
+                bv = ov;
+                be = oe;
+            }
+        }
+        if ((be & 31) == lane)
+            taken |= 1u << (be >> 5);
+        if (lane == k) {
+            my_v = bv;
+            my_e = be;
+        }
+    }
+    const float top = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = lane < K ? expf(my_v - top) : 0.0f;
+    const float ssum = warp_sum(ex);
+    if (lane < K) {
+        topk_idx[t * K + lane] = my_e;
+        topk_w[t * K + lane] = ex / ssum;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Router projection fused with the top-K selection, for many tokens and E >= 32.
 //
 // [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化] the gate's top-k runs
@@ -405,153 +482,27 @@ __global__ void __launch_bounds__(32 * NW)
     }
     __syncthreads();
 
-    // top-K of each token: warp w takes tokens w, w + NW, ...; lane l holds experts l + 32j
-    constexpr int MAXJ = (16 * NW + 31) / 32;
+    // top-K of each token: warp w takes tokens w, w + NW, ...
     for (int tok = warp; tok < kRtTokens; tok += NW) {
         const int t = t0 + tok;
         if (t >= N)
             break;
-        const float *lrow = lt + tok * LR;
-        float v[MAXJ];
-        unsigned taken = 0;
-        bool bad = false;
-#pragma unroll
-        for (int j = 0; j < MAXJ; ++j) {
-            const int e = lane + 32 * j;
-            if (e < E) {
-                float l = lrow[e];
-                if (logits)
-                    logits[(size_t)t * E + e] = l;
-                if (!isfinite(l)) {
-                    bad = true;
-                    if (isnan(l))
-                        l = -INFINITY;
-                }
-                v[j] = l;
-            } else {
-                v[j] = -INFINITY;
-                taken |= 1u << j;
-            }
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) {
-            set_dev_error(MOE_ERR_NONFINITE);
-            if (nonfinite_count)
-                atomicAdd(nonfinite_count, 1ull);
-        }
-        float my_v = 0.0f;
-        int my_e = 0;
-        for (int k = 0; k < K; ++k) {
-            float bv = -INFINITY;
-            int be = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < MAXJ; ++j) {
-                const int e = lane + 32 * j;
-                if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) {
-                    bv = v[j];
-                    be = e;
-                }
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) {
-                    bv = ov;
-                    be = oe;
-                }
-            }
-            if ((be & 31) == lane)
-                taken |= 1u << (be >> 5);
-            if (lane == k) {
-                my_v = bv;
-                my_e = be;
-            }
-        }
-        const float top = __shfl_sync(0xffffffffu, my_v, 0);
-        const float ex = lane < K ? expf(my_v - top) : 0.0f;
-        const float ssum = warp_sum(ex);
-        if (lane < K) {
-            topk_idx[(size_t)t * K + lane] = my_e;
-            topk_w[(size_t)t * K + lane] = ex / ssum;
-        }
+        topk_select_warp<(16 * NW + 31) / 32>(lt + tok * LR, E, K, (size_t)t, logits, topk_idx,
+                                              topk_w, nonfinite_count);
     }
 }
 
-// One warp per token. Lane l holds logits of experts l + 32*j (E <= 256).
-// K rounds of a warp-wide argmax on (value desc, expert asc); then a softmax over
-// the K picked logits. NaN is treated as -inf for the choice; any non-finite
-// logit flags MOE_ERR_NONFINITE (the token's result is then unspecified).
+// One warp per token (E <= 256): topk_select_warp on the token's row of the [N][E] logits.
 __global__ void __launch_bounds__(256)
     topk_softmax_kernel(const float *__restrict__ logits, int N, int E, int K,
                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                         unsigned long long *nonfinite_count)
 {
-    constexpr int MAXJ = 8;
-    const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= N)
         return;
-    const float *lrow = logits + (size_t)t * E;
-    float v[MAXJ];
-    unsigned taken = 0;  // bit j: entry j unavailable (chosen or absent)
-    bool bad = false;
-#pragma unroll
-    for (int j = 0; j < MAXJ; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E) {
-            float l = lrow[e];
-            if (!isfinite(l)) {
-                bad = true;
-                if (isnan(l))
-                    l = -INFINITY;
-            }
-            v[j] = l;
-        } else {
-            v[j] = -INFINITY;
-            taken |= 1u << j;
-        }
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) {
-        set_dev_error(MOE_ERR_NONFINITE);
-        if (nonfinite_count)
-            atomicAdd(nonfinite_count, 1ull);
-    }
-    float my_v = 0.0f;
-    int my_e = 0;
-    for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < MAXJ; ++j) {
-            const int e = lane + 32 * j;
-            if (!((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) {
-                bv = v[j];
-                be = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > bv || (ov == bv && oe < be)) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        if ((be & 31) == lane)
-            taken |= 1u << (be >> 5);
-        if (lane == k) {
-            my_v = bv;
-            my_e = be;
-        }
-    }
-    const float top = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = lane < K ? expf(my_v - top) : 0.0f;
-    const float s = warp_sum(ex);
-    if (lane < K) {
-        topk_idx[(size_t)t * K + lane] = my_e;
-        topk_w[(size_t)t * K + lane] = ex / s;
-    }
+    topk_select_warp<8>(logits + (size_t)t * E, E, K, (size_t)t, nullptr, topk_idx, topk_w,
+                        nonfinite_count);
 }
 
 }  // namespace moe
