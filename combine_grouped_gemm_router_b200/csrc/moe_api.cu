@@ -278,21 +278,21 @@ void launch_router_topk(const moe_shape_t *s, const uint16_t *x, const float *wr
                         int32_t *topk_idx, float *topk_w, float *logits,
                         unsigned long long *nonfinite, cudaStream_t st)
 {
-    using L = RouterTopkTile<NW, TT>;
-    smem_attr_once(router_topk_kernel<NW, TT>, L::SMEM_BYTES);
-    router_topk_kernel<NW, TT><<<(s->N + L::TOK - 1) / L::TOK, L::NT, L::SMEM_BYTES, st>>>(
+    using L = RouterTopkTile<NW, TT, 16>;
+    smem_attr_once(router_topk_kernel<NW, TT, 16>, L::SMEM_BYTES);
+    router_topk_kernel<NW, TT, 16><<<(s->N + L::TOK - 1) / L::TOK, L::NT, L::SMEM_BYTES, st>>>(
         x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
 }
 
-// The fused router with two tokens per lane (64-token CTAs): measured faster than one token per
-// lane (32-token CTAs) even where 64-token CTAs leave SMs idle (155 against 204 us at N = 8192,
-// E = 128), since one token per lane is bound by the broadcast W loads.
-template <int NW>
-void launch_router_topk_any(const moe_shape_t *s, const uint16_t *x, const float *wr,
-                            const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
-                            unsigned long long *nonfinite, cudaStream_t st)
+template <int EPAD, int TM>
+void launch_router_tile8(const moe_shape_t *s, const uint16_t *x, const float *wr,
+                         const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
+                         unsigned long long *nonfinite, cudaStream_t st)
 {
-    launch_router_topk<NW, 2>(s, x, wr, bias, topk_idx, topk_w, logits, nonfinite, st);
+    using L = RouterTile8<EPAD, TM>;
+    smem_attr_once(router_tile8_kernel<EPAD, TM>, L::SMEM_BYTES);
+    router_tile8_kernel<EPAD, TM><<<(s->N + TM - 1) / TM, L::NT, L::SMEM_BYTES, st>>>(
+        x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
 }
 
 // The router projection and the top-K selection. logits_out (nullable) receives the [N][E]
@@ -305,18 +305,25 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
     // Many tokens and E >= 32: the projection and the selection in one kernel (64 tokens x
     // every expert per CTA; the logits reach HBM only when asked for).
     if (E >= 32 && N >= 2048) {
+        // E <= 64 with at least 3 CTAs (6 warps) per SM: the register-tiled form (8 tokens x
+        // 8 experts per thread; measured 510 against 537 us at N = 32768, d = 4096, E = 64).
+        // Fewer logits per SM leave it a warp per scheduler, where the broadcast form is
+        // faster (151 against 167 us at N = 8192, d = 2048, E = 128).
         if (E <= 32)
-            launch_router_topk_any<2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                      nonfinite, st);
+            launch_router_topk<2, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                     nonfinite, st);
+        else if (E <= 64 && (long long)N >= 64LL * 3 * num_sms())
+            launch_router_tile8<64, 64>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                        nonfinite, st);
         else if (E <= 64)
-            launch_router_topk_any<4>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                      nonfinite, st);
+            launch_router_topk<4, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                     nonfinite, st);
         else if (E <= 128)
-            launch_router_topk_any<8>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                      nonfinite, st);
+            launch_router_topk<8, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                     nonfinite, st);
         else
-            launch_router_topk_any<16>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                       nonfinite, st);
+            launch_router_topk<16, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
+                                      nonfinite, st);
         return launch_status();
     }
     float *logits = logits_out ? logits_out : scratch;

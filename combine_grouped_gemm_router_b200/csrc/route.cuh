@@ -339,35 +339,35 @@ __device__ __forceinline__ void topk_select_warp(const float *lrow, int E, int K
 constexpr int kRtKC = 32;      // elements of d per staged chunk
 constexpr int kRtXRow = kRtKC + 8;  // bf16 per staged x row (16-byte pad)
 
-template <int NW, int TT>
+template <int NW, int TT, int EW>
 struct RouterTopkTile {
     static constexpr int NT = 32 * NW;
     static constexpr int TOK = 32 * TT;     // tokens per CTA
-    static constexpr int EP = 16 * NW + 4;  // fp32 per staged W^T row (16-byte pad)
+    static constexpr int EP = EW * NW + 4;  // fp32 per staged W^T row (16-byte pad)
     static constexpr int X_BYTES = TOK * kRtXRow * 2;
     static constexpr int W_BYTES = kRtKC * EP * 4;
     static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
-    static constexpr int LOGIT_BYTES = TOK * (16 * NW + 1) * 4;  // epilogue tile
+    static constexpr int LOGIT_BYTES = TOK * (EW * NW + 1) * 4;  // epilogue tile
     static constexpr int SMEM_BYTES =
         2 * STAGE_BYTES > LOGIT_BYTES ? 2 * STAGE_BYTES : LOGIT_BYTES;
     // W elements each thread carries from global memory to the next stage: E_pad x KC / NT
-    static constexpr int WV = (16 * NW * kRtKC) / (4 * NT);  // float4 per thread
+    static constexpr int WV = (EW * NW * kRtKC) / (4 * NT);  // float4 per thread
 };
 
-template <int NW, int TT>
+template <int NW, int TT, int EW>
 __global__ void __launch_bounds__(32 * NW)
     router_topk_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
                        const float *__restrict__ bias, int N, int d, int E, int K,
                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                        float *__restrict__ logits, unsigned long long *nonfinite_count)
 {
-    using L = RouterTopkTile<NW, TT>;
+    using L = RouterTopkTile<NW, TT, EW>;
     constexpr int kRtTokens = L::TOK;
     extern __shared__ __align__(16) unsigned char rt_smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * kRtTokens;
     const int nchunks = (d + kRtKC - 1) / kRtKC;
-    const int EW = 16 * NW;  // experts covered (E rounded up to 16 per warp)
+    const int EC = EW * NW;  // experts covered (E rounded up to EW per warp)
 
     // x chunk c -> stage s (cp.async, 16 bytes per copy; rows past N are left alone)
     auto stage_x = [&](int c, int s) {
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(32 * NW)
         const int k0 = c * kRtKC, kc = c < nchunks ? min(kRtKC, d - k0) : 0;
 #pragma unroll
         for (int j = 0; j < L::WV; ++j) {
-            const int idx = tid + j * L::NT;  // over EW x (KC / 4), element quad fastest
+            const int idx = tid + j * L::NT;  // over EC x (KC / 4), element quad fastest
             const int e = idx / (kRtKC / 4), q = idx % (kRtKC / 4);
             wreg[j] = (e < E && q * 4 < kc)
                           ? __ldg(reinterpret_cast<const float4 *>(wr + (size_t)e * d + k0) + q)
@@ -409,11 +409,11 @@ __global__ void __launch_bounds__(32 * NW)
         }
     };
 
-    float2 acc[TT][8];  // [token of the lane][expert pair of the warp]
+    float2 acc[TT][EW / 2];  // [token of the lane][expert pair of the warp]
 #pragma unroll
     for (int t = 0; t < TT; ++t)
 #pragma unroll
-        for (int p = 0; p < 8; ++p)
+        for (int p = 0; p < EW / 2; ++p)
             acc[t][p] = make_float2(0.0f, 0.0f);
 
     stage_x(0, 0);
@@ -435,10 +435,10 @@ __global__ void __launch_bounds__(32 * NW)
                 xq[t] = *reinterpret_cast<const uint4 *>(xs + (lane + 32 * t) * kRtXRow + kk);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float *wrow = ws + (kk + q) * L::EP + 16 * warp;
-                float2 wp[8];
+                const float *wrow = ws + (kk + q) * L::EP + EW * warp;
+                float2 wp[EW / 2];
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
+                for (int h = 0; h < EW / 4; ++h) {
                     const float4 v = *reinterpret_cast<const float4 *>(wrow + 4 * h);
                     wp[2 * h] = make_float2(v.x, v.y);
                     wp[2 * h + 1] = make_float2(v.z, v.w);
@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(32 * NW)
                     const float xv = (q & 1) ? bf16_hi(word) : bf16_lo(word);
                     const float2 xx = make_float2(xv, xv);
 #pragma unroll
-                    for (int p = 0; p < 8; ++p)
+                    for (int p = 0; p < EW / 2; ++p)
                         acc[t][p] = __ffma2_rn(xx, wp[p], acc[t][p]);
                 }
             }
@@ -460,15 +460,15 @@ __global__ void __launch_bounds__(32 * NW)
     cp_async_wait<0>();
     __syncthreads();  // every warp is done with the stages: the logit tile may reuse them
 
-    // logits of the tile -> shared memory [token][expert] (row of EW + 1 floats)
+    // logits of the tile -> shared memory [token][expert] (row of EC + 1 floats)
     float *lt = reinterpret_cast<float *>(rt_smem);
-    const int LR = EW + 1;
+    const int LR = EC + 1;
 #pragma unroll
     for (int t = 0; t < TT; ++t) {
         const int tok = lane + 32 * t;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const int e = 16 * warp + 2 * p;
+        for (int p = 0; p < EW / 2; ++p) {
+            const int e = EW * warp + 2 * p;
             float a = acc[t][p].x, b = acc[t][p].y;
             if (bias) {
                 if (e < E)
@@ -487,8 +487,183 @@ __global__ void __launch_bounds__(32 * NW)
         const int t = t0 + tok;
         if (t >= N)
             break;
-        topk_select_warp<(16 * NW + 31) / 32>(lt + tok * LR, E, K, (size_t)t, logits, topk_idx,
+        topk_select_warp<(EW * NW + 31) / 32>(lt + tok * LR, E, K, (size_t)t, logits, topk_idx,
                                               topk_w, nonfinite_count);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Fused router, register-tiled form (E > 32, many tokens). A CTA takes TM tokens and every
+// expert (E padded to EPAD = 64, 128 or 256). A thread owns 8 tokens (two groups of 4:
+// [4 ty, 4 ty + 4) and [TM/2 + 4 ty, ...)) x 8 experts (j TX + tx, j < 8): 64 logits in
+// registers. x is staged in shared memory as fp32 [i][token] (converted and transposed on its way
+// through registers, one chunk ahead) and W in its own layout [expert][i] (cp.async, zero-filled
+// past d and E). Per element i a thread reads its 8 tokens with two 16-byte loads and, once per
+// four elements, its 8 experts with eight: 4 loads per element against 32 packed FMAs on token
+// pairs ((x_t[i], x_t+1[i]) times (W_e[i], W_e[i]) with `__ffma2_rn`: each half rounds like one
+// fmaf, every logit its single ascending chain from +0). A 128-bit shared-memory load is served
+// per half-warp (two wavefronts at least, even when all lanes read one address); a half-warp
+// here reads 2 token groups and 8 consecutive expert rows (36 floats apart: conflict-free), so
+// each load costs exactly two wavefronts: 8 wavefronts per warp and element against 16 SM cycles
+// of FMA-pipe work.
+template <int EPAD, int TM>
+struct RouterTile8 {
+    static constexpr int KC = 32;
+    static constexpr int TX = EPAD / 8, TY = TM / 8;
+    static constexpr int NT = TX * TY, NW = NT / 32;
+    static constexpr int WX = TX / 8;    // warps across the experts (8 thread columns each)
+    static constexpr int XS = TM + 4;    // fp32 per staged x^T row
+    static constexpr int WS = KC + 4;    // fp32 per staged W row
+    static constexpr int STAGE = KC * XS + EPAD * WS;  // fp32 per ring stage
+    static constexpr int XV = (TM * (KC / 8) + NT - 1) / NT;  // 8-element x pieces per thread
+    static constexpr int LR = EPAD + 1;
+    static constexpr int SMEM_BYTES = (2 * STAGE > TM * LR ? 2 * STAGE : TM * LR) * 4;
+    static_assert(TX % 8 == 0 && TY % 4 == 0, "tile");
+};
+
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid)
+{
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem_src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+template <int EPAD, int TM>
+__global__ void __launch_bounds__(RouterTile8<EPAD, TM>::NT)
+    router_tile8_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
+                        const float *__restrict__ bias, int N, int d, int E, int K,
+                        int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                        float *__restrict__ logits, unsigned long long *nonfinite_count)
+{
+    using G = RouterTile8<EPAD, TM>;
+    constexpr int KC = G::KC;
+    extern __shared__ __align__(16) float rt8_smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ty = (warp / G::WX) * 4 + (lane >> 3);
+    const int tx = (warp % G::WX) * 8 + (lane & 7);
+    const int t0 = blockIdx.x * TM;
+    const int nchunks = (d + KC - 1) / KC;
+
+    uint4 xr[G::XV];
+    auto load_x = [&](int c) {  // x chunk c -> registers (zeros past N and d)
+        const int k0 = c * KC;
+#pragma unroll
+        for (int j = 0; j < G::XV; ++j) {
+            const int idx = tid + j * G::NT;
+            const int t = idx % TM, q = idx / TM;
+            xr[j] = (idx < TM * (KC / 8) && t0 + t < N && k0 + 8 * q < d)
+                        ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + t) * d + k0) + q)
+                        : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    auto store_x = [&](int s) {  // registers -> stage s as fp32 [i][token]
+        float *xs = rt8_smem + s * G::STAGE;
+#pragma unroll
+        for (int j = 0; j < G::XV; ++j) {
+            const int idx = tid + j * G::NT;
+            if (idx < TM * (KC / 8)) {
+                const int t = idx % TM, q = idx / TM;
+                const uint32_t w4[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    xs[(8 * q + 2 * h) * G::XS + t] = bf16_lo(w4[h]);
+                    xs[(8 * q + 2 * h + 1) * G::XS + t] = bf16_hi(w4[h]);
+                }
+            }
+        }
+    };
+    auto issue_w = [&](int c, int s) {  // W chunk c -> stage s, [expert][i] (cp.async)
+        float *ws = rt8_smem + s * G::STAGE + KC * G::XS;
+        const int k0 = c * KC;
+        for (int idx = tid; idx < EPAD * (KC / 4); idx += G::NT) {
+            const int e = idx >> 3, q = idx & 7;
+            const bool ok = e < E && k0 + 4 * q < d;
+            cp_async16_zfill(ws + e * G::WS + 4 * q,
+                             ok ? (const void *)(wr + (size_t)e * d + k0 + 4 * q) : (const void *)wr,
+                             ok);
+        }
+    };
+
+    float2 acc[4][8];  // [token pair][expert j]
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            acc[p][j] = make_float2(0.0f, 0.0f);
+
+    load_x(0);
+    store_x(0);
+    issue_w(0, 0);
+    cp_async_commit();
+    if (nchunks > 1)
+        load_x(1);
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1;
+        if (c + 1 < nchunks) {  // the other stage, free since the last barrier
+            store_x(s ^ 1);
+            issue_w(c + 1, s ^ 1);
+        }
+        cp_async_commit();
+        if (c + 2 < nchunks)
+            load_x(c + 2);
+        const float *xs = rt8_smem + s * G::STAGE;
+        const float *ws = xs + KC * G::XS;
+#pragma unroll
+        for (int k4 = 0; k4 < KC / 4; ++k4) {
+            float4 w[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                w[j] = *reinterpret_cast<const float4 *>(ws + (j * G::TX + tx) * G::WS + 4 * k4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int k = 4 * k4 + kk;
+                const float4 xa = *reinterpret_cast<const float4 *>(xs + k * G::XS + 4 * ty);
+                const float4 xb =
+                    *reinterpret_cast<const float4 *>(xs + k * G::XS + TM / 2 + 4 * ty);
+                const float2 pr[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w),
+                                      make_float2(xb.x, xb.y), make_float2(xb.z, xb.w)};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float wv = kk == 0 ? w[j].x : kk == 1 ? w[j].y : kk == 2 ? w[j].z : w[j].w;
+                    const float2 ww = make_float2(wv, wv);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+                        acc[p][j] = __ffma2_rn(pr[p], ww, acc[p][j]);
+                }
+            }
+        }
+        cp_async_wait<0>();
+        __syncthreads();  // stage s is read; chunk c + 1 is in stage s ^ 1
+    }
+
+    // logits (+ bias) of the tile -> shared memory [token][expert]
+    float *lt = rt8_smem;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int ta = (p < 2 ? 4 * ty : TM / 2 + 4 * ty) + 2 * (p & 1);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = j * G::TX + tx;
+            float a = acc[p][j].x, b = acc[p][j].y;
+            if (bias && e < E) {
+                const float be = bias[e];
+                a = __fadd_rn(a, be);
+                b = __fadd_rn(b, be);
+            }
+            lt[ta * G::LR + e] = a;
+            lt[(ta + 1) * G::LR + e] = b;
+        }
+    }
+    __syncthreads();
+    for (int tok = warp; tok < TM; tok += G::NW) {
+        const int t = t0 + tok;
+        if (t >= N)
+            break;
+        topk_select_warp<EPAD / 32>(lt + tok * G::LR, E, K, (size_t)t, logits, topk_idx, topk_w,
+                                    nonfinite_count);
     }
 }
 

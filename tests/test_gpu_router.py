@@ -1,6 +1,7 @@
-"""Parity of the router with the oracle, through moe_route: the fused kernel (projection + top-K
-in one kernel: many tokens, E >= 32) and the chain kernel (few logits: small N or few experts,
-then the top-K kernel). Checked: the logits bit for bit (each one fp32 fmaf chain over d in ascending
+"""Parity of the router with the oracle, through moe_route: the fused kernels (projection + top-K
+in one kernel: many tokens, E >= 32; the broadcast form and, for E <= 64 with many tokens, the
+register-tiled form) and the separate kernels (few logits: small N or few experts, then the
+top-K kernel). Checked: the logits bit for bit (each one fp32 fmaf chain over d in ascending
 order from +0, then + bias), the top-K indices exactly, the gate weights within fp32 rounding of
 the oracle's fp64 softmax. The shapes cover a ragged last token tile, a hidden size that is not
 a multiple of the 32-element chunk, every padded expert width (E rounded up to 32, 64, 128, 256),
@@ -23,7 +24,11 @@ CASES = [
     (4096, 512, 128, 8, 1.1),
     (2048, 1024, 160, 32, 0.0),  # E padded to 256, K = 32
     (2049, 64, 256, 8, 1.2),
-    # the chain kernel: decode-sized, few experts, an odd expert count, one token
+    # the register-tiled fused form (E <= 64, many tokens): ragged last tile, partial chunk,
+    # padded experts
+    (30000, 136, 64, 6, 1.2),
+    (29001, 256, 40, 4, 0.0),
+    # the separate kernels: decode-sized, few experts, an odd expert count, one token
     (16, 7168, 256, 8, 0.0),
     (4096, 512, 8, 2, 0.0),
     (100, 136, 5, 2, 0.9),
