@@ -964,6 +964,9 @@ def parse(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the workload with this many tokens instead of its own N (a reduced "
+                         "case for profiler captures; not a benchmark configuration)")
     return ap.parse_args(argv)
 
 
@@ -973,6 +976,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     from moe_workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.tokens > 0:
+        w = w.with_(N=args.tokens)
     if args.impl == "reference":
         res = run_reference(args, w)
     else:

@@ -154,12 +154,17 @@ __device__ void block_excl_scan_i64(int64_t *a, int n, int64_t *s_warp)
 constexpr int kHistThreads = 256;
 
 // Shared memory of dispatch_hist_kernel: the block's histogram, then (for the block that
-// finishes last) s_a [max(E, W*W) + 1] int64, s_D [W*W] int64, s_warp [32] int64 and
-// s_kh [E][W] int32 (kept rows of expert e from home shard i).
-__host__ __device__ inline size_t hist_smem_bytes(int E, int W)
+// finishes last) s_a [max(E, W*W) + 1] int64, s_D [W*W] int64, s_warp [32] int64, s_kh [E][W]
+// int32 (kept rows of expert e from home shard i) and, when (G + 1) E <= kCumCacheInts, s_cum
+// [G + 1][E] int32: every segment-start prefix the totals read, loaded once, all at a time.
+constexpr int kCumCacheInts = 16384;
+
+__host__ __device__ inline bool cum_cached(int E, int G) { return (size_t)(G + 1) * E <= kCumCacheInts; }
+
+__host__ __device__ inline size_t hist_smem_bytes(int E, int W, int G)
 {
     const size_t scan = ((size_t)(E > W * W ? E : W * W) + 1) * 8 + (size_t)W * W * 8 + 32 * 8 +
-                        (size_t)E * W * 4;
+                        (size_t)E * W * 4 + (cum_cached(E, G) ? (size_t)(G + 1) * E * 4 : 0);
     const size_t hist = (size_t)E * 4;
     return scan > hist ? scan : hist;
 }
@@ -181,10 +186,19 @@ __device__ void pass_totals(const HistArgs &p, unsigned char *smem)
     int64_t *s_D = s_a + scan_len;
     int64_t *s_warp = s_D + W * W;
     int32_t *s_kh = reinterpret_cast<int32_t *>(s_warp + 32);
+    int32_t *s_cum = s_kh + E * W;
+    const bool cached = cum_cached(E, G);
+    if (cached) {
+#pragma unroll 4
+        for (int i = threadIdx.x; i < (G + 1) * E; i += NT)
+            s_cum[i] = seg_cum(p, i % E, i / E);
+        __syncthreads();
+    }
+    auto cum = [&](int e, int g) { return cached ? s_cum[g * E + e] : seg_cum(p, e, g); };
 
     for (int e = threadIdx.x; e < E; e += NT) {
-        const int kp = (int)min((int64_t)seg_cum(p, e, G), C);
-        p.counts[e] = seg_cum(p, e, p.nseg_round);
+        const int kp = (int)min((int64_t)cum(e, G), C);
+        p.counts[e] = cum(e, p.nseg_round);
         p.kept[e] = kp;
         s_a[e] = kp;
     }
@@ -192,7 +206,7 @@ __device__ void pass_totals(const HistArgs &p, unsigned char *smem)
         const int e = ei / W, i = ei % W;
         int64_t s = 0;
         for (int g = i; g < G; g += W)
-            s += min((int64_t)seg_cum(p, e, g + 1), C) - min((int64_t)seg_cum(p, e, g), C);
+            s += min((int64_t)cum(e, g + 1), C) - min((int64_t)cum(e, g), C);
         s_kh[ei] = (int32_t)s;
     }
     __syncthreads();
@@ -231,9 +245,9 @@ __device__ void pass_totals(const HistArgs &p, unsigned char *smem)
             base += s_kh[e2 * W + i];
         int64_t run = 0;
         for (int g = i; g < G; g += W) {
-            const int c0 = seg_cum(p, e, g);
+            const int c0 = cum(e, g);
             p.pk_base[(size_t)g * E + e] = base + run - c0;
-            run += seg_cum(p, e, g + 1) - c0;
+            run += cum(e, g + 1) - c0;
         }
     }
 
@@ -242,11 +256,11 @@ __device__ void pass_totals(const HistArgs &p, unsigned char *smem)
         int mx = 0, mn = 0x7fffffff, act = 0;
         int64_t first = 0;  // rows from round 0
         for (int e = lane; e < E; e += 32) {
-            const int kp = (int)min((int64_t)seg_cum(p, e, G), C);
+            const int kp = (int)min((int64_t)cum(e, G), C);
             mx = max(mx, kp);
             mn = min(mn, kp);
             act += kp > 0;
-            first += min((int64_t)seg_cum(p, e, p.nseg_round), C);
+            first += min((int64_t)cum(e, p.nseg_round), C);
         }
         first = warp_sum(first);
 #pragma unroll
@@ -471,6 +485,687 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// Bulk copy of a token block's bf16 rows (the share of part `part` of `parts`): the block's
+// items are (token, piece) pairs, q = lt * npc + piece; warp w takes q = part + parts * (w + 8 j)
+// of the tokens that keep a slot. Per warp a pipeline over its items: the piece of item c + 1
+// is loaded into its ring slot while item c's stores go out (lane k < K stores slot k's
+// expert-sorted row and, when it has one, its packed row), with up to S - 1 items' stores in
+// flight; a slot is reloaded only once the stores that read it have read it. xb: the block's
+// first token row; s_rk / s_pk: each slot's sorted / packed row or -1 (shared memory); ring_smem:
+// 8 warps x S slots of kPiece bytes, then 8 x S mbarriers. Every wait is bounded.
+__device__ void copy_rows_bulk(const uint16_t *xb, int nt, int K, const int *s_rk, const int *s_pk,
+                               void *x_sorted, void *x_packed, int d, int part, int parts,
+                               unsigned char *ring_smem, int S, uint64_t timeout_ns)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t rb = (uint32_t)d * 2u;
+    const int npc = (int)((rb + kPiece - 1) / kPiece);
+    const int nq = nt * npc, qstep = parts * 8;
+    const uint32_t ring = smem_u32(ring_smem) + warp * S * kPiece;
+    const uint32_t bars = smem_u32(ring_smem) + 8 * S * kPiece + warp * S * 8;
+    if (lane == 0) {
+        for (int j = 0; j < S; ++j)
+            mbar_init(bars + 8 * j, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    // the next item at or after q whose token keeps a slot (nq: none)
+    auto next_item = [&](int q) {
+        for (; q < nq; q += qstep) {
+            const int lt = q / npc;
+            if (__any_sync(0xffffffffu, lane < K && s_rk[lt * K + lane] >= 0))
+                break;
+        }
+        return q < nq ? q : nq;
+    };
+    auto issue_load = [&](int q, int slot) {
+        if (lane == 0) {
+            const int lt = q / npc, pc = q - lt * npc;
+            const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
+            const unsigned char *src = reinterpret_cast<const unsigned char *>(xb) +
+                                       (size_t)lt * rb + (size_t)pc * kPiece;
+            mbar_arrive_expect_tx(bars + 8 * slot, bytes);
+            bulk_load_g2s(ring + slot * kPiece, src, bytes, bars + 8 * slot);
+        }
+    };
+    auto wait_read = [&](int pending) {  // this lane's store groups beyond `pending` read
+        if (pending <= 0)
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        else
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    };
+    unsigned char *dst_s = reinterpret_cast<unsigned char *>(x_sorted);
+    unsigned char *dst_p = reinterpret_cast<unsigned char *>(x_packed);
+    int q_cur = next_item(part + parts * warp);
+    int c = 0;          // items whose stores have been issued
+    int loaded = -1;    // the last item index whose load was issued
+    if (q_cur < nq) {
+        issue_load(q_cur, 0);
+        loaded = 0;
+    }
+    while (q_cur < nq) {
+        const int q_nxt = next_item(q_cur + qstep);
+        if (S > 1 && q_nxt < nq) {  // load item c + 1 (its slot's earlier stores read)
+            wait_read(S - 2);
+            __syncwarp();
+            issue_load(q_nxt, (c + 1) % S);
+            loaded = c + 1;
+        }
+        const int slot = c % S;
+        if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((c / S) & 1), timeout_ns))
+            break;
+        const int lt = q_cur / npc, pc = q_cur - lt * npc;
+        const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
+        const size_t off = (size_t)pc * kPiece;
+        if (lane < K) {  // x_sorted is null for a rank's dispatch (send rows only)
+            const int rk = s_rk[lt * K + lane];
+            if (rk >= 0) {
+                if (dst_s)
+                    bulk_store_s2g(dst_s + (size_t)rk * rb + off, ring + slot * kPiece, bytes);
+                const int pk = s_pk[lt * K + lane];
+                if (pk >= 0)
+                    bulk_store_s2g(dst_p + (size_t)pk * rb + off, ring + slot * kPiece, bytes);
+            }
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        ++c;
+        if (S == 1 && q_nxt < nq) {  // one slot: reload it once this item's stores read it
+            wait_read(0);
+            __syncwarp();
+            issue_load(q_nxt, 0);
+            loaded = c;
+        }
+        q_cur = q_nxt;
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    // loads issued and not consumed (only after a wait that ran out): let them land first
+    if (lane == 0)
+        for (int j = c; j <= loaded; ++j)
+            mbar_wait_bounded(bars + 8 * (j % S), (uint32_t)((j / S) & 1), timeout_ns);
+    __syncwarp();
+}
+
+// Bulk copy by destination row, for a balanced split whatever the routing: warp gw of nw takes
+// a contiguous range of the (row, piece) items of the R expert-sorted rows; row r copies token
+// assign_of_row[r] / K's piece to x_sorted row r and, when there is a packed buffer, to packed
+// row pk_of[assign_of_row[r]]. A token row is read once per kept slot (from L2 after the first).
+// The items' rows are looked up 32 at a time (lane l the l-th item of a batch, the next batch
+// loaded while this one is copied); the copy pipeline is copy_rows_bulk's. ring / bars: this
+// warp's S slots of kPiece bytes and its S mbarriers (shared-memory addresses).
+__device__ void copy_rows_by_row(const uint16_t *x, const int32_t *assign_of_row,
+                                 const int32_t *pk_of, int R, int K, void *x_sorted, void *x_packed,
+                                 int d, int gw, int nw, uint32_t ring, uint32_t bars, int S,
+                                 uint64_t timeout_ns)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t rb = (uint32_t)d * 2u;
+    const int npc = (int)((rb + kPiece - 1) / kPiece);
+    const long long nq = (long long)R * npc;
+    const long long per = (nq + nw - 1) / nw;
+    const long long q0 = min(nq, (long long)gw * per), q1 = min(nq, q0 + per);
+    const int n = (int)(q1 - q0);
+    if (lane == 0) {
+        for (int j = 0; j < S; ++j)
+            mbar_init(bars + 8 * j, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if (n <= 0)
+        return;
+    // item j of the range: lane j % 32 of batch j / 32 holds its token row and packed row
+    auto fetch = [&](int batch, int &tok, int &pk) {
+        const int j = batch * 32 + lane;
+        tok = -1;
+        pk = -1;
+        if (j < n) {
+            const int r = (int)((q0 + j) / npc);
+            const int a = __ldcg(assign_of_row + r);
+            tok = a / K;
+            if (x_packed)
+                pk = __ldcg(pk_of + a);
+        }
+    };
+    int cur_t, cur_p, nxt_t, nxt_p;
+    fetch(0, cur_t, cur_p);
+    fetch(1, nxt_t, nxt_p);
+    auto info = [&](int j, int &tok, int &pk) {  // j in the current or the next batch
+        const bool in_next = (j >> 5) != 0;
+        const int t_src = in_next ? nxt_t : cur_t, p_src = in_next ? nxt_p : cur_p;
+        tok = __shfl_sync(0xffffffffu, t_src, j & 31);
+        pk = __shfl_sync(0xffffffffu, p_src, j & 31);
+    };
+    auto piece = [&](int j, uint32_t &off, uint32_t &bytes) {
+        const int pc = (int)((q0 + j) % npc);
+        off = (uint32_t)pc * kPiece;
+        bytes = min((uint32_t)kPiece, rb - off);
+    };
+    auto issue_load = [&](int j, int jb) {  // item j (index jb inside the held batches)
+        int tok, pk;
+        info(jb, tok, pk);
+        uint32_t off, bytes;
+        piece(j, off, bytes);
+        const int slot = j % S;
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bars + 8 * slot, bytes);
+            bulk_load_g2s(ring + slot * kPiece,
+                          reinterpret_cast<const unsigned char *>(x) + (size_t)tok * rb + off,
+                          bytes, bars + 8 * slot);
+        }
+    };
+    auto wait_read = [&](int pending) {
+        if (pending <= 0)
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        else
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    };
+    unsigned char *dst_s = reinterpret_cast<unsigned char *>(x_sorted);
+    unsigned char *dst_p = reinterpret_cast<unsigned char *>(x_packed);
+    int loaded = 0, c = 0;
+    issue_load(0, 0);
+    for (; c < n; ++c) {
+        if ((c & 31) == 0 && c > 0) {  // the next batch becomes the current one
+            cur_t = nxt_t;
+            cur_p = nxt_p;
+            fetch((c >> 5) + 1, nxt_t, nxt_p);
+        }
+        const int cb = c & 31;
+        if (S > 1 && c + 1 < n) {
+            wait_read(S - 2);
+            __syncwarp();
+            issue_load(c + 1, cb + 1);
+            loaded = c + 1;
+        }
+        const int slot = c % S;
+        if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((c / S) & 1), timeout_ns))
+            break;
+        int tok, pk;
+        info(cb, tok, pk);
+        uint32_t off, bytes;
+        piece(c, off, bytes);
+        const long long r = (q0 + c) / npc;
+        if (lane == 0)
+            bulk_store_s2g(dst_s + (size_t)r * rb + off, ring + slot * kPiece, bytes);
+        else if (lane == 1 && pk >= 0)
+            bulk_store_s2g(dst_p + (size_t)pk * rb + off, ring + slot * kPiece, bytes);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        if (S == 1 && c + 1 < n) {
+            wait_read(0);
+            __syncwarp();
+            issue_load(c + 1, cb + 1);
+            loaded = c + 1;
+        }
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (lane == 0)
+        for (int j = c; j <= loaded; ++j)
+            mbar_wait_bounded(bars + 8 * (j % S), (uint32_t)((j / S) & 1), timeout_ns);
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// The dispatch pass in one kernel (one round, bf16 rows or no copy), for grids that fit on the
+// GPU at once (cooperative launch). CTA (token block tb, part):
+//  1. the block's top-K slice into shared memory; per virtual block of the token block (one,
+//     or K slot-major), per-warp expert counts and each assignment's rank among the block's
+//     assignments to its expert (first come first placed: per-warp bases, then
+//     __match_any_sync inside the warp), and part 0 publishes the block's histogram;
+//  2. one grid barrier (an arrival count, bounded wait);
+//  3. every CTA loads all the histograms (shared memory), scans each expert's column (in
+//     parallel over segments of blocks, then a second pass), and so knows its own blocks'
+//     prefixes, the prefix at every segment start and the totals; from these, like the
+//     totals of the two-kernel pass: kept = min(total, C), offsets, the kept rows of every
+//     (expert, home shard), D, the pack offsets and its own blocks' pack bases. CTA (0, 0)
+//     writes them out;
+//  4. positions = block prefix + rank: the mapping table (part 0) and the dedup counter;
+//  5. the bulk copy of its share of the block's rows (copy_rows_bulk).
+// No position needs a second walk over the top-K, and the histograms are read once per CTA
+// from L2. The arithmetic is the two-kernel pass's, so the results are the same bits.
+struct FusedArgs {
+    const int32_t *topk_idx;
+    VBlocks vbm;  // one round
+    int nvb, bps, nseg;
+    int N, E, K, W, C;
+    unsigned int *ctl;  // [0]: arrivals at the grid barrier (zeroed before the launch)
+    int32_t *agg;       // [nvb][E]
+    int32_t *counts, *kept, *offsets;
+    int64_t *D, *pk_off;
+    int32_t *row_of, *assign_of_row, *expert_of, *packed_row_of;
+    int32_t *pk_of;  // nullable scratch [N*K]: each slot's packed row (for the copy by row)
+    int rank, x_row0;
+    int32_t *send_row_of;
+    int copy;
+    const uint16_t *x;
+    int d;
+    void *x_sorted, *x_packed;
+    moe_stats_t *stats;
+    int slots;
+    uint64_t timeout_ns;
+};
+
+// Shared-memory layout of dispatch_fused_kernel (bytes from the start).
+struct FusedLayout {
+    size_t wcnt, off, e, lr, rk, pk, ex, base, cum, kh, part, a64, warp64, D, pko, pkb, uni, total;
+};
+
+__host__ __device__ inline FusedLayout fused_layout(int E, int K, int W, int nvb, int nseg, int nsub,
+                                                    int slots)
+{
+    FusedLayout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes, size_t align) {
+        o = (o + align - 1) / align * align;
+        const size_t at = o;
+        o += bytes;
+        return at;
+    };
+    const size_t slots_b = (size_t)kDispatchHB * K * 4;
+    L.wcnt = take((size_t)8 * E * 4, 16);
+    L.off = take((size_t)(E + 1) * 4, 16);
+    L.e = take(slots_b, 16);
+    L.lr = take(slots_b, 16);
+    L.rk = take(slots_b, 16);
+    L.pk = take(slots_b, 16);
+    L.ex = take(slots_b, 16);
+    L.base = take((size_t)nsub * E * 4, 16);
+    L.cum = take((size_t)(nseg + 1) * E * 4, 16);
+    L.kh = take((size_t)E * W * 4, 16);
+    L.part = take(256 * 4, 16);
+    L.a64 = take((size_t)((E > W * W ? E : W * W) + 1) * 8, 16);
+    L.warp64 = take(32 * 8, 16);
+    L.D = take((size_t)W * W * 8, 16);
+    L.pko = take((size_t)(W * W + 1) * 8, 16);
+    L.pkb = take((size_t)nsub * E * 8, 16);
+    // the histograms of every block (phase 3), then the copy ring (phase 5), in one region
+    const size_t ring = (size_t)8 * slots * kPiece + (size_t)8 * slots * 8;
+    const size_t aggs = (size_t)nvb * E * 4;
+    L.uni = take(ring > aggs ? ring : aggs, 128);
+    L.total = o;
+    return L;
+}
+
+__global__ void __launch_bounds__(kPlaceThreads) dispatch_fused_kernel(FusedArgs p)
+{
+    extern __shared__ __align__(128) unsigned char fz[];
+    constexpr int NT = kPlaceThreads;
+    const int E = p.E, K = p.K, W = p.W;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tb = blockIdx.x, part = blockIdx.y, parts = gridDim.y;
+    const bool lead = tb == 0 && part == 0;
+    const int nsub = p.vbm.slot_major ? K : 1;
+    const FusedLayout L = fused_layout(E, K, W, p.nvb, p.nseg, nsub, p.slots);
+    int *wcnt = reinterpret_cast<int *>(fz + L.wcnt);
+    int *s_off = reinterpret_cast<int *>(fz + L.off);
+    int *s_e = reinterpret_cast<int *>(fz + L.e);
+    int *s_lr = reinterpret_cast<int *>(fz + L.lr);
+    int *s_rk = reinterpret_cast<int *>(fz + L.rk);
+    int *s_pk = reinterpret_cast<int *>(fz + L.pk);
+    int *s_ex = reinterpret_cast<int *>(fz + L.ex);
+    int *s_base = reinterpret_cast<int *>(fz + L.base);
+    int *s_cum = reinterpret_cast<int *>(fz + L.cum);
+    int *s_kh = reinterpret_cast<int *>(fz + L.kh);
+    int *s_part = reinterpret_cast<int *>(fz + L.part);
+    int64_t *s_a = reinterpret_cast<int64_t *>(fz + L.a64);
+    int64_t *s_warp = reinterpret_cast<int64_t *>(fz + L.warp64);
+    int64_t *s_D = reinterpret_cast<int64_t *>(fz + L.D);
+    int64_t *s_pko = reinterpret_cast<int64_t *>(fz + L.pko);
+    int64_t *s_pkb = reinterpret_cast<int64_t *>(fz + L.pkb);
+    int *s_agg = reinterpret_cast<int *>(fz + L.uni);
+    __shared__ int s_ok, s_dropped;
+
+    int t0, t1;
+    p.vbm.bm.range(tb, t0, t1);
+    const int nt = t1 - t0;
+    unsigned lt_mask;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
+
+    // 1. the block's experts, ranks inside each virtual block, histograms
+    for (int i = tid; i < nt * K; i += NT) {
+        const int e = p.topk_idx[(size_t)t0 * K + i];
+        const bool ok = (unsigned)e < (unsigned)E;
+        if (!ok && part == 0)
+            set_dev_error(MOE_ERR_DEVICE_BOUNDS);
+        s_e[i] = ok ? e : -1;
+        s_rk[i] = -1;
+        s_pk[i] = -1;
+        s_ex[i] = -1;
+    }
+    if (lead && tid == 0 && p.stats)
+        p.stats->dedup_pairs = 0;  // before the barrier: every CTA adds to it after
+    for (int kk = 0; kk < nsub; ++kk) {
+        const int vb = (p.vbm.slot_major ? kk * p.vbm.nblk_tok : 0) + tb;
+        const int na = p.vbm.count(t0, t1);
+        const int per = (na + 7) / 8;
+        const int wb = min(na, warp * per), we = min(na, wb + per);
+        for (int i = tid; i < 8 * E; i += NT)
+            wcnt[i] = 0;
+        __syncthreads();
+        for (int i = wb + lane; i < we; i += 32) {
+            const int e = s_e[p.vbm.assign(t0, kk, i) - t0 * K];
+            if (e >= 0)
+                atomicAdd(&wcnt[warp * E + e], 1);
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += NT) {
+            int run = 0;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const int c = wcnt[w * E + e];
+                wcnt[w * E + e] = run;
+                run += c;
+            }
+            if (part == 0)
+                p.agg[(size_t)vb * E + e] = run;
+        }
+        __syncthreads();
+        for (int g0 = wb; g0 < we; g0 += 32) {
+            const int i = g0 + lane;
+            const bool act = i < we;
+            const int ls = act ? p.vbm.assign(t0, kk, i) - t0 * K : 0;
+            const int e = act ? s_e[ls] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, e);
+            const int rk = __popc(peers & lt_mask);
+            const int base = e >= 0 ? wcnt[warp * E + e] : 0;
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(peers) - 1)
+                wcnt[warp * E + e] = base + __popc(peers);
+            __syncwarp();
+            if (act)
+                s_lr[ls] = base + rk;
+        }
+        __syncthreads();
+    }
+
+    // 2. grid barrier
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned int n_cta = gridDim.x * gridDim.y;
+        atomicAdd(&p.ctl[0], 1u);
+        int ok = 1;
+        if (ld_acquire_u32(&p.ctl[0]) < n_cta) {
+            const uint64_t w0 = global_timer_ns();
+            while (ld_acquire_u32(&p.ctl[0]) < n_cta) {
+                if (global_timer_ns() - w0 > p.timeout_ns) {
+                    set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok)
+        return;  // the histograms are incomplete: write nothing (the error is recorded)
+    __threadfence();
+
+    // 3. every block's histogram; column scans; totals
+    const int nvE = p.nvb * E;
+    {
+        const int n4 = nvE >> 2;  // 16-byte pieces, every load in flight before the first store
+        const int4 *src4 = reinterpret_cast<const int4 *>(p.agg);
+        int4 *dst4 = reinterpret_cast<int4 *>(s_agg);
+#pragma unroll 16
+        for (int i = tid; i < n4; i += NT)
+            dst4[i] = __ldcg(src4 + i);
+        for (int i = 4 * n4 + tid; i < nvE; i += NT)
+            s_agg[i] = __ldcg(p.agg + i);
+    }
+    __syncthreads();
+    const int S = NT / E > 0 ? NT / E : 1;  // segments of blocks per expert column
+    const int Lb = (p.nvb + S - 1) / S;
+    const int col_e = tid % E, col_s = tid / E;
+    const bool col = tid < S * E;
+    const int lo = col ? min(p.nvb, col_s * Lb) : 0, hi = col ? min(p.nvb, lo + Lb) : 0;
+    if (col) {  // pass 1: the segment's sum (8 loads in flight, then their adds)
+        int sum = 0;
+        for (int v0 = lo; v0 < hi; v0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = v0 + u < hi ? s_agg[(v0 + u) * E + col_e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                sum += v[u];
+        }
+        s_part[col_s * E + col_e] = sum;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += NT) {
+        int run = 0;
+        for (int q = 0; q < S; ++q) {
+            const int v = s_part[q * E + e];
+            s_part[q * E + e] = run;
+            run += v;
+        }
+        s_cum[p.nseg * E + e] = run;
+    }
+    __syncthreads();
+    if (col) {  // pass 2: prefixes at segment starts and at this CTA's own blocks
+        int run = s_part[col_s * E + col_e];
+        const int nb = p.vbm.nblk_tok;
+        int to_seg = lo % p.bps;  // blocks since the last segment start
+        int seg = lo / p.bps;
+        // this CTA's next own block at or after lo: tb (+ k nb slot-major)
+        int mine = p.vbm.slot_major ? (lo <= tb ? tb : tb + ((lo - tb + nb - 1) / nb) * nb)
+                                    : (lo <= tb ? tb : 0x7fffffff);
+        for (int v0 = lo; v0 < hi; v0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = v0 + u < hi ? s_agg[(v0 + u) * E + col_e] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int vb = v0 + u;
+                if (vb < hi) {
+                    if (to_seg == 0)
+                        s_cum[seg * E + col_e] = run;
+                    if (vb == mine) {
+                        s_base[(p.vbm.slot_major ? vb / nb : 0) * E + col_e] = run;
+                        mine = p.vbm.slot_major ? mine + nb : 0x7fffffff;
+                    }
+                    run += v[u];
+                    if (++to_seg == p.bps) {
+                        to_seg = 0;
+                        ++seg;
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const int64_t C = p.C;
+    const int G = p.nseg;
+    for (int e = tid; e < E; e += NT)
+        s_a[e] = min((int64_t)s_cum[G * E + e], C);
+    if (warp == 0) {  // drops? (without them every token block keeps all its slots)
+        int over = 0;
+        for (int e = lane; e < E; e += 32)
+            over |= s_cum[G * E + e] > p.C;
+        over = __any_sync(0xffffffffu, over);
+        if (lane == 0)
+            s_dropped = over;
+    }
+    for (int ei = tid; ei < E * W; ei += NT) {
+        const int e = ei / W, i = ei % W;
+        int64_t sk = 0;
+        for (int g = i; g < G; g += W)
+            sk += min((int64_t)s_cum[(g + 1) * E + e], C) - min((int64_t)s_cum[g * E + e], C);
+        s_kh[ei] = (int32_t)sk;
+    }
+    __syncthreads();
+    block_excl_scan_i64<NT>(s_a, E, s_warp);
+    for (int e = tid; e <= E; e += NT)
+        s_off[e] = (int)s_a[e];
+    __syncthreads();
+    const int e_per = E / W;
+    for (int ij = tid; ij < W * W; ij += NT) {
+        const int i = ij / W, j = ij % W;
+        int64_t sd = 0;
+        for (int e = j * e_per; e < (j + 1) * e_per; ++e)
+            sd += s_kh[e * W + i];
+        s_D[ij] = sd;
+    }
+    __syncthreads();
+    for (int ij = tid; ij < W * W; ij += NT)
+        s_pko[ij] = s_D[ij];
+    __syncthreads();
+    block_excl_scan_i64<NT>(s_pko, W * W, s_warp);
+    __syncthreads();
+    // pack bases of this CTA's virtual blocks: a kept assignment to expert e at position pos
+    // from segment g lands on packed row pkb + pos (block (i, j) holds its experts in order,
+    // each expert's rows from shard i in the shard's own order)
+    for (int ke = tid; ke < nsub * E; ke += NT) {
+        const int kk = ke / E, e = ke % E;
+        const int vb = (p.vbm.slot_major ? kk * p.vbm.nblk_tok : 0) + tb;
+        const int g = vb / p.bps, i = g % W, j = e / e_per;
+        int64_t base = s_pko[i * W + j];
+        for (int e2 = j * e_per; e2 < e; ++e2)
+            base += s_kh[e2 * W + i];
+        for (int g2 = i; g2 < g; g2 += W)
+            base += s_cum[(g2 + 1) * E + e] - s_cum[g2 * E + e];
+        s_pkb[ke] = base - s_cum[g * E + e];
+    }
+    if (lead) {
+        for (int e = tid; e < E; e += NT) {
+            p.counts[e] = s_cum[G * E + e];
+            p.kept[e] = s_off[e + 1] - s_off[e];
+        }
+        for (int e = tid; e <= E; e += NT)
+            p.offsets[e] = s_off[e];
+        for (int ij = tid; ij < W * W; ij += NT)
+            p.D[ij] = s_D[ij];
+        for (int ij = tid; ij <= W * W; ij += NT)
+            p.pk_off[ij] = s_pko[ij];
+        if (p.stats && warp == 0) {
+            int mx = 0, mn = 0x7fffffff, act = 0;
+            for (int e = lane; e < E; e += 32) {
+                const int kp = s_off[e + 1] - s_off[e];
+                mx = max(mx, kp);
+                mn = min(mn, kp);
+                act += kp > 0;
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+                act += __shfl_xor_sync(0xffffffffu, act, off);
+            }
+            int64_t diag = 0;
+            for (int i = lane; i < W; i += 32)
+                diag += s_D[i * W + i];
+            diag = warp_sum(diag);
+            if (lane == 0) {
+                const int64_t R = s_pko[W * W];
+                p.stats->rows = R;
+                p.stats->dropped = (int64_t)p.N * p.K - R;
+                p.stats->cross_rows = R - diag;
+                p.stats->capacity = p.C;
+                p.stats->active_experts = act;
+                p.stats->max_kept = mx;
+                p.stats->min_kept = mn;
+                p.stats->rerouted = 0;
+            }
+        }
+    }
+    __syncthreads();
+
+    // 4. positions -> rows, the mapping table
+    for (int kk = 0; kk < nsub; ++kk) {
+        const int na = p.vbm.count(t0, t1);
+        for (int i = tid; i < na; i += NT) {
+            const int a = p.vbm.assign(t0, kk, i);
+            const int ls = a - t0 * K;
+            const int e = s_e[ls];
+            if (e < 0)
+                continue;
+            const int pos = s_base[kk * E + e] + s_lr[ls];
+            const int row = (pos < p.C && s_off[e] + pos < s_off[e + 1]) ? s_off[e] + pos : -1;
+            s_rk[ls] = row;
+            s_ex[ls] = row >= 0 ? e : -1;
+            const int64_t pk = s_pkb[kk * E + e] + pos;
+            s_pk[ls] = (row >= 0 && pk >= 0 && pk < s_off[E]) ? (int)pk : -1;
+            if (row >= 0 && part == 0)
+                p.assign_of_row[row] = a;
+        }
+    }
+    __syncthreads();
+    const bool home_block = p.rank < 0 || tb / p.vbm.bm.bps == p.rank;
+    const int64_t pack_row0 = p.rank < 0 ? 0 : s_pko[(size_t)p.rank * W];
+    if (part == 0) {
+        for (int i = tid; i < nt * K; i += NT) {
+            p.row_of[(size_t)t0 * K + i] = s_rk[i];
+            if (p.expert_of)
+                p.expert_of[(size_t)t0 * K + i] = s_ex[i];
+            if (p.packed_row_of)
+                p.packed_row_of[(size_t)t0 * K + i] = s_pk[i];
+            if (p.pk_of)
+                p.pk_of[(size_t)t0 * K + i] = s_pk[i];
+            if (p.send_row_of && home_block)
+                p.send_row_of[(size_t)(t0 - p.x_row0) * K + i] =
+                    s_pk[i] >= 0 ? (int)(s_pk[i] - pack_row0) : -1;
+        }
+        if (p.stats) {
+            // distinct destination ranks other than the token's home over its kept slots
+            const int home = tb / p.vbm.bm.bps;
+            unsigned long long pairs = 0;
+            for (int l2 = warp; l2 < nt; l2 += 8) {
+                const int ex = lane < K ? s_ex[l2 * K + lane] : -1;
+                const int dest = ex >= 0 ? ex / e_per : -1;
+                const int key = (dest >= 0 && dest != home) ? dest : -1 - lane;
+                const unsigned grp = __match_any_sync(0xffffffffu, key);
+                pairs += __popc(__ballot_sync(0xffffffffu, key >= 0 && (grp & lt_mask) == 0));
+            }
+            if (lane == 0 && pairs)
+                atomicAdd(reinterpret_cast<unsigned long long *>(&p.stats->dedup_pairs), pairs);
+        }
+    }
+    if (!p.copy)
+        return;
+
+    // 5. the rows. The whole batch on one GPU with drops: by destination row, after a second
+    // grid barrier (every CTA's mapping written), an even split whatever the routing (token
+    // blocks keep very different numbers of rows under skew: early tokens claim the capacity).
+    // Without drops (every block keeps all its slots) and for a rank's own send rows: by token
+    // block.
+    if (p.rank < 0 && (p.pk_of || !p.x_packed) && s_dropped) {
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            const unsigned int target = 2u * gridDim.x * gridDim.y;
+            atomicAdd(&p.ctl[0], 1u);
+            int ok = 1;
+            const uint64_t w0 = global_timer_ns();
+            while (ld_acquire_u32(&p.ctl[0]) < target) {
+                if (global_timer_ns() - w0 > p.timeout_ns) {
+                    set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+            }
+            s_ok = ok;
+        }
+        __syncthreads();
+        if (!s_ok)
+            return;
+        __threadfence();
+        const uint32_t ring = smem_u32(fz + L.uni);
+        copy_rows_by_row(p.x, p.assign_of_row, p.pk_of, s_off[E], K, p.x_sorted, p.x_packed, p.d,
+                         (blockIdx.y * gridDim.x + blockIdx.x) * 8 + warp,
+                         gridDim.x * gridDim.y * 8, ring + warp * p.slots * kPiece,
+                         ring + 8 * p.slots * kPiece + warp * p.slots * 8, p.slots, p.timeout_ns);
+        return;
+    }
+    if (!home_block)
+        return;
+    const uint16_t *xb = p.x + (size_t)(t0 - p.x_row0) * p.d;
+    for (int i = tid; i < nt * K; i += NT)
+        s_pk[i] = (!p.x_packed || s_pk[i] < 0) ? -1 : (int)(s_pk[i] - pack_row0);
+    __syncthreads();  // s_agg (in the ring's region) is no longer read
+    copy_rows_bulk(xb, nt, K, s_rk, s_pk, p.x_sorted, p.x_packed, p.d, part, parts, fz + L.uni,
+                   p.slots, p.timeout_ns);
+}
+
 // One CTA per (token block, part). Positions: for every virtual block of the token block (all
 // rounds; each slot k in slot-major order), warps count their sub-ranges per expert, take
 // their bases from the block's exclusive prefix (inclusive minus own), and rank equal experts
@@ -613,99 +1308,9 @@ __global__ void __launch_bounds__(kPlaceThreads) dispatch_place_kernel(PlaceArgs
     __syncthreads();
 
     if (!p.e4m3) {
-        // Bulk copies. The block's items are (token, piece) pairs, q = lt * npc + piece; part
-        // p's warp w takes q = p + parts * (w + 8 j) of the tokens that keep a slot. Per warp a
-        // pipeline over its items: the piece of item c + 1 is loaded into its ring slot while
-        // item c's stores go out (lane k < K stores slot k's expert-sorted and packed rows),
-        // with up to slots - 1 items' stores in flight; a slot is reloaded only once the stores
-        // that read it have read it.
-        const uint32_t rb = (uint32_t)p.d * 2u;
-        const int npc = (int)((rb + kPiece - 1) / kPiece);
-        const int nq = nt * npc, qstep = parts * 8, S = p.slots;
-        unsigned char *smem_b = reinterpret_cast<unsigned char *>(place_smem);
-        const uint32_t ring = smem_u32(smem_b + place_ring_offset(E, K)) + warp * S * kPiece;
-        const uint32_t bars = smem_u32(smem_b + place_ring_offset(E, K)) + 8 * S * kPiece +
-                              warp * S * 8;
-        if (lane == 0) {
-            for (int j = 0; j < S; ++j)
-                mbar_init(bars + 8 * j, 1);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        }
-        __syncwarp();
-        // the next item at or after q whose token keeps a slot (nq: none)
-        auto next_item = [&](int q) {
-            for (; q < nq; q += qstep) {
-                const int lt = q / npc;
-                if (__any_sync(0xffffffffu, lane < K && s_rk[lt * K + lane] >= 0))
-                    break;
-            }
-            return q < nq ? q : nq;
-        };
-        auto issue_load = [&](int q, int slot) {
-            if (lane == 0) {
-                const int lt = q / npc, pc = q - lt * npc;
-                const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
-                const unsigned char *src = reinterpret_cast<const unsigned char *>(xb) +
-                                           (size_t)lt * rb + (size_t)pc * kPiece;
-                mbar_arrive_expect_tx(bars + 8 * slot, bytes);
-                bulk_load_g2s(ring + slot * kPiece, src, bytes, bars + 8 * slot);
-            }
-        };
-        auto wait_read = [&](int pending) {  // this lane's store groups beyond `pending` read
-            if (pending <= 0)
-                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            else
-                asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-        };
-        unsigned char *dst_s = reinterpret_cast<unsigned char *>(p.x_sorted);
-        unsigned char *dst_p = reinterpret_cast<unsigned char *>(p.x_packed);
-        int q_cur = next_item(part + parts * warp);
-        int c = 0;          // items whose stores have been issued
-        int loaded = -1;    // the last item index whose load was issued
-        if (q_cur < nq) {
-            issue_load(q_cur, 0);
-            loaded = 0;
-        }
-        while (q_cur < nq) {
-            const int q_nxt = next_item(q_cur + qstep);
-            if (S > 1 && q_nxt < nq) {  // load item c + 1 (its slot's earlier stores read)
-                wait_read(S - 2);
-                __syncwarp();
-                issue_load(q_nxt, (c + 1) % S);
-                loaded = c + 1;
-            }
-            const int slot = c % S;
-            if (!mbar_wait_bounded(bars + 8 * slot, (uint32_t)((c / S) & 1), p.timeout_ns))
-                break;
-            const int lt = q_cur / npc, pc = q_cur - lt * npc;
-            const uint32_t bytes = min((uint32_t)kPiece, rb - (uint32_t)pc * kPiece);
-            const size_t off = (size_t)pc * kPiece;
-            if (lane < K) {  // x_sorted is null for a rank's dispatch (send rows only)
-                const int rk = s_rk[lt * K + lane];
-                if (rk >= 0) {
-                    if (dst_s)
-                        bulk_store_s2g(dst_s + (size_t)rk * rb + off, ring + slot * kPiece, bytes);
-                    const int pk = s_pk[lt * K + lane];
-                    if (pk >= 0)
-                        bulk_store_s2g(dst_p + (size_t)pk * rb + off, ring + slot * kPiece, bytes);
-                }
-            }
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            ++c;
-            if (S == 1 && q_nxt < nq) {  // one slot: reload it once this item's stores read it
-                wait_read(0);
-                __syncwarp();
-                issue_load(q_nxt, 0);
-                loaded = c;
-            }
-            q_cur = q_nxt;
-        }
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-        // loads issued and not consumed (only after a wait that ran out): let them land first
-        if (lane == 0)
-            for (int j = c; j <= loaded; ++j)
-                mbar_wait_bounded(bars + 8 * (j % S), (uint32_t)((j / S) & 1), p.timeout_ns);
-        __syncwarp();
+        copy_rows_bulk(xb, nt, K, s_rk, s_pk, p.x_sorted, p.x_packed, p.d, part, parts,
+                       reinterpret_cast<unsigned char *>(place_smem) + place_ring_offset(E, K),
+                       p.slots, p.timeout_ns);
         return;
     }
 

@@ -97,15 +97,19 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
 
 // Route/dispatch scratch, carved in this order from the workspace.
 struct ScratchLayout {
-    size_t logits, ctl, agg, incl, pk_base, moved, D, pk_off, total;
+    size_t logits, ctl, agg, incl, pk_base, moved, D, pk_off, pk_of, total;
 };
+
+constexpr size_t kNoScratch = ~(size_t)0;
 
 // The dispatch's own scratch, from offset o: the pass's control words (ticket, finished
 // blocks, one flag per virtual block), the blocks' histograms and inclusive prefixes
 // [nvb][E], the pack bases [nseg][E], the moved-to expert of each assignment (re-routing),
-// the traffic matrix and the pack offsets (when the caller does not want them).
+// the traffic matrix and the pack offsets (when the caller does not want them), and (with_pk)
+// each assignment's packed row for the one-kernel pass's copy by destination row.
 template <typename Layout>
-size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layout &L)
+size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layout &L,
+                        bool with_pk = true)
 {
     L.ctl = o;
     o = align_up(o + ((size_t)g.nvb + 2) * 4);
@@ -122,6 +126,9 @@ size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layou
     o = align_up(o + (size_t)s->W * s->W * 8);
     L.pk_off = o;
     o = align_up(o + ((size_t)s->W * s->W + 1) * 8);
+    L.pk_of = with_pk ? o : kNoScratch;
+    if (with_pk)
+        o = align_up(o + (size_t)s->N * s->K * 4);
     return o;
 }
 
@@ -379,6 +386,7 @@ struct DispatchScratch {
     int32_t *agg, *incl;
     int64_t *pk_base;
     int32_t *moved;
+    int32_t *pk_of;  // null: not available (the fused pass then copies by token block)
 };
 
 // Row pieces of a token block (an upper bound: the block's tokens times pieces per row).
@@ -416,6 +424,93 @@ int place_slots(const moe_shape_t *s, const Geometry &g, int parts)
 // One dispatch pass over `rounds` rounds of virtual blocks: the control words zeroed, the
 // histogram / look-back / totals kernel, then the placement kernel (positions, the mapping
 // table and, when `pay` is given, the copy of the rows).
+// The one-kernel pass (dispatch_fused_kernel) when it applies: one round, bf16 rows or no
+// copy, the layout within a CTA's shared memory, and every CTA of the grid resident at once
+// (a cooperative launch: the grid barrier needs them all). Returns 1 when launched, 0 when the
+// two-kernel pass must run instead, -1 on a CUDA error.
+int dispatch_fused(const moe_shape_t *s, const Geometry &g, const VBlocks &vbm,
+                   const int32_t *topk_idx, int32_t *counts, int32_t *kept, int32_t *offsets,
+                   int32_t *row_of, int32_t *assign_of_row, int32_t *expert_of, const Payload *pay,
+                   const uint16_t *x, int64_t *D, int64_t *pk_off, moe_stats_t *stats,
+                   const DispatchScratch &sc, cudaStream_t st, const RankPack &rk)
+{
+    if (pay && pay->e4m3)
+        return 0;
+    const int nvb = g.nvb_round, nseg = g.nseg_round;
+    const int nsub = g.slot_major ? s->K : 1;
+    constexpr size_t kMaxSmem = 200 * 1024;  // dynamic; the kernel's static part stays below 1 KB
+    const size_t big = fused_layout(s->E, s->K, s->W, nvb, nseg, nsub, 2).total;
+    if (big > kMaxSmem)
+        return 0;
+    int per_sm = 0;
+    if (smem_attr_once(dispatch_fused_kernel, (int)kMaxSmem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_fused_kernel, kPlaceThreads,
+                                                      big) != cudaSuccess) {
+        (void)cudaGetLastError();  // not available here: the two-kernel pass runs instead
+        return 0;
+    }
+    const int capacity = per_sm * num_sms();
+    if (capacity < g.nblk)
+        return 0;
+    int parts = 1, slots = 1;
+    if (pay) {
+        const int items = place_items(s, g);
+        parts = capacity / g.nblk;
+        const int cap = (items + 3) / 4;
+        parts = parts < cap ? parts : cap;
+        parts = parts < 1 ? 1 : parts;
+        slots = 2;  // the copy by destination row deals the rows over every warp of the grid
+    }
+    const size_t smem = fused_layout(s->E, s->K, s->W, nvb, nseg, nsub, slots).total;
+    if (cudaMemsetAsync(sc.ctl, 0, 4, st) != cudaSuccess)
+        return -1;
+    FusedArgs fa = {};
+    fa.topk_idx = topk_idx;
+    fa.vbm = vbm;
+    fa.nvb = nvb;
+    fa.bps = g.bps;
+    fa.nseg = nseg;
+    fa.N = s->N;
+    fa.E = s->E;
+    fa.K = s->K;
+    fa.W = s->W;
+    fa.C = (int)g.C;
+    fa.ctl = sc.ctl;
+    fa.agg = sc.agg;
+    fa.counts = counts;
+    fa.kept = kept;
+    fa.offsets = offsets;
+    fa.D = D;
+    fa.pk_off = pk_off;
+    fa.row_of = row_of;
+    fa.assign_of_row = assign_of_row;
+    fa.expert_of = expert_of;
+    fa.packed_row_of = rk.packed_row_of;
+    fa.rank = rk.rank;
+    fa.x_row0 = rk.x_row0;
+    fa.send_row_of = rk.send_row_of;
+    fa.pk_of = sc.pk_of;
+    fa.copy = pay ? 1 : 0;
+    fa.x = x;
+    fa.d = s->d;
+    fa.x_sorted = pay ? pay->x_sorted : nullptr;
+    fa.x_packed = pay ? pay->x_packed : nullptr;
+    fa.stats = stats;
+    fa.slots = slots;
+    fa.timeout_ns = kWaitTimeoutNs;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(g.nblk, parts);
+    cfg.blockDim = dim3(kPlaceThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, dispatch_fused_kernel, fa) == cudaSuccess ? 1 : -1;
+}
+
 moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
                            const int32_t *moved, const int32_t *topk_idx, int32_t *counts,
                            int32_t *kept, int32_t *offsets, int32_t *row_of,
@@ -432,6 +527,12 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
     vbm.nvb_round = g.nvb_round;
     vbm.moved = moved;
     const int nvb = rounds * g.nvb_round, nseg = rounds * g.nseg_round;
+    if (rounds == 1) {
+        const int f = dispatch_fused(s, g, vbm, topk_idx, counts, kept, offsets, row_of,
+                                     assign_of_row, expert_of, pay, x, D, pk_off, stats, sc, st, rk);
+        if (f != 0)
+            return f > 0 ? launch_status() : MOE_ERR_CUDA;
+    }
     if (cudaMemsetAsync(sc.ctl, 0, ((size_t)nvb + 2) * 4, st) != cudaSuccess)
         return MOE_ERR_CUDA;
     HistArgs ha;
@@ -457,8 +558,10 @@ moe_status_t dispatch_pass(const moe_shape_t *s, const Geometry &g, int rounds,
     ha.pk_base = sc.pk_base;
     ha.stats = stats;
     ha.timeout_ns = kWaitTimeoutNs;
-    const size_t hsm = hist_smem_bytes(s->E, s->W);
-    if (smem_attr_once(dispatch_hist_kernel, (int)hist_smem_bytes(kMaxE, kMaxW)) != cudaSuccess)
+    const size_t hsm = hist_smem_bytes(s->E, s->W, nseg);
+    if (smem_attr_once(dispatch_hist_kernel,
+                       (int)(hist_smem_bytes(kMaxE, kMaxW, 0) + (size_t)kCumCacheInts * 4)) !=
+        cudaSuccess)
         return MOE_ERR_CUDA;
     dispatch_hist_kernel<<<nvb, kHistThreads, hsm, st>>>(ha);
 
@@ -516,7 +619,9 @@ DispatchScratch scratch_at(char *w, const Layout &L)
                            reinterpret_cast<int32_t *>(w + L.agg),
                            reinterpret_cast<int32_t *>(w + L.incl),
                            reinterpret_cast<int64_t *>(w + L.pk_base),
-                           reinterpret_cast<int32_t *>(w + L.moved)};
+                           reinterpret_cast<int32_t *>(w + L.moved),
+                           L.pk_of == kNoScratch ? nullptr
+                                                 : reinterpret_cast<int32_t *>(w + L.pk_of)};
 }
 
 // logits: needed when g.rounds == 2 (re-routing); the moved-to experts then go to sc.moved.
@@ -1895,13 +2000,13 @@ moe_status_t static_scratch_address(void **out)
 }
 
 struct StaticLayout {
-    size_t ctl, agg, incl, pk_base, moved, D, pk_off, total;
+    size_t ctl, agg, incl, pk_base, moved, D, pk_off, pk_of, total;
 };
 
 StaticLayout static_layout(const moe_shape_t *s, const Geometry &g)
 {
     StaticLayout L;
-    L.total = dispatch_scratch(s, g, 0, L);
+    L.total = dispatch_scratch(s, g, 0, L, false);
     return L;
 }
 
