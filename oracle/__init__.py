@@ -77,6 +77,12 @@ def _load():
         lib.orc_quantize_blocks_e4m3.restype = None
         lib.orc_round_bf16.argtypes = [_i64, _p, _p]
         lib.orc_round_bf16.restype = None
+        lib.orc_round_f16.argtypes = [_i64, _p, _p]
+        lib.orc_round_f16.restype = None
+        lib.orc_f16_scale_exponent.argtypes = [ctypes.c_double]
+        lib.orc_f16_scale_exponent.restype = _i64
+        lib.orc_quantize_blocks_f16.argtypes = [_i64, _i64, _i64, _p, _p, _p]
+        lib.orc_quantize_blocks_f16.restype = None
         lib.orc_down_rows.argtypes = [_i64, _p, _i64, _i64, _p, _p, _p]
         lib.orc_down_rows.restype = None
         _lib = lib
@@ -355,6 +361,37 @@ def quantize_blocks_e4m3(v, block: int = 32) -> tuple:
     exps = np.empty((rows, cols // block), np.int32)
     _load().orc_quantize_blocks_e4m3(rows, cols, block, _ptr(a), _ptr(codes), _ptr(exps))
     return codes, exps
+
+
+def round_f16(v: np.ndarray) -> np.ndarray:
+    """Nearest fp16 of each float64 value (ties to even), as uint16 bits."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty(v.shape, np.uint16)
+    _load().orc_round_f16(v.size, _ptr(v), _ptr(out))
+    return out
+
+
+def f16_scale_exponent(amax: float) -> int:
+    return int(_load().orc_f16_scale_exponent(float(amax)))
+
+
+def quantize_blocks_f16(v, block: int = 32) -> tuple:
+    """Block-wise fp16 quantisation of a float matrix [rows][cols] (values taken exactly).
+    Returns (codes uint16 fp16 bits [rows][cols], exps int32 [rows][cols / block]); value =
+    fp16 code value * 2^exp."""
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    rows, cols = a.shape
+    assert cols % block == 0
+    codes = np.empty((rows, cols), np.uint16)
+    exps = np.empty((rows, cols // block), np.int32)
+    _load().orc_quantize_blocks_f16(rows, cols, block, _ptr(a), _ptr(codes), _ptr(exps))
+    return codes, exps
+
+
+def dequantize_blocks_f16(codes: np.ndarray, exps: np.ndarray, block: int = 32) -> np.ndarray:
+    """fp16 code value * 2^exp of every element, float64 (exact)."""
+    v = np.asarray(codes, np.uint16).view(np.float16).astype(np.float64)
+    return v * np.exp2(np.repeat(np.asarray(exps, np.float64), block, axis=1))
 
 
 def dequantize_blocks_e4m3(codes: np.ndarray, exps: np.ndarray, block: int = 32) -> np.ndarray:

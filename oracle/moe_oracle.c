@@ -556,6 +556,79 @@ EXPORT void orc_quantize_blocks_e4m3(int64_t rows, int64_t cols, int64_t block,
     }
 }
 
+/* Nearest fp16 value (1 sign, 5 exponent bits with bias 15, 10 mantissa bits: normal values
+ * 2^-14 .. 65504, subnormals in steps of 2^-24) to a double, ties to even, as fp16 bits; a value
+ * that rounds above 65504 becomes infinity. */
+static uint16_t f16_nearest(double v)
+{
+    if (isnan(v))
+        return 0x7E00;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e); /* binade [2^(e-1), 2^e) */
+    int E = e - 1 < -14 ? -14 : e - 1;
+    double quantum = ldexp(1.0, E - 10);
+    double val = nearbyint(a / quantum) * quantum; /* exact quotient; ties to even */
+    if (val > 65504.0)
+        return sign | 0x7C00;
+    if (val == 0.0)
+        return sign;
+    frexp(val, &e);
+    E = e - 1;
+    if (E < -14) /* subnormal: exponent field 0, mantissa = val / 2^-24 */
+        return sign | (uint16_t)(val / ldexp(1.0, -24));
+    const uint16_t mant = (uint16_t)(ldexp(val, -E) * 1024.0 - 1024.0);
+    return sign | (uint16_t)((E + 15) << 10) | mant;
+}
+
+EXPORT void orc_round_f16(int64_t n, const double *v, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = f16_nearest(v[i]);
+}
+
+/* The exponent j of a block's power-of-two scale for fp16 codes: the smallest j in
+ * [-126, 127] with amax * 2^-j <= 65504 (fp16's largest finite value), 0 for a zero or
+ * non-finite amax: the e4m3 rule above with fp16's bound. */
+EXPORT int64_t orc_f16_scale_exponent(double amax)
+{
+    if (!(amax > 0.0) || !isfinite(amax))
+        return 0;
+    int64_t j = -126;
+    while (j < 127 && ldexp(amax, (int)-j) > 65504.0)
+        j += 1;
+    return j;
+}
+
+/* Block-wise fp16 quantisation of the expert outputs (the return payload in 16 bits, a reading
+ * that extends the FP8 payload's block rule of [MoE 推理服务工程真相 2026, §6.3] to fp16 codes):
+ * every run of `block` consecutive columns of a row takes the exponent j above from its largest
+ * magnitude, each value is stored as the nearest fp16 of value * 2^-j. src [rows][cols] double;
+ * codes [rows][cols] fp16 bits; exps [rows][cols / block] (value = code value * 2^j). */
+EXPORT void orc_quantize_blocks_f16(int64_t rows, int64_t cols, int64_t block,
+                                    const double *src, uint16_t *codes, int32_t *exps)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < cols / block; ++b) {
+            const double *v = src + r * cols + b * block;
+            double amax = 0.0;
+            for (int64_t c = 0; c < block; ++c) {
+                double a = fabs(v[c]);
+                if (a > amax || isnan(a))
+                    amax = a;
+            }
+            int64_t j = orc_f16_scale_exponent(amax);
+            exps[r * (cols / block) + b] = (int32_t)j;
+            for (int64_t c = 0; c < block; ++c)
+                codes[r * cols + b * block + c] = f16_nearest(ldexp(v[c], (int)-j));
+        }
+    }
+}
+
 /* Nearest bf16 value (1 sign, 8 exponent bits, 7 mantissa bits: binary32's range with 8
  * significant bits) to a double, ties to even, as bf16 bits; beyond the largest finite value
  * (2 - 2^-7) * 2^127 rounds to infinity. */

@@ -678,3 +678,76 @@ def test_layer_fp8_down_noise_bounded(orc):
         np.float32).astype(np.float64)
     rel = np.abs(hd - hb) / np.maximum(np.abs(hb), 2.0 ** -6 * q["hs"][:, None])
     assert rel.max() <= 2.0 ** -4
+
+
+# --------------------------------------------------------------------------- fp16 y payload
+# fp16: 1 sign, 5 exponent bits (bias 15), 10 mantissa bits, largest finite 65504.
+
+F16_HAND = [  # (value, bits): format corners and round-to-nearest-even ties, worked by hand
+    (0.0, 0x0000), (-0.0, 0x8000), (1.0, 0x3C00), (-2.0, 0xC000), (65504.0, 0x7BFF),
+    (65520.0, 0x7C00),  # halfway 65504 / 65536: ties to the even, out of range -> infinity
+    (65519.0, 0x7BFF),
+    (2.0 ** -24, 0x0001), (2.0 ** -14, 0x0400), (1023 * 2.0 ** -24, 0x03FF),  # subnormals
+    (2.0 ** -25, 0x0000),  # half the smallest subnormal: ties to the even code 0
+    (3 * 2.0 ** -25, 0x0002),  # 1.5 quanta: ties to 2
+    (1.0 + 2.0 ** -11, 0x3C00),  # halfway 1 / 1 + 2^-10: even mantissa 0
+    (1.0 + 3 * 2.0 ** -11, 0x3C02),  # halfway 1 + 2^-10 / 1 + 2^-9: even mantissa 2
+    (1.0 / 3.0, 0x3555),
+]
+
+
+def test_f16_hand_values(orc):
+    v = np.array([a for a, _ in F16_HAND])
+    np.testing.assert_array_equal(orc.round_f16(v), [c for _, c in F16_HAND])
+    assert orc.round_f16(np.array([np.nan]))[0] & 0x7C00 == 0x7C00
+
+
+def test_f16_matches_torch_float16(orc):
+    """torch's float32 -> float16 conversion is an independent implementation of the same
+    rounding: agree on random fp32 values over the whole range and on every tie of a binade.
+    (From float64 torch rounds twice, through float32, and differs at near-ties: 155.9374935
+    lies below the 155.9375 tie and is 155.875, torch gives 156; the payload's values are
+    fp32, where one rounding is the definition.)"""
+    rng = np.random.default_rng(7)
+    v = np.concatenate([rng.standard_normal(100000) * 100,
+                        np.exp(rng.uniform(-20, 11.2, 100000)) * rng.choice([-1, 1], 100000)])
+    grid = np.arange(0x3C00, 0x4000, dtype=np.uint16).view(np.float16).astype(np.float64)
+    v = np.concatenate([v, (grid[1:] + grid[:-1]) / 2, -(grid[1:] + grid[:-1]) / 2])
+    v32 = v.astype(np.float32)
+    ref = torch.from_numpy(v32).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(orc.round_f16(v32.astype(np.float64)), ref)
+    assert orc.round_f16(np.array([155.93749352322445]))[0] == 0x58DF  # below the tie
+
+
+def test_f16_scale_exponent(orc):
+    assert orc.f16_scale_exponent(0.0) == 0 and orc.f16_scale_exponent(float("nan")) == 0
+    assert orc.f16_scale_exponent(65504.0) == 0 and orc.f16_scale_exponent(65505.0) == 1
+    assert orc.f16_scale_exponent(1.0) == -15  # 2^15 = 32768 <= 65504 < 65536
+    rng = np.random.default_rng(8)
+    for amax in np.exp(rng.uniform(-60, 60, 2000)):
+        j = orc.f16_scale_exponent(amax)
+        assert 32752.0 < math.ldexp(amax, -j) <= 65504.0  # the smallest power of two that fits
+    assert orc.f16_scale_exponent(1e-40) == -126  # clamped: the exponent byte stays in range
+
+
+def test_quantize_blocks_f16(orc):
+    """Each 32-column block: exponent from its largest magnitude by the rule above, codes =
+    torch's float16 conversion of the block scaled by 2^-j; dequantised values within half an
+    fp16 step of the input (relative 2^-11 of the block's scale-adjusted top binade)."""
+    rng = np.random.default_rng(9)
+    v = (rng.standard_normal((20, 128)) * np.exp(rng.uniform(-40, 40, (20, 4))).repeat(32, axis=1)
+         ).astype(np.float32).astype(np.float64)
+    v[4, 64:96] = 0.0
+    codes, exps = orc.quantize_blocks_f16(v)
+    for b in range(4):
+        blk = v[:, 32 * b:32 * b + 32]
+        for r in range(20):
+            j = orc.f16_scale_exponent(np.abs(blk[r]).max())
+            assert exps[r, b] == j
+            ref = torch.from_numpy(np.ldexp(blk[r], -j)).to(torch.float16)
+            np.testing.assert_array_equal(codes[r, 32 * b:32 * b + 32],
+                                          ref.view(torch.int16).numpy().view(np.uint16))
+    assert exps[4, 2] == 0 and np.all(codes[4, 64:96] == 0)
+    back = orc.dequantize_blocks_f16(codes, exps)
+    scale = np.exp2(np.repeat(exps, 32, axis=1).astype(np.float64))
+    assert np.all(np.abs(back - v) <= 2.0 ** -11 * np.maximum(np.abs(v), 2.0 ** -14 * scale))
