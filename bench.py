@@ -328,9 +328,10 @@ def algorithmic_work(w, R: int, E_act: int) -> dict:
         # (the FP8 payload writes one byte per element and a 4-byte scale per row)
         scatter_bytes=(N * d * 2 + 2 * R * (d + 4) + N * K * 4 * 3 if w.fp8
                        else N * d * 2 + 2 * R * d * 2 + N * K * 4 * 3),
-        # combine: read every kept expert row (fp32, or the FP8 return payload: e4m3 codes and
+        # combine: read every kept expert row (fp32, or a block payload: e4m3 or fp16 codes and
         # one exponent byte per 32 columns), the routing, write the bf16 out
-        combine_bytes=(R * (d + d // 32) if w.fp8_return else R * d * 4) + N * K * 8 + N * d * 2,
+        combine_bytes=(R * (d + d // 32) if w.fp8_return else
+                       R * (2 * d + d // 32) if w.y_f16 else R * d * 4) + N * K * 8 + N * d * 2,
     )
 
 
@@ -372,7 +373,7 @@ def run_gpu(args, w) -> dict:
         # the layer's output is bf16, as the hidden states it replaces (a stack's next input)
         return m.make_shape(wl.N, wl.d, wl.f, wl.E, wl.K, wl.W, wl.cf, out_bf16=True,
                             slot_major=wl.slot_major, reroute=wl.reroute,
-                            fp8_return=wl.fp8_return)
+                            fp8_return=wl.fp8_return, y_f16=wl.y_f16)
 
     shape = make(w)
     # a stack also times every point of its capacity-factor x Zipf-skew grid (same weights)
@@ -751,7 +752,8 @@ def run_gpu(args, w) -> dict:
         "dtype": (("e4m3 (dispatch payload, both expert GEMMs' operands and the return "
                    "payload), fp32 accumulate" if w.fp8_return else
                    "e4m3 (dispatch payload and both expert GEMMs' operands), fp32 accumulate")
-                  if w.fp8 else "bf16 (x, W1, W3), fp16 (h, W2), fp32 accumulate"),
+                  if w.fp8 else "bf16 (x, W1, W3), fp16 (h, W2), fp32 accumulate" + (
+                      "; y as fp16 codes + block exponents" if w.y_f16 else "")),
         "data": "synthetic (seeded: x N(0,1), router per the workload, experts N(0,0.02^2); "
                 "random-init weights)",
         "config": {"workload": w.name, "N": N, "d": d, "f": f, "E": E, "K": K, "W": W,
@@ -761,6 +763,8 @@ def run_gpu(args, w) -> dict:
                    "step": (f"the {L}-layer stack, x_(l+1) = bf16(x_l + MoE_l(x_l))" if L > 1
                             else "one layer"),
                    "output": "bf16 [N][d], the fp32 sum rounded once",
+                   "y_payload": ("e4m3 codes + exponent per 32 columns" if w.fp8_return else
+                                 "fp16 codes + exponent per 32 columns" if w.y_f16 else "fp32"),
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {L * 3 * E * d * f * 2 / 1e9:.2f} GB of expert "
                          "weights streamed per step, no flush"},
@@ -964,6 +968,10 @@ def parse(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="time eager launches instead of replaying the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--y-f32", action="store_true",
+                    help="the expert outputs travel to the combine as fp32 rows instead of the "
+                         "default fp16 codes with one power-of-two exponent per 32 columns "
+                         "(bf16-path workloads; the FP8 workloads keep their own payloads)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run the workload with this many tokens instead of its own N (a reduced "
                          "case for profiler captures; not a benchmark configuration)")
@@ -978,6 +986,8 @@ def main(argv=None):
     w = WORKLOADS[args.workload]
     if args.tokens > 0:
         w = w.with_(N=args.tokens)
+    if not w.fp8 and not args.y_f32:
+        w = w.with_(y_f16=True)
     if args.impl == "reference":
         res = run_reference(args, w)
     else:

@@ -163,16 +163,18 @@ MOE_FLAG_SLOT_MAJOR = 2
 MOE_FLAG_REROUTE = 4
 MOE_FLAG_FP8_RETURN = 8
 MOE_FLAG_H_BF16 = 16
+MOE_FLAG_Y_F16 = 32
 
 
 def make_shape(N: int, d: int, f: int, E: int, K: int, W: int, capacity_factor: float = 0.0,
                out_bf16: bool = False, slot_major: bool = False,
-               reroute: bool = False, fp8_return: bool = False, h_bf16: bool = False) -> MoeShape:
+               reroute: bool = False, fp8_return: bool = False, h_bf16: bool = False,
+               y_f16: bool = False) -> MoeShape:
     """h_bf16: the SwiGLU activation h and the down-projection weights in bf16 instead of the
     default fp16 (then W2 is passed as the bf16 weights, not their fp16 copy)."""
     flags = ((MOE_FLAG_OUT_BF16 if out_bf16 else 0) | (MOE_FLAG_SLOT_MAJOR if slot_major else 0)
              | (MOE_FLAG_REROUTE if reroute else 0) | (MOE_FLAG_FP8_RETURN if fp8_return else 0)
-             | (MOE_FLAG_H_BF16 if h_bf16 else 0))
+             | (MOE_FLAG_H_BF16 if h_bf16 else 0) | (MOE_FLAG_Y_F16 if y_f16 else 0))
     return MoeShape(N, d, f, E, K, W, float(capacity_factor), flags)
 
 
@@ -196,8 +198,10 @@ def moe_y_bytes(shape: MoeShape) -> int:
 
 
 def y_payload_stride(shape: MoeShape) -> int:
-    """Row stride in bytes of the FP8 return payload: d codes + d/32 exponents, padded to 16."""
-    return shape.d + ((shape.d // 32 + 15) // 16) * 16
+    """Row stride in bytes of the y payload: d e4m3 codes (FP8 return) or 2d bytes of fp16 codes
+    (MOE_FLAG_Y_F16), then d/32 exponents, padded to 16."""
+    codes = 2 * shape.d if shape.flags & MOE_FLAG_Y_F16 else shape.d
+    return codes + ((shape.d // 32 + 15) // 16) * 16
 
 
 def moe_rows_alloc(shape: MoeShape) -> int:

@@ -17,9 +17,10 @@ namespace moe {
 // result is stored as fp32, or rounded once to bf16 (OUT_BF16).
 // A warp's work item is one token and `seg` 8-column chunks of its row (the whole
 // row for large N; a slice when there are too few tokens to fill the GPU).
-// Y8: the expert outputs arrive as the FP8 return payload (rows of y_stride bytes: d e4m3
-// codes, then one exponent byte j + 127 per 32 columns); each value is decoded exactly
-// (e4m3 -> f16 -> f32, times 2^j) before the same fp32 accumulation.
+// YK: how the expert outputs arrive: 0 fp32 rows; 1 the FP8 return payload (rows of y_stride
+// bytes: d e4m3 codes, then one exponent byte j + 127 per 32 columns); 2 the fp16 payload (2d
+// bytes of fp16 codes, then the exponent bytes). A payload value is decoded exactly (code ->
+// f32, times 2^j) before the same fp32 accumulation.
 __device__ __forceinline__ float f16_to_f32(uint32_t h)
 {
     float f;
@@ -43,7 +44,7 @@ __device__ __forceinline__ void decode_e4m3x8(uint32_t lo, uint32_t hi, float sc
     }
 }
 
-template <bool OUT_BF16, bool Y8>
+template <bool OUT_BF16, int YK>
 __global__ void __launch_bounds__(256)
     combine_kernel(const void *__restrict__ y, int y_stride, const int32_t *__restrict__ row_of,
                    const float *__restrict__ topk_w, const float *__restrict__ shared_y,
@@ -81,7 +82,32 @@ __global__ void __launch_bounds__(256)
                 const float wk = __shfl_sync(0xffffffffu, w, k);
                 if (rk < 0)
                     continue;
-                if constexpr (Y8) {
+                if constexpr (YK == 2) {
+                    const uint8_t *prow = reinterpret_cast<const uint8_t *>(y) +
+                                          (size_t)rk * y_stride;
+                    uint4 v[U];
+                    uint32_t ex[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u)
+                        if (c + 32 * u < cend) {
+                            v[u] = reinterpret_cast<const uint4 *>(prow)[c + 32 * u];
+                            ex[u] = prow[2 * d + (c + 32 * u) / 4];
+                        }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        if (c + 32 * u < cend) {
+                            const float sc = pow2f((int)ex[u] - 127);
+                            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                acc[u][2 * q] = __fmaf_rn(wk, f16_to_f32(w4[q] & 0xFFFFu) * sc,
+                                                          acc[u][2 * q]);
+                                acc[u][2 * q + 1] = __fmaf_rn(wk, f16_to_f32(w4[q] >> 16) * sc,
+                                                              acc[u][2 * q + 1]);
+                            }
+                        }
+                    }
+                } else if constexpr (YK == 1) {
                     const uint8_t *prow = reinterpret_cast<const uint8_t *>(y) +
                                           (size_t)rk * y_stride;
                     uint2 v[U];

@@ -89,6 +89,29 @@ __device__ __forceinline__ int e4m3_scale_exp(float amax)
     return max(-126, min(127, j));
 }
 
+// Exponent j of a block's power-of-two scale for fp16 codes: the smallest j with
+// amax * 2^-j <= 65504 (fp16's largest finite value), clamped to [-126, 127]; 0 for a zero or
+// non-finite amax. From the bits of amax (amax = m * 2^k, m in [1, 2)): 65504 = (2 - 2^-10) *
+// 2^15, so j = k - 15 when m <= 2 - 2^-10 (fraction bits <= 0x7FE000), else k - 14.
+__device__ __forceinline__ int f16_scale_exp(float amax)
+{
+    if (!(amax > 0.0f) || !isfinite(amax))
+        return 0;
+    const uint32_t b = __float_as_uint(amax);
+    int k;
+    uint32_t frac;
+    if (b >= 0x00800000u) {
+        k = (int)(b >> 23) - 127;
+        frac = b & 0x007FFFFFu;
+    } else {  // subnormal: normalise the significand
+        const int lz = __clz(b) - 8;
+        k = -126 - lz;
+        frac = (b << lz) & 0x007FFFFFu;
+    }
+    const int j = frac <= 0x007FE000u ? k - 15 : k - 14;
+    return max(-126, min(127, j));
+}
+
 // 2^j for j in [-126, 127] (a normal float).
 __device__ __forceinline__ float pow2f(int j) { return __uint_as_float((uint32_t)(j + 127) << 23); }
 

@@ -71,7 +71,9 @@ struct Args {
                          // or the FP8 return payload when y_stride > 0
     int ldo;
     int y_stride;        // modes 1, 3: 0, or the payload's row stride in bytes (ldo e4m3 codes,
-                         // then ldo / 32 exponent bytes, padded to 16 bytes)
+                         // or 2 ldo bytes of fp16 codes with y_f16, then ldo / 32 exponent
+                         // bytes, padded to 16 bytes)
+    int y_f16;           // the payload's codes are fp16 (else e4m3)
     const float *row_scale;  // modes 2, 3: scale of each A row [rows_alloc]
     const float *b_scale0;   // mode 2: scale of each W1 row; mode 3: of each W2 row [E * b_rows]
     const float *b_scale1;   // mode 2: scale of each W3 row [E * b_rows]
@@ -147,6 +149,8 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
 }
 // This thread's bulk stores have finished reading shared memory / have completed.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// All but this thread's most recent bulk store have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
@@ -509,6 +513,87 @@ __device__ __forceinline__ void down_epilogue_fp8_return(const Args &args, uint3
     }
 }
 
+// The fp16 return payload: the same blocks with fp16 codes (2 bytes each, the exponent bytes
+// after the 2 ldo code bytes), the block's exponent from f16_scale_exp. When all 32 rows of
+// the warp belong to the expert (wfull), each 32-column piece of codes goes through one of two
+// 2 KB halves of the warp's shared-memory tile (64-byte rows, 64-byte swizzle, as the codes'
+// tensor map expects) and one TMA store of 32 x 32 codes; the pieces alternate halves, so a
+// piece waits only for the store before the previous one. Otherwise (and for the exponent
+// bytes) every thread stores its own row.
+template <int MODE, int BN>
+__device__ __forceinline__ void down_epilogue_f16_return(const Args &args, uint32_t taddr, int n,
+                                                         int row, bool store, float sx,
+                                                         const float *ss, float yscale,
+                                                         const CUtensorMap *ymap, uint32_t ystage,
+                                                         int wrow0, bool wfull)
+{
+    constexpr int CB = epilogue_cols(MODE);
+    const int lane = threadIdx.x & 31;
+    uint8_t *prow = reinterpret_cast<uint8_t *>(args.out) + (size_t)row * args.y_stride;
+    uint64_t exps = 0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += CB) {
+        uint32_t v[CB];
+#pragma unroll
+        for (int q = 0; q < CB / 16; ++q)
+            tmem_ld16(taddr + c + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(v + 16 * q));
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < CB / 32; ++h) {
+            float f[32];
+            uint32_t mx = 0;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                float o = __uint_as_float(v[32 * h + k]);
+                if constexpr (MODE == 3)
+                    o *= sx * ss[c + 32 * h + k];
+                else
+                    o *= yscale;
+                f[k] = o;
+                mx = max(mx, __float_as_uint(o) & 0x7FFFFFFFu);
+            }
+            const int j = f16_scale_exp(__uint_as_float(mx));
+            const float inv = pow2f(-j);
+            uint32_t p[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                p[k] = pack_f16x2(f[2 * k] * inv, f[2 * k + 1] * inv);
+            const int col = c + 32 * h;
+            if (wfull) {
+                const uint32_t half = ystage + (uint32_t)((col / 32) & 1) * 2048u;
+                if (lane == 0)
+                    bulk_wait_read1();  // the store that last read this half has done so
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t addr = half + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                                 "r"(p[4 * k]), "r"(p[4 * k + 1]), "r"(p[4 * k + 2]),
+                                 "r"(p[4 * k + 3])
+                                 : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    tma_store_2d(ymap, half, n * BN + col, wrow0);
+            } else if (store) {
+                uint4 *dst = reinterpret_cast<uint4 *>(prow + 2 * (n * BN + col));
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    dst[k] = make_uint4(p[4 * k], p[4 * k + 1], p[4 * k + 2], p[4 * k + 3]);
+            }
+            exps |= (uint64_t)(uint32_t)(j + 127) << (8 * (col / 32));
+        }
+    }
+    if (store) {
+        uint8_t *eb = prow + 2 * args.ldo + n * (BN / 32);
+        if constexpr (BN == 256)
+            *reinterpret_cast<uint2 *>(eb) = make_uint2((uint32_t)exps, (uint32_t)(exps >> 32));
+        else
+            *reinterpret_cast<uint32_t *>(eb) = (uint32_t)exps;
+    }
+}
+
 // yscale: 2^k when h was stored scaled by 2^-k to stay in fp16's range (1 otherwise).
 template <int MODE, int BN>
 __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, int n, int row,
@@ -517,7 +602,11 @@ __device__ __forceinline__ void down_epilogue(const Args &args, uint32_t taddr, 
                                               int wrow0, bool wfull, float yscale)
 {
     if (args.y_stride > 0) {
-        down_epilogue_fp8_return<MODE, BN>(args, taddr, n, row, store, sx, ss, yscale);
+        if (args.y_f16)
+            down_epilogue_f16_return<MODE, BN>(args, taddr, n, row, store, sx, ss, yscale, ymap,
+                                               ystage, wrow0, wfull);
+        else
+            down_epilogue_fp8_return<MODE, BN>(args, taddr, n, row, store, sx, ss, yscale);
         return;
     }
     constexpr int CB = epilogue_cols(MODE);

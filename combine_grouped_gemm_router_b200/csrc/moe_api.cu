@@ -47,21 +47,28 @@ int64_t capacity_of(const moe_shape_t *s)
     return (int64_t)ceil((double)s->capacity_factor * (double)s->N * (double)s->K / (double)s->E);
 }
 
-// Row stride in bytes of the FP8 return payload (d codes, d/32 exponent bytes padded to 16),
-// or 0 when y is fp32.
+// Row stride in bytes of the y payload: d e4m3 codes (FP8 return) or 2d fp16 codes (fp16
+// return), then d/32 exponent bytes padded to 16; 0 when y is fp32.
 int y_payload_stride(const moe_shape_t *s)
 {
-    if (!(s->flags & MOE_FLAG_FP8_RETURN))
-        return 0;
-    return s->d + ((s->d / 32 + 15) & ~15);
+    const int ex = (s->d / 32 + 15) & ~15;
+    if (s->flags & MOE_FLAG_FP8_RETURN)
+        return s->d + ex;
+    if (s->flags & MOE_FLAG_Y_F16)
+        return 2 * s->d + ex;
+    return 0;
 }
+
+bool y_is_f16(const moe_shape_t *s) { return (s->flags & MOE_FLAG_Y_F16) != 0; }
 
 moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
 {
     if (!s)
         return MOE_ERR_INVALID_ARG;
     if ((s->flags & ~(uint32_t)(MOE_FLAG_OUT_BF16 | MOE_FLAG_SLOT_MAJOR | MOE_FLAG_REROUTE |
-                                MOE_FLAG_FP8_RETURN | MOE_FLAG_H_BF16)) != 0)
+                                MOE_FLAG_FP8_RETURN | MOE_FLAG_H_BF16 | MOE_FLAG_Y_F16)) != 0)
+        return MOE_ERR_INVALID_ARG;
+    if ((s->flags & MOE_FLAG_FP8_RETURN) && (s->flags & MOE_FLAG_Y_F16))
         return MOE_ERR_INVALID_ARG;
     if (s->N < 0 || s->d < 8 || s->E < 1 || s->K < 1 || s->W < 1 || s->f < 0)
         return MOE_ERR_INVALID_ARG;
@@ -73,7 +80,7 @@ moe_status_t check_shape(const moe_shape_t *s, bool gemm, Geometry *g)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (gemm && (s->d % 128 != 0 || s->f < 128 || s->f % 128 != 0))
         return MOE_ERR_UNSUPPORTED_SHAPE;
-    if ((s->flags & MOE_FLAG_FP8_RETURN) && s->d % 128 != 0)
+    if ((s->flags & (MOE_FLAG_FP8_RETURN | MOE_FLAG_Y_F16)) && s->d % 128 != 0)
         return MOE_ERR_UNSUPPORTED_SHAPE;
     if (g) {
         const int64_t NK = (int64_t)s->N * s->K;
@@ -696,19 +703,23 @@ bool make_tmap(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t rows, b
     return r == CUDA_SUCCESS;
 }
 
-// The down projection's output y [rows][inner] fp32 as a store target: box 32 rows x 32
-// columns (128 bytes), 128-byte swizzle (the epilogue's shared-memory tile layout).
-bool make_tmap_y(CUtensorMap *m, float *ptr, uint64_t inner, uint64_t rows)
+// The down projection's output as a store target, box 32 rows x 32 columns: fp32 y
+// [rows][inner] (128-byte rows, 128-byte swizzle), or the fp16 codes of the fp16 return
+// payload (row_bytes apart; 64-byte rows, 64-byte swizzle) -- the epilogue's shared-memory
+// tile layouts.
+bool make_tmap_y(CUtensorMap *m, void *ptr, uint64_t inner, uint64_t rows, bool f16 = false,
+                 uint64_t row_bytes = 0)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
     cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 4};
+    cuuint64_t strides[1] = {f16 ? row_bytes : inner * 4};
     cuuint32_t box[2] = {32, 32};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                     2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     f16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -830,16 +841,16 @@ moe_status_t gemm_up(int E, int d, int f, int64_t a_rows, bool pair, const uint1
 // y_stride > 0: y is the FP8 return payload with that row stride (written by plain stores;
 // the y tensor map, unused then, is a copy of the W2 map).
 moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uint16_t *h,
-                       const int32_t *offsets, const uint16_t *w2, void *y, int y_stride,
+                       const int32_t *offsets, const uint16_t *w2, void *y, int y_stride, bool y_f16,
                        bool f16, uint32_t *h_amax, cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
     if (!make_tmap(&tA, h, f, (uint64_t)a_rows, false, f16) ||
         !make_tmap(&tW2, w2, f, (uint64_t)E * d, false, f16))
         return MOE_ERR_CUDA;
-    if (y_stride > 0)
+    if (y_stride > 0 && !y_f16)
         tY = tW2;
-    else if (!make_tmap_y(&tY, static_cast<float *>(y), d, (uint64_t)a_rows))
+    else if (!make_tmap_y(&tY, y, d, (uint64_t)a_rows, y_f16, (uint64_t)y_stride))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -850,6 +861,7 @@ moe_status_t gemm_down(int E, int d, int f, int64_t a_rows, bool pair, const uin
     args.out = y;
     args.ldo = d;
     args.y_stride = y_stride;
+    args.y_f16 = y_f16 ? 1 : 0;
     args.h_f16 = f16 ? 1 : 0;
     args.h_amax = h_amax;
     args.timeout_ns = kWaitTimeoutNs;
@@ -910,15 +922,15 @@ moe_status_t gemm_up_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const 
 // channel), fp32 y. The pair kernel needs f % 256 == 0 (two atoms per stage).
 moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, const uint8_t *hq,
                             const float *h_scale, const int32_t *offsets, const uint8_t *w2,
-                            const float *s2, void *y, int y_stride, cudaStream_t st)
+                            const float *s2, void *y, int y_stride, bool y_f16, cudaStream_t st)
 {
     CUtensorMap tA, tW2, tY;
     if (!make_tmap(&tA, hq, f, (uint64_t)a_rows, true) ||
         !make_tmap(&tW2, w2, f, (uint64_t)E * d, true))
         return MOE_ERR_CUDA;
-    if (y_stride > 0)
+    if (y_stride > 0 && !y_f16)
         tY = tW2;
-    else if (!make_tmap_y(&tY, static_cast<float *>(y), d, (uint64_t)a_rows))
+    else if (!make_tmap_y(&tY, y, d, (uint64_t)a_rows, y_f16, (uint64_t)y_stride))
         return MOE_ERR_CUDA;
     gg::Args args = {};
     args.offsets = offsets;
@@ -929,6 +941,7 @@ moe_status_t gemm_down_e4m3(int E, int d, int f, int64_t a_rows, bool pair, cons
     args.out = y;
     args.ldo = d;
     args.y_stride = y_stride;
+    args.y_f16 = y_f16 ? 1 : 0;
     args.row_scale = h_scale;
     args.b_scale0 = s2;
     args.timeout_ns = kWaitTimeoutNs;
@@ -981,7 +994,7 @@ moe_status_t expert_down_impl(const moe_shape_t *s, const Geometry &g, const uin
                               cudaStream_t st)
 {
     return gemm_down(s->E, s->d, s->f, g.rows_alloc, use_pair_tiles(s, g), h, offsets, w2, y,
-                     y_payload_stride(s), h_is_f16(s), h_range_word(h, g, s->f), st);
+                     y_payload_stride(s), y_is_f16(s), h_is_f16(s), h_range_word(h, g, s->f), st);
 }
 
 moe_status_t expert_gemm_impl(const moe_shape_t *s, const Geometry &g, const uint16_t *x_sorted,
@@ -1013,7 +1026,8 @@ moe_status_t shared_expert_impl(const moe_shape_t *s, int f_s, const uint16_t *x
                               amax, st);
     if (rc != MOE_OK)
         return rc;
-    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, h_is_f16(s), amax, st);
+    return gemm_down(1, s->d, f_s, s->N, pair, h_s, offsets2, ws2, y_s, 0, false, h_is_f16(s), amax,
+                     st);
 }
 
 moe_status_t combine_impl(const moe_shape_t *s, const void *y, const int32_t *row_of,
@@ -1025,19 +1039,17 @@ moe_status_t combine_impl(const moe_shape_t *s, const void *y, const int32_t *ro
     const int blocks = row_blocks(s->N, nvec, seg);
     const int ys = y_payload_stride(s);
     const bool ob = (s->flags & MOE_FLAG_OUT_BF16) != 0;
-    if (ob && ys)
-        combine_kernel<true, true><<<blocks, 256, 0, st>>>(y, ys, row_of, topk_w, shared_y,
-                                                            residual, s->N, s->d, s->K, seg, out);
-    else if (ob)
-        combine_kernel<true, false><<<blocks, 256, 0, st>>>(y, 0, row_of, topk_w, shared_y,
-                                                             residual, s->N, s->d, s->K, seg, out);
-    else if (ys)
-        combine_kernel<false, true><<<blocks, 256, 0, st>>>(y, ys, row_of, topk_w, shared_y,
-                                                             residual, s->N, s->d, s->K, seg, out);
+    const int yk = ys == 0 ? 0 : y_is_f16(s) ? 2 : 1;  // fp32 y, e4m3 payload, fp16 payload
+    auto go = [&](auto kern) {
+        kern<<<blocks, 256, 0, st>>>(y, ys, row_of, topk_w, shared_y, residual, s->N, s->d, s->K,
+                                     seg, out);
+    };
+    if (ob)
+        yk == 0 ? go(combine_kernel<true, 0>) : yk == 1 ? go(combine_kernel<true, 1>)
+                                                        : go(combine_kernel<true, 2>);
     else
-        combine_kernel<false, false><<<blocks, 256, 0, st>>>(y, 0, row_of, topk_w, shared_y,
-                                                              residual, s->N, s->d, s->K, seg,
-                                                              out);
+        yk == 0 ? go(combine_kernel<false, 0>) : yk == 1 ? go(combine_kernel<false, 1>)
+                                                         : go(combine_kernel<false, 2>);
     return launch_status();
 }
 
@@ -1423,7 +1435,7 @@ moe_expert_down_fp8(const moe_shape_t *shape, const uint8_t *hq, const float *h_
         !aligned4(offsets) || !aligned4(h_scale))
         return MOE_ERR_MISALIGNED;
     return gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc, use_pair_tiles(shape, g),
-                          hq, h_scale, offsets, w2q, w2_scale, y, y_payload_stride(shape),
+                          hq, h_scale, offsets, w2q, w2_scale, y, y_payload_stride(shape), y_is_f16(shape),
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1572,7 +1584,7 @@ moe_status_t layer_run(const moe_shape_t *shape, const Geometry &g, const uint16
             return rc;
         rc = gemm_down_e4m3(shape->E, shape->d, shape->f, g.rows_alloc,
                             use_pair_tiles(shape, g), hq, hs, offsets, up.w2q, up.s2, y,
-                            y_payload_stride(shape), st);
+                            y_payload_stride(shape), y_is_f16(shape), st);
     } else {
         rc = expert_down_impl(shape, g, h, offsets, up.w2, y, st);
     }

@@ -134,6 +134,21 @@ typedef struct moe_shape {
  * quantisation and ignores this flag. */
 #define MOE_FLAG_H_BF16 16u
 
+/* fp16 return payload: the expert outputs y as fp16 codes with one power-of-two exponent per
+ * 32 columns, half the bytes of fp32 y between the down projection and the combine. With this
+ * flag the `y` buffer of moe_expert_down, moe_expert_down_fp8, moe_expert_gemm and moe_combine
+ * (and the layer's internal y) holds, per row, d fp16 codes (2d bytes), then one exponent byte
+ * j + 127 per 32 columns, zero-padded to a multiple of 16 bytes: row stride 2d + roundup16(d/32)
+ * bytes, moe_y_bytes(shape) in all. Block b of row r (columns [32b, 32b + 32)) holds the values
+ * code * 2^j, where j is the smallest power of two with max|block| * 2^-j <= 65504 (fp16's
+ * largest finite value; j in [-126, 127]; 0 for a zero or non-finite block) and each code is the
+ * value * 2^-j rounded to nearest-even fp16: the FP8 payload's block rule with fp16 codes. Every
+ * block is in range whatever the magnitudes, and each value keeps fp16's 11 significant bits
+ * relative to its block's top binade. The values quantised are the fp32 y the plain down GEMM
+ * writes; the combine decodes them exactly and accumulates in fp32. Needs d % 128 == 0; not
+ * with MOE_FLAG_FP8_RETURN. */
+#define MOE_FLAG_Y_F16 32u
+
 /* Per-call dispatch counters, written (not accumulated) by moe_dispatch / moe_layer into
  * DEVICE memory when a non-null pointer is given. Observability signals of
  * "MoE 专家并行的 All-to-All 通信瓶颈", §可观测指标与故障定位, and
@@ -185,8 +200,8 @@ size_t moe_workspace_size(const moe_shape_t *shape);
 size_t moe_layer_workspace_size(const moe_shape_t *shape);
 
 /* Bytes of the y buffer of moe_expert_down / moe_expert_gemm / moe_combine: rows_alloc * d * 4
- * (fp32 y), or rows_alloc * (d + roundup16(d / 32)) with MOE_FLAG_FP8_RETURN. 0 on an invalid
- * shape. */
+ * (fp32 y), rows_alloc * (d + roundup16(d / 32)) with MOE_FLAG_FP8_RETURN, or
+ * rows_alloc * (2d + roundup16(d / 32)) with MOE_FLAG_Y_F16. 0 on an invalid shape. */
 size_t moe_y_bytes(const moe_shape_t *shape);
 
 /* ---------------------------------------------------------------- stages */

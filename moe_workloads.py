@@ -60,6 +60,7 @@ class Workload:
     fp8: bool = False         # e4m3 dispatch payload and gate/up GEMM
     affinity: float = 0.0     # stacks: correlation of a layer's router with the previous one's
     fp8_return: bool = False  # FP8 path: expert outputs travel back as e4m3 + block exponents
+    y_f16: bool = False       # expert outputs travel back as fp16 codes + block exponents
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

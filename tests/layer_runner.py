@@ -13,12 +13,14 @@ def lib():
     return m
 
 
-def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda", h_bf16: bool = False) -> dict:
+def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda", h_bf16: bool = False,
+               y_f16: bool = False) -> dict:
     """route -> dispatch -> expert GEMMs -> combine, each through its C entry point. h and the
-    down-projection weights are fp16 (the library's default) unless h_bf16."""
+    down-projection weights are fp16 (the library's default) unless h_bf16; y is fp32, or the
+    fp16 payload (uint8 bytes) with y_f16."""
     m = lib()
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
-                         reroute=w.reroute, h_bf16=h_bf16)
+                         reroute=w.reroute, h_bf16=h_bf16, y_f16=y_f16)
     dev = torch.device(device)
     x = inp["x"].to(dev)
     wr = inp["w_router"].to(dev)
@@ -56,7 +58,8 @@ def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda", h_bf16: bo
                expert_of=expert_of)
     if w.d % 128 == 0 and w.f % 128 == 0:
         h = torch.zeros(RA, f, dtype=torch.bfloat16 if h_bf16 else torch.float16, device=dev)
-        y = torch.zeros(RA, d, dtype=torch.float32, device=dev)
+        y = (torch.zeros(m.moe_y_bytes(shape), dtype=torch.uint8, device=dev) if y_f16 else
+             torch.zeros(RA, d, dtype=torch.float32, device=dev))
         w2 = m.w2_for(shape, inp["w2"].to(dev))
         m.moe_expert_gemm(shape, x_sorted, offsets, inp["w1"].to(dev), inp["w3"].to(dev),
                           w2, h, y)
@@ -70,10 +73,10 @@ def run_stages(inp: dict, w, pack: bool = True, device: str = "cuda", h_bf16: bo
 
 
 def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True,
-              h_bf16: bool = False) -> dict:
+              h_bf16: bool = False, y_f16: bool = False) -> dict:
     m = lib()
     shape = m.make_shape(w.N, w.d, w.f, w.E, w.K, w.W, w.cf, slot_major=w.slot_major,
-                         reroute=w.reroute, h_bf16=h_bf16)
+                         reroute=w.reroute, h_bf16=h_bf16, y_f16=y_f16)
     dev = torch.device(device)
     ws = torch.empty(m.moe_layer_workspace_size(shape), dtype=torch.uint8, device=dev)
     out = torch.empty(w.N, w.d, dtype=torch.float32, device=dev)
@@ -89,6 +92,28 @@ def run_layer(inp: dict, w, device: str = "cuda", with_stats: bool = True,
         res["stats"] = m.stats_dict(m.read_stats(stats))
     res["dev_error"] = m.moe_get_device_error(True)
     return res
+
+
+def decode_y_payload(shape, ybuf, rows) -> np.ndarray:
+    """Rows `rows` of an fp16 return payload (uint8 bytes on the device) decoded to fp64:
+    code * 2^j per 32-column block."""
+    m = lib()
+    d, st = shape.d, m.y_payload_stride(shape)
+    b = ybuf[:m.moe_rows_alloc(shape) * st].view(-1, st)[rows].cpu().numpy()
+    codes = np.ascontiguousarray(b[:, :2 * d]).view(np.float16).astype(np.float64)
+    j = b[:, 2 * d:2 * d + d // 32].astype(np.int64) - 127
+    return codes * np.exp2(np.repeat(j, 32, axis=1).astype(np.float64))
+
+
+def f16_payload_bound(ybound, y_ref) -> np.ndarray:
+    """ybound (the fp32 y's distance from the oracle's y_ref) widened by the rounding of y to
+    the fp16 block payload: half an fp16 step of |y|, or, where y is subnormal at the block's
+    scale 2^j, half the smallest step there (j is the smallest with blockmax * 2^-j <= 65504,
+    so 2^j < 2 * blockmax / 65504; j >= -126)."""
+    top = np.abs(f64(y_ref)) + ybound
+    bm = top.reshape(*top.shape[:-1], -1, 32).max(-1)
+    s = np.maximum(2.0 * bm / 65504.0, 2.0 ** -126)
+    return ybound + 2.0 ** -11 * top + 2.0 ** -25 * np.repeat(s, 32, axis=-1)
 
 
 def f64(t) -> np.ndarray:

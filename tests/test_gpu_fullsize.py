@@ -15,7 +15,8 @@ import pytest
 import torch
 
 from layer_runner import (assert_rounded_h, assert_within_bound, assert_within_tolerance,
-                          h_bound_rows, run_stages, tolerance_report)
+                          decode_y_payload, f16_payload_bound, h_bound_rows, run_stages,
+                          tolerance_report)
 from moe_workloads import STACK_GRID_CF, STACK_GRID_S, WORKLOADS, make_layer_inputs
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -38,10 +39,12 @@ def host_inputs(inp: dict, experts=None) -> dict:
     return out
 
 
-def check_full_size(orc, w, seed=0, n_sample=24):
+def check_full_size(orc, w, seed=0, n_sample=24, y_f16=False):
+    """With y_f16 the expert outputs travel as the fp16 block payload: its decoded rows are
+    checked against the oracle's y within the fp32 bound widened by the payload's rounding."""
     torch.cuda.empty_cache()
     inp = make_layer_inputs(w, seed=seed, device="cuda")
-    got = run_stages(inp, w)
+    got = run_stages(inp, w, y_f16=y_f16)
     assert got["dev_error"] == 0
     hx = host_inputs(inp, experts=[])  # routing needs no expert weights
     r = orc.route_and_dispatch(hx["x"], hx["w_router"], hx["bias"], w.K, w.W, w.cf,
@@ -93,7 +96,11 @@ def check_full_size(orc, w, seed=0, n_sample=24):
     sample_expert = rr["expert_of"][smp["sample_slots"]]
     ybound = h_bound_rows(smp["sample_h"], hx["w2"], got["w2_used"][torch.from_numpy(used).cuda()],
                           sample_expert)
-    assert_within_bound(got["y"][rows], smp["sample_y"], ybound, "y sample")
+    y_got = got["y"][rows]
+    if y_f16:
+        y_got = decode_y_payload(got["shape"], got["y"], rows)
+        ybound = f16_payload_bound(ybound, smp["sample_y"])
+    assert_within_bound(y_got, smp["sample_y"], ybound, "y sample")
     obound = np.zeros_like(smp["out_tokens"])
     pos = {int(a): i for i, a in enumerate(smp["sample_slots"])}
     for li, t in enumerate(toks):
@@ -106,7 +113,7 @@ def check_full_size(orc, w, seed=0, n_sample=24):
                     smp["sample_y"][yi])
     got_out = got["out"][torch.from_numpy(toks).cuda()]
     assert_within_bound(got_out, smp["out_tokens"], obound, "out sample")
-    rep_y = assert_within_tolerance(got["y"][rows], smp["sample_y"], "y sample")
+    rep_y = assert_within_tolerance(y_got, smp["sample_y"], "y sample")
     rep_o = assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
     # routing margins (reported; the logits are bit-exact, so no seed is rejected)
     lg = np.sort(r["logits"], axis=1)[:, ::-1]
@@ -120,6 +127,13 @@ def check_full_size(orc, w, seed=0, n_sample=24):
 def test_full_size_workload(orc, name, seed):
     rep = check_full_size(orc, WORKLOADS[name], seed=seed)
     print(name, seed, rep)
+
+
+@pytest.mark.parametrize("name", ["mixtral_prefill", "e128_skew", "decode", "stack4"])
+def test_full_size_y_f16(orc, name):
+    """The layers with the fp16 return payload (the bench's default for the non-FP8 path)."""
+    rep = check_full_size(orc, WORKLOADS[name], y_f16=True)
+    print(name, "y fp16 payload", rep)
 
 
 @pytest.mark.parametrize("name", ["e128_skew", "stack4"])
@@ -147,13 +161,14 @@ def test_full_size_stack_layer(orc, cf, s):
     print("stack4 layer 0", cf, s, rep)
 
 
-def full_output_check(orc, w, seed=0):
+def full_output_check(orc, w, seed=0, y_f16=False):
     """The whole output of one layer (every token, every column) against the oracle's layer
     computed in full: routing bit for bit, h within its rounding, y and the output per element
-    within the bound the arithmetic implies and within the stated bar."""
+    within the bound the arithmetic implies and within the stated bar (with y_f16, y is the
+    decoded fp16 block payload and its bound includes the payload's rounding)."""
     torch.cuda.empty_cache()
     inp = make_layer_inputs(w, seed=seed, device="cuda")
-    got = run_stages(inp, w)
+    got = run_stages(inp, w, y_f16=y_f16)
     assert got["dev_error"] == 0
     hx = host_inputs(inp)
     ref = orc.layer(hx, w.K, w.W, w.cf, want_h=True, order=int(w.slot_major), reroute=w.reroute)
@@ -163,7 +178,11 @@ def full_output_check(orc, w, seed=0):
     assert_rounded_h(got["h"][:R], ref["h_rows"], "h", w.d)
     row_expert = ref["expert_of"][ref["assign_of_row"]]
     ybound = h_bound_rows(ref["h_rows"], hx["w2"], got["w2_used"].cpu(), row_expert)
-    assert_within_bound(got["y"][:R], ref["y_rows"], ybound, "y")
+    y_got = got["y"][:R]
+    if y_f16:
+        y_got = decode_y_payload(got["shape"], got["y"], torch.arange(R, device="cuda"))
+        ybound = f16_payload_bound(ybound, ref["y_rows"])
+    assert_within_bound(y_got, ref["y_rows"], ybound, "y")
     kept = np.nonzero(ref["row_of"] >= 0)[0]
     wa = np.abs(ref["topk_w"].reshape(-1)[kept].astype(np.float64))[:, None]
     rows = ref["row_of"][kept]
@@ -171,7 +190,7 @@ def full_output_check(orc, w, seed=0):
     obound = np.zeros((w.N, w.d))
     np.add.at(obound, kept // w.K, per_slot)
     assert_within_bound(got["out"], ref["out"], obound + 1e-30, "out")
-    rep_y = assert_within_tolerance(got["y"][:R], ref["y_rows"], "y")
+    rep_y = assert_within_tolerance(y_got, ref["y_rows"], "y")
     rep_o = assert_within_tolerance(got["out"], ref["out"], "out")
     return dict(R=R, dropped=ref["stats"]["dropped"], y=rep_y, out=rep_o)
 
@@ -183,6 +202,13 @@ def test_full_output_e128_skew(orc, seed):
     rep = full_output_check(orc, WORKLOADS["e128_skew"], seed)
     assert rep["dropped"] > 0
     print("e128_skew full output", seed, rep)
+
+
+@pytest.mark.parametrize("name", ["e128_skew", "decode"])
+def test_full_output_y_f16(orc, name):
+    """Every element of the 128-expert and decode layers with the fp16 return payload."""
+    rep = full_output_check(orc, WORKLOADS[name], 0, y_f16=True)
+    print(name, "full output, y fp16 payload", rep)
 
 
 def test_full_output_decode(orc):
@@ -197,10 +223,11 @@ def test_full_output_mixtral_prefill(orc):
     print("mixtral_prefill full output", rep)
 
 
-def sampled_output_check(orc, inp, w, r, toks, got_out, w2_used):
+def sampled_output_check(orc, inp, w, r, toks, got_out, w2_used, y_f16=False):
     """The layer output of the tokens `toks` (got_out, fp32 rows in the order of toks) against
     the oracle's expert FFN and combine of those tokens under the routing r: per element within
-    the propagated bound, and the stated bar."""
+    the propagated bound (with y_f16, widened by the fp16 payload's rounding), and the stated
+    bar."""
     slots = (toks[:, None] * w.K + np.arange(w.K)[None, :]).reshape(-1)
     eo = r["expert_of"][slots]
     used = np.unique(eo[eo >= 0])
@@ -213,6 +240,8 @@ def sampled_output_check(orc, inp, w, r, toks, got_out, w2_used):
     smp = orc.layer_sampled(hx, w.K, w.W, w.cf, toks, routing=rr, want_h=True)
     sample_expert = rr["expert_of"][smp["sample_slots"]]
     ybound = h_bound_rows(smp["sample_h"], hx["w2"], w2_used[ut].cpu(), sample_expert)
+    if y_f16:
+        ybound = f16_payload_bound(ybound, smp["sample_y"])
     obound = np.zeros_like(smp["out_tokens"])
     pos = {int(a): i for i, a in enumerate(smp["sample_slots"])}
     for li, t in enumerate(toks):
@@ -227,7 +256,7 @@ def sampled_output_check(orc, inp, w, r, toks, got_out, w2_used):
     return assert_within_tolerance(got_out, smp["out_tokens"], "out sample")
 
 
-def stack_teacher_forced(orc, w, n_sample=16):
+def stack_teacher_forced(orc, w, n_sample=16, y_f16=False):
     """The stack of w.layers layers on the GPU, x_{j+1} = bf16(x_j + MoE_j(x_j)), checked layer by
     layer against the oracle fed the GPU's own x_j (teacher forcing, so that the routing
     contract holds per layer):
@@ -235,12 +264,13 @@ def stack_teacher_forced(orc, w, n_sample=16):
      * topk_idx and the dispatch counters of layer j equal the oracle's on x_j, bit for bit;
      * the output of layer j on sampled tokens is within the stated bar of the oracle's;
      * the inter-layer affinity counts moe_affinity_accumulate forms from the GPU's routing
-       equal the oracle's counts from its own routing, bit for bit."""
+       equal the oracle's counts from its own routing, bit for bit.
+    With y_f16 the layers pass their expert outputs to the combine as the fp16 block payload."""
     import combine_grouped_gemm_router_b200 as m
     N, d, E, K = w.N, w.d, w.E, w.K
     torch.cuda.empty_cache()
-    shape32 = m.make_shape(N, d, w.f, E, K, w.W, w.cf)
-    shape16 = m.make_shape(N, d, w.f, E, K, w.W, w.cf, out_bf16=True)
+    shape32 = m.make_shape(N, d, w.f, E, K, w.W, w.cf, y_f16=y_f16)
+    shape16 = m.make_shape(N, d, w.f, E, K, w.W, w.cf, out_bf16=True, y_f16=y_f16)
     ws = torch.empty(m.moe_layer_workspace_size(shape16), dtype=torch.uint8, device="cuda")
     x = make_layer_inputs(w, seed=0, device="cuda", with_x=True)["x"]
     gpu_routes, orc_routes, reports = [], [], []
@@ -270,7 +300,8 @@ def stack_teacher_forced(orc, w, n_sample=16):
                     rs["R"], rs["dropped"], rs["cross_rows"], rs["dedup_pairs"],
                     rs["active_experts"], rs["max_kept"], rs["min_kept"])
         toks = sample_tokens(N, n_sample, seed=layer)
-        rep = sampled_output_check(orc, inp, w, r, toks, moe[torch.from_numpy(toks).cuda()], w2h)
+        rep = sampled_output_check(orc, inp, w, r, toks, moe[torch.from_numpy(toks).cuda()], w2h,
+                                   y_f16=y_f16)
         reports.append(dict(layer=layer, dropped=rs["dropped"], **rep))
         gpu_routes.append(topk)
         orc_routes.append(r["topk_idx"])
@@ -292,6 +323,13 @@ def test_stack_teacher_forced(orc, cf, s):
     skew of its grid, each layer against the oracle on the GPU's own input."""
     reps = stack_teacher_forced(orc, WORKLOADS["stack4"].with_(cf=cf, s=s))
     print("stack4", cf, s, reps)
+
+
+def test_stack_teacher_forced_y_f16(orc):
+    """The stack as the bench runs it (capacity factor 1.25, no skew) with the fp16 return
+    payload between each layer's down projection and combine."""
+    reps = stack_teacher_forced(orc, WORKLOADS["stack4"], y_f16=True)
+    print("stack4 y fp16 payload", reps)
 
 
 def test_stack_teacher_forced_planted_affinity(orc):
