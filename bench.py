@@ -287,8 +287,9 @@ def placement_report(m, counts, L: int, E: int, P: int) -> dict:
 
 def kernel_launches(w) -> int:
     """Kernels the library launches for one layer of workload w, by the same rules as its
-    host code: routing 1 (the fused projection + top-K kernel, E >= 32 and N >= 2048) or 2
-    (projection, then selection); per dispatch pass the histogram / look-back kernel and the
+    host code: routing 2 (the router weights' transposition, then the fused projection + top-K
+    kernel, E > 32 and N >= 2048), 1 (the fused kernel alone, E = 32) or 2 (projection, then
+    selection); per dispatch pass the histogram / look-back kernel and the
     placement kernel (the pass's control words are cleared by a memset, not a kernel); with
     re-routing a positions-only pass, the ranking kernel, then the full pass; each grouped GEMM
     once, or twice (CTA-pair tiles, then single-CTA tiles) when the experts average at least
@@ -299,7 +300,7 @@ def kernel_launches(w) -> int:
     NK = N * K
     C = NK if not w.cf > 0 else min(NK, math.ceil(w.cf * N * K / E))
     pair = min(NK // E, C) >= 768
-    n = 1 if (E >= 32 and N >= 2048) else 2
+    n = (2 if E > 32 else 1) if (E >= 32 and N >= 2048) else 2
     n += (2 + 1 + 2) if w.reroute else 2
     atom = 128 if w.fp8 else 64
     n += 2 if pair and (d // atom) % 2 == 0 else 1                     # gate/up

@@ -28,6 +28,18 @@ __device__ __forceinline__ uint64_t global_timer_ns()
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// (v, v) as the operand pair of a packed fp32 FMA, built by two byte permutes of one word with
+// selector SEL (0x1044: the low bf16 of w as fp32; 0x3244: the high one; 0x3210: w itself).
+// Both halves come from the integer pipe, so the pair costs no move on the FMA pipe, and one
+// asm statement keeps the compiler from merging the two permutes into one register.
+template <uint32_t SEL>
+__device__ __forceinline__ float2 prmt_pair(uint32_t w)
+{
+    uint32_t a, b;
+    asm("prmt.b32 %0, %2, 0, %3;\n\tprmt.b32 %1, %2, 0, %3;" : "=r"(a), "=r"(b) : "r"(w), "n"(SEL));
+    return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+
 // Two fp32 -> one bf16x2 word (round to nearest even), one cvt instruction.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {

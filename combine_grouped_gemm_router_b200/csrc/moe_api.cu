@@ -139,12 +139,26 @@ size_t dispatch_scratch(const moe_shape_t *s, const Geometry &g, size_t o, Layou
     return o;
 }
 
+// The router's one-kernel path: many tokens and E >= 32.
+inline bool router_fused(const moe_shape_t *s) { return s->E >= 32 && s->N >= 2048; }
+
+// Experts the split-warp router form covers (E rounded up to 64, 128 or 256), 0 where another
+// form runs. That form reads the router weights transposed, [d][EC] fp32, from the scratch.
+inline int router_split_ec(const moe_shape_t *s)
+{
+    if (!router_fused(s) || s->E <= 32)
+        return 0;
+    return s->E <= 64 ? 64 : s->E <= 128 ? 128 : 256;
+}
+
 ScratchLayout scratch_layout(const moe_shape_t *s, const Geometry &g)
 {
     ScratchLayout L;
     size_t o = 0;
+    // the router's scratch: the [N][E] logits of its two-kernel path, or the transposed
+    // weights of the split-warp form
     L.logits = o;
-    o = align_up(o + (size_t)s->N * s->E * 4);
+    o = align_up(o + std::max((size_t)s->N * s->E, (size_t)router_split_ec(s) * s->d) * 4);
     L.total = dispatch_scratch(s, g, o, L);
     return L;
 }
@@ -298,15 +312,15 @@ void launch_router_topk(const moe_shape_t *s, const uint16_t *x, const float *wr
         x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
 }
 
-template <int EPAD, int TM>
-void launch_router_tile8(const moe_shape_t *s, const uint16_t *x, const float *wr,
+template <int NE, int TT, int KC, int ST>
+void launch_router_split(const moe_shape_t *s, const uint16_t *x, const float *wt,
                          const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
                          unsigned long long *nonfinite, cudaStream_t st)
 {
-    using L = RouterTile8<EPAD, TM>;
-    smem_attr_once(router_tile8_kernel<EPAD, TM>, L::SMEM_BYTES);
-    router_tile8_kernel<EPAD, TM><<<(s->N + TM - 1) / TM, L::NT, L::SMEM_BYTES, st>>>(
-        x, wr, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
+    using L = RouterSplitTile<NE, TT, KC, ST>;
+    smem_attr_once(router_split_kernel<NE, TT, KC, ST>, L::SMEM_BYTES);
+    router_split_kernel<NE, TT, KC, ST><<<(s->N + kRsTok - 1) / kRsTok, L::NT, L::SMEM_BYTES, st>>>(
+        x, wt, bias, s->N, s->d, s->E, s->K, topk_idx, topk_w, logits, nonfinite);
 }
 
 // The router projection and the top-K selection. logits_out (nullable) receives the [N][E]
@@ -317,27 +331,38 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
 {
     const int N = s->N, d = s->d, E = s->E;
     // Many tokens and E >= 32: the projection and the selection in one kernel (64 tokens x
-    // every expert per CTA; the logits reach HBM only when asked for).
-    if (E >= 32 && N >= 2048) {
-        // E <= 64 with at least 3 CTAs (6 warps) per SM: the register-tiled form (8 tokens x
-        // 8 experts per thread; measured 510 against 537 us at N = 32768, d = 4096, E = 64).
-        // Fewer logits per SM leave it a warp per scheduler, where the broadcast form is
-        // faster (151 against 167 us at N = 8192, d = 2048, E = 128).
-        if (E <= 32)
-            launch_router_topk<2, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                     nonfinite, st);
-        else if (E <= 64 && (long long)N >= 64LL * 3 * num_sms())
-            launch_router_tile8<64, 64>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                        nonfinite, st);
-        else if (E <= 64)
-            launch_router_topk<4, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                     nonfinite, st);
-        else if (E <= 128)
-            launch_router_topk<8, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                     nonfinite, st);
-        else
-            launch_router_topk<16, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out,
-                                      nonfinite, st);
+    // every expert per CTA; the logits reach HBM only when asked for). E > 32: the split-warp
+    // form, on the router weights transposed into the scratch by one small kernel first.
+    if (router_fused(s)) {
+        if (const int EC = router_split_ec(s)) {
+            if (!scratch)
+                return MOE_ERR_WORKSPACE_TOO_SMALL;
+            router_transpose_kernel<<<dim3((d + 31) / 32, EC / 32), 256, 0, st>>>(w_router, E, d,
+                                                                                 EC, scratch);
+#define MOE_RS(NE, TT, KC, ST)                                                                     \
+    launch_router_split<NE, TT, KC, ST>(s, x, scratch, bias, topk_idx, topk_w, logits_out,         \
+                                        nonfinite, st)
+            // E <= 64 with several CTAs per SM: 4 tokens per lane (8 warps per SM at least);
+            // otherwise 2 tokens per lane and twice the warps, 64-element chunks (measured on
+            // the B200: N = 8192, d = 2048, E = 128: 152 -> 141 us against the broadcast form;
+            // N = 32768, d = 4096, E = 64: 509 -> 477 us against the register-tiled form;
+            // N = 8192, d = 2048, E = 256: 266 -> 237 us; N = 8192, d = 2048, E = 64: 111 -> 85 us)
+            const bool many = (long long)N >= 64LL * 3 * num_sms();
+            if (EC == 64) {
+                if (many)
+                    MOE_RS(4, 4, 32, 3);
+                else
+                    MOE_RS(4, 2, 64, 3);
+            } else if (EC == 128) {
+                MOE_RS(8, 2, 64, 3);
+            } else {
+                MOE_RS(16, 4, 64, 2);
+            }
+#undef MOE_RS
+            return launch_status();
+        }
+        launch_router_topk<2, 2>(s, x, w_router, bias, topk_idx, topk_w, logits_out, nonfinite,
+                                 st);  // E == 32: the broadcast form
         return launch_status();
     }
     float *logits = logits_out ? logits_out : scratch;
@@ -1163,7 +1188,7 @@ moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router, co
         !aligned4(topk_idx) || !aligned4(topk_w) || (logits && !aligned4(logits)))
         return MOE_ERR_MISALIGNED;
     float *scratch = nullptr;
-    if (!logits) {
+    if (!logits || router_split_ec(shape)) {
         const ScratchLayout L = scratch_layout(shape, g);
         if (!ws || ws_bytes < L.total)
             return MOE_ERR_WORKSPACE_TOO_SMALL;

@@ -1,8 +1,10 @@
 // Router projection and softmax top-K.
 //
 // [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化] fuses the gate's
-// top-k with the cumsum/scatter that follow; here the gate is two kernels
-// (logits, then selection) and the cumsum/scatter live in dispatch.cuh.
+// top-k with the cumsum/scatter that follow. Here, with many tokens and E >= 32, the
+// projection and the selection are one kernel (router_topk_kernel for E = 32,
+// router_split_kernel after router_transpose_kernel for E > 32); otherwise they are two
+// (router_logits_kernel, then topk_softmax_kernel). The cumsum/scatter live in dispatch.cuh.
 //
 // Logits are defined as one fp32 fused multiply-add per input element in
 // ascending i, from +0, then + bias. That order is kept exactly: the kernel is a
@@ -320,7 +322,7 @@ __device__ __forceinline__ void topk_select_warp(const float *lrow, int E, int K
 }
 
 // ---------------------------------------------------------------------------
-// Router projection fused with the top-K selection, for many tokens and E >= 32.
+// Router projection fused with the top-K selection, broadcast form (many tokens, E = 32).
 //
 // [MoE Inference Communication, §DeepSpeed-MoE › MoE 计算核优化] the gate's top-k runs
 // in the same kernel as the projection: the [N][E] logits need not go to HBM.
@@ -446,8 +448,7 @@ __global__ void __launch_bounds__(32 * NW)
 #pragma unroll
                 for (int t = 0; t < TT; ++t) {
                     const uint32_t word = (q < 2) ? xq[t].x : (q < 4) ? xq[t].y : (q < 6) ? xq[t].z : xq[t].w;
-                    const float xv = (q & 1) ? bf16_hi(word) : bf16_lo(word);
-                    const float2 xx = make_float2(xv, xv);
+                    const float2 xx = (q & 1) ? prmt_pair<0x3244>(word) : prmt_pair<0x1044>(word);
 #pragma unroll
                     for (int p = 0; p < EW / 2; ++p)
                         acc[t][p] = __ffma2_rn(xx, wp[p], acc[t][p]);
@@ -493,177 +494,207 @@ __global__ void __launch_bounds__(32 * NW)
 }
 
 // ---------------------------------------------------------------------------
-// Fused router, register-tiled form (E > 32, many tokens). A CTA takes TM tokens and every
-// expert (E padded to EPAD = 64, 128 or 256). A thread owns 8 tokens (two groups of 4:
-// [4 ty, 4 ty + 4) and [TM/2 + 4 ty, ...)) x 8 experts (j TX + tx, j < 8): 64 logits in
-// registers. x is staged in shared memory as fp32 [i][token] (converted and transposed on its way
-// through registers, one chunk ahead) and W in its own layout [expert][i] (cp.async, zero-filled
-// past d and E). Per element i a thread reads its 8 tokens with two 16-byte loads and, once per
-// four elements, its 8 experts with eight: 4 loads per element against 32 packed FMAs on token
-// pairs ((x_t[i], x_t+1[i]) times (W_e[i], W_e[i]) with `__ffma2_rn`: each half rounds like one
-// fmaf, every logit its single ascending chain from +0). A 128-bit shared-memory load is served
-// per half-warp (two wavefronts at least, even when all lanes read one address); a half-warp
-// here reads 2 token groups and 8 consecutive expert rows (36 floats apart: conflict-free), so
-// each load costs exactly two wavefronts: 8 wavefronts per warp and element against 16 SM cycles
-// of FMA-pipe work.
-template <int EPAD, int TM>
-struct RouterTile8 {
-    static constexpr int KC = 32;
-    static constexpr int TX = EPAD / 8, TY = TM / 8;
-    static constexpr int NT = TX * TY, NW = NT / 32;
-    static constexpr int WX = TX / 8;    // warps across the experts (8 thread columns each)
-    static constexpr int XS = TM + 4;    // fp32 per staged x^T row
-    static constexpr int WS = KC + 4;    // fp32 per staged W row
-    static constexpr int STAGE = KC * XS + EPAD * WS;  // fp32 per ring stage
-    static constexpr int XV = (TM * (KC / 8) + NT - 1) / NT;  // 8-element x pieces per thread
-    static constexpr int LR = EPAD + 1;
-    static constexpr int SMEM_BYTES = (2 * STAGE > TM * LR ? 2 * STAGE : TM * LR) * 4;
-    static_assert(TX % 8 == 0 && TY % 4 == 0, "tile");
-};
-
-__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src, bool valid)
+// The router weights transposed for the split-warp form: wt[i][e] = Wr[e][i] for e < E, 0 for
+// E <= e < EC (a tile of 32 elements x 32 experts per 256-thread CTA, through shared memory).
+__global__ void __launch_bounds__(256)
+    router_transpose_kernel(const float *__restrict__ wr, int E, int d, int EC,
+                            float *__restrict__ wt)
 {
-    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem_src),
-                 "r"(valid ? 16 : 0)
-                 : "memory");
+    __shared__ float tile[32][33];
+    const int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+    for (int r = ty; r < 32; r += 8) {  // r: expert, tx: element
+        const int e = e0 + r, i = i0 + tx;
+        tile[r][tx] = (e < E && i < d) ? wr[(size_t)e * d + i] : 0.0f;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {  // r: element, tx: expert
+        const int i = i0 + r, e = e0 + tx;
+        if (i < d && e < EC)
+            wt[(size_t)i * EC + e] = tile[tx][r];
+    }
 }
 
-template <int EPAD, int TM>
-__global__ void __launch_bounds__(RouterTile8<EPAD, TM>::NT)
-    router_tile8_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr,
+// Fused router, split-warp form (E > 32, many tokens). A CTA takes 64 tokens and EC = 16 NE
+// experts; a warp owns 16 experts: lanes 0-15 the first 8 of them, lanes 16-31 the other 8, and
+// lane j (lane mod 16) of either half owns TT tokens, 16 apart (TT = 4: one token group per
+// expert group; TT = 2: two warps per expert group). A 128-bit shared-memory load is served per
+// half-warp, so when the two halves read two different 16-byte words, one load gives each half
+// four experts' weights of one element at the cost the whole warp pays to read one word: W costs
+// 4 wavefronts per warp and element (a whole-warp broadcast of the same 16 experts pays 8). The
+// arithmetic is that of the other forms: per element a lane forms (x_t[i], x_t[i]) and multiplies
+// it by two neighbouring experts' (W_e[i], W_e+1[i]) in one packed FMA, so every logit is its
+// single ascending fmaf chain from +0. W arrives transposed ([i][e], router_transpose_kernel), so
+// both operands are staged by cp.async alone, STAGES chunks deep; the next element's W and the
+// next 8 elements' x are loaded before the current element's FMAs.
+constexpr int kRsTok = 64;    // tokens per CTA
+
+// NE groups of 16 experts, TT tokens per lane, KC elements of d per staged chunk, ST chunks in
+// flight.
+template <int NE, int TT, int KC, int ST>
+struct RouterSplitTile {
+    static constexpr int TG = 4 / TT;       // token groups of 16 TT tokens
+    static constexpr int NW = NE * TG;
+    static constexpr int NT = 32 * NW;
+    static constexpr int EC = 16 * NE;      // experts covered
+    static constexpr int EP = EC + 4;       // fp32 per staged W^T row
+    static constexpr int XR = KC + 8;       // bf16 per staged x row (16-byte pad: 16-byte loads
+                                            // of 8 consecutive rows hit 8 different bank groups)
+    static constexpr int X_BYTES = kRsTok * XR * 2;
+    static constexpr int W_BYTES = KC * EP * 4;
+    static constexpr int STAGE_BYTES = X_BYTES + W_BYTES;
+    static constexpr int LR = EC + 1;       // fp32 per epilogue logit row
+    static constexpr int LOGIT_BYTES = kRsTok * LR * 4;
+    static constexpr int SMEM_BYTES =
+        ST * STAGE_BYTES > LOGIT_BYTES ? ST * STAGE_BYTES : LOGIT_BYTES;
+    static_assert(TG * TT == 4 && KC % 32 == 0 && ST >= 2, "tile");
+};
+
+// NB 8-element blocks of one staged chunk (NB known at compile time, so the loop is unrolled
+// whole and the loads of the next element and block are scheduled across it).
+template <int NB, int TT, int EP, int XR>
+__device__ __forceinline__ void split_chunk(const uint16_t *xs, const float *ws, int tok0,
+                                            float2 (&acc)[TT][4])
+{
+    uint4 xq[TT];
+#pragma unroll
+    for (int m = 0; m < TT; ++m)
+        xq[m] = *reinterpret_cast<const uint4 *>(xs + (tok0 + 16 * m) * XR);
+    float4 va = *reinterpret_cast<const float4 *>(ws);
+    float4 vb = *reinterpret_cast<const float4 *>(ws + 4);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        uint4 xn[TT];
+        if (b + 1 < NB) {
+#pragma unroll
+            for (int m = 0; m < TT; ++m)
+                xn[m] = *reinterpret_cast<const uint4 *>(xs + (tok0 + 16 * m) * XR + 8 * (b + 1));
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int k = 8 * b + q;
+            float4 na = va, nb = vb;
+            if (k + 1 < 8 * NB) {
+                na = *reinterpret_cast<const float4 *>(ws + (k + 1) * EP);
+                nb = *reinterpret_cast<const float4 *>(ws + (k + 1) * EP + 4);
+            }
+            const float2 wp[4] = {make_float2(va.x, va.y), make_float2(va.z, va.w),
+                                  make_float2(vb.x, vb.y), make_float2(vb.z, vb.w)};
+#pragma unroll
+            for (int m = 0; m < TT; ++m) {
+                const uint32_t word = (q < 2)   ? xq[m].x
+                                      : (q < 4) ? xq[m].y
+                                      : (q < 6) ? xq[m].z
+                                                : xq[m].w;
+                const float2 xx = (q & 1) ? prmt_pair<0x3244>(word) : prmt_pair<0x1044>(word);
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    acc[m][p] = __ffma2_rn(xx, wp[p], acc[m][p]);
+            }
+            va = na;
+            vb = nb;
+        }
+        if (b + 1 < NB) {
+#pragma unroll
+            for (int m = 0; m < TT; ++m)
+                xq[m] = xn[m];
+        }
+    }
+}
+
+template <int NE, int TT, int KC, int ST>
+__global__ void __launch_bounds__(32 * NE * (4 / TT))
+    router_split_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wt,
                         const float *__restrict__ bias, int N, int d, int E, int K,
                         int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
                         float *__restrict__ logits, unsigned long long *nonfinite_count)
 {
-    using G = RouterTile8<EPAD, TM>;
-    constexpr int KC = G::KC;
-    extern __shared__ __align__(16) float rt8_smem[];
+    using L = RouterSplitTile<NE, TT, KC, ST>;
+    extern __shared__ __align__(16) unsigned char rs_smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ty = (warp / G::WX) * 4 + (lane >> 3);
-    const int tx = (warp % G::WX) * 8 + (lane & 7);
-    const int t0 = blockIdx.x * TM;
+    const int half = lane >> 4, j16 = lane & 15;
+    const int t0 = blockIdx.x * kRsTok;
     const int nchunks = (d + KC - 1) / KC;
 
-    uint4 xr[G::XV];
-    auto load_x = [&](int c) {  // x chunk c -> registers (zeros past N and d)
-        const int k0 = c * KC;
-#pragma unroll
-        for (int j = 0; j < G::XV; ++j) {
-            const int idx = tid + j * G::NT;
-            const int t = idx % TM, q = idx / TM;
-            xr[j] = (idx < TM * (KC / 8) && t0 + t < N && k0 + 8 * q < d)
-                        ? __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + t) * d + k0) + q)
-                        : make_uint4(0u, 0u, 0u, 0u);
-        }
-    };
-    auto store_x = [&](int s) {  // registers -> stage s as fp32 [i][token]
-        float *xs = rt8_smem + s * G::STAGE;
-#pragma unroll
-        for (int j = 0; j < G::XV; ++j) {
-            const int idx = tid + j * G::NT;
-            if (idx < TM * (KC / 8)) {
-                const int t = idx % TM, q = idx / TM;
-                const uint32_t w4[4] = {xr[j].x, xr[j].y, xr[j].z, xr[j].w};
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    xs[(8 * q + 2 * h) * G::XS + t] = bf16_lo(w4[h]);
-                    xs[(8 * q + 2 * h + 1) * G::XS + t] = bf16_hi(w4[h]);
-                }
+    // chunk c -> stage c mod ST (cp.async, 16 bytes per copy; x rows past N are left
+    // alone, their logits are never stored): x rows [64][kc] bf16 and W^T rows [kc][EC] fp32
+    auto stage = [&](int c) {
+        if (c < nchunks) {
+            unsigned char *base = rs_smem + (c % ST) * L::STAGE_BYTES;
+            uint16_t *xs = reinterpret_cast<uint16_t *>(base);
+            float *ws = reinterpret_cast<float *>(base + L::X_BYTES);
+            const int k0 = c * KC, kc = min(KC, d - k0);
+            for (int idx = tid; idx < kRsTok * (KC / 8); idx += L::NT) {
+                const int row = idx / (KC / 8), v = idx % (KC / 8);
+                if (t0 + row < N && v * 8 < kc)
+                    cp_async16(xs + row * L::XR + v * 8, x + (size_t)(t0 + row) * d + k0 + v * 8);
             }
-        }
-    };
-    auto issue_w = [&](int c, int s) {  // W chunk c -> stage s, [expert][i] (cp.async)
-        float *ws = rt8_smem + s * G::STAGE + KC * G::XS;
-        const int k0 = c * KC;
-        for (int idx = tid; idx < EPAD * (KC / 4); idx += G::NT) {
-            const int e = idx >> 3, q = idx & 7;
-            const bool ok = e < E && k0 + 4 * q < d;
-            cp_async16_zfill(ws + e * G::WS + 4 * q,
-                             ok ? (const void *)(wr + (size_t)e * d + k0 + 4 * q) : (const void *)wr,
-                             ok);
-        }
-    };
-
-    float2 acc[4][8];  // [token pair][expert j]
-#pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            acc[p][j] = make_float2(0.0f, 0.0f);
-
-    load_x(0);
-    store_x(0);
-    issue_w(0, 0);
-    cp_async_commit();
-    if (nchunks > 1)
-        load_x(1);
-    cp_async_wait<0>();
-    __syncthreads();
-    for (int c = 0; c < nchunks; ++c) {
-        const int s = c & 1;
-        if (c + 1 < nchunks) {  // the other stage, free since the last barrier
-            store_x(s ^ 1);
-            issue_w(c + 1, s ^ 1);
+            for (int idx = tid; idx < kc * (L::EC / 4); idx += L::NT) {
+                const int r = idx / (L::EC / 4), v = idx % (L::EC / 4);
+                cp_async16(ws + r * L::EP + 4 * v, wt + (size_t)(k0 + r) * L::EC + 4 * v);
+            }
         }
         cp_async_commit();
-        if (c + 2 < nchunks)
-            load_x(c + 2);
-        const float *xs = rt8_smem + s * G::STAGE;
-        const float *ws = xs + KC * G::XS;
+    };
+
+    float2 acc[TT][4];  // [token m: tok0 + 16 m][expert pair p of the half]
 #pragma unroll
-        for (int k4 = 0; k4 < KC / 4; ++k4) {
-            float4 w[8];
+    for (int m = 0; m < TT; ++m)
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                w[j] = *reinterpret_cast<const float4 *>(ws + (j * G::TX + tx) * G::WS + 4 * k4);
+        for (int p = 0; p < 4; ++p)
+            acc[m][p] = make_float2(0.0f, 0.0f);
+
+    const int ecol = 16 * (warp % NE) + 8 * half;      // this half's first expert
+    const int tok0 = 16 * TT * (warp / NE) + j16;       // this lane's first token
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int k = 4 * k4 + kk;
-                const float4 xa = *reinterpret_cast<const float4 *>(xs + k * G::XS + 4 * ty);
-                const float4 xb =
-                    *reinterpret_cast<const float4 *>(xs + k * G::XS + TM / 2 + 4 * ty);
-                const float2 pr[4] = {make_float2(xa.x, xa.y), make_float2(xa.z, xa.w),
-                                      make_float2(xb.x, xb.y), make_float2(xb.z, xb.w)};
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float wv = kk == 0 ? w[j].x : kk == 1 ? w[j].y : kk == 2 ? w[j].z : w[j].w;
-                    const float2 ww = make_float2(wv, wv);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p)
-                        acc[p][j] = __ffma2_rn(pr[p], ww, acc[p][j]);
-                }
-            }
+    for (int c = 0; c < ST - 1; ++c)
+        stage(c);
+    for (int c = 0; c < nchunks; ++c) {
+        cp_async_wait<ST - 2>();
+        __syncthreads();  // chunk c has landed; the stage chunk c - 1 used is free
+        stage(c + ST - 1);
+        const unsigned char *base = rs_smem + (c % ST) * L::STAGE_BYTES;
+        const uint16_t *xs = reinterpret_cast<const uint16_t *>(base);
+        const float *ws = reinterpret_cast<const float *>(base + L::X_BYTES) + ecol;
+        const int kc = min(KC, d - c * KC);  // a multiple of 8
+        if (kc == KC) {
+            split_chunk<KC / 8, TT, L::EP, L::XR>(xs, ws, tok0, acc);
+        } else {  // the ragged last chunk, 8 elements at a time
+            for (int k8 = 0; k8 < kc; k8 += 8)
+                split_chunk<1, TT, L::EP, L::XR>(xs + k8, ws + k8 * L::EP, tok0, acc);
         }
-        cp_async_wait<0>();
-        __syncthreads();  // stage s is read; chunk c + 1 is in stage s ^ 1
     }
+    cp_async_wait<0>();
+    __syncthreads();  // every warp is done with the stages: the logit tile may reuse them
 
     // logits (+ bias) of the tile -> shared memory [token][expert]
-    float *lt = rt8_smem;
+    float *lt = reinterpret_cast<float *>(rs_smem);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const int ta = (p < 2 ? 4 * ty : TM / 2 + 4 * ty) + 2 * (p & 1);
+    for (int m = 0; m < TT; ++m) {
+        const int tok = tok0 + 16 * m;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = j * G::TX + tx;
-            float a = acc[p][j].x, b = acc[p][j].y;
-            if (bias && e < E) {
-                const float be = bias[e];
-                a = __fadd_rn(a, be);
-                b = __fadd_rn(b, be);
+        for (int p = 0; p < 4; ++p) {
+            const int e = ecol + 2 * p;
+            float a = acc[m][p].x, b = acc[m][p].y;
+            if (bias) {
+                if (e < E)
+                    a = __fadd_rn(a, bias[e]);
+                if (e + 1 < E)
+                    b = __fadd_rn(b, bias[e + 1]);
             }
-            lt[ta * G::LR + e] = a;
-            lt[(ta + 1) * G::LR + e] = b;
+            lt[tok * L::LR + e] = a;
+            lt[tok * L::LR + e + 1] = b;
         }
     }
     __syncthreads();
-    for (int tok = warp; tok < TM; tok += G::NW) {
+
+    // top-K of each token: warp w takes tokens w, w + NW, ...
+    for (int tok = warp; tok < kRsTok; tok += L::NW) {
         const int t = t0 + tok;
         if (t >= N)
             break;
-        topk_select_warp<EPAD / 32>(lt + tok * G::LR, E, K, (size_t)t, logits, topk_idx, topk_w,
-                                    nonfinite_count);
+        topk_select_warp<(L::EC + 31) / 32>(lt + tok * L::LR, E, K, (size_t)t, logits, topk_idx,
+                                            topk_w, nonfinite_count);
     }
 }
 

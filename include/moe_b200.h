@@ -192,8 +192,9 @@ int64_t moe_capacity(const moe_shape_t *shape);
  * last expert. Returns -1 on an invalid shape. */
 int64_t moe_rows_alloc(const moe_shape_t *shape);
 
-/* Workspace bytes for moe_route (logit scratch when logits == NULL) and moe_dispatch
- * (block histograms, pack bases). 0 on an invalid shape. */
+/* Workspace bytes for moe_route (the router's scratch: the logits when logits == NULL, and the
+ * router weights transposed, [d][E rounded up to 64, 128 or 256] fp32, when N >= 2048 and
+ * E > 32) and moe_dispatch (block histograms, pack bases). 0 on an invalid shape. */
 size_t moe_workspace_size(const moe_shape_t *shape);
 
 /* Workspace bytes for moe_layer: every intermediate of the layer plus the scratch above. */
@@ -215,8 +216,11 @@ size_t moe_y_bytes(const moe_shape_t *shape);
  * topk_idx [N][K] int32: the K largest logits, larger first, equal logits to the lower
  * expert index. topk_w [N][K] fp32: softmax over the K selected logits.
  * logits [N][E] fp32 or NULL (then not returned; the workspace holds them only where the two
- * steps run as separate kernels: few tokens or E < 32). A non-finite logit sets
- * MOE_ERR_NONFINITE in the device error word; that token's result is unspecified. */
+ * steps run as separate kernels: few tokens or E < 32). The workspace (moe_workspace_size
+ * bytes, 16-byte aligned, device) is required when logits == NULL, and always when N >= 2048
+ * and E > 32 (the transposed router weights); MOE_ERR_WORKSPACE_TOO_SMALL otherwise. A
+ * non-finite logit sets MOE_ERR_NONFINITE in the device error word; that token's result is
+ * unspecified. */
 moe_status_t moe_route(const moe_shape_t *shape, const uint16_t *x, const float *w_router,
                        const float *bias, int32_t *topk_idx, float *topk_w, float *logits,
                        void *ws, size_t ws_bytes, moe_stream_t stream);

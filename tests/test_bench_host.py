@@ -16,15 +16,16 @@ sys.path.insert(0, ROOT)
     ("mixtral_prefill", 10),       # E = 8: projection, then selection; pair + single GEMMs,
                                    # the fp16 range pass
     ("mixtral_prefill_fp8", 10),   # e4m3 GEMMs (no range pass) + quantisation of h
-    ("e128_skew", 7),              # fused router; ~165 rows per expert: single-CTA GEMMs only
-    ("e128_skew_fp8", 7),
+    ("e128_skew", 8),              # W_r transposition + fused router; ~165 rows per expert:
+                                   # single-CTA GEMMs only
+    ("e128_skew_fp8", 8),
     ("decode", 8),                 # 16 tokens: projection, then selection
-    ("e128_skew_slot_major", 7),   # the same two dispatch kernels over K times more blocks
-    ("e128_skew_reroute", 10),     # positions-only pass, the ranking kernel, the full pass
-    ("stack4", 9),                 # pair GEMMs
-    ("stack4_affinity", 9),
+    ("e128_skew_slot_major", 8),   # the same two dispatch kernels over K times more blocks
+    ("e128_skew_reroute", 11),     # positions-only pass, the ranking kernel, the full pass
+    ("stack4", 10),                # pair GEMMs
+    ("stack4_affinity", 10),
     ("mixtral_prefill_fp8_return", 10),
-    ("e128_skew_fp8_return", 7),
+    ("e128_skew_fp8_return", 8),
     ("residual_top1", 14),         # shared MLP: offsets, pair + single GEMMs twice, range passes
 ])
 def test_kernel_launch_count(name, count):

@@ -1,12 +1,13 @@
 """Parity of the router with the oracle, through moe_route: the fused kernels (projection + top-K
-in one kernel: many tokens, E >= 32; the broadcast form and, for E <= 64 with many tokens, the
-register-tiled form) and the separate kernels (few logits: small N or few experts, then the
-top-K kernel). Checked: the logits bit for bit (each one fp32 fmaf chain over d in ascending
-order from +0, then + bias), the top-K indices exactly, the gate weights within fp32 rounding of
-the oracle's fp64 softmax. The shapes cover a ragged last token tile, a hidden size that is not
-a multiple of the 32-element chunk, every padded expert width (E rounded up to 32, 64, 128, 256),
-K from 1 to 32, with and without a bias, and planted ties (two experts with identical router
-rows: equal logits, the lower expert index first)."""
+in one kernel: many tokens, E >= 32; the broadcast form for E = 32 and the split-warp form on
+the transposed weights for E > 32, in each of its tile configurations: 64 experts with 2 or 4
+tokens per lane, 128 and 256 experts) and the separate kernels (few logits: small N or few
+experts, then the top-K kernel). Checked: the logits bit for bit (each one fp32 fmaf chain over d
+in ascending order from +0, then + bias), the top-K indices exactly, the gate weights within fp32
+rounding of the oracle's fp64 softmax. The shapes cover a ragged last token tile, hidden sizes
+that are not a multiple of the staged chunk (32 or 64 elements), every padded expert width (E
+rounded up to 32, 64, 128, 256), K from 1 to 32, with and without a bias, and planted ties (two
+experts with identical router rows: equal logits, the lower expert index first)."""
 import numpy as np
 import pytest
 import torch
@@ -24,8 +25,10 @@ CASES = [
     (4096, 512, 128, 8, 1.1),
     (2048, 1024, 160, 32, 0.0),  # E padded to 256, K = 32
     (2049, 64, 256, 8, 1.2),
-    # the register-tiled fused form (E <= 64, many tokens): ragged last tile, partial chunk,
-    # padded experts
+    (2080, 328, 200, 8, 0.0),    # E padded to 256, d = 5 chunks of 64 + 8
+    (2048, 8, 128, 4, 0.0),      # a single ragged chunk
+    # the split-warp form with 4 tokens per lane (E <= 64, several CTAs per SM): ragged last
+    # tile, partial chunk, padded experts
     (30000, 136, 64, 6, 1.2),
     (29001, 256, 40, 4, 0.0),
     # the separate kernels: decode-sized, few experts, an odd expert count, one token
