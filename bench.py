@@ -212,22 +212,24 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- GPU arm
 
-# DRAM bytes per launch of the gate/up grouped GEMM at full size, from ncu captures of the
-# half-size cases (scaled x2: weights, rows and h all double), summarised in profiles/.
+# DRAM bytes per launch of the gate/up grouped GEMM at full size, from one-pass ncu captures
+# (the Mixtral shape from its half-size case, scaled x2: weights, rows and h all double),
+# summarised in profiles/.
 # A figure holds only for the kernel code it was measured on (kernel_source_hash of
 # grouped_gemm.cuh: comments and whitespace do not count).
-_UP_SHA = "677f9b61402ef3adcb881fae89c4b2c3e66732c2611b4496b9bb8e93c6b1a331"
+_UP_SHA = "5d9c986bcab4eb5e75d5a505601235db5f1094189b4665fedb8a52bf68bf5ea7"
 MEASURED_UP_TRAFFIC = {
     # workload: (kernel source sha256, bytes per launch)
-    "mixtral_prefill": (_UP_SHA, 2 * (994.2e6 + 112.2e6)),      # half-size capture x 2
-    "mixtral_prefill_fp8": (_UP_SHA, 2 * (487.8e6 + 104.4e6)),  # half-size capture x 2
-    "e128_skew": (_UP_SHA, 894.0e6 + 34.4e6),
-    "e128_skew_fp8": (_UP_SHA, 444.1e6 + 32.5e6),
+    "mixtral_prefill": (_UP_SHA, 2 * (995.3e6 + 112.5e6)),      # half-size capture x 2
+    "mixtral_prefill_fp8": (_UP_SHA, 2 * (487.8e6 + 104.3e6)),  # half-size capture x 2
+    "e128_skew": (_UP_SHA, 894.8e6 + 34.7e6),
+    "e128_skew_fp8": (_UP_SHA, 444.1e6 + 32.6e6),
     # the return payload changes the down GEMM and the combine, not the gate/up GEMM
-    "mixtral_prefill_fp8_return": (_UP_SHA, 2 * (487.8e6 + 104.4e6)),
-    "e128_skew_fp8_return": (_UP_SHA, 444.1e6 + 32.5e6),
-    "decode": (_UP_SHA, 6081.7e6 + 3.9e6),
-    "decode_fp8": (_UP_SHA, 3042.0e6 + 3.6e6),
+    "mixtral_prefill_fp8_return": (_UP_SHA, 2 * (487.8e6 + 104.3e6)),
+    "e128_skew_fp8_return": (_UP_SHA, 444.1e6 + 32.6e6),
+    "decode": (_UP_SHA, 6080.8e6 + 3.8e6),
+    "decode_fp8": (_UP_SHA, 3042.2e6 + 3.8e6),
+    "stack4": (_UP_SHA, 4041.5e6 + 597.3e6),                    # one layer's launch
 }
 
 
