@@ -17,7 +17,9 @@ path, so every rank runs an independent replica on its own batch (no
 collective on the data path); the reported time is the max over ranks and the
 value counts the tokens of all ranks ("scaling": "weak").
 
-Prints one JSON line on rank 0.
+The headline value times K replays of the step captured once as a CUDA graph; the
+same K steps launched eagerly, with events between the stages, give the per-stage
+times ("eager", "stages_ms"). Prints one JSON line on rank 0.
 """
 from __future__ import annotations
 
@@ -531,16 +533,22 @@ def run_gpu(args, w) -> dict:
     if m.moe_get_device_error(True) != 0:
         raise RuntimeError("device error during warm-up")
 
-    elapsed_s, stage_ms, clock_summary = timed(args.steps, with_clocks=True)
+    # eager launches with CUDA events between the stages: the per-stage times and the
+    # dominant kernel's mean launch duration
+    elapsed_eager_s, stage_ms, clock_summary = timed(args.steps, with_clocks=args.no_graph)
     R_layers = [int(o[E].item()) for o in offsets]
     act_layers = [int(((o[1:] - o[:-1]) > 0).sum().item()) for o in offsets]
     R = R_layers[0]
-    agg = aggregate(float(N * args.steps), elapsed_s, dev)
+    agg_eager = aggregate(float(N * args.steps), elapsed_eager_s, dev)
 
-    # the same step captured once in a CUDA graph and replayed K times: the host launch
-    # overhead disappears, which matters for small (decode) steps
-    graph_res = None
-    if not args.no_graph:
+    # the headline: the same step captured once in a CUDA graph (how a serving loop runs it)
+    # and replayed K times between a barrier and a synchronize, the clocks sampled meanwhile;
+    # the host launch overhead disappears, which matters for small (decode) steps
+    eager_res = {"value": agg_eager["value"], "unit": UNIT,
+                 "ms_per_step": agg_eager["elapsed_max_s"] / args.steps * 1e3}
+    if args.no_graph:
+        agg, elapsed_s, timing = agg_eager, elapsed_eager_s, "eager launches"
+    else:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step()
@@ -550,15 +558,21 @@ def run_gpu(args, w) -> dict:
         barrier()
         g0 = torch.cuda.Event(enable_timing=True)
         g1 = torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler(local)
+        sampler.__enter__()
         g0.record(stream)
         for _ in range(args.steps):
             graph.replay()
         g1.record(stream)
         torch.cuda.synchronize(dev)
+        sampler.__exit__(None, None, None)
         barrier()
-        g_agg = aggregate(float(N * args.steps), g0.elapsed_time(g1) / 1e3, dev)
-        graph_res = {"value": g_agg["value"], "unit": UNIT,
-                     "ms_per_step": g_agg["elapsed_max_s"] / args.steps * 1e3}
+        clock_summary = sampler.summary()
+        elapsed_s = g0.elapsed_time(g1) / 1e3
+        agg = aggregate(float(N * args.steps), elapsed_s, dev)
+        timing = "CUDA graph of one step, replayed"
+        if m.moe_get_device_error(True) != 0:
+            raise RuntimeError("device error during the graph replays")
         del graph
 
     peaks = load_peaks()
@@ -795,7 +809,8 @@ def run_gpu(args, w) -> dict:
         "routing": routing,
         "clocks": clock_summary,
         "gpu_launches": (L * kernel_launches(w) + (L - 1)) * args.steps,
-        "graph": graph_res,
+        "timing": timing,
+        "eager": eager_res,
         "device_error": err,
         "e2e": e2e,
     }
