@@ -342,11 +342,12 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
 #define MOE_RS(NE, TT, KC, ST)                                                                     \
     launch_router_split<NE, TT, KC, ST>(s, x, scratch, bias, topk_idx, topk_w, logits_out,         \
                                         nonfinite, st)
-            // E <= 64 with several CTAs per SM: 4 tokens per lane (8 warps per SM at least);
-            // otherwise 2 tokens per lane and twice the warps, 64-element chunks (measured on
-            // the B200: N = 8192, d = 2048, E = 128: 152 -> 141 us against the broadcast form;
-            // N = 32768, d = 4096, E = 64: 509 -> 477 us against the register-tiled form;
-            // N = 8192, d = 2048, E = 256: 266 -> 237 us; N = 8192, d = 2048, E = 64: 111 -> 85 us)
+            // 4 tokens per lane, except E <= 64 with too few tokens for several CTAs per SM
+            // (2 tokens per lane and twice the warps there); 64-element chunks except the stack
+            // layer's shape (measured on the B200: N = 8192, d = 2048, E = 128: 152 -> 136 us
+            // against the broadcast form; N = 32768, d = 4096, E = 64: 509 -> 477 us against
+            // the register-tiled form; N = 8192, d = 2048, E = 256: 266 -> 237 us; N = 8192,
+            // d = 2048, E = 64: 111 -> 85 us)
             const bool many = (long long)N >= 64LL * 3 * num_sms();
             if (EC == 64) {
                 if (many)
@@ -354,7 +355,7 @@ moe_status_t route_impl(const moe_shape_t *s, const uint16_t *x, const float *w_
                 else
                     MOE_RS(4, 2, 64, 3);
             } else if (EC == 128) {
-                MOE_RS(8, 2, 64, 3);
+                MOE_RS(8, 4, 64, 3);
             } else {
                 MOE_RS(16, 4, 64, 2);
             }
