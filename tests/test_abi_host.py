@@ -110,6 +110,14 @@ def test_argument_errors_return_before_launch(m):
     assert lib.moe_dispatch(by(s), P, P, P, P, P, P, P, P, None, None, None, None, P, need - 1,
                             None) == 3
     assert lib.moe_layer(by(s), P, P, None, P, P, P, None, P, None, None, P, 1024, None) == 3
+    # the fused router (N >= 2048, E > 32) reads the router weights transposed into the
+    # workspace: required even when the logits go to the caller, and sized for [d][E rounded up]
+    big = m.make_shape(4096, 7168, 256, 200, 8, 8)
+    assert lib.moe_route(by(big), P, P, None, P, P, P, None, 0, None) == 3
+    assert lib.moe_route(by(big), P, P, None, P, P, P, P, 16, None) == 3
+    assert m.moe_workspace_size(big) >= 256 * 7168 * 4 > 4096 * 200 * 4
+    few = m.make_shape(2047, 7168, 256, 200, 8, 1)  # the two-kernel router: no workspace needed
+    assert m.moe_workspace_size(few) < 256 * 7168 * 4
     # shape errors
     bad = m.make_shape(64, 128, 256, 8, 9, 4)
     assert lib.moe_route(by(bad), P, P, None, P, P, P, None, 0, None) == 1
