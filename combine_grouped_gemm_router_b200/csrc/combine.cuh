@@ -44,6 +44,220 @@ __device__ __forceinline__ void decode_e4m3x8(uint32_t lo, uint32_t hi, float sc
     }
 }
 
+// ---------------------------------------------------------------------------
+// Bulk-fed combine for the block payloads (YK 1: e4m3, 2: fp16 codes). The combine above is
+// bound by memory latency: a warp gathers one slot's 16-byte pieces per round trip, and its
+// registers cap how many warps keep loads in flight. Here a producer warp brings each token's
+// kept expert rows (whole payload rows, codes and exponent bytes together: one bulk copy per
+// slot), and its residual row and shared-MLP row when given, into a stage of shared memory,
+// kCbMaxStages tokens ahead; eight consumer warps each combine their eighth of the token's
+// columns from shared memory and store it. The bytes in flight cost no registers, and the
+// consumers never wait on global memory. A stage is refilled once all eight have released it.
+// The arithmetic is combine_kernel's, in the same order (slot order k = 0..K-1, then the shared
+// MLP's output, then the residual), so the outputs are the same bits. Every wait is bounded.
+constexpr int kCbConsumers = 8;
+constexpr int kCbMaxStages = 8;
+
+// Shared-memory bytes of one stage: the K payload rows, the residual row (bf16), the shared
+// MLP's row (fp32).
+__host__ __device__ inline size_t cb_stage_bytes(int K, int y_stride, int d, bool residual,
+                                                 bool shared)
+{
+    return (size_t)K * y_stride + (residual ? 2 * (size_t)d : 0) + (shared ? 4 * (size_t)d : 0);
+}
+
+// Total shared memory for S stages: the stages, then per stage its two mbarriers, the K gate
+// weights and the mask of the kept slots.
+__host__ __device__ inline size_t cb_smem_bytes(size_t stage_bytes, int S)
+{
+    return stage_bytes * S + (size_t)S * (16 + 32 * 4 + 4) + 16;
+}
+
+template <bool OUT_BF16, int YK>
+__global__ void __launch_bounds__(32 * (kCbConsumers + 1))
+    combine_bulk_kernel(const void *__restrict__ y, int y_stride, const int32_t *__restrict__ row_of,
+                        const float *__restrict__ topk_w, const float *__restrict__ shared_y,
+                        const uint16_t *__restrict__ residual, int N, int d, int K, int S,
+                        void *__restrict__ out, uint64_t timeout_ns)
+{
+    static_assert(YK == 1 || YK == 2, "block payloads only");
+    extern __shared__ __align__(16) unsigned char cb_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const size_t rows_bytes = (size_t)K * y_stride;
+    const size_t stage_bytes = cb_stage_bytes(K, y_stride, d, residual != nullptr,
+                                              shared_y != nullptr);
+    const size_t meta = stage_bytes * S;
+    const uint32_t full = smem_u32(cb_smem) + (uint32_t)meta;         // [S] mbarriers
+    const uint32_t empty = full + 8u * (uint32_t)S;                     // [S] mbarriers
+    float *s_w = reinterpret_cast<float *>(cb_smem + meta + 16 * S);   // [S][32]
+    uint32_t *s_mask = reinterpret_cast<uint32_t *>(s_w + 32 * S);      // [S]
+    int *s_done = reinterpret_cast<int *>(s_mask + S);                  // tokens every consumer took
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < S; ++j) {
+            mbar_init(full + 8 * j, 1);
+            mbar_init(empty + 8 * j, kCbConsumers);
+        }
+        s_done[0] = 0x7fffffff;
+        s_done[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const int n_mine = (int)blockIdx.x < N ? (N - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x
+                                           : 0;
+    const unsigned char *yb = reinterpret_cast<const unsigned char *>(y);
+    int issued = 0;
+    if (warp == kCbConsumers) {
+        // ---------------- producer: token j of this CTA into stage j mod S. The tokens' rows
+        // and weights are read TB = 32 / K tokens per warp load (lane b K + k: token b, slot k),
+        // one batch ahead, so their latency is paid once per batch and overlaps the copies.
+        const int TB = 32 / K;
+        auto load_batch = [&](int jb, int &rk_, float &w_) {
+            const int b = lane / K, jj = jb + b;
+            rk_ = -1;
+            w_ = 0.0f;
+            if (b < TB && jj < n_mine) {
+                const size_t a = (size_t)((int)blockIdx.x + jj * (int)gridDim.x) * K + lane % K;
+                rk_ = row_of[a];
+                w_ = topk_w[a];
+            }
+        };
+        int brk, nrk;
+        float bw, nw;
+        load_batch(0, nrk, nw);
+        for (int j = 0; j < n_mine; ++j) {
+            const int s = j % S;
+            if (j % TB == 0) {
+                brk = nrk;
+                bw = nw;
+                load_batch(j + TB, nrk, nw);
+            }
+            const int src = (j % TB) * K + (lane < K ? lane : 0);
+            int rk = __shfl_sync(0xffffffffu, brk, src);
+            float w = __shfl_sync(0xffffffffu, bw, src);
+            if (lane >= K) {
+                rk = -1;
+                w = 0.0f;
+            }
+            if (j >= S && !mbar_wait_bounded(empty + 8 * s, (uint32_t)((j / S - 1) & 1), timeout_ns))
+                break;
+            const int t = (int)blockIdx.x + j * (int)gridDim.x;
+            const uint32_t mask = __ballot_sync(0xffffffffu, rk >= 0);
+            s_w[s * 32 + lane] = w;
+            if (lane == 0)
+                s_mask[s] = mask;
+            const uint32_t tx = (uint32_t)(__popc(mask) * y_stride) +
+                                (residual ? 2u * (uint32_t)d : 0u) + (shared_y ? 4u * (uint32_t)d : 0u);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_expect_tx(full + 8 * s, tx);  // also publishes the weights and mask
+            __syncwarp();
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            const uint32_t st = smem_u32(cb_smem) + (uint32_t)(s * stage_bytes);
+            if (rk >= 0)
+                bulk_load_g2s(st + (uint32_t)(lane * y_stride), yb + (size_t)rk * y_stride,
+                              (uint32_t)y_stride, full + 8 * s);
+            if (lane == 0 && residual)
+                bulk_load_g2s(st + (uint32_t)rows_bytes, residual + (size_t)t * d, 2u * (uint32_t)d,
+                              full + 8 * s);
+            if (lane == 0 && shared_y)
+                bulk_load_g2s(st + (uint32_t)(rows_bytes + (residual ? 2 * (size_t)d : 0)),
+                              shared_y + (size_t)t * d, 4u * (uint32_t)d, full + 8 * s);
+            issued = j + 1;
+        }
+    } else {
+        // ---------------- consumers: warp w combines columns [w d / 8, (w + 1) d / 8)
+        const int ng = d / 64;  // 8-column groups per consumer warp
+        const int g0 = warp * ng;
+        const int code_bytes = YK == 2 ? 2 * d : d;
+        int j = 0;
+        for (; j < n_mine; ++j) {
+            const int s = j % S;
+            if (!mbar_wait_bounded(full + 8 * s, (uint32_t)((j / S) & 1), timeout_ns))
+                break;
+            const int t = (int)blockIdx.x + j * (int)gridDim.x;
+            const uint32_t mask = s_mask[s];
+            const float *ws = s_w + s * 32;
+            const unsigned char *st = cb_smem + (size_t)s * stage_bytes;
+            for (int gi = lane; gi < ng; gi += 32) {
+                const int g = g0 + gi;
+                float acc[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    acc[q] = 0.0f;
+                for (int k = 0; k < K; ++k) {
+                    if (!((mask >> k) & 1u))
+                        continue;
+                    const float wk = ws[k];
+                    const unsigned char *row = st + (size_t)k * y_stride;
+                    const float sc = pow2f((int)row[code_bytes + g / 4] - 127);
+                    if constexpr (YK == 2) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * g);
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            acc[2 * q] = __fmaf_rn(wk, f16_to_f32(w4[q] & 0xFFFFu) * sc, acc[2 * q]);
+                            acc[2 * q + 1] =
+                                __fmaf_rn(wk, f16_to_f32(w4[q] >> 16) * sc, acc[2 * q + 1]);
+                        }
+                    } else {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(row + 8 * g);
+                        float f8[8];
+                        decode_e4m3x8(v.x, v.y, sc, f8);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            acc[q] = __fmaf_rn(wk, f8[q], acc[q]);
+                    }
+                }
+                if (shared_y) {
+                    const float4 *sv = reinterpret_cast<const float4 *>(
+                                           st + rows_bytes + (residual ? 2 * (size_t)d : 0)) +
+                                       2 * g;
+                    const float4 a = sv[0], b = sv[1];
+                    const float f8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        acc[q] = __fadd_rn(acc[q], f8[q]);
+                }
+                if (residual) {
+                    const uint4 rv = reinterpret_cast<const uint4 *>(st + rows_bytes)[g];
+                    const uint32_t q4[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[2 * q] = __fadd_rn(acc[2 * q], bf16_lo(q4[q]));
+                        acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], bf16_hi(q4[q]));
+                    }
+                }
+                const size_t chunk = (size_t)t * (d >> 3) + g;
+                if (OUT_BF16) {
+                    uint4 o;
+                    o.x = pack_bf16x2(acc[0], acc[1]);
+                    o.y = pack_bf16x2(acc[2], acc[3]);
+                    o.z = pack_bf16x2(acc[4], acc[5]);
+                    o.w = pack_bf16x2(acc[6], acc[7]);
+                    reinterpret_cast<uint4 *>(out)[chunk] = o;
+                } else {
+                    float4 *o = reinterpret_cast<float4 *>(out) + chunk * 2;
+                    o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(empty + 8 * s);  // this warp is done with the stage
+        }
+        if (lane == 0)
+            atomicMin(s_done, j);
+    }
+    if (warp == kCbConsumers && lane == 0)
+        atomicMax(s_done + 1, issued);
+    __syncthreads();
+    // stages loaded and not consumed (only after a wait that ran out): let them land first
+    if (threadIdx.x == 0)
+        for (int j = *s_done; j < s_done[1]; ++j)
+            mbar_wait_bounded(full + 8 * (j % S), (uint32_t)((j / S) & 1), timeout_ns);
+    __syncthreads();
+}
+
 template <bool OUT_BF16, int YK>
 __global__ void __launch_bounds__(256)
     combine_kernel(const void *__restrict__ y, int y_stride, const int32_t *__restrict__ row_of,

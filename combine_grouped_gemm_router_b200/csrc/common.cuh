@@ -163,6 +163,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Bulk copy global -> shared memory, completing on the mbarrier at `bar` (bytes: a multiple of
+// 16, both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Bounded wait on an mbarrier phase; false (and MOE_ERR_DEVICE_TIMEOUT) when it runs out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > timeout_ns) {
+            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+
 // Token block b of the dispatch: blocks never straddle a home-rank shard, so
 // per-shard prefix counts are available at block boundaries.
 // shard = b / bps, tokens [shard*S + (b%bps)*HB, min(... + HB, (shard+1)*S)).

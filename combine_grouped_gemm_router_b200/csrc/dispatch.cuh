@@ -453,36 +453,11 @@ __host__ __device__ inline size_t place_smem_total(int E, int K, int slots)
     return place_ring_offset(E, K) + (size_t)8 * slots * kPiece + (size_t)8 * slots * 8;
 }
 
-__device__ __forceinline__ void bulk_load_g2s(uint32_t dst, const void *src, uint32_t bytes,
-                                              uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
 __device__ __forceinline__ void bulk_store_s2g(void *dst, uint32_t src, uint32_t bytes)
 {
     asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
                  "r"(bytes)
                  : "memory");
-}
-
-// Bounded wait on an mbarrier phase; false (and MOE_ERR_DEVICE_TIMEOUT) when it runs out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > timeout_ns) {
-            set_dev_error(MOE_ERR_DEVICE_TIMEOUT);
-            return false;
-        }
-    }
-    return true;
 }
 
 // Bulk copy of a token block's bf16 rows (the share of part `part` of `parts`): the block's

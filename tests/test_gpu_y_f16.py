@@ -80,14 +80,15 @@ def test_payload_is_the_block_code_of_y(orc, case, gemm):
     assert np.all(pad == 0xAB) and np.all(tail == 0xAB), "bytes outside the kept rows written"
 
 
-@pytest.mark.parametrize("N", [96, 2048])
-def test_combine_weighs_the_payload_exactly(orc, N):
+@pytest.mark.parametrize("N,d", [(96, 256), (2048, 256), (9600, 512)])
+def test_combine_weighs_the_payload_exactly(orc, N, d):
     """moe_combine on an fp16 payload: out = sum_k w_k * (code * 2^j), fp32 accumulation in k
     order, then the shared MLP's output and the residual when given; the oracle's combine of
     the decoded payload (fp64) bounds the difference per element. N = 96 takes the sliced-row
-    path, N = 2048 the whole-row path."""
+    path, N = 2048 the whole-row path, N = 9600 with d = 512 the bulk-fed kernel
+    (64 or more tokens per SM)."""
     m = lib()
-    K, d, E = 3, 256, 4
+    K, E = 3, 4
     shape = m.make_shape(N, d, 128, E, K, 1, 0.0, y_f16=True)
     RA = m.moe_rows_alloc(shape)
     rng = np.random.default_rng(19)
