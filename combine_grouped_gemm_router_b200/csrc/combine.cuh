@@ -45,12 +45,12 @@ __device__ __forceinline__ void decode_e4m3x8(uint32_t lo, uint32_t hi, float sc
 }
 
 // ---------------------------------------------------------------------------
-// Bulk-fed combine for the block payloads (YK 1: e4m3, 2: fp16 codes). The combine above is
+// Bulk-fed combine for the block payloads (YK 1: e4m3, 2: fp16 codes). combine_kernel (below) is
 // bound by memory latency: a warp gathers one slot's 16-byte pieces per round trip, and its
 // registers cap how many warps keep loads in flight. Here a producer warp brings each token's
 // kept expert rows (whole payload rows, codes and exponent bytes together: one bulk copy per
 // slot), and its residual row and shared-MLP row when given, into a stage of shared memory,
-// kCbMaxStages tokens ahead; eight consumer warps each combine their eighth of the token's
+// up to kCbMaxStages tokens ahead; eight consumer warps each combine their eighth of the token's
 // columns from shared memory and store it. The bytes in flight cost no registers, and the
 // consumers never wait on global memory. A stage is refilled once all eight have released it.
 // The arithmetic is combine_kernel's, in the same order (slot order k = 0..K-1, then the shared
