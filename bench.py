@@ -996,16 +996,23 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
-def main(argv=None):
-    args = parse(argv)
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
+def select_workload(args):
+    """The workload the arguments name: its token count replaced by --tokens, and on the bf16
+    path the fp16 return payload unless --y-f32 (the FP8 workloads keep their own payloads)."""
     from moe_workloads import WORKLOADS
     w = WORKLOADS[args.workload]
     if args.tokens > 0:
         w = w.with_(N=args.tokens)
     if not w.fp8 and not args.y_f32:
         w = w.with_(y_f16=True)
+    return w
+
+
+def main(argv=None):
+    args = parse(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = select_workload(args)
     if args.impl == "reference":
         res = run_reference(args, w)
     else:

@@ -124,3 +124,19 @@ def test_algorithmic_work_counts_the_payload_and_output_bytes():
     up = bench.algorithmic_work(WORKLOADS["mixtral_prefill"], 8192, 8)
     assert up["up_flops"] == 4.0 * 4096 * 14336 * 8192
     assert up["up_bytes"] == 2.0 * 8 * 14336 * 4096 * 2 + 8192 * 4096 * 2 + 8192 * 14336 * 2
+
+
+def test_workload_selection_and_payload_bytes():
+    """The bench runs the bf16-path workloads with the fp16 return payload unless --y-f32, keeps
+    the FP8 workloads' own payloads, and counts the combine's payload bytes accordingly
+    (2d code bytes + d/32 exponent bytes per kept row)."""
+    import bench
+    w = bench.select_workload(bench.parse([]))
+    assert w.name == "stack4" and w.y_f16 and not w.fp8
+    assert not bench.select_workload(bench.parse(["--y-f32"])).y_f16
+    assert not bench.select_workload(bench.parse(["--workload", "e128_skew_fp8"])).y_f16
+    assert bench.select_workload(bench.parse(["--workload", "decode", "--tokens", "8"])).N == 8
+    w = bench.select_workload(bench.parse(["--workload", "e128_skew"]))
+    R, N, d, K = 21185, w.N, w.d, w.K
+    assert bench.algorithmic_work(w, R, 128)["combine_bytes"] == \
+        R * (2 * d + d // 32) + N * K * 8 + N * d * 2
